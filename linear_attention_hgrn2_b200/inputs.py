@@ -1,0 +1,127 @@
+"""Seeded synthetic inputs for the HGRN2 recurrence.
+
+This module is shared by the tests, the benchmark and the smoke check, and it
+holds none of the recurrence's arithmetic: it only draws random tensors with
+the shapes and value distributions of the workloads below and rounds them to
+their storage dtype.  Both the CUDA path and the CPU oracle consume exactly the
+tensors produced here (the oracle after an exact upcast to float64).
+
+Forget gates follow the lower-bounded parameterisation of HGRN ("HGRN2: Gated
+Linear RNNs with State Expansion", §2.2: each layer's forget gate is a learned
+residual above a lower bound ``lb`` that rises with depth):
+
+    f = lb + (1 - lb) * sigmoid(x),  x ~ N(0, 1),     log_f = log(f)
+
+computed in float64, then rounded to the storage dtype.  q, i and dO are
+N(0, 1); initial states are N(0, sigma^2) in float32.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    T: int
+    dk: int
+    dv: int
+    dtype: torch.dtype
+    lb: float
+    chunk: int
+    h0_sigma: float = 0.0     # 0 => no initial state (zeros)
+    want_hT: bool = False
+    bwd: bool = False
+
+
+# The five workloads, named by what they are.  Token tensors are [B, T, H, D].
+TINY = Workload("tiny_fp32_B1_H2_T64_d16", 1, 2, 64, 16, 16, torch.float32, 0.0, 16)
+FWD_LAYER = Workload("fwd_bf16_B4_H8_T2048_d128", 4, 8, 2048, 128, 128, torch.bfloat16, 0.5, 64)
+TRAIN = Workload("train_fwdbwd_bf16_B8_H16_T2048_d128", 8, 16, 2048, 128, 128, torch.bfloat16,
+                 0.95, 64, bwd=True)
+LONG = Workload("long_fwd_bf16_B1_H8_T32768_d128", 1, 8, 32768, 128, 128, torch.bfloat16, 0.9, 64,
+                h0_sigma=0.1, want_hT=True)
+# decode: B=256 sequences, H=16, d=128, one token per step, 1000 steps, S ~ N(0,1)
+DECODE = dict(name="decode_bf16_B256_H16_d128_1000steps", B=256, H=16, dk=128, dv=128,
+              dtype=torch.bfloat16, lb=0.8, steps=1000, S_sigma=1.0)
+
+WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG)}
+
+
+def _gen(seed: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _normal(g: np.random.Generator, shape, sigma: float = 1.0) -> np.ndarray:
+    x = g.standard_normal(size=shape, dtype=np.float32)
+    if sigma != 1.0:
+        x *= np.float32(sigma)
+    return x
+
+
+def gate_log_f(x: np.ndarray, lb: float) -> np.ndarray:
+    """log(lb + (1 - lb) * sigmoid(x)) in float64 (stable for lb = 0)."""
+    x = x.astype(np.float64)
+    if lb == 0.0:
+        return -np.logaddexp(0.0, -x)          # log sigmoid(x)
+    sig = 0.5 * (1.0 + np.tanh(0.5 * x))
+    return np.log(lb + (1.0 - lb) * sig)
+
+
+def _to(x: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dtype)
+
+
+def make_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: torch.dtype, lb: float,
+                seed: int, h0_sigma: float = 0.0, with_dO: bool = False,
+                dhT_sigma: float = 0.0) -> dict:
+    """CPU tensors q, log_f, i [B,T,H,*] in ``dtype``; optional h0, dO, dhT.
+
+    Draw order (fixed): q, i, gate pre-activations, dO, h0, dhT."""
+    g = _gen(seed)
+    out = {}
+    out["q"] = _to(_normal(g, (B, T, H, dk)), dtype)
+    out["i"] = _to(_normal(g, (B, T, H, dv)), dtype)
+    out["log_f"] = _to(gate_log_f(_normal(g, (B, T, H, dk)), lb), dtype)
+    if with_dO:
+        out["dO"] = _to(_normal(g, (B, T, H, dv)), dtype)
+    if h0_sigma > 0:
+        out["h0"] = torch.from_numpy(_normal(g, (B, H, dk, dv), h0_sigma))
+    if dhT_sigma > 0:
+        out["dhT"] = torch.from_numpy(_normal(g, (B, H, dk, dv), dhT_sigma))
+    return out
+
+
+def make_workload(w: Workload, seed: int) -> dict:
+    return make_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.lb, seed,
+                       h0_sigma=w.h0_sigma, with_dO=w.bwd)
+
+
+def make_decode(B: int, H: int, dk: int, dv: int, steps: int, dtype: torch.dtype, lb: float,
+                seed: int, S_sigma: float = 1.0, device: str = "cpu") -> dict:
+    """Decode-step inputs: q, log_f [steps,B,H,dk], i [steps,B,H,dv] and S [B,H,dk,dv] fp32.
+
+    On device='cpu' the draws use NumPy's PCG64 (bit-reproducible everywhere).
+    On a CUDA device they use a seeded torch CUDA generator (for the large
+    benchmark pool only; tests that compare with the oracle use the CPU draws)."""
+    if device == "cpu":
+        g = _gen(seed)
+        q = _to(_normal(g, (steps, B, H, dk)), dtype)
+        i = _to(_normal(g, (steps, B, H, dv)), dtype)
+        lf = _to(gate_log_f(_normal(g, (steps, B, H, dk)), lb), dtype)
+        S = torch.from_numpy(_normal(g, (B, H, dk, dv), S_sigma))
+        return {"q": q, "i": i, "log_f": lf, "S": S}
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    q = torch.randn((steps, B, H, dk), generator=gen, device=device).to(dtype)
+    i = torch.randn((steps, B, H, dv), generator=gen, device=device).to(dtype)
+    x = torch.randn((steps, B, H, dk), generator=gen, device=device, dtype=torch.float64)
+    lf = torch.log(lb + (1.0 - lb) * torch.sigmoid(x)).to(dtype)
+    del x
+    S = torch.randn((B, H, dk, dv), generator=gen, device=device) * S_sigma
+    return {"q": q, "i": i, "log_f": lf, "S": S}

@@ -1,0 +1,104 @@
+"""CPU oracle of the HGRN2 recurrence -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline and
+reference legs) may import this package.  The product library never does, and
+the two share no code: the oracle is ``oracle.c`` (plain sequential fp64 loops,
+see its header for the equations and their source) plus ``brute.py`` (an
+independent quadratic-form restatement in NumPy for tiny inputs).
+
+This module only marshals NumPy arrays to ``oracle.c`` through ctypes and
+builds ``liboracle.so`` with gcc when it is missing or stale.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc -O2 -fopenmp); returns the path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ci = ctypes.c_int
+        lib.oracle_fwd.argtypes = [dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci]
+        lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci]
+        lib.oracle_step.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci]
+        lib.oracle_num_threads.restype = ci
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def fwd(q, log_f, i, h0=None):
+    """o [B,T,H,dv] and hT [B,H,dk,dv] of the recurrence, in fp64.
+
+    q, log_f: [B,T,H,dk]; i: [B,T,H,dv]; h0: [B,H,dk,dv] or None (zeros)."""
+    q, log_f, i, h0 = _f64(q), _f64(log_f), _f64(i), _f64(h0)
+    B, T, H, dk = q.shape
+    dv = i.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    hT = np.zeros((B, H, dk, dv))
+    _load().oracle_fwd(_p(q), _p(log_f), _p(i), _p(h0), _p(o), _p(hT), B, T, H, dk, dv)
+    return o, hT
+
+
+def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dk=False):
+    """Gradients (dq, dlog_f, di, dh0[, dk]) of L = <o, dO> + <hT, dhT>, in fp64."""
+    q, log_f, i, dO, h0, dhT = (_f64(a) for a in (q, log_f, i, dO, h0, dhT))
+    B, T, H, dk = q.shape
+    dv = i.shape[-1]
+    dq = np.zeros_like(q)
+    dlf = np.zeros_like(q)
+    di = np.zeros_like(i)
+    dh0 = np.zeros((B, H, dk, dv))
+    dkk = np.zeros_like(q) if want_dk else None
+    _load().oracle_bwd(_p(q), _p(log_f), _p(i), _p(h0), _p(dO), _p(dhT),
+                       _p(dq), _p(dlf), _p(di), _p(dh0), _p(dkk), B, T, H, dk, dv)
+    if want_dk:
+        return dq, dlf, di, dh0, dkk
+    return dq, dlf, di, dh0
+
+
+def step(q, log_f, i, S):
+    """One decode step.  q, log_f: [B,H,dk]; i: [B,H,dv]; S: [B,H,dk,dv].
+
+    Returns (o [B,H,dv], S_new); the input S is not modified."""
+    q, log_f, i = _f64(q), _f64(log_f), _f64(i)
+    S = np.array(S, dtype=np.float64, copy=True, order="C")
+    B, H, dk = q.shape
+    dv = i.shape[-1]
+    o = np.zeros((B, H, dv))
+    _load().oracle_step(_p(q), _p(log_f), _p(i), _p(S), _p(o), B, H, dk, dv)
+    return o, S

@@ -1,0 +1,222 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics.
+
+Each test checks ``oracle`` (the C fp64 reference) against something other than
+itself: a hand-worked example, an independent quadratic-form restatement, closed
+forms, finite differences, or an algebraic identity.  None needs a GPU.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(rng, B, T, H, dk, dv, lb=0.0, h0=True, scale_a=1.0):
+    q = rng.standard_normal((B, T, H, dk))
+    x = rng.standard_normal((B, T, H, dv))
+    z = rng.standard_normal((B, T, H, dk)) * scale_a
+    sig = 1.0 / (1.0 + np.exp(-z))
+    log_f = np.log(lb + (1 - lb) * sig)
+    h = rng.standard_normal((B, H, dk, dv)) if h0 else None
+    return q, log_f, x, h
+
+
+# ---------------------------------------------------------------- hand-worked example
+def _parse_golden(path):
+    vals = {}
+    for line in open(path):
+        line = line.split("#", 1)[0].strip()
+        if not line or "=" not in line:
+            continue
+        key, rhs = line.split("=", 1)
+        rows = []
+        for row in rhs.split(";"):
+            r = []
+            for tok in row.split():
+                if tok.startswith("ln(") and tok.endswith(")"):
+                    r.append(np.log(float(Fraction(tok[3:-1]))))
+                else:
+                    r.append(float(Fraction(tok)))
+            rows.append(r)
+        vals[key.strip()] = np.array(rows)
+    return vals
+
+
+def test_hand_worked_example_fwd_and_bwd():
+    g = _parse_golden(os.path.join(GOLDEN, "hand_example_T2_dk2_dv2.txt"))
+    sh = lambda a: a[None, :, None, :]  # [T, D] -> [1, T, 1, D]
+    o, hT = oracle.fwd(sh(g["q"]), sh(g["log_f"]), sh(g["i"]))
+    np.testing.assert_allclose(o[0, :, 0], g["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(hT[0, 0], g["hT"], rtol=0, atol=1e-14)
+    dq, dlf, di, dh0 = oracle.bwd(sh(g["q"]), sh(g["log_f"]), sh(g["i"]), sh(g["dO"]))
+    np.testing.assert_allclose(dq[0, :, 0], g["dq"], atol=1e-14)
+    np.testing.assert_allclose(di[0, :, 0], g["di"], atol=1e-14)
+    np.testing.assert_allclose(dlf[0, :, 0], g["dlog_f"], atol=1e-14)
+    np.testing.assert_allclose(dh0[0, 0], g["dh0"], atol=1e-14)
+
+
+# ---------------------------------------------------------------- forward pins
+@pytest.mark.parametrize("shape", [(1, 7, 1, 3, 2), (2, 9, 3, 4, 5), (1, 70, 2, 2, 3)])
+def test_fwd_matches_quadratic_form(shape):
+    rng = np.random.default_rng(1)
+    B, T, H, dk, dv = shape
+    q, lf, x, h0 = _rand(rng, B, T, H, dk, dv)
+    o, hT = oracle.fwd(q, lf, x, h0)
+    o2, hT2 = brute.quadratic_form(q, lf, x, h0)
+    np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hT, hT2, rtol=1e-12, atol=1e-12)
+
+
+def test_fwd_closed_form_f_one_freezes_state():
+    # log f = 0 => f = 1, k = 0: S stays h0 and o_t = h0^T q_t
+    rng = np.random.default_rng(2)
+    q, _, x, h0 = _rand(rng, 2, 11, 2, 4, 3)
+    lf = np.zeros_like(q)
+    o, hT = oracle.fwd(q, lf, x, h0)
+    np.testing.assert_array_equal(hT, h0)
+    np.testing.assert_allclose(o, np.einsum("bthj,bhjv->bthv", q, h0), rtol=1e-13, atol=1e-13)
+    o0, _ = oracle.fwd(q, lf, x, None)
+    assert np.all(o0 == 0.0)
+
+
+def test_fwd_closed_form_f_zero_keeps_last_input():
+    # log f = -40 => f ~ 4e-18 (0 at double precision relative to 1), k = 1:
+    # S_t = 1 i_t^T and o_t = (sum_j q_t[j]) i_t
+    rng = np.random.default_rng(3)
+    q, _, x, h0 = _rand(rng, 1, 13, 2, 5, 4)
+    lf = np.full_like(q, -40.0)
+    o, hT = oracle.fwd(q, lf, x, h0)
+    np.testing.assert_allclose(o, q.sum(-1, keepdims=True) * x, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hT[:, :, 0, :], x[:, -1], rtol=1e-12)
+
+
+def test_fwd_closed_form_constant_scalar_gate_geometric_sum():
+    # scalar f for all t and j, constant input xbar: S_t = f^{t+1} h0 + (1 - f^{t+1}) 1 xbar^T
+    rng = np.random.default_rng(4)
+    B, T, H, dk, dv = 1, 25, 1, 3, 4
+    f = 0.83
+    q = rng.standard_normal((B, T, H, dk))
+    xbar = rng.standard_normal(dv)
+    x = np.broadcast_to(xbar, (B, T, H, dv)).copy()
+    h0 = rng.standard_normal((B, H, dk, dv))
+    lf = np.full((B, T, H, dk), np.log(f))
+    o, hT = oracle.fwd(q, lf, x, h0)
+    t = np.arange(T)
+    ft = f ** (t + 1)
+    expect = (ft[:, None] * (q[0, :, 0] @ h0[0, 0])
+              + (1 - ft)[:, None] * q[0, :, 0].sum(-1, keepdims=True) * xbar[None, :])
+    np.testing.assert_allclose(o[0, :, 0], expect, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hT[0, 0], f ** T * h0[0, 0] + (1 - f ** T) * xbar[None, :],
+                               rtol=1e-12)
+
+
+def test_fwd_literal_masked_attention_when_decay_shared_over_dims():
+    # with one f per token (shared across key dims) O = ((Q K^T) * D) V exactly
+    rng = np.random.default_rng(5)
+    T, dk, dv = 17, 4, 3
+    f = 1 / (1 + np.exp(-rng.standard_normal(T)))
+    q = rng.standard_normal((T, dk))
+    x = rng.standard_normal((T, dv))
+    lf = np.repeat(np.log(f)[:, None], dk, axis=1)
+    o, _ = oracle.fwd(q[None, :, None], lf[None, :, None], x[None, :, None])
+    np.testing.assert_allclose(o[0, :, 0], brute.masked_attention_shared_decay(q, f, x),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_fwd_heads_and_batches_independent():
+    rng = np.random.default_rng(6)
+    q, lf, x, h0 = _rand(rng, 2, 9, 3, 4, 4)
+    o, hT = oracle.fwd(q, lf, x, h0)
+    for b in range(2):
+        for h in range(3):
+            o1, hT1 = oracle.fwd(q[b:b + 1, :, h:h + 1], lf[b:b + 1, :, h:h + 1],
+                                 x[b:b + 1, :, h:h + 1], h0[b:b + 1, h:h + 1])
+            np.testing.assert_array_equal(o1[0, :, 0], o[b, :, h])
+            np.testing.assert_array_equal(hT1[0, 0], hT[b, h])
+
+
+# ---------------------------------------------------------------- step pins
+def test_steps_equal_fwd():
+    rng = np.random.default_rng(7)
+    B, T, H, dk, dv = 2, 12, 3, 4, 5
+    q, lf, x, h0 = _rand(rng, B, T, H, dk, dv)
+    o, hT = oracle.fwd(q, lf, x, h0)
+    S = h0.copy()
+    for t in range(T):
+        ot, S = oracle.step(q[:, t], lf[:, t], x[:, t], S)
+        np.testing.assert_allclose(ot, o[:, t], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S, hT, rtol=1e-13, atol=1e-13)
+
+
+def test_step_reads_updated_state():
+    # one step from S = 0 must already see the current token: o = (q . k) i
+    q = np.array([[[1.0, 2.0]]])
+    lf = np.log(np.array([[[0.25, 0.5]]]))
+    x = np.array([[[3.0]]])
+    o, S = oracle.step(q, lf, x, np.zeros((1, 1, 2, 1)))
+    assert o[0, 0, 0] == pytest.approx((1 * 0.75 + 2 * 0.5) * 3.0, abs=1e-15)
+
+
+# ---------------------------------------------------------------- backward pins
+def _loss(q, lf, x, h0, dO, dhT):
+    o, hT = oracle.fwd(q, lf, x, h0)
+    return float(np.sum(o * dO) + np.sum(hT * dhT))
+
+
+@pytest.mark.parametrize("T", [6, 131])
+def test_bwd_matches_central_finite_differences(T):
+    rng = np.random.default_rng(8 + T)
+    B, H, dk, dv = 1, 2, 3, 2
+    q, lf, x, h0 = _rand(rng, B, T, H, dk, dv, lb=0.3)
+    dO = rng.standard_normal((B, T, H, dv))
+    dhT = rng.standard_normal((B, H, dk, dv))
+    dq, dlf, dx, dh0 = oracle.bwd(q, lf, x, dO, h0, dhT)
+    eps = 1e-6
+    pick = np.random.default_rng(99)
+    for name, arr, grad in (("q", q, dq), ("log_f", lf, dlf), ("i", x, dx), ("h0", h0, dh0)):
+        flat = arr.reshape(-1)
+        idx = pick.choice(flat.size, size=min(flat.size, 24), replace=False)
+        for n in idx:
+            old = flat[n]
+            flat[n] = old + eps
+            lp = _loss(q, lf, x, h0, dO, dhT)
+            flat[n] = old - eps
+            lm = _loss(q, lf, x, h0, dO, dhT)
+            flat[n] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - grad.reshape(-1)[n]) <= 1e-6 * max(1.0, abs(fd)), (name, n, fd)
+
+
+def test_bwd_dlog_f_equals_reverse_cumsum_identity():
+    # d log f_t = sum_{t'>=t} (q*dq - k*dk)_{t'} + rowsum(dhT*hT) - f_t*dk_t
+    # (a rescaling argument on the cumulative log-decay; independent of BPTT's order)
+    rng = np.random.default_rng(9)
+    B, T, H, dk, dv = 2, 40, 2, 4, 3
+    q, lf, x, h0 = _rand(rng, B, T, H, dk, dv, lb=0.2)
+    dO = rng.standard_normal((B, T, H, dv))
+    dhT = rng.standard_normal((B, H, dk, dv))
+    dq, dlf, dx, dh0, dkk = oracle.bwd(q, lf, x, dO, h0, dhT, want_dk=True)
+    _, hT = oracle.fwd(q, lf, x, h0)
+    k = -np.expm1(lf)
+    f = np.exp(lf)
+    w = q * dq - k * dkk
+    rc = np.flip(np.cumsum(np.flip(w, 1), 1), 1)
+    alt = rc + np.sum(dhT * hT, -1)[:, None] - f * dkk
+    np.testing.assert_allclose(dlf, alt, rtol=1e-10, atol=1e-10)
+
+
+def test_bwd_linear_in_dO():
+    rng = np.random.default_rng(10)
+    q, lf, x, h0 = _rand(rng, 1, 15, 2, 3, 3)
+    d1 = rng.standard_normal((1, 15, 2, 3))
+    d2 = rng.standard_normal((1, 15, 2, 3))
+    g1 = oracle.bwd(q, lf, x, d1, h0)
+    g2 = oracle.bwd(q, lf, x, d2, h0)
+    g12 = oracle.bwd(q, lf, x, 2 * d1 - 3 * d2, h0)
+    for a, b, c in zip(g1, g2, g12):
+        np.testing.assert_allclose(c, 2 * a - 3 * b, rtol=1e-11, atol=1e-11)
