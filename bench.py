@@ -1,0 +1,429 @@
+#!/usr/bin/env python3
+"""Benchmark of the HGRN2 hot path on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one training pass of the chunkwise recurrence over one batch: the
+forward (hgrn2_fwd) and the backward (hgrn2_bwd, gradients of q, log f and i)
+on the training workload B=8, H=16, T=2048, d_k=d_v=128, bf16 token tensors,
+fp32 state, forget-gate lower bound 0.95, dO ~ N(0,1).  Inputs (268 MB of
+token tensors per step, more than the 126 MB L2) are resident in HBM before
+the timed region.  Under torchrun each rank runs its own batch on its own GPU
+(data-parallel replicas, no collective on the data path): weak scaling.
+
+The same JSON line also carries the decode step (B=256, H=16, 1000 in-place
+steps of the fp32 state), end-to-end numbers through host buffers, the
+roofline of the dominant call, SM clocks sampled during the timed region, and
+the CPU oracle timed on a bounded sample (rank 0, one GPU only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "HGRN2 fwd+bwd tokens/s (H=16,d=128,T=2048) & % bf16 tensor peak; step GB/s"
+
+# Algorithmic counts per token per head (d_k = d_v = d = 128, chunk C = 64 for accounting,
+# causal half of the intra-chunk products, bf16 token tensors, state recompute not counted):
+D = 128
+C_ACC = 64
+FWD_FLOPS = C_ACC * (D + D) + 4 * D * D           # 81,920
+BWD_FLOPS = C_ACC * (3 * D + 2 * D) + 8 * D * D   # 172,032
+FWD_BYTES = 2 * (D + D + D + D)                   # read q, log f, i; write o = 1,024
+BWD_BYTES = 2 * (4 * D + 3 * D)                   # read q, log f, i, dO; write dq, dlog f, di = 1,792
+STEP_BYTES_PER_BH = 2 * D * D * 4 + 2 * (4 * D)   # decode: S read+write fp32, q/log f/i/o bf16 = 132,096
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def traffic_record(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src_hash = csrc_hash()
+    for line in open(p):
+        if line.startswith("#") or "|" not in line:
+            continue
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == kernel and cells[1] == src_hash:
+            try:
+                return float(cells[3])
+            except ValueError:
+                return None
+    return None
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "linear_attention_hgrn2_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(d, fn), "rb").read())
+    return h.hexdigest()[:12]
+
+
+# ------------------------------------------------------------------------------------------ ours
+def run_ours(args, world, rank, local):
+    import linear_attention_hgrn2_b200 as L
+    from linear_attention_hgrn2_b200 import inputs as I
+
+    L.load_library()
+    w = I.TRAIN
+    B, T, H, dk, dv, chunk = w.B, w.T, w.H, w.dk, w.dv, w.chunk
+    inp = I.make_workload(w, seed=1003 + rank)
+    dev = torch.device("cuda", local)
+    q, lf, x, dO = (inp[k].to(dev) for k in ("q", "log_f", "i", "dO"))
+    ws_f = torch.empty(max(L.workspace_size(B, T, H, dk, dv, chunk, w.dtype, False), 16), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(max(L.workspace_size(B, T, H, dk, dv, chunk, w.dtype, True), 16), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(x)
+
+    def step():
+        L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f)
+        return L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    L.counters(reset=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        t0.record(stream)
+        for k in range(K):
+            evs[k][0].record(stream)
+            L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f)
+            evs[k][1].record(stream)
+            L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b)
+            evs[k][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = L.counters()[2]
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_local, world)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_per_step = ms / K
+    tokens_per_step = B * T
+    value = world * tokens_per_step * K / (ms / 1e3)
+
+    pk = peaks()
+    th = B * T * H   # token-heads per step
+    if bwd_ms >= fwd_ms:
+        dom, dom_ms, dom_bytes = "hgrn2_bwd", bwd_ms, BWD_BYTES * th
+    else:
+        dom, dom_ms, dom_bytes = "hgrn2_fwd", fwd_ms, FWD_BYTES * th
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    tr = traffic_record(dom)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                "traffic": tr, "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)",
+                "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_ms": round(dom_ms, 4),
+                "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4)}
+    flops_step = (FWD_FLOPS + BWD_FLOPS) * th
+    bytes_step = (FWD_BYTES + BWD_BYTES) * th
+    tensor_frac = flops_step / (ms_per_step / 1e3) / (pk["bf16_tflops_sustained"] * 1e12)
+    step_roof = {"achieved_gbs": round(bytes_step / (ms_per_step / 1e3) / 1e9, 1),
+                 "hbm_frac": round(bytes_step / (ms_per_step / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+                 "algorithmic_tflops": round(flops_step / (ms_per_step / 1e3) / 1e12, 2),
+                 "bf16_peak_frac": round(tensor_frac, 4),
+                 "bf16_peak_tflops": pk["bf16_tflops_sustained"]}
+
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
+           "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": w.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv, "chunk": chunk,
+                      "lb": w.lb, "global_batch": B * world, "seq_len": T,
+                      "parallelism": f"dp{world} (independent replicas, no collective)",
+                      "l2": "no flush: 268 MB of token inputs per step > 126 MB L2"},
+           "roofline": roofline, "step_roofline": step_roof, "gpu_launches": launches,
+           "clocks": clk.summary()}
+
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, w, world)
+    if not args.no_decode:
+        out["decode_step"] = run_decode(args, dev, pk)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, w, world):
+    """Same step through host buffers: pinned H2D of the inputs and D2H of all outputs inside the timed region."""
+    import linear_attention_hgrn2_b200 as L
+    hq, hlf, hx, hdO = (t.cpu().pin_memory() for t in (q, lf, x, dO))
+    ho, hdq, hdlf, hdi = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, q, q, x))
+    dq_buf = torch.empty_like(q)
+    K = max(1, min(args.steps, 5))
+
+    def one():
+        q.copy_(hq, non_blocking=True); lf.copy_(hlf, non_blocking=True)
+        x.copy_(hx, non_blocking=True); dO.copy_(hdO, non_blocking=True)
+        L.fwd(q, lf, x, chunk=w.chunk, out=o, workspace=ws_f)
+        dq, dlf, di, _ = L.bwd(q, lf, x, dO, chunk=w.chunk, workspace=ws_b)
+        ho.copy_(o, non_blocking=True); hdq.copy_(dq, non_blocking=True)
+        hdlf.copy_(dlf, non_blocking=True); hdi.copy_(di, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(K):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hlf, hx, hdO))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdlf, hdi))
+    return {"value": round(world * w.B * w.T * K / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": round(ms / K, 3)}
+
+
+def run_decode(args, dev, pk):
+    """Decode workload: B=256, H=16, d=128, 1000 consecutive in-place steps (one timed sequence)."""
+    import linear_attention_hgrn2_b200 as L
+    from linear_attention_hgrn2_b200 import inputs as I
+    cfg = I.DECODE
+    steps = cfg["steps"]
+    d = I.make_decode(cfg["B"], cfg["H"], cfg["dk"], cfg["dv"], steps, cfg["dtype"], cfg["lb"],
+                      seed=1005, device=str(dev))
+    S = d["S"]
+    o = torch.empty((cfg["B"], cfg["H"], cfg["dv"]), dtype=cfg["dtype"], device=dev)
+    for t in range(5):
+        L.step(d["q"][t], d["log_f"][t], d["i"][t], S, out=o)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for t in range(steps):
+        L.step(d["q"][t], d["log_f"][t], d["i"][t], S, out=o)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    nbh = cfg["B"] * cfg["H"]
+    gbs = STEP_BYTES_PER_BH * nbh / (ms / 1e3) / 1e9
+    res = {"workload": cfg["name"], "ms_per_step": round(ms, 5), "tokens_per_s": round(cfg["B"] / (ms / 1e3), 1),
+           "achieved_gbs": round(gbs, 1), "peak_gbs": pk["hbm_gbs"], "frac": round(gbs / pk["hbm_gbs"], 4),
+           "bytes_per_step": STEP_BYTES_PER_BH * nbh, "steps": steps,
+           "l2": "state 268 MB > 126 MB L2, streaming loads/stores"}
+    del d, S
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline(inp, w, budget_s=15.0):
+    """The oracle (unchanged) on the host cores: fwd+bwd of whole (batch, head) sequences of the workload."""
+    import oracle
+    cores = oracle.num_threads()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    # time one pair to size the sample to about budget_s seconds of host time
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+
+    def run(sel):
+        bs = sorted({p[0] for p in sel})
+        hs = sorted({p[1] for p in sel})
+        sl = lambda t: f64(t[bs][:, :, hs].contiguous())
+        qq, ll, xx, gg = (sl(inp[k]) for k in ("q", "log_f", "i", "dO"))
+        t0 = time.perf_counter()
+        oracle.fwd(qq, ll, xx)
+        oracle.bwd(qq, ll, xx, gg)
+        return time.perf_counter() - t0, len(bs) * len(hs)
+
+    dt1, n1 = run(pairs[:1])
+    n_heads = max(1, min(w.H, int(budget_s / max(dt1, 1e-3))))
+    dt, n = run([(0, h) for h in range(n_heads)])
+    tok = n * w.T / w.H                       # token-head sequences -> tokens of all H heads
+    return {"value": round(tok / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fwd+bwd of {n} whole (batch,head) sequences (T={w.T}, d=128) of the workload, "
+                      f"fp64 C oracle, OpenMP over (batch,head); {dt:.2f} s",
+            "seconds": round(dt, 3)}
+
+
+# ------------------------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: same metric and config, bounded samples per step, host cores."""
+    if rank != 0:
+        return
+    import oracle
+    from linear_attention_hgrn2_b200 import inputs as I
+    w = I.TRAIN
+    inp = I.make_workload(w, seed=1003)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    cores = oracle.num_threads()
+    heads = max(1, min(w.H, cores))
+    sl = lambda t: f64(t[:1, :, :heads].contiguous())
+    qq, ll, xx, gg = (sl(inp[k]) for k in ("q", "log_f", "i", "dO"))
+
+    def one():
+        oracle.fwd(qq, ll, xx)
+        oracle.bwd(qq, ll, xx, gg)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = time.perf_counter() - t0
+    tok = args.steps * heads * w.T / w.H
+    value = tok / dt
+    sample = (f"each step: fwd+bwd of {heads} whole (batch,head) sequences (T={w.T}, d=128) of the workload "
+              f"on the fp64 C oracle")
+    out = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                      "chunk": w.chunk, "lb": w.lb, "global_batch": w.B, "seq_len": w.T,
+                      "parallelism": "host cores (OpenMP over batch,head)"},
+           "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

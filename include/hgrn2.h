@@ -1,0 +1,141 @@
+/*
+ * hgrn2.h -- C ABI of the B200 (sm_100a) HGRN2 recurrence library (libhgrn2.so).
+ *
+ * The operation ("HGRN2: Gated Linear RNNs with State Expansion", Qin et al.
+ * 2024, arXiv 2404.07904; section numbers refer to the paper as summarised on
+ * the paperlayer.ai page):
+ *
+ *   per batch b and head h (heads are independent, §3.2 "multihead"), with a
+ *   d_k x d_v fp32 state S (row j = key dimension):
+ *
+ *     f_t = exp(log_f_t)                        forget gate, one per key dim (§5)
+ *     k_t = 1 - f_t = -expm1(log_f_t)           input gate tied to forget gate (§2.1)
+ *     S_t = Diag(f_t) S_{t-1} + k_t i_t^T       outer-product state expansion (§3.2)
+ *     o_t = S_t^T q_t                           matrix-vector output, UPDATED state (§3.2)
+ *
+ *   Read as gated linear attention (§3.2: same recurrence as GLA up to the
+ *   parameterisation) with key k = 1 - f, value v = i and query q, it is
+ *   computed chunkwise on tensor cores.  There is no 1/sqrt(d) scale, no
+ *   normalisation and no output gate inside the library.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layouts (row-major, innermost last, no padding):
+ *      token tensors q, log_f, dlog_f, dq : [B][T][H][d_k]
+ *                    i, o, dO, di         : [B][T][H][d_v]
+ *      states        h0, hT, dhT, dh0, S  : [B][H][d_k][d_v]   always float32
+ *      decode tensors q, log_f            : [B][H][d_k];  i, o : [B][H][d_v]
+ *  - dtype (hgrn2_dtype) is the element type of all token tensors (inputs and
+ *    outputs alike).  States are always float32.
+ *  - All data pointers are DEVICE pointers owned by the caller, aligned to 16
+ *    bytes.  The library allocates no memory, never synchronises inside
+ *    hgrn2_fwd / hgrn2_bwd / hgrn2_step, and keeps no pointer after a call.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
+ *    stream).  Argument checks run on the host before anything is launched: a
+ *    call that returns an error has launched nothing.  A launch failure reported
+ *    by the CUDA runtime returns HGRN2_ERR_CUDA.
+ *  - No exception or abort crosses this ABI.
+ *  - Supported sizes: B, H >= 1; T >= 0 (T = 0 writes hT = h0 and nothing else);
+ *    1 <= d_k, d_v <= 128; chunk in {16, 32, 64, 128}.  The bf16 tensor-core
+ *    path is used when dtype = BF16 and d_k = d_v = 128; every other supported
+ *    shape runs the exact CUDA-core path.  Unsupported shapes return
+ *    HGRN2_ERR_UNSUPPORTED.
+ *  - `chunk` is the length of the chunks of the chunkwise algorithm (§3.2);
+ *    results do not depend on it beyond rounding.  The CUDA-core path caps it at
+ *    what fits in shared memory for the given d_k, d_v.
+ *  - log_f must be finite and <= 0 (f in (0, 1]); other values are outside the
+ *    method's range and their results are unspecified (no fault).
+ *  - Ragged T (not a multiple of the chunk) is handled; the tail is computed
+ *    exactly like any other token.
+ */
+#ifndef HGRN2_H
+#define HGRN2_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HGRN2_OK = 0,
+    HGRN2_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, bad alignment, short workspace */
+    HGRN2_ERR_UNSUPPORTED = 2,   /* valid but unsupported shape / chunk / dtype combination */
+    HGRN2_ERR_CUDA = 3,          /* the CUDA runtime reported an error at launch */
+    HGRN2_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up (see hgrn2_get_device_status) */
+    HGRN2_ERR_DEVICE = 5         /* a device-side consistency check failed (see hgrn2_get_device_status) */
+} hgrn2_status;
+
+typedef enum {
+    HGRN2_FP32 = 0,
+    HGRN2_BF16 = 1
+} hgrn2_dtype;
+
+/* Bytes of device workspace that hgrn2_fwd (want_bwd = 0) or hgrn2_bwd
+ * (want_bwd = 1) needs for these sizes.  May be 0.  Returns (size_t)-1 for
+ * invalid or unsupported arguments.  Host-only, no CUDA call. */
+size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
+                            hgrn2_dtype dtype, int want_bwd);
+
+/* Forward over a whole sequence (§3.2 recurrence above, chunkwise).
+ *   q, log_f : [B,T,H,dk]   i : [B,T,H,dv]          (dtype)
+ *   h0       : [B,H,dk,dv] float32 initial state, or NULL for zeros
+ *   o        : [B,T,H,dv] output (dtype)
+ *   hT       : [B,H,dk,dv] float32 final state S_{T-1}, or NULL to skip
+ *   workspace: device scratch of at least hgrn2_workspace_size(..., 0) bytes
+ *              (may be NULL when that size is 0); contents need no initialisation
+ *              and are undefined afterwards.
+ * Inputs must not alias outputs. */
+hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const float *h0,
+                       void *o, float *hT,
+                       int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                       void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Backward of L(o, hT) through the forward above, given dO = dL/do and an
+ * optional dhT = dL/dhT (NULL = 0).  Writes dq, dlog_f, di (dtype, same layouts
+ * as q, log_f, i) and, when dh0 != NULL, dh0 = dL/dh0 (float32).  h0 must be the
+ * forward's initial state (NULL = zeros).  The gradient of log_f includes both
+ * paths through which it acts: the decay Diag(f) and the tied input gate
+ * k = 1 - f (§2.1).  workspace: at least hgrn2_workspace_size(..., 1) bytes.
+ * dq must not alias any input: the backward reads dq back after writing it. */
+hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const float *h0,
+                       const void *dO, const float *dhT,
+                       void *dq, void *dlog_f, void *di, float *dh0,
+                       int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                       void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* One recurrent decode step for B sequences with one new token each (§1: linear-
+ * time recurrent inference without a KV cache; the §3.2 recurrence for one t):
+ *   S <- Diag(f) S + k i^T  (in place, float32),  then  o = S^T q.
+ *   q, log_f : [B,H,dk]   i, o : [B,H,dv]   (dtype)     S : [B,H,dk,dv] float32
+ * S must not alias q, log_f, i or o.  dv must be a multiple of 4. */
+hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *S, void *o,
+                        int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
+
+/* Synchronises `stream`, then returns and clears the library's device-side
+ * status word of the current device: HGRN2_OK, HGRN2_ERR_TIMEOUT (a bounded
+ * wait gave up) or HGRN2_ERR_DEVICE (a consistency check failed).  Returns
+ * HGRN2_ERR_CUDA if the synchronisation itself fails. */
+hgrn2_status hgrn2_get_device_status(cudaStream_t stream);
+
+/* Diagnostic counters, accumulated since the last reset:
+ *   out[0] = (batch, head) passes that took the exact CUDA-core route because a
+ *            chunk's cumulative log-decay spanned more than the tensor-core
+ *            factorisation allows (device counter of the current device);
+ *   out[1] = tensor-core chunk passes completed (device counter);
+ *   out[2] = kernel launches issued by this library in this process (host count).
+ * Synchronises `stream`.  n = number of entries of `out` (<= 3 are written).
+ * reset != 0 zeroes the counters after reading them. */
+hgrn2_status hgrn2_get_counters(long long *out, int n, int reset, cudaStream_t stream);
+
+/* Static English description of a status code (never NULL). */
+const char *hgrn2_status_string(hgrn2_status s);
+
+/* Library version, e.g. "hgrn2-b200 0.1". */
+const char *hgrn2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HGRN2_H */

@@ -1,0 +1,228 @@
+"""Python binding of libhgrn2.so, the B200 (sm_100a) HGRN2 recurrence library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/hgrn2.h``.  PyTorch supplies
+device memory and the current CUDA stream.  There is no CPU fallback: if the
+shared library is missing or cannot be loaded, every call raises.
+
+Per batch b and head h, with f = exp(log_f) and k = 1 - f ("HGRN2: Gated
+Linear RNNs with State Expansion", §2.1, §3.2):
+
+    S_t = Diag(f_t) S_{t-1} + k_t i_t^T,      o_t = S_t^T q_t
+
+Token tensors are [B, T, H, D]; states [B, H, d_k, d_v] float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhgrn2.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(6)
+FP32, BF16 = 0, 1
+
+# Every extern "C" symbol of include/hgrn2.h.
+EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_step",
+           "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
+
+_lib = None
+
+
+class HGRN2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libhgrn2.so (raises if it is absent: build it with
+    ``python -m linear_attention_hgrn2_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libhgrn2.so not found at {path}; run `python -m linear_attention_hgrn2_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.hgrn2_workspace_size.argtypes = [i32] * 7 + [i32]
+    lib.hgrn2_workspace_size.restype = sz
+    lib.hgrn2_fwd.argtypes = [vp] * 6 + [i32] * 7 + [vp, sz, vp]
+    lib.hgrn2_fwd.restype = i32
+    lib.hgrn2_bwd.argtypes = [vp] * 10 + [i32] * 7 + [vp, sz, vp]
+    lib.hgrn2_bwd.restype = i32
+    lib.hgrn2_step.argtypes = [vp] * 5 + [i32] * 5 + [vp]
+    lib.hgrn2_step.restype = i32
+    lib.hgrn2_get_device_status.argtypes = [vp]
+    lib.hgrn2_get_device_status.restype = i32
+    lib.hgrn2_get_counters.argtypes = [ctypes.POINTER(ctypes.c_longlong), i32, i32, vp]
+    lib.hgrn2_get_counters.restype = i32
+    lib.hgrn2_status_string.argtypes = [i32]
+    lib.hgrn2_status_string.restype = ctypes.c_char_p
+    lib.hgrn2_version.argtypes = []
+    lib.hgrn2_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().hgrn2_status_string(status).decode()
+
+
+def version() -> str:
+    return load_library().hgrn2_version().decode()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _raise(status: int, where: str):
+    if status != OK:
+        raise HGRN2Error(status, where)
+
+
+def workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, want_bwd=False) -> int:
+    n = load_library().hgrn2_workspace_size(B, T, H, dk, dv, chunk,
+                                            BF16 if dtype == torch.bfloat16 else FP32, int(want_bwd))
+    if n == ctypes.c_size_t(-1).value:
+        raise HGRN2Error(ERR_INVALID_ARG, "hgrn2_workspace_size")
+    return int(n)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def fwd(q, log_f, i, h0=None, want_hT=False, chunk=64, out=None, workspace=None):
+    """o = HGRN2(q, log_f, i; h0) and optionally the final state hT.
+
+    q, log_f: [B,T,H,dk]; i: [B,T,H,dv] (float32 or bfloat16, all the same);
+    h0: [B,H,dk,dv] float32 or None.  Returns (o, hT or None)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = i.shape[-1]
+    _check(q, "q")
+    _check(log_f, "log_f", q.dtype, q.shape)
+    _check(i, "i", q.dtype, (B, T, H, dv))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    o = out if out is not None else torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _check(o, "o", q.dtype, (B, T, H, dv))
+    hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_hT else None
+    nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, False)
+    ws = workspace if workspace is not None else _workspace(nws, q.device)
+    st = lib.hgrn2_fwd(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(o), _ptr(hT),
+                       B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
+    _raise(st, "hgrn2_fwd")
+    return o, hT
+
+
+def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dh0=False, chunk=64, workspace=None):
+    """Gradients (dq, dlog_f, di, dh0 or None) of L(o, hT) given dO (and dhT)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = i.shape[-1]
+    _check(q, "q")
+    _check(log_f, "log_f", q.dtype, q.shape)
+    _check(i, "i", q.dtype, (B, T, H, dv))
+    _check(dO, "dO", q.dtype, (B, T, H, dv))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    if dhT is not None:
+        _check(dhT, "dhT", torch.float32, (B, H, dk, dv))
+    dq = torch.empty_like(q)
+    dlf = torch.empty_like(q)
+    di = torch.empty_like(i)
+    dh0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
+    nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, True)
+    ws = workspace if workspace is not None else _workspace(nws, q.device)
+    st = lib.hgrn2_bwd(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(dO), _ptr(dhT),
+                       _ptr(dq), _ptr(dlf), _ptr(di), _ptr(dh0),
+                       B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
+    _raise(st, "hgrn2_bwd")
+    return dq, dlf, di, dh0
+
+
+def step(q, log_f, i, S, out=None):
+    """One decode step: S <- Diag(f) S + k i^T in place; returns o = S^T q.
+
+    q, log_f: [B,H,dk]; i: [B,H,dv]; S: [B,H,dk,dv] float32 (updated in place)."""
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = i.shape[-1]
+    _check(q, "q")
+    _check(log_f, "log_f", q.dtype, q.shape)
+    _check(i, "i", q.dtype, (B, H, dv))
+    _check(S, "S", torch.float32, (B, H, dk, dv))
+    o = out if out is not None else torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = lib.hgrn2_step(_ptr(q), _ptr(log_f), _ptr(i), _ptr(S), _ptr(o), B, H, dk, dv, _dt(q), _stream())
+    _raise(st, "hgrn2_step")
+    return o
+
+
+def device_status() -> int:
+    """Synchronises the current stream; returns and clears the device status word."""
+    return int(load_library().hgrn2_get_device_status(_stream()))
+
+
+def counters(reset: bool = False) -> list[int]:
+    """[exact-route (batch, head) passes, tensor-core chunk passes, kernel launches issued]
+    since the last reset (synchronises the current stream)."""
+    out = (ctypes.c_longlong * 3)()
+    _raise(load_library().hgrn2_get_counters(out, 3, int(reset), _stream()), "hgrn2_get_counters")
+    return [int(out[0]), int(out[1]), int(out[2])]
+
+
+class HGRN2Function(torch.autograd.Function):
+    """Autograd wrapper: o, hT = HGRN2Function.apply(q, log_f, i, h0, chunk)."""
+
+    @staticmethod
+    def forward(ctx, q, log_f, i, h0=None, chunk=64):
+        o, hT = fwd(q.contiguous(), log_f.contiguous(), i.contiguous(),
+                    None if h0 is None else h0.contiguous(), want_hT=True, chunk=chunk)
+        ctx.save_for_backward(q, log_f, i, h0)
+        ctx.chunk = chunk
+        ctx.has_h0 = h0 is not None
+        return o, hT
+
+    @staticmethod
+    def backward(ctx, dO, dhT):
+        q, log_f, i, h0 = ctx.saved_tensors
+        dq, dlf, di, dh0 = bwd(q, log_f, i, dO.contiguous(), h0,
+                               None if dhT is None else dhT.contiguous(),
+                               want_dh0=ctx.has_h0, chunk=ctx.chunk)
+        return dq, dlf, di, dh0, None
+
+
+def hgrn2(q, log_f, i, h0=None, chunk=64):
+    """Differentiable HGRN2 recurrence: returns (o, hT)."""
+    return HGRN2Function.apply(q, log_f, i, h0, chunk)

@@ -1,0 +1,171 @@
+// api.cu -- the extern "C" boundary of libhgrn2.so (declared in include/hgrn2.h).
+//
+// Host-side argument validation, workspace planning and dispatch between the
+// bf16 tensor-core kernels and the exact CUDA-core kernels.  Nothing here
+// allocates device memory or synchronises, except the two status/counter
+// queries, which synchronise the given stream by contract.
+#include <stdint.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace hgrn2;
+
+namespace {
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool chunk_ok(int chunk) { return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128; }
+
+// Largest chunk <= requested whose exact-route shared memory fits.
+int simt_chunk(int chunk, int dk, int dv, bool bwd) {
+    for (int C = chunk; C >= 16; C >>= 1) {
+        size_t s = bwd ? (simt_bwd_dq_smem(C, dk, dv) > simt_bwd_rev_smem(C, dk, dv)
+                              ? simt_bwd_dq_smem(C, dk, dv)
+                              : simt_bwd_rev_smem(C, dk, dv))
+                       : simt_fwd_smem(C, dk, dv);
+        if (s <= kMaxSmem) return C;
+    }
+    return 0;
+}
+
+hgrn2_status check_common(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt) {
+    if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
+    if (dt != HGRN2_FP32 && dt != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
+    if (!chunk_ok(chunk)) return HGRN2_ERR_UNSUPPORTED;
+    if (dk > 128 || dv > 128) return HGRN2_ERR_UNSUPPORTED;
+    // index arithmetic is 64-bit; keep grid dimensions and per-tensor element counts sane
+    if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    return HGRN2_OK;
+}
+
+size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd) {
+    (void)T; (void)dv; (void)chunk; (void)dt;
+    size_t bytes = 0;
+    if (want_bwd) bytes += sizeof(float) * (size_t)B * H * dk;   // rowsum(dhT * hT)
+    return (bytes + 255) & ~(size_t)255;
+}
+
+hgrn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HGRN2_OK : HGRN2_ERR_CUDA; }
+
+std::atomic<long long> g_launches{0};   // kernel launches issued (host side)
+
+}  // namespace
+
+extern "C" {
+
+size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                            int want_bwd) {
+    if (check_common(B, T, H, dk, dv, chunk, dtype) != HGRN2_OK) return (size_t)-1;
+    return ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, want_bwd);
+}
+
+hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o,
+                       float *hT, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                       void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    if (T > 0 && (!q || !log_f || !i || !o)) return HGRN2_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, log_f, i, h0, o, hT, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 0);
+    if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
+    const bool bf16 = dtype == HGRN2_BF16;
+    if (T == 0) {
+        if (!hT) return HGRN2_OK;
+        size_t n = sizeof(float) * (size_t)B * H * dk * dv;
+        cudaError_t e = h0 ? cudaMemcpyAsync(hT, h0, n, cudaMemcpyDeviceToDevice, stream)
+                           : cudaMemsetAsync(hT, 0, n, stream);
+        return from_cuda(e);
+    }
+    int C = simt_chunk(chunk, dk, dv, false);
+    if (!C) return HGRN2_ERR_UNSUPPORTED;
+    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C};
+    g_launches += 1;
+    return from_cuda(launch_simt_fwd(a, bf16, stream));
+}
+
+hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *dO,
+                       const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B, int T,
+                       int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                       size_t ws_bytes, cudaStream_t stream) {
+    hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    if (T > 0 && (!q || !log_f || !i || !dO || !dq || !dlog_f || !di)) return HGRN2_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
+    if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
+    const bool bf16 = dtype == HGRN2_BF16;
+    if (T == 0) {
+        if (!dh0) return HGRN2_OK;
+        size_t n = sizeof(float) * (size_t)B * H * dk * dv;
+        cudaError_t e = dhT ? cudaMemcpyAsync(dh0, dhT, n, cudaMemcpyDeviceToDevice, stream)
+                            : cudaMemsetAsync(dh0, 0, n, stream);
+        return from_cuda(e);
+    }
+    int C = simt_chunk(chunk, dk, dv, true);
+    if (!C) return HGRN2_ERR_UNSUPPORTED;
+    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, (float *)workspace, B, T, H, dk, dv, C};
+    g_launches += 2;
+    return from_cuda(launch_simt_bwd(a, bf16, stream));
+}
+
+hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *S, void *o, int B, int H,
+                        int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
+    if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
+    if (dk > 128 || dv > 128 || (dv & 3)) return HGRN2_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    if (!q || !log_f || !i || !S || !o) return HGRN2_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, log_f, i, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    g_launches += 1;
+    return from_cuda(launch_step(q, log_f, i, S, o, B, H, dk, dv, dtype == HGRN2_BF16, stream));
+}
+
+hgrn2_status hgrn2_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return HGRN2_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return HGRN2_ERR_CUDA;
+    return (hgrn2_status)v;
+}
+
+hgrn2_status hgrn2_get_counters(long long *out, int n, int reset, cudaStream_t stream) {
+    if (!out || n < 0) return HGRN2_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+    unsigned long long c[2] = {0, 0};
+    if (cudaMemcpyFromSymbol(c, g_counters, sizeof(c)) != cudaSuccess) return HGRN2_ERR_CUDA;
+    for (int k = 0; k < n && k < 2; ++k) out[k] = (long long)c[k];
+    if (n > 2) out[2] = g_launches.load();
+    if (reset) {
+        unsigned long long z[2] = {0, 0};
+        if (cudaMemcpyToSymbol(g_counters, z, sizeof(z)) != cudaSuccess) return HGRN2_ERR_CUDA;
+        g_launches = 0;
+    }
+    return HGRN2_OK;
+}
+
+const char *hgrn2_status_string(hgrn2_status s) {
+    switch (s) {
+        case HGRN2_OK: return "ok";
+        case HGRN2_ERR_INVALID_ARG: return "invalid argument";
+        case HGRN2_ERR_UNSUPPORTED: return "unsupported shape, chunk or dtype";
+        case HGRN2_ERR_CUDA: return "CUDA runtime error";
+        case HGRN2_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        case HGRN2_ERR_DEVICE: return "a device-side consistency check failed";
+    }
+    return "unknown status";
+}
+
+const char *hgrn2_version(void) { return "hgrn2-b200 0.1"; }
+
+}  // extern "C"

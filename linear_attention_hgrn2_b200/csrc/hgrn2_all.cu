@@ -1,0 +1,8 @@
+// hgrn2_all.cu -- single translation unit of libhgrn2.so.
+//
+// The kernels share the device-side status word and counters defined in
+// api.cu; compiling them as one unit keeps those references plain (no
+// relocatable device code or device link step).
+#include "api.cu"
+#include "simt.cu"
+#include "step.cu"

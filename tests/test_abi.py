@@ -1,0 +1,91 @@
+"""The C-ABI library loads and exports every symbol include/hgrn2.h declares.
+
+CPU-only: no call here launches anything or touches a CUDA device (only the
+host-side size query and string functions are called).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import linear_attention_hgrn2_b200 as L
+from linear_attention_hgrn2_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hgrn2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hgrn2_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("hgrn2_fwd", "hgrn2_bwd", "hgrn2_step", "hgrn2_workspace_size", "hgrn2_status_string"):
+        assert n in names
+    assert set(names) == set(L.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s(hgrn2_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_status_strings_and_version(lib):
+    for s in range(6):
+        assert isinstance(L.status_string(s), str) and L.status_string(s)
+    assert L.status_string(99) == "unknown status"
+    assert L.version().startswith("hgrn2-b200")
+
+
+def test_workspace_size_rejects_bad_arguments(lib):
+    bad = ctypes.c_size_t(-1).value
+    f = lib.hgrn2_workspace_size
+    assert f(0, 16, 1, 16, 16, 16, 0, 0) == bad          # B < 1
+    assert f(1, -1, 1, 16, 16, 16, 0, 0) == bad          # T < 0
+    assert f(1, 16, 1, 256, 16, 16, 0, 0) == bad         # d_k > 128
+    assert f(1, 16, 1, 16, 16, 48, 0, 0) == bad          # chunk not a power of two in [16,128]
+    assert f(1, 16, 1, 16, 16, 16, 7, 0) == bad          # unknown dtype
+    assert f(1, 16, 1, 16, 16, 16, 0, 0) != bad
+    assert f(8, 2048, 16, 128, 128, 64, 1, 1) != bad
+
+
+def test_bad_arguments_return_errors_before_any_launch(lib):
+    # invalid sizes and null pointers are rejected on the host: no CUDA call is made
+    vp = ctypes.c_void_p
+    st = lib.hgrn2_fwd(None, None, None, None, None, None, 0, 16, 1, 16, 16, 16, 0, None, 0, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_fwd(None, None, None, None, None, None, 1, 16, 1, 16, 16, 16, 0, None, 0, None)
+    assert st == L.ERR_INVALID_ARG       # null q
+    st = lib.hgrn2_fwd(vp(16), vp(16), vp(16), None, vp(16), None, 1, 16, 1, 16, 16, 24, 0, None, 0, None)
+    assert st == L.ERR_UNSUPPORTED       # chunk
+    st = lib.hgrn2_fwd(vp(17), vp(16), vp(16), None, vp(16), None, 1, 16, 1, 16, 16, 16, 0, None, 0, None)
+    assert st == L.ERR_INVALID_ARG       # misaligned
+    st = lib.hgrn2_step(vp(16), vp(16), vp(16), vp(16), vp(16), 1, 1, 16, 6, 0, None)
+    assert st == L.ERR_UNSUPPORTED       # d_v not a multiple of 4
+    st = lib.hgrn2_bwd(*([None] * 10), 1, 8, 1, 16, 16, 16, 1, None, 0, None)
+    assert st == L.ERR_INVALID_ARG
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "linear_attention_hgrn2_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, fn
+                assert "liboracle" not in txt, fn

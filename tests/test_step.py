@@ -1,0 +1,58 @@
+"""GPU parity of the decode step (hgrn2_step) against the oracle, plus step-vs-fwd."""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_hgrn2_b200 as L
+from linear_attention_hgrn2_b200 import inputs as I
+from parity_util import err, np64, tol
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,B,H,dk,dv,steps", [
+    (torch.bfloat16, 4, 3, 128, 128, 30),
+    (torch.float32, 2, 2, 16, 16, 30),
+    (torch.float32, 3, 2, 64, 32, 10),
+    (torch.bfloat16, 2, 2, 100, 12, 10),
+])
+def test_step_matches_oracle(cuda, dtype, B, H, dk, dv, steps):
+    d = I.make_decode(B, H, dk, dv, steps, dtype, 0.8, seed=11)
+    S = d["S"].cuda()
+    S_ref = np64(d["S"])
+    for t in range(steps):
+        o = L.step(d["q"][t].cuda(), d["log_f"][t].cuda(), d["i"][t].cuda(), S)
+        o_ref, S_ref = oracle.step(np64(d["q"][t]), np64(d["log_f"][t]), np64(d["i"][t]), S_ref)
+        assert err(np64(o), o_ref, dtype) <= tol(dtype), t
+    assert err(np64(S), S_ref, dtype) <= tol(dtype)
+
+
+def test_decode_workload_full_size_sampled(cuda):
+    w = I.DECODE
+    steps = 4
+    d = I.make_decode(w["B"], w["H"], w["dk"], w["dv"], steps, w["dtype"], w["lb"], seed=1005)
+    S = d["S"].cuda()
+    pairs = [(0, 0), (17, 3), (255, 15)]
+    S_ref = {p: np64(d["S"][p[0]:p[0] + 1, p[1]:p[1] + 1]) for p in pairs}
+    for t in range(steps):
+        o = L.step(d["q"][t].cuda(), d["log_f"][t].cuda(), d["i"][t].cuda(), S)
+        for (b, h) in pairs:
+            sl = lambda x: np64(x[t][b:b + 1, h:h + 1])
+            o_ref, S_ref[(b, h)] = oracle.step(sl(d["q"]), sl(d["log_f"]), sl(d["i"]), S_ref[(b, h)])
+            assert err(np64(o[b:b + 1, h:h + 1]), o_ref, w["dtype"]) <= tol(w["dtype"])
+    for (b, h) in pairs:
+        assert err(np64(S[b:b + 1, h:h + 1]), S_ref[(b, h)], torch.float32) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_steps_equal_fwd(cuda, dtype):
+    B, T, H, d = 2, 40, 3, 128
+    inp = I.make_inputs(B, T, H, d, d, dtype, 0.5, seed=3, h0_sigma=0.1)
+    g = {k: v.cuda() for k, v in inp.items()}
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=16 if dtype == torch.float32 else 64)
+    S = g["h0"].clone()
+    for t in range(T):
+        ot = L.step(g["q"][:, t].contiguous(), g["log_f"][:, t].contiguous(), g["i"][:, t].contiguous(), S)
+        assert err(np64(ot), np64(o[:, t]), dtype) <= tol(dtype)
+    assert err(np64(S), np64(hT), torch.float32) <= (1e-5 if dtype == torch.float32 else 1e-2)
