@@ -43,11 +43,17 @@ hgrn2_status check_common(int B, int T, int H, int dk, int dv, int chunk, hgrn2_
     return HGRN2_OK;
 }
 
+// The bf16 tensor-core route takes d_k = d_v = 128; everything else runs the exact route.
+bool use_tc(int dk, int dv, hgrn2_dtype dt) { return dt == HGRN2_BF16 && dk == 128 && dv == 128; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
 size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd) {
-    (void)T; (void)dv; (void)chunk; (void)dt;
+    (void)T; (void)chunk;
     size_t bytes = 0;
-    if (want_bwd) bytes += sizeof(float) * (size_t)B * H * dk;   // rowsum(dhT * hT)
-    return (bytes + 255) & ~(size_t)255;
+    if (want_bwd) bytes += align256(sizeof(float) * (size_t)B * H * dk);   // rowsum(dhT * hT)
+    else if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
+    return bytes;
 }
 
 hgrn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HGRN2_OK : HGRN2_ERR_CUDA; }
@@ -85,7 +91,18 @@ hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const fl
     }
     int C = simt_chunk(chunk, dk, dv, false);
     if (!C) return HGRN2_ERR_UNSUPPORTED;
-    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C};
+    if (use_tc(dk, dv, dtype)) {
+        // tensor-core pass; (b,h) pairs whose chunk decay span is too wide are flagged
+        // and recomputed right after by the exact route (same stream, in order)
+        int *flags = (int *)workspace;
+        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, B, T, H};
+        g_launches += 2;
+        cudaError_t e = launch_tc_fwd(t, stream);
+        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+        SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags};
+        return from_cuda(launch_simt_fwd(a, bf16, stream));
+    }
+    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr};
     g_launches += 1;
     return from_cuda(launch_simt_fwd(a, bf16, stream));
 }

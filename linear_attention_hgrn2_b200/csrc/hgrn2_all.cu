@@ -6,3 +6,4 @@
 #include "api.cu"
 #include "simt.cu"
 #include "step.cu"
+#include "tc_fwd.cu"

@@ -12,6 +12,16 @@ struct SimtFwdArgs {
     void *o;
     float *hT;
     int B, T, H, dk, dv, C;
+    const int *only;   // if non-null: only (b,h) with only[b*H+h] != 0 are computed
+};
+
+struct TcFwdArgs {
+    const void *q, *lf, *x;
+    const float *h0;
+    void *o;
+    float *hT;
+    int *flags;        // [B*H] out: 1 where the (b,h) needs the exact route
+    int B, T, H;
 };
 
 struct SimtBwdArgs {
@@ -28,6 +38,9 @@ size_t simt_bwd_dq_smem(int C, int dk, int dv);
 size_t simt_bwd_rev_smem(int C, int dk, int dv);
 cudaError_t launch_simt_fwd(const SimtFwdArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_bwd(const SimtBwdArgs &a, bool bf16, cudaStream_t st);
+
+size_t tc_fwd_smem();
+cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st);
 
 cudaError_t launch_step(const void *q, const void *lf, const void *x, float *S, void *o, int B, int H,
                         int dk, int dv, bool bf16, cudaStream_t st);

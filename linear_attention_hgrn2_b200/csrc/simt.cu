@@ -71,7 +71,8 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
-                int T_, int H, int dk, int dv, int C) {
+                int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+    if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;              // [C][ldk]  q, then q * e^{b}
@@ -337,7 +338,7 @@ static cudaError_t launch_simt_fwd_t(const SimtFwdArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<a.B * a.H, kSimtThreads, smem, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x, a.h0,
-                                             (T *)a.o, a.hT, a.T, a.H, a.dk, a.dv, a.C);
+                                             (T *)a.o, a.hT, a.T, a.H, a.dk, a.dv, a.C, a.only);
     return cudaGetLastError();
 }
 

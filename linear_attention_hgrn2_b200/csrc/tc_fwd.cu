@@ -1,0 +1,422 @@
+// tc_fwd.cu -- chunkwise HGRN2 forward on 5th-generation tensor cores (sm_100a).
+//
+// One CTA walks the 128-token chunks of one (batch, head) (or of one segment of
+// it); d_k = d_v = 128, bf16 token tensors, fp32 state.  Per chunk, with
+// E_t = prod_{r<=t} f_r (cumulative inside the chunk, per key dim j),
+// k = 1 - f, S_in the state entering the chunk and E_B = E at the chunk end
+// ("HGRN2: Gated Linear RNNs with State Expansion", §3.2: gated linear attention
+// with key 1 - f, value i, query q, so chunkwise; §5: per-dimension decay):
+//
+//   Qt = q * E,  Kt = k / E,  Kh = Kt * E_B = k * E_B / E     (all bf16 in smem)
+//   A  = mask_{s<=t}(Qt Kt^T)                                  tcgen05, fp32 in TMEM
+//   O  = Qt bf16(S_in) + bf16(A) V                             tcgen05, fp32 in TMEM
+//   S  = Diag(E_B) S_in + Kh^T V                               fp32 state in TMEM
+//
+// Qt Kt^T realises sum_j q_t[j] k_s[j] exp(b_t[j] - b_s[j]) through factors
+// referenced to the chunk start; it is valid while 1/E stays representable with
+// margin, i.e. min_j E_B[j] >= 1e-26 (a cumulative log-decay span of about 60
+// inside the chunk).  A (batch, head) meeting a chunk beyond that is flagged and
+// recomputed afterwards by the exact CUDA-core route, which forms every
+// exponent as a difference of cumulative sums.
+//
+// Data movement: q, log f, i tiles arrive by TMA (128-byte swizzle, two
+// 64-column boxes per 128 x 128 tile) into a two-stage ring, so the next chunk
+// loads while this one computes; o leaves by TMA store.  The state never leaves
+// TMEM between chunks (d_k lanes x d_v fp32 columns); Diag(E_B) is a per-lane
+// scale applied with tcgen05.ld/st.  The MMAs are issued by one thread;
+// completion is tracked with tcgen05.commit on mbarriers.  Every wait is bounded.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace hgrn2 {
+namespace tcf {
+
+using namespace tc;
+
+constexpr int kThreads = 256;
+constexpr int kTile = 128;               // tokens per chunk
+constexpr int kTileBytes = 128 * 128 * 2;
+constexpr int kBlk = 128 * 128;          // bytes of one 64-column block of a 128-row tile
+constexpr uint32_t kColS = 0, kColO = 128, kColA = 256, kTmemCols = 512;
+constexpr float kMinEB = 1e-26f;
+
+struct __align__(8) Misc {
+    uint64_t full[2];
+    uint64_t barA, barO1, barM;
+    uint32_t tmem_base;
+    int bad;
+    float EB[128];
+    float Ppart[4][128];
+};
+
+constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
+
+struct Params {
+    const float *h0;
+    float *hT;
+    int *flags;     // [B*H] set to 1 when the (b,h) must take the exact route
+    int T, H, ntiles;
+};
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// 1 - exp(a) given f = exp(a): Taylor series of -expm1 for |a| < 0.25 (relative
+// truncation error < 1.5e-6), 1 - f otherwise (no cancellation there).
+__device__ __forceinline__ float k_from(float a, float f) {
+    if (fabsf(a) < 0.25f) {
+        float p = fmaf(a, 1.0f / 120.0f, 1.0f / 24.0f);
+        p = fmaf(p, a, 1.0f / 6.0f);
+        p = fmaf(p, a, 0.5f);
+        p = fmaf(p, a, 1.0f);
+        return -a * p;
+    }
+    return 1.0f - f;
+}
+
+// Row j (lane) of a 64-column half of a TMEM tile -> bf16 row in a swizzled smem block.
+__device__ __forceinline__ void store_row_bf16(uint8_t *blk, int row, const float (&r0)[32], const float (&r1)[32]) {
+    uint8_t *base = blk + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const float *src = c < 4 ? &r0[c * 8] : &r1[(c - 4) * 8];
+        uint4 v;
+        v.x = pack_bf2(src[0], src[1]);
+        v.y = pack_bf2(src[2], src[3]);
+        v.z = pack_bf2(src[4], src[5]);
+        v.w = pack_bf2(src[6], src[7]);
+        *reinterpret_cast<uint4 *>(base + ((c ^ (row & 7)) << 4)) = v;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
+           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o, Params p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *Qb[2] = {smem, smem + 3 * kTileBytes};
+    uint8_t *Gb[2] = {smem + kTileBytes, smem + 4 * kTileBytes};
+    uint8_t *Vb[2] = {smem + 2 * kTileBytes, smem + 5 * kTileBytes};
+    uint8_t *X = smem + 6 * kTileBytes;
+    Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / p.H, h = bh - b * p.H;
+    const int N = p.ntiles;
+    if (smem_u32(smem) & 1023u) {   // the swizzled operand layout needs 1024-byte alignment
+        if (tid == 0) set_status(HGRN2_ERR_DEVICE);
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(&m->full[0], 1);
+        mbar_init(&m->full[1], 1);
+        mbar_init(&m->barA, 1);
+        mbar_init(&m->barO1, 1);
+        mbar_init(&m->barM, 1);
+        fence_mbar_init();
+        m->bad = 0;
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_lf);
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_o);
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = m->tmem_base;
+
+    auto issue_load = [&](int n) {
+        const int s = n & 1;
+        mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
+        for (int c = 0; c < 2; ++c) {
+            tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->full[s], 64 * c, h, n * kTile, b);
+            tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, n * kTile, b);
+            tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, n * kTile, b);
+        }
+    };
+    if (tid == 0) {
+        issue_load(0);
+        if (N > 1) issue_load(1);
+    }
+
+    // TMEM lane quadrant and column half of this warp
+    const int quad = warp & 3, ch = warp >> 2;
+    const int lrow = 32 * quad + lane;                       // TMEM lane = row of the tile
+    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+
+    // state init: S = h0 (or 0), rows j = lrow, columns 64ch .. 64ch+63
+    {
+        float r0[32], r1[32];
+        if (p.h0) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.h0 + ((size_t)bh * 128 + lrow) * 128 + 64 * ch);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float4 a = src[i], c = src[8 + i];
+                r0[4 * i] = a.x; r0[4 * i + 1] = a.y; r0[4 * i + 2] = a.z; r0[4 * i + 3] = a.w;
+                r1[4 * i] = c.x; r1[4 * i + 1] = c.y; r1[4 * i + 2] = c.z; r1[4 * i + 3] = c.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0.0f;
+        }
+        tmem_st32(tl + kColS + 64 * ch, r0);
+        tmem_st32(tl + kColS + 64 * ch + 32, r1);
+        tmem_wait_st();
+    }
+
+    const uint32_t id_kk = idesc_bf16(128, 128, false, false);
+    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
+    const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+    const int pc = tid & 63, rr = tid >> 6;                  // prep: column pair, 32-row range
+    const int col0 = 2 * pc;
+    const uint32_t poff_blk = (uint32_t)(col0 >> 6) * kBlk;
+    const int pchunk = (col0 & 63) >> 3, pin = (col0 & 7) * 2;
+    bool ok = true;
+    int n = 0;
+
+    for (n = 0; n < N; ++n) {
+        const int s = n & 1;
+        if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
+
+        // ---- prep pass 1: f = exp(log f) kept in registers, partial products per 32-row range
+        float f0[32], f1[32];
+        float P0 = 1.0f, P1 = 1.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int t = 32 * rr + i;
+            const uint32_t off = poff_blk + t * 128 + (((uint32_t)pchunk ^ (t & 7)) << 4) + pin;
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + off);
+            f0[i] = __expf(bf_lo(w));
+            f1[i] = __expf(bf_hi(w));
+            P0 *= f0[i];
+            P1 *= f1[i];
+        }
+        m->Ppart[rr][col0] = P0;
+        m->Ppart[rr][col0 + 1] = P1;
+        __syncthreads();
+        // ---- prep pass 2: Qt = q E and Kt = k / E in place
+        float E0 = 1.0f, E1 = 1.0f;
+        for (int r2 = 0; r2 < rr; ++r2) {
+            E0 *= m->Ppart[r2][col0];
+            E1 *= m->Ppart[r2][col0 + 1];
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int t = 32 * rr + i;
+            const uint32_t off = poff_blk + t * 128 + (((uint32_t)pchunk ^ (t & 7)) << 4) + pin;
+            uint32_t *gq = reinterpret_cast<uint32_t *>(Qb[s] + off);
+            uint32_t *gg = reinterpret_cast<uint32_t *>(Gb[s] + off);
+            const uint32_t wa = *gg, wq = *gq;
+            E0 *= f0[i];
+            E1 *= f1[i];
+            const float k0 = k_from(bf_lo(wa), f0[i]), k1 = k_from(bf_hi(wa), f1[i]);
+            *gq = pack_bf2(bf_lo(wq) * E0, bf_hi(wq) * E1);
+            *gg = pack_bf2(k0 * __fdividef(1.0f, E0), k1 * __fdividef(1.0f, E1));
+        }
+        if (rr == 3) {
+            m->EB[col0] = E0;
+            m->EB[col0 + 1] = E1;
+        }
+        fence_proxy_async_smem();
+        const int bad = __syncthreads_or(rr == 3 && !(E0 >= kMinEB && E1 >= kMinEB));
+        if (bad) break;
+
+        // ---- A = Qt Kt^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColA, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Gb[s]) + ko, 16, 1024), id_kk, kk > 0);
+            }
+            mma_commit(&m->barA);
+            tma_store_wait_read0();   // the previous chunk's o store has finished reading X
+        }
+        __syncthreads();
+
+        // ---- S phase: bf16 copy of S_in into X (B operand, MN-major) and S <- Diag(E_B) S
+        {
+            float r0[32], r1[32];
+            tc_fence_after();
+            tmem_ld32(tl + kColS + 64 * ch, r0);
+            tmem_ld32(tl + kColS + 64 * ch + 32, r1);
+            tmem_wait_ld();
+            store_row_bf16(X + ch * kBlk, lrow, r0, r1);
+            const float e = m->EB[lrow];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                r0[i] *= e;
+                r1[i] *= e;
+            }
+            tmem_st32(tl + kColS + 64 * ch, r0);
+            tmem_st32(tl + kColS + 64 * ch + 32, r1);
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(X) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
+            }
+            mma_commit(&m->barO1);
+        }
+
+        // ---- Kh = Kt * E_B in place (after the A MMA has read Kt)
+        if (!mbar_wait(&m->barA, n & 1)) ok = false;
+        tc_fence_after();
+        {
+            const float e0 = m->EB[col0], e1 = m->EB[col0 + 1];
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                const int t = 32 * rr + i;
+                const uint32_t off = poff_blk + t * 128 + (((uint32_t)pchunk ^ (t & 7)) << 4) + pin;
+                uint32_t *gg = reinterpret_cast<uint32_t *>(Gb[s] + off);
+                const uint32_t w = *gg;
+                *gg = pack_bf2(bf_lo(w) * e0, bf_hi(w) * e1);
+            }
+        }
+        // ---- A phase: causal mask, bf16 into X (A operand, K-major) once the inter MMA is done with X
+        {
+            float r0[32], r1[32];
+            tmem_ld32(tl + kColA + 64 * ch, r0);
+            tmem_ld32(tl + kColA + 64 * ch + 32, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (64 * ch + i > lrow) r0[i] = 0.0f;
+                if (64 * ch + 32 + i > lrow) r1[i] = 0.0f;
+            }
+            if (!mbar_wait(&m->barO1, n & 1)) { ok = false; }
+            store_row_bf16(X + ch * kBlk, lrow, r0, r1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(!ok)) { ok = false; break; }
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+            }
+            mma_commit(&m->barM);
+        }
+        if (__syncthreads_or(!mbar_wait(&m->barM, n & 1))) { ok = false; break; }
+        tc_fence_after();
+        if (tid == 0 && n + 2 < N) issue_load(n + 2);
+
+        // ---- epilogue: O (fp32 TMEM) -> bf16 -> X -> TMA store
+        {
+            float r0[32], r1[32];
+            tmem_ld32(tl + kColO + 64 * ch, r0);
+            tmem_ld32(tl + kColO + 64 * ch + 32, r1);
+            tmem_wait_ld();
+            store_row_bf16(X + ch * kBlk, lrow, r0, r1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_o, X, 0, h, n * kTile, b);
+            tma_store_4d(&tm_o, X + kBlk, 64, h, n * kTile, b);
+            tma_store_commit();
+        }
+    }
+
+    const bool fell_back = ok && n < N;
+    if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
+    // drain: a load still in flight into this CTA's shared memory (chunk n+1 was issued
+    // once chunk n-1 completed), and the last o store
+    if (tid == 0) {
+        if (n + 1 < N) mbar_wait(&m->full[(n + 1) & 1], ((n + 1) >> 1) & 1);
+        tma_store_wait_all0();
+    }
+    if (ok && !fell_back && p.hT) {
+        tc_fence_after();
+        float r0[32], r1[32];
+        tmem_ld32(tl + kColS + 64 * ch, r0);
+        tmem_ld32(tl + kColS + 64 * ch + 32, r1);
+        tmem_wait_ld();
+        float4 *dst = reinterpret_cast<float4 *>(p.hT + ((size_t)bh * 128 + lrow) * 128 + 64 * ch);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            dst[i] = make_float4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+            dst[8 + i] = make_float4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
+        }
+    }
+    if (tid == 0) {
+        p.flags[bh] = fell_back ? 1 : 0;
+        if (fell_back) atomicAdd(&g_counters[0], 1ull);
+        if (ok && !fell_back) atomicAdd(&g_counters[1], (unsigned long long)N);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+}  // namespace tcf
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 4-D map over a [B][T][H][128] bf16 tensor: box = 64 features x 1 head x 128 tokens x 1 batch.
+bool make_token_map(CUtensorMap *map, const void *ptr, int B, int T, int H) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)T * H * 256};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t tc_fwd_smem() { return tcf::kSmemBytes; }
+
+cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
+    CUtensorMap mq, ml, mx, mo;
+    if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
+        !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mo, a.o, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(tcf::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcf::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    tcf::Params p{a.h0, a.hT, a.flags, a.T, a.H, (a.T + tcf::kTile - 1) / tcf::kTile};
+    tcf::fwd_kernel<<<a.B * a.H, tcf::kThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, p);
+    return cudaGetLastError();
+}
+
+}  // namespace hgrn2
