@@ -52,7 +52,7 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
     (void)T; (void)chunk;
     size_t bytes = 0;
     if (want_bwd) bytes += align256(sizeof(float) * (size_t)B * H * dk);   // rowsum(dhT * hT)
-    else if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
+    if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
     return bytes;
 }
 
@@ -129,7 +129,17 @@ hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const fl
     }
     int C = simt_chunk(chunk, dk, dv, true);
     if (!C) return HGRN2_ERR_UNSUPPORTED;
-    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, (float *)workspace, B, T, H, dk, dv, C};
+    float *rs = (float *)workspace;
+    if (use_tc(dk, dv, dtype)) {
+        int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
+        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H};
+        g_launches += 4;
+        cudaError_t e = launch_tc_bwd(t, stream);
+        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+        SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, flags};
+        return from_cuda(launch_simt_bwd(a, bf16, stream));
+    }
+    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr};
     g_launches += 2;
     return from_cuda(launch_simt_bwd(a, bf16, stream));
 }

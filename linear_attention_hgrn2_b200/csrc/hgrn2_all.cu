@@ -7,3 +7,4 @@
 #include "simt.cu"
 #include "step.cu"
 #include "tc_fwd.cu"
+#include "tc_bwd.cu"

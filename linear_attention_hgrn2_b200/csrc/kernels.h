@@ -31,6 +31,17 @@ struct SimtBwdArgs {
     float *dh0;
     float *rs;   // [B*H*dk] workspace: rowsum(dhT * hT)
     int B, T, H, dk, dv, C;
+    const int *only;   // if non-null: only (b,h) with only[b*H+h] != 0 are computed
+};
+
+struct TcBwdArgs {
+    const void *q, *lf, *x, *dO;
+    const float *h0, *dhT;
+    void *dq, *dlf, *dx;
+    float *dh0;
+    float *rs;         // [B*H*128] workspace
+    int *flags;        // [B*H] workspace, out: 1 where the (b,h) needs the exact route
+    int B, T, H;
 };
 
 size_t simt_fwd_smem(int C, int dk, int dv);
@@ -40,6 +51,8 @@ cudaError_t launch_simt_fwd(const SimtFwdArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_bwd(const SimtBwdArgs &a, bool bf16, cudaStream_t st);
 
 size_t tc_fwd_smem();
+size_t tc_bwd_smem();
+cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st);
 
 cudaError_t launch_step(const void *q, const void *lf, const void *x, float *S, void *o, int B, int H,

@@ -148,7 +148,8 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
-                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C) {
+                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+    if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Bs = sm;              // [C][ldk]
@@ -224,7 +225,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
-                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C) {
+                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+    if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;               // [C][ldk] q, later q e^{b}
@@ -356,12 +358,12 @@ static cudaError_t launch_simt_bwd_t(const SimtBwdArgs &a, cudaStream_t st) {
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     if (e != cudaSuccess) return e;
     k1<<<a.B * a.H, kSimtThreads, s1, st>>>((const T *)a.lf, (const T *)a.x, a.h0, (const T *)a.dO,
-                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C);
+                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C, a.only);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k2<<<a.B * a.H, kSimtThreads, s2, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x,
                                             (const T *)a.dO, a.dhT, (const T *)a.dq, a.rs,
-                                            (T *)a.dlf, (T *)a.dx, a.dh0, a.T, a.H, a.dk, a.dv, a.C);
+                                            (T *)a.dlf, (T *)a.dx, a.dh0, a.T, a.H, a.dk, a.dv, a.C, a.only);
     return cudaGetLastError();
 }
 

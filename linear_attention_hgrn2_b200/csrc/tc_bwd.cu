@@ -1,0 +1,681 @@
+// tc_bwd.cu -- chunkwise HGRN2 backward on 5th-generation tensor cores (sm_100a).
+//
+// Two sweeps per (batch, head), d_k = d_v = 128, bf16 token tensors, 128-token
+// chunks, same factorisation as the forward: E_t = prod_{r<=t} f_r inside a
+// chunk, Qt = q E, Kt = k / E, E_B = E at the chunk end.
+//
+// Forward sweep (dq_kernel): the fp32 state is recomputed in TMEM and
+//   dq = E * (dO S_in^T + mask(dO V^T) Kt)                                 (1)
+// is formed transposed (TMEM lane = key dim j, column = token t), so the
+// decay factor E[j][t] that finishes it sits in the same thread's lane.  The
+// state is post-scaled: the MMA accumulates S_in + Kt^T V, and the next chunk
+// multiplies its rows by E_B before using it.  At the end it writes
+// rowsum(dhT * hT) for the reverse sweep's carry.
+//
+// Reverse sweep (rev_kernel), chunks last to first, dS = dL/dS_out in TMEM:
+//   dSh  = Diag(E_B) dS                                   (also the new dS)
+//   di   = mask(A)^T dO + Kt dSh                            A = Qt Kt^T
+//   dk^T = (Qt^T mask(dO V^T) + dSh V^T) / E               (lane j, column s)
+//   dS   = dSh + Qt^T dO
+//   dlog f_t = sum_{t'>=t} (q dq - k dk)_{t'} + rowsum(dhT hT) - f_t dk_t
+// The last line is the gradient through both the decay and the tied input gate
+// k = 1 - f ("HGRN2: Gated Linear RNNs with State Expansion", §2.1 tied gate,
+// §3.2 outer-product state, §5 per-dimension decay); its reverse cumulative sum
+// runs inside the chunk per key dim (thread-local, lane = j) and across chunks
+// through a carry.  q, log f and dq for that line are read back from global
+// memory (they were just streamed through L2) so that the next chunk's TMA
+// load can start as soon as the MMAs are done.
+//
+// Validity and fallback are those of the forward: a (batch, head) whose chunk
+// decay span exceeds the factorisation's range is flagged by the forward sweep,
+// skipped by the reverse sweep, and recomputed by the exact route.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace hgrn2 {
+namespace tcb {
+
+using namespace tc;
+using namespace tcc;
+
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ void st_bar_expect(uint64_t *bar, uint32_t bytes) { mbar_arrive_expect_tx(bar, bytes); }
+
+// ------------------------------------------------------------------ forward sweep: dq
+namespace fsw {
+constexpr uint32_t kColS = 0, kColDA = 128, kColDQ = 256, kColE = 384;
+
+struct __align__(8) Misc {
+    uint64_t full[2];
+    uint64_t barA, barQ1, barM;
+    uint32_t tmem_base;
+    int pad;
+    float EBr[2][128];     // E_B of the last two chunks (post-scaling of the state)
+    float Ppart[2][128];   // prep partial products; after the loop, rowsum(dhT*hT) halves
+};
+constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
+}  // namespace fsw
+
+struct DqParams {
+    const float *h0, *dhT;
+    float *rs;       // [B*H*128] rowsum(dhT * hT)
+    int *flags;      // [B*H]
+    int T, H, ntiles;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUtensorMap tm_x,
+          const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dq, DqParams p) {
+    using namespace fsw;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *Gb[2] = {smem, smem + 3 * kTileBytes};
+    uint8_t *Vb[2] = {smem + kTileBytes, smem + 4 * kTileBytes};
+    uint8_t *Ob[2] = {smem + 2 * kTileBytes, smem + 5 * kTileBytes};
+    uint8_t *X = smem + 6 * kTileBytes;
+    Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / p.H, h = bh - b * p.H;
+    const int N = p.ntiles;
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0) set_status(HGRN2_ERR_DEVICE);
+        return;
+    }
+    const int quad = warp & 3, half = warp >> 2;
+    const int j = 32 * quad + lane;                         // key dim / TMEM lane / tile row
+    if (tid == 0) {
+        mbar_init(&m->full[0], 1);
+        mbar_init(&m->full[1], 1);
+        mbar_init(&m->barA, 1);
+        mbar_init(&m->barQ1, 1);
+        mbar_init(&m->barM, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = m->tmem_base;
+    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+
+    auto issue_load = [&](int n) {
+        const int s = n & 1;
+        mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
+        for (int c = 0; c < 2; ++c) {
+            tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, n * kTile, b);
+            tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, n * kTile, b);
+            tma_load_4d(Ob[s] + c * kBlk, &tm_do, &m->full[s], 64 * c, h, n * kTile, b);
+        }
+    };
+    if (tid == 0) {
+        issue_load(0);
+        if (N > 1) issue_load(1);
+    }
+    {   // state init S = h0 (or 0); previous E_B = 1
+        float r0[32], r1[32];
+        if (p.h0) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.h0 + ((size_t)bh * 128 + j) * 128 + 64 * half);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float4 a = src[i], c = src[8 + i];
+                r0[4 * i] = a.x; r0[4 * i + 1] = a.y; r0[4 * i + 2] = a.z; r0[4 * i + 3] = a.w;
+                r1[4 * i] = c.x; r1[4 * i + 1] = c.y; r1[4 * i + 2] = c.z; r1[4 * i + 3] = c.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0.0f;
+        }
+        tmem_st32(tl + kColS + 64 * half, r0);
+        tmem_st32(tl + kColS + 64 * half + 32, r1);
+        tmem_wait_st();
+        if (half == 0) m->EBr[1][j] = 1.0f;
+    }
+
+    const uint32_t id_kk = idesc_bf16(128, 128, false, false);
+    const uint32_t id_mnk = idesc_bf16(128, 128, true, false);
+    const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+    const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
+    bool ok = true;
+    int n = 0;
+    for (n = 0; n < N; ++n) {
+        const int s = n & 1;
+        if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
+        // ---- prep: column j, rows 64*half .. +63: Kt = k / E in place of log f, E -> TMEM
+        float fv[64];
+        float P = 1.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const int t = 64 * half + i;
+            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+            fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + off)));
+            P *= fv[i];
+        }
+        m->Ppart[half][j] = P;
+        __syncthreads();
+        float E = half ? m->Ppart[0][j] : 1.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const int t = 64 * half + i;
+            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+            __nv_bfloat16 *g = reinterpret_cast<__nv_bfloat16 *>(Gb[s] + off);
+            const float a = __bfloat162float(*g);
+            E *= fv[i];
+            const float k = k_from(a, fv[i]);
+            *g = __float2bfloat16_rn(k * __fdividef(1.0f, E));
+            fv[i] = E;
+        }
+        if (half == 1) m->EBr[s][j] = E;
+        {
+            float *e0 = fv, *e1 = fv + 32;
+            tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(e0));
+            tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(e1));
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(half == 1 && !(E >= kMinEB))) break;
+
+        // ---- dA = dO V^T
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColDA, sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Vb[s]) + ko, 16, 1024), id_kk, kk > 0);
+            }
+            mma_commit(&m->barA);
+            tma_store_wait_read0();
+        }
+        __syncthreads();
+        // ---- S phase: S_in = Diag(E_B of the previous chunk) * accumulator; bf16 copy into X
+        {
+            float r0[32], r1[32];
+            tc_fence_after();
+            tmem_ld32(tl + kColS + 64 * half, r0);
+            tmem_ld32(tl + kColS + 64 * half + 32, r1);
+            tmem_wait_ld();
+            const float e = m->EBr[s ^ 1][j];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                r0[i] *= e;
+                r1[i] *= e;
+            }
+            store_row_bf16(X + half * kBlk, j, r0, r1);
+            tmem_st32(tl + kColS + 64 * half, r0);
+            tmem_st32(tl + kColS + 64 * half + 32, r1);
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- dq_pre^T = S_in dO^T   (M = j, N = t, K = v)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024), id_kk, kk > 0);
+            }
+            mma_commit(&m->barQ1);
+        }
+        // ---- dA phase: causal mask, bf16 into X (rows t) once the previous MMA is done with X
+        {
+            if (!mbar_wait(&m->barA, n & 1)) ok = false;
+            tc_fence_after();
+            float r0[32], r1[32];
+            tmem_ld32(tl + kColDA + 64 * half, r0);
+            tmem_ld32(tl + kColDA + 64 * half + 32, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (64 * half + i > j) r0[i] = 0.0f;
+                if (64 * half + 32 + i > j) r1[i] = 0.0f;
+            }
+            if (!mbar_wait(&m->barQ1, n & 1)) ok = false;
+            store_row_bf16(X + half * kBlk, j, r0, r1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(!ok)) { ok = false; break; }
+        // ---- dq_pre^T += Kt^T dA^T (M = j, N = t, K = s);  S += Kt^T V (M = j, N = v, K = t)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(X) + ko, 16, 1024), id_mnk, true);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+            }
+            mma_commit(&m->barM);
+        }
+        if (__syncthreads_or(!mbar_wait(&m->barM, n & 1))) { ok = false; break; }
+        tc_fence_after();
+        if (tid == 0 && n + 2 < N) issue_load(n + 2);
+        // ---- epilogue: dq[t][j] = E[j][t] * dq_pre^T[j][t] -> X (rows t) -> TMA store
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float d[32], e[32];
+            tmem_ld32(tl + kColDQ + 64 * half + 32 * c, d);
+            tmem_ld32(tl + kColE + 64 * half + 32 * c, e);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int t = 64 * half + 32 * c + i;
+                *reinterpret_cast<__nv_bfloat16 *>(X + cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin) =
+                    __float2bfloat16_rn(d[i] * e[i]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_dq, X, 0, h, n * kTile, b);
+            tma_store_4d(&tm_dq, X + kBlk, 64, h, n * kTile, b);
+            tma_store_commit();
+        }
+    }
+    const bool fell_back = ok && n < N;
+    if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
+    if (tid == 0) {
+        if (n + 1 < N) mbar_wait(&m->full[(n + 1) & 1], ((n + 1) >> 1) & 1);
+        tma_store_wait_all0();
+    }
+    if (ok && !fell_back && p.dhT && p.rs) {
+        // hT = Diag(E_B of the last chunk) * accumulator;  rs[j] = sum_v dhT[j,v] hT[j,v]
+        tc_fence_after();
+        float r0[32], r1[32];
+        tmem_ld32(tl + kColS + 64 * half, r0);
+        tmem_ld32(tl + kColS + 64 * half + 32, r1);
+        tmem_wait_ld();
+        const float e = N > 0 ? m->EBr[(N - 1) & 1][j] : 1.0f;
+        const float *g = p.dhT + ((size_t)bh * 128 + j) * 128 + 64 * half;
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            acc = fmaf(g[i], r0[i] * e, acc);
+            acc = fmaf(g[32 + i], r1[i] * e, acc);
+        }
+        m->Ppart[half][j] = acc;
+    }
+    __syncthreads();
+    if (ok && !fell_back && p.dhT && p.rs && half == 0) p.rs[(size_t)bh * 128 + j] = m->Ppart[0][j] + m->Ppart[1][j];
+    if (tid == 0) {
+        p.flags[bh] = fell_back ? 1 : 0;
+        if (fell_back) atomicAdd(&g_counters[0], 1ull);
+        if (ok && !fell_back) atomicAdd(&g_counters[1], (unsigned long long)N);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+// ------------------------------------------------------------------ reverse sweep
+namespace rsw {
+constexpr uint32_t kColDS = 0, kColX1 = 128, kColX2 = 256, kColE = 384;
+
+struct __align__(8) Misc {
+    uint64_t full, barP1, barP2;
+    uint32_t tmem_base;
+    int pad;
+    float EB[128];
+    float Ppart[2][128];   // prep partial products; in the epilogue, per-half suffix totals
+    float carry[128];
+};
+constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
+}  // namespace rsw
+
+struct RevParams {
+    const __nv_bfloat16 *q, *lf, *dq;   // read back in the d log f epilogue
+    const float *dhT, *rs;
+    float *dh0;
+    const int *flags;
+    int T, H, ntiles;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
+           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
+           const __grid_constant__ CUtensorMap tm_di, const __grid_constant__ CUtensorMap tm_dlf, RevParams p) {
+    using namespace rsw;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *Qb = smem, *Gb = smem + kTileBytes, *Vb = smem + 2 * kTileBytes, *Ob = smem + 3 * kTileBytes;
+    uint8_t *D16 = smem + 4 * kTileBytes, *AT = smem + 5 * kTileBytes, *DA = smem + 6 * kTileBytes;
+    Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / p.H, h = bh - b * p.H;
+    const int N = p.ntiles;
+    if (p.flags[bh] != 0) return;   // this (b,h) takes the exact route
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0) set_status(HGRN2_ERR_DEVICE);
+        return;
+    }
+    const int quad = warp & 3, half = warp >> 2;
+    const int j = 32 * quad + lane;
+    if (tid == 0) {
+        mbar_init(&m->full, 1);
+        mbar_init(&m->barP1, 1);
+        mbar_init(&m->barP2, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = m->tmem_base;
+    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+
+    auto issue_load = [&](int n) {
+        mbar_arrive_expect_tx(&m->full, 4 * kTileBytes);
+        for (int c = 0; c < 2; ++c) {
+            tma_load_4d(Qb + c * kBlk, &tm_q, &m->full, 64 * c, h, n * kTile, b);
+            tma_load_4d(Gb + c * kBlk, &tm_lf, &m->full, 64 * c, h, n * kTile, b);
+            tma_load_4d(Vb + c * kBlk, &tm_x, &m->full, 64 * c, h, n * kTile, b);
+            tma_load_4d(Ob + c * kBlk, &tm_do, &m->full, 64 * c, h, n * kTile, b);
+        }
+    };
+    if (tid == 0 && N > 0) issue_load(N - 1);
+    {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
+        float r0[32], r1[32];
+        if (p.dhT) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * 128 + j) * 128 + 64 * half);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float4 a = src[i], c = src[8 + i];
+                r0[4 * i] = a.x; r0[4 * i + 1] = a.y; r0[4 * i + 2] = a.z; r0[4 * i + 3] = a.w;
+                r1[4 * i] = c.x; r1[4 * i + 1] = c.y; r1[4 * i + 2] = c.z; r1[4 * i + 3] = c.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0.0f;
+        }
+        tmem_st32(tl + kColDS + 64 * half, r0);
+        tmem_st32(tl + kColDS + 64 * half + 32, r1);
+        tmem_wait_st();
+        if (half == 0) m->carry[j] = (p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
+    }
+
+    const uint32_t id_kk = idesc_bf16(128, 128, false, false);
+    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
+    const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+    const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
+    const size_t tok_stride = (size_t)p.H * 128;
+    bool ok = true;
+    int it = 0, n = N - 1;
+    for (; n >= 0; --n, ++it) {
+        if (__syncthreads_or(!mbar_wait(&m->full, it & 1))) { ok = false; break; }
+        // ---- prep: Qt = q E (in place), Kt = k / E (in place of log f), E -> TMEM
+        float fv[64];
+        float P = 1.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const int t = 64 * half + i;
+            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+            fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb + off)));
+            P *= fv[i];
+        }
+        m->Ppart[half][j] = P;
+        __syncthreads();
+        float E = half ? m->Ppart[0][j] : 1.0f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const int t = 64 * half + i;
+            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+            __nv_bfloat16 *g = reinterpret_cast<__nv_bfloat16 *>(Gb + off);
+            __nv_bfloat16 *qq = reinterpret_cast<__nv_bfloat16 *>(Qb + off);
+            const float a = __bfloat162float(*g);
+            E *= fv[i];
+            const float k = k_from(a, fv[i]);
+            *g = __float2bfloat16_rn(k * __fdividef(1.0f, E));
+            *qq = __float2bfloat16_rn(__bfloat162float(*qq) * E);
+            fv[i] = E;
+        }
+        if (half == 1) m->EB[j] = E;
+        tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(fv));
+        tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(fv + 32));
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(half == 1 && !(E >= kMinEB))) {
+            if (tid == 0) set_status(HGRN2_ERR_DEVICE);   // the forward sweep passed this (b,h)
+            ok = false;
+            break;
+        }
+        // ---- phase 1: A^T = Kt Qt^T (M = s, N = t), dA = dO V^T (M = t, N = s)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Qb) + ko, 16, 1024), id_kk, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(Ob) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, kk > 0);
+            }
+            mma_commit(&m->barP1);
+            tma_store_wait_read0();   // previous chunk's di / d log f stores have read AT / DA
+        }
+        __syncthreads();
+        // ---- dS phase: dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16
+        {
+            float r0[32], r1[32];
+            tc_fence_after();
+            tmem_ld32(tl + kColDS + 64 * half, r0);
+            tmem_ld32(tl + kColDS + 64 * half + 32, r1);
+            tmem_wait_ld();
+            const float e = m->EB[j];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                r0[i] *= e;
+                r1[i] *= e;
+            }
+            store_row_bf16(D16 + half * kBlk, j, r0, r1);
+            tmem_st32(tl + kColDS + 64 * half, r0);
+            tmem_st32(tl + kColDS + 64 * half + 32, r1);
+            tmem_wait_st();
+        }
+        // ---- masks: A^T keeps t >= s (lane s), dA keeps s <= t (lane t)
+        {
+            if (!mbar_wait(&m->barP1, it & 1)) ok = false;
+            tc_fence_after();
+            float r0[32], r1[32];
+            tmem_ld32(tl + kColX1 + 64 * half, r0);
+            tmem_ld32(tl + kColX1 + 64 * half + 32, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (64 * half + i < j) r0[i] = 0.0f;
+                if (64 * half + 32 + i < j) r1[i] = 0.0f;
+            }
+            store_row_bf16(AT + half * kBlk, j, r0, r1);
+            tmem_ld32(tl + kColX2 + 64 * half, r0);
+            tmem_ld32(tl + kColX2 + 64 * half + 32, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (64 * half + i > j) r0[i] = 0.0f;
+                if (64 * half + 32 + i > j) r1[i] = 0.0f;
+            }
+            store_row_bf16(DA + half * kBlk, j, r0, r1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(!ok)) { ok = false; break; }
+        // ---- phase 2
+        if (tid == 0) {
+            tc_fence_after();
+            // di = mask(A)^T dO + Kt dSh          (M = s, N = v)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(AT) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(D16) + kk * 2048, kBlk, 1024), id_kmn, true);
+            }
+            // dk_pre^T = Qt^T mask(dA) + dSh V^T   (M = j, N = s)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(DA) + kk * 2048, kBlk, 1024), id_mnmn, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, true);
+            }
+            // dS = dSh + Qt^T dO                    (M = j, N = v)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ss(tbase + kColDS, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_mnmn, true);
+            }
+            mma_commit(&m->barP2);
+        }
+        if (__syncthreads_or(!mbar_wait(&m->barP2, it & 1))) { ok = false; break; }
+        tc_fence_after();
+        if (tid == 0 && n > 0) issue_load(n - 1);   // inputs of this chunk are no longer read
+
+        // ---- di (lane s) -> AT (rows s) for the TMA store
+        {
+            float r0[32], r1[32];
+            tmem_ld32(tl + kColX1 + 64 * half, r0);
+            tmem_ld32(tl + kColX1 + 64 * half + 32, r1);
+            tmem_wait_ld();
+            store_row_bf16(AT + half * kBlk, j, r0, r1);
+        }
+        // ---- d log f (lane j, tokens 64*half .. +63), reverse cumulative sum with carry
+        float dap[64];
+        float suf = 0.0f;
+        const int t_base = n * kTile + 64 * half;
+#pragma unroll
+        for (int c = 1; c >= 0; --c) {
+            float dk[32], e[32];
+            tmem_ld32(tl + kColX2 + 64 * half + 32 * c, dk);
+            tmem_ld32(tl + kColE + 64 * half + 32 * c, e);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 31; i >= 0; --i) {
+                const int tg = t_base + 32 * c + i;
+                float w = 0.0f, fdk = 0.0f;
+                if (tg < p.T) {
+                    const size_t gi = ((size_t)b * p.T + tg) * tok_stride + (size_t)h * 128 + j;
+                    const float a = __bfloat162float(p.lf[gi]);
+                    const float qv = __bfloat162float(p.q[gi]);
+                    const float dqv = __bfloat162float(p.dq[gi]);
+                    const float f = __expf(a);
+                    const float k = k_from(a, f);
+                    const float dkv = dk[i] * __fdividef(1.0f, e[i]);
+                    w = qv * dqv - k * dkv;
+                    fdk = f * dkv;
+                }
+                suf += w;
+                dap[32 * c + i] = suf - fdk;
+            }
+        }
+        m->Ppart[half][j] = suf;
+        __syncthreads();
+        {
+            const float carry = m->carry[j] + (half == 0 ? m->Ppart[1][j] : 0.0f);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const int t = 64 * half + i;
+                *reinterpret_cast<__nv_bfloat16 *>(DA + cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin) =
+                    __float2bfloat16_rn(dap[i] + carry);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (half == 0) m->carry[j] += m->Ppart[0][j] + m->Ppart[1][j];
+        if (tid == 0) {
+            tma_store_4d(&tm_di, AT, 0, h, n * kTile, b);
+            tma_store_4d(&tm_di, AT + kBlk, 64, h, n * kTile, b);
+            tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
+            tma_store_4d(&tm_dlf, DA + kBlk, 64, h, n * kTile, b);
+            tma_store_commit();
+        }
+    }
+    if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
+    if (tid == 0) {
+        // a load was issued for chunk n-1 only after chunk n's MMAs completed; after a break
+        // at chunk n before that point, nothing is in flight except chunk n itself (waited)
+        tma_store_wait_all0();
+    }
+    if (ok && p.dh0) {
+        tc_fence_after();
+        float r0[32], r1[32];
+        tmem_ld32(tl + kColDS + 64 * half, r0);
+        tmem_ld32(tl + kColDS + 64 * half + 32, r1);
+        tmem_wait_ld();
+        float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * 128 + j) * 128 + 64 * half);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            dst[i] = make_float4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+            dst[8 + i] = make_float4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
+        }
+    }
+    if (tid == 0 && ok) atomicAdd(&g_counters[1], (unsigned long long)N);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+}  // namespace tcb
+
+static_assert(tcb::fsw::kSmemBytes <= 227 * 1024, "forward-sweep shared memory");
+static_assert(tcb::rsw::kSmemBytes <= 227 * 1024, "reverse-sweep shared memory");
+
+size_t tc_bwd_smem() { return tcb::fsw::kSmemBytes > tcb::rsw::kSmemBytes ? tcb::fsw::kSmemBytes : tcb::rsw::kSmemBytes; }
+
+cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
+    CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl;
+    if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
+        !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mdo, a.dO, a.B, a.T, a.H) ||
+        !make_token_map(&mdq, a.dq, a.B, a.T, a.H) || !make_token_map(&mdi, a.dx, a.B, a.T, a.H) ||
+        !make_token_map(&mdl, a.dlf, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(tcb::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcb::fsw::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tcb::rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcb::rsw::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
+    tcb::DqParams p1{a.h0, a.dhT, a.rs, a.flags, a.T, a.H, ntiles};
+    tcb::dq_kernel<<<a.B * a.H, tcb::kThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    tcb::RevParams p2{(const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.dq,
+                      a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles};
+    tcb::rev_kernel<<<a.B * a.H, tcb::kThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdi, mdl, p2);
+    return cudaGetLastError();
+}
+
+}  // namespace hgrn2

@@ -1,0 +1,85 @@
+// tc_common.cuh -- device and host helpers shared by the tensor-core kernels.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace hgrn2 {
+namespace tcc {
+
+constexpr int kTile = 128;               // tokens per chunk (one M = 128 MMA tile)
+constexpr int kTileBytes = 128 * 128 * 2;
+constexpr int kBlk = 128 * 128;          // bytes of one 64-column block of a 128-row tile
+constexpr float kMinEB = 1e-26f;         // factorisation range: min_j E_B[j] (decay span ~60)
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// 1 - exp(a) given f = exp(a): Taylor series of -expm1 for |a| < 0.25 (relative
+// truncation error < 1.5e-6), 1 - f otherwise (no cancellation there).
+__device__ __forceinline__ float k_from(float a, float f) {
+    if (fabsf(a) < 0.25f) {
+        float p = fmaf(a, 1.0f / 120.0f, 1.0f / 24.0f);
+        p = fmaf(p, a, 1.0f / 6.0f);
+        p = fmaf(p, a, 0.5f);
+        p = fmaf(p, a, 1.0f);
+        return -a * p;
+    }
+    return 1.0f - f;
+}
+
+// Row j (lane) of a 64-column half of a TMEM tile -> bf16 row in a swizzled smem block.
+__device__ __forceinline__ void store_row_bf16(uint8_t *blk, int row, const float (&r0)[32], const float (&r1)[32]) {
+    uint8_t *base = blk + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const float *src = c < 4 ? &r0[c * 8] : &r1[(c - 4) * 8];
+        uint4 v;
+        v.x = pack_bf2(src[0], src[1]);
+        v.y = pack_bf2(src[2], src[3]);
+        v.z = pack_bf2(src[4], src[5]);
+        v.w = pack_bf2(src[6], src[7]);
+        *reinterpret_cast<uint4 *>(base + ((c ^ (row & 7)) << 4)) = v;
+    }
+}
+
+
+// bf16 element (row, col) of a 128 x 128 tile in the two-block 128-byte-swizzled layout.
+__device__ __forceinline__ __nv_bfloat16 *tile_elem(uint8_t *tile, int row, int col) {
+    return reinterpret_cast<__nv_bfloat16 *>(tile + tc::sw128_off(row, col, 128));
+}
+
+}  // namespace tcc
+
+// ------------------------------------------------------------------ host side
+inline PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 4-D map over a [B][T][H][128] bf16 tensor: box = 64 features x 1 head x 128 tokens x 1 batch.
+inline bool make_token_map(CUtensorMap *map, const void *ptr, int B, int T, int H) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)T * H * 256};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace hgrn2

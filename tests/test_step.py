@@ -55,4 +55,4 @@ def test_steps_equal_fwd(cuda, dtype):
     for t in range(T):
         ot = L.step(g["q"][:, t].contiguous(), g["log_f"][:, t].contiguous(), g["i"][:, t].contiguous(), S)
         assert err(np64(ot), np64(o[:, t]), dtype) <= tol(dtype)
-    assert err(np64(S), np64(hT), torch.float32) <= (1e-4 if dtype == torch.float32 else 1e-2)
+    assert err(np64(S), np64(hT), dtype) <= tol(dtype)
