@@ -53,6 +53,7 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
     size_t bytes = 0;
     if (want_bwd) bytes += align256(sizeof(float) * (size_t)B * H * dk);   // rowsum(dhT * hT)
     if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
+    if (!want_bwd && use_tc(dk, dv, dt) && T > 0) bytes += align256(tc_fwd_workspace(B, T, H));  // segments
     return bytes;
 }
 
@@ -95,8 +96,11 @@ hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const fl
         // tensor-core pass; (b,h) pairs whose chunk decay span is too wide are flagged
         // and recomputed right after by the exact route (same stream, in order)
         int *flags = (int *)workspace;
-        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, B, T, H};
-        g_launches += 2;
+        float *seg_ws = (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
+        int nseg, tps;
+        tc_fwd_segments(B, T, H, &nseg, &tps);
+        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H};
+        g_launches += nseg > 1 ? 4 : 2;
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags};

@@ -21,6 +21,7 @@ struct TcFwdArgs {
     void *o;
     float *hT;
     int *flags;        // [B*H] out: 1 where the (b,h) needs the exact route
+    float *seg_ws;     // segment aggregates, tc_fwd_workspace(B, T, H) bytes (may be null if 0)
     int B, T, H;
 };
 
@@ -51,6 +52,8 @@ cudaError_t launch_simt_fwd(const SimtFwdArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_bwd(const SimtBwdArgs &a, bool bf16, cudaStream_t st);
 
 size_t tc_fwd_smem();
+void tc_fwd_segments(int B, int T, int H, int *nseg, int *tps);
+size_t tc_fwd_workspace(int B, int T, int H);
 size_t tc_bwd_smem();
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st);
