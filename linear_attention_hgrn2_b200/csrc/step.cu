@@ -25,7 +25,7 @@ constexpr int kStepThreads = 256;
 constexpr int kStepMaxRows = 16;   // ceil(128 * 32 / 256): d_k <= 128, d_v <= 128
 
 template <typename T>
-__global__ void __launch_bounds__(kStepThreads)
+__global__ void __launch_bounds__(kStepThreads, 2)
 step_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
             float *__restrict__ S, T *__restrict__ o, int dk, int dv) {
     __shared__ float sq[128], sf[128], sk[128];

@@ -104,8 +104,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     const uint32_t tbase = m->tmem_base;
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
 
+    int issued = 0, waited = 0;
     auto issue_load = [&](int n) {
         const int s = n & 1;
+        ++issued;
         mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
         for (int c = 0; c < 2; ++c) {
             tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, n * kTile, b);
@@ -146,6 +148,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     for (n = 0; n < N; ++n) {
         const int s = n & 1;
         if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
+        waited = n + 1;
         // ---- prep: column j, rows 64*half .. +63: Kt = k / E in place of log f, E -> TMEM
         float fv[64];
         float P = 1.0f;
@@ -289,8 +292,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     }
     const bool fell_back = ok && n < N;
     if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
-    if (tid == 0) {
-        if (n + 1 < N) mbar_wait(&m->full[(n + 1) & 1], ((n + 1) >> 1) & 1);
+    if (tid == 0) {   // drain loads still landing in this CTA's shared memory, and the stores
+        for (int k = waited; k < issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
         tma_store_wait_all0();
     }
     if (ok && !fell_back && p.dhT && p.rs) {
@@ -328,7 +331,7 @@ namespace rsw {
 constexpr uint32_t kColDS = 0, kColX1 = 128, kColX2 = 256, kColE = 384;
 
 struct __align__(8) Misc {
-    uint64_t full, barP1, barP2;
+    uint64_t barIn, barDO, barDQ, barP1, barP2;
     uint32_t tmem_base;
     int pad;
     float EB[128];
@@ -339,17 +342,22 @@ constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
 }  // namespace rsw
 
 struct RevParams {
-    const __nv_bfloat16 *q, *lf, *dq;   // read back in the d log f epilogue
     const float *dhT, *rs;
     float *dh0;
     const int *flags;
     int T, H, ntiles;
 };
 
+// Shared-memory plan per chunk (7 tiles of 32 KB): Qb q -> Qt, Gb log f -> Kt, Vb v (then
+// the dq tile for the d log f epilogue), Ob dO, D16 bf16(dSh), AT mask(A)^T (then di
+// staging), DA mask(dA) (then d log f staging).  Loads: q, log f, v of the next chunk
+// start once this chunk's epilogue has read Qb, Gb, Vb; dO of the next chunk and dq of
+// this one start as soon as the MMAs are done, under the epilogue.
 __global__ void __launch_bounds__(kThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
-           const __grid_constant__ CUtensorMap tm_di, const __grid_constant__ CUtensorMap tm_dlf, RevParams p) {
+           const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_di,
+           const __grid_constant__ CUtensorMap tm_dlf, RevParams p) {
     using namespace rsw;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *Qb = smem, *Gb = smem + kTileBytes, *Vb = smem + 2 * kTileBytes, *Ob = smem + 3 * kTileBytes;
@@ -367,7 +375,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int quad = warp & 3, half = warp >> 2;
     const int j = 32 * quad + lane;
     if (tid == 0) {
-        mbar_init(&m->full, 1);
+        mbar_init(&m->barIn, 1);
+        mbar_init(&m->barDO, 1);
+        mbar_init(&m->barDQ, 1);
         mbar_init(&m->barP1, 1);
         mbar_init(&m->barP2, 1);
         fence_mbar_init();
@@ -382,16 +392,27 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t tbase = m->tmem_base;
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
 
-    auto issue_load = [&](int n) {
-        mbar_arrive_expect_tx(&m->full, 4 * kTileBytes);
+    // loads issued / arrivals waited for, per barrier (thread 0's view): [barIn, barDO, barDQ]
+    int issued[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
+    auto issue_in = [&](int n) {
+        ++issued[0];
+        mbar_arrive_expect_tx(&m->barIn, 3 * kTileBytes);
         for (int c = 0; c < 2; ++c) {
-            tma_load_4d(Qb + c * kBlk, &tm_q, &m->full, 64 * c, h, n * kTile, b);
-            tma_load_4d(Gb + c * kBlk, &tm_lf, &m->full, 64 * c, h, n * kTile, b);
-            tma_load_4d(Vb + c * kBlk, &tm_x, &m->full, 64 * c, h, n * kTile, b);
-            tma_load_4d(Ob + c * kBlk, &tm_do, &m->full, 64 * c, h, n * kTile, b);
+            tma_load_4d(Qb + c * kBlk, &tm_q, &m->barIn, 64 * c, h, n * kTile, b);
+            tma_load_4d(Gb + c * kBlk, &tm_lf, &m->barIn, 64 * c, h, n * kTile, b);
+            tma_load_4d(Vb + c * kBlk, &tm_x, &m->barIn, 64 * c, h, n * kTile, b);
         }
     };
-    if (tid == 0 && N > 0) issue_load(N - 1);
+    auto issue_one = [&](uint8_t *dst, const CUtensorMap *tm, uint64_t *bar, int n) {
+        ++issued[bar == &m->barDO ? 1 : 2];
+        mbar_arrive_expect_tx(bar, kTileBytes);
+        tma_load_4d(dst, tm, bar, 0, h, n * kTile, b);
+        tma_load_4d(dst + kBlk, tm, bar, 64, h, n * kTile, b);
+    };
+    if (tid == 0 && N > 0) {
+        issue_in(N - 1);
+        issue_one(Ob, &tm_do, &m->barDO, N - 1);
+    }
     {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
         float r0[32], r1[32];
         if (p.dhT) {
@@ -416,19 +437,19 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
     const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
     const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
-    const size_t tok_stride = (size_t)p.H * 128;
+    auto elem_off = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
     bool ok = true;
     int it = 0, n = N - 1;
     for (; n >= 0; --n, ++it) {
-        if (__syncthreads_or(!mbar_wait(&m->full, it & 1))) { ok = false; break; }
+        const uint32_t par = it & 1;
+        if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
+        waited[0] = it + 1;
         // ---- prep: Qt = q E (in place), Kt = k / E (in place of log f), E -> TMEM
         float fv[64];
         float P = 1.0f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-            const int t = 64 * half + i;
-            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
-            fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb + off)));
+            fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb + elem_off(64 * half + i))));
             P *= fv[i];
         }
         m->Ppart[half][j] = P;
@@ -436,8 +457,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         float E = half ? m->Ppart[0][j] : 1.0f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-            const int t = 64 * half + i;
-            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+            const uint32_t off = elem_off(64 * half + i);
             __nv_bfloat16 *g = reinterpret_cast<__nv_bfloat16 *>(Gb + off);
             __nv_bfloat16 *qq = reinterpret_cast<__nv_bfloat16 *>(Qb + off);
             const float a = __bfloat162float(*g);
@@ -460,6 +480,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         // ---- phase 1: A^T = Kt Qt^T (M = s, N = t), dA = dO V^T (M = t, N = s)
         if (tid == 0) {
+            if (!mbar_wait(&m->barDO, par)) ok = false;
+            else waited[1] = it + 1;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -497,7 +519,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         // ---- masks: A^T keeps t >= s (lane s), dA keeps s <= t (lane t)
         {
-            if (!mbar_wait(&m->barP1, it & 1)) ok = false;
+            if (!mbar_wait(&m->barP1, par)) ok = false;
             tc_fence_after();
             float r0[32], r1[32];
             tmem_ld32(tl + kColX1 + 64 * half, r0);
@@ -558,10 +580,12 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
             mma_commit(&m->barP2);
         }
-        if (__syncthreads_or(!mbar_wait(&m->barP2, it & 1))) { ok = false; break; }
+        if (__syncthreads_or(!mbar_wait(&m->barP2, par))) { ok = false; break; }
         tc_fence_after();
-        if (tid == 0 && n > 0) issue_load(n - 1);   // inputs of this chunk are no longer read
-
+        if (tid == 0) {
+            issue_one(Vb, &tm_dq, &m->barDQ, n);                  // dq of this chunk, for d log f
+            if (n > 0) issue_one(Ob, &tm_do, &m->barDO, n - 1);   // dO of the next chunk
+        }
         // ---- di (lane s) -> AT (rows s) for the TMA store
         {
             float r0[32], r1[32];
@@ -570,44 +594,49 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tmem_wait_ld();
             store_row_bf16(AT + half * kBlk, j, r0, r1);
         }
-        // ---- d log f (lane j, tokens 64*half .. +63), reverse cumulative sum with carry
-        float dap[64];
+        // ---- d log f (lane j, tokens 64*half .. +63): partial values (without the carry)
+        // d'_t = sum_{t<=t'<chunk half end} (q dq - k dk)_{t'} - f_t dk_t, kept in TMEM X1
+        // (di has been read out), with q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}.
+        if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
+        waited[2] = it + 1;
         float suf = 0.0f;
-        const int t_base = n * kTile + 64 * half;
 #pragma unroll
         for (int c = 1; c >= 0; --c) {
-            float dk[32], e[32];
-            tmem_ld32(tl + kColX2 + 64 * half + 32 * c, dk);
-            tmem_ld32(tl + kColE + 64 * half + 32 * c, e);
+            float dkp[32], e[32], dap[32];
+            const int col = 64 * half + 32 * c;
+            tmem_ld32(tl + kColX2 + col, dkp);
+            tmem_ld32(tl + kColE + col, e);
+            const float eprev = col > 0 ? tmem_ld1(tl + kColE + col - 1) : 1.0f;
             tmem_wait_ld();
+            float invE = __fdividef(1.0f, e[31]);
 #pragma unroll
             for (int i = 31; i >= 0; --i) {
-                const int tg = t_base + 32 * c + i;
-                float w = 0.0f, fdk = 0.0f;
-                if (tg < p.T) {
-                    const size_t gi = ((size_t)b * p.T + tg) * tok_stride + (size_t)h * 128 + j;
-                    const float a = __bfloat162float(p.lf[gi]);
-                    const float qv = __bfloat162float(p.q[gi]);
-                    const float dqv = __bfloat162float(p.dq[gi]);
-                    const float f = __expf(a);
-                    const float k = k_from(a, f);
-                    const float dkv = dk[i] * __fdividef(1.0f, e[i]);
-                    w = qv * dqv - k * dkv;
-                    fdk = f * dkv;
-                }
-                suf += w;
-                dap[32 * c + i] = suf - fdk;
+                const int t = col + i;
+                const uint32_t off = elem_off(t);
+                const float qt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Qb + off));
+                const float kt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb + off));
+                const float dq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Vb + off));
+                const float invEm1 = __fdividef(1.0f, i > 0 ? e[i - 1] : eprev);
+                suf += qt * invE * dq - kt * dkp[i];
+                dap[i] = suf - dkp[i] * invEm1;
+                invE = invEm1;
             }
+            tmem_st32(tl + kColX1 + col, dap);
         }
+        tmem_wait_st();
         m->Ppart[half][j] = suf;
         __syncthreads();
         {
             const float carry = m->carry[j] + (half == 0 ? m->Ppart[1][j] : 0.0f);
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const int t = 64 * half + i;
-                *reinterpret_cast<__nv_bfloat16 *>(DA + cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin) =
-                    __float2bfloat16_rn(dap[i] + carry);
+            for (int c = 0; c < 2; ++c) {
+                float dap[32];
+                const int col = 64 * half + 32 * c;
+                tmem_ld32(tl + kColX1 + col, dap);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(DA + elem_off(col + i)) = __float2bfloat16_rn(dap[i] + carry);
             }
         }
         fence_proxy_async_smem();
@@ -620,15 +649,17 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA + kBlk, 64, h, n * kTile, b);
             tma_store_commit();
+            if (n > 0) issue_in(n - 1);   // the epilogue has read Qb, Gb, Vb
         }
     }
     if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
-    if (tid == 0) {
-        // a load was issued for chunk n-1 only after chunk n's MMAs completed; after a break
-        // at chunk n before that point, nothing is in flight except chunk n itself (waited)
+    if (tid == 0) {   // drain loads that may still be landing in this CTA's shared memory
+        uint64_t *bars[3] = {&m->barIn, &m->barDO, &m->barDQ};
+        for (int q = 0; q < 3; ++q)
+            for (int k = waited[q]; k < issued[q]; ++k) mbar_wait(bars[q], k & 1, 2000000u);
         tma_store_wait_all0();
     }
-    if (ok && p.dh0) {
+    if (ok && n < 0 && p.dh0) {
         tc_fence_after();
         float r0[32], r1[32];
         tmem_ld32(tl + kColDS + 64 * half, r0);
@@ -641,7 +672,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             dst[8 + i] = make_float4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
         }
     }
-    if (tid == 0 && ok) atomicAdd(&g_counters[1], (unsigned long long)N);
+    if (tid == 0 && ok && n < 0) atomicAdd(&g_counters[1], (unsigned long long)N);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -672,9 +703,8 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     tcb::dq_kernel<<<a.B * a.H, tcb::kThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    tcb::RevParams p2{(const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.dq,
-                      a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles};
-    tcb::rev_kernel<<<a.B * a.H, tcb::kThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdi, mdl, p2);
+    tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles};
+    tcb::rev_kernel<<<a.B * a.H, tcb::kThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, p2);
     return cudaGetLastError();
 }
 

@@ -100,8 +100,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
 
+    int issued = 0, waited = 0;   // chunks whose loads were issued / whose arrival was waited for
     auto issue_load = [&](int n) {
         const int s = n & 1;
+        ++issued;
         mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
         for (int c = 0; c < 2; ++c) {
             tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
@@ -155,6 +157,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     for (n = 0; n < N; ++n) {
         const int s = n & 1;
         if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
+        waited = n + 1;
 
         // ---- prep pass 1: f = exp(log f) kept in registers, partial products per 32-row range
         float f0[32], f1[32];
@@ -315,10 +318,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
     const bool fell_back = ok && n < N;
     if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
-    // drain: a load still in flight into this CTA's shared memory (chunk n+1 was issued
-    // once chunk n-1 completed), and the last o store
+    // drain: loads still landing in this CTA's shared memory, and the last o store
     if (tid == 0) {
-        if (n + 1 < N) mbar_wait(&m->full[(n + 1) & 1], ((n + 1) >> 1) & 1);
+        for (int k = waited; k < issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
         tma_store_wait_all0();
     }
     if (ok && !fell_back && p.hT && seg == p.nseg - 1) {
@@ -400,8 +402,10 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
+    int issued = 0, waited = 0;
     auto issue_load = [&](int n) {
         const int s = n & 1;
+        ++issued;
         mbar_arrive_expect_tx(&m->full[s], 2 * kTileBytes);
         for (int c = 0; c < 2; ++c) {
             tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
@@ -431,6 +435,7 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
     for (int n = 0; n < N; ++n) {
         const int s = n & 1;
         if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
+        waited = n + 1;
         float f0[32], f1[32];
         float P0 = 1.0f, P1 = 1.0f;
 #pragma unroll
@@ -498,7 +503,10 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
         tc_fence_after();
         if (tid == 0 && n + 2 < N) issue_load(n + 2);
     }
-    if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
+    if (!ok && tid == 0) {
+        set_status(HGRN2_ERR_TIMEOUT);
+        for (int k = waited; k < issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
+    }
     if (ok) {
         float r0[32], r1[32];
         tmem_ld32(tl + 64 * ch, r0);
