@@ -105,6 +105,30 @@ hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const fl
                        int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
                        void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* Allocation-free variant of hgrn2_bwd.  The paper has no counterpart: this
+ * entry point exists for callers that cannot give the library a device
+ * buffer -- for example a plain C host program that links only this library
+ * and owns no device allocator, or a service whose memory policy forbids new
+ * device allocations once it is running (cudaMalloc and cudaFree synchronise
+ * the device and can stall unrelated work).  Arguments and results are those
+ * of hgrn2_bwd without the workspace.  Its scratch is a fixed array of
+ * HGRN2_NOALLOC_SCRATCH_BYTES bytes inside the library, which every GPU that
+ * loads the library keeps until the process exits; sizes whose backward needs
+ * more scratch than that (for d_k = 128 and bf16: B*H > 2032) return
+ * HGRN2_ERR_UNSUPPORTED and launch nothing.  The first call on a device looks
+ * up the array's device address on that device (make that first call before
+ * any stream capture on it).  All calls share the one array and it keeps the
+ * last call's contents; nothing in it needs to start at zero, because each call
+ * writes what it reads.  Calls that may overlap on the GPU (on different
+ * streams, or from different host threads) race on the array: serialise them.
+ * This entry point calls no device allocation routine. */
+#define HGRN2_NOALLOC_SCRATCH_BYTES (1u << 20)
+hgrn2_status hgrn2_bwd_noalloc(const void *q, const void *log_f, const void *i, const float *h0,
+                               const void *dO, const float *dhT,
+                               void *dq, void *dlog_f, void *di, float *dh0,
+                               int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                               cudaStream_t stream);
+
 /* One recurrent decode step for B sequences with one new token each (§1: linear-
  * time recurrent inference without a KV cache; the §3.2 recurrence for one t):
  *   S <- Diag(f) S + k i^T  (in place, float32),  then  o = S^T q.

@@ -26,7 +26,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(
 FP32, BF16 = 0, 1
 
 # Every extern "C" symbol of include/hgrn2.h.
-EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_step",
+EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_bwd_noalloc", "hgrn2_step",
            "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
 
 _lib = None
@@ -54,6 +54,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_fwd.restype = i32
     lib.hgrn2_bwd.argtypes = [vp] * 10 + [i32] * 7 + [vp, sz, vp]
     lib.hgrn2_bwd.restype = i32
+    lib.hgrn2_bwd_noalloc.argtypes = [vp] * 10 + [i32] * 7 + [vp]
+    lib.hgrn2_bwd_noalloc.restype = i32
     lib.hgrn2_step.argtypes = [vp] * 5 + [i32] * 5 + [vp]
     lib.hgrn2_step.restype = i32
     lib.hgrn2_get_device_status.argtypes = [vp]

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -200,3 +201,47 @@ const char *hgrn2_status_string(hgrn2_status s) {
 const char *hgrn2_version(void) { return "hgrn2-b200 0.1"; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free backward
+// Scratch of hgrn2_bwd_noalloc: a fixed-size array in the library's own device
+// memory, present on every GPU the library is loaded on for the life of the
+// process.  Host code only ever sees a stand-in for this symbol; the device
+// address is looked up per device with cudaGetSymbolAddress and cached.
+namespace {
+constexpr size_t kNoAllocScratchBytes = HGRN2_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device (looked up once per device).
+hgrn2_status noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return HGRN2_ERR_CUDA;
+    if (dev >= kMaxDevices) return HGRN2_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HGRN2_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return HGRN2_OK;
+}
+}  // namespace
+
+extern "C" hgrn2_status hgrn2_bwd_noalloc(const void *q, const void *log_f, const void *i, const float *h0,
+                                          const void *dO, const float *dhT, void *dq, void *dlog_f, void *di,
+                                          float *dh0, int B, int T, int H, int dk, int dv, int chunk,
+                                          hgrn2_dtype dtype, cudaStream_t stream) {
+    hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    const size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
+    if (need > kNoAllocScratchBytes) return HGRN2_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    s = noalloc_scratch(&scratch);
+    if (s != HGRN2_OK) return s;
+    return hgrn2_bwd(q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype, scratch,
+                     kNoAllocScratchBytes, stream);
+}
