@@ -7,24 +7,30 @@
 // ("HGRN2: Gated Linear RNNs with State Expansion", §3.2: gated linear attention
 // with key 1 - f, value i, query q, so chunkwise; §5: per-dimension decay):
 //
-//   Qt = q * E,  Kt = k / E,  Kh = Kt * E_B = k * E_B / E     (all bf16 in smem)
+//   Qt = q * E,  Kt = k / E                                    (bf16 in smem)
 //   A  = mask_{s<=t}(Qt Kt^T)                                  tcgen05, fp32 in TMEM
 //   O  = Qt bf16(S_in) + bf16(A) V                             tcgen05, fp32 in TMEM
-//   S  = Diag(E_B) S_in + Kh^T V                               fp32 state in TMEM
+//   S' = S_in + Kt^T V,   S_out = Diag(E_B) S'                 fp32 state in TMEM
 //
-// Qt Kt^T realises sum_j q_t[j] k_s[j] exp(b_t[j] - b_s[j]) through factors
-// referenced to the chunk start; it is valid while 1/E stays representable with
-// margin, i.e. min_j E_B[j] >= 1e-26 (a cumulative log-decay span of about 60
-// inside the chunk).  A (batch, head) meeting a chunk beyond that is flagged and
-// recomputed afterwards by the exact CUDA-core route, which forms every
-// exponent as a difference of cumulative sums.
+// The state is post-scaled: the MMA accumulates Kt^T V onto S_in, and the next
+// chunk multiplies the rows by this chunk's E_B before using it (the products
+// Kt * E_B = k * E_B / E <= k are never formed in bf16 at all).  Qt Kt^T realises
+// sum_j q_t[j] k_s[j] exp(b_t[j] - b_s[j]) through factors referenced to the
+// chunk start; it is valid while 1/E stays representable with margin, i.e.
+// min_j E_B[j] >= 1e-26 (a cumulative log-decay span of about 60 inside the
+// chunk).  A (batch, head) meeting a chunk beyond that is flagged and recomputed
+// afterwards by the exact CUDA-core route, which forms every exponent as a
+// difference of cumulative sums.
 //
-// Data movement: q, log f, i tiles arrive by TMA (128-byte swizzle, two
-// 64-column boxes per 128 x 128 tile) into a two-stage ring, so the next chunk
-// loads while this one computes; o leaves by TMA store.  The state never leaves
-// TMEM between chunks (d_k lanes x d_v fp32 columns); Diag(E_B) is a per-lane
-// scale applied with tcgen05.ld/st.  The MMAs are issued by one thread;
-// completion is tracked with tcgen05.commit on mbarriers.  Every wait is bounded.
+// Warp roles (16 warps), coordinated by mbarriers only:
+//   warp 0      TMA producer: q, log f, i tiles (128-byte swizzle) into a 2-stage ring
+//   warp 1      TMEM allocator and the single MMA-issuing thread
+//   warps 4-7   TMEM warps (one thread per TMEM lane): S phase (bf16 copy of S_in,
+//               Diag(E_B) scale), causal mask of A, o epilogue (stored from registers)
+//   warps 8-15  prep warps: f, E, k, Qt, Kt for the next chunk while the current one
+//               is on the tensor cores
+// Every wait is bounded; a wait that gives up records HGRN2_ERR_TIMEOUT.
+#include <climits>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -37,16 +43,19 @@ namespace tcf {
 using namespace tc;
 using namespace tcc;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;        // aggregate kernel
+constexpr int kFwdThreads = 512;     // forward kernel: 16 warps
 constexpr uint32_t kColS = 0, kColO = 128, kColA = 256, kTmemCols = 512;
 
 struct __align__(8) Misc {
-    uint64_t full[2];
-    uint64_t barA, barO1, barM;
+    uint64_t full[2], prepped[2], empty[2];
+    uint64_t barA, barO1, barS, barO2;      // MMA completions (tcgen05.commit)
+    uint64_t sdone, adone, ofree;           // TMEM-warp arrivals (128 each)
     uint32_t tmem_base;
-    int bad;
-    float EB[128];
-    float Ppart[4][128];
+    int bad_tile;                           // first chunk whose decay span is too wide
+    int waited_full;                        // chunks whose arrival the prep warps consumed
+    float EB[3][128];                       // E_B ring (read one chunk later by the S phase)
+    float Ppart[128];                       // product of f over rows 0..63, per key dim
 };
 
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
@@ -54,15 +63,48 @@ constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
 struct Params {
     const float *h0;
     float *hT;
+    __nv_bfloat16 *o;
     int *flags;       // [B*H] set to 1 when the (b,h) must take the exact route
     const float *Sin; // [B*H][nseg-1][128][128] state entering segments 1.. (from the scan)
     int T, H, ntiles;
     int nseg, tps;    // sequence segments per (b,h) and chunks per segment
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
+
+// Waits for phase `parity` of `bar`, or returns false early once `*bad <= tile` (the
+// pipeline stopped before that phase could complete) or after a bounded number of polls.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const int *bad, int tile) {
+    for (uint32_t it = 0; it < 20000000u; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (ld_volatile(bad) <= tile) return false;
+        if (it > 64) __nanosleep(32);
+    }
+    set_status(HGRN2_ERR_TIMEOUT);
+    return false;
+}
+
+// One 32-column chunk (c = 0..3) of a TMEM row -> bf16 into row `row` of a swizzled 128 x 128 tile.
+__device__ __forceinline__ void store_chunk_bf16(uint8_t *tile, int row, int c, const float (&r)[32]) {
+    uint8_t *base = tile + (c >> 1) * kBlk + row * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int chunk = 4 * (c & 1) + q;
+        uint4 v;
+        v.x = pack_bf2(r[8 * q + 0], r[8 * q + 1]);
+        v.y = pack_bf2(r[8 * q + 2], r[8 * q + 3]);
+        v.z = pack_bf2(r[8 * q + 4], r[8 * q + 5]);
+        v.w = pack_bf2(r[8 * q + 6], r[8 * q + 7]);
+        *reinterpret_cast<uint4 *>(base + ((chunk ^ (row & 7)) << 4)) = v;
+    }
+}
+
+__global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
-           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o, Params p) {
+           const __grid_constant__ CUtensorMap tm_x, Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *Qb[2] = {smem, smem + 3 * kTileBytes};
     uint8_t *Gb[2] = {smem + kTileBytes, smem + 4 * kTileBytes};
@@ -79,19 +121,26 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         return;
     }
     if (tid == 0) {
-        mbar_init(&m->full[0], 1);
-        mbar_init(&m->full[1], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->prepped[s], 256);
+            mbar_init(&m->empty[s], 1);
+        }
         mbar_init(&m->barA, 1);
         mbar_init(&m->barO1, 1);
-        mbar_init(&m->barM, 1);
+        mbar_init(&m->barS, 1);
+        mbar_init(&m->barO2, 1);
+        mbar_init(&m->sdone, 128);
+        mbar_init(&m->adone, 128);
+        mbar_init(&m->ofree, 128);
+        m->bad_tile = INT_MAX;
+        m->waited_full = 0;
         fence_mbar_init();
-        m->bad = 0;
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_lf);
         tma_prefetch_desc(&tm_x);
-        tma_prefetch_desc(&tm_o);
     }
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(&m->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -99,255 +148,237 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
+    int producer_issued = 0;
 
-    int issued = 0, waited = 0;   // chunks whose loads were issued / whose arrival was waited for
-    auto issue_load = [&](int n) {
-        const int s = n & 1;
-        ++issued;
-        mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
-        for (int c = 0; c < 2; ++c) {
-            tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
-            tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
-            tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
-        }
-    };
-    if (tid == 0) {
-        issue_load(0);
-        if (N > 1) issue_load(1);
-    }
-
-    // TMEM lane quadrant and column half of this warp
-    const int quad = warp & 3, ch = warp >> 2;
-    const int lrow = 32 * quad + lane;                       // TMEM lane = row of the tile
-    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
-
-    // state init: S = h0 (or 0) for the first segment, the scanned incoming state otherwise;
-    // rows j = lrow, columns 64ch .. 64ch+63
-    {
-        float r0[32], r1[32];
-        const float *init = seg == 0 ? (p.h0 ? p.h0 + (size_t)bh * 16384 : nullptr)
-                                     : p.Sin + ((size_t)bh * (p.nseg - 1) + seg - 1) * 16384;
-        if (init) {
-            const float4 *src = reinterpret_cast<const float4 *>(init + (size_t)lrow * 128 + 64 * ch);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float4 a = src[i], c = src[8 + i];
-                r0[4 * i] = a.x; r0[4 * i + 1] = a.y; r0[4 * i + 2] = a.z; r0[4 * i + 3] = a.w;
-                r1[4 * i] = c.x; r1[4 * i + 1] = c.y; r1[4 * i + 2] = c.z; r1[4 * i + 3] = c.w;
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            for (int n = 0; n < N; ++n) {
+                const int s = n & 1;
+                if (ld_volatile(&m->bad_tile) < n) break;
+                if (n >= 2 && !wait_or_abort(&m->empty[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
+                mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
+                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
+                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
+                }
+                ++producer_issued;
             }
-        } else {
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_kk = idesc_bf16(128, 128, false, false);
+            const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
+            const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+            for (int n = 0; n < N; ++n) {
+                const int s = n & 1;
+                if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                if (ld_volatile(&m->bad_tile) <= n) break;
+                tc_fence_after();
+                // A = Qt Kt^T
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0.0f;
-        }
-        tmem_st32(tl + kColS + 64 * ch, r0);
-        tmem_st32(tl + kColS + 64 * ch + 32, r1);
-        tmem_wait_st();
-    }
-
-    const uint32_t id_kk = idesc_bf16(128, 128, false, false);
-    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
-    const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
-    const int pc = tid & 63, rr = tid >> 6;                  // prep: column pair, 32-row range
-    const int col0 = 2 * pc;
-    const uint32_t poff_blk = (uint32_t)(col0 >> 6) * kBlk;
-    const int pchunk = (col0 & 63) >> 3, pin = (col0 & 7) * 2;
-    bool ok = true;
-    int n = 0;
-
-    for (n = 0; n < N; ++n) {
-        const int s = n & 1;
-        if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
-        waited = n + 1;
-
-        // ---- prep pass 1: f = exp(log f) kept in registers, partial products per 32-row range
-        float f0[32], f1[32];
-        float P0 = 1.0f, P1 = 1.0f;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColA, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
+                                sdesc_sw128(smem_u32(Gb[s]) + ko, 16, 1024), id_kk, kk > 0);
+                }
+                mma_commit(&m->barA);
+                // O = Qt bf16(S_in) once the S phase wrote it and the last epilogue read O;
+                // S' = S_in + Kt^T V
+                if (!mbar_wait(&m->sdone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                if (n >= 1 && !mbar_wait(&m->ofree, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int t = 32 * rr + i;
-            const uint32_t off = poff_blk + t * 128 + (((uint32_t)pchunk ^ (t & 7)) << 4) + pin;
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + off);
-            f0[i] = __expf(bf_lo(w));
-            f1[i] = __expf(bf_hi(w));
-            P0 *= f0[i];
-            P1 *= f1[i];
-        }
-        m->Ppart[rr][col0] = P0;
-        m->Ppart[rr][col0 + 1] = P1;
-        __syncthreads();
-        // ---- prep pass 2: Qt = q E and Kt = k / E in place
-        float E0 = 1.0f, E1 = 1.0f;
-        for (int r2 = 0; r2 < rr; ++r2) {
-            E0 *= m->Ppart[r2][col0];
-            E1 *= m->Ppart[r2][col0 + 1];
-        }
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
+                                sdesc_sw128(smem_u32(X) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
+                }
+                mma_commit(&m->barO1);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int t = 32 * rr + i;
-            const uint32_t off = poff_blk + t * 128 + (((uint32_t)pchunk ^ (t & 7)) << 4) + pin;
-            uint32_t *gq = reinterpret_cast<uint32_t *>(Qb[s] + off);
-            uint32_t *gg = reinterpret_cast<uint32_t *>(Gb[s] + off);
-            const uint32_t wa = *gg, wq = *gq;
-            E0 *= f0[i];
-            E1 *= f1[i];
-            const float k0 = k_from(bf_lo(wa), f0[i]), k1 = k_from(bf_hi(wa), f1[i]);
-            *gq = pack_bf2(bf_lo(wq) * E0, bf_hi(wq) * E1);
-            *gg = pack_bf2(k0 * __fdividef(1.0f, E0), k1 * __fdividef(1.0f, E1));
-        }
-        if (rr == 3) {
-            m->EB[col0] = E0;
-            m->EB[col0 + 1] = E1;
-        }
-        fence_proxy_async_smem();
-        const int bad = __syncthreads_or(rr == 3 && !(E0 >= kMinEB && E1 >= kMinEB));
-        if (bad) break;
-
-        // ---- A = Qt Kt^T
-        if (tid == 0) {
-            tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
+                                sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                mma_commit(&m->barS);
+                // O += bf16(mask(A)) V once the TMEM warps wrote it
+                if (!mbar_wait(&m->adone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColA, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Gb[s]) + ko, 16, 1024), id_kk, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
+                                sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
+                }
+                mma_commit(&m->barO2);
+                mma_commit(&m->empty[s]);   // stage s is free once everything above completed
             }
-            mma_commit(&m->barA);
-            tma_store_wait_read0();   // the previous chunk's o store has finished reading X
         }
-        __syncthreads();
-
-        // ---- S phase: bf16 copy of S_in into X (B operand, MN-major) and S <- Diag(E_B) S
-        {
-            float r0[32], r1[32];
-            tc_fence_after();
-            tmem_ld32(tl + kColS + 64 * ch, r0);
-            tmem_ld32(tl + kColS + 64 * ch + 32, r1);
-            tmem_wait_ld();
-            store_row_bf16(X + ch * kBlk, lrow, r0, r1);
-            const float e = m->EB[lrow];
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ TMEM warps
+        const int quad = warp & 3, r = 32 * quad + lane;             // TMEM lane = tile row
+        const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+        {   // S = h0 / scanned incoming state / 0
+            const float *init = seg == 0 ? (p.h0 ? p.h0 + (size_t)bh * 16384 : nullptr)
+                                         : p.Sin + ((size_t)bh * (p.nseg - 1) + seg - 1) * 16384;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                r0[i] *= e;
-                r1[i] *= e;
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                if (init) {
+                    const float4 *src = reinterpret_cast<const float4 *>(init + (size_t)r * 128 + 32 * c);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 a = src[i];
+                        v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                }
+                tmem_st32(tl + kColS + 32 * c, v);
             }
-            tmem_st32(tl + kColS + 64 * ch, r0);
-            tmem_st32(tl + kColS + 64 * ch + 32, r1);
             tmem_wait_st();
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+        const size_t orow_stride = (size_t)p.H * 128;
+        int n = 0;
+        for (; n < N; ++n) {
+            const int s = n & 1;
+            if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (ld_volatile(&m->bad_tile) <= n) break;
+            // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand)
+            if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            tc_fence_after();
+            const float e = n >= 1 ? m->EB[(n - 1) % 3][r] : 1.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColS + 32 * c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= e;
+                store_chunk_bf16(X, r, c, v);
+                tmem_st32(tl + kColS + 32 * c, v);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->sdone);
+            // causal mask of A, bf16 -> X (A operand) once the inter-chunk MMA has read X
+            if (!mbar_wait(&m->barA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (!mbar_wait(&m->barO1, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(X) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
-            }
-            mma_commit(&m->barO1);
-        }
-
-        // ---- Kh = Kt * E_B in place (after the A MMA has read Kt)
-        if (!mbar_wait(&m->barA, n & 1)) ok = false;
-        tc_fence_after();
-        {
-            const float e0 = m->EB[col0], e1 = m->EB[col0 + 1];
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) {
-                const int t = 32 * rr + i;
-                const uint32_t off = poff_blk + t * 128 + (((uint32_t)pchunk ^ (t & 7)) << 4) + pin;
-                uint32_t *gg = reinterpret_cast<uint32_t *>(Gb[s] + off);
-                const uint32_t w = *gg;
-                *gg = pack_bf2(bf_lo(w) * e0, bf_hi(w) * e1);
-            }
-        }
-        // ---- A phase: causal mask, bf16 into X (A operand, K-major) once the inter MMA is done with X
-        {
-            float r0[32], r1[32];
-            tmem_ld32(tl + kColA + 64 * ch, r0);
-            tmem_ld32(tl + kColA + 64 * ch + 32, r1);
-            tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColA + 32 * c, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (64 * ch + i > lrow) r0[i] = 0.0f;
-                if (64 * ch + 32 + i > lrow) r1[i] = 0.0f;
+                for (int i = 0; i < 32; ++i)
+                    if (32 * c + i > r) v[i] = 0.0f;
+                store_chunk_bf16(X, r, c, v);
             }
-            if (!mbar_wait(&m->barO1, n & 1)) { ok = false; }
-            store_row_bf16(X + ch * kBlk, lrow, r0, r1);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(!ok)) { ok = false; break; }
-        if (tid == 0) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->adone);
+            // o epilogue: row r of the chunk, straight from TMEM to global memory
+            if (!mbar_wait(&m->barO2, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
+            const int t = (g0 + n) * kTile + r;
+            __nv_bfloat16 *orow = p.o + ((size_t)b * p.T + t) * orow_stride + (size_t)h * 128;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColO + 32 * c, v);
+                tmem_wait_ld();
+                if (t < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pack_bf2(v[8 * q], v[8 * q + 1]), pack_bf2(v[8 * q + 2], v[8 * q + 3]),
+                                            pack_bf2(v[8 * q + 4], v[8 * q + 5]), pack_bf2(v[8 * q + 6], v[8 * q + 7]));
+                }
             }
+            tc_fence_before();
+            mbar_arrive(&m->ofree);
+        }
+        // the last state MMA must be complete before hT is read or TMEM is released
+        if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
+        tc_fence_after();
+        if (n == N && p.hT && seg == p.nseg - 1) {
+            const float e = m->EB[(N - 1) % 3][r];
+            float *dst = p.hT + ((size_t)bh * 128 + r) * 128;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColS + 32 * c, v);
+                tmem_wait_ld();
+                float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    d4[i] = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
             }
-            mma_commit(&m->barM);
         }
-        if (__syncthreads_or(!mbar_wait(&m->barM, n & 1))) { ok = false; break; }
-        tc_fence_after();
-        if (tid == 0 && n + 2 < N) issue_load(n + 2);
-
-        // ---- epilogue: O (fp32 TMEM) -> bf16 -> X -> TMA store
-        {
-            float r0[32], r1[32];
-            tmem_ld32(tl + kColO + 64 * ch, r0);
-            tmem_ld32(tl + kColO + 64 * ch + 32, r1);
-            tmem_wait_ld();
-            store_row_bf16(X + ch * kBlk, lrow, r0, r1);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_4d(&tm_o, X, 0, h, (g0 + n) * kTile, b);
-            tma_store_4d(&tm_o, X + kBlk, 64, h, (g0 + n) * kTile, b);
-            tma_store_commit();
-        }
-    }
-
-    const bool fell_back = ok && n < N;
-    if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
-    // drain: loads still landing in this CTA's shared memory, and the last o store
-    if (tid == 0) {
-        for (int k = waited; k < issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
-        tma_store_wait_all0();
-    }
-    if (ok && !fell_back && p.hT && seg == p.nseg - 1) {
-        tc_fence_after();
-        float r0[32], r1[32];
-        tmem_ld32(tl + kColS + 64 * ch, r0);
-        tmem_ld32(tl + kColS + 64 * ch + 32, r1);
-        tmem_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(p.hT + ((size_t)bh * 128 + lrow) * 128 + 64 * ch);
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ prep warps
+        // thread = one key dim j (column) and one half of the chunk's rows
+        const int ptid = tid - 256;
+        const int j = ptid & 127, half = ptid >> 7;
+        const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
+        for (int n = 0; n < N; ++n) {
+            const int s = n & 1;
+            if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (ptid == 0) m->waited_full = n + 1;
+            float fv[64];
+            float P = 1.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            dst[i] = make_float4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
-            dst[8 + i] = make_float4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
+            for (int i = 0; i < 64; ++i) {
+                const int t = 64 * half + i;
+                const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+                fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + off)));
+                P *= fv[i];
+            }
+            if (half == 0) m->Ppart[j] = P;
+            named_bar_sync(1, 256);
+            float E = half ? m->Ppart[j] : 1.0f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const int t = 64 * half + i;
+                const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
+                __nv_bfloat16 *gq = reinterpret_cast<__nv_bfloat16 *>(Qb[s] + off);
+                __nv_bfloat16 *gg = reinterpret_cast<__nv_bfloat16 *>(Gb[s] + off);
+                const float a = __bfloat162float(*gg);
+                E *= fv[i];
+                *gq = __float2bfloat16_rn(__bfloat162float(*gq) * E);
+                *gg = __float2bfloat16_rn(k_from(a, fv[i]) * __fdividef(1.0f, E));
+            }
+            if (half == 1) {
+                m->EB[n % 3][j] = E;
+                if (!(E >= kMinEB)) atomicMin(&m->bad_tile, n);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 256);   // bad_tile settled, Ppart free for the next chunk
+            mbar_arrive(&m->prepped[s]);
+            if (ld_volatile(&m->bad_tile) <= n) break;
         }
     }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int bad = m->bad_tile;
+    const bool fell_back = bad < N;
+    if (warp == 0 && lane == 0)   // drain loads still landing in this CTA's shared memory
+        for (int k = m->waited_full; k < producer_issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
     if (tid == 0) {
         if (p.nseg == 1) p.flags[bh] = fell_back ? 1 : 0;   // sole writer
         else if (fell_back) p.flags[bh] = 1;                  // zeroed by the aggregate kernel
         if (fell_back) atomicAdd(&g_counters[0], 1ull);
-        if (ok && !fell_back) atomicAdd(&g_counters[1], (unsigned long long)N);
+        else atomicAdd(&g_counters[1], (unsigned long long)N);
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+    __syncwarp();
+    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
-
 
 // ------------------------------------------------------------------ sequence segments
 // For few (batch, head) pairs, each sequence is cut into segments of `tps` chunks run by
@@ -573,9 +604,9 @@ size_t tc_fwd_workspace(int B, int T, int H) {
 size_t tc_fwd_smem() { return tcf::kSmemBytes; }
 
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
-    CUtensorMap mq, ml, mx, mo;
+    CUtensorMap mq, ml, mx;
     if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
-        !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mo, a.o, a.B, a.T, a.H))
+        !make_token_map(&mx, a.x, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(tcf::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcf::kSmemBytes);
@@ -594,8 +625,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
         tcf::scan_kernel<<<BH * 16, 256, 0, st>>>(a.h0, U, g, nseg);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    tcf::Params p{a.h0, a.hT, a.flags, U, a.T, a.H, ntiles, nseg, tps};
-    tcf::fwd_kernel<<<BH * nseg, tcf::kThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, p);
+    tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, a.flags, U, a.T, a.H, ntiles, nseg, tps};
+    tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, p);
     return cudaGetLastError();
 }
 
