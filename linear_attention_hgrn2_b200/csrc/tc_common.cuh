@@ -13,6 +13,7 @@ constexpr int kTile = 128;               // tokens per chunk (one M = 128 MMA ti
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kBlk = 128 * 128;          // bytes of one 64-column block of a 128-row tile
 constexpr float kMinEB = 1e-26f;         // factorisation range: min_j E_B[j] (decay span ~60)
+constexpr float kMinLogEB = -59.8f;      // the same bound on the chunk's summed log decay
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

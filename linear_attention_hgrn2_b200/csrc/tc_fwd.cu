@@ -55,7 +55,6 @@ struct __align__(8) Misc {
     int bad_tile;                           // first chunk whose decay span is too wide
     int waited_full;                        // chunks whose arrival the prep warps consumed
     float EB[3][128];                       // E_B ring (read one chunk later by the S phase)
-    float Ppart[128];                       // product of f over rows 0..63, per key dim
 };
 
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
@@ -81,7 +80,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, co
     for (uint32_t it = 0; it < 20000000u; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (ld_volatile(bad) <= tile) return false;
-        if (it > 64) __nanosleep(32);
+        if (it > (1u << 20)) __nanosleep(64);
     }
     set_status(HGRN2_ERR_TIMEOUT);
     return false;
@@ -104,7 +103,7 @@ __device__ __forceinline__ void store_chunk_bf16(uint8_t *tile, int row, int c, 
 
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
-           const __grid_constant__ CUtensorMap tm_x, Params p) {
+           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o, Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *Qb[2] = {smem, smem + 3 * kTileBytes};
     uint8_t *Gb[2] = {smem + kTileBytes, smem + 4 * kTileBytes};
@@ -139,6 +138,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_lf);
         tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_o);
     }
     if (warp == 1) {
         tmem_alloc(&m->tmem_base, kTmemCols);
@@ -212,7 +212,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
                 }
                 mma_commit(&m->barO2);
-                mma_commit(&m->empty[s]);   // stage s is free once everything above completed
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -240,7 +239,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
             tmem_wait_st();
         }
-        const size_t orow_stride = (size_t)p.H * 128;
         int n = 0;
         for (; n < N; ++n) {
             const int s = n & 1;
@@ -281,27 +279,30 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->adone);
-            // o epilogue: row r of the chunk, straight from TMEM to global memory
+            // o epilogue: O -> bf16 rows in the chunk's q buffer (free: every MMA of the chunk
+            // completed) -> TMA store; the stage is released once the store has read it
             if (!mbar_wait(&m->barO2, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
-            const int t = (g0 + n) * kTile + r;
-            __nv_bfloat16 *orow = p.o + ((size_t)b * p.T + t) * orow_stride + (size_t)h * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
                 tmem_ld32(tl + kColO + 32 * c, v);
                 tmem_wait_ld();
-                if (t < p.T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(pack_bf2(v[8 * q], v[8 * q + 1]), pack_bf2(v[8 * q + 2], v[8 * q + 3]),
-                                            pack_bf2(v[8 * q + 4], v[8 * q + 5]), pack_bf2(v[8 * q + 6], v[8 * q + 7]));
-                }
+                store_chunk_bf16(Qb[s], r, c, v);
             }
+            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->ofree);
+            named_bar_sync(2, 128);
+            if (r == 0) {
+                tma_store_4d(&tm_o, Qb[s], 0, h, (g0 + n) * kTile, b);
+                tma_store_4d(&tm_o, Qb[s] + kBlk, 64, h, (g0 + n) * kTile, b);
+                tma_store_commit();
+                tma_store_wait_read0();
+                mbar_arrive(&m->empty[s]);
+            }
         }
+        if (r == 0) tma_store_wait_all0();
         // the last state MMA must be complete before hT is read or TMEM is released
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
@@ -321,43 +322,55 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ prep warps
-        // thread = one key dim j (column) and one half of the chunk's rows
+        // thread = one key dim j (column) and one half of the chunk's rows.  The decay is
+        // formed from the running sum b of log f: E = exp(b), 1/E = exp(-b); threads of the
+        // second half first sum log f over the first half.  Rows go in batches of 16: all
+        // loads, then the arithmetic, then all stores (so loads are not held behind stores).
         const int ptid = tid - 256;
         const int j = ptid & 127, half = ptid >> 7;
         const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
+        auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
         for (int n = 0; n < N; ++n) {
             const int s = n & 1;
             if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ptid == 0) m->waited_full = n + 1;
-            float fv[64];
-            float P = 1.0f;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const int t = 64 * half + i;
-                const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
-                fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + off)));
-                P *= fv[i];
+            float bsum = 0.0f;
+            if (half) {
+#pragma unroll 16
+                for (int t = 0; t < 64; ++t) bsum += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t)));
             }
-            if (half == 0) m->Ppart[j] = P;
-            named_bar_sync(1, 256);
-            float E = half ? m->Ppart[j] : 1.0f;
+            float invEprev = __expf(-bsum);
+#pragma unroll 1
+            for (int bt = 0; bt < 4; ++bt) {
+                const int t0 = 64 * half + 16 * bt;
+                float av[16], qv[16];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const int t = 64 * half + i;
-                const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
-                __nv_bfloat16 *gq = reinterpret_cast<__nv_bfloat16 *>(Qb[s] + off);
-                __nv_bfloat16 *gg = reinterpret_cast<__nv_bfloat16 *>(Gb[s] + off);
-                const float a = __bfloat162float(*gg);
-                E *= fv[i];
-                *gq = __float2bfloat16_rn(__bfloat162float(*gq) * E);
-                *gg = __float2bfloat16_rn(k_from(a, fv[i]) * __fdividef(1.0f, E));
+                for (int i = 0; i < 16; ++i) {
+                    av[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t0 + i)));
+                    qv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Qb[s] + eoff(t0 + i)));
+                }
+                __nv_bfloat16 oq[16], ok[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    bsum += av[i];
+                    const float E = __expf(bsum), invE = __expf(-bsum);
+                    const float k = fabsf(av[i]) < 0.25f ? k_from(av[i], 0.0f) : 1.0f - E * invEprev;
+                    oq[i] = __float2bfloat16_rn(qv[i] * E);
+                    ok[i] = __float2bfloat16_rn(k * invE);
+                    invEprev = invE;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    *reinterpret_cast<__nv_bfloat16 *>(Qb[s] + eoff(t0 + i)) = oq[i];
+                    *reinterpret_cast<__nv_bfloat16 *>(Gb[s] + eoff(t0 + i)) = ok[i];
+                }
             }
             if (half == 1) {
-                m->EB[n % 3][j] = E;
-                if (!(E >= kMinEB)) atomicMin(&m->bad_tile, n);
+                m->EB[n % 3][j] = __expf(bsum);
+                if (!(bsum >= kMinLogEB)) atomicMin(&m->bad_tile, n);
             }
             fence_proxy_async_smem();
-            named_bar_sync(1, 256);   // bad_tile settled, Ppart free for the next chunk
+            named_bar_sync(1, 256);   // bad_tile settled
             mbar_arrive(&m->prepped[s]);
             if (ld_volatile(&m->bad_tile) <= n) break;
         }
@@ -604,9 +617,9 @@ size_t tc_fwd_workspace(int B, int T, int H) {
 size_t tc_fwd_smem() { return tcf::kSmemBytes; }
 
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
-    CUtensorMap mq, ml, mx;
+    CUtensorMap mq, ml, mx, mo;
     if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
-        !make_token_map(&mx, a.x, a.B, a.T, a.H))
+        !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mo, a.o, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(tcf::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcf::kSmemBytes);
@@ -626,7 +639,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, a.flags, U, a.T, a.H, ntiles, nseg, tps};
-    tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, p);
+    tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, p);
     return cudaGetLastError();
 }
 

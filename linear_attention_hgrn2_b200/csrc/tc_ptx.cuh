@@ -47,10 +47,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait on phase `parity`.  Returns false (and the caller records a
 // timeout status) if the phase did not complete within ~`max_iters` polls
 // with backoff; it never spins forever.
+// try_wait itself suspends the thread for a short hardware-defined window, so the
+// first million polls spin without sleeping (hand-offs on the hot path stay fast);
+// after that the poll backs off with __nanosleep.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_iters = 20000000u) {
     for (uint32_t it = 0; it < max_iters; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (it > 64) __nanosleep(32);
+        if (it > (1u << 20)) __nanosleep(64);
     }
     return false;
 }
