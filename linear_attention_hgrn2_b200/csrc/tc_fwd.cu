@@ -339,6 +339,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll 16
                 for (int t = 0; t < 64; ++t) bsum += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t)));
             }
+            named_bar_sync(1, 256);   // rows 0..63 of log f are read before the first half overwrites them
             float invEprev = __expf(-bsum);
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
