@@ -54,7 +54,8 @@ struct __align__(8) Misc {
     uint32_t tmem_base;
     int bad_tile;                           // first chunk whose decay span is too wide
     int waited_full;                        // chunks whose arrival the prep warps consumed
-    float EB[3][128];                       // E_B ring (read one chunk later by the S phase)
+    float EB[2][128];                       // E_B ring: read by the TMEM warps while that chunk is current
+    float Ppart[3][128];                    // per 32-row range sums of log f (ranges 0..2)
 };
 
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
@@ -240,14 +241,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tmem_wait_st();
         }
         int n = 0;
+        float e_prev = 1.0f, e_cur = 1.0f;   // E_B of the previous and the current chunk, key dim r
         for (; n < N; ++n) {
             const int s = n & 1;
             if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ld_volatile(&m->bad_tile) <= n) break;
+            e_prev = e_cur;
+            e_cur = m->EB[s][r];   // the prep warps rewrite this slot only after this chunk's stage is released
             // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand)
             if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
-            const float e = n >= 1 ? m->EB[(n - 1) % 3][r] : 1.0f;
+            const float e = e_prev;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
@@ -307,7 +311,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
         if (n == N && p.hT && seg == p.nseg - 1) {
-            const float e = m->EB[(N - 1) % 3][r];
+            const float e = e_cur;
             float *dst = p.hT + ((size_t)bh * 128 + r) * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -322,56 +326,71 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ prep warps
-        // thread = one key dim j (column) and one half of the chunk's rows.  The decay is
-        // formed from the running sum b of log f: E = exp(b), 1/E = exp(-b); threads of the
-        // second half first sum log f over the first half.  Rows go in batches of 16: all
-        // loads, then the arithmetic, then all stores (so loads are not held behind stores).
+        // thread = one column pair (2 key dims, 4-byte smem accesses) and one 32-row range.
+        // The decay is formed from the running sum b of log f: E = exp(b), 1/E = exp(-b).
+        // Each range first sums its own rows; ranges exchange sums through shared memory.
+        // Rows go in batches of 8: all loads, then the arithmetic, then all stores.
         const int ptid = tid - 256;
-        const int j = ptid & 127, half = ptid >> 7;
-        const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
+        const int pc = ptid & 63, rr = ptid >> 6, col0 = 2 * pc;
+        const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
         auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
         for (int n = 0; n < N; ++n) {
             const int s = n & 1;
             if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ptid == 0) m->waited_full = n + 1;
-            float bsum = 0.0f;
-            if (half) {
-#pragma unroll 16
-                for (int t = 0; t < 64; ++t) bsum += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t)));
+            if (rr < 3) {
+                float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(32 * rr + i));
+                    s0 += bf_lo(w);
+                    s1 += bf_hi(w);
+                }
+                m->Ppart[rr][col0] = s0;
+                m->Ppart[rr][col0 + 1] = s1;
             }
-            named_bar_sync(1, 256);   // rows 0..63 of log f are read before the first half overwrites them
-            float invEprev = __expf(-bsum);
+            named_bar_sync(1, 256);
+            float b0 = 0.0f, b1 = 0.0f;
+            for (int r2 = 0; r2 < rr; ++r2) {
+                b0 += m->Ppart[r2][col0];
+                b1 += m->Ppart[r2][col0 + 1];
+            }
+            float ip0 = __expf(-b0), ip1 = __expf(-b1);   // 1/E of the row before the range
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
-                const int t0 = 64 * half + 16 * bt;
-                float av[16], qv[16];
+                const int t0 = 32 * rr + 8 * bt;
+                uint32_t wa[8], wq[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    av[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t0 + i)));
-                    qv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Qb[s] + eoff(t0 + i)));
-                }
-                __nv_bfloat16 oq[16], ok[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    bsum += av[i];
-                    const float E = __expf(bsum), invE = __expf(-bsum);
-                    const float k = fabsf(av[i]) < 0.25f ? k_from(av[i], 0.0f) : 1.0f - E * invEprev;
-                    oq[i] = __float2bfloat16_rn(qv[i] * E);
-                    ok[i] = __float2bfloat16_rn(k * invE);
-                    invEprev = invE;
+                for (int i = 0; i < 8; ++i) {
+                    wa[i] = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(t0 + i));
+                    wq[i] = *reinterpret_cast<const uint32_t *>(Qb[s] + eoff(t0 + i));
                 }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    *reinterpret_cast<__nv_bfloat16 *>(Qb[s] + eoff(t0 + i)) = oq[i];
-                    *reinterpret_cast<__nv_bfloat16 *>(Gb[s] + eoff(t0 + i)) = ok[i];
+                for (int i = 0; i < 8; ++i) {
+                    const float a0 = bf_lo(wa[i]), a1 = bf_hi(wa[i]);
+                    b0 += a0;
+                    b1 += a1;
+                    const float E0 = __expf(b0), E1 = __expf(b1), iE0 = __expf(-b0), iE1 = __expf(-b1);
+                    const float k0 = fabsf(a0) < 0.25f ? k_from(a0, 0.0f) : 1.0f - E0 * ip0;
+                    const float k1 = fabsf(a1) < 0.25f ? k_from(a1, 0.0f) : 1.0f - E1 * ip1;
+                    wq[i] = pack_bf2(bf_lo(wq[i]) * E0, bf_hi(wq[i]) * E1);
+                    wa[i] = pack_bf2(k0 * iE0, k1 * iE1);
+                    ip0 = iE0;
+                    ip1 = iE1;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    *reinterpret_cast<uint32_t *>(Qb[s] + eoff(t0 + i)) = wq[i];
+                    *reinterpret_cast<uint32_t *>(Gb[s] + eoff(t0 + i)) = wa[i];
                 }
             }
-            if (half == 1) {
-                m->EB[n % 3][j] = __expf(bsum);
-                if (!(bsum >= kMinLogEB)) atomicMin(&m->bad_tile, n);
+            if (rr == 3) {
+                m->EB[s][col0] = __expf(b0);
+                m->EB[s][col0 + 1] = __expf(b1);
+                if (!(b0 >= kMinLogEB && b1 >= kMinLogEB)) atomicMin(&m->bad_tile, n);
             }
             fence_proxy_async_smem();
-            named_bar_sync(1, 256);   // bad_tile settled
+            named_bar_sync(1, 256);   // bad_tile settled; Ppart free for the next chunk
             mbar_arrive(&m->prepped[s]);
             if (ld_volatile(&m->bad_tile) <= n) break;
         }
