@@ -34,6 +34,22 @@ __device__ __forceinline__ float k_from(float a, float f) {
     return 1.0f - f;
 }
 
+// 2^x on the FMA pipe (keeps the MUFU unit free for the other half of the exponentials).
+// Range reduction x = n + f with n = rint(x), |f| <= 1/2; 2^f = e^(f ln 2) by its Taylor
+// series to degree 4 (relative error < 6e-5 over the range); 2^n placed in the exponent
+// field.  x is clamped to [-126, 126] (no inf/denormal results).
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fminf(fmaxf(x, -126.0f), 126.0f);
+    const float n = rintf(x);
+    const float u = (x - n) * 0.69314718056f;
+    float p = fmaf(u, 1.0f / 24.0f, 1.0f / 6.0f);
+    p = fmaf(p, u, 0.5f);
+    p = fmaf(p, u, 1.0f);
+    p = fmaf(p, u, 1.0f);
+    return p * __int_as_float(((int)n + 127) << 23);
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 // Row j (lane) of a 64-column half of a TMEM tile -> bf16 row in a swizzled smem block.
 __device__ __forceinline__ void store_row_bf16(uint8_t *blk, int row, const float (&r0)[32], const float (&r1)[32]) {
     uint8_t *base = blk + row * 128;

@@ -355,7 +355,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 b0 += m->Ppart[r2][col0];
                 b1 += m->Ppart[r2][col0 + 1];
             }
-            float ip0 = __expf(-b0), ip1 = __expf(-b1);   // 1/E of the row before the range
+            float ip0 = exp2_fma(-b0 * kLog2e), ip1 = exp2_fma(-b1 * kLog2e);   // 1/E before the range
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
                 const int t0 = 32 * rr + 8 * bt;
@@ -370,7 +370,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     const float a0 = bf_lo(wa[i]), a1 = bf_hi(wa[i]);
                     b0 += a0;
                     b1 += a1;
-                    const float E0 = __expf(b0), E1 = __expf(b1), iE0 = __expf(-b0), iE1 = __expf(-b1);
+                    const float E0 = __expf(b0), E1 = __expf(b1);
+                    const float iE0 = exp2_fma(-b0 * kLog2e), iE1 = exp2_fma(-b1 * kLog2e);
                     const float k0 = fabsf(a0) < 0.25f ? k_from(a0, 0.0f) : 1.0f - E0 * ip0;
                     const float k1 = fabsf(a1) < 0.25f ? k_from(a1, 0.0f) : 1.0f - E1 * ip1;
                     wq[i] = pack_bf2(bf_lo(wq[i]) * E0, bf_hi(wq[i]) * E1);

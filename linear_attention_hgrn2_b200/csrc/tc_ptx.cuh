@@ -47,10 +47,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait on phase `parity`.  Returns false (and the caller records a
 // timeout status) if the phase did not complete within ~`max_iters` polls
 // with backoff; it never spins forever.
-// try_wait itself suspends the thread for a short hardware-defined window, so the
-// first million polls spin without sleeping (hand-offs on the hot path stay fast);
-// after that the poll backs off with __nanosleep.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait on phase `parity`: the first polls use the non-blocking test_wait (a
+// hand-off is seen within a few cycles), then try_wait (which suspends the thread for
+// a short hardware-defined window), and after a million polls __nanosleep back-off.
+// Returns false if the phase did not complete within `max_iters` polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_iters = 20000000u) {
+    for (uint32_t it = 0; it < 4096u; ++it)
+        if (mbar_test_wait(bar, parity)) return true;
     for (uint32_t it = 0; it < max_iters; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (it > (1u << 20)) __nanosleep(64);
