@@ -50,6 +50,16 @@ __device__ __forceinline__ float exp2_fma(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
+// k = 1 - f for the prep: -expm1(a) by its Taylor series to degree 4 in a when |a| < 1/4
+// (relative truncation error < 3e-5, below bf16 rounding), else 1 - f with f = E_t / E_{t-1}
+// supplied by the caller as `f` (no cancellation there: f <= e^-1/4).  Branch-free.
+__device__ __forceinline__ float k_gate(float a, float f) {
+    float p = fmaf(a, 1.0f / 24.0f, 1.0f / 6.0f);
+    p = fmaf(p, a, 0.5f);
+    p = fmaf(p, a, 1.0f);
+    return fabsf(a) < 0.25f ? -a * p : 1.0f - f;
+}
+
 // Row j (lane) of a 64-column half of a TMEM tile -> bf16 row in a swizzled smem block.
 __device__ __forceinline__ void store_row_bf16(uint8_t *blk, int row, const float (&r0)[32], const float (&r1)[32]) {
     uint8_t *base = blk + row * 128;

@@ -26,7 +26,7 @@
 //   warp 0      TMA producer: q, log f, i tiles (128-byte swizzle) into a 2-stage ring
 //   warp 1      TMEM allocator and the single MMA-issuing thread
 //   warps 4-7   TMEM warps (one thread per TMEM lane): S phase (bf16 copy of S_in,
-//               Diag(E_B) scale), causal mask of A, o epilogue (stored from registers)
+//               Diag(E_B) scale), causal mask of A, o epilogue (staged in smem, TMA store)
 //   warps 8-15  prep warps: f, E, k, Qt, Kt for the next chunk while the current one
 //               is on the tensor cores
 // Every wait is bounded; a wait that gives up records HGRN2_ERR_TIMEOUT.
@@ -213,6 +213,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
                 }
                 mma_commit(&m->barO2);
+                mma_commit(&m->empty[s]);   // stage s is free once every MMA above completed
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -248,8 +249,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (ld_volatile(&m->bad_tile) <= n) break;
             e_prev = e_cur;
             e_cur = m->EB[s][r];   // the prep warps rewrite this slot only after this chunk's stage is released
-            // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand)
+            // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand),
+            // once the previous chunk's o store has read X
             if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (n >= 1) {
+                if (r == 0) tma_store_wait_read0();
+                named_bar_sync(2, 128);
+            }
             tc_fence_after();
             const float e = e_prev;
 #pragma unroll
@@ -283,8 +289,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->adone);
-            // o epilogue: O -> bf16 rows in the chunk's q buffer (free: every MMA of the chunk
-            // completed) -> TMA store; the stage is released once the store has read it
+            // o epilogue: O -> bf16 rows in X (free: the last MMA of the chunk completed) ->
+            // TMA store; the next S phase waits until the store has read X
             if (!mbar_wait(&m->barO2, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
 #pragma unroll
@@ -292,18 +298,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 float v[32];
                 tmem_ld32(tl + kColO + 32 * c, v);
                 tmem_wait_ld();
-                store_chunk_bf16(Qb[s], r, c, v);
+                store_chunk_bf16(X, r, c, v);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->ofree);
             named_bar_sync(2, 128);
             if (r == 0) {
-                tma_store_4d(&tm_o, Qb[s], 0, h, (g0 + n) * kTile, b);
-                tma_store_4d(&tm_o, Qb[s] + kBlk, 64, h, (g0 + n) * kTile, b);
+                tma_store_4d(&tm_o, X, 0, h, (g0 + n) * kTile, b);
+                tma_store_4d(&tm_o, X + kBlk, 64, h, (g0 + n) * kTile, b);
                 tma_store_commit();
-                tma_store_wait_read0();
-                mbar_arrive(&m->empty[s]);
             }
         }
         if (r == 0) tma_store_wait_all0();
@@ -355,7 +359,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 b0 += m->Ppart[r2][col0];
                 b1 += m->Ppart[r2][col0 + 1];
             }
-            float ip0 = exp2_fma(-b0 * kLog2e), ip1 = exp2_fma(-b1 * kLog2e);   // 1/E before the range
+            float ip0 = __expf(-b0), ip1 = __expf(-b1);   // 1/E of the row before the range
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
                 const int t0 = 32 * rr + 8 * bt;
@@ -370,10 +374,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     const float a0 = bf_lo(wa[i]), a1 = bf_hi(wa[i]);
                     b0 += a0;
                     b1 += a1;
-                    const float E0 = __expf(b0), E1 = __expf(b1);
-                    const float iE0 = exp2_fma(-b0 * kLog2e), iE1 = exp2_fma(-b1 * kLog2e);
-                    const float k0 = fabsf(a0) < 0.25f ? k_from(a0, 0.0f) : 1.0f - E0 * ip0;
-                    const float k1 = fabsf(a1) < 0.25f ? k_from(a1, 0.0f) : 1.0f - E1 * ip1;
+                    const float E0 = __expf(b0), E1 = __expf(b1), iE0 = __expf(-b0), iE1 = __expf(-b1);
+                    const float k0 = k_gate(a0, E0 * ip0), k1 = k_gate(a1, E1 * ip1);
                     wq[i] = pack_bf2(bf_lo(wq[i]) * E0, bf_hi(wq[i]) * E1);
                     wa[i] = pack_bf2(k0 * iE0, k1 * iE1);
                     ip0 = iE0;

@@ -56,13 +56,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait on phase `parity`: the first polls use the non-blocking test_wait (a
-// hand-off is seen within a few cycles), then try_wait (which suspends the thread for
-// a short hardware-defined window), and after a million polls __nanosleep back-off.
-// Returns false if the phase did not complete within `max_iters` polls.
+// Bounded wait on phase `parity`.  try_wait suspends the thread for a short
+// hardware-defined window, so the first million polls run without sleeping (hand-offs
+// on the hot path stay fast and idle pollers do not take issue slots from working
+// warps); after that the poll backs off with __nanosleep.  Returns false if the phase
+// did not complete within `max_iters` polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_iters = 20000000u) {
-    for (uint32_t it = 0; it < 4096u; ++it)
-        if (mbar_test_wait(bar, parity)) return true;
     for (uint32_t it = 0; it < max_iters; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (it > (1u << 20)) __nanosleep(64);
