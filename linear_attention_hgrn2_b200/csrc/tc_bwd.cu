@@ -45,16 +45,29 @@ constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ void st_bar_expect(uint64_t *bar, uint32_t bytes) { mbar_arrive_expect_tx(bar, bytes); }
 
 // ------------------------------------------------------------------ forward sweep: dq
+// Warp roles (16 warps), coordinated by mbarriers:
+//   warp 0      TMA producer: log f, i, dO tiles into a 2-stage ring
+//   warp 1      TMEM allocator, MMA thread: dA = dO V^T as soon as a chunk lands, then
+//               dq_pre^T = S_in dO^T + Kt^T mask(dA)^T and S' = S_in + Kt^T V
+//   warps 4-7   TMEM warps: S phase (Diag(E_B) post-scale, bf16 copy), causal mask of
+//               dA, dq = E * dq_pre epilogue (lane = key dim j) staged in smem, TMA store
+//   warps 8-15  prep warps (thread = key dim j, half of the rows): Kt = k / E in place
+//               of log f, and E into TMEM lane j for the epilogue
 namespace fsw {
 constexpr uint32_t kColS = 0, kColDA = 128, kColDQ = 256, kColE = 384;
+constexpr int kDqThreads = 512;
 
 struct __align__(8) Misc {
-    uint64_t full[2];
-    uint64_t barA, barQ1, barM;
+    uint64_t full[2], prepped[2], empty[2];
+    uint64_t barDA, barQ1, barS, barQ;       // MMA completions (tcgen05.commit)
+    uint64_t sdone, dadone, dqfree, efree;   // TMEM-warp arrivals (128 each)
     uint32_t tmem_base;
+    int bad_tile;
+    int waited_full;
     int pad;
-    float EBr[2][128];     // E_B of the last two chunks (post-scaling of the state)
-    float Ppart[2][128];   // prep partial products; after the loop, rowsum(dhT*hT) halves
+    float EB[2][128];
+    float Bpart[128];                        // sum of log f over rows 0..63, per key dim
+    float rs_part[128];
 };
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
 }  // namespace fsw
@@ -66,7 +79,7 @@ struct DqParams {
     int T, H, ntiles;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(fsw::kDqThreads, 1)
 dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUtensorMap tm_x,
           const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dq, DqParams p) {
     using namespace fsw;
@@ -84,17 +97,29 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
     }
-    const int quad = warp & 3, half = warp >> 2;
-    const int j = 32 * quad + lane;                         // key dim / TMEM lane / tile row
     if (tid == 0) {
-        mbar_init(&m->full[0], 1);
-        mbar_init(&m->full[1], 1);
-        mbar_init(&m->barA, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&m->full[s], 1);
+            mbar_init(&m->prepped[s], 256);
+            mbar_init(&m->empty[s], 1);
+        }
+        mbar_init(&m->barDA, 1);
         mbar_init(&m->barQ1, 1);
-        mbar_init(&m->barM, 1);
+        mbar_init(&m->barS, 1);
+        mbar_init(&m->barQ, 1);
+        mbar_init(&m->sdone, 128);
+        mbar_init(&m->dadone, 128);
+        mbar_init(&m->dqfree, 128);
+        mbar_init(&m->efree, 128);
+        m->bad_tile = INT_MAX;
+        m->waited_full = 0;
         fence_mbar_init();
+        tma_prefetch_desc(&tm_lf);
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_do);
+        tma_prefetch_desc(&tm_dq);
     }
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(&m->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -102,228 +127,265 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
-    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+    int producer_issued = 0;
+    bool fell_back_here = false;
 
-    int issued = 0, waited = 0;
-    auto issue_load = [&](int n) {
-        const int s = n & 1;
-        ++issued;
-        mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
-        for (int c = 0; c < 2; ++c) {
-            tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, n * kTile, b);
-            tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, n * kTile, b);
-            tma_load_4d(Ob[s] + c * kBlk, &tm_do, &m->full[s], 64 * c, h, n * kTile, b);
-        }
-    };
-    if (tid == 0) {
-        issue_load(0);
-        if (N > 1) issue_load(1);
-    }
-    {   // state init S = h0 (or 0); previous E_B = 1
-        float r0[32], r1[32];
-        if (p.h0) {
-            const float4 *src = reinterpret_cast<const float4 *>(p.h0 + ((size_t)bh * 128 + j) * 128 + 64 * half);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float4 a = src[i], c = src[8 + i];
-                r0[4 * i] = a.x; r0[4 * i + 1] = a.y; r0[4 * i + 2] = a.z; r0[4 * i + 3] = a.w;
-                r1[4 * i] = c.x; r1[4 * i + 1] = c.y; r1[4 * i + 2] = c.z; r1[4 * i + 3] = c.w;
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            for (int n = 0; n < N; ++n) {
+                const int s = n & 1;
+                if (ld_volatile(&m->bad_tile) < n) break;
+                if (n >= 2 && !wait_or_abort(&m->empty[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
+                mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, n * kTile, b);
+                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, n * kTile, b);
+                    tma_load_4d(Ob[s] + c * kBlk, &tm_do, &m->full[s], 64 * c, h, n * kTile, b);
+                }
+                ++producer_issued;
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0.0f;
         }
-        tmem_st32(tl + kColS + 64 * half, r0);
-        tmem_st32(tl + kColS + 64 * half + 32, r1);
-        tmem_wait_st();
-        if (half == 0) m->EBr[1][j] = 1.0f;
-    }
-
-    const uint32_t id_kk = idesc_bf16(128, 128, false, false);
-    const uint32_t id_mnk = idesc_bf16(128, 128, true, false);
-    const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
-    const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
-    bool ok = true;
-    int n = 0;
-    for (n = 0; n < N; ++n) {
-        const int s = n & 1;
-        if (__syncthreads_or(!mbar_wait(&m->full[s], (n >> 1) & 1))) { ok = false; break; }
-        waited = n + 1;
-        // ---- prep: column j, rows 64*half .. +63: Kt = k / E in place of log f, E -> TMEM
-        float fv[64];
-        float P = 1.0f;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_kk = idesc_bf16(128, 128, false, false);
+            const uint32_t id_mnk = idesc_bf16(128, 128, true, false);
+            const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+            for (int n = 0; n < N; ++n) {
+                const int s = n & 1;
+                // dA = dO V^T (does not need the prep)
+                if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const int t = 64 * half + i;
-            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
-            fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + off)));
-            P *= fv[i];
-        }
-        m->Ppart[half][j] = P;
-        __syncthreads();
-        float E = half ? m->Ppart[0][j] : 1.0f;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColDA, sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024),
+                                sdesc_sw128(smem_u32(Vb[s]) + ko, 16, 1024), id_kk, kk > 0);
+                }
+                mma_commit(&m->barDA);
+                if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                if (ld_volatile(&m->bad_tile) <= n) {
+                    mbar_wait(&m->barDA, n & 1);   // nothing left in flight
+                    break;
+                }
+                // dq_pre^T = S_in dO^T (M = j, N = t); S' = S_in + Kt^T V
+                if (!mbar_wait(&m->sdone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                if (n >= 1 && !mbar_wait(&m->dqfree, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const int t = 64 * half + i;
-            const uint32_t off = cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin;
-            __nv_bfloat16 *g = reinterpret_cast<__nv_bfloat16 *>(Gb[s] + off);
-            const float a = __bfloat162float(*g);
-            E *= fv[i];
-            const float k = k_from(a, fv[i]);
-            *g = __float2bfloat16_rn(k * __fdividef(1.0f, E));
-            fv[i] = E;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
+                                sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024), id_kk, kk > 0);
+                }
+                mma_commit(&m->barQ1);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
+                                sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                mma_commit(&m->barS);
+                // dq_pre^T += Kt^T mask(dA)^T (M = j, N = t, K = s)
+                if (!mbar_wait(&m->dadone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
+                                sdesc_sw128(smem_u32(X) + ko, 16, 1024), id_mnk, true);
+                }
+                mma_commit(&m->barQ);
+                mma_commit(&m->empty[s]);
+            }
         }
-        if (half == 1) m->EBr[s][j] = E;
-        {
-            float *e0 = fv, *e1 = fv + 32;
-            tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(e0));
-            tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(e1));
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ TMEM warps
+        const int quad = warp & 3, r = 32 * quad + lane;
+        const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+        const uint32_t cblk = (uint32_t)(r >> 6) * kBlk, cch = (uint32_t)((r & 63) >> 3), cin = (uint32_t)(r & 7) * 2;
+        {   // S = h0 (or 0)
+            const float *init = p.h0 ? p.h0 + (size_t)bh * 16384 : nullptr;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                if (init) {
+                    const float4 *src = reinterpret_cast<const float4 *>(init + (size_t)r * 128 + 32 * c);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 a = src[i];
+                        v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                }
+                tmem_st32(tl + kColS + 32 * c, v);
+            }
             tmem_wait_st();
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(half == 1 && !(E >= kMinEB))) break;
-
-        // ---- dA = dO V^T
-        if (tid == 0) {
+        int n = 0;
+        float e_prev = 1.0f, e_cur = 1.0f;
+        for (; n < N; ++n) {
+            const int s = n & 1;
+            if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (ld_volatile(&m->bad_tile) <= n) break;
+            e_prev = e_cur;
+            e_cur = m->EB[s][r];
+            // S phase
+            if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (n >= 1) {
+                if (r == 0) tma_store_wait_read0();   // the previous dq store has read X
+                named_bar_sync(2, 128);
+            }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColDA, sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Vb[s]) + ko, 16, 1024), id_kk, kk > 0);
-            }
-            mma_commit(&m->barA);
-            tma_store_wait_read0();
-        }
-        __syncthreads();
-        // ---- S phase: S_in = Diag(E_B of the previous chunk) * accumulator; bf16 copy into X
-        {
-            float r0[32], r1[32];
-            tc_fence_after();
-            tmem_ld32(tl + kColS + 64 * half, r0);
-            tmem_ld32(tl + kColS + 64 * half + 32, r1);
-            tmem_wait_ld();
-            const float e = m->EBr[s ^ 1][j];
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColS + 32 * c, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                r0[i] *= e;
-                r1[i] *= e;
+                for (int i = 0; i < 32; ++i) v[i] *= e_prev;
+                store_chunk_bf16(X, r, c, v);
+                tmem_st32(tl + kColS + 32 * c, v);
             }
-            store_row_bf16(X + half * kBlk, j, r0, r1);
-            tmem_st32(tl + kColS + 64 * half, r0);
-            tmem_st32(tl + kColS + 64 * half + 32, r1);
             tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // ---- dq_pre^T = S_in dO^T   (M = j, N = t, K = v)
-        if (tid == 0) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->sdone);
+            // causal mask of dA (lane = t), bf16 -> X (rows t) once S_in dO^T has read X
+            if (!mbar_wait(&m->barDA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (!mbar_wait(&m->barQ1, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024), id_kk, kk > 0);
-            }
-            mma_commit(&m->barQ1);
-        }
-        // ---- dA phase: causal mask, bf16 into X (rows t) once the previous MMA is done with X
-        {
-            if (!mbar_wait(&m->barA, n & 1)) ok = false;
-            tc_fence_after();
-            float r0[32], r1[32];
-            tmem_ld32(tl + kColDA + 64 * half, r0);
-            tmem_ld32(tl + kColDA + 64 * half + 32, r1);
-            tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColDA + 32 * c, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (64 * half + i > j) r0[i] = 0.0f;
-                if (64 * half + 32 + i > j) r1[i] = 0.0f;
+                for (int i = 0; i < 32; ++i)
+                    if (32 * c + i > r) v[i] = 0.0f;
+                store_chunk_bf16(X, r, c, v);
             }
-            if (!mbar_wait(&m->barQ1, n & 1)) ok = false;
-            store_row_bf16(X + half * kBlk, j, r0, r1);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(!ok)) { ok = false; break; }
-        // ---- dq_pre^T += Kt^T dA^T (M = j, N = t, K = s);  S += Kt^T V (M = j, N = v, K = t)
-        if (tid == 0) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->dadone);
+            // dq[t][j] = E[j][t] * dq_pre^T[j][t]  (lane j = r) -> X as the [t][j] tile
+            if (!mbar_wait(&m->barQ, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(X) + ko, 16, 1024), id_mnk, true);
-            }
+            for (int c = 0; c < 4; ++c) {
+                float d[32], e[32];
+                tmem_ld32(tl + kColDQ + 32 * c, d);
+                tmem_ld32(tl + kColE + 32 * c, e);
+                tmem_wait_ld();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                for (int i = 0; i < 32; ++i) {
+                    const int t = 32 * c + i;
+                    *reinterpret_cast<__nv_bfloat16 *>(X + cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin) =
+                        __float2bfloat16_rn(d[i] * e[i]);
+                }
             }
-            mma_commit(&m->barM);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&m->dqfree);
+            mbar_arrive(&m->efree);
+            named_bar_sync(2, 128);
+            if (r == 0) {
+                tma_store_4d(&tm_dq, X, 0, h, n * kTile, b);
+                tma_store_4d(&tm_dq, X + kBlk, 64, h, n * kTile, b);
+                tma_store_commit();
+            }
         }
-        if (__syncthreads_or(!mbar_wait(&m->barM, n & 1))) { ok = false; break; }
+        if (r == 0) tma_store_wait_all0();
+        if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        if (tid == 0 && n + 2 < N) issue_load(n + 2);
-        // ---- epilogue: dq[t][j] = E[j][t] * dq_pre^T[j][t] -> X (rows t) -> TMA store
+        fell_back_here = n < N;
+        if (n == N && p.dhT && p.rs) {
+            // hT = Diag(E_B of the last chunk) S';  rs[j] = sum_v dhT[j,v] hT[j,v]
+            const float *g = p.dhT + ((size_t)bh * 128 + r) * 128;
+            float acc = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            float d[32], e[32];
-            tmem_ld32(tl + kColDQ + 64 * half + 32 * c, d);
-            tmem_ld32(tl + kColE + 64 * half + 32 * c, e);
-            tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(tl + kColS + 32 * c, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int t = 64 * half + 32 * c + i;
-                *reinterpret_cast<__nv_bfloat16 *>(X + cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin) =
-                    __float2bfloat16_rn(d[i] * e[i]);
+                for (int i = 0; i < 32; ++i) acc = fmaf(g[32 * c + i], v[i] * e_cur, acc);
             }
+            p.rs[(size_t)bh * 128 + r] = acc;
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_4d(&tm_dq, X, 0, h, n * kTile, b);
-            tma_store_4d(&tm_dq, X + kBlk, 64, h, n * kTile, b);
-            tma_store_commit();
-        }
-    }
-    const bool fell_back = ok && n < N;
-    if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
-    if (tid == 0) {   // drain loads still landing in this CTA's shared memory, and the stores
-        for (int k = waited; k < issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
-        tma_store_wait_all0();
-    }
-    if (ok && !fell_back && p.dhT && p.rs) {
-        // hT = Diag(E_B of the last chunk) * accumulator;  rs[j] = sum_v dhT[j,v] hT[j,v]
-        tc_fence_after();
-        float r0[32], r1[32];
-        tmem_ld32(tl + kColS + 64 * half, r0);
-        tmem_ld32(tl + kColS + 64 * half + 32, r1);
-        tmem_wait_ld();
-        const float e = N > 0 ? m->EBr[(N - 1) & 1][j] : 1.0f;
-        const float *g = p.dhT + ((size_t)bh * 128 + j) * 128 + 64 * half;
-        float acc = 0.0f;
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ prep warps
+        // thread = key dim j (TMEM lane j, in this warp's lane quadrant) and 64 rows.
+        const int j = 32 * (warp & 3) + lane, half = (warp - 8) >> 2;
+        const uint32_t tl = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
+        const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
+        auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+        for (int n = 0; n < N; ++n) {
+            const int s = n & 1;
+            if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (warp == 8 && lane == 0) m->waited_full = n + 1;
+            if (half == 1) {
+                float sum = 0.0f;
+#pragma unroll 16
+                for (int t = 0; t < 64; ++t)
+                    sum += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t)));
+                m->Bpart[j] = sum;
+            }
+            named_bar_sync(1, 256);   // rows 0..63 of log f are read before the first half overwrites them
+            float bsum = half ? m->Bpart[j] : 0.0f;
+            float ip = __expf(-bsum);
+            float ev[64];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            acc = fmaf(g[i], r0[i] * e, acc);
-            acc = fmaf(g[32 + i], r1[i] * e, acc);
+            for (int bt = 0; bt < 8; ++bt) {
+                const int t0 = 64 * half + 8 * bt;
+                float av[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    av[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t0 + i)));
+                __nv_bfloat16 ok[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    bsum += av[i];
+                    const float E = __expf(bsum), iE = __expf(-bsum);
+                    ok[i] = __float2bfloat16_rn(k_gate(av[i], E * ip) * iE);
+                    ev[8 * bt + i] = E;
+                    ip = iE;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) *reinterpret_cast<__nv_bfloat16 *>(Gb[s] + eoff(t0 + i)) = ok[i];
+            }
+            if (half == 1) {
+                m->EB[s][j] = __expf(bsum);
+                if (!(bsum >= kMinLogEB)) atomicMin(&m->bad_tile, n);
+            }
+            fence_proxy_async_smem();
+            // E -> TMEM lane j once the previous chunk's dq epilogue has read it
+            if (n >= 1 && !mbar_wait(&m->efree, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(ev));
+            tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(ev + 32));
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar_sync(1, 256);   // bad_tile settled, Bpart free
+            mbar_arrive(&m->prepped[s]);
+            if (ld_volatile(&m->bad_tile) <= n) break;
         }
-        m->Ppart[half][j] = acc;
     }
-    __syncthreads();
-    if (ok && !fell_back && p.dhT && p.rs && half == 0) p.rs[(size_t)bh * 128 + j] = m->Ppart[0][j] + m->Ppart[1][j];
-    if (tid == 0) {
-        p.flags[bh] = fell_back ? 1 : 0;
-        if (fell_back) atomicAdd(&g_counters[0], 1ull);
-        if (ok && !fell_back) atomicAdd(&g_counters[1], (unsigned long long)N);
-    }
+
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+    const bool fell_back = m->bad_tile < N;
+    (void)fell_back_here;
+    if (warp == 0 && lane == 0)
+        for (int k = m->waited_full; k < producer_issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
+    if (tid == 0) {
+        p.flags[bh] = fell_back ? 1 : 0;
+        if (fell_back) atomicAdd(&g_counters[0], 1ull);
+        else atomicAdd(&g_counters[1], (unsigned long long)N);
+    }
+    __syncwarp();
+    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
 
 // ------------------------------------------------------------------ reverse sweep
@@ -700,7 +762,7 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     tcb::DqParams p1{a.h0, a.dhT, a.rs, a.flags, a.T, a.H, ntiles};
-    tcb::dq_kernel<<<a.B * a.H, tcb::kThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
+    tcb::dq_kernel<<<a.B * a.H, tcb::fsw::kDqThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles};

@@ -1,6 +1,7 @@
 // tc_common.cuh -- device and host helpers shared by the tensor-core kernels.
 #pragma once
 
+#include <climits>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -75,6 +76,38 @@ __device__ __forceinline__ void store_row_bf16(uint8_t *blk, int row, const floa
     }
 }
 
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
+
+// Waits for phase `parity` of `bar`, or returns false early once `*bad <= tile` (the
+// pipeline stopped before that phase could complete) or after a bounded number of polls.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const int *bad, int tile) {
+    for (uint32_t it = 0; it < 20000000u; ++it) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if (ld_volatile(bad) <= tile) return false;
+        if (it > (1u << 20)) __nanosleep(64);
+    }
+    set_status(HGRN2_ERR_TIMEOUT);
+    return false;
+}
+
+// One 32-column chunk (c = 0..3) of a TMEM row -> bf16 into row `row` of a swizzled 128 x 128 tile.
+__device__ __forceinline__ void store_chunk_bf16(uint8_t *tile, int row, int c, const float (&r)[32]) {
+    uint8_t *base = tile + (c >> 1) * kBlk + row * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int chunk = 4 * (c & 1) + q;
+        uint4 v;
+        v.x = pack_bf2(r[8 * q + 0], r[8 * q + 1]);
+        v.y = pack_bf2(r[8 * q + 2], r[8 * q + 3]);
+        v.z = pack_bf2(r[8 * q + 4], r[8 * q + 5]);
+        v.w = pack_bf2(r[8 * q + 6], r[8 * q + 7]);
+        *reinterpret_cast<uint4 *>(base + ((chunk ^ (row & 7)) << 4)) = v;
+    }
+}
 
 // bf16 element (row, col) of a 128 x 128 tile in the two-block 128-byte-swizzled layout.
 __device__ __forceinline__ __nv_bfloat16 *tile_elem(uint8_t *tile, int row, int col) {

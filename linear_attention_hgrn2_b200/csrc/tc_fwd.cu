@@ -70,38 +70,6 @@ struct Params {
     int nseg, tps;    // sequence segments per (b,h) and chunks per segment
 };
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
-
-// Waits for phase `parity` of `bar`, or returns false early once `*bad <= tile` (the
-// pipeline stopped before that phase could complete) or after a bounded number of polls.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const int *bad, int tile) {
-    for (uint32_t it = 0; it < 20000000u; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (ld_volatile(bad) <= tile) return false;
-        if (it > (1u << 20)) __nanosleep(64);
-    }
-    set_status(HGRN2_ERR_TIMEOUT);
-    return false;
-}
-
-// One 32-column chunk (c = 0..3) of a TMEM row -> bf16 into row `row` of a swizzled 128 x 128 tile.
-__device__ __forceinline__ void store_chunk_bf16(uint8_t *tile, int row, int c, const float (&r)[32]) {
-    uint8_t *base = tile + (c >> 1) * kBlk + row * 128;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int chunk = 4 * (c & 1) + q;
-        uint4 v;
-        v.x = pack_bf2(r[8 * q + 0], r[8 * q + 1]);
-        v.y = pack_bf2(r[8 * q + 2], r[8 * q + 3]);
-        v.z = pack_bf2(r[8 * q + 4], r[8 * q + 5]);
-        v.w = pack_bf2(r[8 * q + 6], r[8 * q + 7]);
-        *reinterpret_cast<uint4 *>(base + ((chunk ^ (row & 7)) << 4)) = v;
-    }
-}
-
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o, Params p) {
