@@ -389,15 +389,23 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 }
 
 // ------------------------------------------------------------------ reverse sweep
+// 16 warps; every phase is spread over all of them.  TMEM lane quadrant = warp & 3,
+// quarter = warp >> 2 selects 32 TMEM columns (or 32 rows of the chunk in the prep).
+// Shared memory (7 tiles of 32 KB): Qb q -> Qt, Gb log f -> Kt, Vb v, Ob dO, D16 bf16(dSh)
+// then the dq tile, AT mask(A)^T then di staging, DA mask(dA) then d log f staging.
+// As soon as the MMAs of a chunk are done, dq of this chunk lands in D16 and v, dO of the
+// next chunk in Vb, Ob; q and log f of the next chunk follow once the epilogue has read
+// Qt and Kt.
 namespace rsw {
 constexpr uint32_t kColDS = 0, kColX1 = 128, kColX2 = 256, kColE = 384;
+constexpr int kRevThreads = 512;
 
 struct __align__(8) Misc {
-    uint64_t barIn, barDO, barDQ, barP1, barP2;
+    uint64_t barIn, barVO, barDQ, barP1, barP2;
     uint32_t tmem_base;
     int pad;
     float EB[128];
-    float Ppart[2][128];   // prep partial products; in the epilogue, per-half suffix totals
+    float Bpart[3][128];   // per 32-row range sums of log f; in the epilogue, quarter suffix totals
     float carry[128];
 };
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
@@ -410,12 +418,7 @@ struct RevParams {
     int T, H, ntiles;
 };
 
-// Shared-memory plan per chunk (7 tiles of 32 KB): Qb q -> Qt, Gb log f -> Kt, Vb v (then
-// the dq tile for the d log f epilogue), Ob dO, D16 bf16(dSh), AT mask(A)^T (then di
-// staging), DA mask(dA) (then d log f staging).  Loads: q, log f, v of the next chunk
-// start once this chunk's epilogue has read Qb, Gb, Vb; dO of the next chunk and dq of
-// this one start as soon as the MMAs are done, under the epilogue.
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(rsw::kRevThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
            const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_di,
@@ -434,11 +437,12 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
     }
-    const int quad = warp & 3, half = warp >> 2;
-    const int j = 32 * quad + lane;
+    const int quad = warp & 3, q4 = warp >> 2;
+    const int j = 32 * quad + lane;      // TMEM lane / key dim / tile row
+    const int c0 = 32 * q4;              // this thread's 32 TMEM columns (or rows, in the prep)
     if (tid == 0) {
         mbar_init(&m->barIn, 1);
-        mbar_init(&m->barDO, 1);
+        mbar_init(&m->barVO, 1);
         mbar_init(&m->barDQ, 1);
         mbar_init(&m->barP1, 1);
         mbar_init(&m->barP2, 1);
@@ -454,95 +458,105 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t tbase = m->tmem_base;
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
 
-    // loads issued / arrivals waited for, per barrier (thread 0's view): [barIn, barDO, barDQ]
+    // loads issued / arrivals waited for, per barrier (thread 0's view): [barIn, barVO, barDQ]
     int issued[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
-    auto issue_in = [&](int n) {
-        ++issued[0];
-        mbar_arrive_expect_tx(&m->barIn, 3 * kTileBytes);
+    auto issue2 = [&](uint8_t *d0, const CUtensorMap *t0, uint8_t *d1, const CUtensorMap *t1, uint64_t *bar,
+                      int q, int n) {
+        ++issued[q];
+        mbar_arrive_expect_tx(bar, 2 * kTileBytes);
         for (int c = 0; c < 2; ++c) {
-            tma_load_4d(Qb + c * kBlk, &tm_q, &m->barIn, 64 * c, h, n * kTile, b);
-            tma_load_4d(Gb + c * kBlk, &tm_lf, &m->barIn, 64 * c, h, n * kTile, b);
-            tma_load_4d(Vb + c * kBlk, &tm_x, &m->barIn, 64 * c, h, n * kTile, b);
+            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, h, n * kTile, b);
+            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, h, n * kTile, b);
         }
     };
-    auto issue_one = [&](uint8_t *dst, const CUtensorMap *tm, uint64_t *bar, int n) {
-        ++issued[bar == &m->barDO ? 1 : 2];
-        mbar_arrive_expect_tx(bar, kTileBytes);
-        tma_load_4d(dst, tm, bar, 0, h, n * kTile, b);
-        tma_load_4d(dst + kBlk, tm, bar, 64, h, n * kTile, b);
-    };
     if (tid == 0 && N > 0) {
-        issue_in(N - 1);
-        issue_one(Ob, &tm_do, &m->barDO, N - 1);
+        issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, N - 1);
+        issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, N - 1);
     }
     {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
-        float r0[32], r1[32];
+        float v[32];
         if (p.dhT) {
-            const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * 128 + j) * 128 + 64 * half);
+            const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * 128 + j) * 128 + c0);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float4 a = src[i], c = src[8 + i];
-                r0[4 * i] = a.x; r0[4 * i + 1] = a.y; r0[4 * i + 2] = a.z; r0[4 * i + 3] = a.w;
-                r1[4 * i] = c.x; r1[4 * i + 1] = c.y; r1[4 * i + 2] = c.z; r1[4 * i + 3] = c.w;
+                const float4 a = src[i];
+                v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r0[i] = r1[i] = 0.0f;
+            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
         }
-        tmem_st32(tl + kColDS + 64 * half, r0);
-        tmem_st32(tl + kColDS + 64 * half + 32, r1);
+        tmem_st32(tl + kColDS + c0, v);
         tmem_wait_st();
-        if (half == 0) m->carry[j] = (p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
+        if (q4 == 0) m->carry[j] = (p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
     }
 
     const uint32_t id_kk = idesc_bf16(128, 128, false, false);
     const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
     const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
     const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
-    auto elem_off = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+    auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+    auto bfat = [&](const uint8_t *tile, int t) -> float {
+        return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + eoff(t)));
+    };
     bool ok = true;
     int it = 0, n = N - 1;
     for (; n >= 0; --n, ++it) {
         const uint32_t par = it & 1;
         if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
         waited[0] = it + 1;
-        // ---- prep: Qt = q E (in place), Kt = k / E (in place of log f), E -> TMEM
-        float fv[64];
-        float P = 1.0f;
+        // ---- prep: column j, rows c0 .. c0+31: Qt = q E, Kt = k / E in place; E -> TMEM
+        {
+            float sum = 0.0f;
+            if (q4 < 3) {
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) sum += bfat(Gb, c0 + i);
+                m->Bpart[q4][j] = sum;
+            }
+            __syncthreads();
+            float bsum = 0.0f;
+            for (int r2 = 0; r2 < q4; ++r2) bsum += m->Bpart[r2][j];
+            float ip = __expf(-bsum);
+            float ev[32];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            fv[i] = __expf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb + elem_off(64 * half + i))));
-            P *= fv[i];
-        }
-        m->Ppart[half][j] = P;
-        __syncthreads();
-        float E = half ? m->Ppart[0][j] : 1.0f;
+            for (int bt = 0; bt < 4; ++bt) {
+                const int t0 = c0 + 8 * bt;
+                float av[8], qv[8];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const uint32_t off = elem_off(64 * half + i);
-            __nv_bfloat16 *g = reinterpret_cast<__nv_bfloat16 *>(Gb + off);
-            __nv_bfloat16 *qq = reinterpret_cast<__nv_bfloat16 *>(Qb + off);
-            const float a = __bfloat162float(*g);
-            E *= fv[i];
-            const float k = k_from(a, fv[i]);
-            *g = __float2bfloat16_rn(k * __fdividef(1.0f, E));
-            *qq = __float2bfloat16_rn(__bfloat162float(*qq) * E);
-            fv[i] = E;
-        }
-        if (half == 1) m->EB[j] = E;
-        tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(fv));
-        tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(fv + 32));
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(half == 1 && !(E >= kMinEB))) {
-            if (tid == 0) set_status(HGRN2_ERR_DEVICE);   // the forward sweep passed this (b,h)
-            ok = false;
-            break;
+                for (int i = 0; i < 8; ++i) {
+                    av[i] = bfat(Gb, t0 + i);
+                    qv[i] = bfat(Qb, t0 + i);
+                }
+                __nv_bfloat16 oq[8], ok2[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    bsum += av[i];
+                    const float E = __expf(bsum), iE = __expf(-bsum);
+                    ok2[i] = __float2bfloat16_rn(k_gate(av[i], E * ip) * iE);
+                    oq[i] = __float2bfloat16_rn(qv[i] * E);
+                    ev[8 * bt + i] = E;
+                    ip = iE;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    *reinterpret_cast<__nv_bfloat16 *>(Gb + eoff(t0 + i)) = ok2[i];
+                    *reinterpret_cast<__nv_bfloat16 *>(Qb + eoff(t0 + i)) = oq[i];
+                }
+            }
+            tmem_st32(tl + kColE + c0, ev);
+            tmem_wait_st();
+            if (q4 == 3) m->EB[j] = __expf(bsum);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (__syncthreads_or(q4 == 3 && !(bsum >= kMinLogEB))) {
+                if (tid == 0) set_status(HGRN2_ERR_DEVICE);   // the forward sweep passed this (b,h)
+                ok = false;
+                break;
+            }
         }
         // ---- phase 1: A^T = Kt Qt^T (M = s, N = t), dA = dO V^T (M = t, N = s)
         if (tid == 0) {
-            if (!mbar_wait(&m->barDO, par)) ok = false;
+            if (!mbar_wait(&m->barVO, par)) ok = false;
             else waited[1] = it + 1;
             tc_fence_after();
 #pragma unroll
@@ -563,45 +577,34 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         __syncthreads();
         // ---- dS phase: dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16
         {
-            float r0[32], r1[32];
+            float v[32];
             tc_fence_after();
-            tmem_ld32(tl + kColDS + 64 * half, r0);
-            tmem_ld32(tl + kColDS + 64 * half + 32, r1);
+            tmem_ld32(tl + kColDS + c0, v);
             tmem_wait_ld();
             const float e = m->EB[j];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                r0[i] *= e;
-                r1[i] *= e;
-            }
-            store_row_bf16(D16 + half * kBlk, j, r0, r1);
-            tmem_st32(tl + kColDS + 64 * half, r0);
-            tmem_st32(tl + kColDS + 64 * half + 32, r1);
+            for (int i = 0; i < 32; ++i) v[i] *= e;
+            store_chunk_bf16(D16, j, q4, v);
+            tmem_st32(tl + kColDS + c0, v);
             tmem_wait_st();
         }
         // ---- masks: A^T keeps t >= s (lane s), dA keeps s <= t (lane t)
         {
             if (!mbar_wait(&m->barP1, par)) ok = false;
             tc_fence_after();
-            float r0[32], r1[32];
-            tmem_ld32(tl + kColX1 + 64 * half, r0);
-            tmem_ld32(tl + kColX1 + 64 * half + 32, r1);
+            float v[32];
+            tmem_ld32(tl + kColX1 + c0, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (64 * half + i < j) r0[i] = 0.0f;
-                if (64 * half + 32 + i < j) r1[i] = 0.0f;
-            }
-            store_row_bf16(AT + half * kBlk, j, r0, r1);
-            tmem_ld32(tl + kColX2 + 64 * half, r0);
-            tmem_ld32(tl + kColX2 + 64 * half + 32, r1);
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i < j) v[i] = 0.0f;
+            store_chunk_bf16(AT, j, q4, v);
+            tmem_ld32(tl + kColX2 + c0, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (64 * half + i > j) r0[i] = 0.0f;
-                if (64 * half + 32 + i > j) r1[i] = 0.0f;
-            }
-            store_row_bf16(DA + half * kBlk, j, r0, r1);
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i > j) v[i] = 0.0f;
+            store_chunk_bf16(DA, j, q4, v);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -645,94 +648,88 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (__syncthreads_or(!mbar_wait(&m->barP2, par))) { ok = false; break; }
         tc_fence_after();
         if (tid == 0) {
-            issue_one(Vb, &tm_dq, &m->barDQ, n);                  // dq of this chunk, for d log f
-            if (n > 0) issue_one(Ob, &tm_do, &m->barDO, n - 1);   // dO of the next chunk
+            // dq of this chunk into D16; v and dO of the next chunk into Vb, Ob
+            ++issued[2];
+            mbar_arrive_expect_tx(&m->barDQ, kTileBytes);
+            tma_load_4d(D16, &tm_dq, &m->barDQ, 0, h, n * kTile, b);
+            tma_load_4d(D16 + kBlk, &tm_dq, &m->barDQ, 64, h, n * kTile, b);
+            if (n > 0) issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
         }
         // ---- di (lane s) -> AT (rows s) for the TMA store
         {
-            float r0[32], r1[32];
-            tmem_ld32(tl + kColX1 + 64 * half, r0);
-            tmem_ld32(tl + kColX1 + 64 * half + 32, r1);
+            float v[32];
+            tmem_ld32(tl + kColX1 + c0, v);
             tmem_wait_ld();
-            store_row_bf16(AT + half * kBlk, j, r0, r1);
+            store_chunk_bf16(AT, j, q4, v);
         }
-        // ---- d log f (lane j, tokens 64*half .. +63): partial values (without the carry)
-        // d'_t = sum_{t<=t'<chunk half end} (q dq - k dk)_{t'} - f_t dk_t, kept in TMEM X1
-        // (di has been read out), with q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}.
+        // ---- d log f (lane j, tokens c0 .. c0+31): partial values kept in TMEM X1 (di has
+        // been read out): d'_t = sum_{t<=t'<quarter end} (q dq - k dk)_{t'} - f_t dk_t with
+        // q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}
         if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
         waited[2] = it + 1;
         float suf = 0.0f;
-#pragma unroll
-        for (int c = 1; c >= 0; --c) {
+        {
             float dkp[32], e[32], dap[32];
-            const int col = 64 * half + 32 * c;
-            tmem_ld32(tl + kColX2 + col, dkp);
-            tmem_ld32(tl + kColE + col, e);
-            const float eprev = col > 0 ? tmem_ld1(tl + kColE + col - 1) : 1.0f;
+            tmem_ld32(tl + kColX2 + c0, dkp);
+            tmem_ld32(tl + kColE + c0, e);
+            const float eprev = c0 > 0 ? tmem_ld1(tl + kColE + c0 - 1) : 1.0f;
             tmem_wait_ld();
             float invE = __fdividef(1.0f, e[31]);
 #pragma unroll
             for (int i = 31; i >= 0; --i) {
-                const int t = col + i;
-                const uint32_t off = elem_off(t);
-                const float qt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Qb + off));
-                const float kt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb + off));
-                const float dq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Vb + off));
+                const int t = c0 + i;
+                const float qt = bfat(Qb, t), kt = bfat(Gb, t), dq = bfat(D16, t);
                 const float invEm1 = __fdividef(1.0f, i > 0 ? e[i - 1] : eprev);
                 suf += qt * invE * dq - kt * dkp[i];
                 dap[i] = suf - dkp[i] * invEm1;
                 invE = invEm1;
             }
-            tmem_st32(tl + kColX1 + col, dap);
+            tmem_st32(tl + kColX1 + c0, dap);
+            tmem_wait_st();
         }
-        tmem_wait_st();
-        m->Ppart[half][j] = suf;
+        // quarter totals: quarters 0..2 in Bpart, quarter 3 in EB (free until the next prep)
+        if (q4 < 3) m->Bpart[q4][j] = suf;
+        else m->EB[j] = suf;
         __syncthreads();
         {
-            const float carry = m->carry[j] + (half == 0 ? m->Ppart[1][j] : 0.0f);
+            float carry = m->carry[j];   // from later chunks (and rowsum(dhT * hT))
+            if (q4 < 3) carry += m->EB[j];
+            for (int r2 = q4 + 1; r2 < 3; ++r2) carry += m->Bpart[r2][j];
+            float dap[32];
+            tmem_ld32(tl + kColX1 + c0, dap);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float dap[32];
-                const int col = 64 * half + 32 * c;
-                tmem_ld32(tl + kColX1 + col, dap);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    *reinterpret_cast<__nv_bfloat16 *>(DA + elem_off(col + i)) = __float2bfloat16_rn(dap[i] + carry);
-            }
+            for (int i = 0; i < 32; ++i)
+                *reinterpret_cast<__nv_bfloat16 *>(DA + eoff(c0 + i)) = __float2bfloat16_rn(dap[i] + carry);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (half == 0) m->carry[j] += m->Ppart[0][j] + m->Ppart[1][j];
+        if (q4 == 0) m->carry[j] += m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
         if (tid == 0) {
             tma_store_4d(&tm_di, AT, 0, h, n * kTile, b);
             tma_store_4d(&tm_di, AT + kBlk, 64, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA + kBlk, 64, h, n * kTile, b);
             tma_store_commit();
-            if (n > 0) issue_in(n - 1);   // the epilogue has read Qb, Gb, Vb
+            if (n > 0) issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, n - 1);   // epilogue read Qt, Kt
         }
     }
     if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
     if (tid == 0) {   // drain loads that may still be landing in this CTA's shared memory
-        uint64_t *bars[3] = {&m->barIn, &m->barDO, &m->barDQ};
+        uint64_t *bars[3] = {&m->barIn, &m->barVO, &m->barDQ};
         for (int q = 0; q < 3; ++q)
             for (int k = waited[q]; k < issued[q]; ++k) mbar_wait(bars[q], k & 1, 2000000u);
         tma_store_wait_all0();
     }
     if (ok && n < 0 && p.dh0) {
         tc_fence_after();
-        float r0[32], r1[32];
-        tmem_ld32(tl + kColDS + 64 * half, r0);
-        tmem_ld32(tl + kColDS + 64 * half + 32, r1);
+        float v[32];
+        tmem_ld32(tl + kColDS + c0, v);
         tmem_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * 128 + j) * 128 + 64 * half);
+        float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * 128 + j) * 128 + c0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            dst[i] = make_float4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
-            dst[8 + i] = make_float4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
-        }
+        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
     if (tid == 0 && ok && n < 0) atomicAdd(&g_counters[1], (unsigned long long)N);
     tc_fence_before();
@@ -766,7 +763,7 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles};
-    tcb::rev_kernel<<<a.B * a.H, tcb::kThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, p2);
+    tcb::rev_kernel<<<a.B * a.H, tcb::rsw::kRevThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, p2);
     return cudaGetLastError();
 }
 
