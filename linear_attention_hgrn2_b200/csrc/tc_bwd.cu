@@ -144,6 +144,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
                     tma_load_4d(Ob[s] + c * kBlk, &tm_do, &m->full[s], 64 * c, h, n * kTile, b);
                 }
                 ++producer_issued;
+                if (n + 2 < N)   // warm L2 for the chunk after next (its load waits for a free stage)
+                    for (int c = 0; c < 2; ++c) {
+                        tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (n + 2) * kTile, b);
+                        tma_prefetch_l2_4d(&tm_x, 64 * c, h, (n + 2) * kTile, b);
+                        tma_prefetch_l2_4d(&tm_do, 64 * c, h, (n + 2) * kTile, b);
+                    }
             }
         }
     } else if (warp == 1) {
@@ -404,6 +410,7 @@ struct __align__(8) Misc {
     uint64_t barIn, barVO, barDQ, barP1, barP2;
     uint32_t tmem_base;
     int pad;
+    int issued[3], waited[3];   // loads issued / arrivals waited for: [barIn, barVO, barDQ]
     float EB[128];
     float Bpart[3][128];   // per 32-row range sums of log f; in the epilogue, quarter suffix totals
     float carry[128];
@@ -458,8 +465,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t tbase = m->tmem_base;
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
 
-    // loads issued / arrivals waited for, per barrier (thread 0's view): [barIn, barVO, barDQ]
-    int issued[3] = {0, 0, 0}, waited[3] = {0, 0, 0};
+    int *issued = m->issued, *waited = m->waited;   // thread 0 issues; waits are recorded by thread 0
+    if (tid == 0)
+        for (int q = 0; q < 3; ++q) issued[q] = waited[q] = 0;
     auto issue2 = [&](uint8_t *d0, const CUtensorMap *t0, uint8_t *d1, const CUtensorMap *t1, uint64_t *bar,
                       int q, int n) {
         ++issued[q];
@@ -504,7 +512,18 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     for (; n >= 0; --n, ++it) {
         const uint32_t par = it & 1;
         if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
-        waited[0] = it + 1;
+        if (tid == 0) waited[0] = it + 1;
+        if (tid == 0) {   // warm L2: this chunk's dq, the next chunk's inputs
+            for (int c = 0; c < 2; ++c) {
+                tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
+                if (n > 0) {
+                    tma_prefetch_l2_4d(&tm_q, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_x, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_do, 64 * c, h, (n - 1) * kTile, b);
+                }
+            }
+        }
         // ---- prep: column j, rows c0 .. c0+31: Qt = q E, Kt = k / E in place; E -> TMEM
         {
             float sum = 0.0f;
@@ -664,29 +683,41 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         // ---- d log f (lane j, tokens c0 .. c0+31): partial values kept in TMEM X1 (di has
         // been read out): d'_t = sum_{t<=t'<quarter end} (q dq - k dk)_{t'} - f_t dk_t with
-        // q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}
-        if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
-        waited[2] = it + 1;
-        float suf = 0.0f;
-        {
-            float dkp[32], e[32], dap[32];
-            tmem_ld32(tl + kColX2 + c0, dkp);
-            tmem_ld32(tl + kColE + c0, e);
-            const float eprev = c0 > 0 ? tmem_ld1(tl + kColE + c0 - 1) : 1.0f;
-            tmem_wait_ld();
-            float invE = __fdividef(1.0f, e[31]);
+        // q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}.  Qt and Kt are copied to
+        // registers first, so that q and log f of the next chunk can load during the epilogue.
+        uint32_t qk[32];
 #pragma unroll
-            for (int i = 31; i >= 0; --i) {
-                const int t = c0 + i;
-                const float qt = bfat(Qb, t), kt = bfat(Gb, t), dq = bfat(D16, t);
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t off = eoff(c0 + i);
+            qk[i] = (uint32_t)*reinterpret_cast<const uint16_t *>(Qb + off) |
+                    ((uint32_t)*reinterpret_cast<const uint16_t *>(Gb + off) << 16);
+        }
+        __syncthreads();
+        if (tid == 0 && n > 0) issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, n - 1);
+        if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
+        if (tid == 0) waited[2] = it + 1;
+        float suf = 0.0f;
+#pragma unroll
+        for (int hh = 1; hh >= 0; --hh) {
+            float dkp[16], e[16], dap[16];
+            const int col = c0 + 16 * hh;
+            tmem_ld16(tl + kColX2 + col, dkp);
+            tmem_ld16(tl + kColE + col, e);
+            const float eprev = col > 0 ? tmem_ld1(tl + kColE + col - 1) : 1.0f;
+            tmem_wait_ld();
+            float invE = __fdividef(1.0f, e[15]);
+#pragma unroll
+            for (int i = 15; i >= 0; --i) {
+                const int t = col + i;
+                const float qt = bf_lo(qk[16 * hh + i]), kt = bf_hi(qk[16 * hh + i]), dq = bfat(D16, t);
                 const float invEm1 = __fdividef(1.0f, i > 0 ? e[i - 1] : eprev);
                 suf += qt * invE * dq - kt * dkp[i];
                 dap[i] = suf - dkp[i] * invEm1;
                 invE = invEm1;
             }
-            tmem_st32(tl + kColX1 + c0, dap);
-            tmem_wait_st();
+            tmem_st16(tl + kColX1 + col, dap);
         }
+        tmem_wait_st();
         // quarter totals: quarters 0..2 in Bpart, quarter 3 in EB (free until the next prep)
         if (q4 < 3) m->Bpart[q4][j] = suf;
         else m->EB[j] = suf;
@@ -712,7 +743,6 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA + kBlk, 64, h, n * kTile, b);
             tma_store_commit();
-            if (n > 0) issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, n - 1);   // epilogue read Qt, Kt
         }
     }
     if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
