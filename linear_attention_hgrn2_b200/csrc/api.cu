@@ -100,10 +100,15 @@ hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const fl
         float *seg_ws = (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
         int nseg, tps;
         tc_fwd_segments(B, T, H, &nseg, &tps);
-        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H};
-        g_launches += nseg > 1 ? 4 : 2;
+        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H, C};
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+        if (nseg == 1) {   // the exact route, if needed, runs inside the tensor-core kernel
+            g_launches += 1;
+            return HGRN2_OK;
+        }
+        // segmented: aggregate, scan, segments, then the exact route for flagged (b,h)
+        g_launches += 4;
         SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags};
         return from_cuda(launch_simt_fwd(a, bf16, stream));
     }
@@ -137,12 +142,9 @@ hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const fl
     float *rs = (float *)workspace;
     if (use_tc(dk, dv, dtype)) {
         int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
-        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H};
-        g_launches += 4;
-        cudaError_t e = launch_tc_bwd(t, stream);
-        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
-        SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, flags};
-        return from_cuda(launch_simt_bwd(a, bf16, stream));
+        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C};
+        g_launches += 2;   // the exact route, if needed, runs inside the forward-sweep kernel
+        return from_cuda(launch_tc_bwd(t, stream));
     }
     SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr};
     g_launches += 2;

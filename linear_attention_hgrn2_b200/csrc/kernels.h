@@ -23,6 +23,7 @@ struct TcFwdArgs {
     int *flags;        // [B*H] out: 1 where the (b,h) needs the exact route
     float *seg_ws;     // segment aggregates, tc_fwd_workspace(B, T, H) bytes (may be null if 0)
     int B, T, H;
+    int simt_C;        // chunk of the exact route
 };
 
 struct SimtBwdArgs {
@@ -43,6 +44,7 @@ struct TcBwdArgs {
     float *rs;         // [B*H*128] workspace
     int *flags;        // [B*H] workspace, out: 1 where the (b,h) needs the exact route
     int B, T, H;
+    int simt_C;        // chunk of the exact route (run inside the forward-sweep kernel)
 };
 
 size_t simt_fwd_smem(int C, int dk, int dv);

@@ -68,12 +68,10 @@ static __device__ __forceinline__ void cumsum_gates(float *Bs, float *Ks, int ld
 
 // ------------------------------------------------------------------ forward
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
-simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
+__device__ __forceinline__ void
+simt_fwd_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
-                int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
-    if (only && only[blockIdx.x] == 0) return;
-    extern __shared__ float sm[];
+                int T_, int H, int dk, int dv, int C, float *sm, int bh) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;              // [C][ldk]  q, then q * e^{b}
     float *Bs = Qs + C * ldk;    // [C][ldk]  log f, then cumulative b
@@ -81,7 +79,7 @@ simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__re
     float *Vs = Ks + C * ldk;    // [C][ldv]
     float *As = Vs + C * ldv;    // [C][ldc]
     float *Ss = As + C * ldc;    // [dk][ldv] running state (fp32)
-    const int bh = blockIdx.x, b = bh / H, h = bh % H, tid = threadIdx.x;
+    const int b = bh / H, h = bh % H, tid = threadIdx.x;
     const size_t sbase = (size_t)bh * dk * dv;
 
     for (int idx = tid; idx < dk * dv; idx += blockDim.x) {
@@ -145,12 +143,10 @@ simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__re
 // dA_ts = dO_t . v_s.  Also writes rs[j] = sum_v dhT[j,v] hT[j,v] when dhT != NULL (used by the
 // reverse sweep's d log f carry).
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
-simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
+__device__ __forceinline__ void
+simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
-                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
-    if (only && only[blockIdx.x] == 0) return;
-    extern __shared__ float sm[];
+                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, float *sm, int bh) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Bs = sm;              // [C][ldk]
     float *Ks = Bs + C * ldk;    // [C][ldk]
@@ -158,7 +154,7 @@ simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const floa
     float *Gs = Vs + C * ldv;    // [C][ldv] dO
     float *As = Gs + C * ldv;    // [C][ldc] dA
     float *Ss = As + C * ldc;    // [dk][ldv]
-    const int bh = blockIdx.x, b = bh / H, h = bh % H, tid = threadIdx.x;
+    const int b = bh / H, h = bh % H, tid = threadIdx.x;
     const size_t sbase = (size_t)bh * dk * dv;
 
     for (int idx = tid; idx < dk * dv; idx += blockDim.x) {
@@ -221,13 +217,11 @@ simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const floa
 //   dS_in = Diag(e^B) dS + sum_t (q_t e^{b_t}) dO_t^T
 // The reverse cumulative sum runs across chunks through `carry`.
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
-simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
+__device__ __forceinline__ void
+simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
-                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
-    if (only && only[blockIdx.x] == 0) return;
-    extern __shared__ float sm[];
+                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, float *sm, int bh) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;               // [C][ldk] q, later q e^{b}
     float *Bs = Qs + C * ldk;     // [C][ldk] b
@@ -241,7 +235,7 @@ simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *
     float *dAs = As + C * ldc;    // [C][ldc]
     float *dS = dAs + C * ldc;    // [dk][ldv]
     float *carry = dS + dk * ldv; // [dk]
-    const int bh = blockIdx.x, b = bh / H, h = bh % H, tid = threadIdx.x;
+    const int b = bh / H, h = bh % H, tid = threadIdx.x;
     const size_t sbase = (size_t)bh * dk * dv;
 
     for (int idx = tid; idx < dk * dv; idx += blockDim.x) {
@@ -330,6 +324,39 @@ simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *
             int j = idx / dv, v = idx - j * dv;
             dh0[sbase + idx] = dS[j * ldv + v];
         }
+}
+
+
+// ------------------------------------------------------------------ kernels (one CTA per (b,h))
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
+                const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
+                int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+    if (only && only[blockIdx.x] == 0) return;
+    extern __shared__ float sm[];
+    simt_fwd_body<T>(q, lf, x, h0, o, hT, T_, H, dk, dv, C, sm, blockIdx.x);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
+                   const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
+                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+    if (only && only[blockIdx.x] == 0) return;
+    extern __shared__ float sm[];
+    simt_bwd_dq_body<T>(lf, x, h0, dO, dhT, dq, rs, T_, H, dk, dv, C, sm, blockIdx.x);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
+                    const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
+                    const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
+                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+    if (only && only[blockIdx.x] == 0) return;
+    extern __shared__ float sm[];
+    simt_bwd_rev_body<T>(q, lf, x, dO, dhT, dq, rs, dlf, dx, dh0, T_, H, dk, dv, C, sm, blockIdx.x);
 }
 
 // ------------------------------------------------------------------ launchers

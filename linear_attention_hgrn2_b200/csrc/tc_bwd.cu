@@ -77,6 +77,11 @@ struct DqParams {
     float *rs;       // [B*H*128] rowsum(dhT * hT)
     int *flags;      // [B*H]
     int T, H, ntiles;
+    // for the in-kernel exact route
+    const __nv_bfloat16 *q, *lf, *x, *dO;
+    __nv_bfloat16 *dq, *dlf, *dx;
+    float *dh0;
+    int simt_chunk;
 };
 
 __global__ void __launch_bounds__(fsw::kDqThreads, 1)
@@ -392,6 +397,17 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     }
     __syncwarp();
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+    // exact route for this (b,h): both sweeps on CUDA cores in the drained CTA (the reverse
+    // tensor-core kernel skips flagged pairs)
+    if (fell_back) {
+        __syncthreads();
+        float *sm = reinterpret_cast<float *>(smem);
+        simt_bwd_dq_body<__nv_bfloat16>(p.lf, p.x, p.h0, p.dO, p.dhT, p.dq, p.rs, p.T, p.H, 128, 128,
+                                        p.simt_chunk, sm, bh);
+        __syncthreads();
+        simt_bwd_rev_body<__nv_bfloat16>(p.q, p.lf, p.x, p.dO, p.dhT, p.dq, p.rs, p.dlf, p.dx, p.dh0, p.T, p.H,
+                                         128, 128, p.simt_chunk, sm, bh);
+    }
 }
 
 // ------------------------------------------------------------------ reverse sweep
@@ -788,7 +804,10 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     e = cudaFuncSetAttribute(tcb::rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcb::rsw::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
-    tcb::DqParams p1{a.h0, a.dhT, a.rs, a.flags, a.T, a.H, ntiles};
+    tcb::DqParams p1{a.h0, a.dhT, a.rs, a.flags, a.T, a.H, ntiles,
+                     (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
+                     (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
+                     (__nv_bfloat16 *)a.dx, a.dh0, a.simt_C};
     tcb::dq_kernel<<<a.B * a.H, tcb::fsw::kDqThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -64,6 +64,8 @@ struct Params {
     const float *h0;
     float *hT;
     __nv_bfloat16 *o;
+    const __nv_bfloat16 *q, *lf, *x;   // for the in-kernel exact route
+    int simt_chunk;
     int *flags;       // [B*H] set to 1 when the (b,h) must take the exact route
     const float *Sin; // [B*H][nseg-1][128][128] state entering segments 1.. (from the scan)
     int T, H, ntiles;
@@ -388,6 +390,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     __syncwarp();
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+    // exact route for this (b,h) when it runs unsegmented: the pipeline is drained, so the
+    // CTA's shared memory is free for the CUDA-core chunkwise forward of the whole sequence
+    if (fell_back && p.nseg == 1) {
+        __syncthreads();
+        simt_fwd_body<__nv_bfloat16>(p.q, p.lf, p.x, p.h0, p.o, p.hT, p.T, p.H, 128, 128, p.simt_chunk,
+                                     reinterpret_cast<float *>(smem), bh);
+    }
 }
 
 // ------------------------------------------------------------------ sequence segments
@@ -635,7 +644,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
         tcf::scan_kernel<<<BH * 16, 256, 0, st>>>(a.h0, U, g, nseg);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, a.flags, U, a.T, a.H, ntiles, nseg, tps};
+    tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
+                  (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps};
     tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, p);
     return cudaGetLastError();
 }
