@@ -4,8 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one training pass of the chunkwise recurrence over one batch: the
-forward (hgrn2_fwd) and the backward (hgrn2_bwd, gradients of q, log f and i)
-on the training workload B=8, H=16, T=2048, d_k=d_v=128, bf16 token tensors,
+forward that keeps the chunk states (hgrn2_fwd_train) and the backward that
+reads them (hgrn2_bwd_saved, gradients of q, log f and i) on the training workload B=8, H=16, T=2048, d_k=d_v=128, bf16 token tensors,
 fp32 state, forget-gate lower bound 0.95, dO ~ N(0,1).  Inputs (268 MB of
 token tensors per step, more than the 126 MB L2) are resident in HBM before
 the timed region.  Under torchrun each rank runs its own batch on its own GPU
@@ -185,10 +185,11 @@ def run_ours(args, world, rank, local):
     ws_f = torch.empty(max(L.workspace_size(B, T, H, dk, dv, chunk, w.dtype, False), 16), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(max(L.workspace_size(B, T, H, dk, dv, chunk, w.dtype, True), 16), dtype=torch.uint8, device=dev)
     o = torch.empty_like(x)
+    sv = L.new_saved(q)   # chunk states kept by the training forward for the backward
 
     def step():
-        L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f)
-        return L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b)
+        L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f, saved=sv)
+        return L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b, saved=sv)
 
     for _ in range(args.warmup):
         step()
@@ -206,9 +207,9 @@ def run_ours(args, world, rank, local):
         t0.record(stream)
         for k in range(K):
             evs[k][0].record(stream)
-            L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f)
+            L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f, saved=sv)
             evs[k][1].record(stream)
-            L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b)
+            L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b, saved=sv)
             evs[k][2].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
@@ -225,9 +226,9 @@ def run_ours(args, world, rank, local):
     pk = peaks()
     th = B * T * H   # token-heads per step
     if bwd_ms >= fwd_ms:
-        dom, dom_ms, dom_bytes = "hgrn2_bwd", bwd_ms, BWD_BYTES * th
+        dom, dom_ms, dom_bytes = "hgrn2_bwd_saved", bwd_ms, BWD_BYTES * th
     else:
-        dom, dom_ms, dom_bytes = "hgrn2_fwd", fwd_ms, FWD_BYTES * th
+        dom, dom_ms, dom_bytes = "hgrn2_fwd_train", fwd_ms, FWD_BYTES * th
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     tr = traffic_record(dom)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
@@ -250,12 +251,13 @@ def run_ours(args, world, rank, local):
            "config": {"workload": w.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv, "chunk": chunk,
                       "lb": w.lb, "global_batch": B * world, "seq_len": T,
                       "parallelism": f"dp{world} (independent replicas, no collective)",
+                      "calls": "hgrn2_fwd_train + hgrn2_bwd_saved",
                       "l2": "no flush: 268 MB of token inputs per step > 126 MB L2"},
            "roofline": roofline, "step_roofline": step_roof, "gpu_launches": launches,
            "clocks": clk.summary()}
 
     if not args.no_e2e:
-        out["e2e"] = run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, w, world)
+        out["e2e"] = run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, sv, w, world)
     if not args.no_decode:
         out["decode_step"] = run_decode(args, dev, pk)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -264,7 +266,7 @@ def run_ours(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
-def run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, w, world):
+def run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, sv, w, world):
     """Same step through host buffers: pinned H2D of the inputs and D2H of all outputs inside the timed region."""
     import linear_attention_hgrn2_b200 as L
     hq, hlf, hx, hdO = (t.cpu().pin_memory() for t in (q, lf, x, dO))
@@ -275,8 +277,8 @@ def run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, w, world):
     def one():
         q.copy_(hq, non_blocking=True); lf.copy_(hlf, non_blocking=True)
         x.copy_(hx, non_blocking=True); dO.copy_(hdO, non_blocking=True)
-        L.fwd(q, lf, x, chunk=w.chunk, out=o, workspace=ws_f)
-        dq, dlf, di, _ = L.bwd(q, lf, x, dO, chunk=w.chunk, workspace=ws_b)
+        L.fwd(q, lf, x, chunk=w.chunk, out=o, workspace=ws_f, saved=sv)
+        dq, dlf, di, _ = L.bwd(q, lf, x, dO, chunk=w.chunk, workspace=ws_b, saved=sv)
         ho.copy_(o, non_blocking=True); hdq.copy_(dq, non_blocking=True)
         hdlf.copy_(dlf, non_blocking=True); hdi.copy_(di, non_blocking=True)
 

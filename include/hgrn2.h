@@ -105,6 +105,44 @@ hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const fl
                        int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
                        void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* Training pair: a forward that keeps the chunk states, and a backward that reads
+ * them instead of recomputing them.  Chunkwise training (§3.2: the GLA-style
+ * chunkwise algorithm) needs the state entering every chunk in both passes;
+ * storing it in the forward halves the backward's sweeps over the sequence.
+ *
+ * hgrn2_saved_size: bytes of the saved-state buffer for these sizes.  0 when the
+ * configuration has no saved-state path (the exact CUDA-core route, or T = 0):
+ * hgrn2_fwd_train and hgrn2_bwd_saved then behave exactly as hgrn2_fwd and
+ * hgrn2_bwd and ignore `saved` (which may be NULL).  (size_t)-1 for invalid or
+ * unsupported arguments.  Host-only, no CUDA call.
+ *
+ * The buffer (device memory, caller-owned, 16-byte aligned, no initialisation
+ * needed) is opaque.  For the bf16 tensor-core route it holds, per (b,h), the
+ * bf16-rounded state entering each 128-token chunk (the same operand the forward
+ * multiplies with; ceil(T/128) x 128 x 128 x 2 bytes), the float32 final state,
+ * and which (b,h) took the exact route.
+ *
+ * hgrn2_fwd_train: hgrn2_fwd (same arguments and results) that also fills
+ *   `saved` (saved_bytes >= hgrn2_saved_size, else HGRN2_ERR_INVALID_ARG).
+ * hgrn2_bwd_saved: hgrn2_bwd (same arguments and results, same workspace size)
+ *   for a forward made by hgrn2_fwd_train with the same q, log_f, i, h0 and
+ *   sizes, whose `saved` buffer is passed unchanged.  A buffer from other inputs
+ *   gives wrong gradients (it is not checked).  dq is only written, never read
+ *   back, on this path.  The bf16 route runs one kernel launch. */
+size_t hgrn2_saved_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype);
+
+hgrn2_status hgrn2_fwd_train(const void *q, const void *log_f, const void *i, const float *h0,
+                             void *o, float *hT, void *saved, size_t saved_bytes,
+                             int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                             void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+hgrn2_status hgrn2_bwd_saved(const void *q, const void *log_f, const void *i, const float *h0,
+                             const void *saved, size_t saved_bytes,
+                             const void *dO, const float *dhT,
+                             void *dq, void *dlog_f, void *di, float *dh0,
+                             int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                             void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Allocation-free variant of hgrn2_bwd.  The paper has no counterpart: this
  * entry point exists for callers that cannot give the library a device
  * buffer -- for example a plain C host program that links only this library

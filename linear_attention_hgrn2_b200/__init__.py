@@ -26,8 +26,9 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(
 FP32, BF16 = 0, 1
 
 # Every extern "C" symbol of include/hgrn2.h.
-EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_bwd_noalloc", "hgrn2_step",
-           "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
+EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size", "hgrn2_fwd_train",
+           "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_step", "hgrn2_get_device_status",
+           "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
 
 _lib = None
 
@@ -54,6 +55,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_fwd.restype = i32
     lib.hgrn2_bwd.argtypes = [vp] * 10 + [i32] * 7 + [vp, sz, vp]
     lib.hgrn2_bwd.restype = i32
+    lib.hgrn2_saved_size.argtypes = [i32] * 6
+    lib.hgrn2_saved_size.restype = sz
+    lib.hgrn2_fwd_train.argtypes = [vp] * 7 + [sz] + [i32] * 7 + [vp, sz, vp]
+    lib.hgrn2_fwd_train.restype = i32
+    lib.hgrn2_bwd_saved.argtypes = [vp] * 5 + [sz] + [vp] * 6 + [i32] * 7 + [vp, sz, vp]
+    lib.hgrn2_bwd_saved.restype = i32
     lib.hgrn2_bwd_noalloc.argtypes = [vp] * 10 + [i32] * 7 + [vp]
     lib.hgrn2_bwd_noalloc.restype = i32
     lib.hgrn2_step.argtypes = [vp] * 5 + [i32] * 5 + [vp]
@@ -124,11 +131,29 @@ def _workspace(nbytes: int, device) -> torch.Tensor | None:
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def fwd(q, log_f, i, h0=None, want_hT=False, chunk=64, out=None, workspace=None):
+def saved_size(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Bytes of the buffer that fwd(..., saved=) fills for bwd(..., saved=); 0 when
+    this configuration has no saved-state path (the backward then recomputes)."""
+    n = load_library().hgrn2_saved_size(B, T, H, dk, dv, BF16 if dtype == torch.bfloat16 else FP32)
+    if n == ctypes.c_size_t(-1).value:
+        raise HGRN2Error(ERR_INVALID_ARG, "hgrn2_saved_size")
+    return int(n)
+
+
+def new_saved(q: torch.Tensor, dv: int | None = None) -> torch.Tensor | None:
+    """An uninitialised saved-state buffer for a forward on q (None if not needed)."""
+    B, T, H, dk = q.shape
+    n = saved_size(B, T, H, dk, dk if dv is None else dv, q.dtype)
+    return torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+
+
+def fwd(q, log_f, i, h0=None, want_hT=False, chunk=64, out=None, workspace=None, saved=None):
     """o = HGRN2(q, log_f, i; h0) and optionally the final state hT.
 
     q, log_f: [B,T,H,dk]; i: [B,T,H,dv] (float32 or bfloat16, all the same);
-    h0: [B,H,dk,dv] float32 or None.  Returns (o, hT or None)."""
+    h0: [B,H,dk,dv] float32 or None.  saved: a uint8 CUDA buffer of saved_size()
+    bytes (see new_saved) that receives the chunk states for bwd(..., saved=), or
+    None.  Returns (o, hT or None)."""
     lib = load_library()
     B, T, H, dk = q.shape
     dv = i.shape[-1]
@@ -142,14 +167,23 @@ def fwd(q, log_f, i, h0=None, want_hT=False, chunk=64, out=None, workspace=None)
     hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_hT else None
     nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, False)
     ws = workspace if workspace is not None else _workspace(nws, q.device)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8)
+        st = lib.hgrn2_fwd_train(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(o), _ptr(hT), _ptr(saved),
+                                 saved.numel(), B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
+        _raise(st, "hgrn2_fwd_train")
+        return o, hT
     st = lib.hgrn2_fwd(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(o), _ptr(hT),
                        B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
     _raise(st, "hgrn2_fwd")
     return o, hT
 
 
-def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dh0=False, chunk=64, workspace=None):
-    """Gradients (dq, dlog_f, di, dh0 or None) of L(o, hT) given dO (and dhT)."""
+def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dh0=False, chunk=64, workspace=None, saved=None):
+    """Gradients (dq, dlog_f, di, dh0 or None) of L(o, hT) given dO (and dhT).
+
+    saved: the buffer a fwd(..., saved=) on the same q, log_f, i, h0 filled (the
+    states are then read instead of recomputed), or None."""
     lib = load_library()
     B, T, H, dk = q.shape
     dv = i.shape[-1]
@@ -167,6 +201,13 @@ def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dh0=False, chunk=64, workspace=
     dh0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
     nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, True)
     ws = workspace if workspace is not None else _workspace(nws, q.device)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8)
+        st = lib.hgrn2_bwd_saved(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(saved), saved.numel(),
+                                 _ptr(dO), _ptr(dhT), _ptr(dq), _ptr(dlf), _ptr(di), _ptr(dh0),
+                                 B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
+        _raise(st, "hgrn2_bwd_saved")
+        return dq, dlf, di, dh0
     st = lib.hgrn2_bwd(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(dO), _ptr(dhT),
                        _ptr(dq), _ptr(dlf), _ptr(di), _ptr(dh0),
                        B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
@@ -209,19 +250,21 @@ class HGRN2Function(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, log_f, i, h0=None, chunk=64):
-        o, hT = fwd(q.contiguous(), log_f.contiguous(), i.contiguous(),
-                    None if h0 is None else h0.contiguous(), want_hT=True, chunk=chunk)
-        ctx.save_for_backward(q, log_f, i, h0)
+        q, log_f, i = q.contiguous(), log_f.contiguous(), i.contiguous()
+        h0 = None if h0 is None else h0.contiguous()
+        saved = new_saved(q, i.shape[-1])   # chunk states for the backward (None: recompute)
+        o, hT = fwd(q, log_f, i, h0, want_hT=True, chunk=chunk, saved=saved)
+        ctx.save_for_backward(q, log_f, i, h0, saved)
         ctx.chunk = chunk
         ctx.has_h0 = h0 is not None
         return o, hT
 
     @staticmethod
     def backward(ctx, dO, dhT):
-        q, log_f, i, h0 = ctx.saved_tensors
+        q, log_f, i, h0, saved = ctx.saved_tensors
         dq, dlf, di, dh0 = bwd(q, log_f, i, dO.contiguous(), h0,
                                None if dhT is None else dhT.contiguous(),
-                               want_dh0=ctx.has_h0, chunk=ctx.chunk)
+                               want_dh0=ctx.has_h0, chunk=ctx.chunk, saved=saved)
         return dq, dlf, di, dh0, None
 
 

@@ -58,6 +58,24 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
     return bytes;
 }
 
+// Saved-state buffer of the tensor-core route (written by hgrn2_fwd_train, read by
+// hgrn2_bwd_saved): bf16 state entering every 128-token chunk, fp32 final state, and the
+// forward's exact-route flags.
+struct SavedLayout {
+    size_t hTs, flags, total;   // byte offsets (the bf16 states start at 0)
+};
+SavedLayout saved_layout(int B, int T, int H) {
+    const size_t BH = (size_t)B * H, nt = (size_t)(T + 127) / 128;
+    SavedLayout l;
+    l.hTs = align256(BH * nt * 128 * 128 * 2);
+    l.flags = l.hTs + align256(BH * 128 * 128 * sizeof(float));
+    l.total = l.flags + align256(BH * sizeof(int));
+    return l;
+}
+size_t saved_bytes_needed(int B, int T, int H, int dk, int dv, hgrn2_dtype dt) {
+    return (use_tc(dk, dv, dt) && T > 0) ? saved_layout(B, T, H).total : 0;
+}
+
 hgrn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HGRN2_OK : HGRN2_ERR_CUDA; }
 
 std::atomic<long long> g_launches{0};   // kernel launches issued (host side)
@@ -72,13 +90,18 @@ size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk, hgrn
     return ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, want_bwd);
 }
 
-hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o,
-                       float *hT, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
-                       void *workspace, size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Forward; `saved` (null, or saved_bytes_needed bytes) receives what hgrn2_bwd_saved reads.
+hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
+                      void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                      void *workspace, size_t ws_bytes, cudaStream_t stream) {
     hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !log_f || !i || !o)) return HGRN2_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, log_f, i, h0, o, hT, workspace};
+    const void *ptrs[] = {q, log_f, i, h0, o, hT, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
     size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 0);
@@ -96,11 +119,13 @@ hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const fl
     if (use_tc(dk, dv, dtype)) {
         // tensor-core pass; (b,h) pairs whose chunk decay span is too wide are flagged
         // and recomputed right after by the exact route (same stream, in order)
-        int *flags = (int *)workspace;
+        const SavedLayout sl = saved_layout(B, T, H);
+        int *flags = saved ? (int *)((char *)saved + sl.flags) : (int *)workspace;
         float *seg_ws = (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
         int nseg, tps;
         tc_fwd_segments(B, T, H, &nseg, &tps);
-        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H, C};
+        TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H, C, saved,
+                    saved ? (float *)((char *)saved + sl.hTs) : nullptr};
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         if (nseg == 1) {   // the exact route, if needed, runs inside the tensor-core kernel
@@ -117,14 +142,15 @@ hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const fl
     return from_cuda(launch_simt_fwd(a, bf16, stream));
 }
 
-hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *dO,
-                       const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B, int T,
-                       int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
-                       size_t ws_bytes, cudaStream_t stream) {
+// Backward; with `saved` (from fwd_impl on the same inputs) the states are read, not recomputed.
+hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                      const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
+                      int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                      size_t ws_bytes, cudaStream_t stream) {
     hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !log_f || !i || !dO || !dq || !dlog_f || !di)) return HGRN2_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, workspace};
+    const void *ptrs[] = {q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
     size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
@@ -141,14 +167,69 @@ hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const fl
     if (!C) return HGRN2_ERR_UNSUPPORTED;
     float *rs = (float *)workspace;
     if (use_tc(dk, dv, dtype)) {
+        if (saved) {   // one launch: reverse sweep from the saved states (exact route inside)
+            const SavedLayout sl = saved_layout(B, T, H);
+            TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs,
+                        (int *)((char *)saved + sl.flags), B, T, H, C, saved,
+                        (const float *)((const char *)saved + sl.hTs)};
+            g_launches += 1;
+            return from_cuda(launch_tc_bwd(t, stream));
+        }
         int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
-        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C};
+        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C, nullptr, nullptr};
         g_launches += 2;   // the exact route, if needed, runs inside the forward-sweep kernel
         return from_cuda(launch_tc_bwd(t, stream));
     }
     SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr};
     g_launches += 2;
     return from_cuda(launch_simt_bwd(a, bf16, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+hgrn2_status hgrn2_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o,
+                       float *hT, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                       void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    return fwd_impl(q, log_f, i, h0, o, hT, nullptr, B, T, H, dk, dv, chunk, dtype, workspace, ws_bytes, stream);
+}
+
+hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *dO,
+                       const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B, int T,
+                       int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                       size_t ws_bytes, cudaStream_t stream) {
+    return bwd_impl(q, log_f, i, h0, nullptr, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype,
+                    workspace, ws_bytes, stream);
+}
+
+size_t hgrn2_saved_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    if (check_common(B, T, H, dk, dv, 64, dtype) != HGRN2_OK) return (size_t)-1;
+    return saved_bytes_needed(B, T, H, dk, dv, dtype);
+}
+
+hgrn2_status hgrn2_fwd_train(const void *q, const void *log_f, const void *i, const float *h0, void *o,
+                             float *hT, void *saved, size_t saved_bytes, int B, int T, int H, int dk, int dv,
+                             int chunk, hgrn2_dtype dtype, void *workspace, size_t ws_bytes,
+                             cudaStream_t stream) {
+    hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    const size_t need = saved_bytes_needed(B, T, H, dk, dv, dtype);
+    if (need && (!saved || saved_bytes < need)) return HGRN2_ERR_INVALID_ARG;
+    return fwd_impl(q, log_f, i, h0, o, hT, need ? saved : nullptr, B, T, H, dk, dv, chunk, dtype, workspace,
+                    ws_bytes, stream);
+}
+
+hgrn2_status hgrn2_bwd_saved(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                             size_t saved_bytes, const void *dO, const float *dhT, void *dq, void *dlog_f,
+                             void *di, float *dh0, int B, int T, int H, int dk, int dv, int chunk,
+                             hgrn2_dtype dtype, void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    const size_t need = saved_bytes_needed(B, T, H, dk, dv, dtype);
+    if (need && (!saved || saved_bytes < need)) return HGRN2_ERR_INVALID_ARG;
+    return bwd_impl(q, log_f, i, h0, need ? saved : nullptr, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv,
+                    chunk, dtype, workspace, ws_bytes, stream);
 }
 
 hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *S, void *o, int B, int H,

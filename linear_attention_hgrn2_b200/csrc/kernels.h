@@ -24,6 +24,8 @@ struct TcFwdArgs {
     float *seg_ws;     // segment aggregates, tc_fwd_workspace(B, T, H) bytes (may be null if 0)
     int B, T, H;
     int simt_C;        // chunk of the exact route
+    void *st16;        // out, or null: bf16 state entering every chunk [B*H][ntiles][128][128]
+    float *hTs;        // out (with st16): final state [B*H][128][128]
 };
 
 struct SimtBwdArgs {
@@ -42,9 +44,11 @@ struct TcBwdArgs {
     void *dq, *dlf, *dx;
     float *dh0;
     float *rs;         // [B*H*128] workspace
-    int *flags;        // [B*H] workspace, out: 1 where the (b,h) needs the exact route
+    int *flags;        // [B*H] recompute: workspace, out; saved states: in, from the forward
     int B, T, H;
-    int simt_C;        // chunk of the exact route (run inside the forward-sweep kernel)
+    int simt_C;        // chunk of the exact route
+    const void *st16;  // saved bf16 chunk-entry states [B*H][ntiles][128][128], or null (recompute)
+    const float *hTs;  // saved final state [B*H][128][128] (with st16)
 };
 
 size_t simt_fwd_smem(int C, int dk, int dv);

@@ -133,7 +133,6 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
     int producer_issued = 0;
-    bool fell_back_here = false;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -310,7 +309,6 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
         if (r == 0) tma_store_wait_all0();
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        fell_back_here = n < N;
         if (n == N && p.dhT && p.rs) {
             // hT = Diag(E_B of the last chunk) S';  rs[j] = sum_v dhT[j,v] hT[j,v]
             const float *g = p.dhT + ((size_t)bh * 128 + r) * 128;
@@ -387,7 +385,6 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const bool fell_back = m->bad_tile < N;
-    (void)fell_back_here;
     if (warp == 0 && lane == 0)
         for (int k = m->waited_full; k < producer_issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
     if (tid == 0) {
@@ -415,15 +412,23 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 // quarter = warp >> 2 selects 32 TMEM columns (or 32 rows of the chunk in the prep).
 // Shared memory (7 tiles of 32 KB): Qb q -> Qt, Gb log f -> Kt, Vb v, Ob dO, D16 bf16(dSh)
 // then the dq tile, AT mask(A)^T then di staging, DA mask(dA) then d log f staging.
-// As soon as the MMAs of a chunk are done, dq of this chunk lands in D16 and v, dO of the
-// next chunk in Vb, Ob; q and log f of the next chunk follow once the epilogue has read
-// Qt and Kt.
+//
+// Two modes.  Recompute mode (kSaved = false) follows the forward-sweep kernel: as soon
+// as the MMAs of a chunk are done, dq of this chunk (written by that kernel) lands in D16
+// and v, dO of the next chunk in Vb, Ob; q and log f of the next chunk follow once the
+// epilogue has read Qt and Kt.  Saved-state mode (kSaved = true) needs no forward sweep:
+// the bf16 state entering each chunk, stored by the training forward, lands in D16 and a
+// third MMA phase forms dq itself, transposed (lane j, tokens along the columns),
+//     dq_pre^T = S_in dO^T + Kt^T mask(dA)^T,      dq = E * dq_pre,
+// reusing the masked dA of this chunk; q dq = Qt dq_pre then enters d log f without
+// reading dq back.  A (batch, head) that the forward flagged for the exact route runs
+// both exact sweeps here, on CUDA cores.
 namespace rsw {
 constexpr uint32_t kColDS = 0, kColX1 = 128, kColX2 = 256, kColE = 384;
 constexpr int kRevThreads = 512;
 
 struct __align__(8) Misc {
-    uint64_t barIn, barVO, barDQ, barP1, barP2;
+    uint64_t barIn, barVO, barDQ, barP1, barP2, barP3;   // barDQ: dq (recompute) or S_in (saved)
     uint32_t tmem_base;
     int pad;
     int issued[3], waited[3];   // loads issued / arrivals waited for: [barIn, barVO, barDQ]
@@ -435,17 +440,25 @@ constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
 }  // namespace rsw
 
 struct RevParams {
-    const float *dhT, *rs;
+    const float *dhT;
+    float *rs;           // rowsum(dhT * hT) from the forward sweep; exact-route workspace (saved mode)
     float *dh0;
-    const int *flags;
+    const int *flags;    // [B*H] 1: the (b,h) takes the exact route
     int T, H, ntiles;
+    // saved-state mode
+    const float *hTs;    // [B*H][128][128] final state saved by the forward
+    const float *h0;
+    const __nv_bfloat16 *q, *lf, *x, *dO;   // for the exact route
+    __nv_bfloat16 *dq, *dlf, *dx;
+    int simt_chunk;
 };
 
+template <bool kSaved>
 __global__ void __launch_bounds__(rsw::kRevThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
            const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_di,
-           const __grid_constant__ CUtensorMap tm_dlf, RevParams p) {
+           const __grid_constant__ CUtensorMap tm_dlf, const __grid_constant__ CUtensorMap tm_st, RevParams p) {
     using namespace rsw;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *Qb = smem, *Gb = smem + kTileBytes, *Vb = smem + 2 * kTileBytes, *Ob = smem + 3 * kTileBytes;
@@ -455,7 +468,18 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / p.H, h = bh - b * p.H;
     const int N = p.ntiles;
-    if (p.flags[bh] != 0) return;   // this (b,h) takes the exact route
+    if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
+        if (kSaved) {         // both sweeps here (recompute mode: in the forward-sweep kernel)
+            float *sm = reinterpret_cast<float *>(smem);
+            simt_bwd_dq_body<__nv_bfloat16>(p.lf, p.x, p.h0, p.dO, p.dhT, p.dq, p.rs, p.T, p.H, 128, 128,
+                                            p.simt_chunk, sm, bh);
+            __syncthreads();
+            simt_bwd_rev_body<__nv_bfloat16>(p.q, p.lf, p.x, p.dO, p.dhT, p.dq, p.rs, p.dlf, p.dx, p.dh0, p.T,
+                                             p.H, 128, 128, p.simt_chunk, sm, bh);
+            if (tid == 0) atomicAdd(&g_counters[0], 1ull);
+        }
+        return;
+    }
     if (smem_u32(smem) & 1023u) {
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
@@ -469,6 +493,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->barDQ, 1);
         mbar_init(&m->barP1, 1);
         mbar_init(&m->barP2, 1);
+        mbar_init(&m->barP3, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -499,6 +524,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
         float v[32];
+        float part = 0.0f;   // saved mode: this quarter's share of rowsum(dhT * hT)
         if (p.dhT) {
             const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * 128 + j) * 128 + c0);
 #pragma unroll
@@ -506,18 +532,34 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const float4 a = src[i];
                 v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
             }
+            if (kSaved) {
+                const float4 *hs = reinterpret_cast<const float4 *>(p.hTs + ((size_t)bh * 128 + j) * 128 + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 a = hs[i];
+                    part += v[4 * i] * a.x + v[4 * i + 1] * a.y + v[4 * i + 2] * a.z + v[4 * i + 3] * a.w;
+                }
+            }
         } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.0f;
         }
         tmem_st32(tl + kColDS + c0, v);
         tmem_wait_st();
-        if (q4 == 0) m->carry[j] = (p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
+        if (kSaved) {
+            if (q4 < 3) m->Bpart[q4][j] = part;
+            else m->EB[j] = part;
+            __syncthreads();
+            if (q4 == 0) m->carry[j] = m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
+        } else if (q4 == 0) {
+            m->carry[j] = (p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
+        }
     }
 
     const uint32_t id_kk = idesc_bf16(128, 128, false, false);
     const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
     const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+    const uint32_t id_mnk = idesc_bf16(128, 128, true, false);
     const uint32_t cblk = (uint32_t)(j >> 6) * kBlk, cch = (uint32_t)((j & 63) >> 3), cin = (uint32_t)(j & 7) * 2;
     auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
     auto bfat = [&](const uint8_t *tile, int t) -> float {
@@ -529,9 +571,10 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const uint32_t par = it & 1;
         if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
         if (tid == 0) waited[0] = it + 1;
-        if (tid == 0) {   // warm L2: this chunk's dq, the next chunk's inputs
+        if (tid == 0) {   // warm L2: this chunk's dq (or saved state), the next chunk's inputs
             for (int c = 0; c < 2; ++c) {
-                tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
+                if (kSaved) tma_prefetch_l2_4d(&tm_st, 64 * c, 0, 0, bh * N + n);
+                else tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
                 if (n > 0) {
                     tma_prefetch_l2_4d(&tm_q, 64 * c, h, (n - 1) * kTile, b);
                     tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (n - 1) * kTile, b);
@@ -683,12 +726,16 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (__syncthreads_or(!mbar_wait(&m->barP2, par))) { ok = false; break; }
         tc_fence_after();
         if (tid == 0) {
-            // dq of this chunk into D16; v and dO of the next chunk into Vb, Ob
             ++issued[2];
             mbar_arrive_expect_tx(&m->barDQ, kTileBytes);
-            tma_load_4d(D16, &tm_dq, &m->barDQ, 0, h, n * kTile, b);
-            tma_load_4d(D16 + kBlk, &tm_dq, &m->barDQ, 64, h, n * kTile, b);
-            if (n > 0) issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
+            if (kSaved) {   // the saved bf16 state entering this chunk into D16
+                tma_load_4d(D16, &tm_st, &m->barDQ, 0, 0, 0, bh * N + n);
+                tma_load_4d(D16 + kBlk, &tm_st, &m->barDQ, 64, 0, 0, bh * N + n);
+            } else {        // dq of this chunk into D16; v and dO of the next chunk into Vb, Ob
+                tma_load_4d(D16, &tm_dq, &m->barDQ, 0, h, n * kTile, b);
+                tma_load_4d(D16 + kBlk, &tm_dq, &m->barDQ, 64, h, n * kTile, b);
+                if (n > 0) issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
+            }
         }
         // ---- di (lane s) -> AT (rows s) for the TMA store
         {
@@ -708,10 +755,39 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             qk[i] = (uint32_t)*reinterpret_cast<const uint16_t *>(Qb + off) |
                     ((uint32_t)*reinterpret_cast<const uint16_t *>(Gb + off) << 16);
         }
-        __syncthreads();
-        if (tid == 0 && n > 0) issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, n - 1);
-        if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
-        if (tid == 0) waited[2] = it + 1;
+        if (kSaved) {
+            // phase 3 once di has left X1: dq_pre^T = S_in dO^T + Kt^T mask(dA)^T   (M = j, N = t)
+            tc_fence_before();
+            if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
+            if (tid == 0) {
+                waited[2] = it + 1;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
+                                sdesc_sw128(smem_u32(Ob) + ko, 16, 1024), id_kk, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                    mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + kk * 2048, kBlk, 1024),
+                                sdesc_sw128(smem_u32(DA) + ko, 16, 1024), id_mnk, true);
+                }
+                mma_commit(&m->barP3);
+            }
+            if (__syncthreads_or(!mbar_wait(&m->barP3, par))) { ok = false; break; }
+            tc_fence_after();
+            if (tid == 0 && n > 0) {   // every operand tile of this chunk has been read
+                issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
+                issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, n - 1);
+            }
+        } else {
+            __syncthreads();
+            if (tid == 0 && n > 0) issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, n - 1);
+            if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
+            if (tid == 0) waited[2] = it + 1;
+        }
         float suf = 0.0f;
 #pragma unroll
         for (int hh = 1; hh >= 0; --hh) {
@@ -719,15 +795,21 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const int col = c0 + 16 * hh;
             tmem_ld16(tl + kColX2 + col, dkp);
             tmem_ld16(tl + kColE + col, e);
+            if (kSaved) tmem_ld16(tl + kColX1 + col, dap);   // dq_pre of these tokens
             const float eprev = col > 0 ? tmem_ld1(tl + kColE + col - 1) : 1.0f;
             tmem_wait_ld();
             float invE = __fdividef(1.0f, e[15]);
 #pragma unroll
             for (int i = 15; i >= 0; --i) {
                 const int t = col + i;
-                const float qt = bf_lo(qk[16 * hh + i]), kt = bf_hi(qk[16 * hh + i]), dq = bfat(D16, t);
+                const float qt = bf_lo(qk[16 * hh + i]), kt = bf_hi(qk[16 * hh + i]);
                 const float invEm1 = __fdividef(1.0f, i > 0 ? e[i - 1] : eprev);
-                suf += qt * invE * dq - kt * dkp[i];
+                if (kSaved) {   // dq = E dq_pre into D16 (row t); q dq = Qt dq_pre
+                    *reinterpret_cast<__nv_bfloat16 *>(D16 + eoff(t)) = __float2bfloat16_rn(e[i] * dap[i]);
+                    suf += qt * dap[i] - kt * dkp[i];
+                } else {
+                    suf += qt * invE * bfat(D16, t) - kt * dkp[i];
+                }
                 dap[i] = suf - dkp[i] * invEm1;
                 invE = invEm1;
             }
@@ -758,6 +840,10 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tma_store_4d(&tm_di, AT + kBlk, 64, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA + kBlk, 64, h, n * kTile, b);
+            if (kSaved) {
+                tma_store_4d(&tm_dq, D16, 0, h, n * kTile, b);
+                tma_store_4d(&tm_dq, D16 + kBlk, 64, h, n * kTile, b);
+            }
             tma_store_commit();
         }
     }
@@ -792,18 +878,37 @@ static_assert(tcb::rsw::kSmemBytes <= 227 * 1024, "reverse-sweep shared memory")
 size_t tc_bwd_smem() { return tcb::fsw::kSmemBytes > tcb::rsw::kSmemBytes ? tcb::fsw::kSmemBytes : tcb::rsw::kSmemBytes; }
 
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
-    CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl;
+    const bool saved = a.st16 != nullptr;
+    const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
+    CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl, mst;
     if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
         !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mdo, a.dO, a.B, a.T, a.H) ||
         !make_token_map(&mdq, a.dq, a.B, a.T, a.H) || !make_token_map(&mdi, a.dx, a.B, a.T, a.H) ||
         !make_token_map(&mdl, a.dlf, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tcb::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tcb::fsw::kSmemBytes);
+    // saved states [B*H*ntiles][128][128] bf16, addressed as 128-row "token" tiles
+    if (saved && !make_token_map(&mst, a.st16, a.B * a.H * ntiles, 128, 1)) return cudaErrorInvalidValue;
+    if (!saved) mst = mq;   // unused
+    tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles, a.hTs, a.h0,
+                      (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
+                      (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
+                      (__nv_bfloat16 *)a.dx, a.simt_C};
+    cudaError_t e;
+    if (saved) {
+        // one launch; the exact route of a flagged (b,h) runs in the same shared memory
+        size_t smem = tcb::rsw::kSmemBytes;
+        if (simt_bwd_dq_smem(a.simt_C, 128, 128) > smem) smem = simt_bwd_dq_smem(a.simt_C, 128, 128);
+        if (simt_bwd_rev_smem(a.simt_C, 128, 128) > smem) smem = simt_bwd_rev_smem(a.simt_C, 128, 128);
+        e = cudaFuncSetAttribute(tcb::rev_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        tcb::rev_kernel<true><<<a.B * a.H, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);
+        return cudaGetLastError();
+    }
+    e = cudaFuncSetAttribute(tcb::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcb::fsw::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tcb::rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcb::rsw::kSmemBytes);
+    e = cudaFuncSetAttribute(tcb::rev_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tcb::rsw::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     tcb::DqParams p1{a.h0, a.dhT, a.rs, a.flags, a.T, a.H, ntiles,
                      (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                      (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
@@ -811,8 +916,8 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     tcb::dq_kernel<<<a.B * a.H, tcb::fsw::kDqThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles};
-    tcb::rev_kernel<<<a.B * a.H, tcb::rsw::kRevThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, p2);
+    tcb::rev_kernel<false><<<a.B * a.H, tcb::rsw::kRevThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi,
+                                                                                           mdl, mst, p2);
     return cudaGetLastError();
 }
 

@@ -12,6 +12,10 @@
 //   O  = Qt bf16(S_in) + bf16(A) V                             tcgen05, fp32 in TMEM
 //   S' = S_in + Kt^T V,   S_out = Diag(E_B) S'                 fp32 state in TMEM
 //
+// For training, the forward can also keep what the backward needs: bf16(S_in) of every
+// chunk (the operand it builds anyway for the inter-chunk MMA, written out by a TMA store)
+// and the fp32 final state.
+//
 // The state is post-scaled: the MMA accumulates Kt^T V onto S_in, and the next
 // chunk multiplies the rows by this chunk's E_B before using it (the products
 // Kt * E_B = k * E_B / E <= k are never formed in bf16 at all).  Qt Kt^T realises
@@ -70,11 +74,14 @@ struct Params {
     const float *Sin; // [B*H][nseg-1][128][128] state entering segments 1.. (from the scan)
     int T, H, ntiles;
     int nseg, tps;    // sequence segments per (b,h) and chunks per segment
+    bool save;        // store bf16(S_in) of every chunk through tm_st
+    float *hTs;       // with save: the final state [B*H][128][128]
 };
 
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
-           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o, Params p) {
+           const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o,
+           const __grid_constant__ CUtensorMap tm_st, Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *Qb[2] = {smem, smem + 3 * kTileBytes};
     uint8_t *Gb[2] = {smem + kTileBytes, smem + 4 * kTileBytes};
@@ -248,9 +255,23 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->sdone);
-            // causal mask of A, bf16 -> X (A operand) once the inter-chunk MMA has read X
+            if (p.save) {   // bf16(S_in) of this chunk, kept for the backward
+                named_bar_sync(2, 128);
+                if (r == 0) {
+                    const int slot = bh * p.ntiles + g0 + n;
+                    tma_store_4d(&tm_st, X, 0, 0, 0, slot);
+                    tma_store_4d(&tm_st, X + kBlk, 64, 0, 0, slot);
+                    tma_store_commit();
+                }
+            }
+            // causal mask of A, bf16 -> X (A operand) once the inter-chunk MMA (and the state
+            // store) have read X
             if (!mbar_wait(&m->barA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (!mbar_wait(&m->barO1, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (p.save) {
+                if (r == 0) tma_store_wait_read0();
+                named_bar_sync(2, 128);
+            }
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -290,18 +311,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // the last state MMA must be complete before hT is read or TMEM is released
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        if (n == N && p.hT && seg == p.nseg - 1) {
+        if (n == N && (p.hT || p.hTs) && seg == p.nseg - 1) {
             const float e = e_cur;
-            float *dst = p.hT + ((size_t)bh * 128 + r) * 128;
+            float *dst = p.hT ? p.hT + ((size_t)bh * 128 + r) * 128 : nullptr;
+            float *dsv = p.hTs ? p.hTs + ((size_t)bh * 128 + r) * 128 : nullptr;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
                 tmem_ld32(tl + kColS + 32 * c, v);
                 tmem_wait_ld();
-                float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * c);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    d4[i] = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
+                for (int i = 0; i < 8; ++i) {
+                    const float4 w = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
+                    if (dst) reinterpret_cast<float4 *>(dst + 32 * c)[i] = w;
+                    if (dsv) reinterpret_cast<float4 *>(dsv + 32 * c)[i] = w;
+                }
             }
         }
     } else if (warp >= 8) {
@@ -623,10 +647,14 @@ size_t tc_fwd_workspace(int B, int T, int H) {
 size_t tc_fwd_smem() { return tcf::kSmemBytes; }
 
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
-    CUtensorMap mq, ml, mx, mo;
+    CUtensorMap mq, ml, mx, mo, mst;
     if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
         !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mo, a.o, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
+    // saved states [B*H*ntiles][128][128] bf16, addressed as 128-row "token" tiles
+    const int ntiles_all = (a.T + tcc::kTile - 1) / tcc::kTile;
+    if (a.st16 && !make_token_map(&mst, a.st16, a.B * a.H * ntiles_all, 128, 1)) return cudaErrorInvalidValue;
+    if (!a.st16) mst = mo;   // unused
     cudaError_t e = cudaFuncSetAttribute(tcf::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcf::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -645,8 +673,9 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
-                  (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps};
-    tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, p);
+                  (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps,
+                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr};
+    tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     return cudaGetLastError();
 }
 

@@ -89,3 +89,28 @@ def test_product_path_does_not_import_the_oracle():
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, fn
                 assert "liboracle" not in txt, fn
+
+
+def test_saved_size_and_training_pair_argument_checks(lib):
+    bad = ctypes.c_size_t(-1).value
+    f = lib.hgrn2_saved_size
+    # bf16, d = 128: per (b,h) ceil(T/128) bf16 chunk states, one fp32 final state, one flag
+    B, T, H = 2, 300, 3
+    nt = (T + 127) // 128
+    up = lambda x: (x + 255) // 256 * 256
+    want = up(B * H * nt * 128 * 128 * 2) + up(B * H * 128 * 128 * 4) + up(B * H * 4)
+    assert f(B, T, H, 128, 128, L.BF16) == want
+    assert f(B, T, H, 64, 64, L.BF16) == 0        # exact route: nothing saved
+    assert f(B, T, H, 128, 128, L.FP32) == 0
+    assert f(B, 0, H, 128, 128, L.BF16) == 0
+    assert f(0, T, H, 128, 128, L.BF16) == bad
+    vp = ctypes.c_void_p
+    # a saved buffer shorter than hgrn2_saved_size is rejected before any launch
+    st = lib.hgrn2_fwd_train(vp(16), vp(16), vp(16), None, vp(16), None, vp(256), want - 1,
+                             B, T, H, 128, 128, 64, L.BF16, vp(256), 1 << 30, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_bwd_saved(vp(16), vp(16), vp(16), None, None, 0, vp(16), None, vp(16), vp(16), vp(16),
+                             None, B, T, H, 128, 128, 64, L.BF16, vp(256), 1 << 30, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_bwd_saved(*([None] * 5), 0, *([None] * 6), 1, 8, 1, 16, 16, 16, 1, None, 0, None)
+    assert st == L.ERR_INVALID_ARG       # null inputs (exact route: the buffer is not needed)

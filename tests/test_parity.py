@@ -79,16 +79,20 @@ BF16_CASES = [
 ]
 
 
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
 @pytest.mark.parametrize("case", BF16_CASES)
-def test_bf16_fwd_bwd(cuda, case):
+def test_bf16_fwd_bwd(cuda, case, saved):
     B, T, H, lb, chunk, with_h0, with_dhT = case
     inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, lb, seed=100 + T,
                         h0_sigma=0.1 if with_h0 else 0.0, with_dO=True,
                         dhT_sigma=0.1 if with_dhT else 0.0)
     g = to_cuda(inp)
     h0, dhT = g.get("h0"), g.get("dhT")
-    o, hT = L.fwd(g["q"], g["log_f"], g["i"], h0, want_hT=True, chunk=chunk)
-    dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], h0, dhT, want_dh0=True, chunk=chunk)
+    sv = L.new_saved(g["q"]) if saved else None
+    assert (sv is not None) == saved
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], h0, want_hT=True, chunk=chunk, saved=sv)
+    dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], h0, dhT, want_dh0=True, chunk=chunk,
+                             saved=sv)
     ref = oracle_heads(inp, _all_pairs(B, H), want_bwd=True, dhT=inp.get("dhT"))
     for n, (b, h) in enumerate(_all_pairs(B, H)):
         for name, got in (("o", o[b, :, h]), ("hT", hT[b, h]), ("dq", dq[b, :, h]),
@@ -114,12 +118,15 @@ def test_workload_fwd_layer_full_size(cuda):
     _check_fwd(inp, o, None, _sample_pairs(w.B, w.H, 4, 1), w.dtype)
 
 
-def test_workload_train_full_size_fwd_bwd(cuda):
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_workload_train_full_size_fwd_bwd(cuda, saved):
+    # saved=True is the pair the benchmark times: hgrn2_fwd_train + hgrn2_bwd_saved
     w = I.TRAIN
     inp = I.make_workload(w, seed=1003)
     g = to_cuda(inp)
-    o, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=w.chunk)
-    dq, dlf, di, _ = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=w.chunk)
+    sv = L.new_saved(g["q"]) if saved else None
+    o, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=w.chunk, saved=sv)
+    dq, dlf, di, _ = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=w.chunk, saved=sv)
     torch.cuda.synchronize()
     pairs = _sample_pairs(w.B, w.H, 3, 2)
     ref = oracle_heads(inp, pairs, want_bwd=True)
@@ -191,15 +198,68 @@ def test_gate_zero_keeps_last_input(cuda, dtype):
     assert np.max(np.abs(np64(dlf) - r[1])) <= tol(dtype) * scale
 
 
-def test_reports_exact_route_is_finite_for_strong_decay(cuda):
-    # lb = 0 at chunk 128: cumulative log-decay spans of ~-100 inside a chunk
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_reports_exact_route_is_finite_for_strong_decay(cuda, saved):
+    # lb = 0 at chunk 128: cumulative log-decay spans of ~-100 inside a chunk (B*H = 2: the
+    # forward runs in sequence segments, then the exact route for the flagged pairs)
     inp = I.make_inputs(1, 384, 2, 128, 128, torch.bfloat16, 0.0, seed=5, with_dO=True)
     g = to_cuda(inp)
-    o, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=128)
-    dq, dlf, di, _ = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=128)
+    sv = L.new_saved(g["q"]) if saved else None
+    o, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=128, saved=sv)
+    dq, dlf, di, _ = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=128, saved=sv)
     ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True)
     for n, h in enumerate((0, 1)):
         for name, got in (("o", o[0, :, h]), ("dq", dq[0, :, h]), ("dlog_f", dlf[0, :, h]),
                           ("di", di[0, :, h])):
             assert np.isfinite(np64(got)).all()
             assert err(np64(got), ref[name][n], torch.bfloat16) <= 2e-2, name
+
+
+def test_saved_pair_launch_counts_and_mixed_routes(cuda):
+    # B*H = 80 > 148 / 2: one CTA per (b,h), no sequence segments.  Head 3 of batch 1 gets a
+    # strong decay (exact route), every other pair stays on the tensor cores; the saved
+    # backward is one launch and computes both kinds of pair.
+    B, T, H = 10, 600, 8
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.9, seed=77, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    strong = I.make_inputs(1, T, 1, 128, 128, torch.bfloat16, 0.0, seed=78)
+    inp["log_f"][1, :, 3] = strong["log_f"][0, :, 0]
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"])
+    L.counters(reset=True)
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    c_fwd = L.counters(reset=True)
+    dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
+                             saved=sv)
+    c_bwd = L.counters(reset=True)
+    assert c_fwd[2] == 1 and c_bwd[2] == 1, (c_fwd, c_bwd)
+    assert c_fwd[0] == 1 and c_bwd[0] == 1, (c_fwd, c_bwd)   # one exact-route pair in each pass
+    assert L.device_status() == L.OK
+    pairs = [(1, 3), (0, 0), (1, 7)]
+    ref = oracle_heads(inp, pairs, want_bwd=True, dhT=inp["dhT"])
+    for n, (b, h) in enumerate(pairs):
+        for name, got in (("o", o[b, :, h]), ("hT", hT[b, h]), ("dq", dq[b, :, h]),
+                          ("dlog_f", dlf[b, :, h]), ("di", di[b, :, h]), ("dh0", dh0[b, h])):
+            e = err(np64(got), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, b, h, e)
+
+
+def test_autograd_function_uses_saved_states(cuda):
+    B, T, H = 1, 260, 2
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.95, seed=9, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    g = to_cuda(inp)
+    q, lf, x = (g[k].clone().requires_grad_(True) for k in ("q", "log_f", "i"))
+    h0 = g["h0"].clone().requires_grad_(True)
+    L.counters(reset=True)
+    o, hT = L.hgrn2(q, lf, x, h0, chunk=64)
+    loss = (o.float() * g["dO"].float()).sum() + (hT * g["dhT"]).sum()
+    loss.backward()
+    c = L.counters(reset=True)
+    assert c[2] == 4 + 1, c   # segmented forward (4 launches) + one saved backward launch
+    ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True, dhT=inp["dhT"])
+    for n, h in enumerate((0, 1)):
+        for name, got in (("dq", q.grad[0, :, h]), ("dlog_f", lf.grad[0, :, h]), ("di", x.grad[0, :, h]),
+                          ("dh0", h0.grad[0, h])):
+            e = err(np64(got), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, h, e)
