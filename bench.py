@@ -191,34 +191,58 @@ def run_ours(args, world, rank, local):
         L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f, saved=sv)
         return L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b, saved=sv)
 
+    def fwd_call():
+        L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f, saved=sv)
+
+    def bwd_call():
+        L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b, saved=sv)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # estimate the step time, to keep the GPU busy for ~50 ms before the timed region
+    w0 = time.perf_counter()
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n_spin = max(1, int(0.05 / max((time.perf_counter() - w0) / 3, 1e-6)))
     stream = torch.cuda.current_stream()
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    L.counters(reset=True)
-    barrier(world)
-    torch.cuda.synchronize()
+    gate = 2_000_000   # cycles of a device-side sleep that holds the queue while the host fills it
     with ClockSampler(local) as clk:
-        time.sleep(0.3)
+        time.sleep(0.1)              # nvidia-smi starting up
+        for _ in range(n_spin):      # clocks back up after that idle period
+            step()
+        launches0 = L.counters()[2]  # synchronises
+        barrier(world)
+        torch.cuda.synchronize()
+        # timed region: only the two bracketing events, so nothing but the calls runs between
+        # them; the sleep ahead of t0 lets the host queue the K steps before the GPU reaches them
+        torch.cuda._sleep(gate)
         t0.record(stream)
-        for k in range(K):
-            evs[k][0].record(stream)
-            L.fwd(q, lf, x, chunk=chunk, out=o, workspace=ws_f, saved=sv)
-            evs[k][1].record(stream)
-            L.bwd(q, lf, x, dO, chunk=chunk, workspace=ws_b, saved=sv)
-            evs[k][2].record(stream)
+        for _ in range(K):
+            step()
         t1.record(stream)
         torch.cuda.synchronize()
-    barrier(world)
-    launches = L.counters()[2]
+        barrier(world)
+        launches = L.counters()[2] - launches0
+        # per-call durations, same data and clocks: K forward calls, then K backward calls
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        torch.cuda._sleep(gate)
+        ev[0].record(stream)
+        for _ in range(K):
+            fwd_call()
+        ev[1].record(stream)
+        for _ in range(K):
+            bwd_call()
+        ev[2].record(stream)
+        torch.cuda.synchronize()
     ms_local = t0.elapsed_time(t1)
     ms = max_over_ranks(ms_local, world)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    fwd_ms = ev[0].elapsed_time(ev[1]) / K
+    bwd_ms = ev[1].elapsed_time(ev[2]) / K
     ms_per_step = ms / K
     tokens_per_step = B * T
     value = world * tokens_per_step * K / (ms / 1e3)

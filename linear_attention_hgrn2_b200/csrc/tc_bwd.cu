@@ -343,7 +343,6 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
             }
             named_bar_sync(1, 256);   // rows 0..63 of log f are read before the first half overwrites them
             float bsum = half ? m->Bpart[j] : 0.0f;
-            float ip = __expf(-bsum);
             float ev[64];
 #pragma unroll
             for (int bt = 0; bt < 8; ++bt) {
@@ -357,9 +356,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
                 for (int i = 0; i < 8; ++i) {
                     bsum += av[i];
                     const float E = __expf(bsum), iE = __expf(-bsum);
-                    ok[i] = __float2bfloat16_rn(k_gate(av[i], E * ip) * iE);
+                    ok[i] = __float2bfloat16_rn((1.0f - __expf(av[i])) * iE);
                     ev[8 * bt + i] = E;
-                    ip = iE;
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) *reinterpret_cast<__nv_bfloat16 *>(Gb[s] + eoff(t0 + i)) = ok[i];
@@ -583,7 +581,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
             }
         }
-        // ---- prep: column j, rows c0 .. c0+31: Qt = q E, Kt = k / E in place; E -> TMEM
+        // ---- prep: column j, rows c0 .. c0+31: Qt = q E, Kt = k / E in place; E -> TMEM.
+        // f = e^a directly, so k = 1 - f has an absolute error of a few 1e-8; E is the running
+        // product of f from the range start, 1/E = e^{-b}.
         {
             float sum = 0.0f;
             if (q4 < 3) {
@@ -594,7 +594,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             __syncthreads();
             float bsum = 0.0f;
             for (int r2 = 0; r2 < q4; ++r2) bsum += m->Bpart[r2][j];
-            float ip = __expf(-bsum);
+            float E = __expf(bsum);
             float ev[32];
 #pragma unroll
             for (int bt = 0; bt < 4; ++bt) {
@@ -609,11 +609,11 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     bsum += av[i];
-                    const float E = __expf(bsum), iE = __expf(-bsum);
-                    ok2[i] = __float2bfloat16_rn(k_gate(av[i], E * ip) * iE);
+                    const float f = __expf(av[i]);
+                    E *= f;
+                    ok2[i] = __float2bfloat16_rn((1.0f - f) * __expf(-bsum));
                     oq[i] = __float2bfloat16_rn(qv[i] * E);
                     ev[8 * bt + i] = E;
-                    ip = iE;
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {

@@ -27,7 +27,9 @@
 // difference of cumulative sums.
 //
 // Warp roles (16 warps), coordinated by mbarriers only:
-//   warp 0      TMA producer: q, log f, i tiles (128-byte swizzle) into a 2-stage ring
+//   warp 0      TMA producer: q, log f, i tiles (128-byte swizzle) into a 2-stage ring; q and
+//               log f of a stage are refilled as soon as the state MMA has read Qt and Kt,
+//               i once the last MMA of the chunk has read it
 //   warp 1      TMEM allocator and the single MMA-issuing thread
 //   warps 4-7   TMEM warps (one thread per TMEM lane): S phase (bf16 copy of S_in,
 //               Diag(E_B) scale), causal mask of A, o epilogue (staged in smem, TMA store)
@@ -52,12 +54,14 @@ constexpr int kFwdThreads = 512;     // forward kernel: 16 warps
 constexpr uint32_t kColS = 0, kColO = 128, kColA = 256, kTmemCols = 512;
 
 struct __align__(8) Misc {
-    uint64_t full[2], prepped[2], empty[2];
+    uint64_t fullQG[2], fullV[2], prepped[2];   // stage s: q and log f / i landed; prep done
+    uint64_t emptyQG[2], emptyV[2];             // stage s: Qt, Kt / v read by every MMA of its chunk
     uint64_t barA, barO1, barS, barO2;      // MMA completions (tcgen05.commit)
     uint64_t sdone, adone, ofree;           // TMEM-warp arrivals (128 each)
     uint32_t tmem_base;
     int bad_tile;                           // first chunk whose decay span is too wide
-    int waited_full;                        // chunks whose arrival the prep warps consumed
+    int waited_full;                        // q / log f arrivals the prep warps consumed
+    int waited_v;                           // v arrivals the MMA thread consumed
     float EB[2][128];                       // E_B ring: read by the TMEM warps while that chunk is current
     float Ppart[3][128];                    // per 32-row range sums of log f (ranges 0..2)
 };
@@ -99,9 +103,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&m->full[s], 1);
+            mbar_init(&m->fullQG[s], 1);
+            mbar_init(&m->fullV[s], 1);
             mbar_init(&m->prepped[s], 256);
-            mbar_init(&m->empty[s], 1);
+            mbar_init(&m->emptyQG[s], 1);
+            mbar_init(&m->emptyV[s], 1);
         }
         mbar_init(&m->barA, 1);
         mbar_init(&m->barO1, 1);
@@ -112,6 +118,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->ofree, 128);
         m->bad_tile = INT_MAX;
         m->waited_full = 0;
+        m->waited_v = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_lf);
@@ -126,7 +133,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
-    int producer_issued = 0;
+    int issued_qg = 0, issued_v = 0;   // producer: loads issued per barrier pair
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -134,14 +141,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             for (int n = 0; n < N; ++n) {
                 const int s = n & 1;
                 if (ld_volatile(&m->bad_tile) < n) break;
-                if (n >= 2 && !wait_or_abort(&m->empty[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
-                mbar_arrive_expect_tx(&m->full[s], 3 * kTileBytes);
+                // q and log f once the state MMA of chunk n-2 has read Qt, Kt; i once its last
+                // MMA has read v
+                if (n >= 2 && !wait_or_abort(&m->emptyQG[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
+                mbar_arrive_expect_tx(&m->fullQG[s], 2 * kTileBytes);
                 for (int c = 0; c < 2; ++c) {
-                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
-                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
-                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->full[s], 64 * c, h, (g0 + n) * kTile, b);
+                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, h, (g0 + n) * kTile, b);
+                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, h, (g0 + n) * kTile, b);
                 }
-                ++producer_issued;
+                ++issued_qg;
+                if (n >= 2 && !wait_or_abort(&m->emptyV[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
+                mbar_arrive_expect_tx(&m->fullV[s], kTileBytes);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, h, (g0 + n) * kTile, b);
+                ++issued_v;
                 if (n + 2 < N)   // warm L2 for the chunk after next (its load waits for a free stage)
                     for (int c = 0; c < 2; ++c) {
                         tma_prefetch_l2_4d(&tm_q, 64 * c, h, (g0 + n + 2) * kTile, b);
@@ -181,11 +194,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(X) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
                 }
                 mma_commit(&m->barO1);
+                if (!mbar_wait(&m->fullV[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                m->waited_v = n + 1;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
                                 sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
                 mma_commit(&m->barS);
+                mma_commit(&m->emptyQG[s]);   // Qt and Kt of stage s are free once the MMAs above completed
                 // O += bf16(mask(A)) V once the TMEM warps wrote it
                 if (!mbar_wait(&m->adone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
                 tc_fence_after();
@@ -196,7 +213,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
                 }
                 mma_commit(&m->barO2);
-                mma_commit(&m->empty[s]);   // stage s is free once every MMA above completed
+                mma_commit(&m->emptyV[s]);   // v of stage s is free once every MMA above completed
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -331,16 +348,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     } else if (warp >= 8) {
         // ------------------------------------------------------------ prep warps
         // thread = one column pair (2 key dims, 4-byte smem accesses) and one 32-row range.
-        // The decay is formed from the running sum b of log f: E = exp(b), 1/E = exp(-b).
-        // Each range first sums its own rows; ranges exchange sums through shared memory.
-        // Rows go in batches of 8: all loads, then the arithmetic, then all stores.
+        // Each range first sums its own rows of log f; ranges exchange sums through shared
+        // memory.  Then f = e^a directly (so k = 1 - f has an absolute error of a few 1e-8),
+        // E = running product of f from the range start, 1/E = e^{-b} with b the running sum
+        // of log f.  Rows go in batches of 8: all loads, then the arithmetic, then all stores.
         const int ptid = tid - 256;
         const int pc = ptid & 63, rr = ptid >> 6, col0 = 2 * pc;
         const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
         auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
         for (int n = 0; n < N; ++n) {
             const int s = n & 1;
-            if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (!mbar_wait(&m->fullQG[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ptid == 0) m->waited_full = n + 1;
             if (rr < 3) {
                 float s0 = 0.0f, s1 = 0.0f;
@@ -359,7 +377,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 b0 += m->Ppart[r2][col0];
                 b1 += m->Ppart[r2][col0 + 1];
             }
-            float ip0 = __expf(-b0), ip1 = __expf(-b1);   // 1/E of the row before the range
+            float E0 = __expf(b0), E1 = __expf(b1);   // E of the row before the range
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
                 const int t0 = 32 * rr + 8 * bt;
@@ -374,12 +392,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     const float a0 = bf_lo(wa[i]), a1 = bf_hi(wa[i]);
                     b0 += a0;
                     b1 += a1;
-                    const float E0 = __expf(b0), E1 = __expf(b1), iE0 = __expf(-b0), iE1 = __expf(-b1);
-                    const float k0 = k_gate(a0, E0 * ip0), k1 = k_gate(a1, E1 * ip1);
+                    const float f0 = __expf(a0), f1 = __expf(a1);
+                    E0 *= f0;
+                    E1 *= f1;
                     wq[i] = pack_bf2(bf_lo(wq[i]) * E0, bf_hi(wq[i]) * E1);
-                    wa[i] = pack_bf2(k0 * iE0, k1 * iE1);
-                    ip0 = iE0;
-                    ip1 = iE1;
+                    wa[i] = pack_bf2((1.0f - f0) * __expf(-b0), (1.0f - f1) * __expf(-b1));
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -405,7 +422,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int bad = m->bad_tile;
     const bool fell_back = bad < N;
     if (warp == 0 && lane == 0)   // drain loads still landing in this CTA's shared memory
-        for (int k = m->waited_full; k < producer_issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
+    {
+        for (int k = m->waited_full; k < issued_qg; ++k) mbar_wait(&m->fullQG[k & 1], (k >> 1) & 1, 2000000u);
+        for (int k = m->waited_v; k < issued_v; ++k) mbar_wait(&m->fullV[k & 1], (k >> 1) & 1, 2000000u);
+    }
     if (tid == 0) {
         if (p.nseg == 1) p.flags[bh] = fell_back ? 1 : 0;   // sole writer
         else if (fell_back) p.flags[bh] = 1;                  // zeroed by the aggregate kernel
