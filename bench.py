@@ -291,37 +291,76 @@ def run_ours(args, world, rank, local):
 
 
 def run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, sv, w, world):
-    """Same step through host buffers: pinned H2D of the inputs and D2H of all outputs inside the timed region."""
+    """Same step through host buffers: every step's inputs go host -> device from pinned memory and
+    all its outputs (o, dq, d log f, di) come back device -> host, inside the timed region.
+
+    The copies are pipelined as a training input pipeline would be: the upload of step k+1 (one
+    stream), the compute of step k (the current stream) and the download of step k-1 (a third
+    stream) overlap, with two device buffer sets.  The timed region includes the pipeline's fill
+    (the first upload) and drain (the last download)."""
     import linear_attention_hgrn2_b200 as L
-    hq, hlf, hx, hdO = (t.cpu().pin_memory() for t in (q, lf, x, dO))
-    ho, hdq, hdlf, hdi = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, q, q, x))
-    dq_buf = torch.empty_like(q)
-    K = max(1, min(args.steps, 5))
+    hin = [t.cpu().pin_memory() for t in (q, lf, x, dO)]
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, q, q, x)]
+    din = [[q, lf, x, dO], [torch.empty_like(t) for t in (q, lf, x, dO)]]
+    dout_o = [o, torch.empty_like(o)]
+    K = max(3, min(args.steps, 8))
+    comp = torch.cuda.current_stream()
+    s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    up_done, comp_done, down_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    first = [True, True]
 
-    def one():
-        q.copy_(hq, non_blocking=True); lf.copy_(hlf, non_blocking=True)
-        x.copy_(hx, non_blocking=True); dO.copy_(hdO, non_blocking=True)
-        L.fwd(q, lf, x, chunk=w.chunk, out=o, workspace=ws_f, saved=sv)
-        dq, dlf, di, _ = L.bwd(q, lf, x, dO, chunk=w.chunk, workspace=ws_b, saved=sv)
-        ho.copy_(o, non_blocking=True); hdq.copy_(dq, non_blocking=True)
-        hdlf.copy_(dlf, non_blocking=True); hdi.copy_(di, non_blocking=True)
+    def upload(k):
+        sl = k % 2
+        with torch.cuda.stream(s_up):
+            if not first[sl]:
+                s_up.wait_event(comp_done[sl])      # step k-2 has finished reading this buffer set
+            for d, h in zip(din[sl], hin):
+                d.copy_(h, non_blocking=True)
+            up_done[sl].record(s_up)
 
-    one()
+    def compute_and_download(k):
+        sl = k % 2
+        comp.wait_event(up_done[sl])
+        if not first[sl]:
+            comp.wait_event(down_done[sl])          # step k-2's outputs have left this buffer set
+        qq, ll, xx, dd = din[sl]
+        L.fwd(qq, ll, xx, chunk=w.chunk, out=dout_o[sl], workspace=ws_f, saved=sv)
+        dq, dlf, di, _ = L.bwd(qq, ll, xx, dd, chunk=w.chunk, workspace=ws_b, saved=sv)
+        comp_done[sl].record(comp)
+        first[sl] = False
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(comp_done[sl])
+            for h, d in zip(hout, (dout_o[sl], dq, dlf, di)):
+                d.record_stream(s_down)
+                h.copy_(d, non_blocking=True)
+            down_done[sl].record(s_down)
+
+    def run(nsteps):
+        upload(0)
+        for k in range(nsteps):
+            if k + 1 < nsteps:
+                upload(k + 1)
+            compute_and_download(k)
+        comp.wait_stream(s_down)
+
+    run(2)
     torch.cuda.synchronize()
     barrier(world)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(K):
-        one()
-    b.record()
+    a.record(comp)
+    s_up.wait_event(a)
+    run(K)
+    b.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hlf, hx, hdO))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdlf, hdi))
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
     return {"value": round(world * w.B * w.T * K / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
-            "ms_per_step": round(ms / K, 3)}
+            "ms_per_step": round(ms / K, 3),
+            "pipeline": "upload k+1 | compute k | download k-1 on three streams; fill and drain timed"}
 
 
 def run_decode(args, dev, pk):
