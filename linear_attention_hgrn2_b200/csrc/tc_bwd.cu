@@ -427,6 +427,7 @@ constexpr int kRevThreads = 512;
 
 struct __align__(8) Misc {
     uint64_t barIn, barVO, barDQ, barP1, barP2, barP3;   // barDQ: dq (recompute) or S_in (saved)
+    uint64_t barDS;                                      // all 512 threads wrote dSh into TMEM
     uint32_t tmem_base;
     int pad;
     int issued[3], waited[3];   // loads issued / arrivals waited for: [barIn, barVO, barDQ]
@@ -492,6 +493,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->barP1, 1);
         mbar_init(&m->barP2, 1);
         mbar_init(&m->barP3, 1);
+        mbar_init(&m->barDS, kRevThreads);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -665,23 +667,50 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             store_chunk_bf16(D16, j, q4, v);
             tmem_st32(tl + kColDS + c0, v);
             tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&m->barDS);
+        }
+        if (tid == 0) {   // the recurrence step, issued as soon as dSh is in TMEM: dS = dSh + Qt^T dO
+            if (!mbar_wait(&m->barDS, par)) ok = false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ss(tbase + kColDS, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_mnmn, true);
+            }
         }
         // ---- masks: A^T keeps t >= s (lane s), dA keeps s <= t (lane t)
         {
             if (!mbar_wait(&m->barP1, par)) ok = false;
             tc_fence_after();
+            // this thread's 32 columns are all kept (q4 > quad), all dropped (q4 < quad) or the
+            // diagonal block (q4 == quad, compare per element); the branch is warp-uniform
             float v[32];
-            tmem_ld32(tl + kColX1 + c0, v);
-            tmem_wait_ld();
+            if (q4 >= quad) {
+                tmem_ld32(tl + kColX1 + c0, v);
+                tmem_wait_ld();
+                if (q4 == quad) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (c0 + i < j) v[i] = 0.0f;
+                    for (int i = 0; i < 32; ++i)
+                        if (i < lane) v[i] = 0.0f;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            }
             store_chunk_bf16(AT, j, q4, v);
-            tmem_ld32(tl + kColX2 + c0, v);
-            tmem_wait_ld();
+            if (q4 <= quad) {
+                tmem_ld32(tl + kColX2 + c0, v);
+                tmem_wait_ld();
+                if (q4 == quad) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (c0 + i > j) v[i] = 0.0f;
+                    for (int i = 0; i < 32; ++i)
+                        if (i > lane) v[i] = 0.0f;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            }
             store_chunk_bf16(DA, j, q4, v);
         }
         fence_proxy_async_smem();
@@ -715,13 +744,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
                             sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, true);
             }
-            // dS = dSh + Qt^T dO                    (M = j, N = v)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + kColDS, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_mnmn, true);
-            }
-            mma_commit(&m->barP2);
+            mma_commit(&m->barP2);   // also covers the recurrence step issued after the dS phase
         }
         if (__syncthreads_or(!mbar_wait(&m->barP2, par))) { ok = false; break; }
         tc_fence_after();

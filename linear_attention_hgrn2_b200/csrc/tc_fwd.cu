@@ -290,14 +290,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 named_bar_sync(2, 128);
             }
             tc_fence_after();
+            // column block c is kept (c < quad), dropped (c > quad) or diagonal (per element)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
-                tmem_ld32(tl + kColA + 32 * c, v);
-                tmem_wait_ld();
+                if (c <= quad) {
+                    tmem_ld32(tl + kColA + 32 * c, v);
+                    tmem_wait_ld();
+                    if (c == quad) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (32 * c + i > r) v[i] = 0.0f;
+                        for (int i = 0; i < 32; ++i)
+                            if (i > lane) v[i] = 0.0f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                }
                 store_chunk_bf16(X, r, c, v);
             }
             fence_proxy_async_smem();
