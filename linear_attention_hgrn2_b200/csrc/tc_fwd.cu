@@ -32,7 +32,8 @@
 //               i once the last MMA of the chunk has read it
 //   warp 1      TMEM allocator and the single MMA-issuing thread
 //   warps 4-7   TMEM warps (one thread per TMEM lane): S phase (bf16 copy of S_in,
-//               Diag(E_B) scale), causal mask of A, o epilogue (staged in smem, TMA store)
+//               Diag(E_B) scale), causal mask of A (bf16 pairs back into TMEM: the intra
+//               MMA reads its A operand from TMEM), o epilogue (staged in smem, TMA store)
 //   warps 8-15  prep warps: f, E, k, Qt, Kt for the next chunk while the current one
 //               is on the tensor cores
 // Every wait is bounded; a wait that gives up records HGRN2_ERR_TIMEOUT.
@@ -51,7 +52,7 @@ using namespace tcc;
 
 constexpr int kThreads = 256;        // aggregate kernel
 constexpr int kFwdThreads = 512;     // forward kernel: 16 warps
-constexpr uint32_t kColS = 0, kColO = 128, kColA = 256, kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 128, kColA = 256, kColP = 384, kTmemCols = 512;   // P: bf16 mask(A)
 
 struct __align__(8) Misc {
     uint64_t fullQG[2], fullV[2], prepped[2];   // stage s: q and log f / i landed; prep done
@@ -203,15 +204,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
                 mma_commit(&m->barS);
                 mma_commit(&m->emptyQG[s]);   // Qt and Kt of stage s are free once the MMAs above completed
-                // O += bf16(mask(A)) V once the TMEM warps wrote it
+                // O += bf16(mask(A)) V once the TMEM warps wrote it (A operand in TMEM)
                 if (!mbar_wait(&m->adone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tbase + kColO, tbase + kColP + 8 * kk,
                                 sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
-                }
                 mma_commit(&m->barO2);
                 mma_commit(&m->emptyV[s]);   // v of stage s is free once every MMA above completed
             }
@@ -281,19 +280,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     tma_store_commit();
                 }
             }
-            // causal mask of A, bf16 -> X (A operand) once the inter-chunk MMA (and the state
-            // store) have read X
+            // causal mask of A -> bf16 pairs in TMEM columns P (the A operand of the intra MMA),
+            // as soon as A is complete.  Column block c is kept (c < quad), dropped (c > quad) or
+            // diagonal (per element).  The MMA that read the previous chunk's P completed before A.
             if (!mbar_wait(&m->barA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (!mbar_wait(&m->barO1, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (p.save) {
-                if (r == 0) tma_store_wait_read0();
-                named_bar_sync(2, 128);
-            }
             tc_fence_after();
-            // column block c is kept (c < quad), dropped (c > quad) or diagonal (per element)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float v[32];
+                float v[32], pk[16];
                 if (c <= quad) {
                     tmem_ld32(tl + kColA + 32 * c, v);
                     tmem_wait_ld();
@@ -302,18 +296,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         for (int i = 0; i < 32; ++i)
                             if (i > lane) v[i] = 0.0f;
                     }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pk[i] = __uint_as_float(pack_bf2(v[2 * i], v[2 * i + 1]));
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                    for (int i = 0; i < 16; ++i) pk[i] = 0.0f;
                 }
-                store_chunk_bf16(X, r, c, v);
+                tmem_st16(tl + kColP + 16 * c, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&m->adone);
-            // o epilogue: O -> bf16 rows in X (free: the last MMA of the chunk completed) ->
-            // TMA store; the next S phase waits until the store has read X
+            // o epilogue: O -> bf16 rows in X (free: the last MMA of the chunk completed, and the
+            // state store has read it) -> TMA store; the next S phase waits until the store has read X
             if (!mbar_wait(&m->barO2, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            if (p.save) {
+                if (r == 0) tma_store_wait_read0();
+                named_bar_sync(2, 128);
+            }
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
