@@ -263,3 +263,67 @@ def test_autograd_function_uses_saved_states(cuda):
                           ("dh0", h0.grad[0, h])):
             e = err(np64(got), ref[name][n], torch.bfloat16)
             assert e <= 2e-2, (name, h, e)
+
+
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_more_pairs_than_sms(cuda, saved):
+    # B*H = 192 > 148 SMs: the one-CTA-per-(b,h) kernels run in more than one wave; ragged T
+    B, T, H = 2, 200, 96
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.9, seed=31, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"]) if saved else None
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
+                             saved=sv)
+    assert L.device_status() == L.OK
+    pairs = [(0, 0), (0, 95), (1, 0), (1, 47), (1, 95)]
+    ref = oracle_heads(inp, pairs, want_bwd=True, dhT=inp["dhT"])
+    for n, (b, h) in enumerate(pairs):
+        for name, got in (("o", o[b, :, h]), ("hT", hT[b, h]), ("dq", dq[b, :, h]), ("dlog_f", dlf[b, :, h]),
+                          ("di", di[b, :, h]), ("dh0", dh0[b, h])):
+            e = err(np64(got), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, b, h, e)
+
+
+def test_saved_pair_long_segmented_sequence(cuda):
+    # B*H = 2: the forward cuts each sequence into up to 74 segments (aggregate, fp32 scan, then
+    # every segment from its incoming state) and saves the chunk states of all of them; the
+    # backward walks all 32 chunks of each sequence from the saved states
+    B, T, H = 1, 4096, 2
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.95, seed=41, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"])
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
+                             saved=sv)
+    assert L.device_status() == L.OK
+    ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True, dhT=inp["dhT"])
+    for n, h in enumerate((0, 1)):
+        for name, got in (("o", o[0, :, h]), ("hT", hT[0, h]), ("dq", dq[0, :, h]), ("dlog_f", dlf[0, :, h]),
+                          ("di", di[0, :, h]), ("dh0", dh0[0, h])):
+            e = err(np64(got), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, h, e)
+
+
+def test_calls_on_a_side_stream(cuda):
+    # every call is asynchronous on torch's current stream; results on a side stream match the
+    # default stream's bit for bit
+    inp = I.make_inputs(2, 300, 4, 128, 128, torch.bfloat16, 0.9, seed=51, with_dO=True)
+    g = to_cuda(inp)
+    sv0 = L.new_saved(g["q"])
+    o0, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=64, saved=sv0)
+    r0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=64, saved=sv0)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        sv1 = L.new_saved(g["q"])
+        o1, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=64, saved=sv1)
+        r1 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=64, saved=sv1)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert torch.equal(o0, o1)
+    for a, b in zip(r0[:3], r1[:3]):
+        assert torch.equal(a, b)
