@@ -114,18 +114,20 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun sets RANK / WORLD_SIZE / LOCAL_RANK / MASTER_*).  The data
+    path has no collective: the process group only carries the barriers and the max over ranks
+    of the device times.  backend "gloo" (CPU) is for tests of this host logic."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -136,12 +138,24 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: the whole job is done when every rank is."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(tokens_per_rank_step: int, steps: int, ms: float, world: int) -> float:
+    """Tokens per second of the whole job: every rank processes its own batch (weak scaling)."""
+    return world * tokens_per_rank_step * steps / (ms / 1e3)
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch."""
+    return 1003 + rank
 
 
 def traffic_record(kernel: str):
@@ -179,7 +193,7 @@ def run_ours(args, world, rank, local):
     L.load_library()
     w = I.TRAIN
     B, T, H, dk, dv, chunk = w.B, w.T, w.H, w.dk, w.dv, w.chunk
-    inp = I.make_workload(w, seed=1003 + rank)
+    inp = I.make_workload(w, seed=rank_seed(rank))
     dev = torch.device("cuda", local)
     q, lf, x, dO = (inp[k].to(dev) for k in ("q", "log_f", "i", "dO"))
     ws_f = torch.empty(max(L.workspace_size(B, T, H, dk, dv, chunk, w.dtype, False), 16), dtype=torch.uint8, device=dev)
@@ -245,7 +259,7 @@ def run_ours(args, world, rank, local):
     bwd_ms = ev[1].elapsed_time(ev[2]) / K
     ms_per_step = ms / K
     tokens_per_step = B * T
-    value = world * tokens_per_step * K / (ms / 1e3)
+    value = whole_job_value(tokens_per_step, K, ms, world)
 
     pk = peaks()
     th = B * T * H   # token-heads per step
@@ -357,7 +371,7 @@ def run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, sv, w, world):
     ms = max_over_ranks(a.elapsed_time(b), world)
     h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = sum(t.numel() * t.element_size() for t in hout)
-    return {"value": round(world * w.B * w.T * K / (ms / 1e3), 1), "unit": "tokens/s",
+    return {"value": round(whole_job_value(w.B * w.T, K, ms, world), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
             "ms_per_step": round(ms / K, 3),
             "pipeline": "upload k+1 | compute k | download k-1 on three streams; fill and drain timed"}

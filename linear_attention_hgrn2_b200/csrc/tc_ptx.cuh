@@ -192,6 +192,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) 
         "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&r)[8]) {
+    const uint32_t *u = reinterpret_cast<const uint32_t *>(r);
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(u[0]),
+                 "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+                 : "memory");
+}
 // One 32-bit TMEM column of the thread's lane.
 __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     uint32_t u;
