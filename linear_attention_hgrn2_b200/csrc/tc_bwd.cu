@@ -571,18 +571,6 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const uint32_t par = it & 1;
         if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
         if (tid == 0) waited[0] = it + 1;
-        if (tid == 0) {   // warm L2: this chunk's dq (or saved state), the next chunk's inputs
-            for (int c = 0; c < 2; ++c) {
-                if (kSaved) tma_prefetch_l2_4d(&tm_st, 64 * c, 0, 0, bh * N + n);
-                else tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
-                if (n > 0) {
-                    tma_prefetch_l2_4d(&tm_q, 64 * c, h, (n - 1) * kTile, b);
-                    tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (n - 1) * kTile, b);
-                    tma_prefetch_l2_4d(&tm_x, 64 * c, h, (n - 1) * kTile, b);
-                    tma_prefetch_l2_4d(&tm_do, 64 * c, h, (n - 1) * kTile, b);
-                }
-            }
-        }
         // ---- prep: column j, rows c0 .. c0+31: Qt = q E, Kt = k / E in place; E -> TMEM.
         // f = e^a directly, so k = 1 - f has an absolute error of a few 1e-8; E is the running
         // product of f from the range start, 1/E = e^{-b}.
@@ -652,6 +640,19 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                             sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, kk > 0);
             }
             mma_commit(&m->barP1);
+            // warm L2: this chunk's dq (or saved state), the next chunk's inputs.  Issued here,
+            // where this thread would otherwise only wait: a prefetch holds up its issuing thread,
+            // and at the top of the chunk that delayed every warp at the next block barrier.
+            for (int c = 0; c < 2; ++c) {
+                if (kSaved) tma_prefetch_l2_4d(&tm_st, 64 * c, 0, 0, bh * N + n);
+                else tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
+                if (n > 0) {
+                    tma_prefetch_l2_4d(&tm_q, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_x, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_do, 64 * c, h, (n - 1) * kTile, b);
+                }
+            }
             tma_store_wait_read0();   // previous chunk's di / d log f stores have read AT / DA
         }
         __syncthreads();

@@ -156,12 +156,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 for (int c = 0; c < 2; ++c)
                     tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, h, (g0 + n) * kTile, b);
                 ++issued_v;
-                if (n + 2 < N)   // warm L2 for the chunk after next (its load waits for a free stage)
-                    for (int c = 0; c < 2; ++c) {
-                        tma_prefetch_l2_4d(&tm_q, 64 * c, h, (g0 + n + 2) * kTile, b);
-                        tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (g0 + n + 2) * kTile, b);
-                        tma_prefetch_l2_4d(&tm_x, 64 * c, h, (g0 + n + 2) * kTile, b);
-                    }
             }
         }
     } else if (warp == 1) {
