@@ -424,6 +424,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 namespace rsw {
 constexpr uint32_t kColDS = 0, kColX1 = 128, kColX2 = 256, kColE = 384;
 constexpr int kRevThreads = 512;
+constexpr int kStoreTid = 256;   // issues the output TMA stores (thread 0 issues loads and MMAs)
 
 struct __align__(8) Misc {
     uint64_t barIn, barVO, barDQ, barP1, barP2, barP3;   // barDQ: dq (recompute) or S_in (saved)
@@ -653,8 +654,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     tma_prefetch_l2_4d(&tm_do, 64 * c, h, (n - 1) * kTile, b);
                 }
             }
-            tma_store_wait_read0();   // previous chunk's di / d log f stores have read AT / DA
         }
+        // the previous chunk's output stores have read their staging tiles (the issuing thread)
+        if (tid == kStoreTid) tma_store_wait_read0();
         __syncthreads();
         // ---- dS phase: dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16
         {
@@ -859,7 +861,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tc_fence_before();
         __syncthreads();
         if (q4 == 0) m->carry[j] += m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
-        if (tid == 0) {
+        if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
             tma_store_4d(&tm_di, AT, 0, h, n * kTile, b);
             tma_store_4d(&tm_di, AT + kBlk, 64, h, n * kTile, b);
             tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
@@ -876,8 +878,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         uint64_t *bars[3] = {&m->barIn, &m->barVO, &m->barDQ};
         for (int q = 0; q < 3; ++q)
             for (int k = waited[q]; k < issued[q]; ++k) mbar_wait(bars[q], k & 1, 2000000u);
-        tma_store_wait_all0();
     }
+    if (tid == kStoreTid) tma_store_wait_all0();
     if (ok && n < 0 && p.dh0) {
         tc_fence_after();
         float v[32];
