@@ -749,6 +749,14 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
             mma_commit(&m->barP2);   // also covers the recurrence step issued after the dS phase
         }
+        // Qt and Kt to registers for the epilogue while the phase-2 MMAs run
+        uint32_t qk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t off = eoff(c0 + i);
+            qk[i] = (uint32_t)*reinterpret_cast<const uint16_t *>(Qb + off) |
+                    ((uint32_t)*reinterpret_cast<const uint16_t *>(Gb + off) << 16);
+        }
         if (__syncthreads_or(!mbar_wait(&m->barP2, par))) { ok = false; break; }
         tc_fence_after();
         if (tid == 0) {
@@ -772,15 +780,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         // ---- d log f (lane j, tokens c0 .. c0+31): partial values kept in TMEM X1 (di has
         // been read out): d'_t = sum_{t<=t'<quarter end} (q dq - k dk)_{t'} - f_t dk_t with
-        // q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}.  Qt and Kt are copied to
-        // registers first, so that q and log f of the next chunk can load during the epilogue.
-        uint32_t qk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const uint32_t off = eoff(c0 + i);
-            qk[i] = (uint32_t)*reinterpret_cast<const uint16_t *>(Qb + off) |
-                    ((uint32_t)*reinterpret_cast<const uint16_t *>(Gb + off) << 16);
-        }
+        // q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}.  Qt and Kt were copied to
+        // registers, so that q and log f of the next chunk can load during the epilogue.
         if (kSaved) {
             // phase 3 once di has left X1: dq_pre^T = S_in dO^T + Kt^T mask(dA)^T   (M = j, N = t)
             tc_fence_before();
