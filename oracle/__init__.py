@@ -102,3 +102,17 @@ def step(q, log_f, i, S):
     o = np.zeros((B, H, dv))
     _load().oracle_step(_p(q), _p(log_f), _p(i), _p(S), _p(o), B, H, dk, dv)
     return o, S
+
+
+def lower_bound_log_f(g, lb: float):
+    """log f for the lower-bounded forget gate f = lb + (1 - lb) * sigmoid(g), in fp64.
+
+    ("HGRN2: Gated Linear RNNs with State Expansion", §2.2: the forget gate of each layer is
+    kept above a learnable lower bound lb in [0, 1).)  Written as
+        log f = log(1 + lb e^{-g}) - log(1 + e^{-g}),
+    both terms through log-add-exp, so that neither g -> +inf nor g -> -inf overflows; lb = 0
+    gives log sigmoid(g)."""
+    g = np.asarray(g, dtype=np.float64)
+    if lb == 0.0:
+        return -np.logaddexp(0.0, -g)
+    return np.logaddexp(0.0, np.log(lb) - g) - np.logaddexp(0.0, -g)

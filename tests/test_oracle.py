@@ -220,3 +220,32 @@ def test_bwd_linear_in_dO():
     g12 = oracle.bwd(q, lf, x, 2 * d1 - 3 * d2, h0)
     for a, b, c in zip(g1, g2, g12):
         np.testing.assert_allclose(c, 2 * a - 3 * b, rtol=1e-11, atol=1e-11)
+
+
+# ---------------------------------------------------------------- lower-bounded forget gate
+def test_lower_bound_gate_closed_forms():
+    # f = lb + (1 - lb) sigmoid(g) ("HGRN2: Gated Linear RNNs with State Expansion", §2.2)
+    for lb in (0.0, 0.5, 0.9, 0.99):
+        # g = 0: sigmoid = 1/2, f = (1 + lb) / 2
+        assert oracle.lower_bound_log_f(0.0, lb) == pytest.approx(np.log((1 + lb) / 2), rel=1e-15, abs=1e-15)
+        # g -> +inf: f -> 1 from below, 1 - f = (1 - lb) e^{-g} (1 + O(e^{-g}))
+        g = 40.0
+        assert -oracle.lower_bound_log_f(g, lb) == pytest.approx((1 - lb) * np.exp(-g), rel=1e-9)
+        if lb > 0:   # g -> -inf: f -> lb
+            assert oracle.lower_bound_log_f(-40.0, lb) == pytest.approx(np.log(lb), rel=1e-12)
+    # lb = 0 is the textbook log-sigmoid: -log1p(e^{-g}) for g >= 0, g - log1p(e^{g}) for g < 0
+    g = np.linspace(-20, 20, 41)
+    logsig = np.where(g >= 0, -np.log1p(np.exp(-np.abs(g))), g - np.log1p(np.exp(-np.abs(g))))
+    np.testing.assert_allclose(oracle.lower_bound_log_f(g, 0.0), logsig, rtol=1e-13)
+
+
+def test_lower_bound_gate_matches_direct_formula_and_is_monotone():
+    rng = np.random.default_rng(3)
+    g = rng.normal(0, 3, 1000).clip(-10, 10)
+    for lb in (0.1, 0.5, 0.95):
+        direct = np.log(lb + (1 - lb) / (1 + np.exp(-g)))
+        np.testing.assert_allclose(oracle.lower_bound_log_f(g, lb), direct, rtol=1e-9, atol=1e-15)
+    gs = np.sort(g)
+    assert np.all(np.diff(oracle.lower_bound_log_f(gs, 0.5)) >= 0)          # increasing in g
+    assert np.all(oracle.lower_bound_log_f(g, 0.9) >= oracle.lower_bound_log_f(g, 0.5))   # and in lb
+    assert np.all(oracle.lower_bound_log_f(g, 0.5) <= 0) and np.all(oracle.lower_bound_log_f(g, 0.5) >= np.log(0.5))
