@@ -175,6 +175,15 @@ hgrn2_status hgrn2_bwd_noalloc(const void *q, const void *log_f, const void *i, 
 hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *S, void *o,
                         int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
 
+/* hgrn2_step with the lower-bounded forget gate formed in the kernel from raw gate
+ * logits (§2.2: each layer keeps its forget gate above a lower bound lb):
+ *   f = lb + (1 - lb) sigmoid(g),   k = 1 - f = (1 - lb) sigmoid(-g)
+ *   g : [B,H,dk] (dtype), the gate pre-activations of this token; 0 <= lb < 1 (else
+ *   HGRN2_ERR_INVALID_ARG).  Everything else as hgrn2_step.  It saves the separate
+ *   elementwise pass that would write log f for hgrn2_step. */
+hgrn2_status hgrn2_step_lb(const void *q, const void *g, const void *i, float lb, float *S, void *o,
+                           int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the library's device-side
  * status word of the current device: HGRN2_OK, HGRN2_ERR_TIMEOUT (a bounded
  * wait gave up) or HGRN2_ERR_DEVICE (a consistency check failed).  Returns

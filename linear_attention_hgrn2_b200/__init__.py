@@ -27,7 +27,7 @@ FP32, BF16 = 0, 1
 
 # Every extern "C" symbol of include/hgrn2.h.
 EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size", "hgrn2_fwd_train",
-           "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_step", "hgrn2_get_device_status",
+           "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_step", "hgrn2_step_lb", "hgrn2_get_device_status",
            "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
 
 _lib = None
@@ -65,6 +65,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_bwd_noalloc.restype = i32
     lib.hgrn2_step.argtypes = [vp] * 5 + [i32] * 5 + [vp]
     lib.hgrn2_step.restype = i32
+    lib.hgrn2_step_lb.argtypes = [vp] * 3 + [ctypes.c_float] + [vp] * 2 + [i32] * 5 + [vp]
+    lib.hgrn2_step_lb.restype = i32
     lib.hgrn2_get_device_status.argtypes = [vp]
     lib.hgrn2_get_device_status.restype = i32
     lib.hgrn2_get_counters.argtypes = [ctypes.POINTER(ctypes.c_longlong), i32, i32, vp]
@@ -229,6 +231,23 @@ def step(q, log_f, i, S, out=None):
     o = out if out is not None else torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     st = lib.hgrn2_step(_ptr(q), _ptr(log_f), _ptr(i), _ptr(S), _ptr(o), B, H, dk, dv, _dt(q), _stream())
     _raise(st, "hgrn2_step")
+    return o
+
+
+def step_lb(q, g, i, lb: float, S, out=None):
+    """One decode step with the lower-bounded forget gate f = lb + (1 - lb) sigmoid(g)
+    formed in the kernel from the raw gate logits g [B,H,dk]; otherwise as step()."""
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = i.shape[-1]
+    _check(q, "q")
+    _check(g, "g", q.dtype, q.shape)
+    _check(i, "i", q.dtype, (B, H, dv))
+    _check(S, "S", torch.float32, (B, H, dk, dv))
+    o = out if out is not None else torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = lib.hgrn2_step_lb(_ptr(q), _ptr(g), _ptr(i), ctypes.c_float(lb), _ptr(S), _ptr(o), B, H, dk, dv, _dt(q),
+                           _stream())
+    _raise(st, "hgrn2_step_lb")
     return o
 
 

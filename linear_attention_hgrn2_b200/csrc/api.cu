@@ -185,6 +185,20 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     return from_cuda(launch_simt_bwd(a, bf16, stream));
 }
 
+hgrn2_status step_impl(const void *q, const void *lf, const void *i, float *S, void *o, int B, int H, int dk, int dv,
+                       hgrn2_dtype dtype, bool gate_lb, float lb, cudaStream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
+    if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
+    if (dk > 128 || dv > 128 || (dv & 3)) return HGRN2_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    if (!q || !lf || !i || !S || !o) return HGRN2_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, lf, i, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    g_launches += 1;
+    return from_cuda(launch_step(q, lf, i, S, o, B, H, dk, dv, dtype == HGRN2_BF16, gate_lb, lb, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -234,16 +248,13 @@ hgrn2_status hgrn2_bwd_saved(const void *q, const void *log_f, const void *i, co
 
 hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *S, void *o, int B, int H,
                         int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream) {
-    if (B < 1 || H < 1 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
-    if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
-    if (dk > 128 || dv > 128 || (dv & 3)) return HGRN2_ERR_UNSUPPORTED;
-    if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
-    if (!q || !log_f || !i || !S || !o) return HGRN2_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, log_f, i, S, o};
-    for (const void *p : ptrs)
-        if (!aligned16(p)) return HGRN2_ERR_INVALID_ARG;
-    g_launches += 1;
-    return from_cuda(launch_step(q, log_f, i, S, o, B, H, dk, dv, dtype == HGRN2_BF16, stream));
+    return step_impl(q, log_f, i, S, o, B, H, dk, dv, dtype, false, 0.0f, stream);
+}
+
+hgrn2_status hgrn2_step_lb(const void *q, const void *g, const void *i, float lb, float *S, void *o, int B, int H,
+                           int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream) {
+    if (!(lb >= 0.0f && lb < 1.0f)) return HGRN2_ERR_INVALID_ARG;   // also rejects NaN
+    return step_impl(q, g, i, S, o, B, H, dk, dv, dtype, true, lb, stream);
 }
 
 hgrn2_status hgrn2_get_device_status(cudaStream_t stream) {

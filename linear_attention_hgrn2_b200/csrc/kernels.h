@@ -64,7 +64,8 @@ size_t tc_bwd_smem();
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st);
 
+// gate_lb: `lf` holds raw gate logits g and f = lb + (1 - lb) sigmoid(g); else `lf` is log f.
 cudaError_t launch_step(const void *q, const void *lf, const void *x, float *S, void *o, int B, int H,
-                        int dk, int dv, bool bf16, cudaStream_t st);
+                        int dk, int dv, bool bf16, bool gate_lb, float lb, cudaStream_t st);
 
 }  // namespace hgrn2

@@ -16,6 +16,12 @@
 // larger than L2 at serving batch sizes, so it should not displace other data.
 // The d_k-long dot products for o are reduced across row groups in shared
 // memory.
+//
+// Lower-bounded gate (the kLB instantiation): the call passes the raw gate logits g
+// instead of log f, and f = lb + (1 - lb) sigmoid(g) ("HGRN2", §2.2: each layer's forget
+// gate is kept above a lower bound lb in [0, 1)) is formed here, with
+// k = 1 - f = (1 - lb) sigmoid(-g) taken directly, so neither f nor k loses precision and
+// no separate pass writes log f.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,10 +30,10 @@ namespace hgrn2 {
 constexpr int kStepThreads = 256;
 constexpr int kStepMaxRows = 16;   // ceil(128 * 32 / 256): d_k <= 128, d_v <= 128
 
-template <typename T>
+template <typename T, bool kLB>
 __global__ void __launch_bounds__(kStepThreads, 2)
 step_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
-            float *__restrict__ S, T *__restrict__ o, int dk, int dv) {
+            float *__restrict__ S, T *__restrict__ o, int dk, int dv, float lb) {
     __shared__ float sq[128], sf[128], sk[128];
     __shared__ float4 red[kStepThreads];
     const int bh = blockIdx.x, tid = threadIdx.x;
@@ -45,8 +51,14 @@ step_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restri
     }
     for (int j = tid; j < dk; j += kStepThreads) {
         const float a = to_f<T>(lf[(size_t)bh * dk + j]);
-        sf[j] = expf(a);
-        sk[j] = one_minus_exp(a);
+        if (kLB) {   // a = g: sigmoid(|g|) and sigmoid(-|g|) from e^{-|g|} in (0, 1]
+            const float e = expf(-fabsf(a)), sp = 1.0f / (1.0f + e), sn = e * sp;
+            sf[j] = lb + (1.0f - lb) * (a >= 0.0f ? sp : sn);
+            sk[j] = (1.0f - lb) * (a >= 0.0f ? sn : sp);
+        } else {
+            sf[j] = expf(a);
+            sk[j] = one_minus_exp(a);
+        }
         sq[j] = to_f<T>(q[(size_t)bh * dk + j]);
     }
     float4 xv = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -89,16 +101,24 @@ step_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restri
     }
 }
 
+template <typename T>
+static void launch_step_t(const void *q, const void *lf, const void *x, float *S, void *o, int grid, int dk, int dv,
+                          bool gate_lb, float lb, cudaStream_t st) {
+    if (gate_lb)
+        step_kernel<T, true><<<grid, kStepThreads, 0, st>>>((const T *)q, (const T *)lf, (const T *)x, S, (T *)o, dk,
+                                                            dv, lb);
+    else
+        step_kernel<T, false><<<grid, kStepThreads, 0, st>>>((const T *)q, (const T *)lf, (const T *)x, S, (T *)o, dk,
+                                                             dv, 0.0f);
+}
+
 cudaError_t launch_step(const void *q, const void *lf, const void *x, float *S, void *o, int B, int H,
-                        int dk, int dv, bool bf16, cudaStream_t st) {
+                        int dk, int dv, bool bf16, bool gate_lb, float lb, cudaStream_t st) {
     const int grid = B * H;
     if (bf16)
-        step_kernel<__nv_bfloat16><<<grid, kStepThreads, 0, st>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)lf, (const __nv_bfloat16 *)x, S,
-            (__nv_bfloat16 *)o, dk, dv);
+        launch_step_t<__nv_bfloat16>(q, lf, x, S, o, grid, dk, dv, gate_lb, lb, st);
     else
-        step_kernel<float><<<grid, kStepThreads, 0, st>>>((const float *)q, (const float *)lf,
-                                                          (const float *)x, S, (float *)o, dk, dv);
+        launch_step_t<float>(q, lf, x, S, o, grid, dk, dv, gate_lb, lb, st);
     return cudaGetLastError();
 }
 

@@ -104,7 +104,9 @@ def make_workload(w: Workload, seed: int) -> dict:
 
 def make_decode(B: int, H: int, dk: int, dv: int, steps: int, dtype: torch.dtype, lb: float,
                 seed: int, S_sigma: float = 1.0, device: str = "cpu") -> dict:
-    """Decode-step inputs: q, log_f [steps,B,H,dk], i [steps,B,H,dv] and S [B,H,dk,dv] fp32.
+    """Decode-step inputs: q, log_f [steps,B,H,dk], i [steps,B,H,dv] and S [B,H,dk,dv] fp32,
+    plus g [steps,B,H,dk]: the gate pre-activations log_f was made from, rounded to dtype
+    (for the lower-bounded-gate step, which takes them raw).
 
     On device='cpu' the draws use NumPy's PCG64 (bit-reproducible everywhere).
     On a CUDA device they use a seeded torch CUDA generator (for the large
@@ -113,15 +115,17 @@ def make_decode(B: int, H: int, dk: int, dv: int, steps: int, dtype: torch.dtype
         g = _gen(seed)
         q = _to(_normal(g, (steps, B, H, dk)), dtype)
         i = _to(_normal(g, (steps, B, H, dv)), dtype)
-        lf = _to(gate_log_f(_normal(g, (steps, B, H, dk)), lb), dtype)
+        x = _normal(g, (steps, B, H, dk))
+        lf = _to(gate_log_f(x, lb), dtype)
         S = torch.from_numpy(_normal(g, (B, H, dk, dv), S_sigma))
-        return {"q": q, "i": i, "log_f": lf, "S": S}
+        return {"q": q, "i": i, "log_f": lf, "S": S, "g": _to(x, dtype)}
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     q = torch.randn((steps, B, H, dk), generator=gen, device=device).to(dtype)
     i = torch.randn((steps, B, H, dv), generator=gen, device=device).to(dtype)
     x = torch.randn((steps, B, H, dk), generator=gen, device=device, dtype=torch.float64)
     lf = torch.log(lb + (1.0 - lb) * torch.sigmoid(x)).to(dtype)
+    graw = x.to(dtype)
     del x
     S = torch.randn((B, H, dk, dv), generator=gen, device=device) * S_sigma
-    return {"q": q, "i": i, "log_f": lf, "S": S}
+    return {"q": q, "i": i, "log_f": lf, "S": S, "g": graw}

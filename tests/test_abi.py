@@ -114,3 +114,10 @@ def test_saved_size_and_training_pair_argument_checks(lib):
     assert st == L.ERR_INVALID_ARG
     st = lib.hgrn2_bwd_saved(*([None] * 5), 0, *([None] * 6), 1, 8, 1, 16, 16, 16, 1, None, 0, None)
     assert st == L.ERR_INVALID_ARG       # null inputs (exact route: the buffer is not needed)
+
+
+def test_step_lb_checks_the_bound_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    for lb in (-0.5, 1.0, 2.0, float("nan")):
+        st = lib.hgrn2_step_lb(vp(16), vp(16), vp(16), ctypes.c_float(lb), vp(16), vp(16), 1, 1, 16, 16, 0, None)
+        assert st == L.ERR_INVALID_ARG, lb

@@ -56,3 +56,50 @@ def test_steps_equal_fwd(cuda, dtype):
         ot = L.step(g["q"][:, t].contiguous(), g["log_f"][:, t].contiguous(), g["i"][:, t].contiguous(), S)
         assert err(np64(ot), np64(o[:, t]), dtype) <= tol(dtype)
     assert err(np64(S), np64(hT), dtype) <= tol(dtype)
+
+
+# ---------------------------------------------------------------- lower-bounded gate in the kernel
+@pytest.mark.parametrize("dtype,B,H,dk,dv,lb", [
+    (torch.bfloat16, 4, 3, 128, 128, 0.8),
+    (torch.float32, 2, 2, 16, 16, 0.0),
+    (torch.float32, 3, 2, 64, 32, 0.95),
+    (torch.bfloat16, 2, 2, 100, 12, 0.5),
+])
+def test_step_lb_matches_oracle(cuda, dtype, B, H, dk, dv, lb):
+    steps = 20
+    d = I.make_decode(B, H, dk, dv, steps, dtype, lb, seed=13)
+    S = d["S"].cuda()
+    S_ref = np64(d["S"])
+    for t in range(steps):
+        g = d["g"][t] * 3.0   # wider than N(0,1): both saturation sides of the sigmoid
+        o = L.step_lb(d["q"][t].cuda(), g.cuda(), d["i"][t].cuda(), lb, S)
+        lf_ref = oracle.lower_bound_log_f(np64(g), lb)
+        o_ref, S_ref = oracle.step(np64(d["q"][t]), lf_ref, np64(d["i"][t]), S_ref)
+        assert err(np64(o), o_ref, dtype) <= tol(dtype), t
+    assert err(np64(S), S_ref, dtype) <= tol(dtype)
+
+
+def test_step_lb_extreme_logits_and_full_size_sample(cuda):
+    w = I.DECODE
+    d = I.make_decode(w["B"], w["H"], w["dk"], w["dv"], 2, w["dtype"], w["lb"], seed=1006)
+    S = d["S"].cuda()
+    g = d["g"][0].clone()
+    g[0, 0, :64] = 40.0     # f -> 1: the state is kept, nothing is written
+    g[0, 0, 64:] = -40.0    # f -> lb
+    o = L.step_lb(d["q"][0].cuda(), g.cuda(), d["i"][0].cuda(), w["lb"], S)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    for (b, h) in [(0, 0), (17, 3), (255, 15)]:
+        sl = lambda x: np64(x[b:b + 1, h:h + 1])
+        o_ref, S_ref = oracle.step(sl(d["q"][0]), oracle.lower_bound_log_f(sl(g), w["lb"]), sl(d["i"][0]),
+                                   sl(d["S"]))
+        assert err(np64(o[b:b + 1, h:h + 1]), o_ref, w["dtype"]) <= tol(w["dtype"])
+        assert err(np64(S[b:b + 1, h:h + 1]), S_ref, torch.float32) <= 1e-5
+
+
+def test_step_lb_rejects_bounds_outside_unit_interval(cuda):
+    q = torch.zeros(1, 1, 16, device="cuda")
+    S = torch.zeros(1, 1, 16, 16, device="cuda")
+    for lb in (-0.1, 1.0, float("nan")):
+        with pytest.raises(L.HGRN2Error):
+            L.step_lb(q, q, q, lb, S)
