@@ -143,6 +143,43 @@ hgrn2_status hgrn2_bwd_saved(const void *q, const void *log_f, const void *i, co
                              int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
                              void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* Packed variable-length sequences.  The paper trains on concatenated documents
+ * (§4 language modelling); packing several sequences into one token tensor without
+ * padding is how that is fed to a per-sequence recurrence.  The recurrence restarts
+ * at every sequence boundary.
+ *   token tensors q, log_f, dq, dlog_f: [total_T][H][dk];  i, o, dO, di: [total_T][H][dv]
+ *   cu_seqlens: DEVICE int32 [nseq + 1], 16-byte aligned; sequence s is tokens
+ *     cu_seqlens[s] .. cu_seqlens[s+1]-1 (0 = cu[0] <= cu[1] <= ... <= cu[nseq] = total_T;
+ *     not checked on the host: values are clamped to [0, total_T] on the device, so a
+ *     malformed array gives wrong results, never an out-of-range access).  Sequences may
+ *     be empty and may start at any token.
+ *   states h0, hT, dhT, dh0: [nseq][H][dk][dv] float32, one per sequence and head.
+ * hgrn2_workspace_size_varlen: workspace bytes of both calls (never 0).
+ * hgrn2_saved_size_varlen: bytes of the optional saved-state buffer (0 where there is
+ *   no saved-state path: the exact route, or total_T = 0); (size_t)-1 for bad sizes.
+ * hgrn2_fwd_varlen: forward of every sequence; `saved` (may be NULL) receives what
+ *   hgrn2_bwd_varlen reads, as for hgrn2_fwd_train.
+ * hgrn2_bwd_varlen: backward of every sequence.  With the `saved` buffer of the
+ *   matching hgrn2_fwd_varlen call it is one reverse-sweep launch on tensor cores;
+ *   without it (NULL) the exact CUDA-core route computes it. */
+size_t hgrn2_workspace_size_varlen(int nseq, int total_T, int H, int dk, int dv, int chunk,
+                                   hgrn2_dtype dtype);
+size_t hgrn2_saved_size_varlen(int nseq, int total_T, int H, int dk, int dv, hgrn2_dtype dtype);
+
+hgrn2_status hgrn2_fwd_varlen(const void *q, const void *log_f, const void *i, const float *h0,
+                              void *o, float *hT, const int *cu_seqlens, int nseq, int total_T,
+                              int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                              void *saved, size_t saved_bytes, void *workspace, size_t ws_bytes,
+                              cudaStream_t stream);
+
+hgrn2_status hgrn2_bwd_varlen(const void *q, const void *log_f, const void *i, const float *h0,
+                              const void *saved, size_t saved_bytes,
+                              const void *dO, const float *dhT,
+                              void *dq, void *dlog_f, void *di, float *dh0,
+                              const int *cu_seqlens, int nseq, int total_T, int H, int dk, int dv,
+                              int chunk, hgrn2_dtype dtype, void *workspace, size_t ws_bytes,
+                              cudaStream_t stream);
+
 /* Allocation-free variant of hgrn2_bwd.  The paper has no counterpart: this
  * entry point exists for callers that cannot give the library a device
  * buffer -- for example a plain C host program that links only this library

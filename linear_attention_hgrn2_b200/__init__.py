@@ -27,7 +27,8 @@ FP32, BF16 = 0, 1
 
 # Every extern "C" symbol of include/hgrn2.h.
 EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size", "hgrn2_fwd_train",
-           "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_step", "hgrn2_step_lb", "hgrn2_get_device_status",
+           "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_workspace_size_varlen", "hgrn2_saved_size_varlen",
+           "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_lb", "hgrn2_get_device_status",
            "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
 
 _lib = None
@@ -63,6 +64,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_bwd_saved.restype = i32
     lib.hgrn2_bwd_noalloc.argtypes = [vp] * 10 + [i32] * 7 + [vp]
     lib.hgrn2_bwd_noalloc.restype = i32
+    lib.hgrn2_workspace_size_varlen.argtypes = [i32] * 7
+    lib.hgrn2_workspace_size_varlen.restype = sz
+    lib.hgrn2_saved_size_varlen.argtypes = [i32] * 6
+    lib.hgrn2_saved_size_varlen.restype = sz
+    lib.hgrn2_fwd_varlen.argtypes = [vp] * 7 + [i32] * 7 + [vp, sz, vp, sz, vp]
+    lib.hgrn2_fwd_varlen.restype = i32
+    lib.hgrn2_bwd_varlen.argtypes = [vp] * 5 + [sz] + [vp] * 7 + [i32] * 7 + [vp, sz, vp]
+    lib.hgrn2_bwd_varlen.restype = i32
     lib.hgrn2_step.argtypes = [vp] * 5 + [i32] * 5 + [vp]
     lib.hgrn2_step.restype = i32
     lib.hgrn2_step_lb.argtypes = [vp] * 3 + [ctypes.c_float] + [vp] * 2 + [i32] * 5 + [vp]
@@ -214,6 +223,94 @@ def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dh0=False, chunk=64, workspace=
                        _ptr(dq), _ptr(dlf), _ptr(di), _ptr(dh0),
                        B, T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
     _raise(st, "hgrn2_bwd")
+    return dq, dlf, di, dh0
+
+
+def _size_or_raise(n: int, where: str) -> int:
+    if n == ctypes.c_size_t(-1).value:
+        raise HGRN2Error(ERR_INVALID_ARG, where)
+    return int(n)
+
+
+def saved_size_varlen(nseq, total_T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Bytes of the saved-state buffer of fwd_varlen (0: no saved-state path)."""
+    return _size_or_raise(load_library().hgrn2_saved_size_varlen(nseq, total_T, H, dk, dv,
+                                                                  BF16 if dtype == torch.bfloat16 else FP32),
+                          "hgrn2_saved_size_varlen")
+
+
+def workspace_size_varlen(nseq, total_T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    return _size_or_raise(load_library().hgrn2_workspace_size_varlen(nseq, total_T, H, dk, dv, chunk,
+                                                                      BF16 if dtype == torch.bfloat16 else FP32),
+                          "hgrn2_workspace_size_varlen")
+
+
+def new_saved_varlen(q: torch.Tensor, cu_seqlens: torch.Tensor, dv: int | None = None) -> torch.Tensor | None:
+    """An uninitialised saved-state buffer for fwd_varlen on packed q [total_T,H,dk]."""
+    total_T, H, dk = q.shape
+    n = saved_size_varlen(cu_seqlens.numel() - 1, total_T, H, dk, dk if dv is None else dv, q.dtype)
+    return torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+
+
+def _check_varlen(q, log_f, i, cu_seqlens):
+    _check(q, "q")
+    if q.dim() != 3:
+        raise ValueError("packed token tensors are [total_T, H, D]")
+    total_T, H, dk = q.shape
+    dv = i.shape[-1]
+    _check(log_f, "log_f", q.dtype, q.shape)
+    _check(i, "i", q.dtype, (total_T, H, dv))
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be [nseq + 1] with nseq >= 1")
+    return total_T, H, dk, dv, cu_seqlens.numel() - 1
+
+
+def fwd_varlen(q, log_f, i, cu_seqlens, h0=None, want_hT=False, chunk=64, out=None, saved=None):
+    """Packed variable-length sequences: q, log_f [total_T,H,dk], i [total_T,H,dv];
+    sequence s is tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 (int32 CUDA tensor), each
+    with its own state (h0, hT: [nseq,H,dk,dv] float32).  saved: new_saved_varlen()
+    or None.  Returns (o [total_T,H,dv], hT or None)."""
+    lib = load_library()
+    total_T, H, dk, dv, nseq = _check_varlen(q, log_f, i, cu_seqlens)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (nseq, H, dk, dv))
+    o = out if out is not None else torch.empty((total_T, H, dv), dtype=q.dtype, device=q.device)
+    _check(o, "o", q.dtype, (total_T, H, dv))
+    hT = torch.empty((nseq, H, dk, dv), dtype=torch.float32, device=q.device) if want_hT else None
+    nws = workspace_size_varlen(nseq, total_T, H, dk, dv, chunk, q.dtype)
+    ws = _workspace(nws, q.device)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8)
+    st = lib.hgrn2_fwd_varlen(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(o), _ptr(hT), _ptr(cu_seqlens),
+                              nseq, total_T, H, dk, dv, chunk, _dt(q), _ptr(saved),
+                              0 if saved is None else saved.numel(), _ptr(ws), nws, _stream())
+    _raise(st, "hgrn2_fwd_varlen")
+    return o, hT
+
+
+def bwd_varlen(q, log_f, i, dO, cu_seqlens, h0=None, dhT=None, want_dh0=False, chunk=64, saved=None):
+    """Gradients (dq, dlog_f, di, dh0 or None) of packed sequences (see fwd_varlen)."""
+    lib = load_library()
+    total_T, H, dk, dv, nseq = _check_varlen(q, log_f, i, cu_seqlens)
+    _check(dO, "dO", q.dtype, (total_T, H, dv))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (nseq, H, dk, dv))
+    if dhT is not None:
+        _check(dhT, "dhT", torch.float32, (nseq, H, dk, dv))
+    dq = torch.empty_like(q)
+    dlf = torch.empty_like(q)
+    di = torch.empty_like(i)
+    dh0 = torch.empty((nseq, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
+    nws = workspace_size_varlen(nseq, total_T, H, dk, dv, chunk, q.dtype)
+    ws = _workspace(nws, q.device)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8)
+    st = lib.hgrn2_bwd_varlen(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(saved),
+                              0 if saved is None else saved.numel(), _ptr(dO), _ptr(dhT),
+                              _ptr(dq), _ptr(dlf), _ptr(di), _ptr(dh0), _ptr(cu_seqlens),
+                              nseq, total_T, H, dk, dv, chunk, _dt(q), _ptr(ws), nws, _stream())
+    _raise(st, "hgrn2_bwd_varlen")
     return dq, dlf, di, dh0
 
 

@@ -64,16 +64,21 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
 struct SavedLayout {
     size_t hTs, flags, total;   // byte offsets (the bf16 states start at 0)
 };
-SavedLayout saved_layout(int B, int T, int H) {
-    const size_t BH = (size_t)B * H, nt = (size_t)(T + 127) / 128;
+SavedLayout saved_layout(int B, int T, int H, bool packed = false) {
+    const size_t BH = (size_t)B * H, slots = (size_t)tc_saved_slots(B, T, H, packed);
     SavedLayout l;
-    l.hTs = align256(BH * nt * 128 * 128 * 2);
+    l.hTs = align256(slots * 128 * 128 * 2);
     l.flags = l.hTs + align256(BH * 128 * 128 * sizeof(float));
     l.total = l.flags + align256(BH * sizeof(int));
     return l;
 }
 size_t saved_bytes_needed(int B, int T, int H, int dk, int dv, hgrn2_dtype dt) {
     return (use_tc(dk, dv, dt) && T > 0) ? saved_layout(B, T, H).total : 0;
+}
+
+// Workspace of the packed-sequence calls: rowsum(dhT * hT) [nseq*H*dk] and flags [nseq*H].
+size_t ws_bytes_varlen(int nseq, int H, int dk) {
+    return align256(sizeof(float) * (size_t)nseq * H * dk) + align256(sizeof(int) * (size_t)nseq * H);
 }
 
 hgrn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HGRN2_OK : HGRN2_ERR_CUDA; }
@@ -97,14 +102,14 @@ namespace {
 // Forward; `saved` (null, or saved_bytes_needed bytes) receives what hgrn2_bwd_saved reads.
 hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
                       void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
-                      void *workspace, size_t ws_bytes, cudaStream_t stream) {
+                      void *workspace, size_t ws_bytes, cudaStream_t stream, const int *cu = nullptr) {
     hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !log_f || !i || !o)) return HGRN2_ERR_INVALID_ARG;
     const void *ptrs[] = {q, log_f, i, h0, o, hT, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
-    size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 0);
+    size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 0);
     if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
     const bool bf16 = dtype == HGRN2_BF16;
     if (T == 0) {
@@ -119,13 +124,14 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
     if (use_tc(dk, dv, dtype)) {
         // tensor-core pass; (b,h) pairs whose chunk decay span is too wide are flagged
         // and recomputed right after by the exact route (same stream, in order)
-        const SavedLayout sl = saved_layout(B, T, H);
-        int *flags = saved ? (int *)((char *)saved + sl.flags) : (int *)workspace;
-        float *seg_ws = (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
-        int nseg, tps;
-        tc_fwd_segments(B, T, H, &nseg, &tps);
+        const SavedLayout sl = saved_layout(B, T, H, cu != nullptr);
+        int *flags = saved ? (int *)((char *)saved + sl.flags)
+                           : (int *)((char *)workspace + (cu ? align256(sizeof(float) * (size_t)B * H * dk) : 0));
+        float *seg_ws = cu ? nullptr : (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
+        int nseg = 1, tps = 1;
+        if (!cu) tc_fwd_segments(B, T, H, &nseg, &tps);
         TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H, C, saved,
-                    saved ? (float *)((char *)saved + sl.hTs) : nullptr};
+                    saved ? (float *)((char *)saved + sl.hTs) : nullptr, cu};
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         if (nseg == 1) {   // the exact route, if needed, runs inside the tensor-core kernel
@@ -134,10 +140,10 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
         }
         // segmented: aggregate, scan, segments, then the exact route for flagged (b,h)
         g_launches += 4;
-        SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags};
+        SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags, nullptr};
         return from_cuda(launch_simt_fwd(a, bf16, stream));
     }
-    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr};
+    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr, cu};
     g_launches += 1;
     return from_cuda(launch_simt_fwd(a, bf16, stream));
 }
@@ -146,14 +152,14 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
 hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
                       const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
                       int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
-                      size_t ws_bytes, cudaStream_t stream) {
+                      size_t ws_bytes, cudaStream_t stream, const int *cu = nullptr) {
     hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !log_f || !i || !dO || !dq || !dlog_f || !di)) return HGRN2_ERR_INVALID_ARG;
     const void *ptrs[] = {q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
-    size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
+    size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
     if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
     const bool bf16 = dtype == HGRN2_BF16;
     if (T == 0) {
@@ -166,21 +172,21 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     int C = simt_chunk(chunk, dk, dv, true);
     if (!C) return HGRN2_ERR_UNSUPPORTED;
     float *rs = (float *)workspace;
-    if (use_tc(dk, dv, dtype)) {
+    if (use_tc(dk, dv, dtype) && (saved || !cu)) {
         if (saved) {   // one launch: reverse sweep from the saved states (exact route inside)
-            const SavedLayout sl = saved_layout(B, T, H);
+            const SavedLayout sl = saved_layout(B, T, H, cu != nullptr);
             TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs,
                         (int *)((char *)saved + sl.flags), B, T, H, C, saved,
-                        (const float *)((const char *)saved + sl.hTs)};
+                        (const float *)((const char *)saved + sl.hTs), cu};
             g_launches += 1;
             return from_cuda(launch_tc_bwd(t, stream));
         }
         int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
-        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C, nullptr, nullptr};
+        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C, nullptr, nullptr, nullptr};
         g_launches += 2;   // the exact route, if needed, runs inside the forward-sweep kernel
         return from_cuda(launch_tc_bwd(t, stream));
     }
-    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr};
+    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr, cu};
     g_launches += 2;
     return from_cuda(launch_simt_bwd(a, bf16, stream));
 }
@@ -244,6 +250,43 @@ hgrn2_status hgrn2_bwd_saved(const void *q, const void *log_f, const void *i, co
     if (need && (!saved || saved_bytes < need)) return HGRN2_ERR_INVALID_ARG;
     return bwd_impl(q, log_f, i, h0, need ? saved : nullptr, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv,
                     chunk, dtype, workspace, ws_bytes, stream);
+}
+
+size_t hgrn2_saved_size_varlen(int nseq, int total_T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    if (check_common(nseq, total_T, H, dk, dv, 64, dtype) != HGRN2_OK) return (size_t)-1;
+    return (use_tc(dk, dv, dtype) && total_T > 0) ? saved_layout(nseq, total_T, H, true).total : 0;
+}
+
+size_t hgrn2_workspace_size_varlen(int nseq, int total_T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype) {
+    if (check_common(nseq, total_T, H, dk, dv, chunk, dtype) != HGRN2_OK) return (size_t)-1;
+    return ws_bytes_varlen(nseq, H, dk);
+}
+
+hgrn2_status hgrn2_fwd_varlen(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
+                              const int *cu_seqlens, int nseq, int total_T, int H, int dk, int dv, int chunk,
+                              hgrn2_dtype dtype, void *saved, size_t saved_bytes, void *workspace, size_t ws_bytes,
+                              cudaStream_t stream) {
+    hgrn2_status s = check_common(nseq, total_T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    if (!cu_seqlens || !aligned16(cu_seqlens)) return HGRN2_ERR_INVALID_ARG;
+    const size_t need = hgrn2_saved_size_varlen(nseq, total_T, H, dk, dv, dtype);
+    if (saved && saved_bytes < need) return HGRN2_ERR_INVALID_ARG;
+    return fwd_impl(q, log_f, i, h0, o, hT, need ? saved : nullptr, nseq, total_T, H, dk, dv, chunk, dtype,
+                    workspace, ws_bytes, stream, cu_seqlens);
+}
+
+hgrn2_status hgrn2_bwd_varlen(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                              size_t saved_bytes, const void *dO, const float *dhT, void *dq, void *dlog_f,
+                              void *di, float *dh0, const int *cu_seqlens, int nseq, int total_T, int H, int dk,
+                              int dv, int chunk, hgrn2_dtype dtype, void *workspace, size_t ws_bytes,
+                              cudaStream_t stream) {
+    hgrn2_status s = check_common(nseq, total_T, H, dk, dv, chunk, dtype);
+    if (s != HGRN2_OK) return s;
+    if (!cu_seqlens || !aligned16(cu_seqlens)) return HGRN2_ERR_INVALID_ARG;
+    const size_t need = hgrn2_saved_size_varlen(nseq, total_T, H, dk, dv, dtype);
+    if (saved && saved_bytes < need) return HGRN2_ERR_INVALID_ARG;
+    return bwd_impl(q, log_f, i, h0, need ? saved : nullptr, dO, dhT, dq, dlog_f, di, dh0, nseq, total_T, H, dk, dv,
+                    chunk, dtype, workspace, ws_bytes, stream, cu_seqlens);
 }
 
 hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *S, void *o, int B, int H,

@@ -13,6 +13,7 @@ struct SimtFwdArgs {
     float *hT;
     int B, T, H, dk, dv, C;
     const int *only;   // if non-null: only (b,h) with only[b*H+h] != 0 are computed
+    const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
 };
 
 struct TcFwdArgs {
@@ -24,8 +25,9 @@ struct TcFwdArgs {
     float *seg_ws;     // segment aggregates, tc_fwd_workspace(B, T, H) bytes (may be null if 0)
     int B, T, H;
     int simt_C;        // chunk of the exact route
-    void *st16;        // out, or null: bf16 state entering every chunk [B*H][ntiles][128][128]
+    void *st16;        // out, or null: bf16 state entering every chunk, tc_saved_slots() tiles
     float *hTs;        // out (with st16): final state [B*H][128][128]
+    const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
 };
 
 struct SimtBwdArgs {
@@ -36,6 +38,7 @@ struct SimtBwdArgs {
     float *rs;   // [B*H*dk] workspace: rowsum(dhT * hT)
     int B, T, H, dk, dv, C;
     const int *only;   // if non-null: only (b,h) with only[b*H+h] != 0 are computed
+    const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
 };
 
 struct TcBwdArgs {
@@ -47,8 +50,9 @@ struct TcBwdArgs {
     int *flags;        // [B*H] recompute: workspace, out; saved states: in, from the forward
     int B, T, H;
     int simt_C;        // chunk of the exact route
-    const void *st16;  // saved bf16 chunk-entry states [B*H][ntiles][128][128], or null (recompute)
+    const void *st16;  // saved bf16 chunk-entry states (tc_saved_slots() tiles), or null (recompute)
     const float *hTs;  // saved final state [B*H][128][128] (with st16)
+    const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens (needs st16)
 };
 
 size_t simt_fwd_smem(int C, int dk, int dv);
@@ -58,6 +62,7 @@ cudaError_t launch_simt_fwd(const SimtFwdArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_bwd(const SimtBwdArgs &a, bool bf16, cudaStream_t st);
 
 size_t tc_fwd_smem();
+int tc_saved_slots(int B, int T, int H, bool packed);
 void tc_fwd_segments(int B, int T, int H, int *nseg, int *tps);
 size_t tc_fwd_workspace(int B, int T, int H);
 size_t tc_bwd_smem();

@@ -71,7 +71,7 @@ template <typename T>
 __device__ __forceinline__ void
 simt_fwd_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
-                int T_, int H, int dk, int dv, int C, float *sm, int bh) {
+                int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;              // [C][ldk]  q, then q * e^{b}
     float *Bs = Qs + C * ldk;    // [C][ldk]  log f, then cumulative b
@@ -79,8 +79,8 @@ simt_fwd_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__rest
     float *Vs = Ks + C * ldk;    // [C][ldv]
     float *As = Vs + C * ldv;    // [C][ldc]
     float *Ss = As + C * ldc;    // [dk][ldv] running state (fp32)
-    const int b = bh / H, h = bh % H, tid = threadIdx.x;
-    const size_t sbase = (size_t)bh * dk * dv;
+    const int tid = threadIdx.x;
+    const size_t sbase = (size_t)sidx * dk * dv;
 
     for (int idx = tid; idx < dk * dv; idx += blockDim.x) {
         int j = idx / dv, v = idx - j * dv;
@@ -146,7 +146,7 @@ template <typename T>
 __device__ __forceinline__ void
 simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
-                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, float *sm, int bh) {
+                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Bs = sm;              // [C][ldk]
     float *Ks = Bs + C * ldk;    // [C][ldk]
@@ -154,8 +154,8 @@ simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float 
     float *Gs = Vs + C * ldv;    // [C][ldv] dO
     float *As = Gs + C * ldv;    // [C][ldc] dA
     float *Ss = As + C * ldc;    // [dk][ldv]
-    const int b = bh / H, h = bh % H, tid = threadIdx.x;
-    const size_t sbase = (size_t)bh * dk * dv;
+    const int tid = threadIdx.x;
+    const size_t sbase = (size_t)sidx * dk * dv;
 
     for (int idx = tid; idx < dk * dv; idx += blockDim.x) {
         int j = idx / dv, v = idx - j * dv;
@@ -205,7 +205,7 @@ simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float 
         for (int j = tid; j < dk; j += blockDim.x) {
             float acc = 0.0f;
             for (int v = 0; v < dv; ++v) acc = fmaf(dhT[sbase + (size_t)j * dv + v], Ss[j * ldv + v], acc);
-            rs[(size_t)bh * dk + j] = acc;
+            rs[(size_t)sidx * dk + j] = acc;
         }
 }
 
@@ -221,7 +221,7 @@ __device__ __forceinline__ void
 simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
-                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, float *sm, int bh) {
+                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;               // [C][ldk] q, later q e^{b}
     float *Bs = Qs + C * ldk;     // [C][ldk] b
@@ -235,14 +235,14 @@ simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__
     float *dAs = As + C * ldc;    // [C][ldc]
     float *dS = dAs + C * ldc;    // [dk][ldv]
     float *carry = dS + dk * ldv; // [dk]
-    const int b = bh / H, h = bh % H, tid = threadIdx.x;
-    const size_t sbase = (size_t)bh * dk * dv;
+    const int tid = threadIdx.x;
+    const size_t sbase = (size_t)sidx * dk * dv;
 
     for (int idx = tid; idx < dk * dv; idx += blockDim.x) {
         int j = idx / dv, v = idx - j * dv;
         dS[j * ldv + v] = dhT ? dhT[sbase + idx] : 0.0f;
     }
-    for (int j = tid; j < dk; j += blockDim.x) carry[j] = (dhT && rs) ? rs[(size_t)bh * dk + j] : 0.0f;
+    for (int j = tid; j < dk; j += blockDim.x) carry[j] = (dhT && rs) ? rs[(size_t)sidx * dk + j] : 0.0f;
 
     const int nchunks = (T_ + C - 1) / C;
     for (int c = nchunks - 1; c >= 0; --c) {
@@ -328,24 +328,53 @@ simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__
 
 
 // ------------------------------------------------------------------ kernels (one CTA per (b,h))
+// With cu (variable-length packed sequences: token tensors [total_T][H][D], sequence s at
+// tokens cu[s] .. cu[s+1]-1), CTA (s,h) runs the body on pointers offset to the sequence's
+// first token, with batch 0 and T = its length; cu values are clamped to [0, total_T].
+struct SeqView {
+    int b, h, T;
+    size_t tok0;
+};
+__device__ __forceinline__ SeqView seq_view(const int *cu, int bid, int H, int T_) {
+    SeqView v;
+    v.h = bid % H;
+    if (cu) {
+        const int s = bid / H;
+        const int a = min(max(cu[s], 0), T_), e = min(max(cu[s + 1], a), T_);
+        v.b = 0;
+        v.T = e - a;
+        v.tok0 = (size_t)a;
+    } else {
+        v.b = bid / H;
+        v.T = T_;
+        v.tok0 = 0;
+    }
+    return v;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
-                int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+                int T_, int H, int dk, int dv, int C, const int *__restrict__ only, const int *__restrict__ cu) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
-    simt_fwd_body<T>(q, lf, x, h0, o, hT, T_, H, dk, dv, C, sm, blockIdx.x);
+    const SeqView v = seq_view(cu, blockIdx.x, H, T_);
+    const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
+    simt_fwd_body<T>(q + ok, lf + ok, x + ov, h0, o + ov, hT, v.T, H, dk, dv, C, sm, v.b, v.h, blockIdx.x);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
-                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only,
+                   const int *__restrict__ cu) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
-    simt_bwd_dq_body<T>(lf, x, h0, dO, dhT, dq, rs, T_, H, dk, dv, C, sm, blockIdx.x);
+    const SeqView v = seq_view(cu, blockIdx.x, H, T_);
+    const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
+    simt_bwd_dq_body<T>(lf + ok, x + ov, h0, dO + ov, dhT, dq + ok, rs, v.T, H, dk, dv, C, sm, v.b, v.h, blockIdx.x);
 }
 
 template <typename T>
@@ -353,10 +382,14 @@ __global__ void __launch_bounds__(kSimtThreads)
 simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
-                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, const int *__restrict__ only) {
+                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, const int *__restrict__ only,
+                    const int *__restrict__ cu) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
-    simt_bwd_rev_body<T>(q, lf, x, dO, dhT, dq, rs, dlf, dx, dh0, T_, H, dk, dv, C, sm, blockIdx.x);
+    const SeqView v = seq_view(cu, blockIdx.x, H, T_);
+    const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
+    simt_bwd_rev_body<T>(q + ok, lf + ok, x + ov, dO + ov, dhT, dq + ok, rs, dlf + ok, dx + ov, dh0, v.T, H, dk, dv, C,
+                         sm, v.b, v.h, blockIdx.x);
 }
 
 // ------------------------------------------------------------------ launchers
@@ -367,7 +400,7 @@ static cudaError_t launch_simt_fwd_t(const SimtFwdArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<a.B * a.H, kSimtThreads, smem, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x, a.h0,
-                                             (T *)a.o, a.hT, a.T, a.H, a.dk, a.dv, a.C, a.only);
+                                             (T *)a.o, a.hT, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu);
     return cudaGetLastError();
 }
 
@@ -385,12 +418,12 @@ static cudaError_t launch_simt_bwd_t(const SimtBwdArgs &a, cudaStream_t st) {
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     if (e != cudaSuccess) return e;
     k1<<<a.B * a.H, kSimtThreads, s1, st>>>((const T *)a.lf, (const T *)a.x, a.h0, (const T *)a.dO,
-                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C, a.only);
+                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k2<<<a.B * a.H, kSimtThreads, s2, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x,
                                             (const T *)a.dO, a.dhT, (const T *)a.dq, a.rs,
-                                            (T *)a.dlf, (T *)a.dx, a.dh0, a.T, a.H, a.dk, a.dv, a.C, a.only);
+                                            (T *)a.dlf, (T *)a.dx, a.dh0, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu);
     return cudaGetLastError();
 }
 

@@ -398,10 +398,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
         __syncthreads();
         float *sm = reinterpret_cast<float *>(smem);
         simt_bwd_dq_body<__nv_bfloat16>(p.lf, p.x, p.h0, p.dO, p.dhT, p.dq, p.rs, p.T, p.H, 128, 128,
-                                        p.simt_chunk, sm, bh);
+                                        p.simt_chunk, sm, b, h, bh);
         __syncthreads();
         simt_bwd_rev_body<__nv_bfloat16>(p.q, p.lf, p.x, p.dO, p.dhT, p.dq, p.rs, p.dlf, p.dx, p.dh0, p.T, p.H,
-                                         128, 128, p.simt_chunk, sm, bh);
+                                         128, 128, p.simt_chunk, sm, b, h, bh);
     }
 }
 
@@ -451,6 +451,7 @@ struct RevParams {
     const __nv_bfloat16 *q, *lf, *x, *dO;   // for the exact route
     __nv_bfloat16 *dq, *dlf, *dx;
     int simt_chunk;
+    const int *cu;       // packed sequences (saved mode only), or null; B = their number
 };
 
 template <bool kSaved>
@@ -466,16 +467,33 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, b = bh / p.H, h = bh - b * p.H;
-    const int N = p.ntiles;
+    const int bh = blockIdx.x, h = bh % p.H;
+    // token of chunk n: tok0 + n * kTile of batch bc; saved-state slot: slot0 + n * sstride.
+    // Packed sequences (saved mode only): rows from the sequence's end on (valid(n) < kTile)
+    // are masked in the prep and not stored.
+    int b = bh / p.H, bc = b, tok0 = 0, len = p.T, N = p.ntiles, slot0 = bh * p.ntiles, sstride = 1;
+    if (kSaved && p.cu) {
+        const int sq = bh / p.H;
+        const int a = min(max(p.cu[sq], 0), p.T), e = min(max(p.cu[sq + 1], a), p.T);
+        b = bc = 0;
+        tok0 = a;
+        len = e - a;
+        N = (len + kTile - 1) / kTile;
+        slot0 = ((a >> 7) + sq) * p.H + h;
+        sstride = p.H;
+    }
+    auto valid_rows = [&](int n) -> int { return (kSaved && p.cu) ? min(kTile, len - n * kTile) : kTile; };
     if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
         if (kSaved) {         // both sweeps here (recompute mode: in the forward-sweep kernel)
             float *sm = reinterpret_cast<float *>(smem);
-            simt_bwd_dq_body<__nv_bfloat16>(p.lf, p.x, p.h0, p.dO, p.dhT, p.dq, p.rs, p.T, p.H, 128, 128,
-                                            p.simt_chunk, sm, bh);
+            const size_t ok = (size_t)tok0 * p.H * 128;   // 0 unless packed sequences
+            const int Tl = p.cu ? len : p.T;
+            simt_bwd_dq_body<__nv_bfloat16>(p.lf + ok, p.x + ok, p.h0, p.dO + ok, p.dhT, p.dq + ok, p.rs, Tl, p.H,
+                                            128, 128, p.simt_chunk, sm, b, h, bh);
             __syncthreads();
-            simt_bwd_rev_body<__nv_bfloat16>(p.q, p.lf, p.x, p.dO, p.dhT, p.dq, p.rs, p.dlf, p.dx, p.dh0, p.T,
-                                             p.H, 128, 128, p.simt_chunk, sm, bh);
+            simt_bwd_rev_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.dO + ok, p.dhT, p.dq + ok, p.rs,
+                                             p.dlf + ok, p.dx + ok, p.dh0, Tl, p.H, 128, 128, p.simt_chunk, sm,
+                                             b, h, bh);
             if (tid == 0) atomicAdd(&g_counters[0], 1ull);
         }
         return;
@@ -515,8 +533,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         ++issued[q];
         mbar_arrive_expect_tx(bar, 2 * kTileBytes);
         for (int c = 0; c < 2; ++c) {
-            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, h, n * kTile, b);
-            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, h, n * kTile, b);
+            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, h, tok0 + n * kTile, bc);
+            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, h, tok0 + n * kTile, bc);
         }
     };
     if (tid == 0 && N > 0) {
@@ -576,10 +594,11 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // f = e^a directly, so k = 1 - f has an absolute error of a few 1e-8; E is the running
         // product of f from the range start, 1/E = e^{-b}.
         {
+            const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
             float sum = 0.0f;
             if (q4 < 3) {
 #pragma unroll 8
-                for (int i = 0; i < 32; ++i) sum += bfat(Gb, c0 + i);
+                for (int i = 0; i < 32; ++i) sum += c0 + i < vr ? bfat(Gb, c0 + i) : 0.0f;
                 m->Bpart[q4][j] = sum;
             }
             __syncthreads();
@@ -593,8 +612,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 float av[8], qv[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    av[i] = bfat(Gb, t0 + i);
-                    qv[i] = bfat(Qb, t0 + i);
+                    av[i] = t0 + i < vr ? bfat(Gb, t0 + i) : 0.0f;
+                    qv[i] = t0 + i < vr ? bfat(Qb, t0 + i) : 0.0f;
                 }
                 __nv_bfloat16 oq[8], ok2[8];
 #pragma unroll
@@ -645,13 +664,13 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             // where this thread would otherwise only wait: a prefetch holds up its issuing thread,
             // and at the top of the chunk that delayed every warp at the next block barrier.
             for (int c = 0; c < 2; ++c) {
-                if (kSaved) tma_prefetch_l2_4d(&tm_st, 64 * c, 0, 0, bh * N + n);
+                if (kSaved) tma_prefetch_l2_4d(&tm_st, 64 * c, 0, 0, slot0 + n * sstride);
                 else tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
                 if (n > 0) {
-                    tma_prefetch_l2_4d(&tm_q, 64 * c, h, (n - 1) * kTile, b);
-                    tma_prefetch_l2_4d(&tm_lf, 64 * c, h, (n - 1) * kTile, b);
-                    tma_prefetch_l2_4d(&tm_x, 64 * c, h, (n - 1) * kTile, b);
-                    tma_prefetch_l2_4d(&tm_do, 64 * c, h, (n - 1) * kTile, b);
+                    tma_prefetch_l2_4d(&tm_q, 64 * c, h, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_lf, 64 * c, h, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_x, 64 * c, h, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_do, 64 * c, h, tok0 + (n - 1) * kTile, bc);
                 }
             }
         }
@@ -763,8 +782,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             ++issued[2];
             mbar_arrive_expect_tx(&m->barDQ, kTileBytes);
             if (kSaved) {   // the saved bf16 state entering this chunk into D16
-                tma_load_4d(D16, &tm_st, &m->barDQ, 0, 0, 0, bh * N + n);
-                tma_load_4d(D16 + kBlk, &tm_st, &m->barDQ, 64, 0, 0, bh * N + n);
+                tma_load_4d(D16, &tm_st, &m->barDQ, 0, 0, 0, slot0 + n * sstride);
+                tma_load_4d(D16 + kBlk, &tm_st, &m->barDQ, 64, 0, 0, slot0 + n * sstride);
             } else {        // dq of this chunk into D16; v and dO of the next chunk into Vb, Ob
                 tma_load_4d(D16, &tm_dq, &m->barDQ, 0, h, n * kTile, b);
                 tma_load_4d(D16 + kBlk, &tm_dq, &m->barDQ, 64, h, n * kTile, b);
@@ -862,16 +881,28 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tc_fence_before();
         __syncthreads();
         if (q4 == 0) m->carry[j] += m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
-        if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
-            tma_store_4d(&tm_di, AT, 0, h, n * kTile, b);
-            tma_store_4d(&tm_di, AT + kBlk, 64, h, n * kTile, b);
-            tma_store_4d(&tm_dlf, DA, 0, h, n * kTile, b);
-            tma_store_4d(&tm_dlf, DA + kBlk, 64, h, n * kTile, b);
-            if (kSaved) {
-                tma_store_4d(&tm_dq, D16, 0, h, n * kTile, b);
-                tma_store_4d(&tm_dq, D16 + kBlk, 64, h, n * kTile, b);
+        const int vr = valid_rows(n);
+        if (vr == kTile) {
+            if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
+                tma_store_4d(&tm_di, AT, 0, h, tok0 + n * kTile, bc);
+                tma_store_4d(&tm_di, AT + kBlk, 64, h, tok0 + n * kTile, bc);
+                tma_store_4d(&tm_dlf, DA, 0, h, tok0 + n * kTile, bc);
+                tma_store_4d(&tm_dlf, DA + kBlk, 64, h, tok0 + n * kTile, bc);
+                if (kSaved) {
+                    tma_store_4d(&tm_dq, D16, 0, h, tok0 + n * kTile, bc);
+                    tma_store_4d(&tm_dq, D16 + kBlk, 64, h, tok0 + n * kTile, bc);
+                }
+                tma_store_commit();
             }
-            tma_store_commit();
+        } else {   // a packed sequence's last chunk: rows 0 .. vr-1 of the three tiles, 16 bytes a thread
+            for (int idx = tid; idx < 3 * vr * 16; idx += kRevThreads) {
+                const int tsel = idx / (vr * 16), rem = idx - tsel * vr * 16, row = rem >> 4, ch = rem & 15;
+                const uint8_t *tile = tsel == 0 ? AT : tsel == 1 ? DA : D16;
+                __nv_bfloat16 *out = tsel == 0 ? p.dx : tsel == 1 ? p.dlf : p.dq;
+                const uint4 w = *reinterpret_cast<const uint4 *>(tile + (ch >> 3) * kBlk + row * 128 +
+                                                                 (((ch & 7) ^ (row & 7)) << 4));
+                *reinterpret_cast<uint4 *>(out + ((size_t)(tok0 + n * kTile + row) * p.H + h) * 128 + 8 * ch) = w;
+            }
         }
     }
     if (!ok && tid == 0) set_status(HGRN2_ERR_TIMEOUT);
@@ -906,20 +937,24 @@ size_t tc_bwd_smem() { return tcb::fsw::kSmemBytes > tcb::rsw::kSmemBytes ? tcb:
 
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     const bool saved = a.st16 != nullptr;
+    const bool packed = a.cu != nullptr;   // saved mode only; a.B is then the number of sequences
+    if (packed && !saved) return cudaErrorInvalidValue;
+    const int Bm = packed ? 1 : a.B;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl, mst;
-    if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
-        !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mdo, a.dO, a.B, a.T, a.H) ||
-        !make_token_map(&mdq, a.dq, a.B, a.T, a.H) || !make_token_map(&mdi, a.dx, a.B, a.T, a.H) ||
-        !make_token_map(&mdl, a.dlf, a.B, a.T, a.H))
+    if (!make_token_map(&mq, a.q, Bm, a.T, a.H) || !make_token_map(&ml, a.lf, Bm, a.T, a.H) ||
+        !make_token_map(&mx, a.x, Bm, a.T, a.H) || !make_token_map(&mdo, a.dO, Bm, a.T, a.H) ||
+        !make_token_map(&mdq, a.dq, Bm, a.T, a.H) || !make_token_map(&mdi, a.dx, Bm, a.T, a.H) ||
+        !make_token_map(&mdl, a.dlf, Bm, a.T, a.H))
         return cudaErrorInvalidValue;
-    // saved states [B*H*ntiles][128][128] bf16, addressed as 128-row "token" tiles
-    if (saved && !make_token_map(&mst, a.st16, a.B * a.H * ntiles, 128, 1)) return cudaErrorInvalidValue;
+    // saved states: 128-row "token" tiles
+    if (saved && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
+        return cudaErrorInvalidValue;
     if (!saved) mst = mq;   // unused
     tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles, a.hTs, a.h0,
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
-                      (__nv_bfloat16 *)a.dx, a.simt_C};
+                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu};
     cudaError_t e;
     if (saved) {
         // one launch; the exact route of a flagged (b,h) runs in the same shared memory

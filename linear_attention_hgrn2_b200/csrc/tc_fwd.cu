@@ -81,6 +81,8 @@ struct Params {
     int nseg, tps;    // sequence segments per (b,h) and chunks per segment
     bool save;        // store bf16(S_in) of every chunk through tm_st
     float *hTs;       // with save: the final state [B*H][128][128]
+    const int *cu;    // packed sequences (or null): sequence s at tokens cu[s] .. cu[s+1]-1 of a
+                      // [1][T][H][128] tensor; CTA (s,h); no segments
 };
 
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -95,9 +97,25 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x / p.nseg, seg = blockIdx.x - bh * p.nseg, b = bh / p.H, h = bh - b * p.H;
+    const int bh = blockIdx.x / p.nseg, seg = blockIdx.x - bh * p.nseg, h = bh % p.H;
     const int g0 = seg * p.tps;                                   // first chunk of this segment
-    const int N = min(p.ntiles - g0, p.tps);                      // chunks of this segment
+    // token of chunk n: tok0 + n * kTile of batch bc; saved-state slot: slot0 + n * sstride.
+    // Packed sequences: rows from the sequence's end on (valid(n) < kTile) are masked in the
+    // prep and not stored; a sequence may start at any token.
+    int b = bh / p.H, bc = b, tok0 = g0 * kTile, len = p.T, N = min(p.ntiles - g0, p.tps);
+    int slot0 = bh * p.ntiles + g0, sstride = 1;
+    if (p.cu) {
+        const int sq = bh / p.H;
+        const int a = min(max(p.cu[sq], 0), p.T), e = min(max(p.cu[sq + 1], a), p.T);
+        b = 0;
+        bc = 0;
+        tok0 = a;
+        len = e - a;
+        N = (len + kTile - 1) / kTile;
+        slot0 = ((a >> 7) + sq) * p.H + h;
+        sstride = p.H;
+    }
+    auto valid_rows = [&](int n) -> int { return p.cu ? min(kTile, len - n * kTile) : kTile; };
     if (smem_u32(smem) & 1023u) {   // the swizzled operand layout needs 1024-byte alignment
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
@@ -147,14 +165,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 if (n >= 2 && !wait_or_abort(&m->emptyQG[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
                 mbar_arrive_expect_tx(&m->fullQG[s], 2 * kTileBytes);
                 for (int c = 0; c < 2; ++c) {
-                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, h, (g0 + n) * kTile, b);
-                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, h, (g0 + n) * kTile, b);
+                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, h, tok0 + n * kTile, bc);
+                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, h, tok0 + n * kTile, bc);
                 }
                 ++issued_qg;
                 if (n >= 2 && !wait_or_abort(&m->emptyV[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
                 mbar_arrive_expect_tx(&m->fullV[s], kTileBytes);
                 for (int c = 0; c < 2; ++c)
-                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, h, (g0 + n) * kTile, b);
+                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, h, tok0 + n * kTile, bc);
                 ++issued_v;
             }
         }
@@ -268,7 +286,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (p.save) {   // bf16(S_in) of this chunk, kept for the backward
                 named_bar_sync(2, 128);
                 if (r == 0) {
-                    const int slot = bh * p.ntiles + g0 + n;
+                    const int slot = slot0 + n * sstride;
                     tma_store_4d(&tm_st, X, 0, 0, 0, slot);
                     tma_store_4d(&tm_st, X + kBlk, 64, 0, 0, slot);
                     tma_store_commit();
@@ -309,21 +327,42 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 named_bar_sync(2, 128);
             }
             tc_fence_after();
+            const int vr = valid_rows(n);
+            if (vr == kTile) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float v[32];
-                tmem_ld32(tl + kColO + 32 * c, v);
-                tmem_wait_ld();
-                store_chunk_bf16(X, r, c, v);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&m->ofree);
-            named_bar_sync(2, 128);
-            if (r == 0) {
-                tma_store_4d(&tm_o, X, 0, h, (g0 + n) * kTile, b);
-                tma_store_4d(&tm_o, X + kBlk, 64, h, (g0 + n) * kTile, b);
-                tma_store_commit();
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tl + kColO + 32 * c, v);
+                    tmem_wait_ld();
+                    store_chunk_bf16(X, r, c, v);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&m->ofree);
+                named_bar_sync(2, 128);
+                if (r == 0) {
+                    tma_store_4d(&tm_o, X, 0, h, tok0 + n * kTile, bc);
+                    tma_store_4d(&tm_o, X + kBlk, 64, h, tok0 + n * kTile, bc);
+                    tma_store_commit();
+                }
+            } else {   // a packed sequence's last chunk: its rows only, stored by their threads
+                uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(tok0 + n * kTile + r) * p.H + h) * 128);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tl + kColO + 32 * c, v);
+                    tmem_wait_ld();
+                    if (r < vr) {
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq)
+                            dst[4 * c + qq] = make_uint4(pack_bf2(v[8 * qq], v[8 * qq + 1]),
+                                                         pack_bf2(v[8 * qq + 2], v[8 * qq + 3]),
+                                                         pack_bf2(v[8 * qq + 4], v[8 * qq + 5]),
+                                                         pack_bf2(v[8 * qq + 6], v[8 * qq + 7]));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&m->ofree);
             }
         }
         if (r == 0) tma_store_wait_all0();
@@ -362,11 +401,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const int s = n & 1;
             if (!mbar_wait(&m->fullQG[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ptid == 0) m->waited_full = n + 1;
+            const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
             if (rr < 3) {
                 float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll 8
                 for (int i = 0; i < 32; ++i) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(32 * rr + i));
+                    uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(32 * rr + i));
+                    if (32 * rr + i >= vr) w = 0u;
                     s0 += bf_lo(w);
                     s1 += bf_hi(w);
                 }
@@ -388,6 +429,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 for (int i = 0; i < 8; ++i) {
                     wa[i] = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(t0 + i));
                     wq[i] = *reinterpret_cast<const uint32_t *>(Qb[s] + eoff(t0 + i));
+                    if (t0 + i >= vr) wa[i] = wq[i] = 0u;
                 }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -440,8 +482,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     // CTA's shared memory is free for the CUDA-core chunkwise forward of the whole sequence
     if (fell_back && p.nseg == 1) {
         __syncthreads();
-        simt_fwd_body<__nv_bfloat16>(p.q, p.lf, p.x, p.h0, p.o, p.hT, p.T, p.H, 128, 128, p.simt_chunk,
-                                     reinterpret_cast<float *>(smem), bh);
+        const size_t ok = (size_t)tok0 * p.H * 128;   // 0 unless packed sequences
+        simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, p.cu ? len : p.T, p.H, 128,
+                                     128, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
     }
 }
 
@@ -668,21 +711,30 @@ size_t tc_fwd_workspace(int B, int T, int H) {
 
 size_t tc_fwd_smem() { return tcf::kSmemBytes; }
 
+// Slots of the saved bf16 chunk states: [B*H*ntiles] (slot bh * ntiles + n), or for packed
+// sequences [(T / 128 + nseq) * H] (slot ((cu[s] / 128) + s + n) * H + h: sequence s's chunks
+// never reach sequence s+1's first slot, whatever the lengths).
+int tc_saved_slots(int B, int T, int H, bool packed) {
+    return packed ? ((T >> 7) + B) * H : B * H * ((T + tcc::kTile - 1) / tcc::kTile);
+}
+
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
+    const bool packed = a.cu != nullptr;   // a.B is then the number of sequences
+    const int Bm = packed ? 1 : a.B;
     CUtensorMap mq, ml, mx, mo, mst;
-    if (!make_token_map(&mq, a.q, a.B, a.T, a.H) || !make_token_map(&ml, a.lf, a.B, a.T, a.H) ||
-        !make_token_map(&mx, a.x, a.B, a.T, a.H) || !make_token_map(&mo, a.o, a.B, a.T, a.H))
+    if (!make_token_map(&mq, a.q, Bm, a.T, a.H) || !make_token_map(&ml, a.lf, Bm, a.T, a.H) ||
+        !make_token_map(&mx, a.x, Bm, a.T, a.H) || !make_token_map(&mo, a.o, Bm, a.T, a.H))
         return cudaErrorInvalidValue;
-    // saved states [B*H*ntiles][128][128] bf16, addressed as 128-row "token" tiles
-    const int ntiles_all = (a.T + tcc::kTile - 1) / tcc::kTile;
-    if (a.st16 && !make_token_map(&mst, a.st16, a.B * a.H * ntiles_all, 128, 1)) return cudaErrorInvalidValue;
+    // saved states: 128-row "token" tiles
+    if (a.st16 && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
+        return cudaErrorInvalidValue;
     if (!a.st16) mst = mo;   // unused
     cudaError_t e = cudaFuncSetAttribute(tcf::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcf::kSmemBytes);
     if (e != cudaSuccess) return e;
-    int nseg, tps;
-    tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
+    int nseg = 1, tps = ntiles;
+    if (!packed) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);
     const int BH = a.B * a.H;
     float *U = a.seg_ws, *g = a.seg_ws ? a.seg_ws + (size_t)BH * (nseg - 1) * 16384 : nullptr;
     if (nseg > 1) {
@@ -696,7 +748,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps,
-                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr};
+                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu};
     tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     return cudaGetLastError();
 }

@@ -129,3 +129,38 @@ def make_decode(B: int, H: int, dk: int, dv: int, steps: int, dtype: torch.dtype
     del x
     S = torch.randn((B, H, dk, dv), generator=gen, device=device) * S_sigma
     return {"q": q, "i": i, "log_f": lf, "S": S, "g": graw}
+
+
+def make_varlen(lens, H: int, dk: int, dv: int, dtype: torch.dtype, lb: float, seed: int,
+                h0_sigma: float = 0.0, with_dO: bool = False, dhT_sigma: float = 0.0) -> dict:
+    """Packed variable-length sequences: CPU tensors q, log_f [total_T,H,dk], i (and dO)
+    [total_T,H,dv] in ``dtype``, cu_seqlens int32 [nseq+1] (sequence s is tokens
+    cu_seqlens[s] .. cu_seqlens[s+1]-1), optional h0, dhT [nseq,H,dk,dv] float32.
+
+    The tokens are the draws of make_inputs(1, total_T, ...) with the same seed, so a
+    sequence is a slice of one long stream; the states are drawn per sequence."""
+    lens = [int(n) for n in lens]
+    total = sum(lens)
+    inp = make_inputs(1, total, H, dk, dv, dtype, lb, seed, with_dO=with_dO)
+    out = {k: v[0] for k, v in inp.items()}
+    out["cu_seqlens"] = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    g = _gen(seed + 1)
+    if h0_sigma > 0:
+        out["h0"] = torch.from_numpy(_normal(g, (len(lens), H, dk, dv), h0_sigma))
+    if dhT_sigma > 0:
+        out["dhT"] = torch.from_numpy(_normal(g, (len(lens), H, dk, dv), dhT_sigma))
+    return out
+
+
+def document_lengths(total: int, mean: int, seed: int, min_len: int = 1) -> list:
+    """Lengths of documents packed into ``total`` tokens: exponential with the given mean
+    (many short documents, a few long ones), at least ``min_len``; the last one is cut to
+    fill ``total`` exactly."""
+    g = _gen(seed)
+    lens, used = [], 0
+    while used < total:
+        n = max(min_len, int(g.exponential(mean)))
+        n = min(n, total - used)
+        lens.append(n)
+        used += n
+    return lens

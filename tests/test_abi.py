@@ -121,3 +121,40 @@ def test_step_lb_checks_the_bound_before_any_launch(lib):
     for lb in (-0.5, 1.0, 2.0, float("nan")):
         st = lib.hgrn2_step_lb(vp(16), vp(16), vp(16), ctypes.c_float(lb), vp(16), vp(16), 1, 1, 16, 16, 0, None)
         assert st == L.ERR_INVALID_ARG, lb
+
+
+def test_packed_sequence_sizes_and_argument_checks(lib):
+    bad = ctypes.c_size_t(-1).value
+    up = lambda x: (x + 255) // 256 * 256
+    nseq, T, H = 5, 700, 3
+    # chunk-state slots: sequence s's chunk n sits at ((cu[s] >> 7) + s + n) * H + h, so
+    # (T >> 7) + nseq slot rows cover any packing of T tokens into nseq sequences
+    slots = ((T >> 7) + nseq) * H
+    want = up(slots * 128 * 128 * 2) + up(nseq * H * 128 * 128 * 4) + up(nseq * H * 4)
+    assert lib.hgrn2_saved_size_varlen(nseq, T, H, 128, 128, L.BF16) == want
+    assert lib.hgrn2_saved_size_varlen(nseq, T, H, 64, 64, L.BF16) == 0
+    assert lib.hgrn2_saved_size_varlen(nseq, 0, H, 128, 128, L.BF16) == 0
+    assert lib.hgrn2_saved_size_varlen(0, T, H, 128, 128, L.BF16) == bad
+    ws = lib.hgrn2_workspace_size_varlen(nseq, T, H, 128, 128, 64, L.BF16)
+    assert ws == up(nseq * H * 128 * 4) + up(nseq * H * 4)
+    assert lib.hgrn2_workspace_size_varlen(nseq, T, H, 128, 128, 48, L.BF16) == bad
+    vp = ctypes.c_void_p
+    args = (nseq, T, H, 128, 128, 64, L.BF16)
+    # null or misaligned cu_seqlens, a short saved buffer: rejected before any launch
+    for cu in (None, vp(20)):
+        st = lib.hgrn2_fwd_varlen(vp(16), vp(16), vp(16), None, vp(16), None, cu, *args, None, 0,
+                                  vp(256), ws, None)
+        assert st == L.ERR_INVALID_ARG
+        st = lib.hgrn2_bwd_varlen(vp(16), vp(16), vp(16), None, None, 0, vp(16), None, vp(16), vp(16),
+                                  vp(16), None, cu, *args, vp(256), ws, None)
+        assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_fwd_varlen(vp(16), vp(16), vp(16), None, vp(16), None, vp(16), *args, vp(256), want - 1,
+                              vp(256), ws, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_bwd_varlen(vp(16), vp(16), vp(16), None, vp(256), want - 1, vp(16), None, vp(16), vp(16),
+                              vp(16), None, vp(16), *args, vp(256), ws, None)
+    assert st == L.ERR_INVALID_ARG
+    # workspace shorter than hgrn2_workspace_size_varlen
+    st = lib.hgrn2_fwd_varlen(vp(16), vp(16), vp(16), None, vp(16), None, vp(16), *args, None, 0,
+                              vp(256), ws - 1, None)
+    assert st == L.ERR_INVALID_ARG
