@@ -12,7 +12,8 @@ the timed region.  Under torchrun each rank runs its own batch on its own GPU
 (data-parallel replicas, no collective on the data path): weak scaling.
 
 The same JSON line also carries the decode step (B=256, H=16, 1000 in-place
-steps of the fp32 state), end-to-end numbers through host buffers, the
+steps of the fp32 state), the training pair on packed documents of varied
+length (16,384 tokens, H=16), end-to-end numbers through host buffers, the
 roofline of the dominant call, SM clocks sampled during the timed region, and
 the CPU oracle timed on a bounded sample (rank 0, one GPU only).
 """
@@ -298,6 +299,8 @@ def run_ours(args, world, rank, local):
         out["e2e"] = run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, sv, w, world)
     if not args.no_decode:
         out["decode_step"] = run_decode(args, dev, pk)
+    if not args.no_varlen:
+        out["varlen"] = run_varlen(args, dev, pk, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_seconds)
     if rank == 0:
@@ -423,6 +426,60 @@ def run_decode(args, dev, pk):
     return res
 
 
+def run_varlen(args, dev, pk, rank):
+    """Packed documents: the training pair (hgrn2_fwd_varlen with saved states, then
+    hgrn2_bwd_varlen) over 16,384 tokens cut into documents of exponential length."""
+    import linear_attention_hgrn2_b200 as L
+    from linear_attention_hgrn2_b200 import inputs as I
+    cfg = I.VARLEN
+    lens = I.document_lengths(cfg["total_T"], cfg["mean_len"], seed=rank_seed(rank) + 7)
+    inp = I.make_varlen(lens, cfg["H"], cfg["dk"], cfg["dv"], cfg["dtype"], cfg["lb"], seed=rank_seed(rank) + 8,
+                        with_dO=True)
+    q, lf, x, dO, cu = (inp[k].to(dev) for k in ("q", "log_f", "i", "dO", "cu_seqlens"))
+    sv = L.new_saved_varlen(q, cu)
+    o = torch.empty_like(x)
+    chunk = cfg["chunk"]
+
+    def fwd_call():
+        L.fwd_varlen(q, lf, x, cu, chunk=chunk, out=o, saved=sv)
+
+    def bwd_call():
+        L.bwd_varlen(q, lf, x, dO, cu, chunk=chunk, saved=sv)
+
+    for _ in range(max(args.warmup, 3)):
+        fwd_call()
+        bwd_call()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    torch.cuda._sleep(2_000_000)
+    ev[0].record()
+    for _ in range(K):
+        fwd_call()
+        bwd_call()
+    ev[1].record()
+    for _ in range(K):
+        fwd_call()
+    ev[2].record()
+    for _ in range(K):
+        bwd_call()
+    ev[3].record()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / K
+    fwd_ms = ev[1].elapsed_time(ev[2]) / K
+    bwd_ms = ev[2].elapsed_time(ev[3]) / K
+    th = cfg["total_T"] * cfg["H"]
+    gbs_b = BWD_BYTES * th / (bwd_ms / 1e3) / 1e9
+    res = {"workload": cfg["name"], "documents": len(lens), "min_len": min(lens), "max_len": max(lens),
+           "tokens_per_s": round(cfg["total_T"] / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+           "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+           "bwd_achieved_gbs": round(gbs_b, 1), "bwd_frac": round(gbs_b / pk["hbm_gbs"], 4),
+           "calls": "hgrn2_fwd_varlen (saved states) + hgrn2_bwd_varlen", "steps": K}
+    del inp, q, lf, x, dO, sv, o
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(inp, w, budget_s=15.0):
     """The oracle (unchanged) on the host cores: fwd+bwd of whole (batch, head) sequences of the workload.
 
@@ -501,6 +558,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

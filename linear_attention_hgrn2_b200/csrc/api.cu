@@ -62,23 +62,29 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
 // hgrn2_bwd_saved): bf16 state entering every 128-token chunk, fp32 final state, and the
 // forward's exact-route flags.
 struct SavedLayout {
-    size_t hTs, flags, total;   // byte offsets (the bf16 states start at 0)
+    size_t hTs, flags, perm, total;   // byte offsets (the bf16 states start at 0)
 };
 SavedLayout saved_layout(int B, int T, int H, bool packed = false) {
     const size_t BH = (size_t)B * H, slots = (size_t)tc_saved_slots(B, T, H, packed);
     SavedLayout l;
     l.hTs = align256(slots * 128 * 128 * 2);
     l.flags = l.hTs + align256(BH * 128 * 128 * sizeof(float));
-    l.total = l.flags + align256(BH * sizeof(int));
+    l.perm = l.flags + align256(BH * sizeof(int));
+    l.total = l.perm + (packed ? align256((size_t)B * sizeof(int)) : 0);   // packed: launch order
     return l;
 }
 size_t saved_bytes_needed(int B, int T, int H, int dk, int dv, hgrn2_dtype dt) {
     return (use_tc(dk, dv, dt) && T > 0) ? saved_layout(B, T, H).total : 0;
 }
 
-// Workspace of the packed-sequence calls: rowsum(dhT * hT) [nseq*H*dk] and flags [nseq*H].
+// Workspace of the packed-sequence calls: rowsum(dhT * hT) [nseq*H*dk], flags [nseq*H] and the
+// launch order [nseq].
+size_t ws_flags_varlen(int nseq, int H, int dk) { return align256(sizeof(float) * (size_t)nseq * H * dk); }
+size_t ws_perm_varlen(int nseq, int H, int dk) {
+    return ws_flags_varlen(nseq, H, dk) + align256(sizeof(int) * (size_t)nseq * H);
+}
 size_t ws_bytes_varlen(int nseq, int H, int dk) {
-    return align256(sizeof(float) * (size_t)nseq * H * dk) + align256(sizeof(int) * (size_t)nseq * H);
+    return ws_perm_varlen(nseq, H, dk) + align256(sizeof(int) * (size_t)nseq);
 }
 
 hgrn2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HGRN2_OK : HGRN2_ERR_CUDA; }
@@ -121,17 +127,23 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
     }
     int C = simt_chunk(chunk, dk, dv, false);
     if (!C) return HGRN2_ERR_UNSUPPORTED;
+    const SavedLayout sl = saved_layout(B, T, H, cu != nullptr);
+    int *perm = nullptr;
+    if (cu) {   // longest sequences first; kept in the saved buffer for the backward
+        perm = saved ? (int *)((char *)saved + sl.perm) : (int *)((char *)workspace + ws_perm_varlen(B, H, dk));
+        if (launch_lpt_order(cu, B, T, perm, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+        g_launches += 1;
+    }
     if (use_tc(dk, dv, dtype)) {
         // tensor-core pass; (b,h) pairs whose chunk decay span is too wide are flagged
         // and recomputed right after by the exact route (same stream, in order)
-        const SavedLayout sl = saved_layout(B, T, H, cu != nullptr);
         int *flags = saved ? (int *)((char *)saved + sl.flags)
-                           : (int *)((char *)workspace + (cu ? align256(sizeof(float) * (size_t)B * H * dk) : 0));
+                           : (int *)((char *)workspace + (cu ? ws_flags_varlen(B, H, dk) : 0));
         float *seg_ws = cu ? nullptr : (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
         int nseg = 1, tps = 1;
         if (!cu) tc_fwd_segments(B, T, H, &nseg, &tps);
         TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H, C, saved,
-                    saved ? (float *)((char *)saved + sl.hTs) : nullptr, cu};
+                    saved ? (float *)((char *)saved + sl.hTs) : nullptr, cu, perm};
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         if (nseg == 1) {   // the exact route, if needed, runs inside the tensor-core kernel
@@ -140,10 +152,10 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
         }
         // segmented: aggregate, scan, segments, then the exact route for flagged (b,h)
         g_launches += 4;
-        SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags, nullptr};
+        SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags, nullptr, nullptr};
         return from_cuda(launch_simt_fwd(a, bf16, stream));
     }
-    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr, cu};
+    SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr, cu, perm};
     g_launches += 1;
     return from_cuda(launch_simt_fwd(a, bf16, stream));
 }
@@ -172,21 +184,31 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     int C = simt_chunk(chunk, dk, dv, true);
     if (!C) return HGRN2_ERR_UNSUPPORTED;
     float *rs = (float *)workspace;
+    const SavedLayout sl = saved_layout(B, T, H, cu != nullptr);
+    const int *perm = nullptr;
+    if (cu && saved) {   // the order the forward chose
+        perm = (const int *)((const char *)saved + sl.perm);
+    } else if (cu) {
+        int *p = (int *)((char *)workspace + ws_perm_varlen(B, H, dk));
+        if (launch_lpt_order(cu, B, T, p, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+        g_launches += 1;
+        perm = p;
+    }
     if (use_tc(dk, dv, dtype) && (saved || !cu)) {
         if (saved) {   // one launch: reverse sweep from the saved states (exact route inside)
-            const SavedLayout sl = saved_layout(B, T, H, cu != nullptr);
             TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs,
                         (int *)((char *)saved + sl.flags), B, T, H, C, saved,
-                        (const float *)((const char *)saved + sl.hTs), cu};
+                        (const float *)((const char *)saved + sl.hTs), cu, perm};
             g_launches += 1;
             return from_cuda(launch_tc_bwd(t, stream));
         }
         int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
-        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C, nullptr, nullptr, nullptr};
+        TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C, nullptr, nullptr, nullptr,
+                    nullptr};
         g_launches += 2;   // the exact route, if needed, runs inside the forward-sweep kernel
         return from_cuda(launch_tc_bwd(t, stream));
     }
-    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr, cu};
+    SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr, cu, perm};
     g_launches += 2;
     return from_cuda(launch_simt_bwd(a, bf16, stream));
 }

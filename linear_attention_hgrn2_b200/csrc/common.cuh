@@ -17,6 +17,17 @@ __device__ unsigned long long g_counters[2] = {0ull, 0ull};
 
 __device__ __forceinline__ void set_status(int s) { atomicCAS(&g_status, 0, s); }
 
+// Packed sequences: the sequence that CTA row r runs, perm[r] (r without perm).  An entry out
+// of [0, nseq) (a saved buffer that does not belong to this call) sets the status and maps to
+// r, so no access leaves the caller's tensors.
+__device__ __forceinline__ int packed_seq(const int *perm, int r, int nseq) {
+    if (!perm) return r;
+    const int s = perm[r];
+    if ((unsigned)s < (unsigned)nseq) return s;
+    set_status(HGRN2_ERR_DEVICE);
+    return r;
+}
+
 // ---- element conversion -----------------------------------------------------
 template <typename T> __device__ __forceinline__ float to_f(T x);
 template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }

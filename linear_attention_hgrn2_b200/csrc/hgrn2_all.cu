@@ -6,5 +6,6 @@
 #include "api.cu"
 #include "simt.cu"
 #include "step.cu"
+#include "varlen.cu"
 #include "tc_fwd.cu"
 #include "tc_bwd.cu"

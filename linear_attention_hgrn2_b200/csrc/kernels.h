@@ -14,6 +14,7 @@ struct SimtFwdArgs {
     int B, T, H, dk, dv, C;
     const int *only;   // if non-null: only (b,h) with only[b*H+h] != 0 are computed
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
+    const int *perm;   // with cu: launch order of the sequences (longest first), or null
 };
 
 struct TcFwdArgs {
@@ -28,6 +29,7 @@ struct TcFwdArgs {
     void *st16;        // out, or null: bf16 state entering every chunk, tc_saved_slots() tiles
     float *hTs;        // out (with st16): final state [B*H][128][128]
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
+    const int *perm;   // with cu: launch order of the sequences (longest first), or null
 };
 
 struct SimtBwdArgs {
@@ -39,6 +41,7 @@ struct SimtBwdArgs {
     int B, T, H, dk, dv, C;
     const int *only;   // if non-null: only (b,h) with only[b*H+h] != 0 are computed
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
+    const int *perm;   // with cu: launch order of the sequences (longest first), or null
 };
 
 struct TcBwdArgs {
@@ -53,7 +56,12 @@ struct TcBwdArgs {
     const void *st16;  // saved bf16 chunk-entry states (tc_saved_slots() tiles), or null (recompute)
     const float *hTs;  // saved final state [B*H][128][128] (with st16)
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens (needs st16)
+    const int *perm;   // with cu: launch order of the sequences (longest first), or null
 };
+
+// Longest-first launch order of packed sequences: perm[r] = the sequence that CTA row r runs,
+// ordered by decreasing number of 128-token chunks (one CTA; any nseq).
+cudaError_t launch_lpt_order(const int *cu, int nseq, int T, int *perm, cudaStream_t st);
 
 size_t simt_fwd_smem(int C, int dk, int dv);
 size_t simt_bwd_dq_smem(int C, int dk, int dv);

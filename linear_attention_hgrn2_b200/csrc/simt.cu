@@ -329,21 +329,24 @@ simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__
 
 // ------------------------------------------------------------------ kernels (one CTA per (b,h))
 // With cu (variable-length packed sequences: token tensors [total_T][H][D], sequence s at
-// tokens cu[s] .. cu[s+1]-1), CTA (s,h) runs the body on pointers offset to the sequence's
-// first token, with batch 0 and T = its length; cu values are clamped to [0, total_T].
+// tokens cu[s] .. cu[s+1]-1), CTA (r,h) runs sequence s = perm[r] (r without perm) on pointers
+// offset to the sequence's first token, with batch 0 and T = its length; its states are those
+// of pair s*H+h.  cu values are clamped to [0, total_T].
 struct SeqView {
-    int b, h, T;
+    int b, h, T, sidx;
     size_t tok0;
 };
-__device__ __forceinline__ SeqView seq_view(const int *cu, int bid, int H, int T_) {
+__device__ __forceinline__ SeqView seq_view(const int *cu, const int *perm, int bid, int H, int T_) {
     SeqView v;
     v.h = bid % H;
+    v.sidx = bid;
     if (cu) {
-        const int s = bid / H;
+        const int s = packed_seq(perm, bid / H, gridDim.x / H);
         const int a = min(max(cu[s], 0), T_), e = min(max(cu[s + 1], a), T_);
         v.b = 0;
         v.T = e - a;
         v.tok0 = (size_t)a;
+        v.sidx = s * H + v.h;
     } else {
         v.b = bid / H;
         v.T = T_;
@@ -356,12 +359,13 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_fwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
-                int T_, int H, int dk, int dv, int C, const int *__restrict__ only, const int *__restrict__ cu) {
+                int T_, int H, int dk, int dv, int C, const int *__restrict__ only, const int *__restrict__ cu,
+                const int *__restrict__ perm) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
-    const SeqView v = seq_view(cu, blockIdx.x, H, T_);
+    const SeqView v = seq_view(cu, perm, blockIdx.x, H, T_);
     const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
-    simt_fwd_body<T>(q + ok, lf + ok, x + ov, h0, o + ov, hT, v.T, H, dk, dv, C, sm, v.b, v.h, blockIdx.x);
+    simt_fwd_body<T>(q + ok, lf + ok, x + ov, h0, o + ov, hT, v.T, H, dk, dv, C, sm, v.b, v.h, v.sidx);
 }
 
 template <typename T>
@@ -369,12 +373,12 @@ __global__ void __launch_bounds__(kSimtThreads)
 simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
                    float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only,
-                   const int *__restrict__ cu) {
+                   const int *__restrict__ cu, const int *__restrict__ perm) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
-    const SeqView v = seq_view(cu, blockIdx.x, H, T_);
+    const SeqView v = seq_view(cu, perm, blockIdx.x, H, T_);
     const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
-    simt_bwd_dq_body<T>(lf + ok, x + ov, h0, dO + ov, dhT, dq + ok, rs, v.T, H, dk, dv, C, sm, v.b, v.h, blockIdx.x);
+    simt_bwd_dq_body<T>(lf + ok, x + ov, h0, dO + ov, dhT, dq + ok, rs, v.T, H, dk, dv, C, sm, v.b, v.h, v.sidx);
 }
 
 template <typename T>
@@ -383,13 +387,13 @@ simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
                     float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, const int *__restrict__ only,
-                    const int *__restrict__ cu) {
+                    const int *__restrict__ cu, const int *__restrict__ perm) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
-    const SeqView v = seq_view(cu, blockIdx.x, H, T_);
+    const SeqView v = seq_view(cu, perm, blockIdx.x, H, T_);
     const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
     simt_bwd_rev_body<T>(q + ok, lf + ok, x + ov, dO + ov, dhT, dq + ok, rs, dlf + ok, dx + ov, dh0, v.T, H, dk, dv, C,
-                         sm, v.b, v.h, blockIdx.x);
+                         sm, v.b, v.h, v.sidx);
 }
 
 // ------------------------------------------------------------------ launchers
@@ -400,7 +404,7 @@ static cudaError_t launch_simt_fwd_t(const SimtFwdArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<a.B * a.H, kSimtThreads, smem, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x, a.h0,
-                                             (T *)a.o, a.hT, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu);
+                                             (T *)a.o, a.hT, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu, a.perm);
     return cudaGetLastError();
 }
 
@@ -418,12 +422,12 @@ static cudaError_t launch_simt_bwd_t(const SimtBwdArgs &a, cudaStream_t st) {
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     if (e != cudaSuccess) return e;
     k1<<<a.B * a.H, kSimtThreads, s1, st>>>((const T *)a.lf, (const T *)a.x, a.h0, (const T *)a.dO,
-                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu);
+                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu, a.perm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k2<<<a.B * a.H, kSimtThreads, s2, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x,
                                             (const T *)a.dO, a.dhT, (const T *)a.dq, a.rs,
-                                            (T *)a.dlf, (T *)a.dx, a.dh0, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu);
+                                            (T *)a.dlf, (T *)a.dx, a.dh0, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu, a.perm);
     return cudaGetLastError();
 }
 

@@ -452,9 +452,12 @@ struct RevParams {
     __nv_bfloat16 *dq, *dlf, *dx;
     int simt_chunk;
     const int *cu;       // packed sequences (saved mode only), or null; B = their number
+    const int *perm;     // with cu: CTA row r runs sequence perm[r]
 };
 
-template <bool kSaved>
+// kPacked (saved mode only): p.cu holds packed sequences; compiled apart so the dense path
+// carries no row masks
+template <bool kSaved, bool kPacked>
 __global__ void __launch_bounds__(rsw::kRevThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
@@ -467,13 +470,16 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, h = bh % p.H;
+    int bh = blockIdx.x;
+    const int h = bh % p.H;
     // token of chunk n: tok0 + n * kTile of batch bc; saved-state slot: slot0 + n * sstride.
     // Packed sequences (saved mode only): rows from the sequence's end on (valid(n) < kTile)
     // are masked in the prep and not stored.
     int b = bh / p.H, bc = b, tok0 = 0, len = p.T, N = p.ntiles, slot0 = bh * p.ntiles, sstride = 1;
-    if (kSaved && p.cu) {
-        const int sq = bh / p.H;
+    static_assert(kSaved || !kPacked, "packed sequences need the saved states");
+    if (kPacked) {
+        const int sq = packed_seq(p.perm, bh / p.H, gridDim.x / p.H);
+        bh = sq * p.H + h;   // the pair whose states, flag and gradients this CTA owns
         const int a = min(max(p.cu[sq], 0), p.T), e = min(max(p.cu[sq + 1], a), p.T);
         b = bc = 0;
         tok0 = a;
@@ -482,12 +488,12 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         slot0 = ((a >> 7) + sq) * p.H + h;
         sstride = p.H;
     }
-    auto valid_rows = [&](int n) -> int { return (kSaved && p.cu) ? min(kTile, len - n * kTile) : kTile; };
+    auto valid_rows = [&](int n) -> int { return kPacked ? min(kTile, len - n * kTile) : kTile; };
     if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
         if (kSaved) {         // both sweeps here (recompute mode: in the forward-sweep kernel)
             float *sm = reinterpret_cast<float *>(smem);
             const size_t ok = (size_t)tok0 * p.H * 128;   // 0 unless packed sequences
-            const int Tl = p.cu ? len : p.T;
+            const int Tl = kPacked ? len : p.T;
             simt_bwd_dq_body<__nv_bfloat16>(p.lf + ok, p.x + ok, p.h0, p.dO + ok, p.dhT, p.dq + ok, p.rs, Tl, p.H,
                                             128, 128, p.simt_chunk, sm, b, h, bh);
             __syncthreads();
@@ -954,21 +960,22 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles, a.hTs, a.h0,
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
-                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu};
+                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm};
     cudaError_t e;
     if (saved) {
         // one launch; the exact route of a flagged (b,h) runs in the same shared memory
         size_t smem = tcb::rsw::kSmemBytes;
         if (simt_bwd_dq_smem(a.simt_C, 128, 128) > smem) smem = simt_bwd_dq_smem(a.simt_C, 128, 128);
         if (simt_bwd_rev_smem(a.simt_C, 128, 128) > smem) smem = simt_bwd_rev_smem(a.simt_C, 128, 128);
-        e = cudaFuncSetAttribute(tcb::rev_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        auto kern = packed ? tcb::rev_kernel<true, true> : tcb::rev_kernel<true, false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        tcb::rev_kernel<true><<<a.B * a.H, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);
+        kern<<<a.B * a.H, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);
         return cudaGetLastError();
     }
     e = cudaFuncSetAttribute(tcb::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcb::fsw::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tcb::rev_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tcb::rev_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tcb::rsw::kSmemBytes);
     if (e != cudaSuccess) return e;
     tcb::DqParams p1{a.h0, a.dhT, a.rs, a.flags, a.T, a.H, ntiles,
@@ -978,7 +985,7 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     tcb::dq_kernel<<<a.B * a.H, tcb::fsw::kDqThreads, tcb::fsw::kSmemBytes, st>>>(ml, mx, mdo, mdq, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    tcb::rev_kernel<false><<<a.B * a.H, tcb::rsw::kRevThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi,
+    tcb::rev_kernel<false, false><<<a.B * a.H, tcb::rsw::kRevThreads, tcb::rsw::kSmemBytes, st>>>(mq, ml, mx, mdo, mdq, mdi,
                                                                                            mdl, mst, p2);
     return cudaGetLastError();
 }

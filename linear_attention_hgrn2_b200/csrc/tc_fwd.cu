@@ -82,9 +82,12 @@ struct Params {
     bool save;        // store bf16(S_in) of every chunk through tm_st
     float *hTs;       // with save: the final state [B*H][128][128]
     const int *cu;    // packed sequences (or null): sequence s at tokens cu[s] .. cu[s+1]-1 of a
-                      // [1][T][H][128] tensor; CTA (s,h); no segments
+                      // [1][T][H][128] tensor; CTA (r,h) runs sequence perm[r]; no segments
+    const int *perm;
 };
 
+// kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks)
+template <bool kPacked>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o,
@@ -97,15 +100,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x / p.nseg, seg = blockIdx.x - bh * p.nseg, h = bh % p.H;
+    int bh = blockIdx.x / p.nseg;
+    const int seg = blockIdx.x - bh * p.nseg, h = bh % p.H;
     const int g0 = seg * p.tps;                                   // first chunk of this segment
     // token of chunk n: tok0 + n * kTile of batch bc; saved-state slot: slot0 + n * sstride.
     // Packed sequences: rows from the sequence's end on (valid(n) < kTile) are masked in the
     // prep and not stored; a sequence may start at any token.
     int b = bh / p.H, bc = b, tok0 = g0 * kTile, len = p.T, N = min(p.ntiles - g0, p.tps);
     int slot0 = bh * p.ntiles + g0, sstride = 1;
-    if (p.cu) {
-        const int sq = bh / p.H;
+    if (kPacked) {
+        const int sq = packed_seq(p.perm, bh / p.H, gridDim.x / p.H);
+        bh = sq * p.H + h;   // the pair whose states and flag this CTA owns
         const int a = min(max(p.cu[sq], 0), p.T), e = min(max(p.cu[sq + 1], a), p.T);
         b = 0;
         bc = 0;
@@ -115,7 +120,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         slot0 = ((a >> 7) + sq) * p.H + h;
         sstride = p.H;
     }
-    auto valid_rows = [&](int n) -> int { return p.cu ? min(kTile, len - n * kTile) : kTile; };
+    auto valid_rows = [&](int n) -> int { return kPacked ? min(kTile, len - n * kTile) : kTile; };
     if (smem_u32(smem) & 1023u) {   // the swizzled operand layout needs 1024-byte alignment
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
@@ -483,7 +488,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (fell_back && p.nseg == 1) {
         __syncthreads();
         const size_t ok = (size_t)tok0 * p.H * 128;   // 0 unless packed sequences
-        simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, p.cu ? len : p.T, p.H, 128,
+        simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T, p.H, 128,
                                      128, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
     }
 }
@@ -729,8 +734,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     if (a.st16 && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
         return cudaErrorInvalidValue;
     if (!a.st16) mst = mo;   // unused
-    cudaError_t e = cudaFuncSetAttribute(tcf::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tcf::kSmemBytes);
+    auto kern = packed ? tcf::fwd_kernel<true> : tcf::fwd_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     int nseg = 1, tps = ntiles;
@@ -748,8 +753,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps,
-                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu};
-    tcf::fwd_kernel<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
+                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm};
+    kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     return cudaGetLastError();
 }
 

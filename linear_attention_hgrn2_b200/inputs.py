@@ -50,6 +50,11 @@ LONG = Workload("long_fwd_bf16_B1_H8_T32768_d128", 1, 8, 32768, 128, 128, torch.
 DECODE = dict(name="decode_bf16_B256_H16_d128_1000steps", B=256, H=16, dk=128, dv=128,
               dtype=torch.bfloat16, lb=0.8, steps=1000, S_sigma=1.0)
 
+# packed documents: the training step's 16,384 tokens per batch cut into documents of
+# exponentially distributed length (mean 512 tokens), H=16, d=128, one state per document
+VARLEN = dict(name="varlen_train_bf16_T16384_H16_d128_docmean512", total_T=16384, H=16, dk=128, dv=128,
+              dtype=torch.bfloat16, lb=0.95, mean_len=512, chunk=64)
+
 WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG)}
 
 

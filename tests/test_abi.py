@@ -130,13 +130,14 @@ def test_packed_sequence_sizes_and_argument_checks(lib):
     # chunk-state slots: sequence s's chunk n sits at ((cu[s] >> 7) + s + n) * H + h, so
     # (T >> 7) + nseq slot rows cover any packing of T tokens into nseq sequences
     slots = ((T >> 7) + nseq) * H
-    want = up(slots * 128 * 128 * 2) + up(nseq * H * 128 * 128 * 4) + up(nseq * H * 4)
+    # + final states, flags, and the launch order of the sequences
+    want = up(slots * 128 * 128 * 2) + up(nseq * H * 128 * 128 * 4) + up(nseq * H * 4) + up(nseq * 4)
     assert lib.hgrn2_saved_size_varlen(nseq, T, H, 128, 128, L.BF16) == want
     assert lib.hgrn2_saved_size_varlen(nseq, T, H, 64, 64, L.BF16) == 0
     assert lib.hgrn2_saved_size_varlen(nseq, 0, H, 128, 128, L.BF16) == 0
     assert lib.hgrn2_saved_size_varlen(0, T, H, 128, 128, L.BF16) == bad
     ws = lib.hgrn2_workspace_size_varlen(nseq, T, H, 128, 128, 64, L.BF16)
-    assert ws == up(nseq * H * 128 * 4) + up(nseq * H * 4)
+    assert ws == up(nseq * H * 128 * 4) + up(nseq * H * 4) + up(nseq * 4)
     assert lib.hgrn2_workspace_size_varlen(nseq, T, H, 128, 128, 48, L.BF16) == bad
     vp = ctypes.c_void_p
     args = (nseq, T, H, 128, 128, 64, L.BF16)

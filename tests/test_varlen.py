@@ -86,7 +86,9 @@ def test_bf16_edge_lengths(cuda, saved, states):
     _check(inp, got, range(len(EDGE_LENS)), range(2), torch.bfloat16, 2e-2)
 
 
-def test_bf16_launch_count_is_one_per_pass(cuda):
+def test_bf16_launch_counts(cuda):
+    # forward: the longest-first order of the sequences, then one tensor-core launch; the
+    # backward reads that order and the chunk states from the saved buffer: one launch
     inp = I.make_varlen(EDGE_LENS, 2, 128, 128, torch.bfloat16, 0.9, seed=602, with_dO=True)
     g = to_cuda(inp)
     sv = L.new_saved_varlen(g["q"], g["cu_seqlens"])
@@ -95,7 +97,7 @@ def test_bf16_launch_count_is_one_per_pass(cuda):
     c_fwd = L.counters(reset=True)
     L.bwd_varlen(g["q"], g["log_f"], g["i"], g["dO"], g["cu_seqlens"], saved=sv)
     c_bwd = L.counters(reset=True)
-    assert c_fwd[2] == 1 and c_bwd[2] == 1, (c_fwd, c_bwd)
+    assert c_fwd[2] == 2 and c_bwd[2] == 1, (c_fwd, c_bwd)
     assert c_fwd[0] == 0 and c_bwd[0] == 0, (c_fwd, c_bwd)
 
 
@@ -171,3 +173,26 @@ def test_packed_equal_lengths_match_the_batched_call(cuda):
     for a, b in zip((dq, dlf, di), r2[:3]):
         assert torch.equal(pk(a), b)
     assert torch.equal(dh0, r2[3])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_repacking_in_reverse_order_changes_no_bit(cuda, dtype):
+    # each (sequence, head) pair depends on its own tokens and states only: packing the same
+    # documents in the opposite order moves them to other token offsets, other chunk-state
+    # slots and another launch order, and must reproduce every output bit for bit
+    lens = EDGE_LENS
+    inp = I.make_varlen(lens, 2, 128, 128, dtype, 0.9, seed=610, h0_sigma=0.1, with_dO=True, dhT_sigma=0.1)
+    cu = inp["cu_seqlens"].tolist()
+    order = list(reversed(range(len(lens))))
+    rev = {k: torch.cat([inp[k][cu[s]:cu[s + 1]] for s in order]) for k in ("q", "log_f", "i", "dO")}
+    rev["h0"], rev["dhT"] = inp["h0"][order].contiguous(), inp["dhT"][order].contiguous()
+    rev["cu_seqlens"] = torch.tensor([0] + list(np.cumsum([lens[s] for s in order])), dtype=torch.int32)
+    saved = dtype == torch.bfloat16
+    a = _run(to_cuda(inp), saved=saved)
+    b = _run(to_cuda(rev), saved=saved)
+    rcu = rev["cu_seqlens"].tolist()
+    for j, s in enumerate(order):
+        for name in ("o", "dq", "dlog_f", "di"):
+            assert torch.equal(a[name][cu[s]:cu[s + 1]], b[name][rcu[j]:rcu[j + 1]]), (name, s)
+        for name in ("hT", "dh0"):
+            assert torch.equal(a[name][s], b[name][j]), (name, s)
