@@ -116,3 +116,28 @@ def lower_bound_log_f(g, lb: float):
     if lb == 0.0:
         return -np.logaddexp(0.0, -g)
     return np.logaddexp(0.0, np.log(lb) - g) - np.logaddexp(0.0, -g)
+
+
+def step_bwd(q, log_f, i, S, dO, dS=None):
+    """Gradients (dq, dlog_f, di, dS_prev) of one decode step, for L = <o, dO> + <S_new, dS>
+    with (o, S_new) = step(q, log_f, i, S).  One step is the recurrence over a single token
+    starting from h0 = S, so this is bwd() at T = 1 with h0 = S and dhT = dS.
+
+    q, log_f: [B,H,dk]; i, dO: [B,H,dv]; S, dS: [B,H,dk,dv] (dS None: zero)."""
+    dq, dlf, di, dS0 = bwd(_f64(q)[:, None], _f64(log_f)[:, None], _f64(i)[:, None], _f64(dO)[:, None],
+                           h0=S, dhT=dS)
+    return dq[:, 0], dlf[:, 0], di[:, 0], dS0
+
+
+def lower_bound_dlog_f_dg(g, lb: float):
+    """d log f / d g of the lower-bounded gate (see lower_bound_log_f), in fp64.
+
+    f = lb + (1 - lb) sigmoid(g) gives df/dg = (1 - lb) sigmoid(g) sigmoid(-g), and
+    d log f / dg = (df/dg) / f.  With u = e^{-|g|} in (0, 1] this is
+        (1 - lb) u / ((1 + u) (1 + lb u))     for g >= 0,
+        (1 - lb) u / ((1 + u) (lb + u))       for g < 0,
+    a ratio of positive terms, so it keeps full relative precision in both tails."""
+    g = np.asarray(g, dtype=np.float64)
+    u = np.exp(-np.abs(g))
+    den = np.where(g >= 0, (1.0 + u) * (1.0 + lb * u), (1.0 + u) * (lb + u))
+    return (1.0 - lb) * u / den

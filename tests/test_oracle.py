@@ -249,3 +249,58 @@ def test_lower_bound_gate_matches_direct_formula_and_is_monotone():
     assert np.all(np.diff(oracle.lower_bound_log_f(gs, 0.5)) >= 0)          # increasing in g
     assert np.all(oracle.lower_bound_log_f(g, 0.9) >= oracle.lower_bound_log_f(g, 0.5))   # and in lb
     assert np.all(oracle.lower_bound_log_f(g, 0.5) <= 0) and np.all(oracle.lower_bound_log_f(g, 0.5) >= np.log(0.5))
+
+
+def test_lower_bound_gate_derivative_matches_finite_differences():
+    # central differences of lower_bound_log_f itself, and the closed form at g = 0:
+    # d log f / dg = (1 - lb) sigmoid'(0) / f(0) = (1 - lb) / 4 / ((1 + lb) / 2)
+    # (for g well below 0, log f is log lb plus a tiny term, and a difference quotient of it
+    # loses the digits; the tails are checked against their asymptotes instead)
+    g = np.linspace(-6.0, 12.0, 73)
+    h = 1e-5
+    for lb in (0.0, 0.3, 0.9, 0.99):
+        fd = (oracle.lower_bound_log_f(g + h, lb) - oracle.lower_bound_log_f(g - h, lb)) / (2 * h)
+        np.testing.assert_allclose(oracle.lower_bound_dlog_f_dg(g, lb), fd, rtol=2e-6, atol=1e-12)
+        assert oracle.lower_bound_dlog_f_dg(0.0, lb) == pytest.approx((1 - lb) / (2 * (1 + lb)), rel=1e-14)
+    # far tails: e^{-g} (1 - lb) for g -> +inf; -> 0 for g -> -inf when lb > 0, -> 1 when lb = 0
+    assert oracle.lower_bound_dlog_f_dg(30.0, 0.5) == pytest.approx(0.5 * np.exp(-30.0), rel=1e-6)
+    assert oracle.lower_bound_dlog_f_dg(-30.0, 0.5) == pytest.approx(0.5 * np.exp(-30.0) / 0.5, rel=1e-6)
+    # and it is the derivative of the log-add-exp form: sigmoid(-g) - sigmoid(log lb - g), where
+    # that difference does not cancel (g >= -4)
+    gg = np.linspace(-4.0, 12.0, 33)
+    sig = lambda x: 1.0 / (1.0 + np.exp(-x))
+    for lb in (0.3, 0.9):
+        np.testing.assert_allclose(oracle.lower_bound_dlog_f_dg(gg, lb), sig(-gg) - sig(np.log(lb) - gg), rtol=1e-9)
+    assert oracle.lower_bound_dlog_f_dg(-30.0, 0.0) == pytest.approx(1.0, rel=1e-12)
+
+
+@pytest.mark.parametrize("with_dS", [False, True])
+def test_step_bwd_matches_central_finite_differences_of_step(with_dS):
+    # L = <o, dO> + <S_new, dS> through oracle.step (the C decode step, not the BPTT code)
+    rng = np.random.default_rng(17)
+    B, H, dk, dv = 2, 1, 3, 2
+    q = rng.standard_normal((B, H, dk))
+    lf = -np.abs(rng.standard_normal((B, H, dk))) - 0.05
+    x = rng.standard_normal((B, H, dv))
+    S = rng.standard_normal((B, H, dk, dv))
+    dO = rng.standard_normal((B, H, dv))
+    dS = rng.standard_normal((B, H, dk, dv)) if with_dS else None
+
+    def loss(q_, lf_, x_, S_):
+        o, Sn = oracle.step(q_, lf_, x_, S_)
+        return float(np.sum(o * dO) + (np.sum(Sn * dS) if with_dS else 0.0))
+
+    dq, dlf, di, dSp = oracle.step_bwd(q, lf, x, S, dO, dS)
+    h = 1e-6
+    for arr, grad, idx in ((q, dq, 0), (lf, dlf, 1), (x, di, 2), (S, dSp, 3)):
+        fd = np.zeros_like(arr)
+        for k in np.ndindex(arr.shape):
+            args = [q, lf, x, S]
+            p, m = arr.copy(), arr.copy()
+            p[k] += h
+            m[k] -= h
+            args[idx] = p
+            lp = loss(*args)
+            args[idx] = m
+            fd[k] = (lp - loss(*args)) / (2 * h)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8)
