@@ -44,6 +44,9 @@ BWD_FLOPS = C_ACC * (3 * D + 2 * D) + 8 * D * D   # 172,032
 FWD_BYTES = 2 * (D + D + D + D)                   # read q, log f, i; write o = 1,024
 BWD_BYTES = 2 * (4 * D + 3 * D)                   # read q, log f, i, dO; write dq, dlog f, di = 1,792
 STEP_BYTES_PER_BH = 2 * D * D * 4 + 2 * (4 * D)   # decode: S read+write fp32, q/log f/i/o bf16 = 132,096
+# decode-step backward: S and dS read, dS_prev written (fp32); q, log f, i, dO read and dq, dlog f,
+# di written (bf16) = 198,400
+STEP_BWD_BYTES_PER_BH = 3 * D * D * 4 + 2 * (7 * D)
 
 
 def peaks():
@@ -411,7 +414,24 @@ def run_decode(args, dev, pk):
     b.record()
     torch.cuda.synchronize()
     ms_lb = a.elapsed_time(b) / steps
+    # the step backward, from the last token to the first, dS carried in place (truncated BPTT
+    # through decode steps); one state buffer stands for the per-step states (268 MB > L2)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1006)
+    dO = torch.randn((steps,) + tuple(o.shape), generator=gen, device=dev).to(cfg["dtype"])
+    dS = torch.randn(tuple(S.shape), generator=gen, device=dev)
+    for t in range(5):
+        L.step_bwd(d["q"][t], d["log_f"][t], d["i"][t], S, dO[t], dS, dS_out=dS)
+    torch.cuda.synchronize()
+    a.record()
+    for t in reversed(range(steps)):
+        L.step_bwd(d["q"][t], d["log_f"][t], d["i"][t], S, dO[t], dS, dS_out=dS)
+    b.record()
+    torch.cuda.synchronize()
+    ms_bwd = a.elapsed_time(b) / steps
     nbh = cfg["B"] * cfg["H"]
+    gbs_bwd = STEP_BWD_BYTES_PER_BH * nbh / (ms_bwd / 1e3) / 1e9
+    del dO, dS
     gbs = STEP_BYTES_PER_BH * nbh / (ms / 1e3) / 1e9
     gbs_lb = STEP_BYTES_PER_BH * nbh / (ms_lb / 1e3) / 1e9
     res = {"workload": cfg["name"], "ms_per_step": round(ms, 5), "tokens_per_s": round(cfg["B"] / (ms / 1e3), 1),
@@ -420,7 +440,10 @@ def run_decode(args, dev, pk):
            "l2": "state 268 MB > 126 MB L2, streaming loads/stores",
            "lower_bound_gate": {"call": "hgrn2_step_lb (f = lb + (1-lb) sigmoid(g) in the kernel)",
                                 "ms_per_step": round(ms_lb, 5), "achieved_gbs": round(gbs_lb, 1),
-                                "frac": round(gbs_lb / pk["hbm_gbs"], 4)}}
+                                "frac": round(gbs_lb / pk["hbm_gbs"], 4)},
+           "backward": {"call": "hgrn2_step_bwd (dS in place, last token to first)",
+                        "ms_per_step": round(ms_bwd, 5), "bytes_per_step": STEP_BWD_BYTES_PER_BH * nbh,
+                        "achieved_gbs": round(gbs_bwd, 1), "frac": round(gbs_bwd / pk["hbm_gbs"], 4)}}
     del d, S
     torch.cuda.empty_cache()
     return res

@@ -221,6 +221,31 @@ hgrn2_status hgrn2_step(const void *q, const void *log_f, const void *i, float *
 hgrn2_status hgrn2_step_lb(const void *q, const void *g, const void *i, float lb, float *S, void *o,
                            int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
 
+/* Backward of one hgrn2_step, for a loss L(o, S_new) of the step's output and updated
+ * state (truncated backpropagation through recurrent decode steps):
+ *   S       : [B,H,dk,dv] float32, the state BEFORE the step (what hgrn2_step read)
+ *   dO      : [B,H,dv] (dtype), dL/do
+ *   dS      : [B,H,dk,dv] float32, dL/dS_new, or NULL (zero)
+ *   dS_prev : out [B,H,dk,dv] float32, dL/dS, or NULL; may be dS itself (in place), else
+ *             must not overlap it (HGRN2_ERR_INVALID_ARG)
+ *   dq, dlog_f : out [B,H,dk] (dtype);  di : out [B,H,dv] (dtype)
+ * With G = dS + q dO^T:  dq = S_new dO,  dlog f = f . rowsum(G . (S - 1 i^T)),
+ * di = G^T k,  dS_prev = Diag(f) G  (the §3.2 recurrence for one token, differentiated
+ * with k = 1 - f tied to f as in §2.1).  It reads S and dS and writes dS_prev once.
+ * Same size limits as hgrn2_step. */
+hgrn2_status hgrn2_step_bwd(const void *q, const void *log_f, const void *i, const float *S,
+                            const void *dO, const float *dS, float *dS_prev,
+                            void *dq, void *dlog_f, void *di,
+                            int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
+
+/* Backward of one hgrn2_step_lb: as hgrn2_step_bwd, with the gate logits g and lb of that
+ * step in place of log f, and dg = dL/dg = dL/dlog f . (1 - lb) sigmoid(g) sigmoid(-g) / f
+ * written in place of dlog f.  0 <= lb < 1, else HGRN2_ERR_INVALID_ARG. */
+hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, float lb, const float *S,
+                               const void *dO, const float *dS, float *dS_prev,
+                               void *dq, void *dg, void *di,
+                               int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the library's device-side
  * status word of the current device: HGRN2_OK, HGRN2_ERR_TIMEOUT (a bounded
  * wait gave up) or HGRN2_ERR_DEVICE (a consistency check failed).  Returns

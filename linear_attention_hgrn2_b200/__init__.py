@@ -28,7 +28,7 @@ FP32, BF16 = 0, 1
 # Every extern "C" symbol of include/hgrn2.h.
 EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size", "hgrn2_fwd_train",
            "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_workspace_size_varlen", "hgrn2_saved_size_varlen",
-           "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_lb", "hgrn2_get_device_status",
+           "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_bwd", "hgrn2_step_lb_bwd", "hgrn2_step_lb", "hgrn2_get_device_status",
            "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
 
 _lib = None
@@ -73,6 +73,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_bwd_varlen.argtypes = [vp] * 5 + [sz] + [vp] * 7 + [i32] * 7 + [vp, sz, vp]
     lib.hgrn2_bwd_varlen.restype = i32
     lib.hgrn2_step.argtypes = [vp] * 5 + [i32] * 5 + [vp]
+    lib.hgrn2_step_bwd.argtypes = [vp] * 10 + [i32] * 5 + [vp]
+    lib.hgrn2_step_bwd.restype = i32
+    lib.hgrn2_step_lb_bwd.argtypes = [vp] * 3 + [ctypes.c_float] + [vp] * 7 + [i32] * 5 + [vp]
+    lib.hgrn2_step_lb_bwd.restype = i32
     lib.hgrn2_step.restype = i32
     lib.hgrn2_step_lb.argtypes = [vp] * 3 + [ctypes.c_float] + [vp] * 2 + [i32] * 5 + [vp]
     lib.hgrn2_step_lb.restype = i32
@@ -346,6 +350,41 @@ def step_lb(q, g, i, lb: float, S, out=None):
                            _stream())
     _raise(st, "hgrn2_step_lb")
     return o
+
+
+def _step_bwd(fn, name, q, gate, i, S, dO, dS, lb, dS_out):
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = i.shape[-1]
+    _check(q, "q")
+    _check(gate, "gate", q.dtype, q.shape)
+    _check(i, "i", q.dtype, (B, H, dv))
+    _check(S, "S", torch.float32, (B, H, dk, dv))
+    _check(dO, "dO", q.dtype, (B, H, dv))
+    if dS is not None:
+        _check(dS, "dS", torch.float32, (B, H, dk, dv))
+    if dS_out is None:
+        dS_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check(dS_out, "dS_prev", torch.float32, (B, H, dk, dv))
+    dq = torch.empty_like(q)
+    dg = torch.empty_like(q)
+    di = torch.empty_like(i)
+    args = [_ptr(q), _ptr(gate), _ptr(i)] + ([ctypes.c_float(lb)] if lb is not None else [])
+    st = fn(*args, _ptr(S), _ptr(dO), _ptr(dS), _ptr(dS_out), _ptr(dq), _ptr(dg), _ptr(di), B, H, dk, dv, _dt(q),
+            _stream())
+    _raise(st, name)
+    return dq, dg, di, dS_out
+
+
+def step_bwd(q, log_f, i, S, dO, dS=None, dS_out=None):
+    """Backward of step(): S is the state before the step, dO = dL/do, dS = dL/dS_new (None:
+    zero).  Returns (dq, dlog_f, di, dS_prev); dS_out (may be dS, for in place) receives dS_prev."""
+    return _step_bwd(load_library().hgrn2_step_bwd, "hgrn2_step_bwd", q, log_f, i, S, dO, dS, None, dS_out)
+
+
+def step_lb_bwd(q, g, i, lb: float, S, dO, dS=None, dS_out=None):
+    """Backward of step_lb(): as step_bwd, returning dL/dg in place of dlog_f."""
+    return _step_bwd(load_library().hgrn2_step_lb_bwd, "hgrn2_step_lb_bwd", q, g, i, S, dO, dS, lb, dS_out)
 
 
 def device_status() -> int:

@@ -227,6 +227,28 @@ hgrn2_status step_impl(const void *q, const void *lf, const void *i, float *S, v
     return from_cuda(launch_step(q, lf, i, S, o, B, H, dk, dv, dtype == HGRN2_BF16, gate_lb, lb, stream));
 }
 
+hgrn2_status step_bwd_impl(const void *q, const void *lf, const void *i, const float *S, const void *dO,
+                           const float *dS, float *dS_prev, void *dq, void *dlf, void *di, int B, int H, int dk,
+                           int dv, hgrn2_dtype dtype, bool gate_lb, float lb, cudaStream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
+    if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
+    if (dk > 128 || dv > 128 || (dv & 3)) return HGRN2_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    if (!q || !lf || !i || !S || !dO || !dq || !dlf || !di) return HGRN2_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, lf, i, S, dO, dS, dS_prev, dq, dlf, di};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    // dS_prev is dS itself or does not overlap it
+    if (dS && dS_prev && dS != dS_prev) {
+        const size_t n = sizeof(float) * (size_t)B * H * dk * dv;
+        const char *a = (const char *)dS, *b = (const char *)dS_prev;
+        if (a < b + n && b < a + n) return HGRN2_ERR_INVALID_ARG;
+    }
+    StepBwdArgs a{q, lf, i, S, dO, dS, dS_prev, dq, dlf, di, B, H, dk, dv, gate_lb, lb};
+    g_launches += 1;
+    return from_cuda(launch_step_bwd(a, dtype == HGRN2_BF16, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -320,6 +342,19 @@ hgrn2_status hgrn2_step_lb(const void *q, const void *g, const void *i, float lb
                            int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream) {
     if (!(lb >= 0.0f && lb < 1.0f)) return HGRN2_ERR_INVALID_ARG;   // also rejects NaN
     return step_impl(q, g, i, S, o, B, H, dk, dv, dtype, true, lb, stream);
+}
+
+hgrn2_status hgrn2_step_bwd(const void *q, const void *log_f, const void *i, const float *S, const void *dO,
+                            const float *dS, float *dS_prev, void *dq, void *dlog_f, void *di, int B, int H, int dk,
+                            int dv, hgrn2_dtype dtype, cudaStream_t stream) {
+    return step_bwd_impl(q, log_f, i, S, dO, dS, dS_prev, dq, dlog_f, di, B, H, dk, dv, dtype, false, 0.0f, stream);
+}
+
+hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, float lb, const float *S, const void *dO,
+                               const float *dS, float *dS_prev, void *dq, void *dg, void *di, int B, int H, int dk,
+                               int dv, hgrn2_dtype dtype, cudaStream_t stream) {
+    if (!(lb >= 0.0f && lb < 1.0f)) return HGRN2_ERR_INVALID_ARG;
+    return step_bwd_impl(q, g, i, S, dO, dS, dS_prev, dq, dg, di, B, H, dk, dv, dtype, true, lb, stream);
 }
 
 hgrn2_status hgrn2_get_device_status(cudaStream_t stream) {

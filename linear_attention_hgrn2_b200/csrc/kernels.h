@@ -59,6 +59,19 @@ struct TcBwdArgs {
     const int *perm;   // with cu: launch order of the sequences (longest first), or null
 };
 
+struct StepBwdArgs {
+    const void *q, *lf, *x;   // lf: log f, or the gate logits g with gate_lb
+    const float *S;           // state before the step
+    const void *dO;
+    const float *dS;          // dL/dS_new or null
+    float *dS_prev;           // out or null; may equal dS
+    void *dq, *dlf, *dx;      // dlf: d log f, or dL/dg with gate_lb
+    int B, H, dk, dv;
+    bool gate_lb;
+    float lb;
+};
+cudaError_t launch_step_bwd(const StepBwdArgs &a, bool bf16, cudaStream_t st);
+
 // Longest-first launch order of packed sequences: perm[r] = the sequence that CTA row r runs,
 // ordered by decreasing number of 128-token chunks (one CTA; any nseq).
 cudaError_t launch_lpt_order(const int *cu, int nseq, int T, int *perm, cudaStream_t st);

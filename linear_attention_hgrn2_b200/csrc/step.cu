@@ -101,6 +101,139 @@ step_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restri
     }
 }
 
+// Backward of one step, for L(o, S_new) with dO = dL/do and dS = dL/dS_new (null: zero), from
+// the state S the step read.  Per element, with G = dS + q dO^T the whole gradient at S_new:
+//
+//   dq[j]      = sum_v S_new[j,v] dO[v]              (S_new recomputed from S, f, k, i)
+//   dL/df[j]   = sum_v G[j,v] (S[j,v] - i[v])        (k = 1 - f moves against f)
+//   di[v]      = sum_j G[j,v] k[j]
+//   dS_prev    = Diag(f) G
+//
+// and d log f = f dL/df, or, for the lower-bounded gate, dL/dg = dL/df (1 - lb) sigmoid(g)
+// sigmoid(-g).  The two d_k x d_v fp32 reads and one write dominate: 3 * 4 * d_k * d_v bytes per
+// (batch, head).  Same thread layout as the step: each thread holds 16-byte column groups of up
+// to 16 rows of S and dS in registers, all loads issued first (128 KB in flight per block);
+// row sums go through padded shared memory, column sums through a second buffer.
+// dS_prev may be dS itself (each element is read before its owner thread overwrites it), so
+// neither pointer is declared restrict.
+template <typename T, bool kLB>
+__global__ void __launch_bounds__(kStepThreads, 1)
+step_bwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
+                const float *__restrict__ S, const T *__restrict__ dO, const float *dS, float *dSp,
+                T *__restrict__ dq, T *__restrict__ dlf, T *__restrict__ dx, int dk, int dv, float lb) {
+    __shared__ float sq[128], sf[128], sk[128], sd[128];
+    __shared__ float rows[2][128][33];   // [dq | dL/df][row][column group], padded against conflicts
+    __shared__ float4 red[kStepThreads];
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    const int CG = dv >> 2, RG = kStepThreads / CG;
+    const int cg = tid % CG, rg = tid / CG;
+    const bool active = rg < RG;
+    const size_t so = (size_t)bh * dk * dv;
+    const float4 *Sp = reinterpret_cast<const float4 *>(S + so);
+    const float4 *Dp = dS ? reinterpret_cast<const float4 *>(dS + so) : nullptr;
+    float4 *Pp = dSp ? reinterpret_cast<float4 *>(dSp + so) : nullptr;
+
+    float4 r[kStepMaxRows], d[kStepMaxRows];
+#pragma unroll
+    for (int i = 0; i < kStepMaxRows; ++i) {
+        const int j = rg + i * RG;
+        if (active && j < dk) {
+            r[i] = __ldcs(Sp + (size_t)j * CG + cg);
+            d[i] = Dp ? __ldcs(Dp + (size_t)j * CG + cg) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    for (int j = tid; j < dk; j += kStepThreads) {
+        const float a = to_f<T>(lf[(size_t)bh * dk + j]);
+        if (kLB) {   // a = g; sp = sigmoid(|g|), sn = sigmoid(-|g|)
+            const float e = expf(-fabsf(a)), sp = 1.0f / (1.0f + e), sn = e * sp;
+            sf[j] = lb + (1.0f - lb) * (a >= 0.0f ? sp : sn);
+            sk[j] = (1.0f - lb) * (a >= 0.0f ? sn : sp);
+            sd[j] = (1.0f - lb) * sp * sn;   // df/dg
+        } else {
+            const float f = expf(a);
+            sf[j] = f;
+            sk[j] = one_minus_exp(a);
+            sd[j] = f;                       // df/dlog f
+        }
+        sq[j] = to_f<T>(q[(size_t)bh * dk + j]);
+    }
+    float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), gv = xv;
+    if (active) {
+        const T *xp = x + (size_t)bh * dv + 4 * cg, *gp = dO + (size_t)bh * dv + 4 * cg;
+        xv = make_float4(to_f<T>(xp[0]), to_f<T>(xp[1]), to_f<T>(xp[2]), to_f<T>(xp[3]));
+        gv = make_float4(to_f<T>(gp[0]), to_f<T>(gp[1]), to_f<T>(gp[2]), to_f<T>(gp[3]));
+    }
+    __syncthreads();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);   // di partial over this thread's rows
+#pragma unroll
+    for (int i = 0; i < kStepMaxRows; ++i) {
+        const int j = rg + i * RG;
+        if (active && j < dk) {
+            const float f = sf[j], k = sk[j], qj = sq[j];
+            const float4 s = r[i];
+            float4 G = d[i];
+            G.x = fmaf(qj, gv.x, G.x);
+            G.y = fmaf(qj, gv.y, G.y);
+            G.z = fmaf(qj, gv.z, G.z);
+            G.w = fmaf(qj, gv.w, G.w);
+            const float pq = fmaf(f, s.x, k * xv.x) * gv.x + fmaf(f, s.y, k * xv.y) * gv.y +
+                             fmaf(f, s.z, k * xv.z) * gv.z + fmaf(f, s.w, k * xv.w) * gv.w;
+            const float pf = G.x * (s.x - xv.x) + G.y * (s.y - xv.y) + G.z * (s.z - xv.z) + G.w * (s.w - xv.w);
+            acc.x = fmaf(G.x, k, acc.x);
+            acc.y = fmaf(G.y, k, acc.y);
+            acc.z = fmaf(G.z, k, acc.z);
+            acc.w = fmaf(G.w, k, acc.w);
+            if (Pp) __stcs(Pp + (size_t)j * CG + cg, make_float4(f * G.x, f * G.y, f * G.z, f * G.w));
+            rows[0][j][cg] = pq;
+            rows[1][j][cg] = pf;
+        }
+    }
+    red[tid] = acc;
+    __syncthreads();
+    for (int t = tid; t < 2 * dk; t += kStepThreads) {
+        const int w = t >= dk, j = t - w * dk;
+        float sum = 0.0f;
+        for (int c = 0; c < CG; ++c) sum += rows[w][j][c];
+        if (w == 0)
+            dq[(size_t)bh * dk + j] = from_f<T>(sum);
+        else
+            dlf[(size_t)bh * dk + j] = from_f<T>(sum * sd[j]);
+    }
+    if (tid < CG) {
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int g = 0; g < RG; ++g) {
+            const float4 p = red[g * CG + tid];
+            s.x += p.x; s.y += p.y; s.z += p.z; s.w += p.w;
+        }
+        T *op = dx + (size_t)bh * dv + 4 * tid;
+        op[0] = from_f<T>(s.x);
+        op[1] = from_f<T>(s.y);
+        op[2] = from_f<T>(s.z);
+        op[3] = from_f<T>(s.w);
+    }
+}
+
+template <typename T>
+static void launch_step_bwd_t(const StepBwdArgs &a, int grid, cudaStream_t st) {
+    if (a.gate_lb)
+        step_bwd_kernel<T, true><<<grid, kStepThreads, 0, st>>>(
+            (const T *)a.q, (const T *)a.lf, (const T *)a.x, a.S, (const T *)a.dO, a.dS, a.dS_prev, (T *)a.dq,
+            (T *)a.dlf, (T *)a.dx, a.dk, a.dv, a.lb);
+    else
+        step_bwd_kernel<T, false><<<grid, kStepThreads, 0, st>>>(
+            (const T *)a.q, (const T *)a.lf, (const T *)a.x, a.S, (const T *)a.dO, a.dS, a.dS_prev, (T *)a.dq,
+            (T *)a.dlf, (T *)a.dx, a.dk, a.dv, 0.0f);
+}
+
+cudaError_t launch_step_bwd(const StepBwdArgs &a, bool bf16, cudaStream_t st) {
+    const int grid = a.B * a.H;
+    if (bf16)
+        launch_step_bwd_t<__nv_bfloat16>(a, grid, st);
+    else
+        launch_step_bwd_t<float>(a, grid, st);
+    return cudaGetLastError();
+}
+
 template <typename T>
 static void launch_step_t(const void *q, const void *lf, const void *x, float *S, void *o, int grid, int dk, int dv,
                           bool gate_lb, float lb, cudaStream_t st) {

@@ -169,3 +169,12 @@ def document_lengths(total: int, mean: int, seed: int, min_len: int = 1) -> list
         lens.append(n)
         used += n
     return lens
+
+
+def make_step_grads(B: int, H: int, dk: int, dv: int, dtype: torch.dtype, seed: int,
+                    dS_sigma: float = 1.0) -> dict:
+    """Upstream gradients of one decode step: dO [B,H,dv] in ``dtype`` (N(0,1)) and
+    dS [B,H,dk,dv] float32 (N(0, dS_sigma^2)), drawn in that order."""
+    g = _gen(seed)
+    return {"dO": _to(_normal(g, (B, H, dv)), dtype),
+            "dS": torch.from_numpy(_normal(g, (B, H, dk, dv), dS_sigma))}

@@ -159,3 +159,29 @@ def test_packed_sequence_sizes_and_argument_checks(lib):
     st = lib.hgrn2_fwd_varlen(vp(16), vp(16), vp(16), None, vp(16), None, vp(16), *args, None, 0,
                               vp(256), ws - 1, None)
     assert st == L.ERR_INVALID_ARG
+
+
+def test_step_bwd_argument_checks_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    B, H, dk, dv = 2, 2, 16, 16
+    n = B * H * dk * dv * 4
+    base = [vp(256), vp(256), vp(256), vp(4096)]   # q, log_f, i, S
+    # dS_prev overlapping dS without being it
+    st = lib.hgrn2_step_bwd(*base, vp(256), vp(1 << 20), vp((1 << 20) + 16), vp(256), vp(256), vp(256),
+                            B, H, dk, dv, L.FP32, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_step_bwd(*base, vp(256), vp(1 << 20), vp((1 << 20) + n - 16), vp(256), vp(256), vp(256),
+                            B, H, dk, dv, L.FP32, None)
+    assert st == L.ERR_INVALID_ARG
+    # null outputs, dv not a multiple of 4, misaligned state
+    st = lib.hgrn2_step_bwd(*base, vp(256), None, None, None, vp(256), vp(256), B, H, dk, dv, L.FP32, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_step_bwd(*base, vp(256), None, None, vp(256), vp(256), vp(256), B, H, dk, 6, L.FP32, None)
+    assert st == L.ERR_UNSUPPORTED
+    st = lib.hgrn2_step_bwd(vp(256), vp(256), vp(256), vp(4100), vp(256), None, None, vp(256), vp(256), vp(256),
+                            B, H, dk, dv, L.FP32, None)
+    assert st == L.ERR_INVALID_ARG
+    for lb in (-0.1, 1.0, float("nan")):
+        st = lib.hgrn2_step_lb_bwd(vp(256), vp(256), vp(256), ctypes.c_float(lb), vp(4096), vp(256), None, None,
+                                   vp(256), vp(256), vp(256), B, H, dk, dv, L.FP32, None)
+        assert st == L.ERR_INVALID_ARG, lb
