@@ -233,7 +233,7 @@ hgrn2_status step_bwd_impl(const void *q, const void *lf, const void *i, const f
     if (B < 1 || H < 1 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
     if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
     if (dk > 128 || dv > 128 || (dv & 3)) return HGRN2_ERR_UNSUPPORTED;
-    if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 29)) return HGRN2_ERR_UNSUPPORTED;   // two blocks per (b,h)
     if (!q || !lf || !i || !S || !dO || !dq || !dlf || !di) return HGRN2_ERR_INVALID_ARG;
     const void *ptrs[] = {q, lf, i, S, dO, dS, dS_prev, dq, dlf, di};
     for (const void *p : ptrs)

@@ -22,6 +22,8 @@
 // gate is kept above a lower bound lb in [0, 1)) is formed here, with
 // k = 1 - f = (1 - lb) sigmoid(-g) taken directly, so neither f nor k loses precision and
 // no separate pass writes log f.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -111,39 +113,48 @@ step_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restri
 //
 // and d log f = f dL/df, or, for the lower-bounded gate, dL/dg = dL/df (1 - lb) sigmoid(g)
 // sigmoid(-g).  The two d_k x d_v fp32 reads and one write dominate: 3 * 4 * d_k * d_v bytes per
-// (batch, head).  Same thread layout as the step: each thread holds 16-byte column groups of up
-// to 16 rows of S and dS in registers, all loads issued first (128 KB in flight per block);
-// row sums go through padded shared memory, column sums through a second buffer.
+// (batch, head).  A cluster of two blocks shares one (batch, head), each block half of the rows,
+// so that a thread holds at most 8 rows of S and dS (16-byte column groups, all loads issued
+// first) and two blocks fit on an SM: one block's loads overlap the other's arithmetic and
+// stores.  Row sums stay inside a block (padded shared memory); the column sum di crosses the
+// pair once, through distributed shared memory.
 // dS_prev may be dS itself (each element is read before its owner thread overwrites it), so
 // neither pointer is declared restrict.
+constexpr int kStepBwdRows = 8;   // ceil(64 * 32 / 256): half of d_k <= 128 rows, d_v <= 128
+
 template <typename T, bool kLB>
-__global__ void __launch_bounds__(kStepThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kStepThreads, 2)
 step_bwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ S, const T *__restrict__ dO, const float *dS, float *dSp,
                 T *__restrict__ dq, T *__restrict__ dlf, T *__restrict__ dx, int dk, int dv, float lb) {
-    __shared__ float sq[128], sf[128], sk[128], sd[128];
-    __shared__ float rows[2][128][33];   // [dq | dL/df][row][column group], padded against conflicts
+    __shared__ float sq[64], sf[64], sk[64], sd[64];
+    __shared__ float rows[2][64][33];   // [dq | dL/df][row][column group], padded against conflicts
     __shared__ float4 red[kStepThreads];
-    const int bh = blockIdx.x, tid = threadIdx.x;
+    __shared__ float4 peer[32];         // the other block's di partials (block 0 only)
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int bh = blockIdx.x >> 1, tid = threadIdx.x;
+    const int half = (dk + 1) >> 1, j0 = rank ? half : 0, nr = rank ? dk - half : half;
     const int CG = dv >> 2, RG = kStepThreads / CG;
     const int cg = tid % CG, rg = tid / CG;
     const bool active = rg < RG;
-    const size_t so = (size_t)bh * dk * dv;
+    const size_t so = ((size_t)bh * dk + j0) * dv;
     const float4 *Sp = reinterpret_cast<const float4 *>(S + so);
     const float4 *Dp = dS ? reinterpret_cast<const float4 *>(dS + so) : nullptr;
     float4 *Pp = dSp ? reinterpret_cast<float4 *>(dSp + so) : nullptr;
 
-    float4 r[kStepMaxRows], d[kStepMaxRows];
+    float4 r[kStepBwdRows], d[kStepBwdRows];
 #pragma unroll
-    for (int i = 0; i < kStepMaxRows; ++i) {
+    for (int i = 0; i < kStepBwdRows; ++i) {
         const int j = rg + i * RG;
-        if (active && j < dk) {
+        if (active && j < nr) {
             r[i] = __ldcs(Sp + (size_t)j * CG + cg);
             d[i] = Dp ? __ldcs(Dp + (size_t)j * CG + cg) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    for (int j = tid; j < dk; j += kStepThreads) {
-        const float a = to_f<T>(lf[(size_t)bh * dk + j]);
+    const size_t vo = (size_t)bh * dk + j0;   // this block's first row in the [B,H,dk] vectors
+    for (int j = tid; j < nr; j += kStepThreads) {
+        const float a = to_f<T>(lf[vo + j]);
         if (kLB) {   // a = g; sp = sigmoid(|g|), sn = sigmoid(-|g|)
             const float e = expf(-fabsf(a)), sp = 1.0f / (1.0f + e), sn = e * sp;
             sf[j] = lb + (1.0f - lb) * (a >= 0.0f ? sp : sn);
@@ -155,7 +166,7 @@ step_bwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__re
             sk[j] = one_minus_exp(a);
             sd[j] = f;                       // df/dlog f
         }
-        sq[j] = to_f<T>(q[(size_t)bh * dk + j]);
+        sq[j] = to_f<T>(q[vo + j]);
     }
     float4 xv = make_float4(0.f, 0.f, 0.f, 0.f), gv = xv;
     if (active) {
@@ -166,9 +177,9 @@ step_bwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__re
     __syncthreads();
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);   // di partial over this thread's rows
 #pragma unroll
-    for (int i = 0; i < kStepMaxRows; ++i) {
+    for (int i = 0; i < kStepBwdRows; ++i) {
         const int j = rg + i * RG;
-        if (active && j < dk) {
+        if (active && j < nr) {
             const float f = sf[j], k = sk[j], qj = sq[j];
             const float4 s = r[i];
             float4 G = d[i];
@@ -190,26 +201,31 @@ step_bwd_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *__re
     }
     red[tid] = acc;
     __syncthreads();
-    for (int t = tid; t < 2 * dk; t += kStepThreads) {
-        const int w = t >= dk, j = t - w * dk;
+    for (int t = tid; t < 2 * nr; t += kStepThreads) {
+        const int w = t >= nr, j = t - w * nr;
         float sum = 0.0f;
         for (int c = 0; c < CG; ++c) sum += rows[w][j][c];
         if (w == 0)
-            dq[(size_t)bh * dk + j] = from_f<T>(sum);
+            dq[vo + j] = from_f<T>(sum);
         else
-            dlf[(size_t)bh * dk + j] = from_f<T>(sum * sd[j]);
+            dlf[vo + j] = from_f<T>(sum * sd[j]);
     }
+    float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
     if (tid < CG) {
-        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int g = 0; g < RG; ++g) {
             const float4 p = red[g * CG + tid];
-            s.x += p.x; s.y += p.y; s.z += p.z; s.w += p.w;
+            part.x += p.x; part.y += p.y; part.z += p.z; part.w += p.w;
         }
+        if (rank == 1) cluster.map_shared_rank(peer, 0)[tid] = part;
+    }
+    cluster.sync();   // block 1's partials are in block 0's shared memory
+    if (rank == 0 && tid < CG) {
+        const float4 p = peer[tid];
         T *op = dx + (size_t)bh * dv + 4 * tid;
-        op[0] = from_f<T>(s.x);
-        op[1] = from_f<T>(s.y);
-        op[2] = from_f<T>(s.z);
-        op[3] = from_f<T>(s.w);
+        op[0] = from_f<T>(part.x + p.x);
+        op[1] = from_f<T>(part.y + p.y);
+        op[2] = from_f<T>(part.z + p.z);
+        op[3] = from_f<T>(part.w + p.w);
     }
 }
 
@@ -226,7 +242,7 @@ static void launch_step_bwd_t(const StepBwdArgs &a, int grid, cudaStream_t st) {
 }
 
 cudaError_t launch_step_bwd(const StepBwdArgs &a, bool bf16, cudaStream_t st) {
-    const int grid = a.B * a.H;
+    const int grid = 2 * a.B * a.H;   // a cluster of two blocks per (batch, head)
     if (bf16)
         launch_step_bwd_t<__nv_bfloat16>(a, grid, st);
     else
