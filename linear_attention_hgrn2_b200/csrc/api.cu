@@ -45,7 +45,9 @@ hgrn2_status check_common(int B, int T, int H, int dk, int dv, int chunk, hgrn2_
 }
 
 // The bf16 tensor-core route takes d_k = d_v = 128; everything else runs the exact route.
-bool use_tc(int dk, int dv, hgrn2_dtype dt) { return dt == HGRN2_BF16 && dk == 128 && dv == 128; }
+// The tensor-core route: bf16 with d_k = d_v = 128, or 64 (run as 128-wide tiles whose second
+// half is held at zero).
+bool use_tc(int dk, int dv, hgrn2_dtype dt) { return dt == HGRN2_BF16 && dk == dv && (dk == 128 || dk == 64); }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -141,9 +143,9 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
                            : (int *)((char *)workspace + (cu ? ws_flags_varlen(B, H, dk) : 0));
         float *seg_ws = cu ? nullptr : (float *)((char *)workspace + align256(sizeof(int) * (size_t)B * H));
         int nseg = 1, tps = 1;
-        if (!cu) tc_fwd_segments(B, T, H, &nseg, &tps);
+        if (!cu && dk == 128) tc_fwd_segments(B, T, H, &nseg, &tps);   // as the launcher decides
         TcFwdArgs t{q, log_f, i, h0, o, hT, flags, seg_ws, B, T, H, C, saved,
-                    saved ? (float *)((char *)saved + sl.hTs) : nullptr, cu, perm};
+                    saved ? (float *)((char *)saved + sl.hTs) : nullptr, cu, perm, dk};
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         if (nseg == 1) {   // the exact route, if needed, runs inside the tensor-core kernel
@@ -194,17 +196,19 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
         g_launches += 1;
         perm = p;
     }
-    if (use_tc(dk, dv, dtype) && (saved || !cu)) {
+    // without saved states only d = 128 has a tensor-core backward (recompute); the rest take the
+    // exact route
+    if (use_tc(dk, dv, dtype) && (saved || (!cu && dk == 128))) {
         if (saved) {   // one launch: reverse sweep from the saved states (exact route inside)
             TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs,
                         (int *)((char *)saved + sl.flags), B, T, H, C, saved,
-                        (const float *)((const char *)saved + sl.hTs), cu, perm};
+                        (const float *)((const char *)saved + sl.hTs), cu, perm, dk};
             g_launches += 1;
             return from_cuda(launch_tc_bwd(t, stream));
         }
         int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
         TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, flags, B, T, H, C, nullptr, nullptr, nullptr,
-                    nullptr};
+                    nullptr, 128};
         g_launches += 2;   // the exact route, if needed, runs inside the forward-sweep kernel
         return from_cuda(launch_tc_bwd(t, stream));
     }

@@ -30,6 +30,7 @@ struct TcFwdArgs {
     float *hTs;        // out (with st16): final state [B*H][128][128]
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
     const int *perm;   // with cu: launch order of the sequences (longest first), or null
+    int D;             // head size d_k = d_v: 128 or 64
 };
 
 struct SimtBwdArgs {
@@ -57,6 +58,7 @@ struct TcBwdArgs {
     const float *hTs;  // saved final state [B*H][128][128] (with st16)
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens (needs st16)
     const int *perm;   // with cu: launch order of the sequences (longest first), or null
+    int D;             // head size d_k = d_v: 128 or 64 (64: saved-state mode only)
 };
 
 struct StepBwdArgs {

@@ -453,6 +453,8 @@ struct RevParams {
     int simt_chunk;
     const int *cu;       // packed sequences (saved mode only), or null; B = their number
     const int *perm;     // with cu: CTA row r runs sequence perm[r]
+    int D;               // head size d_k = d_v: 128, or 64 (saved mode; the second 64-column half of
+                         // every operand tile is held at zero, which is exactly neutral)
 };
 
 // kPacked (saved mode only): p.cu holds packed sequences; compiled apart so the dense path
@@ -492,13 +494,13 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
         if (kSaved) {         // both sweeps here (recompute mode: in the forward-sweep kernel)
             float *sm = reinterpret_cast<float *>(smem);
-            const size_t ok = (size_t)tok0 * p.H * 128;   // 0 unless packed sequences
+            const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
             const int Tl = kPacked ? len : p.T;
             simt_bwd_dq_body<__nv_bfloat16>(p.lf + ok, p.x + ok, p.h0, p.dO + ok, p.dhT, p.dq + ok, p.rs, Tl, p.H,
-                                            128, 128, p.simt_chunk, sm, b, h, bh);
+                                            p.D, p.D, p.simt_chunk, sm, b, h, bh);
             __syncthreads();
             simt_bwd_rev_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.dO + ok, p.dhT, p.dq + ok, p.rs,
-                                             p.dlf + ok, p.dx + ok, p.dh0, Tl, p.H, 128, 128, p.simt_chunk, sm,
+                                             p.dlf + ok, p.dx + ok, p.dh0, Tl, p.H, p.D, p.D, p.simt_chunk, sm,
                                              b, h, bh);
             if (tid == 0) atomicAdd(&g_counters[0], 1ull);
         }
@@ -525,6 +527,15 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tmem_alloc(&m->tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    const int nblk = p.D >> 6;   // 64-column blocks loaded and stored per tile
+    if (nblk == 1) {             // d = 64: the unloaded halves of the input tiles stay zero
+        for (int i = tid; i < 4 * (int)(kBlk / 16); i += kRevThreads) {
+            const int t = i / (int)(kBlk / 16), o = i - t * (int)(kBlk / 16);
+            uint8_t *base = t == 0 ? Qb : t == 1 ? Gb : t == 2 ? Vb : Ob;
+            reinterpret_cast<uint4 *>(base + kBlk)[o] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -537,8 +548,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     auto issue2 = [&](uint8_t *d0, const CUtensorMap *t0, uint8_t *d1, const CUtensorMap *t1, uint64_t *bar,
                       int q, int n) {
         ++issued[q];
-        mbar_arrive_expect_tx(bar, 2 * kTileBytes);
-        for (int c = 0; c < 2; ++c) {
+        mbar_arrive_expect_tx(bar, 2 * nblk * kBlk);
+        for (int c = 0; c < nblk; ++c) {
             tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, h, tok0 + n * kTile, bc);
             tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, h, tok0 + n * kTile, bc);
         }
@@ -550,15 +561,15 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
         float v[32];
         float part = 0.0f;   // saved mode: this quarter's share of rowsum(dhT * hT)
-        if (p.dhT) {
-            const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * 128 + j) * 128 + c0);
+        if (p.dhT && j < p.D && c0 < p.D) {   // d x d; zero outside for d = 64
+            const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * p.D + j) * p.D + c0);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 a = src[i];
                 v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
             }
             if (kSaved) {
-                const float4 *hs = reinterpret_cast<const float4 *>(p.hTs + ((size_t)bh * 128 + j) * 128 + c0);
+                const float4 *hs = reinterpret_cast<const float4 *>(p.hTs + ((size_t)bh * p.D + j) * p.D + c0);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 a = hs[i];
@@ -890,24 +901,22 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const int vr = valid_rows(n);
         if (vr == kTile) {
             if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
-                tma_store_4d(&tm_di, AT, 0, h, tok0 + n * kTile, bc);
-                tma_store_4d(&tm_di, AT + kBlk, 64, h, tok0 + n * kTile, bc);
-                tma_store_4d(&tm_dlf, DA, 0, h, tok0 + n * kTile, bc);
-                tma_store_4d(&tm_dlf, DA + kBlk, 64, h, tok0 + n * kTile, bc);
-                if (kSaved) {
-                    tma_store_4d(&tm_dq, D16, 0, h, tok0 + n * kTile, bc);
-                    tma_store_4d(&tm_dq, D16 + kBlk, 64, h, tok0 + n * kTile, bc);
+                for (int c = 0; c < nblk; ++c) {
+                    tma_store_4d(&tm_di, AT + c * kBlk, 64 * c, h, tok0 + n * kTile, bc);
+                    tma_store_4d(&tm_dlf, DA + c * kBlk, 64 * c, h, tok0 + n * kTile, bc);
+                    if (kSaved) tma_store_4d(&tm_dq, D16 + c * kBlk, 64 * c, h, tok0 + n * kTile, bc);
                 }
                 tma_store_commit();
             }
         } else {   // a packed sequence's last chunk: rows 0 .. vr-1 of the three tiles, 16 bytes a thread
-            for (int idx = tid; idx < 3 * vr * 16; idx += kRevThreads) {
-                const int tsel = idx / (vr * 16), rem = idx - tsel * vr * 16, row = rem >> 4, ch = rem & 15;
+            const int nch = 8 * nblk;   // 16-byte chunks per row
+            for (int idx = tid; idx < 3 * vr * nch; idx += kRevThreads) {
+                const int tsel = idx / (vr * nch), rem = idx - tsel * vr * nch, row = rem / nch, ch = rem - row * nch;
                 const uint8_t *tile = tsel == 0 ? AT : tsel == 1 ? DA : D16;
                 __nv_bfloat16 *out = tsel == 0 ? p.dx : tsel == 1 ? p.dlf : p.dq;
                 const uint4 w = *reinterpret_cast<const uint4 *>(tile + (ch >> 3) * kBlk + row * 128 +
                                                                  (((ch & 7) ^ (row & 7)) << 4));
-                *reinterpret_cast<uint4 *>(out + ((size_t)(tok0 + n * kTile + row) * p.H + h) * 128 + 8 * ch) = w;
+                *reinterpret_cast<uint4 *>(out + ((size_t)(tok0 + n * kTile + row) * p.H + h) * p.D + 8 * ch) = w;
             }
         }
     }
@@ -918,12 +927,12 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             for (int k = waited[q]; k < issued[q]; ++k) mbar_wait(bars[q], k & 1, 2000000u);
     }
     if (tid == kStoreTid) tma_store_wait_all0();
-    if (ok && n < 0 && p.dh0) {
+    if (ok && n < 0 && p.dh0 && j < p.D && c0 < p.D) {   // warp-uniform
         tc_fence_after();
         float v[32];
         tmem_ld32(tl + kColDS + c0, v);
         tmem_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * 128 + j) * 128 + c0);
+        float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * p.D + j) * p.D + c0);
 #pragma unroll
         for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
@@ -944,14 +953,14 @@ size_t tc_bwd_smem() { return tcb::fsw::kSmemBytes > tcb::rsw::kSmemBytes ? tcb:
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     const bool saved = a.st16 != nullptr;
     const bool packed = a.cu != nullptr;   // saved mode only; a.B is then the number of sequences
-    if (packed && !saved) return cudaErrorInvalidValue;
-    const int Bm = packed ? 1 : a.B;
+    if ((packed || a.D != 128) && !saved) return cudaErrorInvalidValue;
+    const int Bm = packed ? 1 : a.B, D = a.D;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl, mst;
-    if (!make_token_map(&mq, a.q, Bm, a.T, a.H) || !make_token_map(&ml, a.lf, Bm, a.T, a.H) ||
-        !make_token_map(&mx, a.x, Bm, a.T, a.H) || !make_token_map(&mdo, a.dO, Bm, a.T, a.H) ||
-        !make_token_map(&mdq, a.dq, Bm, a.T, a.H) || !make_token_map(&mdi, a.dx, Bm, a.T, a.H) ||
-        !make_token_map(&mdl, a.dlf, Bm, a.T, a.H))
+    if (!make_token_map(&mq, a.q, Bm, a.T, a.H, D) || !make_token_map(&ml, a.lf, Bm, a.T, a.H, D) ||
+        !make_token_map(&mx, a.x, Bm, a.T, a.H, D) || !make_token_map(&mdo, a.dO, Bm, a.T, a.H, D) ||
+        !make_token_map(&mdq, a.dq, Bm, a.T, a.H, D) || !make_token_map(&mdi, a.dx, Bm, a.T, a.H, D) ||
+        !make_token_map(&mdl, a.dlf, Bm, a.T, a.H, D))
         return cudaErrorInvalidValue;
     // saved states: 128-row "token" tiles
     if (saved && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
@@ -960,13 +969,13 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles, a.hTs, a.h0,
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
-                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm};
+                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm, D};
     cudaError_t e;
     if (saved) {
         // one launch; the exact route of a flagged (b,h) runs in the same shared memory
         size_t smem = tcb::rsw::kSmemBytes;
-        if (simt_bwd_dq_smem(a.simt_C, 128, 128) > smem) smem = simt_bwd_dq_smem(a.simt_C, 128, 128);
-        if (simt_bwd_rev_smem(a.simt_C, 128, 128) > smem) smem = simt_bwd_rev_smem(a.simt_C, 128, 128);
+        if (simt_bwd_dq_smem(a.simt_C, D, D) > smem) smem = simt_bwd_dq_smem(a.simt_C, D, D);
+        if (simt_bwd_rev_smem(a.simt_C, D, D) > smem) smem = simt_bwd_rev_smem(a.simt_C, D, D);
         auto kern = packed ? tcb::rev_kernel<true, true> : tcb::rev_kernel<true, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

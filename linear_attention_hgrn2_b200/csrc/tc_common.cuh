@@ -129,12 +129,14 @@ inline PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 4-D map over a [B][T][H][128] bf16 tensor: box = 64 features x 1 head x 128 tokens x 1 batch.
-inline bool make_token_map(CUtensorMap *map, const void *ptr, int B, int T, int H) {
+// 4-D map over a [B][T][H][D] bf16 tensor (D = 128 or 64): box = 64 features x 1 head x 128 tokens
+// x 1 batch, so a 128 x 128 tile takes D / 64 boxes.
+inline bool make_token_map(CUtensorMap *map, const void *ptr, int B, int T, int H, int D = 128) {
     auto enc = get_encode();
     if (!enc) return false;
-    cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)T * H * 256};
+    const cuuint64_t row = (cuuint64_t)D * 2;   // bytes of one (token, head) row: 256 or 128
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {row, (cuuint64_t)H * row, (cuuint64_t)T * H * row};
     cuuint32_t box[4] = {64, 1, 128, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, es,

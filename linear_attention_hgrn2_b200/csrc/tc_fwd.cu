@@ -84,6 +84,8 @@ struct Params {
     const int *cu;    // packed sequences (or null): sequence s at tokens cu[s] .. cu[s+1]-1 of a
                       // [1][T][H][128] tensor; CTA (r,h) runs sequence perm[r]; no segments
     const int *perm;
+    int D;            // head size d_k = d_v: 128, or 64 (the second 64-column half of every operand
+                      // tile is held at zero: log f = 0, q = i = 0 there, exactly neutral)
 };
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks)
@@ -153,6 +155,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tmem_alloc(&m->tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    const int nblk = p.D >> 6;   // 64-column blocks loaded and stored per tile
+    if (nblk == 1) {             // d = 64: the unloaded halves of the input tiles stay zero
+        for (int i = tid; i < 6 * (int)(kBlk / 16); i += kFwdThreads) {
+            const int t = i / (int)(kBlk / 16), o = i - t * (int)(kBlk / 16);
+            uint8_t *base = t < 2 ? Qb[t] : t < 4 ? Gb[t - 2] : Vb[t - 4];
+            reinterpret_cast<uint4 *>(base + kBlk)[o] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -168,15 +179,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 // q and log f once the state MMA of chunk n-2 has read Qt, Kt; i once its last
                 // MMA has read v
                 if (n >= 2 && !wait_or_abort(&m->emptyQG[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
-                mbar_arrive_expect_tx(&m->fullQG[s], 2 * kTileBytes);
-                for (int c = 0; c < 2; ++c) {
+                mbar_arrive_expect_tx(&m->fullQG[s], 2 * nblk * kBlk);
+                for (int c = 0; c < nblk; ++c) {
                     tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, h, tok0 + n * kTile, bc);
                     tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, h, tok0 + n * kTile, bc);
                 }
                 ++issued_qg;
                 if (n >= 2 && !wait_or_abort(&m->emptyV[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
-                mbar_arrive_expect_tx(&m->fullV[s], kTileBytes);
-                for (int c = 0; c < 2; ++c)
+                mbar_arrive_expect_tx(&m->fullV[s], nblk * kBlk);
+                for (int c = 0; c < nblk; ++c)
                     tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, h, tok0 + n * kTile, bc);
                 ++issued_v;
             }
@@ -236,14 +247,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // ------------------------------------------------------------ TMEM warps
         const int quad = warp & 3, r = 32 * quad + lane;             // TMEM lane = tile row
         const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
-        {   // S = h0 / scanned incoming state / 0
-            const float *init = seg == 0 ? (p.h0 ? p.h0 + (size_t)bh * 16384 : nullptr)
+        {   // S = h0 / scanned incoming state / 0 (d x d, zero outside for d = 64)
+            const float *init = seg == 0 ? (p.h0 ? p.h0 + (size_t)bh * p.D * p.D : nullptr)
                                          : p.Sin + ((size_t)bh * (p.nseg - 1) + seg - 1) * 16384;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
-                if (init) {
-                    const float4 *src = reinterpret_cast<const float4 *>(init + (size_t)r * 128 + 32 * c);
+                if (init && r < p.D && 32 * c < p.D) {
+                    const float4 *src = reinterpret_cast<const float4 *>(init + (size_t)r * p.D + 32 * c);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float4 a = src[i];
@@ -347,13 +358,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 named_bar_sync(2, 128);
                 if (r == 0) {
                     tma_store_4d(&tm_o, X, 0, h, tok0 + n * kTile, bc);
-                    tma_store_4d(&tm_o, X + kBlk, 64, h, tok0 + n * kTile, bc);
+                    if (nblk == 2) tma_store_4d(&tm_o, X + kBlk, 64, h, tok0 + n * kTile, bc);
                     tma_store_commit();
                 }
             } else {   // a packed sequence's last chunk: its rows only, stored by their threads
-                uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(tok0 + n * kTile + r) * p.H + h) * 128);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(tok0 + n * kTile + r) * p.H + h) * p.D);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    if (32 * c >= p.D) break;
                     float v[32];
                     tmem_ld32(tl + kColO + 32 * c, v);
                     tmem_wait_ld();
@@ -374,12 +386,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // the last state MMA must be complete before hT is read or TMEM is released
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        if (n == N && (p.hT || p.hTs) && seg == p.nseg - 1) {
+        if (n == N && (p.hT || p.hTs) && seg == p.nseg - 1 && r < p.D) {   // warp-uniform
             const float e = e_cur;
-            float *dst = p.hT ? p.hT + ((size_t)bh * 128 + r) * 128 : nullptr;
-            float *dsv = p.hTs ? p.hTs + ((size_t)bh * 128 + r) * 128 : nullptr;
+            float *dst = p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
+            float *dsv = p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
+                if (32 * c >= p.D) break;
                 float v[32];
                 tmem_ld32(tl + kColS + 32 * c, v);
                 tmem_wait_ld();
@@ -487,9 +500,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     // CTA's shared memory is free for the CUDA-core chunkwise forward of the whole sequence
     if (fell_back && p.nseg == 1) {
         __syncthreads();
-        const size_t ok = (size_t)tok0 * p.H * 128;   // 0 unless packed sequences
-        simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T, p.H, 128,
-                                     128, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
+        const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
+        simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T, p.H, p.D,
+                                     p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
     }
 }
 
@@ -727,8 +740,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     const bool packed = a.cu != nullptr;   // a.B is then the number of sequences
     const int Bm = packed ? 1 : a.B;
     CUtensorMap mq, ml, mx, mo, mst;
-    if (!make_token_map(&mq, a.q, Bm, a.T, a.H) || !make_token_map(&ml, a.lf, Bm, a.T, a.H) ||
-        !make_token_map(&mx, a.x, Bm, a.T, a.H) || !make_token_map(&mo, a.o, Bm, a.T, a.H))
+    if (!make_token_map(&mq, a.q, Bm, a.T, a.H, a.D) || !make_token_map(&ml, a.lf, Bm, a.T, a.H, a.D) ||
+        !make_token_map(&mx, a.x, Bm, a.T, a.H, a.D) || !make_token_map(&mo, a.o, Bm, a.T, a.H, a.D))
         return cudaErrorInvalidValue;
     // saved states: 128-row "token" tiles
     if (a.st16 && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
@@ -739,7 +752,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     int nseg = 1, tps = ntiles;
-    if (!packed) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);
+    if (!packed && a.D == 128) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);   // d = 64: one CTA per (b,h)
     const int BH = a.B * a.H;
     float *U = a.seg_ws, *g = a.seg_ws ? a.seg_ws + (size_t)BH * (nseg - 1) * 16384 : nullptr;
     if (nseg > 1) {
@@ -753,7 +766,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps,
-                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm};
+                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D};
     kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     return cudaGetLastError();
 }

@@ -100,7 +100,9 @@ def test_saved_size_and_training_pair_argument_checks(lib):
     up = lambda x: (x + 255) // 256 * 256
     want = up(B * H * nt * 128 * 128 * 2) + up(B * H * 128 * 128 * 4) + up(B * H * 4)
     assert f(B, T, H, 128, 128, L.BF16) == want
-    assert f(B, T, H, 64, 64, L.BF16) == 0        # exact route: nothing saved
+    assert f(B, T, H, 64, 64, L.BF16) == want     # d = 64: the same zero-padded 128 x 128 slots
+    assert f(B, T, H, 32, 32, L.BF16) == 0        # exact route: nothing saved
+    assert f(B, T, H, 64, 128, L.BF16) == 0
     assert f(B, T, H, 128, 128, L.FP32) == 0
     assert f(B, 0, H, 128, 128, L.BF16) == 0
     assert f(0, T, H, 128, 128, L.BF16) == bad
@@ -133,7 +135,8 @@ def test_packed_sequence_sizes_and_argument_checks(lib):
     # + final states, flags, and the launch order of the sequences
     want = up(slots * 128 * 128 * 2) + up(nseq * H * 128 * 128 * 4) + up(nseq * H * 4) + up(nseq * 4)
     assert lib.hgrn2_saved_size_varlen(nseq, T, H, 128, 128, L.BF16) == want
-    assert lib.hgrn2_saved_size_varlen(nseq, T, H, 64, 64, L.BF16) == 0
+    assert lib.hgrn2_saved_size_varlen(nseq, T, H, 64, 64, L.BF16) == want
+    assert lib.hgrn2_saved_size_varlen(nseq, T, H, 32, 32, L.BF16) == 0
     assert lib.hgrn2_saved_size_varlen(nseq, 0, H, 128, 128, L.BF16) == 0
     assert lib.hgrn2_saved_size_varlen(0, T, H, 128, 128, L.BF16) == bad
     ws = lib.hgrn2_workspace_size_varlen(nseq, T, H, 128, 128, 64, L.BF16)
