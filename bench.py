@@ -13,7 +13,8 @@ the timed region.  Under torchrun each rank runs its own batch on its own GPU
 
 The same JSON line also carries the decode step (B=256, H=16, 1000 in-place
 steps of the fp32 state), the training pair on packed documents of varied
-length (16,384 tokens, H=16), end-to-end numbers through host buffers, the
+length (16,384 tokens, H=16), the training pair with 64-wide heads (H=32),
+end-to-end numbers through host buffers, the
 roofline of the dominant call, SM clocks sampled during the timed region, and
 the CPU oracle timed on a bounded sample (rank 0, one GPU only).
 """
@@ -304,6 +305,8 @@ def run_ours(args, world, rank, local):
         out["decode_step"] = run_decode(args, dev, pk)
     if not args.no_varlen:
         out["varlen"] = run_varlen(args, dev, pk, rank)
+    if not args.no_d64:
+        out["head_dim_64"] = run_d64(args, dev, pk, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_seconds)
     if rank == 0:
@@ -503,6 +506,55 @@ def run_varlen(args, dev, pk, rank):
     return res
 
 
+def run_d64(args, dev, pk, rank):
+    """The training pair with 64-wide heads at the same hidden size (B=8, H=32, T=2048, d=64)."""
+    import linear_attention_hgrn2_b200 as L
+    from linear_attention_hgrn2_b200 import inputs as I
+    w = I.TRAIN_D64
+    inp = I.make_workload(w, seed=rank_seed(rank) + 9)
+    q, lf, x, dO = (inp[k].to(dev) for k in ("q", "log_f", "i", "dO"))
+    sv = L.new_saved(q)
+    o = torch.empty_like(x)
+
+    def fwd_call():
+        L.fwd(q, lf, x, chunk=w.chunk, out=o, saved=sv)
+
+    def bwd_call():
+        L.bwd(q, lf, x, dO, chunk=w.chunk, saved=sv)
+
+    for _ in range(max(args.warmup, 3)):
+        fwd_call()
+        bwd_call()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    torch.cuda._sleep(2_000_000)
+    ev[0].record()
+    for _ in range(K):
+        fwd_call()
+        bwd_call()
+    ev[1].record()
+    for _ in range(K):
+        fwd_call()
+    ev[2].record()
+    for _ in range(K):
+        bwd_call()
+    ev[3].record()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / K
+    fwd_ms = ev[1].elapsed_time(ev[2]) / K
+    bwd_ms = ev[2].elapsed_time(ev[3]) / K
+    th = w.B * w.T * w.H
+    bwd_bytes = 2 * 7 * w.dk * th   # read q, log f, i, dO; write dq, dlog f, di (bf16)
+    gbs_b = bwd_bytes / (bwd_ms / 1e3) / 1e9
+    res = {"workload": w.name, "tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+           "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4), "bwd_achieved_gbs": round(gbs_b, 1),
+           "bwd_frac": round(gbs_b / pk["hbm_gbs"], 4), "calls": "hgrn2_fwd_train + hgrn2_bwd_saved", "steps": K}
+    del inp, q, lf, x, dO, sv, o
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(inp, w, budget_s=15.0):
     """The oracle (unchanged) on the host cores: fwd+bwd of whole (batch, head) sequences of the workload.
 
@@ -582,6 +634,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-d64", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

@@ -55,7 +55,10 @@ DECODE = dict(name="decode_bf16_B256_H16_d128_1000steps", B=256, H=16, dk=128, d
 VARLEN = dict(name="varlen_train_bf16_T16384_H16_d128_docmean512", total_T=16384, H=16, dk=128, dv=128,
               dtype=torch.bfloat16, lb=0.95, mean_len=512, chunk=64)
 
-WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG)}
+# the training workload's hidden size (2048) with 64-wide heads
+TRAIN_D64 = Workload("train_fwdbwd_bf16_B8_H32_T2048_d64", 8, 32, 2048, 64, 64, torch.bfloat16, 0.95, 64, bwd=True)
+
+WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG, TRAIN_D64)}
 
 
 def _gen(seed: int) -> np.random.Generator:
