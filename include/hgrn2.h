@@ -72,9 +72,12 @@ typedef enum {
     HGRN2_BF16 = 1
 } hgrn2_dtype;
 
-/* Bytes of device workspace that hgrn2_fwd (want_bwd = 0) or hgrn2_bwd
- * (want_bwd = 1) needs for these sizes.  May be 0.  Returns (size_t)-1 for
- * invalid or unsupported arguments.  Host-only, no CUDA call. */
+/* Bytes of device workspace that hgrn2_fwd (want_bwd = 0), hgrn2_bwd (want_bwd = 1)
+ * or hgrn2_bwd_saved (want_bwd = 2; never more than for 1) needs for these sizes.
+ * May be 0.  For bf16 heads of 64, the hgrn2_bwd size includes room for the chunk
+ * states and an o scratch: that backward runs the tensor-core forward into them,
+ * then the saved-state backward.  Returns (size_t)-1 for invalid or unsupported
+ * arguments.  Host-only, no CUDA call. */
 size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
                             hgrn2_dtype dtype, int want_bwd);
 

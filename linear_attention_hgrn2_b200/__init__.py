@@ -133,6 +133,7 @@ def _raise(status: int, where: str):
 
 
 def workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, want_bwd=False) -> int:
+    """want_bwd: False (forward), True (backward), or 2 (backward given saved states)."""
     n = load_library().hgrn2_workspace_size(B, T, H, dk, dv, chunk,
                                             BF16 if dtype == torch.bfloat16 else FP32, int(want_bwd))
     if n == ctypes.c_size_t(-1).value:
@@ -144,6 +145,11 @@ def _workspace(nbytes: int, device) -> torch.Tensor | None:
     if nbytes == 0:
         return None
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _caller_workspace(t: torch.Tensor) -> torch.Tensor:
+    _check(t, "workspace", torch.uint8)
+    return t
 
 
 def saved_size(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
@@ -181,7 +187,9 @@ def fwd(q, log_f, i, h0=None, want_hT=False, chunk=64, out=None, workspace=None,
     _check(o, "o", q.dtype, (B, T, H, dv))
     hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_hT else None
     nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, False)
-    ws = workspace if workspace is not None else _workspace(nws, q.device)
+    ws = _caller_workspace(workspace) if workspace is not None else _workspace(nws, q.device)
+    if workspace is not None:
+        nws = workspace.numel()   # the library checks it against what it needs
     if saved is not None:
         _check(saved, "saved", torch.uint8)
         st = lib.hgrn2_fwd_train(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(o), _ptr(hT), _ptr(saved),
@@ -214,8 +222,10 @@ def bwd(q, log_f, i, dO, h0=None, dhT=None, want_dh0=False, chunk=64, workspace=
     dlf = torch.empty_like(q)
     di = torch.empty_like(i)
     dh0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
-    nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, True)
-    ws = workspace if workspace is not None else _workspace(nws, q.device)
+    nws = workspace_size(B, T, H, dk, dv, chunk, q.dtype, 2 if saved is not None else True)
+    ws = _caller_workspace(workspace) if workspace is not None else _workspace(nws, q.device)
+    if workspace is not None:
+        nws = workspace.numel()   # the library checks it against what it needs
     if saved is not None:
         _check(saved, "saved", torch.uint8)
         st = lib.hgrn2_bwd_saved(_ptr(q), _ptr(log_f), _ptr(i), _ptr(h0), _ptr(saved), saved.numel(),

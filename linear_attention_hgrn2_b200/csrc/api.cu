@@ -51,15 +51,6 @@ bool use_tc(int dk, int dv, hgrn2_dtype dt) { return dt == HGRN2_BF16 && dk == d
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd) {
-    (void)T; (void)chunk;
-    size_t bytes = 0;
-    if (want_bwd) bytes += align256(sizeof(float) * (size_t)B * H * dk);   // rowsum(dhT * hT)
-    if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
-    if (!want_bwd && use_tc(dk, dv, dt) && T > 0) bytes += align256(tc_fwd_workspace(B, T, H));  // segments
-    return bytes;
-}
-
 // Saved-state buffer of the tensor-core route (written by hgrn2_fwd_train, read by
 // hgrn2_bwd_saved): bf16 state entering every 128-token chunk, fp32 final state, and the
 // forward's exact-route flags.
@@ -75,6 +66,27 @@ SavedLayout saved_layout(int B, int T, int H, bool packed = false) {
     l.total = l.perm + (packed ? align256((size_t)B * sizeof(int)) : 0);   // packed: launch order
     return l;
 }
+
+// Workspace of hgrn2_fwd / hgrn2_bwd.  The backward of 64-wide heads without saved states
+// (tc64) runs the tensor-core forward into a saved-state buffer and an o scratch inside the
+// workspace, then the saved-state backward; the no-alloc backward passes tc64 = false and
+// takes the exact route instead.
+size_t ws_bytes_base(int B, int H, int dk, int dv, hgrn2_dtype dt, int want_bwd) {
+    size_t bytes = 0;
+    if (want_bwd) bytes += align256(sizeof(float) * (size_t)B * H * dk);   // rowsum(dhT * hT)
+    if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
+    return bytes;
+}
+size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd,
+                       bool tc64 = true) {
+    (void)chunk;
+    size_t bytes = ws_bytes_base(B, H, dk, dv, dt, want_bwd);
+    if (!want_bwd && use_tc(dk, dv, dt) && dk == 128 && T > 0) bytes += align256(tc_fwd_workspace(B, T, H));
+    if (want_bwd && tc64 && use_tc(dk, dv, dt) && dk == 64 && T > 0)   // saved states + o scratch
+        bytes += saved_layout(B, T, H).total + align256((size_t)B * T * H * dv * 2);
+    return bytes;
+}
+
 size_t saved_bytes_needed(int B, int T, int H, int dk, int dv, hgrn2_dtype dt) {
     return (use_tc(dk, dv, dt) && T > 0) ? saved_layout(B, T, H).total : 0;
 }
@@ -100,7 +112,8 @@ extern "C" {
 size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
                             int want_bwd) {
     if (check_common(B, T, H, dk, dv, chunk, dtype) != HGRN2_OK) return (size_t)-1;
-    return ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, want_bwd);
+    if (want_bwd < 0 || want_bwd > 2) return (size_t)-1;
+    return ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, want_bwd != 0, want_bwd != 2);
 }
 
 }  // extern "C"
@@ -166,16 +179,28 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
 hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
                       const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
                       int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
-                      size_t ws_bytes, cudaStream_t stream, const int *cu = nullptr) {
+                      size_t ws_bytes, cudaStream_t stream, const int *cu = nullptr, bool tc64 = true) {
     hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !log_f || !i || !dO || !dq || !dlog_f || !di)) return HGRN2_ERR_INVALID_ARG;
     const void *ptrs[] = {q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
-    size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
+    size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1, tc64 && !saved);
     if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
     const bool bf16 = dtype == HGRN2_BF16;
+    if (T > 0 && !saved && !cu && tc64 && use_tc(dk, dv, dtype) && dk == 64) {
+        // 64-wide heads: the tensor-core forward keeps the chunk states in the workspace (its o
+        // goes to scratch there too), then the saved-state backward reads them
+        const size_t base = ws_bytes_base(B, H, dk, dv, dtype, 1);
+        char *sv = (char *)workspace + base;
+        void *o2 = sv + saved_layout(B, T, H).total;
+        hgrn2_status st = fwd_impl(q, log_f, i, h0, o2, nullptr, sv, B, T, H, dk, dv, chunk, dtype, workspace, base,
+                                   stream);
+        if (st != HGRN2_OK) return st;
+        return bwd_impl(q, log_f, i, h0, sv, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype, workspace,
+                        base, stream);
+    }
     if (T == 0) {
         if (!dh0) return HGRN2_OK;
         size_t n = sizeof(float) * (size_t)B * H * dk * dv;
@@ -435,11 +460,13 @@ extern "C" hgrn2_status hgrn2_bwd_noalloc(const void *q, const void *log_f, cons
                                           hgrn2_dtype dtype, cudaStream_t stream) {
     hgrn2_status s = check_common(B, T, H, dk, dv, chunk, dtype);
     if (s != HGRN2_OK) return s;
-    const size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1);
+    // 64-wide heads take the exact route here: their tensor-core recompute needs a workspace
+    // the size of the chunk states
+    const size_t need = ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1, false);
     if (need > kNoAllocScratchBytes) return HGRN2_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     s = noalloc_scratch(&scratch);
     if (s != HGRN2_OK) return s;
-    return hgrn2_bwd(q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype, scratch,
-                     kNoAllocScratchBytes, stream);
+    return bwd_impl(q, log_f, i, h0, nullptr, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype, scratch,
+                    kNoAllocScratchBytes, stream, nullptr, false);
 }

@@ -188,3 +188,18 @@ def test_step_bwd_argument_checks_before_any_launch(lib):
         st = lib.hgrn2_step_lb_bwd(vp(256), vp(256), vp(256), ctypes.c_float(lb), vp(4096), vp(256), None, None,
                                    vp(256), vp(256), vp(256), B, H, dk, dv, L.FP32, None)
         assert st == L.ERR_INVALID_ARG, lb
+
+
+def test_workspace_size_of_the_backward_with_saved_states(lib):
+    f = lib.hgrn2_workspace_size
+    bad = ctypes.c_size_t(-1).value
+    up = lambda x: (x + 255) // 256 * 256
+    B, T, H = 2, 300, 3
+    for d in (128, 64):
+        assert f(B, T, H, d, d, 64, L.BF16, 2) <= f(B, T, H, d, d, 64, L.BF16, 1)
+    # d = 64 without saved states: room for the chunk states and an o scratch on top
+    extra = lib.hgrn2_saved_size(B, T, H, 64, 64, L.BF16) + up(B * T * H * 64 * 2)
+    assert f(B, T, H, 64, 64, 64, L.BF16, 1) == f(B, T, H, 64, 64, 64, L.BF16, 2) + extra
+    assert f(B, T, H, 128, 128, 64, L.BF16, 1) == f(B, T, H, 128, 128, 64, L.BF16, 2)
+    assert f(B, T, H, 64, 64, 64, L.BF16, 3) == bad
+    assert f(B, T, H, 64, 64, 64, L.BF16, -1) == bad

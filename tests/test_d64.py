@@ -57,6 +57,12 @@ def test_d64_fwd_bwd(cuda, case, saved):
     assert c[2] == 1 and c[1] + c[0] > 0, c
     dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g.get("h0"), g.get("dhT"), want_dh0=True,
                              chunk=chunk, saved=sv)
+    c = L.counters(reset=True)
+    # saved: one reverse-sweep launch; recompute: the forward into the workspace's saved-state
+    # buffer, then that launch.  Neither touches the exact route unless a head is flagged.
+    assert c[2] == (1 if saved else 2), c
+    if lb > 0:
+        assert c[0] == 0, c
     assert L.device_status() == L.OK
     _check(inp, (o, hT, dq, dlf, di, dh0), _pairs(B, H), inp.get("dhT"))
 
