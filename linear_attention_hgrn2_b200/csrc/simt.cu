@@ -17,6 +17,10 @@
 //
 // Every exponent formed is <= 0 when log f <= 0, so nothing overflows however
 // strong the decay.  One thread block walks the chunks of one (batch, head).
+//
+// The bodies are device functions kept out of line (__noinline__): the tensor-core
+// kernels call them only for flagged pairs, and inlined there they made those kernels'
+// code large enough that instruction fetch cost the reverse sweep 10% of its time.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -68,7 +72,7 @@ static __device__ __forceinline__ void cumsum_gates(float *Bs, float *Ks, int ld
 
 // ------------------------------------------------------------------ forward
 template <typename T>
-__device__ __forceinline__ void
+__device__ __noinline__ void
 simt_fwd_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                 const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT,
                 int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
@@ -143,7 +147,7 @@ simt_fwd_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__rest
 // dA_ts = dO_t . v_s.  Also writes rs[j] = sum_v dhT[j,v] hT[j,v] when dhT != NULL (used by the
 // reverse sweep's d log f carry).
 template <typename T>
-__device__ __forceinline__ void
+__device__ __noinline__ void
 simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
                    float *__restrict__ rs, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
@@ -217,7 +221,7 @@ simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float 
 //   dS_in = Diag(e^B) dS + sum_t (q_t e^{b_t}) dO_t^T
 // The reverse cumulative sum runs across chunks through `carry`.
 template <typename T>
-__device__ __forceinline__ void
+__device__ __noinline__ void
 simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
