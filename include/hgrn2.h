@@ -249,6 +249,14 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
                                void *dq, void *dg, void *di,
                                int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
 
+/* Check of the failure reporting: launches one block that waits, through the bounded
+ * wait every kernel of the library uses, on a barrier that nothing arrives at.  The
+ * wait gives up after `polls` polls (1 .. 2^24; each poll lasts at most the hardware's
+ * short try-wait window), records HGRN2_ERR_TIMEOUT in the device status word and the
+ * block exits normally: no fault, the context stays usable.  hgrn2_get_device_status
+ * then returns HGRN2_ERR_TIMEOUT (and clears it). */
+hgrn2_status hgrn2_selftest_wait_timeout(unsigned int polls, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the library's device-side
  * status word of the current device: HGRN2_OK, HGRN2_ERR_TIMEOUT (a bounded
  * wait gave up) or HGRN2_ERR_DEVICE (a consistency check failed).  Returns

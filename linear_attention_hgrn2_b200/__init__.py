@@ -28,8 +28,9 @@ FP32, BF16 = 0, 1
 # Every extern "C" symbol of include/hgrn2.h.
 EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size", "hgrn2_fwd_train",
            "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_workspace_size_varlen", "hgrn2_saved_size_varlen",
-           "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_bwd", "hgrn2_step_lb_bwd", "hgrn2_step_lb", "hgrn2_get_device_status",
-           "hgrn2_get_counters", "hgrn2_status_string", "hgrn2_version")
+           "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_lb", "hgrn2_step_bwd",
+           "hgrn2_step_lb_bwd", "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string",
+           "hgrn2_version", "hgrn2_selftest_wait_timeout")
 
 _lib = None
 
@@ -81,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_step_lb.argtypes = [vp] * 3 + [ctypes.c_float] + [vp] * 2 + [i32] * 5 + [vp]
     lib.hgrn2_step_lb.restype = i32
     lib.hgrn2_get_device_status.argtypes = [vp]
+    lib.hgrn2_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.hgrn2_selftest_wait_timeout.restype = i32
     lib.hgrn2_get_device_status.restype = i32
     lib.hgrn2_get_counters.argtypes = [ctypes.POINTER(ctypes.c_longlong), i32, i32, vp]
     lib.hgrn2_get_counters.restype = i32
@@ -400,6 +403,12 @@ def step_lb_bwd(q, g, i, lb: float, S, dO, dS=None, dS_out=None):
 def device_status() -> int:
     """Synchronises the current stream; returns and clears the device status word."""
     return int(load_library().hgrn2_get_device_status(_stream()))
+
+
+def selftest_wait_timeout(polls: int = 1000) -> None:
+    """Launches the bounded-wait check (see include/hgrn2.h): afterwards device_status()
+    returns ERR_TIMEOUT."""
+    _raise(load_library().hgrn2_selftest_wait_timeout(polls, _stream()), "hgrn2_selftest_wait_timeout")
 
 
 def counters(reset: bool = False) -> list[int]:

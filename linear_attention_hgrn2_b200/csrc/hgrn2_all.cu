@@ -7,5 +7,6 @@
 #include "simt.cu"
 #include "step.cu"
 #include "varlen.cu"
+#include "selftest.cu"
 #include "tc_fwd.cu"
 #include "tc_bwd.cu"

@@ -203,3 +203,8 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
     assert f(B, T, H, 128, 128, 64, L.BF16, 1) == f(B, T, H, 128, 128, 64, L.BF16, 2)
     assert f(B, T, H, 64, 64, 64, L.BF16, 3) == bad
     assert f(B, T, H, 64, 64, 64, L.BF16, -1) == bad
+
+
+def test_selftest_checks_its_poll_count_before_any_launch(lib):
+    assert lib.hgrn2_selftest_wait_timeout(0, None) == L.ERR_INVALID_ARG
+    assert lib.hgrn2_selftest_wait_timeout((1 << 24) + 1, None) == L.ERR_INVALID_ARG
