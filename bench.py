@@ -13,8 +13,8 @@ the timed region.  Under torchrun each rank runs its own batch on its own GPU
 
 The same JSON line also carries the decode step (B=256, H=16, 1000 in-place
 steps of the fp32 state), the training pair on packed documents of varied
-length (16,384 tokens, H=16), the training pair with 64-wide heads (H=32),
-end-to-end numbers through host buffers, the
+length (16,384 tokens, H=16), the training pair with 64-wide heads (H=32), the two
+forward-only workloads (forward layer, long sequence), end-to-end numbers through host buffers, the
 roofline of the dominant call, SM clocks sampled during the timed region, and
 the CPU oracle timed on a bounded sample (rank 0, one GPU only).
 """
@@ -307,6 +307,8 @@ def run_ours(args, world, rank, local):
         out["varlen"] = run_varlen(args, dev, pk, rank)
     if not args.no_d64:
         out["head_dim_64"] = run_d64(args, dev, pk, rank)
+    if not args.no_fwd_configs:
+        out["forward_configs"] = run_fwd_configs(args, dev, pk, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_seconds)
     if rank == 0:
@@ -555,6 +557,50 @@ def run_d64(args, dev, pk, rank):
     return res
 
 
+def run_fwd_configs(args, dev, pk, rank):
+    """The two forward-only workloads: the forward layer (B=4, H=8, T=2048, lb=0.5) and the long
+    sequence (B=1, H=8, T=32768, lb=0.9, h0 in, hT out).  With 32 and 8 (b,h) pairs they run the
+    segmented forward: segment aggregates, an fp32 scan over segments, then every segment from
+    its incoming state (4 launches)."""
+    import linear_attention_hgrn2_b200 as L
+    from linear_attention_hgrn2_b200 import inputs as I
+    res = {}
+    for w in (I.FWD_LAYER, I.LONG):
+        inp = I.make_workload(w, seed=rank_seed(rank) + 11)
+        q, lf, x = (inp[k].to(dev) for k in ("q", "log_f", "i"))
+        h0 = inp["h0"].to(dev) if "h0" in inp else None
+        o = torch.empty_like(x)
+        ws = torch.empty(max(L.workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.dtype, False), 16),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            return L.fwd(q, lf, x, h0, want_hT=w.want_hT, chunk=w.chunk, out=o, workspace=ws)
+
+        for _ in range(max(args.warmup, 3)):
+            call()
+        torch.cuda.synchronize()
+        K = args.steps
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        L.counters(reset=True)
+        torch.cuda._sleep(2_000_000)
+        a.record()
+        for _ in range(K):
+            call()
+        b.record()
+        torch.cuda.synchronize()
+        launches = L.counters(reset=True)[2] // K
+        ms = a.elapsed_time(b) / K
+        th = w.B * w.T * w.H
+        nbytes = FWD_BYTES * th + (2 * w.B * w.H * w.dk * w.dv * 4 if w.want_hT else 0)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[w.name] = {"tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_call": round(ms, 4),
+                       "launches_per_call": launches, "achieved_gbs": round(gbs, 1),
+                       "frac": round(gbs / pk["hbm_gbs"], 4), "calls": K}
+        del inp, q, lf, x, o, ws, h0
+        torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(inp, w, budget_s=15.0):
     """The oracle (unchanged) on the host cores: fwd+bwd of whole (batch, head) sequences of the workload.
 
@@ -635,6 +681,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-d64", action="store_true")
+    ap.add_argument("--no-fwd-configs", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
