@@ -41,6 +41,8 @@ def _load():
         lib.oracle_fwd.argtypes = [dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci]
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci]
         lib.oracle_step.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci]
+        lib.oracle_sd_fwd.argtypes = [dp] * 7 + [ci] * 5
+        lib.oracle_sd_bwd.argtypes = [dp] * 12 + [ci] * 5
         lib.oracle_num_threads.restype = ci
         _lib = lib
     return _lib
@@ -141,3 +143,32 @@ def lower_bound_dlog_f_dg(g, lb: float):
     u = np.exp(-np.abs(g))
     den = np.where(g >= 0, (1.0 + u) * (1.0 + lb * u), (1.0 + u) * (lb + u))
     return (1.0 - lb) * u / den
+
+
+def sd_fwd(q, k, v, log_g, h0=None):
+    """Scalar-decay variant, in fp64: S_t = g_t S_{t-1} + k_t v_t^T, o_t = S_t^T q_t with
+    g_t = exp(log_g_t) one decay per (batch, token, head) (the per-head decay of Mamba2/RetNet
+    that "HGRN2: Gated Linear RNNs with State Expansion", §5, contrasts with its per-dimension
+    decay).  q, k: [B,T,H,dk]; v: [B,T,H,dv]; log_g: [B,T,H]; h0: [B,H,dk,dv] or None.
+    Returns (o [B,T,H,dv], hT)."""
+    q, k, v, log_g, h0 = (_f64(a) for a in (q, k, v, log_g, h0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    hT = np.zeros((B, H, dk, dv))
+    _load().oracle_sd_fwd(_p(q), _p(k), _p(v), _p(log_g), _p(h0), _p(o), _p(hT), B, T, H, dk, dv)
+    return o, hT
+
+
+def sd_bwd(q, k, v, log_g, dO, h0=None, dhT=None):
+    """Gradients (dq, dk, dv, dlog_g, dh0) of L = <o, dO> + <hT, dhT> for sd_fwd, in fp64
+    (back-propagation through time)."""
+    q, k, v, log_g, dO, h0, dhT = (_f64(a) for a in (q, k, v, log_g, dO, h0, dhT))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dq, dk_, dv_ = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg = np.zeros_like(log_g)
+    dh0 = np.zeros((B, H, dk, dv))
+    _load().oracle_sd_bwd(_p(q), _p(k), _p(v), _p(log_g), _p(h0), _p(dO), _p(dhT), _p(dq), _p(dk_), _p(dv_),
+                          _p(dg), _p(dh0), B, T, H, dk, dv)
+    return dq, dk_, dv_, dg, dh0

@@ -198,6 +198,124 @@ void oracle_bwd(const double *q, const double *log_f, const double *x,
     }
 }
 
+/* ------------------------------------------------------------------------
+ * Scalar-decay variant (the contrast of §5: models such as Mamba2 or RetNet
+ * keep ONE decay per head and token, and a key of their own):
+ *
+ *   S_t = g_t S_{t-1} + k_t v_t^T,      o_t = S_t^T q_t,      g_t = exp(log_g_t)
+ *
+ * q, k: [B][T][H][dk]; v, o: [B][T][H][dv]; log_g: [B][T][H]; states as above.
+ * ------------------------------------------------------------------------ */
+#define GATE(b, t, h, T, H) (((size_t)(b) * (T) + (t)) * (H) + (h))
+
+void oracle_sd_fwd(const double *q, const double *k, const double *v, const double *log_g,
+                   const double *h0, double *o, double *hT, int B, int T, int H, int dk, int dv)
+{
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double *S = (double *)calloc((size_t)dk * dv, sizeof(double));
+            if (h0) memcpy(S, h0 + ST(b, h, B, H, dk, dv), sizeof(double) * dk * dv);
+            for (int t = 0; t < T; ++t) {
+                double g = exp(log_g[GATE(b, t, h, T, H)]);
+                for (int j = 0; j < dk; ++j) {
+                    double kj = k[TOK(b, t, h, j, T, H, dk)];
+                    for (int c = 0; c < dv; ++c)
+                        S[j * dv + c] = g * S[j * dv + c] + kj * v[TOK(b, t, h, c, T, H, dv)];
+                }
+                for (int c = 0; c < dv; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dk; ++j) acc += q[TOK(b, t, h, j, T, H, dk)] * S[j * dv + c];
+                    o[TOK(b, t, h, c, T, H, dv)] = acc;
+                }
+            }
+            if (hT) memcpy(hT + ST(b, h, B, H, dk, dv), S, sizeof(double) * dk * dv);
+            free(S);
+        }
+    }
+}
+
+/* Backward of oracle_sd_fwd by back-propagation through time.  Going backwards
+ * over t, with dS the gradient w.r.t. S_t:
+ *
+ *   dS      += q_t dO_t^T
+ *   dq_t     = S_t dO_t
+ *   dk_t     = dS v_t
+ *   dv_t     = dS^T k_t
+ *   dlog_g_t = g_t * sum_{j,c} dS[j,c] S_{t-1}[j,c]
+ *   dS       = g_t dS
+ *
+ * and dh0 = dS; S_{t-1} is recomputed from checkpoints as in oracle_bwd. */
+void oracle_sd_bwd(const double *q, const double *k, const double *v, const double *log_g,
+                   const double *h0, const double *dO, const double *dhT,
+                   double *dq, double *dk_, double *dv_, double *dlog_g, double *dh0,
+                   int B, int T, int H, int dk, int dv)
+{
+    int nck = (T + CKPT - 1) / CKPT;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            size_t sd = (size_t)dk * dv;
+            double *ck = (double *)calloc((size_t)(nck + 1) * sd, sizeof(double));
+            double *seg = (double *)malloc((size_t)(CKPT + 1) * sd * sizeof(double));
+            double *dS = (double *)calloc(sd, sizeof(double));
+            double *S = (double *)calloc(sd, sizeof(double));
+            if (h0) memcpy(S, h0 + ST(b, h, B, H, dk, dv), sizeof(double) * sd);
+            for (int t = 0; t < T; ++t) {
+                if (t % CKPT == 0) memcpy(ck + (size_t)(t / CKPT) * sd, S, sizeof(double) * sd);
+                double g = exp(log_g[GATE(b, t, h, T, H)]);
+                for (int j = 0; j < dk; ++j) {
+                    double kj = k[TOK(b, t, h, j, T, H, dk)];
+                    for (int c = 0; c < dv; ++c)
+                        S[j * dv + c] = g * S[j * dv + c] + kj * v[TOK(b, t, h, c, T, H, dv)];
+                }
+            }
+            if (dhT) memcpy(dS, dhT + ST(b, h, B, H, dk, dv), sizeof(double) * sd);
+            for (int c0 = nck - 1; c0 >= 0; --c0) {
+                int t0 = c0 * CKPT, t1 = t0 + CKPT < T ? t0 + CKPT : T;
+                memcpy(seg, ck + (size_t)c0 * sd, sizeof(double) * sd);
+                for (int t = t0; t < t1; ++t) {
+                    double *prev = seg + (size_t)(t - t0) * sd, *cur = prev + sd;
+                    double g = exp(log_g[GATE(b, t, h, T, H)]);
+                    for (int j = 0; j < dk; ++j) {
+                        double kj = k[TOK(b, t, h, j, T, H, dk)];
+                        for (int c = 0; c < dv; ++c)
+                            cur[j * dv + c] = g * prev[j * dv + c] + kj * v[TOK(b, t, h, c, T, H, dv)];
+                    }
+                }
+                for (int t = t1 - 1; t >= t0; --t) {
+                    const double *Sp = seg + (size_t)(t - t0) * sd, *St = Sp + sd;
+                    const double *qt = q + TOK(b, t, h, 0, T, H, dk), *kt = k + TOK(b, t, h, 0, T, H, dk);
+                    const double *vt = v + TOK(b, t, h, 0, T, H, dv), *gt = dO + TOK(b, t, h, 0, T, H, dv);
+                    double g = exp(log_g[GATE(b, t, h, T, H)]);
+                    for (int j = 0; j < dk; ++j)
+                        for (int c = 0; c < dv; ++c) dS[j * dv + c] += qt[j] * gt[c];
+                    double dg = 0.0;
+                    for (int j = 0; j < dk; ++j) {
+                        double aq = 0.0, ak = 0.0;
+                        for (int c = 0; c < dv; ++c) {
+                            aq += St[j * dv + c] * gt[c];
+                            ak += dS[j * dv + c] * vt[c];
+                            dg += dS[j * dv + c] * Sp[j * dv + c];
+                        }
+                        dq[TOK(b, t, h, j, T, H, dk)] = aq;
+                        dk_[TOK(b, t, h, j, T, H, dk)] = ak;
+                    }
+                    for (int c = 0; c < dv; ++c) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dk; ++j) acc += dS[j * dv + c] * kt[j];
+                        dv_[TOK(b, t, h, c, T, H, dv)] = acc;
+                    }
+                    dlog_g[GATE(b, t, h, T, H)] = g * dg;
+                    for (size_t e = 0; e < sd; ++e) dS[e] *= g;
+                }
+            }
+            if (dh0) memcpy(dh0 + ST(b, h, B, H, dk, dv), dS, sizeof(double) * sd);
+            free(ck); free(seg); free(dS); free(S);
+        }
+    }
+}
+
 /* Number of threads OpenMP will use (1 when built without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

@@ -304,3 +304,103 @@ def test_step_bwd_matches_central_finite_differences_of_step(with_dS):
             args[idx] = m
             fd[k] = (lp - loss(*args)) / (2 * h)
         np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-8)
+
+
+# ---------------------------------------------------------------- scalar-decay variant
+def _sd_inputs(B, T, H, dk, dv, seed, h0=True):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk))
+    v = rng.standard_normal((B, T, H, dv))
+    lg = -np.abs(rng.standard_normal((B, T, H))) * 0.5
+    S0 = rng.standard_normal((B, H, dk, dv)) if h0 else None
+    return q, k, v, lg, S0
+
+
+def test_sd_fwd_matches_quadratic_masked_form():
+    # O = ((Q K^T) . D) V + Diag(prod_{r<=t} g_r) Q h0,  D_ts = prod_{s<r<=t} g_r for s <= t
+    B, T, H, dk, dv = 1, 9, 2, 3, 4
+    q, k, v, lg, S0 = _sd_inputs(B, T, H, dk, dv, 31)
+    o, hT = oracle.sd_fwd(q, k, v, lg, S0)
+    g = np.exp(lg)
+    for h in range(H):
+        Q, K, V = q[0, :, h], k[0, :, h], v[0, :, h]
+        D = np.zeros((T, T))
+        for t in range(T):
+            for s in range(t + 1):
+                D[t, s] = np.prod(g[0, s + 1:t + 1, h])
+        G = np.array([np.prod(g[0, :t + 1, h]) for t in range(T)])
+        ref = ((Q @ K.T) * D) @ V + G[:, None] * (Q @ S0[0, h])
+        np.testing.assert_allclose(o[0, :, h], ref, rtol=1e-12, atol=1e-12)
+        Sref = G[-1] * S0[0, h] + sum(D[T - 1, s] * np.outer(K[s], V[s]) for s in range(T))
+        np.testing.assert_allclose(hT[0, h], Sref, rtol=1e-12, atol=1e-12)
+
+
+def test_sd_fwd_closed_forms():
+    B, T, H, dk, dv = 1, 6, 1, 3, 2
+    q, k, v, _, S0 = _sd_inputs(B, T, H, dk, dv, 32)
+    # g = 1: the state accumulates every k v^T on top of h0
+    o, _ = oracle.sd_fwd(q, k, v, np.zeros((B, T, H)), S0)
+    for t in range(T):
+        S = S0[0, 0] + sum(np.outer(k[0, s, 0], v[0, s, 0]) for s in range(t + 1))
+        np.testing.assert_allclose(o[0, t, 0], S.T @ q[0, t, 0], rtol=1e-12, atol=1e-12)
+    # g -> 0 (log g = -80): only the current token survives, o_t = (q_t . k_t) v_t
+    o, _ = oracle.sd_fwd(q, k, v, np.full((B, T, H), -80.0), S0)
+    np.testing.assert_allclose(o[0, :, 0], (q[0, :, 0] * k[0, :, 0]).sum(-1)[:, None] * v[0, :, 0],
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_sd_equals_hgrn2_when_the_key_is_one_minus_a_shared_gate():
+    # HGRN2 with every key dim's forget gate equal to g_t has key 1 - g_t in every dim: the
+    # scalar-decay form with k_t = (1 - g_t) 1 and the same gate computes the same o and hT, and
+    # the chain rule through k = 1 - g links the gradients:
+    #   sum_j dlog_f[t, j] = dlog_g[t] - g_t sum_j dk[t, j]
+    B, T, H, dk, dv = 2, 70, 2, 3, 4     # T crosses the oracle's 64-step checkpoint
+    q, _, v, lg, S0 = _sd_inputs(B, T, H, dk, dv, 33)
+    rng = np.random.default_rng(34)
+    dO = rng.standard_normal((B, T, H, dv))
+    dhT = rng.standard_normal((B, H, dk, dv))
+    g = np.exp(lg)
+    k = np.repeat((1.0 - g)[..., None], dk, axis=-1)
+    lf = np.repeat(lg[..., None], dk, axis=-1)
+    o1, h1 = oracle.sd_fwd(q, k, v, lg, S0)
+    o2, h2 = oracle.fwd(q, lf, v, S0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(h1, h2, rtol=1e-10, atol=1e-12)
+    dq1, dk1, dv1, dg1, dh1 = oracle.sd_bwd(q, k, v, lg, dO, S0, dhT)
+    dq2, dlf2, di2, dh2 = oracle.bwd(q, lf, v, dO, S0, dhT)
+    np.testing.assert_allclose(dq1, dq2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv1, di2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dh1, dh2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dlf2.sum(-1), dg1 - g * dk1.sum(-1), rtol=1e-9, atol=1e-10)
+
+
+def test_sd_bwd_matches_central_finite_differences():
+    B, T, H, dk, dv = 1, 67, 1, 2, 3
+    q, k, v, lg, S0 = _sd_inputs(B, T, H, dk, dv, 35)
+    rng = np.random.default_rng(36)
+    dO = rng.standard_normal((B, T, H, dv))
+    dhT = rng.standard_normal((B, H, dk, dv))
+
+    def loss(q_, k_, v_, lg_, S_):
+        o, hT = oracle.sd_fwd(q_, k_, v_, lg_, S_)
+        return float(np.sum(o * dO) + np.sum(hT * dhT))
+
+    grads = oracle.sd_bwd(q, k, v, lg, dO, S0, dhT)
+    args = [q, k, v, lg, S0]
+    h = 1e-6
+    pick = np.random.default_rng(37)
+    for ai in range(5):   # gradient ai is w.r.t. argument ai
+        arr = args[ai]
+        # a few entries each, including the first and the last token (a checkpoint boundary at 64)
+        picks = {tuple(int(pick.integers(0, n)) for n in arr.shape) for _ in range(4)}
+        if arr.ndim >= 3:
+            picks |= {tuple(0 for _ in arr.shape), tuple(n - 1 for n in arr.shape)}
+        for p in picks:
+            a_p, a_m = arr.copy(), arr.copy()
+            a_p[p] += h
+            a_m[p] -= h
+            ap, am = list(args), list(args)
+            ap[ai], am[ai] = a_p, a_m
+            fd = (loss(*ap) - loss(*am)) / (2 * h)
+            assert grads[ai][p] == pytest.approx(fd, rel=1e-5, abs=1e-7), (ai, p)
