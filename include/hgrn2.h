@@ -249,6 +249,30 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
                                void *dq, void *dg, void *di,
                                int B, int H, int dk, int dv, hgrn2_dtype dtype, cudaStream_t stream);
 
+/* Scalar-decay variant: one decay per head and token and a key of its own, the per-head
+ * decay of models such as Mamba2 and RetNet that §5 contrasts with HGRN2's per-dimension
+ * decay (where the masked form ((Q K^T) . D) V holds exactly):
+ *   S_t = g_t S_{t-1} + k_t v_t^T,   o_t = S_t^T q_t,   g_t = exp(log_g_t)  (log_g <= 0)
+ *   q, k : [B,T,H,dk]   v, o : [B,T,H,dv]   log_g : [B,T,H]   (all dtype)
+ *   h0, hT : [B,H,dk,dv] float32 (NULL allowed, as for hgrn2_fwd)
+ * Computed chunkwise on CUDA cores in fp32 arithmetic (exact route: every exponent formed
+ * is a difference of in-chunk cumulative sums, so any decay strength is exact).
+ * 1 <= dk, dv <= 128; any T >= 0; pointers 16-byte aligned.
+ * hgrn2_scalar_bwd: gradients dq, dk_out (of k), dv_out (of v), dlog_g (same shapes and dtype
+ * as the inputs) and
+ * dh0 (NULL: not computed) of L(o, hT) given dO and dhT (NULL: zero).  workspace: device
+ * scratch of at least hgrn2_scalar_workspace_size(B, H) bytes ((size_t)-1 for bad sizes). */
+size_t hgrn2_scalar_workspace_size(int B, int H);
+hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g,
+                              const float *h0, void *o, float *hT,
+                              int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                              cudaStream_t stream);
+hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const void *log_g,
+                              const float *h0, const void *dO, const float *dhT,
+                              void *dq, void *dk_out, void *dv_out, void *dlog_g, float *dh0,
+                              int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                              void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Check of the failure reporting: launches one block that waits, through the bounded
  * wait every kernel of the library uses, on a barrier that nothing arrives at.  The
  * wait gives up after `polls` polls (1 .. 2^24; each poll lasts at most the hardware's

@@ -30,7 +30,8 @@ EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size",
            "hgrn2_bwd_saved", "hgrn2_bwd_noalloc", "hgrn2_workspace_size_varlen", "hgrn2_saved_size_varlen",
            "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_lb", "hgrn2_step_bwd",
            "hgrn2_step_lb_bwd", "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string",
-           "hgrn2_version", "hgrn2_selftest_wait_timeout")
+           "hgrn2_version", "hgrn2_selftest_wait_timeout", "hgrn2_scalar_workspace_size", "hgrn2_scalar_fwd",
+           "hgrn2_scalar_bwd")
 
 _lib = None
 
@@ -83,6 +84,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_step_lb.restype = i32
     lib.hgrn2_get_device_status.argtypes = [vp]
     lib.hgrn2_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.hgrn2_scalar_workspace_size.argtypes = [i32, i32]
+    lib.hgrn2_scalar_workspace_size.restype = sz
+    lib.hgrn2_scalar_fwd.argtypes = [vp] * 7 + [i32] * 6 + [vp]
+    lib.hgrn2_scalar_fwd.restype = i32
+    lib.hgrn2_scalar_bwd.argtypes = [vp] * 12 + [i32] * 6 + [vp, sz, vp]
+    lib.hgrn2_scalar_bwd.restype = i32
     lib.hgrn2_selftest_wait_timeout.restype = i32
     lib.hgrn2_get_device_status.restype = i32
     lib.hgrn2_get_counters.argtypes = [ctypes.POINTER(ctypes.c_longlong), i32, i32, vp]
@@ -398,6 +405,53 @@ def step_bwd(q, log_f, i, S, dO, dS=None, dS_out=None):
 def step_lb_bwd(q, g, i, lb: float, S, dO, dS=None, dS_out=None):
     """Backward of step_lb(): as step_bwd, returning dL/dg in place of dlog_f."""
     return _step_bwd(load_library().hgrn2_step_lb_bwd, "hgrn2_step_lb_bwd", q, g, i, S, dO, dS, lb, dS_out)
+
+
+def scalar_fwd(q, k, v, log_g, h0=None, want_hT=False):
+    """Scalar-decay variant: S_t = g_t S_{t-1} + k_t v_t^T, o_t = S_t^T q_t, g_t = exp(log_g_t).
+
+    q, k: [B,T,H,dk]; v: [B,T,H,dv]; log_g: [B,T,H] (same dtype); h0: [B,H,dk,dv] float32 or
+    None.  Returns (o, hT or None)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q")
+    _check(k, "k", q.dtype, q.shape)
+    _check(v, "v", q.dtype, (B, T, H, dv))
+    _check(log_g, "log_g", q.dtype, (B, T, H))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_hT else None
+    st = lib.hgrn2_scalar_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(o), _ptr(hT),
+                              B, T, H, dk, dv, _dt(q), _stream())
+    _raise(st, "hgrn2_scalar_fwd")
+    return o, hT
+
+
+def scalar_bwd(q, k, v, log_g, dO, h0=None, dhT=None, want_dh0=False):
+    """Gradients (dq, dk, dv, dlog_g, dh0 or None) of the scalar-decay variant."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q")
+    _check(k, "k", q.dtype, q.shape)
+    _check(v, "v", q.dtype, (B, T, H, dv))
+    _check(log_g, "log_g", q.dtype, (B, T, H))
+    _check(dO, "dO", q.dtype, (B, T, H, dv))
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv))
+    if dhT is not None:
+        _check(dhT, "dhT", torch.float32, (B, H, dk, dv))
+    dq, dk_, dv_, dg = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g)
+    dh0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
+    nws = _size_or_raise(lib.hgrn2_scalar_workspace_size(B, H), "hgrn2_scalar_workspace_size")
+    ws = _workspace(nws, q.device)
+    st = lib.hgrn2_scalar_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(dq),
+                              _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dh0), B, T, H, dk, dv, _dt(q), _ptr(ws), nws,
+                              _stream())
+    _raise(st, "hgrn2_scalar_bwd")
+    return dq, dk_, dv_, dg, dh0
 
 
 def device_status() -> int:

@@ -12,6 +12,8 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <initializer_list>
+
 using namespace hgrn2;
 
 namespace {
@@ -384,6 +386,69 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
                                int dv, hgrn2_dtype dtype, cudaStream_t stream) {
     if (!(lb >= 0.0f && lb < 1.0f)) return HGRN2_ERR_INVALID_ARG;
     return step_bwd_impl(q, g, i, S, dO, dS, dS_prev, dq, dg, di, B, H, dk, dv, dtype, true, lb, stream);
+}
+
+// ------------------------------------------------------------------ scalar-decay variant
+namespace {
+hgrn2_status check_scalar(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
+    if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
+    if (dk > 128 || dv > 128) return HGRN2_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1ll << 30) || (long long)B * T * H > (1ll << 40)) return HGRN2_ERR_UNSUPPORTED;
+    return HGRN2_OK;
+}
+bool all_aligned(std::initializer_list<const void *> ptrs) {
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return false;
+    return true;
+}
+}  // namespace
+
+size_t hgrn2_scalar_workspace_size(int B, int H) {
+    if (B < 1 || H < 1) return (size_t)-1;
+    return align256(sizeof(float) * (size_t)B * H);
+}
+
+hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                              void *o, float *hT, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                              cudaStream_t stream) {
+    hgrn2_status s = check_scalar(B, T, H, dk, dv, dtype);
+    if (s != HGRN2_OK) return s;
+    if (T > 0 && (!q || !k || !v || !log_g || !o)) return HGRN2_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, log_g, h0, o, hT})) return HGRN2_ERR_INVALID_ARG;
+    if (T == 0) {
+        if (!hT) return HGRN2_OK;
+        const size_t n = sizeof(float) * (size_t)B * H * dk * dv;
+        return from_cuda(h0 ? cudaMemcpyAsync(hT, h0, n, cudaMemcpyDeviceToDevice, stream)
+                            : cudaMemsetAsync(hT, 0, n, stream));
+    }
+    ScalarArgs a{q, k, v, log_g, h0, o, hT, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                 nullptr, B, T, H, dk, dv};
+    g_launches += 1;
+    return from_cuda(launch_scalar_fwd(a, dtype == HGRN2_BF16, stream));
+}
+
+hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                              const void *dO, const float *dhT, void *dq, void *dk_out, void *dv_out, void *dlog_g,
+                              float *dh0, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype, void *workspace,
+                              size_t ws_bytes, cudaStream_t stream) {
+    hgrn2_status s = check_scalar(B, T, H, dk, dv, dtype);
+    if (s != HGRN2_OK) return s;
+    if (T > 0 && (!q || !k || !v || !log_g || !dO || !dq || !dk_out || !dv_out || !dlog_g))
+        return HGRN2_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, log_g, h0, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, workspace}))
+        return HGRN2_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < hgrn2_scalar_workspace_size(B, H)) return HGRN2_ERR_INVALID_ARG;
+    if (T == 0) {
+        if (!dh0) return HGRN2_OK;
+        const size_t n = sizeof(float) * (size_t)B * H * dk * dv;
+        return from_cuda(dhT ? cudaMemcpyAsync(dh0, dhT, n, cudaMemcpyDeviceToDevice, stream)
+                             : cudaMemsetAsync(dh0, 0, n, stream));
+    }
+    ScalarArgs a{q, k, v, log_g, h0, nullptr, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0,
+                 (float *)workspace, B, T, H, dk, dv};
+    g_launches += 2;
+    return from_cuda(launch_scalar_bwd(a, dtype == HGRN2_BF16, stream));
 }
 
 hgrn2_status hgrn2_get_device_status(cudaStream_t stream) {

@@ -7,6 +7,7 @@
 #include "simt.cu"
 #include "step.cu"
 #include "varlen.cu"
+#include "scalar.cu"
 #include "selftest.cu"
 #include "tc_fwd.cu"
 #include "tc_bwd.cu"

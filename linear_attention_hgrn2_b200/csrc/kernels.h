@@ -74,6 +74,22 @@ struct StepBwdArgs {
 };
 cudaError_t launch_step_bwd(const StepBwdArgs &a, bool bf16, cudaStream_t st);
 
+// Scalar-decay variant (one decay per head and token, explicit key): exact route on CUDA cores.
+struct ScalarArgs {
+    const void *q, *k, *v, *lg;     // lg: log g [B][T][H]
+    const float *h0;
+    void *o;                        // forward outputs
+    float *hT;
+    const void *dO;                 // backward inputs / outputs
+    const float *dhT;
+    void *dq, *dk_out, *dv_out, *dlg;
+    float *dh0;
+    float *rs;                      // backward workspace: <dhT, hT> per (b,h)
+    int B, T, H, dk, dv;
+};
+cudaError_t launch_scalar_fwd(const ScalarArgs &a, bool bf16, cudaStream_t st);
+cudaError_t launch_scalar_bwd(const ScalarArgs &a, bool bf16, cudaStream_t st);
+
 // Longest-first launch order of packed sequences: perm[r] = the sequence that CTA row r runs,
 // ordered by decreasing number of 128-token chunks (one CTA; any nseq).
 cudaError_t launch_lpt_order(const int *cu, int nseq, int T, int *perm, cudaStream_t st);

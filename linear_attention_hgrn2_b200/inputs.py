@@ -181,3 +181,27 @@ def make_step_grads(B: int, H: int, dk: int, dv: int, dtype: torch.dtype, seed: 
     g = _gen(seed)
     return {"dO": _to(_normal(g, (B, H, dv)), dtype),
             "dS": torch.from_numpy(_normal(g, (B, H, dk, dv), dS_sigma))}
+
+
+# Scalar-decay variant at the training workload's shape: one decay per head and token,
+# g = lb + (1 - lb) sigmoid(x) as for the per-dimension gates, an explicit key k ~ N(0, 1/d_k)
+SCALAR_TRAIN = Workload("scalar_fwdbwd_bf16_B8_H16_T2048_d128", 8, 16, 2048, 128, 128, torch.bfloat16, 0.95,
+                        32, bwd=True)
+
+
+def make_scalar_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: torch.dtype, lb: float, seed: int,
+                       h0_sigma: float = 0.0, with_dO: bool = False, dhT_sigma: float = 0.0) -> dict:
+    """CPU tensors for the scalar-decay variant: q, k [B,T,H,dk], v [B,T,H,dv], log_g [B,T,H]
+    in ``dtype``; optional h0, dO, dhT.  Draw order (fixed): q, k, v, gate, dO, h0, dhT."""
+    g = _gen(seed)
+    out = {"q": _to(_normal(g, (B, T, H, dk)), dtype),
+           "k": _to(_normal(g, (B, T, H, dk), 1.0 / np.sqrt(dk)), dtype),
+           "v": _to(_normal(g, (B, T, H, dv)), dtype)}
+    out["log_g"] = _to(gate_log_f(_normal(g, (B, T, H)), lb), dtype)
+    if with_dO:
+        out["dO"] = _to(_normal(g, (B, T, H, dv)), dtype)
+    if h0_sigma > 0:
+        out["h0"] = torch.from_numpy(_normal(g, (B, H, dk, dv), h0_sigma))
+    if dhT_sigma > 0:
+        out["dhT"] = torch.from_numpy(_normal(g, (B, H, dk, dv), dhT_sigma))
+    return out

@@ -208,3 +208,19 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
 def test_selftest_checks_its_poll_count_before_any_launch(lib):
     assert lib.hgrn2_selftest_wait_timeout(0, None) == L.ERR_INVALID_ARG
     assert lib.hgrn2_selftest_wait_timeout((1 << 24) + 1, None) == L.ERR_INVALID_ARG
+
+
+def test_scalar_decay_argument_checks_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    bad = ctypes.c_size_t(-1).value
+    assert lib.hgrn2_scalar_workspace_size(0, 4) == bad
+    assert lib.hgrn2_scalar_workspace_size(2, 3) == 256
+    f = lib.hgrn2_scalar_fwd
+    assert f(vp(16), vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 256, 16, L.FP32, None) == L.ERR_UNSUPPORTED
+    assert f(None, vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 16, 16, L.FP32, None) == L.ERR_INVALID_ARG
+    assert f(vp(18), vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 16, 16, L.FP32, None) == L.ERR_INVALID_ARG
+    g = lib.hgrn2_scalar_bwd
+    # workspace missing or short
+    args = [vp(16)] * 4 + [None, vp(16), None] + [vp(16)] * 4 + [None]
+    assert g(*args, 2, 8, 3, 16, 16, L.BF16, None, 0, None) == L.ERR_INVALID_ARG
+    assert g(*args, 2, 8, 3, 16, 16, L.BF16, vp(256), 255, None) == L.ERR_INVALID_ARG

@@ -196,3 +196,32 @@ def test_repacking_in_reverse_order_changes_no_bit(cuda, dtype):
             assert torch.equal(a[name][cu[s]:cu[s + 1]], b[name][rcu[j]:rcu[j + 1]]), (name, s)
         for name in ("hT", "dh0"):
             assert torch.equal(a[name][s], b[name][j]), (name, s)
+
+
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_tokens_outside_every_sequence_are_left_untouched(cuda, saved):
+    # cu_seqlens = [3, 3, 140, 140] over 200 tokens: sequence 1 is tokens 3..139, sequences 0
+    # and 2 are empty; tokens 0..2 and 140..199 belong to none and keep what the buffers held
+    H = 2
+    inp = I.make_varlen([200], H, 128, 128, torch.bfloat16, 0.9, seed=611, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    g = to_cuda(inp)
+    nseq = 3
+    cu = torch.tensor([3, 3, 140, 140], dtype=torch.int32, device="cuda")
+    gen = torch.Generator().manual_seed(5)
+    h0 = (0.1 * torch.randn((nseq, H, 128, 128), generator=gen)).cuda()
+    dhT = (0.1 * torch.randn((nseq, H, 128, 128), generator=gen)).cuda()
+    sentinel = 7.0
+    o = torch.full((200, H, 128), sentinel, dtype=torch.bfloat16, device="cuda")
+    sv = L.new_saved_varlen(g["q"], cu) if saved else None
+    _, hT = L.fwd_varlen(g["q"], g["log_f"], g["i"], cu, h0, want_hT=True, out=o, saved=sv)
+    dq, dlf, di, dh0 = L.bwd_varlen(g["q"], g["log_f"], g["i"], g["dO"], cu, h0, dhT, want_dh0=True, saved=sv)
+    assert L.device_status() == L.OK
+    outside = torch.cat([o[:3], o[140:]])
+    assert torch.all(outside == sentinel)
+    for s in (0, 2):   # empty: states pass through
+        assert torch.equal(hT[s], h0[s]) and torch.equal(dh0[s], dhT[s])
+    ref_in = {"q": inp["q"], "log_f": inp["log_f"], "i": inp["i"], "dO": inp["dO"],
+              "h0": h0.cpu(), "dhT": dhT.cpu(), "cu_seqlens": torch.tensor([3, 3, 140, 140], dtype=torch.int32)}
+    _check(ref_in, {"o": o, "hT": hT, "dq": dq, "dlog_f": dlf, "di": di, "dh0": dh0}, [1], range(H),
+           torch.bfloat16, 2e-2)
