@@ -14,7 +14,8 @@ the timed region.  Under torchrun each rank runs its own batch on its own GPU
 The same JSON line also carries the decode step (B=256, H=16, 1000 in-place
 steps of the fp32 state), the training pair on packed documents of varied
 length (16,384 tokens, H=16), the training pair with 64-wide heads (H=32), the two
-forward-only workloads (forward layer, long sequence), end-to-end numbers through host buffers, the
+forward-only workloads (forward layer, long sequence), the scalar-decay variant,
+end-to-end numbers through host buffers, the
 roofline of the dominant call, SM clocks sampled during the timed region, and
 the CPU oracle timed on a bounded sample (rank 0, one GPU only).
 """
@@ -309,6 +310,8 @@ def run_ours(args, world, rank, local):
         out["head_dim_64"] = run_d64(args, dev, pk, rank)
     if not args.no_fwd_configs:
         out["forward_configs"] = run_fwd_configs(args, dev, pk, rank)
+    if not args.no_scalar:
+        out["scalar_decay"] = run_scalar(args, dev, pk, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_seconds)
     if rank == 0:
@@ -601,6 +604,58 @@ def run_fwd_configs(args, dev, pk, rank):
     return res
 
 
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA/clock x 2 flop x 1.965 GHz (max SM clock)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_scalar(args, dev, pk, rank):
+    """The scalar-decay variant (one decay per head and token, explicit key) at the training
+    workload's shape: hgrn2_scalar_fwd + hgrn2_scalar_bwd, CUDA cores, chunks of 32."""
+    import linear_attention_hgrn2_b200 as L
+    from linear_attention_hgrn2_b200 import inputs as I
+    w = I.SCALAR_TRAIN
+    inp = I.make_scalar_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.lb, seed=rank_seed(rank) + 13, with_dO=True)
+    g = {k: t.to(dev) for k, t in inp.items()}
+
+    def fwd_call():
+        L.scalar_fwd(g["q"], g["k"], g["v"], g["log_g"])
+
+    def bwd_call():
+        L.scalar_bwd(g["q"], g["k"], g["v"], g["log_g"], g["dO"])
+
+    for _ in range(2):
+        fwd_call()
+        bwd_call()
+    torch.cuda.synchronize()
+    K = max(3, min(args.steps, 10))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for _ in range(K):
+        fwd_call()
+    ev[1].record()
+    for _ in range(K):
+        bwd_call()
+    ev[2].record()
+    torch.cuda.synchronize()
+    fwd_ms = ev[0].elapsed_time(ev[1]) / K
+    bwd_ms = ev[1].elapsed_time(ev[2]) / K
+    # algorithmic flops of the chunkwise forward per token-head at chunk C: causal scores
+    # (C/2 * dk * 2), intra outputs (C/2 * dv * 2), inter outputs and state update (2 * dk*dv * 2)
+    C, dk, dv = 32, w.dk, w.dv
+    fwd_flops = (C // 2) * (dk + dv) * 2 + 4 * dk * dv
+    th = w.B * w.T * w.H
+    tf = fwd_flops * th / (fwd_ms / 1e3) / 1e12
+    res = {"workload": w.name, "tokens_per_s": round(w.B * w.T / ((fwd_ms + bwd_ms) / 1e3), 1),
+           "fwd_ms": round(fwd_ms, 3), "bwd_ms": round(bwd_ms, 3), "route": "exact (CUDA cores, fp32 arithmetic)",
+           "fwd_roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(FP32_PEAK_TFLOPS, 1),
+                            "unit": "TFLOP/s", "frac": round(tf / FP32_PEAK_TFLOPS, 4),
+                            "peak_source": "148 SMs x 128 fp32 FMA/clock x 1.965 GHz"},
+           "calls": "hgrn2_scalar_fwd + hgrn2_scalar_bwd", "steps": K}
+    del g, inp
+    torch.cuda.empty_cache()
+    return res
+
+
 def cpu_baseline(inp, w, budget_s=15.0):
     """The oracle (unchanged) on the host cores: fwd+bwd of whole (batch, head) sequences of the workload.
 
@@ -682,6 +737,7 @@ def main():
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-d64", action="store_true")
     ap.add_argument("--no-fwd-configs", action="store_true")
+    ap.add_argument("--no-scalar", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
