@@ -255,8 +255,10 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
  *   S_t = g_t S_{t-1} + k_t v_t^T,   o_t = S_t^T q_t,   g_t = exp(log_g_t)  (log_g <= 0)
  *   q, k : [B,T,H,dk]   v, o : [B,T,H,dv]   log_g : [B,T,H]   (all dtype)
  *   h0, hT : [B,H,dk,dv] float32 (NULL allowed, as for hgrn2_fwd)
- * Computed chunkwise on CUDA cores in fp32 arithmetic (exact route: every exponent formed
- * is a difference of in-chunk cumulative sums, so any decay strength is exact).
+ * The forward runs on tensor cores for bf16 with dk = dv = 128 or 64 (128-token chunks,
+ * bf16 operands, fp32 accumulation and state); everything else, and the backward, runs
+ * chunkwise on CUDA cores in fp32 arithmetic.  Both routes form only exponents that are
+ * differences of in-chunk cumulative sums, so any decay strength is exact.
  * 1 <= dk, dv <= 128; any T >= 0; pointers 16-byte aligned.
  * hgrn2_scalar_bwd: gradients dq, dk_out (of k), dv_out (of v), dlog_g (same shapes and dtype
  * as the inputs) and

@@ -422,9 +422,14 @@ hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const
         return from_cuda(h0 ? cudaMemcpyAsync(hT, h0, n, cudaMemcpyDeviceToDevice, stream)
                             : cudaMemsetAsync(hT, 0, n, stream));
     }
+    g_launches += 1;
+    if (use_tc(dk, dv, dtype)) {   // tensor cores: the kScalar instance of the forward kernel
+        TcFwdArgs t{q, k, v, h0, o, hT, nullptr, nullptr, B, T, H, 32, nullptr, nullptr, nullptr, nullptr, dk,
+                    log_g};
+        return from_cuda(launch_tc_fwd(t, stream));
+    }
     ScalarArgs a{q, k, v, log_g, h0, o, hT, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                  nullptr, B, T, H, dk, dv};
-    g_launches += 1;
     return from_cuda(launch_scalar_fwd(a, dtype == HGRN2_BF16, stream));
 }
 

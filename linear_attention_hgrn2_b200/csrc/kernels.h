@@ -31,6 +31,7 @@ struct TcFwdArgs {
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens
     const int *perm;   // with cu: launch order of the sequences (longest first), or null
     int D;             // head size d_k = d_v: 128 or 64
+    const void *lgs;   // scalar-decay variant: log g [B][T][H] (lf is then the key k); else null
 };
 
 struct SimtBwdArgs {

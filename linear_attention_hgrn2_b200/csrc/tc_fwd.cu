@@ -86,10 +86,16 @@ struct Params {
     const int *perm;
     int D;            // head size d_k = d_v: 128, or 64 (the second 64-column half of every operand
                       // tile is held at zero: log f = 0, q = i = 0 there, exactly neutral)
+    const __nv_bfloat16 *lgs;   // scalar-decay variant: log g [B][T][H]; tm_lf then maps the key k
 };
 
-// kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks)
-template <bool kPacked>
+// kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
+// kScalar: the scalar-decay variant S_t = g_t S_{t-1} + k_t v_t^T (one decay per head and token,
+// key k loaded in place of log f).  Its decay factors exactly: A = Q K^T on the raw tiles, the
+// exact e^{b_t - b_s} applied where the TMEM warps mask A, Q rows scaled by e^{b_t} and K rows by
+// e^{B - b_t} after that MMA has read them, and the state scaled by e^{B} before the state MMA
+// adds to it.  Every exponent is <= 0, so nothing is ever flagged.
+template <bool kPacked, bool kScalar = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o,
@@ -200,7 +206,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
             for (int n = 0; n < N; ++n) {
                 const int s = n & 1;
-                if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                // scalar decay: A needs only the raw tiles; otherwise the prepped Qt, Kt
+                if (!mbar_wait(kScalar ? &m->fullQG[s] : &m->prepped[s], (n >> 1) & 1)) {
+                    set_status(HGRN2_ERR_TIMEOUT);
+                    break;
+                }
                 if (ld_volatile(&m->bad_tile) <= n) break;
                 tc_fence_after();
                 // A = Qt Kt^T
@@ -211,6 +221,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(Gb[s]) + ko, 16, 1024), id_kk, kk > 0);
                 }
                 mma_commit(&m->barA);
+                if (kScalar) {   // the prep scales Q and K in place once A has read them
+                    if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+                    tc_fence_after();
+                }
                 // O = Qt bf16(S_in) once the S phase wrote it and the last epilogue read O;
                 // S' = S_in + Kt^T V
                 if (!mbar_wait(&m->sdone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -275,7 +289,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ld_volatile(&m->bad_tile) <= n) break;
             e_prev = e_cur;
-            e_cur = m->EB[s][r];   // the prep warps rewrite this slot only after this chunk's stage is released
+            if (kScalar) e_cur = __expf(m->Ppart[n % 3][kTile - 1]);   // e^{B}, B = the chunk's total log g
+            else e_cur = m->EB[s][r];   // the prep warps rewrite this slot only after this chunk's stage is released
             // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand),
             // once the previous chunk's o store has read X
             if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -284,15 +299,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 named_bar_sync(2, 128);
             }
             tc_fence_after();
-            const float e = e_prev;
+            // scalar decay: S_in is exact already; it is scaled by this chunk's e^{B} for the state MMA
+            const float e = kScalar ? e_cur : e_prev;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
                 tmem_ld32(tl + kColS + 32 * c, v);
                 tmem_wait_ld();
+                if (!kScalar) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= e;
+                    for (int i = 0; i < 32; ++i) v[i] *= e;
+                }
                 store_chunk_bf16(X, r, c, v);
+                if (kScalar) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= e;
+                }
                 tmem_st32(tl + kColS + 32 * c, v);
             }
             tmem_wait_st();
@@ -323,6 +345,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (i > lane) v[i] = 0.0f;
+                    }
+                    if (kScalar) {   // A_rs = (q_r . k_s) e^{b_r - b_s} for s <= r
+                        const float *bv = m->Ppart[n % 3];
+                        const float br = bv[r];
+                        if (c < quad) {
+                            // every column precedes r: e^{b_r - b_e} e^{b_e - b_s} with b_e at the
+                            // block's last column, both factors <= 1; lane l forms column 32c + l's
+                            const float be = bv[32 * c + 31];
+                            const float alpha = __expf(br - be), beta = __expf(be - bv[32 * c + lane]);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= alpha * __shfl_sync(0xffffffffu, beta, i);
+                        } else {   // the diagonal block (columns past r were zeroed above)
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] *= i <= lane ? __expf(br - bv[32 * c + i]) : 0.0f;
+                        }
                     }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = __uint_as_float(pack_bf2(v[2 * i], v[2 * i + 1]));
@@ -387,7 +424,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
         if (n == N && (p.hT || p.hTs) && seg == p.nseg - 1 && r < p.D) {   // warp-uniform
-            const float e = e_cur;
+            const float e = kScalar ? 1.0f : e_cur;   // scalar decay: the state is complete
             float *dst = p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
             float *dsv = p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
 #pragma unroll
@@ -419,6 +456,50 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const int s = n & 1;
             if (!mbar_wait(&m->fullQG[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ptid == 0) m->waited_full = n + 1;
+            if constexpr (kScalar) {
+                // b_t = cumulative log g from the chunk start into a 3-slot ring (the TMEM warps read
+                // slot n % 3 while masking chunk n, which may be after this stage is released: the
+                // prep two chunks ahead writes another slot); 0 past the sequence end
+                float *bv = m->Ppart[n % 3];
+                float *wtot = m->EB[0];   // warp totals of the scan (E_B is not kept for this variant)
+                float a = 0.0f;
+                if (ptid < kTile) {
+                    const int t = tok0 + n * kTile + ptid;
+                    if (t < p.T) a = __bfloat162float(p.lgs[((size_t)bc * p.T + t) * p.H + h]);
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, a, o);
+                        if (lane >= o) a += y;
+                    }
+                    if (lane == 31) wtot[ptid >> 5] = a;
+                }
+                named_bar_sync(1, 256);
+                if (ptid < kTile) {
+                    for (int w = 0; w < (ptid >> 5); ++w) a += wtot[w];
+                    bv[ptid] = a;
+                }
+                named_bar_sync(1, 256);
+                const float Bt = bv[kTile - 1];
+                // Q rows times e^{b_t}, K rows times e^{B - b_t} (both <= 1) once the A MMA has read the
+                // raw tiles; lane l forms the factors of row 32 rr + l and the warp shares them
+                const float bl = bv[32 * rr + lane];
+                const float el = __expf(bl), wl = __expf(Bt - bl);
+                if (!mbar_wait(&m->barA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const int t = 32 * rr + i;
+                    const float et = __shfl_sync(0xffffffffu, el, i), wt = __shfl_sync(0xffffffffu, wl, i);
+                    uint32_t *pq = reinterpret_cast<uint32_t *>(Qb[s] + eoff(t));
+                    uint32_t *pk = reinterpret_cast<uint32_t *>(Gb[s] + eoff(t));
+                    const uint32_t wq = *pq, wk = *pk;
+                    *pq = pack_bf2(bf_lo(wq) * et, bf_hi(wq) * et);
+                    *pk = pack_bf2(bf_lo(wk) * wt, bf_hi(wk) * wt);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 256);
+                mbar_arrive(&m->prepped[s]);
+                continue;
+            }
             const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
             if (rr < 3) {
                 float s0 = 0.0f, s1 = 0.0f;
@@ -489,7 +570,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         for (int k = m->waited_v; k < issued_v; ++k) mbar_wait(&m->fullV[k & 1], (k >> 1) & 1, 2000000u);
     }
     if (tid == 0) {
-        if (p.nseg == 1) p.flags[bh] = fell_back ? 1 : 0;   // sole writer
+        if (kScalar) {}                                       // nothing is ever flagged
+        else if (p.nseg == 1) p.flags[bh] = fell_back ? 1 : 0;   // sole writer
         else if (fell_back) p.flags[bh] = 1;                  // zeroed by the aggregate kernel
         if (fell_back) atomicAdd(&g_counters[0], 1ull);
         else atomicAdd(&g_counters[1], (unsigned long long)N);
@@ -498,7 +580,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
     // exact route for this (b,h) when it runs unsegmented: the pipeline is drained, so the
     // CTA's shared memory is free for the CUDA-core chunkwise forward of the whole sequence
-    if (fell_back && p.nseg == 1) {
+    if (!kScalar && fell_back && p.nseg == 1) {
         __syncthreads();
         const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
         simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T, p.H, p.D,
@@ -747,12 +829,13 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     if (a.st16 && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
         return cudaErrorInvalidValue;
     if (!a.st16) mst = mo;   // unused
-    auto kern = packed ? tcf::fwd_kernel<true> : tcf::fwd_kernel<false>;
+    const bool scalar = a.lgs != nullptr;   // the scalar-decay variant (a.lf is then the key k)
+    auto kern = packed ? tcf::fwd_kernel<true> : scalar ? tcf::fwd_kernel<false, true> : tcf::fwd_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     int nseg = 1, tps = ntiles;
-    if (!packed && a.D == 128) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);   // d = 64: one CTA per (b,h)
+    if (!packed && !scalar && a.D == 128) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);   // else one CTA per (b,h)
     const int BH = a.B * a.H;
     float *U = a.seg_ws, *g = a.seg_ws ? a.seg_ws + (size_t)BH * (nseg - 1) * 16384 : nullptr;
     if (nseg > 1) {
@@ -766,7 +849,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps,
-                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D};
+                  a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D,
+                  (const __nv_bfloat16 *)a.lgs};
     kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     return cudaGetLastError();
 }

@@ -122,3 +122,29 @@ def test_scalar_empty_sequence_passes_states_through(cuda):
     g = to_cuda(inp)
     got = _run(g)
     assert torch.equal(got["hT"], g["h0"]) and torch.equal(got["dh0"], g["dhT"])
+
+
+@pytest.mark.parametrize("d,lb,strong", [(128, 0.5, False), (64, 0.9, False), (128, 0.5, True)],
+                         ids=["d128", "d64", "d128_strong_decay"])
+def test_scalar_tensor_core_forward(cuda, d, lb, strong):
+    # bf16 with d = 128 or 64 runs the scalar-decay instance of the tensor-core forward: chunk
+    # passes are counted on the device, no pair takes another route; with log g = -12 per token
+    # the decay inside a 128-token chunk reaches e^{-1536}, and every factor it forms is <= 1
+    B, T, H = 2, 300, 3
+    inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, lb, seed=1300 + d, h0_sigma=0.1)
+    if strong:
+        inp["log_g"][:] = -12.0
+    g = to_cuda(inp)
+    L.counters(reset=True)
+    o, hT = L.scalar_fwd(g["q"], g["k"], g["v"], g["log_g"], g["h0"], want_hT=True)
+    c = L.counters(reset=True)
+    assert c[1] == B * H * ((T + 127) // 128) and c[0] == 0 and c[2] == 1, c
+    assert L.device_status() == L.OK
+    assert np.isfinite(np64(o)).all() and np.isfinite(np64(hT)).all()
+    for b in range(B):
+        for h in range(H):
+            sl = lambda t: np64(t[b:b + 1, :, h:h + 1])
+            ro, rh = oracle.sd_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["log_g"]),
+                                   np64(inp["h0"][b:b + 1, h:h + 1]))
+            assert err(np64(o[b, :, h]), ro[0, :, 0], torch.bfloat16) <= 2e-2, (b, h)
+            assert err(np64(hT[b, h]), rh[0, 0], torch.bfloat16) <= 2e-2, (b, h)
