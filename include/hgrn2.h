@@ -255,16 +255,17 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
  *   S_t = g_t S_{t-1} + k_t v_t^T,   o_t = S_t^T q_t,   g_t = exp(log_g_t)  (log_g <= 0)
  *   q, k : [B,T,H,dk]   v, o : [B,T,H,dv]   log_g : [B,T,H]   (all dtype)
  *   h0, hT : [B,H,dk,dv] float32 (NULL allowed, as for hgrn2_fwd)
- * The forward runs on tensor cores for bf16 with dk = dv = 128 or 64 (128-token chunks,
- * bf16 operands, fp32 accumulation and state); everything else, and the backward, runs
- * chunkwise on CUDA cores in fp32 arithmetic.  Both routes form only exponents that are
- * differences of in-chunk cumulative sums, so any decay strength is exact.
+ * Forward and backward run on tensor cores for bf16 with dk = dv = 128 or 64 (128-token
+ * chunks, bf16 operands, fp32 accumulation and state); everything else runs chunkwise on
+ * CUDA cores in fp32 arithmetic, exact for any decay strength.
  * 1 <= dk, dv <= 128; any T >= 0; pointers 16-byte aligned.
  * hgrn2_scalar_bwd: gradients dq, dk_out (of k), dv_out (of v), dlog_g (same shapes and dtype
- * as the inputs) and
- * dh0 (NULL: not computed) of L(o, hT) given dO and dhT (NULL: zero).  workspace: device
- * scratch of at least hgrn2_scalar_workspace_size(B, H) bytes ((size_t)-1 for bad sizes). */
-size_t hgrn2_scalar_workspace_size(int B, int H);
+ * as the inputs) and dh0 (NULL: not computed) of L(o, hT) given dO and dhT (NULL: zero).
+ * workspace: device scratch of at least hgrn2_scalar_workspace_size(...) bytes ((size_t)-1 for
+ * bad sizes).  On the tensor-core route (bf16, dk = dv = 128 or 64) the backward runs the forward
+ * again with its chunk states saved into that workspace, then a reverse sweep over them; pairs
+ * whose summed log decay over a 128-token chunk is below -59.8 are recomputed on CUDA cores. */
+size_t hgrn2_scalar_workspace_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype);
 hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g,
                               const float *h0, void *o, float *hT,
                               int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,

@@ -84,7 +84,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_step_lb.restype = i32
     lib.hgrn2_get_device_status.argtypes = [vp]
     lib.hgrn2_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
-    lib.hgrn2_scalar_workspace_size.argtypes = [i32, i32]
+    lib.hgrn2_scalar_workspace_size.argtypes = [i32] * 6
     lib.hgrn2_scalar_workspace_size.restype = sz
     lib.hgrn2_scalar_fwd.argtypes = [vp] * 7 + [i32] * 6 + [vp]
     lib.hgrn2_scalar_fwd.restype = i32
@@ -445,7 +445,7 @@ def scalar_bwd(q, k, v, log_g, dO, h0=None, dhT=None, want_dh0=False):
         _check(dhT, "dhT", torch.float32, (B, H, dk, dv))
     dq, dk_, dv_, dg = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g)
     dh0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
-    nws = _size_or_raise(lib.hgrn2_scalar_workspace_size(B, H), "hgrn2_scalar_workspace_size")
+    nws = _size_or_raise(lib.hgrn2_scalar_workspace_size(B, T, H, dk, dv, _dt(q)), "hgrn2_scalar_workspace_size")
     ws = _workspace(nws, q.device)
     st = lib.hgrn2_scalar_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(dq),
                               _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dh0), B, T, H, dk, dv, _dt(q), _ptr(ws), nws,

@@ -397,6 +397,14 @@ hgrn2_status check_scalar(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype
     if ((long long)B * H > (1ll << 30) || (long long)B * T * H > (1ll << 40)) return HGRN2_ERR_UNSUPPORTED;
     return HGRN2_OK;
 }
+// Workspace of hgrn2_scalar_bwd: <dhT, hT> per (b,h) and q . dq per token (exact route); on the
+// tensor-core route also the chunk states its forward saves and an o scratch.
+size_t scalar_ws_bytes(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    size_t n = align256(sizeof(float) * (size_t)B * H) + align256(sizeof(float) * (size_t)B * T * H);   // rs, q.dq
+    if (use_tc(dk, dv, dtype) && T > 0) n += saved_layout(B, T, H).total + align256((size_t)B * T * H * dv * 2);
+    return n;
+}
+
 bool all_aligned(std::initializer_list<const void *> ptrs) {
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return false;
@@ -404,9 +412,9 @@ bool all_aligned(std::initializer_list<const void *> ptrs) {
 }
 }  // namespace
 
-size_t hgrn2_scalar_workspace_size(int B, int H) {
-    if (B < 1 || H < 1) return (size_t)-1;
-    return align256(sizeof(float) * (size_t)B * H);
+size_t hgrn2_scalar_workspace_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    if (check_scalar(B, T, H, dk, dv, dtype) != HGRN2_OK) return (size_t)-1;
+    return scalar_ws_bytes(B, T, H, dk, dv, dtype);
 }
 
 hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
@@ -429,7 +437,7 @@ hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const
         return from_cuda(launch_tc_fwd(t, stream));
     }
     ScalarArgs a{q, k, v, log_g, h0, o, hT, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                 nullptr, B, T, H, dk, dv};
+                 nullptr, nullptr, B, T, H, dk, dv, nullptr};
     return from_cuda(launch_scalar_fwd(a, dtype == HGRN2_BF16, stream));
 }
 
@@ -443,15 +451,39 @@ hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const
         return HGRN2_ERR_INVALID_ARG;
     if (!all_aligned({q, k, v, log_g, h0, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, workspace}))
         return HGRN2_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < hgrn2_scalar_workspace_size(B, H)) return HGRN2_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < scalar_ws_bytes(B, T, H, dk, dv, dtype)) return HGRN2_ERR_INVALID_ARG;
     if (T == 0) {
         if (!dh0) return HGRN2_OK;
         const size_t n = sizeof(float) * (size_t)B * H * dk * dv;
         return from_cuda(dhT ? cudaMemcpyAsync(dh0, dhT, n, cudaMemcpyDeviceToDevice, stream)
                              : cudaMemsetAsync(dh0, 0, n, stream));
     }
-    ScalarArgs a{q, k, v, log_g, h0, nullptr, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0,
-                 (float *)workspace, B, T, H, dk, dv};
+    float *rs = (float *)workspace;
+    float *qdq = (float *)((char *)workspace + align256(sizeof(float) * (size_t)B * H));
+    const size_t base = align256(sizeof(float) * (size_t)B * H) + align256(sizeof(float) * (size_t)B * T * H);
+    if (use_tc(dk, dv, dtype)) {
+        // tensor cores: the forward keeps its chunk states in the workspace (o goes to scratch),
+        // the reverse sweep reads them; pairs whose chunk decay leaves the factorised form's range
+        // are flagged by the forward and recomputed on the exact route
+        char *sv = (char *)workspace + base;
+        const SavedLayout sl = saved_layout(B, T, H);
+        int *flags = (int *)(sv + sl.flags);
+        float *hTs = (float *)(sv + sl.hTs);
+        TcFwdArgs f{q, k, v, h0, sv + sl.total, nullptr, flags, nullptr, B, T, H, 32, sv, hTs, nullptr, nullptr, dk,
+                    log_g};
+        cudaError_t e = launch_tc_fwd(f, stream);
+        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+        TcBwdArgs r{q, k, v, dO, h0, dhT, dq, dk_out, dv_out, dh0, rs, flags, B, T, H, 32, sv, hTs, nullptr, nullptr,
+                    dk, log_g, dlog_g};
+        e = launch_tc_bwd(r, stream);
+        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+        ScalarArgs a{q, k, v, log_g, h0, nullptr, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, rs, qdq, B, T, H,
+                     dk, dv, flags};
+        g_launches += 4;
+        return from_cuda(launch_scalar_bwd(a, dtype == HGRN2_BF16, stream));
+    }
+    ScalarArgs a{q, k, v, log_g, h0, nullptr, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, rs, qdq, B, T, H, dk,
+                 dv, nullptr};
     g_launches += 2;
     return from_cuda(launch_scalar_bwd(a, dtype == HGRN2_BF16, stream));
 }

@@ -60,6 +60,8 @@ struct TcBwdArgs {
     const int *cu;     // if non-null: packed sequences, B = their number, T = total tokens (needs st16)
     const int *perm;   // with cu: launch order of the sequences (longest first), or null
     int D;             // head size d_k = d_v: 128 or 64 (64: saved-state mode only)
+    const void *lgs;   // scalar-decay variant (saved mode): log g [B][T][H]; lf is then k, dlf dk
+    void *dlg;         // scalar-decay variant: d log g [B][T][H]
 };
 
 struct StepBwdArgs {
@@ -86,7 +88,9 @@ struct ScalarArgs {
     void *dq, *dk_out, *dv_out, *dlg;
     float *dh0;
     float *rs;                      // backward workspace: <dhT, hT> per (b,h)
+    float *qdq;                     // backward workspace: q_t . dq_t per token [B][T][H], fp32
     int B, T, H, dk, dv;
+    const int *only;                // backward: if non-null, only (b,h) with only[b*H+h] != 0
 };
 cudaError_t launch_scalar_fwd(const ScalarArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_scalar_bwd(const ScalarArgs &a, bool bf16, cudaStream_t st);

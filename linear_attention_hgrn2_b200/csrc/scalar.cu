@@ -24,6 +24,8 @@
 // The last line follows from o and hT being homogeneous in the decays; it runs as a reverse
 // cumulative sum across chunks.  One thread block walks the chunks of one (batch, head); the
 // state (or its gradient) stays in shared memory in fp32.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -90,7 +92,9 @@ __device__ __forceinline__ void decay_scores(float *M, const float *X, const flo
 size_t fwd_smem(int dk, int dv) {
     return sizeof(float) * ((size_t)dk * (dv + 1) + 2 * kC * (dk + 1) + kC * (dv + 1) + kC * (kC + 1) + 3 * kC);
 }
-size_t dq_smem(int dk, int dv) { return fwd_smem(dk, dv) + sizeof(float) * kC * (dv + 1); }
+size_t dq_smem(int dk, int dv) {
+    return sizeof(float) * ((size_t)dk * (dv + 1) + 2 * kC * (dk + 1) + 2 * kC * (dv + 1) + kC * (kC + 1) + 4 * kC);
+}
 size_t rev_smem(int dk, int dv) {
     return sizeof(float) * ((size_t)dk * (dv + 1) + 3 * kC * (dk + 1) + 2 * kC * (dv + 1) + 2 * kC * (kC + 1) +
                             5 * kC);
@@ -138,22 +142,26 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
         for (int e = tid; e < dk * dv; e += kThreads) hT[so + e] = S[(e / dv) * lds + e % dv];
 }
 
-// Forward sweep of the backward: dq of every token, and rs = <dhT, hT> for the reverse sweep.
+// Forward sweep of the backward: dq of every token, q_t . dq_t in fp32 (for the reverse sweep's
+// d log g, so that it does not read back the rounded dq), and rs = <dhT, hT>.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-bwd_dq_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ lg,
+bwd_dq_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ lg,
               const float *__restrict__ h0, const T *__restrict__ dO, const float *__restrict__ dhT,
-              T *__restrict__ dq, float *__restrict__ rs, int T_, int H, int dk, int dv) {
+              T *__restrict__ dq, float *__restrict__ qdq, float *__restrict__ rs, int T_, int H, int dk, int dv,
+              const int *only) {
+    if (only && only[blockIdx.x] == 0) return;   // only the pairs the tensor-core route flagged
     extern __shared__ float sm[];
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H, tid = threadIdx.x;
     const int lds = dv + 1, ldk = dk + 1, ldv = dv + 1, lda = kC + 1;
     float *S = sm, *Ks = S + dk * lds, *Vs = Ks + kC * ldk, *Gs = Vs + kC * ldv, *dA = Gs + kC * ldv;
-    float *bs = dA + kC * lda, *es = bs + kC, *ws = es + kC;
+    float *bs = dA + kC * lda, *es = bs + kC, *ws = es + kC, *Qs = ws + kC;
     const size_t so = (size_t)bh * dk * dv;
     for (int e = tid; e < dk * dv; e += kThreads) S[(e / dv) * lds + e % dv] = h0 ? h0[so + e] : 0.0f;
     for (int t0 = 0; t0 < T_; t0 += kC) {
         const int n = min(kC, T_ - t0);
         __syncthreads();
+        load_rows<T>(Qs, ldk, q, b, h, t0, n, T_, H, dk);
         load_rows<T>(Ks, ldk, k, b, h, t0, n, T_, H, dk);
         load_rows<T>(Vs, ldv, v, b, h, t0, n, T_, H, dv);
         load_rows<T>(Gs, ldv, dO, b, h, t0, n, T_, H, dv);
@@ -166,9 +174,16 @@ bwd_dq_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__restr
             float inter = 0.0f, intra = 0.0f;
             for (int c = 0; c < dv; ++c) inter = fmaf(Gs[t * ldv + c], S[j * lds + c], inter);
             for (int s = 0; s <= t; ++s) intra = fmaf(dA[t * lda + s], Ks[s * ldk + j], intra);
-            dq[tidx(b, t0 + t, h, T_, H, dk) + j] = from_f<T>(fmaf(es[t], inter, intra));
+            const float g = fmaf(es[t], inter, intra);
+            dq[tidx(b, t0 + t, h, T_, H, dk) + j] = from_f<T>(g);
+            Qs[t * ldk + j] *= g;   // q dq per element (nothing else reads Qs in this phase)
         }
         __syncthreads();
+        if (tid < n) {   // q_t . dq_t, summed in a fixed order
+            float acc = 0.0f;
+            for (int j = 0; j < dk; ++j) acc += Qs[tid * ldk + j];
+            qdq[gidx(b, t0 + tid, h, T_, H)] = acc;
+        }
         const float eB = es[kC - 1];
         for (int e = tid; e < dk * dv; e += kThreads) {
             const int j = e / dv, c = e - j * dv;
@@ -198,8 +213,10 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ lg,
                const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
-               const float *__restrict__ rs, T *__restrict__ dk_out, T *__restrict__ dv_out,
-               T *__restrict__ dlg, float *__restrict__ dh0, int T_, int H, int dk, int dv) {
+               const float *__restrict__ qdq, const float *__restrict__ rs, T *__restrict__ dk_out,
+               T *__restrict__ dv_out,
+               T *__restrict__ dlg, float *__restrict__ dh0, int T_, int H, int dk, int dv, const int *only) {
+    if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
     const int bh = blockIdx.x, b = bh / H, h = bh - b * H, tid = threadIdx.x;
     const int lds = dv + 1, ldk = dk + 1, ldv = dv + 1, lda = kC + 1;
@@ -243,9 +260,14 @@ bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
             const int t = tid;
             float acc = 0.0f;
             if (t < n) {
-                const size_t r = tidx(b, t0 + t, h, T_, H, dk);
-                for (int j = 0; j < dk; ++j)
-                    acc += Qs[t * ldk + j] * to_f<T>(dq[r + j]) - Ks[t * ldk + j] * DK[t * ldk + j];
+                if (std::is_same<T, float>::value) {   // dq is exact: pair the terms element by element
+                    const size_t r = tidx(b, t0 + t, h, T_, H, dk);
+                    for (int j = 0; j < dk; ++j)
+                        acc += Qs[t * ldk + j] * to_f<T>(dq[r + j]) - Ks[t * ldk + j] * DK[t * ldk + j];
+                } else {   // dq was rounded to bf16: q . dq from the forward sweep's fp32 sum
+                    acc = qdq[gidx(b, t0 + t, h, T_, H)];
+                    for (int j = 0; j < dk; ++j) acc -= Ks[t * ldk + j] * DK[t * ldk + j];
+                }
             }
             term[t] = acc;
         }
@@ -298,14 +320,14 @@ static cudaError_t launch_sd_bwd_t(const ScalarArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(sd::bwd_rev_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     if (e != cudaSuccess) return e;
-    sd::bwd_dq_kernel<T><<<a.B * a.H, sd::kThreads, s1, st>>>((const T *)a.k, (const T *)a.v, (const T *)a.lg, a.h0,
-                                                               (const T *)a.dO, a.dhT, (T *)a.dq, a.rs, a.T, a.H,
-                                                               a.dk, a.dv);
+    sd::bwd_dq_kernel<T><<<a.B * a.H, sd::kThreads, s1, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
+                                                               (const T *)a.lg, a.h0, (const T *)a.dO, a.dhT,
+                                                               (T *)a.dq, a.qdq, a.rs, a.T, a.H, a.dk, a.dv, a.only);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     sd::bwd_rev_kernel<T><<<a.B * a.H, sd::kThreads, s2, st>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.lg, (const T *)a.dO, a.dhT, (const T *)a.dq,
-        a.rs, (T *)a.dk_out, (T *)a.dv_out, (T *)a.dlg, a.dh0, a.T, a.H, a.dk, a.dv);
+        a.qdq, a.rs, (T *)a.dk_out, (T *)a.dv_out, (T *)a.dlg, a.dh0, a.T, a.H, a.dk, a.dv, a.only);
     return cudaGetLastError();
 }
 

@@ -29,6 +29,8 @@
 // Validity and fallback are those of the forward: a (batch, head) whose chunk
 // decay span exceeds the factorisation's range is flagged by the forward sweep,
 // skipped by the reverse sweep, and recomputed by the exact route.
+#include <cstddef>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -437,6 +439,8 @@ struct __align__(8) Misc {
     float carry[128];
 };
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
+static_assert(offsetof(Misc, Bpart) == offsetof(Misc, EB) + sizeof(float) * 128,
+              "the scalar-decay reduction uses EB and Bpart as one [4][128] array");
 }  // namespace rsw
 
 struct RevParams {
@@ -455,11 +459,18 @@ struct RevParams {
     const int *perm;     // with cu: CTA row r runs sequence perm[r]
     int D;               // head size d_k = d_v: 128, or 64 (saved mode; the second 64-column half of
                          // every operand tile is held at zero, which is exactly neutral)
+    const __nv_bfloat16 *lgs;   // scalar decay: log g [B][T][H] (lf is then the key k, dlf its gradient)
+    __nv_bfloat16 *dlg;         // scalar decay: d log g [B][T][H]
 };
 
 // kPacked (saved mode only): p.cu holds packed sequences; compiled apart so the dense path
-// carries no row masks
-template <bool kSaved, bool kPacked>
+// carries no row masks.
+// kScalar (saved mode only): the scalar-decay variant S_t = g_t S_{t-1} + k_t v_t^T.  Its chunk
+// math is this kernel's with Qt = q E_t, Kt = k / E_t for a decay E_t shared by every key dim:
+// the prep scans the gate per row instead of forming k = 1 - f; the epilogue writes dk = dk_pre /
+// E in place of d log f, has no tied-key term, and sums the per-dim reverse sums over d_k into
+// d log g_t.  Flagged pairs return at once; the host recomputes them on the exact route.
+template <bool kSaved, bool kPacked, bool kScalar = false>
 __global__ void __launch_bounds__(rsw::kRevThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
@@ -492,7 +503,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     auto valid_rows = [&](int n) -> int { return kPacked ? min(kTile, len - n * kTile) : kTile; };
     if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
-        if (kSaved) {         // both sweeps here (recompute mode: in the forward-sweep kernel)
+        if (kSaved && !kScalar) {   // both sweeps here (recompute mode: in the forward-sweep kernel)
             float *sm = reinterpret_cast<float *>(smem);
             const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
             const int Tl = kPacked ? len : p.T;
@@ -612,6 +623,52 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // product of f from the range start, 1/E = e^{-b}.
         {
             const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
+            float bsum = 0.0f;   // per-dim: the running log-decay sum; scalar decay: the chunk's total
+            float ev[32];
+            if constexpr (kScalar) {
+                // b_t = cumulative log g from the chunk start (0 past the sequence end), threads 0..127
+                float a = 0.0f;
+                if (tid < kTile) {
+                    const int t = tok0 + n * kTile + tid;
+                    if (t < p.T) a = __bfloat162float(p.lgs[((size_t)bc * p.T + t) * p.H + h]);
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, a, o);
+                        if (lane >= o) a += y;
+                    }
+                    if (lane == 31) m->Bpart[1][tid >> 5] = a;
+                }
+                __syncthreads();
+                if (tid < kTile) {
+                    for (int w = 0; w < (tid >> 5); ++w) a += m->Bpart[1][w];
+                    m->Bpart[0][tid] = a;
+                }
+                __syncthreads();
+                bsum = m->Bpart[0][kTile - 1];
+#pragma unroll
+                for (int bt = 0; bt < 4; ++bt) {   // Qt = q e^{b_t}, Kt = k e^{-b_t} (b_t >= the range bound)
+                    const int t0 = c0 + 8 * bt;
+                    float kv[8], qv[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        kv[i] = bfat(Gb, t0 + i);
+                        qv[i] = bfat(Qb, t0 + i);
+                    }
+                    __nv_bfloat16 oq[8], ok2[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float b = m->Bpart[0][t0 + i], E = __expf(b);
+                        ok2[i] = __float2bfloat16_rn(kv[i] * __expf(-b));
+                        oq[i] = __float2bfloat16_rn(qv[i] * E);
+                        ev[8 * bt + i] = E;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        *reinterpret_cast<__nv_bfloat16 *>(Gb + eoff(t0 + i)) = ok2[i];
+                        *reinterpret_cast<__nv_bfloat16 *>(Qb + eoff(t0 + i)) = oq[i];
+                    }
+                }
+            } else {
             float sum = 0.0f;
             if (q4 < 3) {
 #pragma unroll 8
@@ -619,10 +676,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 m->Bpart[q4][j] = sum;
             }
             __syncthreads();
-            float bsum = 0.0f;
             for (int r2 = 0; r2 < q4; ++r2) bsum += m->Bpart[r2][j];
             float E = __expf(bsum);
-            float ev[32];
 #pragma unroll
             for (int bt = 0; bt < 4; ++bt) {
                 const int t0 = c0 + 8 * bt;
@@ -648,6 +703,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     *reinterpret_cast<__nv_bfloat16 *>(Qb + eoff(t0 + i)) = oq[i];
                 }
             }
+            }   // per-dim prep
             tmem_st32(tl + kColE + c0, ev);
             tmem_wait_st();
             if (q4 == 3) m->EB[j] = __expf(bsum);
@@ -873,7 +929,12 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 } else {
                     suf += qt * invE * bfat(D16, t) - kt * dkp[i];
                 }
-                dap[i] = suf - dkp[i] * invEm1;
+                if (kScalar) {   // dk = dk_pre / E into DA (row t); no tied-key term
+                    *reinterpret_cast<__nv_bfloat16 *>(DA + eoff(t)) = __float2bfloat16_rn(dkp[i] * __fdividef(1.0f, e[i]));
+                    dap[i] = suf;
+                } else {
+                    dap[i] = suf - dkp[i] * invEm1;
+                }
                 invE = invEm1;
             }
             tmem_st16(tl + kColX1 + col, dap);
@@ -890,14 +951,42 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             float dap[32];
             tmem_ld32(tl + kColX1 + c0, dap);
             tmem_wait_ld();
+            if constexpr (kScalar) {
+                // d log g_t = sum_j (d'_t[j] + carry_j): the warp's 32 key dims by a butterfly (lane l
+                // ends with token c0 + l), then the four key-dim quarters through shared memory (EB and
+                // Bpart, free once every thread has read its carry and the next carry is in a register)
+                const float nc = m->carry[j] + m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                *reinterpret_cast<__nv_bfloat16 *>(DA + eoff(c0 + i)) = __float2bfloat16_rn(dap[i] + carry);
+                for (int i = 0; i < 32; ++i) dap[i] += carry;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    const bool up = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < o; ++i) {
+                        const float send = up ? dap[i] : dap[i + o];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+                        dap[i] = (up ? dap[i + o] : dap[i]) + recv;
+                    }
+                }
+                __syncthreads();
+                if (q4 == 0) m->carry[j] = nc;
+                float *red = m->EB;   // EB[128] and Bpart[3][128], contiguous: [key-dim quarter][token]
+                red[quad * kTile + c0 + lane] = dap[0];
+                __syncthreads();
+                const int tok = n * kTile + tid;
+                if (tid < kTile && tok < p.T)
+                    p.dlg[((size_t)bc * p.T + tok) * p.H + h] =
+                        __float2bfloat16_rn(red[tid] + red[kTile + tid] + red[2 * kTile + tid] + red[3 * kTile + tid]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(DA + eoff(c0 + i)) = __float2bfloat16_rn(dap[i] + carry);
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (q4 == 0) m->carry[j] += m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
+        if (!kScalar && q4 == 0) m->carry[j] += m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
         const int vr = valid_rows(n);
         if (vr == kTile) {
             if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
@@ -953,7 +1042,8 @@ size_t tc_bwd_smem() { return tcb::fsw::kSmemBytes > tcb::rsw::kSmemBytes ? tcb:
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     const bool saved = a.st16 != nullptr;
     const bool packed = a.cu != nullptr;   // saved mode only; a.B is then the number of sequences
-    if ((packed || a.D != 128) && !saved) return cudaErrorInvalidValue;
+    if ((packed || a.D != 128 || a.lgs) && !saved) return cudaErrorInvalidValue;
+    if (a.lgs && packed) return cudaErrorInvalidValue;
     const int Bm = packed ? 1 : a.B, D = a.D;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl, mst;
@@ -969,14 +1059,16 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     tcb::RevParams p2{a.dhT, a.rs, a.dh0, a.flags, a.T, a.H, ntiles, a.hTs, a.h0,
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
-                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm, D};
+                      (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm, D, (const __nv_bfloat16 *)a.lgs,
+                      (__nv_bfloat16 *)a.dlg};
     cudaError_t e;
     if (saved) {
         // one launch; the exact route of a flagged (b,h) runs in the same shared memory
         size_t smem = tcb::rsw::kSmemBytes;
         if (simt_bwd_dq_smem(a.simt_C, D, D) > smem) smem = simt_bwd_dq_smem(a.simt_C, D, D);
         if (simt_bwd_rev_smem(a.simt_C, D, D) > smem) smem = simt_bwd_rev_smem(a.simt_C, D, D);
-        auto kern = packed ? tcb::rev_kernel<true, true> : tcb::rev_kernel<true, false>;
+        auto kern = packed ? tcb::rev_kernel<true, true>
+                    : a.lgs ? tcb::rev_kernel<true, false, true> : tcb::rev_kernel<true, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         kern<<<a.B * a.H, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);

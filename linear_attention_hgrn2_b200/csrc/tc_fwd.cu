@@ -61,6 +61,7 @@ struct __align__(8) Misc {
     uint64_t sdone, adone, ofree;           // TMEM-warp arrivals (128 each)
     uint32_t tmem_base;
     int bad_tile;                           // first chunk whose decay span is too wide
+    int sflag;                              // scalar decay: a chunk's total log g < kMinLogEB (for the backward)
     int waited_full;                        // q / log f arrivals the prep warps consumed
     int waited_v;                           // v arrivals the MMA thread consumed
     float EB[2][128];                       // E_B ring: read by the TMEM warps while that chunk is current
@@ -94,7 +95,8 @@ struct Params {
 // key k loaded in place of log f).  Its decay factors exactly: A = Q K^T on the raw tiles, the
 // exact e^{b_t - b_s} applied where the TMEM warps mask A, Q rows scaled by e^{b_t} and K rows by
 // e^{B - b_t} after that MMA has read them, and the state scaled by e^{B} before the state MMA
-// adds to it.  Every exponent is <= 0, so nothing is ever flagged.
+// adds to it.  Every exponent is <= 0, so the forward is exact for any decay; a pair whose chunk
+// decay leaves the backward's factorisation range is flagged for the backward.
 template <bool kPacked, bool kScalar = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
@@ -149,6 +151,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->adone, 128);
         mbar_init(&m->ofree, 128);
         m->bad_tile = INT_MAX;
+        m->sflag = 0;
         m->waited_full = 0;
         m->waited_v = 0;
         fence_mbar_init();
@@ -480,6 +483,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
                 named_bar_sync(1, 256);
                 const float Bt = bv[kTile - 1];
+                // the forward is exact for any decay; the backward's factorised form is not past this
+                if (ptid == 0 && !(Bt >= kMinLogEB)) m->sflag = 1;
                 // Q rows times e^{b_t}, K rows times e^{B - b_t} (both <= 1) once the A MMA has read the
                 // raw tiles; lane l forms the factors of row 32 rr + l and the warp shares them
                 const float bl = bv[32 * rr + lane];
@@ -570,7 +575,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         for (int k = m->waited_v; k < issued_v; ++k) mbar_wait(&m->fullV[k & 1], (k >> 1) & 1, 2000000u);
     }
     if (tid == 0) {
-        if (kScalar) {}                                       // nothing is ever flagged
+        if (kScalar) { if (p.flags) p.flags[bh] = m->sflag; }   // for the backward only
         else if (p.nseg == 1) p.flags[bh] = fell_back ? 1 : 0;   // sole writer
         else if (fell_back) p.flags[bh] = 1;                  // zeroed by the aggregate kernel
         if (fell_back) atomicAdd(&g_counters[0], 1ull);

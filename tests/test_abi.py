@@ -213,8 +213,13 @@ def test_selftest_checks_its_poll_count_before_any_launch(lib):
 def test_scalar_decay_argument_checks_before_any_launch(lib):
     vp = ctypes.c_void_p
     bad = ctypes.c_size_t(-1).value
-    assert lib.hgrn2_scalar_workspace_size(0, 4) == bad
-    assert lib.hgrn2_scalar_workspace_size(2, 3) == 256
+    up = lambda x: (x + 255) // 256 * 256
+    assert lib.hgrn2_scalar_workspace_size(0, 8, 4, 16, 16, L.FP32) == bad
+    # exact route: <dhT, hT> per (b,h) and q . dq per token, fp32
+    assert lib.hgrn2_scalar_workspace_size(2, 8, 3, 16, 16, L.FP32) == up(4 * 2 * 3) + up(4 * 2 * 8 * 3)
+    B, T, H = 2, 300, 3   # tensor-core route: + the saved chunk states and an o scratch
+    assert lib.hgrn2_scalar_workspace_size(B, T, H, 128, 128, L.BF16) == (
+        up(4 * B * H) + up(4 * B * T * H) + lib.hgrn2_saved_size(B, T, H, 128, 128, L.BF16) + up(B * T * H * 128 * 2))
     f = lib.hgrn2_scalar_fwd
     assert f(vp(16), vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 256, 16, L.FP32, None) == L.ERR_UNSUPPORTED
     assert f(None, vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 16, 16, L.FP32, None) == L.ERR_INVALID_ARG
@@ -224,3 +229,4 @@ def test_scalar_decay_argument_checks_before_any_launch(lib):
     args = [vp(16)] * 4 + [None, vp(16), None] + [vp(16)] * 4 + [None]
     assert g(*args, 2, 8, 3, 16, 16, L.BF16, None, 0, None) == L.ERR_INVALID_ARG
     assert g(*args, 2, 8, 3, 16, 16, L.BF16, vp(256), 255, None) == L.ERR_INVALID_ARG
+    assert g(*args, 2, 300, 3, 128, 128, L.BF16, vp(256), 256, None) == L.ERR_INVALID_ARG   # no room for states

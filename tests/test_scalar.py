@@ -148,3 +148,26 @@ def test_scalar_tensor_core_forward(cuda, d, lb, strong):
                                    np64(inp["h0"][b:b + 1, h:h + 1]))
             assert err(np64(o[b, :, h]), ro[0, :, 0], torch.bfloat16) <= 2e-2, (b, h)
             assert err(np64(hT[b, h]), rh[0, 0], torch.bfloat16) <= 2e-2, (b, h)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_scalar_tensor_core_backward_with_a_flagged_head(cuda, d):
+    # bf16 d = 128 / 64: the backward runs the forward again (chunk states saved into the workspace)
+    # and the tensor-core reverse sweep: 4 launches (forward, reverse sweep, the exact route's two
+    # kernels for flagged pairs).  Head (1, 2) has log g = -1 per token, a chunk total of -128,
+    # past the factorised form's range: it is recomputed on CUDA cores; the rest stays on the
+    # tensor cores.  Every gradient must match the oracle.
+    B, T, H = 2, 300, 3
+    inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, 0.9, seed=1400 + d, h0_sigma=0.1, with_dO=True,
+                               dhT_sigma=0.1)
+    inp["log_g"][1, :, 2] = -1.0
+    g = to_cuda(inp)
+    L.counters(reset=True)
+    dq, dk, dv, dg, dh0 = L.scalar_bwd(g["q"], g["k"], g["v"], g["log_g"], g["dO"], g["h0"], g["dhT"],
+                                       want_dh0=True)
+    c = L.counters(reset=True)
+    assert c[2] == 4, c
+    assert L.device_status() == L.OK
+    o, hT = L.scalar_fwd(g["q"], g["k"], g["v"], g["log_g"], g["h0"], want_hT=True)
+    got = {"o": o, "hT": hT, "dq": dq, "dk": dk, "dv": dv, "dlog_g": dg, "dh0": dh0}
+    _check(inp, got, [(b, h) for b in range(B) for h in range(H)], torch.bfloat16, 2e-2)
