@@ -604,13 +604,9 @@ def run_fwd_configs(args, dev, pk, rank):
     return res
 
 
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA/clock x 2 flop x 1.965 GHz (max SM clock)
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-
-
 def run_scalar(args, dev, pk, rank):
     """The scalar-decay variant (one decay per head and token, explicit key) at the training
-    workload's shape: hgrn2_scalar_fwd + hgrn2_scalar_bwd, CUDA cores, chunks of 32."""
+    workload's shape: hgrn2_scalar_fwd + hgrn2_scalar_bwd."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
     w = I.SCALAR_TRAIN
@@ -627,7 +623,7 @@ def run_scalar(args, dev, pk, rank):
         fwd_call()
         bwd_call()
     torch.cuda.synchronize()
-    K = max(3, min(args.steps, 10))
+    K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     ev[0].record()
     for _ in range(K):
@@ -639,17 +635,18 @@ def run_scalar(args, dev, pk, rank):
     torch.cuda.synchronize()
     fwd_ms = ev[0].elapsed_time(ev[1]) / K
     bwd_ms = ev[1].elapsed_time(ev[2]) / K
-    # algorithmic flops of the chunkwise forward per token-head at chunk C: causal scores
-    # (C/2 * dk * 2), intra outputs (C/2 * dv * 2), inter outputs and state update (2 * dk*dv * 2)
-    C, dk, dv = 32, w.dk, w.dv
-    fwd_flops = (C // 2) * (dk + dv) * 2 + 4 * dk * dv
+    # algorithmic bytes per token-head (bf16): forward reads q, k, v, log g and writes o; backward
+    # reads q, k, v, log g, dO and writes dq, dk, dv, d log g
+    dk, dv = w.dk, w.dv
+    step_bytes = 2 * (2 * dk + dv + 1 + dv) + 2 * (2 * dk + 2 * dv + 1 + 2 * dk + dv + 1)
     th = w.B * w.T * w.H
-    tf = fwd_flops * th / (fwd_ms / 1e3) / 1e12
     res = {"workload": w.name, "tokens_per_s": round(w.B * w.T / ((fwd_ms + bwd_ms) / 1e3), 1),
-           "fwd_ms": round(fwd_ms, 3), "bwd_ms": round(bwd_ms, 3), "route": "exact (CUDA cores, fp32 arithmetic)",
-           "fwd_roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(FP32_PEAK_TFLOPS, 1),
-                            "unit": "TFLOP/s", "frac": round(tf / FP32_PEAK_TFLOPS, 4),
-                            "peak_source": "148 SMs x 128 fp32 FMA/clock x 1.965 GHz"},
+           "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+           "route": "tensor cores (the backward re-runs the forward to save chunk states, then a reverse sweep)",
+           "step_hbm": {"achieved_gbs": round(step_bytes * th / ((fwd_ms + bwd_ms) / 1e3) / 1e9, 1),
+                        "peak_gbs": pk["hbm_gbs"],
+                        "frac": round(step_bytes * th / ((fwd_ms + bwd_ms) / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+                        "bytes_per_token_head": step_bytes},
            "calls": "hgrn2_scalar_fwd + hgrn2_scalar_bwd", "steps": K}
     del g, inp
     torch.cuda.empty_cache()
