@@ -261,11 +261,13 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
  * 1 <= dk, dv <= 128; any T >= 0; pointers 16-byte aligned.
  * hgrn2_scalar_bwd: gradients dq, dk_out (of k), dv_out (of v), dlog_g (same shapes and dtype
  * as the inputs) and dh0 (NULL: not computed) of L(o, hT) given dO and dhT (NULL: zero).
- * workspace: device scratch of at least hgrn2_scalar_workspace_size(...) bytes ((size_t)-1 for
- * bad sizes).  On the tensor-core route (bf16, dk = dv = 128 or 64) the backward runs the forward
- * again with its chunk states saved into that workspace, then a reverse sweep over them; pairs
- * whose summed log decay over a 128-token chunk is below -59.8 are recomputed on CUDA cores. */
-size_t hgrn2_scalar_workspace_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype);
+ * workspace: device scratch of at least hgrn2_scalar_workspace_size(..., 1) bytes.  On the
+ * tensor-core route (bf16, dk = dv = 128 or 64) this backward runs the forward again with its
+ * chunk states saved into that workspace, then a reverse sweep over them; pairs whose summed log
+ * decay over a 128-token chunk is below -59.8 are recomputed on CUDA cores.
+ * hgrn2_scalar_workspace_size: bytes of workspace for the forward (want_bwd = 0: none),
+ * hgrn2_scalar_bwd (1) or hgrn2_scalar_bwd_saved (2); (size_t)-1 for bad sizes. */
+size_t hgrn2_scalar_workspace_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype, int want_bwd);
 hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g,
                               const float *h0, void *o, float *hT,
                               int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
@@ -275,6 +277,26 @@ hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const
                               void *dq, void *dk_out, void *dv_out, void *dlog_g, float *dh0,
                               int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
                               void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* The scalar-decay training pair: hgrn2_scalar_fwd_train is hgrn2_scalar_fwd that also keeps
+ * what hgrn2_scalar_bwd_saved reads (the bf16 state entering every 128-token chunk, the fp32 final
+ * state and the range flags) in `saved`, a device buffer of hgrn2_scalar_saved_size(...) bytes
+ * (0 where there is no saved-state path: fp32, other head sizes or T = 0; then `saved` may be
+ * NULL and the backward takes the exact route).  hgrn2_scalar_bwd_saved is hgrn2_scalar_bwd
+ * reading that buffer instead of running the forward again; its workspace is
+ * hgrn2_scalar_workspace_size(..., 2) bytes.  A buffer shorter than the saved size returns
+ * HGRN2_ERR_INVALID_ARG before any launch. */
+size_t hgrn2_scalar_saved_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype);
+hgrn2_status hgrn2_scalar_fwd_train(const void *q, const void *k, const void *v, const void *log_g,
+                                    const float *h0, void *o, float *hT, void *saved, size_t saved_bytes,
+                                    int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                                    cudaStream_t stream);
+hgrn2_status hgrn2_scalar_bwd_saved(const void *q, const void *k, const void *v, const void *log_g,
+                                    const float *h0, const void *saved, size_t saved_bytes,
+                                    const void *dO, const float *dhT,
+                                    void *dq, void *dk_out, void *dv_out, void *dlog_g, float *dh0,
+                                    int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                                    void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* Check of the failure reporting: launches one block that waits, through the bounded
  * wait every kernel of the library uses, on a barrier that nothing arrives at.  The

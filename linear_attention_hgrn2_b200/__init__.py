@@ -31,7 +31,7 @@ EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size",
            "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_lb", "hgrn2_step_bwd",
            "hgrn2_step_lb_bwd", "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string",
            "hgrn2_version", "hgrn2_selftest_wait_timeout", "hgrn2_scalar_workspace_size", "hgrn2_scalar_fwd",
-           "hgrn2_scalar_bwd")
+           "hgrn2_scalar_bwd", "hgrn2_scalar_saved_size", "hgrn2_scalar_fwd_train", "hgrn2_scalar_bwd_saved")
 
 _lib = None
 
@@ -84,7 +84,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_step_lb.restype = i32
     lib.hgrn2_get_device_status.argtypes = [vp]
     lib.hgrn2_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
-    lib.hgrn2_scalar_workspace_size.argtypes = [i32] * 6
+    lib.hgrn2_scalar_workspace_size.argtypes = [i32] * 7
+    lib.hgrn2_scalar_saved_size.argtypes = [i32] * 6
+    lib.hgrn2_scalar_saved_size.restype = sz
+    lib.hgrn2_scalar_fwd_train.argtypes = [vp] * 8 + [sz] + [i32] * 6 + [vp]
+    lib.hgrn2_scalar_fwd_train.restype = i32
+    lib.hgrn2_scalar_bwd_saved.argtypes = [vp] * 6 + [sz] + [vp] * 7 + [i32] * 6 + [vp, sz, vp]
+    lib.hgrn2_scalar_bwd_saved.restype = i32
     lib.hgrn2_scalar_workspace_size.restype = sz
     lib.hgrn2_scalar_fwd.argtypes = [vp] * 7 + [i32] * 6 + [vp]
     lib.hgrn2_scalar_fwd.restype = i32
@@ -407,11 +413,26 @@ def step_lb_bwd(q, g, i, lb: float, S, dO, dS=None, dS_out=None):
     return _step_bwd(load_library().hgrn2_step_lb_bwd, "hgrn2_step_lb_bwd", q, g, i, S, dO, dS, lb, dS_out)
 
 
-def scalar_fwd(q, k, v, log_g, h0=None, want_hT=False):
+def scalar_saved_size(B, T, H, dk, dv, dtype=torch.bfloat16) -> int:
+    """Bytes of the buffer scalar_fwd(..., saved=) fills for scalar_bwd(..., saved=) (0: none)."""
+    return _size_or_raise(load_library().hgrn2_scalar_saved_size(B, T, H, dk, dv,
+                                                                  BF16 if dtype == torch.bfloat16 else FP32),
+                          "hgrn2_scalar_saved_size")
+
+
+def new_scalar_saved(q: torch.Tensor, dv: int | None = None) -> torch.Tensor | None:
+    """An uninitialised saved-state buffer for a scalar-decay forward on q (None if not needed)."""
+    B, T, H, dk = q.shape
+    n = scalar_saved_size(B, T, H, dk, dk if dv is None else dv, q.dtype)
+    return torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+
+
+def scalar_fwd(q, k, v, log_g, h0=None, want_hT=False, saved=None):
     """Scalar-decay variant: S_t = g_t S_{t-1} + k_t v_t^T, o_t = S_t^T q_t, g_t = exp(log_g_t).
 
     q, k: [B,T,H,dk]; v: [B,T,H,dv]; log_g: [B,T,H] (same dtype); h0: [B,H,dk,dv] float32 or
-    None.  Returns (o, hT or None)."""
+    None.  saved: new_scalar_saved() buffer that receives the chunk states for
+    scalar_bwd(..., saved=), or None.  Returns (o, hT or None)."""
     lib = load_library()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -423,14 +444,21 @@ def scalar_fwd(q, k, v, log_g, h0=None, want_hT=False):
         _check(h0, "h0", torch.float32, (B, H, dk, dv))
     o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_hT else None
+    if saved is not None:
+        _check(saved, "saved", torch.uint8)
+        st = lib.hgrn2_scalar_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(o), _ptr(hT),
+                                        _ptr(saved), saved.numel(), B, T, H, dk, dv, _dt(q), _stream())
+        _raise(st, "hgrn2_scalar_fwd_train")
+        return o, hT
     st = lib.hgrn2_scalar_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(o), _ptr(hT),
                               B, T, H, dk, dv, _dt(q), _stream())
     _raise(st, "hgrn2_scalar_fwd")
     return o, hT
 
 
-def scalar_bwd(q, k, v, log_g, dO, h0=None, dhT=None, want_dh0=False):
-    """Gradients (dq, dk, dv, dlog_g, dh0 or None) of the scalar-decay variant."""
+def scalar_bwd(q, k, v, log_g, dO, h0=None, dhT=None, want_dh0=False, saved=None):
+    """Gradients (dq, dk, dv, dlog_g, dh0 or None) of the scalar-decay variant.  saved: the buffer
+    a scalar_fwd(..., saved=) on the same inputs filled, or None (the forward then runs again)."""
     lib = load_library()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -445,8 +473,16 @@ def scalar_bwd(q, k, v, log_g, dO, h0=None, dhT=None, want_dh0=False):
         _check(dhT, "dhT", torch.float32, (B, H, dk, dv))
     dq, dk_, dv_, dg = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_g)
     dh0 = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None
-    nws = _size_or_raise(lib.hgrn2_scalar_workspace_size(B, T, H, dk, dv, _dt(q)), "hgrn2_scalar_workspace_size")
+    nws = _size_or_raise(lib.hgrn2_scalar_workspace_size(B, T, H, dk, dv, _dt(q), 2 if saved is not None else 1),
+                         "hgrn2_scalar_workspace_size")
     ws = _workspace(nws, q.device)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8)
+        st = lib.hgrn2_scalar_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(saved), saved.numel(),
+                                        _ptr(dO), _ptr(dhT), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dh0),
+                                        B, T, H, dk, dv, _dt(q), _ptr(ws), nws, _stream())
+        _raise(st, "hgrn2_scalar_bwd_saved")
+        return dq, dk_, dv_, dg, dh0
     st = lib.hgrn2_scalar_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_g), _ptr(h0), _ptr(dO), _ptr(dhT), _ptr(dq),
                               _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dh0), B, T, H, dk, dv, _dt(q), _ptr(ws), nws,
                               _stream())
@@ -499,3 +535,30 @@ class HGRN2Function(torch.autograd.Function):
 def hgrn2(q, log_f, i, h0=None, chunk=64):
     """Differentiable HGRN2 recurrence: returns (o, hT)."""
     return HGRN2Function.apply(q, log_f, i, h0, chunk)
+
+
+class ScalarDecayFunction(torch.autograd.Function):
+    """Autograd wrapper of the scalar-decay variant: o, hT = ScalarDecayFunction.apply(q, k, v, log_g, h0)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_g, h0=None):
+        q, k, v, log_g = q.contiguous(), k.contiguous(), v.contiguous(), log_g.contiguous()
+        h0 = None if h0 is None else h0.contiguous()
+        saved = new_scalar_saved(q, v.shape[-1])   # chunk states for the backward (None: recompute)
+        o, hT = scalar_fwd(q, k, v, log_g, h0, want_hT=True, saved=saved)
+        ctx.save_for_backward(q, k, v, log_g, h0, saved)
+        ctx.has_h0 = h0 is not None
+        return o, hT
+
+    @staticmethod
+    def backward(ctx, dO, dhT):
+        q, k, v, log_g, h0, saved = ctx.saved_tensors
+        dq, dk, dv, dg, dh0 = scalar_bwd(q, k, v, log_g, dO.contiguous(), h0,
+                                         None if dhT is None else dhT.contiguous(), want_dh0=ctx.has_h0,
+                                         saved=saved)
+        return dq, dk, dv, dg, dh0
+
+
+def scalar_decay(q, k, v, log_g, h0=None):
+    """Differentiable scalar-decay variant: returns (o, hT)."""
+    return ScalarDecayFunction.apply(q, k, v, log_g, h0)

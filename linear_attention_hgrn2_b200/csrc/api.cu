@@ -399,9 +399,11 @@ hgrn2_status check_scalar(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype
 }
 // Workspace of hgrn2_scalar_bwd: <dhT, hT> per (b,h) and q . dq per token (exact route); on the
 // tensor-core route also the chunk states its forward saves and an o scratch.
-size_t scalar_ws_bytes(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+size_t scalar_ws_bytes(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype, int want) {
+    if (want == 0) return 0;   // the forward needs none
     size_t n = align256(sizeof(float) * (size_t)B * H) + align256(sizeof(float) * (size_t)B * T * H);   // rs, q.dq
-    if (use_tc(dk, dv, dtype) && T > 0) n += saved_layout(B, T, H).total + align256((size_t)B * T * H * dv * 2);
+    if (want == 1 && use_tc(dk, dv, dtype) && T > 0)   // no saved states: room for them and an o scratch
+        n += saved_layout(B, T, H).total + align256((size_t)B * T * H * dv * 2);
     return n;
 }
 
@@ -412,18 +414,19 @@ bool all_aligned(std::initializer_list<const void *> ptrs) {
 }
 }  // namespace
 
-size_t hgrn2_scalar_workspace_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
-    if (check_scalar(B, T, H, dk, dv, dtype) != HGRN2_OK) return (size_t)-1;
-    return scalar_ws_bytes(B, T, H, dk, dv, dtype);
-}
+}  // extern "C"
 
-hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
-                              void *o, float *hT, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
-                              cudaStream_t stream) {
+namespace {
+
+// Scalar-decay forward; `saved` (null, or scalar_saved_bytes) receives the chunk states and the
+// range flags that the reverse sweep reads (tensor-core route only).
+hgrn2_status scalar_fwd_impl(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                             void *o, float *hT, void *saved, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                             cudaStream_t stream) {
     hgrn2_status s = check_scalar(B, T, H, dk, dv, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !k || !v || !log_g || !o)) return HGRN2_ERR_INVALID_ARG;
-    if (!all_aligned({q, k, v, log_g, h0, o, hT})) return HGRN2_ERR_INVALID_ARG;
+    if (!all_aligned({q, k, v, log_g, h0, o, hT, saved})) return HGRN2_ERR_INVALID_ARG;
     if (T == 0) {
         if (!hT) return HGRN2_OK;
         const size_t n = sizeof(float) * (size_t)B * H * dk * dv;
@@ -432,8 +435,10 @@ hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const
     }
     g_launches += 1;
     if (use_tc(dk, dv, dtype)) {   // tensor cores: the kScalar instance of the forward kernel
-        TcFwdArgs t{q, k, v, h0, o, hT, nullptr, nullptr, B, T, H, 32, nullptr, nullptr, nullptr, nullptr, dk,
-                    log_g};
+        const SavedLayout sl = saved_layout(B, T, H);
+        int *flags = saved ? (int *)((char *)saved + sl.flags) : nullptr;
+        float *hTs = saved ? (float *)((char *)saved + sl.hTs) : nullptr;
+        TcFwdArgs t{q, k, v, h0, o, hT, flags, nullptr, B, T, H, 32, saved, hTs, nullptr, nullptr, dk, log_g};
         return from_cuda(launch_tc_fwd(t, stream));
     }
     ScalarArgs a{q, k, v, log_g, h0, o, hT, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
@@ -441,17 +446,24 @@ hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const
     return from_cuda(launch_scalar_fwd(a, dtype == HGRN2_BF16, stream));
 }
 
-hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
-                              const void *dO, const float *dhT, void *dq, void *dk_out, void *dv_out, void *dlog_g,
-                              float *dh0, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype, void *workspace,
-                              size_t ws_bytes, cudaStream_t stream) {
+size_t scalar_saved_bytes(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    return (use_tc(dk, dv, dtype) && T > 0) ? saved_layout(B, T, H).total : 0;
+}
+
+// Scalar-decay backward.  With `saved` (from scalar_fwd_impl on the same inputs) the reverse sweep
+// reads its chunk states; without it, on the tensor-core route, the forward runs again into the
+// workspace first.
+hgrn2_status scalar_bwd_impl(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                             const void *saved, const void *dO, const float *dhT, void *dq, void *dk_out,
+                             void *dv_out, void *dlog_g, float *dh0, int B, int T, int H, int dk, int dv,
+                             hgrn2_dtype dtype, void *workspace, size_t ws_bytes, cudaStream_t stream) {
     hgrn2_status s = check_scalar(B, T, H, dk, dv, dtype);
     if (s != HGRN2_OK) return s;
     if (T > 0 && (!q || !k || !v || !log_g || !dO || !dq || !dk_out || !dv_out || !dlog_g))
         return HGRN2_ERR_INVALID_ARG;
-    if (!all_aligned({q, k, v, log_g, h0, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, workspace}))
+    if (!all_aligned({q, k, v, log_g, h0, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, workspace, saved}))
         return HGRN2_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < scalar_ws_bytes(B, T, H, dk, dv, dtype)) return HGRN2_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < scalar_ws_bytes(B, T, H, dk, dv, dtype, saved ? 2 : 1)) return HGRN2_ERR_INVALID_ARG;
     if (T == 0) {
         if (!dh0) return HGRN2_OK;
         const size_t n = sizeof(float) * (size_t)B * H * dk * dv;
@@ -462,30 +474,77 @@ hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const
     float *qdq = (float *)((char *)workspace + align256(sizeof(float) * (size_t)B * H));
     const size_t base = align256(sizeof(float) * (size_t)B * H) + align256(sizeof(float) * (size_t)B * T * H);
     if (use_tc(dk, dv, dtype)) {
-        // tensor cores: the forward keeps its chunk states in the workspace (o goes to scratch),
-        // the reverse sweep reads them; pairs whose chunk decay leaves the factorised form's range
-        // are flagged by the forward and recomputed on the exact route
-        char *sv = (char *)workspace + base;
+        // the reverse sweep over the saved chunk states; pairs whose chunk decay leaves the factorised
+        // form's range were flagged by the forward and are recomputed on the exact route
         const SavedLayout sl = saved_layout(B, T, H);
+        char *sv = (char *)saved;
+        if (!sv) {   // no saved states: the forward again, into the workspace (o to scratch)
+            sv = (char *)workspace + base;
+            s = scalar_fwd_impl(q, k, v, log_g, h0, sv + sl.total, nullptr, sv, B, T, H, dk, dv, dtype, stream);
+            if (s != HGRN2_OK) return s;
+        }
         int *flags = (int *)(sv + sl.flags);
         float *hTs = (float *)(sv + sl.hTs);
-        TcFwdArgs f{q, k, v, h0, sv + sl.total, nullptr, flags, nullptr, B, T, H, 32, sv, hTs, nullptr, nullptr, dk,
-                    log_g};
-        cudaError_t e = launch_tc_fwd(f, stream);
-        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         TcBwdArgs r{q, k, v, dO, h0, dhT, dq, dk_out, dv_out, dh0, rs, flags, B, T, H, 32, sv, hTs, nullptr, nullptr,
                     dk, log_g, dlog_g};
-        e = launch_tc_bwd(r, stream);
-        if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+        if (launch_tc_bwd(r, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
         ScalarArgs a{q, k, v, log_g, h0, nullptr, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, rs, qdq, B, T, H,
                      dk, dv, flags};
-        g_launches += 4;
+        g_launches += 3;
         return from_cuda(launch_scalar_bwd(a, dtype == HGRN2_BF16, stream));
     }
     ScalarArgs a{q, k, v, log_g, h0, nullptr, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, rs, qdq, B, T, H, dk,
                  dv, nullptr};
     g_launches += 2;
     return from_cuda(launch_scalar_bwd(a, dtype == HGRN2_BF16, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hgrn2_scalar_workspace_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype, int want_bwd) {
+    if (check_scalar(B, T, H, dk, dv, dtype) != HGRN2_OK || want_bwd < 0 || want_bwd > 2) return (size_t)-1;
+    return scalar_ws_bytes(B, T, H, dk, dv, dtype, want_bwd);
+}
+
+size_t hgrn2_scalar_saved_size(int B, int T, int H, int dk, int dv, hgrn2_dtype dtype) {
+    if (check_scalar(B, T, H, dk, dv, dtype) != HGRN2_OK) return (size_t)-1;
+    return scalar_saved_bytes(B, T, H, dk, dv, dtype);
+}
+
+hgrn2_status hgrn2_scalar_fwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                              void *o, float *hT, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                              cudaStream_t stream) {
+    return scalar_fwd_impl(q, k, v, log_g, h0, o, hT, nullptr, B, T, H, dk, dv, dtype, stream);
+}
+
+hgrn2_status hgrn2_scalar_fwd_train(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                                    void *o, float *hT, void *saved, size_t saved_bytes, int B, int T, int H, int dk,
+                                    int dv, hgrn2_dtype dtype, cudaStream_t stream) {
+    if (check_scalar(B, T, H, dk, dv, dtype) != HGRN2_OK) return check_scalar(B, T, H, dk, dv, dtype);
+    const size_t need = scalar_saved_bytes(B, T, H, dk, dv, dtype);
+    if (need && (!saved || saved_bytes < need)) return HGRN2_ERR_INVALID_ARG;
+    return scalar_fwd_impl(q, k, v, log_g, h0, o, hT, need ? saved : nullptr, B, T, H, dk, dv, dtype, stream);
+}
+
+hgrn2_status hgrn2_scalar_bwd(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                              const void *dO, const float *dhT, void *dq, void *dk_out, void *dv_out, void *dlog_g,
+                              float *dh0, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype, void *workspace,
+                              size_t ws_bytes, cudaStream_t stream) {
+    return scalar_bwd_impl(q, k, v, log_g, h0, nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, B, T, H, dk, dv,
+                           dtype, workspace, ws_bytes, stream);
+}
+
+hgrn2_status hgrn2_scalar_bwd_saved(const void *q, const void *k, const void *v, const void *log_g, const float *h0,
+                                    const void *saved, size_t saved_bytes, const void *dO, const float *dhT, void *dq,
+                                    void *dk_out, void *dv_out, void *dlog_g, float *dh0, int B, int T, int H, int dk,
+                                    int dv, hgrn2_dtype dtype, void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (check_scalar(B, T, H, dk, dv, dtype) != HGRN2_OK) return check_scalar(B, T, H, dk, dv, dtype);
+    const size_t need = scalar_saved_bytes(B, T, H, dk, dv, dtype);
+    if (need && (!saved || saved_bytes < need)) return HGRN2_ERR_INVALID_ARG;
+    return scalar_bwd_impl(q, k, v, log_g, h0, need ? saved : nullptr, dO, dhT, dq, dk_out, dv_out, dlog_g, dh0, B, T,
+                           H, dk, dv, dtype, workspace, ws_bytes, stream);
 }
 
 hgrn2_status hgrn2_get_device_status(cudaStream_t stream) {

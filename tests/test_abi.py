@@ -214,12 +214,26 @@ def test_scalar_decay_argument_checks_before_any_launch(lib):
     vp = ctypes.c_void_p
     bad = ctypes.c_size_t(-1).value
     up = lambda x: (x + 255) // 256 * 256
-    assert lib.hgrn2_scalar_workspace_size(0, 8, 4, 16, 16, L.FP32) == bad
+    ws = lib.hgrn2_scalar_workspace_size
+    assert ws(0, 8, 4, 16, 16, L.FP32, 1) == bad
+    assert ws(2, 8, 3, 16, 16, L.FP32, 3) == bad
+    assert ws(2, 8, 3, 16, 16, L.FP32, 0) == 0                      # the forward needs none
     # exact route: <dhT, hT> per (b,h) and q . dq per token, fp32
-    assert lib.hgrn2_scalar_workspace_size(2, 8, 3, 16, 16, L.FP32) == up(4 * 2 * 3) + up(4 * 2 * 8 * 3)
-    B, T, H = 2, 300, 3   # tensor-core route: + the saved chunk states and an o scratch
-    assert lib.hgrn2_scalar_workspace_size(B, T, H, 128, 128, L.BF16) == (
-        up(4 * B * H) + up(4 * B * T * H) + lib.hgrn2_saved_size(B, T, H, 128, 128, L.BF16) + up(B * T * H * 128 * 2))
+    assert ws(2, 8, 3, 16, 16, L.FP32, 1) == up(4 * 2 * 3) + up(4 * 2 * 8 * 3)
+    B, T, H = 2, 300, 3   # tensor-core route: + the saved chunk states and an o scratch, unless given
+    saved = lib.hgrn2_saved_size(B, T, H, 128, 128, L.BF16)
+    assert lib.hgrn2_scalar_saved_size(B, T, H, 128, 128, L.BF16) == saved
+    assert lib.hgrn2_scalar_saved_size(B, T, H, 32, 32, L.BF16) == 0
+    assert ws(B, T, H, 128, 128, L.BF16, 2) == up(4 * B * H) + up(4 * B * T * H)
+    assert ws(B, T, H, 128, 128, L.BF16, 1) == ws(B, T, H, 128, 128, L.BF16, 2) + saved + up(B * T * H * 128 * 2)
+    # a saved buffer shorter than the saved size: rejected before any launch
+    st = lib.hgrn2_scalar_fwd_train(vp(16), vp(16), vp(16), vp(16), None, vp(16), None, vp(256), saved - 1,
+                                    B, T, H, 128, 128, L.BF16, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_scalar_bwd_saved(vp(16), vp(16), vp(16), vp(16), None, vp(256), saved - 1, vp(16), None,
+                                    vp(16), vp(16), vp(16), vp(16), None, B, T, H, 128, 128, L.BF16, vp(256),
+                                    1 << 30, None)
+    assert st == L.ERR_INVALID_ARG
     f = lib.hgrn2_scalar_fwd
     assert f(vp(16), vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 256, 16, L.FP32, None) == L.ERR_UNSUPPORTED
     assert f(None, vp(16), vp(16), vp(16), None, vp(16), None, 1, 8, 1, 16, 16, L.FP32, None) == L.ERR_INVALID_ARG

@@ -171,3 +171,40 @@ def test_scalar_tensor_core_backward_with_a_flagged_head(cuda, d):
     o, hT = L.scalar_fwd(g["q"], g["k"], g["v"], g["log_g"], g["h0"], want_hT=True)
     got = {"o": o, "hT": hT, "dq": dq, "dk": dk, "dv": dv, "dlog_g": dg, "dh0": dh0}
     _check(inp, got, [(b, h) for b in range(B) for h in range(H)], torch.bfloat16, 2e-2)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_scalar_saved_state_pair(cuda, d):
+    # the training pair: the forward keeps its chunk states, the backward reads them (one reverse
+    # sweep plus the exact route's kernels for flagged pairs: 3 launches), with a flagged head
+    B, T, H = 2, 300, 3
+    inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, 0.9, seed=1500 + d, h0_sigma=0.1, with_dO=True,
+                               dhT_sigma=0.1)
+    inp["log_g"][0, :, 1] = -1.0
+    g = to_cuda(inp)
+    sv = L.new_scalar_saved(g["q"])
+    assert sv is not None
+    L.counters(reset=True)
+    o, hT = L.scalar_fwd(g["q"], g["k"], g["v"], g["log_g"], g["h0"], want_hT=True, saved=sv)
+    c_fwd = L.counters(reset=True)
+    dq, dk, dv, dg, dh0 = L.scalar_bwd(g["q"], g["k"], g["v"], g["log_g"], g["dO"], g["h0"], g["dhT"], want_dh0=True,
+                                       saved=sv)
+    c_bwd = L.counters(reset=True)
+    assert c_fwd[2] == 1 and c_bwd[2] == 3, (c_fwd, c_bwd)
+    assert L.device_status() == L.OK
+    got = {"o": o, "hT": hT, "dq": dq, "dk": dk, "dv": dv, "dlog_g": dg, "dh0": dh0}
+    _check(inp, got, [(b, h) for b in range(B) for h in range(H)], torch.bfloat16, 2e-2)
+
+
+def test_scalar_autograd_function(cuda):
+    B, T, H, d = 1, 260, 2, 128
+    inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, 0.9, seed=1600, h0_sigma=0.1, with_dO=True,
+                               dhT_sigma=0.1)
+    g = to_cuda(inp)
+    leaves = [g[n].clone().requires_grad_(True) for n in ("q", "k", "v", "log_g", "h0")]
+    o, hT = L.scalar_decay(*leaves)
+    loss = (o.float() * g["dO"].float()).sum() + (hT * g["dhT"]).sum()
+    loss.backward()
+    got = {"o": o.detach(), "hT": hT.detach(), "dq": leaves[0].grad, "dk": leaves[1].grad, "dv": leaves[2].grad,
+           "dlog_g": leaves[3].grad, "dh0": leaves[4].grad}
+    _check(inp, got, [(0, 0), (0, 1)], torch.bfloat16, 2e-2)
