@@ -256,8 +256,10 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
  *   q, k : [B,T,H,dk]   v, o : [B,T,H,dv]   log_g : [B,T,H]   (all dtype)
  *   h0, hT : [B,H,dk,dv] float32 (NULL allowed, as for hgrn2_fwd)
  * Forward and backward run on tensor cores for bf16 with dk = dv = 128 or 64 (128-token
- * chunks, bf16 operands, fp32 accumulation and state); everything else runs chunkwise on
- * CUDA cores in fp32 arithmetic, exact for any decay strength.
+ * chunks, bf16 operands, fp32 accumulation and state; a (batch, head) with a chunk whose
+ * summed log decay is below -59.8 is recomputed on CUDA cores, by the forward inside its own
+ * launch); everything else runs chunkwise on CUDA cores in fp32 arithmetic, exact for any
+ * decay strength.
  * 1 <= dk, dv <= 128; any T >= 0; pointers 16-byte aligned.
  * hgrn2_scalar_bwd: gradients dq, dk_out (of k), dv_out (of v), dlog_g (same shapes and dtype
  * as the inputs) and dh0 (NULL: not computed) of L(o, hT) given dO and dhT (NULL: zero).

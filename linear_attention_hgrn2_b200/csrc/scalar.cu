@@ -49,7 +49,7 @@ __device__ __forceinline__ size_t tidx(int b, int t, int h, int T_, int H, int D
 template <typename T>
 __device__ __forceinline__ void load_rows(float *dst, int ld, const T *src, int b, int h, int t0, int n, int T_,
                                           int H, int D) {
-    for (int e = threadIdx.x; e < kC * D; e += kThreads) {
+    for (int e = threadIdx.x; e < kC * D; e += blockDim.x) {
         const int t = e / D, j = e - t * D;
         dst[t * ld + j] = t < n ? to_f<T>(src[tidx(b, t0 + t, h, T_, H, D) + j]) : 0.0f;
     }
@@ -78,7 +78,7 @@ __device__ __forceinline__ void gate_prefix(float *bs, float *es, float *ws, con
 // M[t][s] = s <= t ? (X_t . Y_s) e^{b_t - b_s} : 0, for the chunk's kC x kC pairs.
 __device__ __forceinline__ void decay_scores(float *M, const float *X, const float *Y, int ld, int D,
                                              const float *bs) {
-    for (int e = threadIdx.x; e < kC * kC; e += kThreads) {
+    for (int e = threadIdx.x; e < kC * kC; e += blockDim.x) {
         const int t = e / kC, s = e - t * kC;
         float acc = 0.0f;
         if (s <= t) {
@@ -89,7 +89,7 @@ __device__ __forceinline__ void decay_scores(float *M, const float *X, const flo
     }
 }
 
-size_t fwd_smem(int dk, int dv) {
+constexpr size_t fwd_smem(int dk, int dv) {
     return sizeof(float) * ((size_t)dk * (dv + 1) + 2 * kC * (dk + 1) + kC * (dv + 1) + kC * (kC + 1) + 3 * kC);
 }
 size_t dq_smem(int dk, int dv) {
@@ -100,17 +100,20 @@ size_t rev_smem(int dk, int dv) {
                             5 * kC);
 }
 
+// The forward of one (b, h) by the whole thread block (any multiple of 32 threads), in the shared
+// memory at sm (fwd_smem bytes).  Kept out of line: the tensor-core forward calls it only for the
+// pairs whose chunk decay leaves its factorised form's range.
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
-fwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ lg,
-           const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT, int T_, int H, int dk, int dv) {
-    extern __shared__ float sm[];
-    const int bh = blockIdx.x, b = bh / H, h = bh - b * H, tid = threadIdx.x;
+__device__ __noinline__ void fwd_body(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                                      const T *__restrict__ lg, const float *__restrict__ h0, T *__restrict__ o,
+                                      float *__restrict__ hT, int T_, int H, int dk, int dv, float *sm, int b, int h,
+                                      int bh) {
+    const int tid = threadIdx.x, nt = blockDim.x;
     const int lds = dv + 1, ldk = dk + 1, ldv = dv + 1, lda = kC + 1;
     float *S = sm, *Qs = S + dk * lds, *Ks = Qs + kC * ldk, *Vs = Ks + kC * ldk, *A = Vs + kC * ldv;
     float *bs = A + kC * lda, *es = bs + kC, *ws = es + kC;
     const size_t so = (size_t)bh * dk * dv;
-    for (int e = tid; e < dk * dv; e += kThreads) S[(e / dv) * lds + e % dv] = h0 ? h0[so + e] : 0.0f;
+    for (int e = tid; e < dk * dv; e += nt) S[(e / dv) * lds + e % dv] = h0 ? h0[so + e] : 0.0f;
     for (int t0 = 0; t0 < T_; t0 += kC) {
         const int n = min(kC, T_ - t0);
         __syncthreads();   // the previous chunk is done with every tile
@@ -121,7 +124,7 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
         __syncthreads();
         decay_scores(A, Qs, Ks, ldk, dk, bs);
         __syncthreads();
-        for (int e = tid; e < n * dv; e += kThreads) {   // o_t (reads S_in)
+        for (int e = tid; e < n * dv; e += nt) {   // o_t (reads S_in)
             const int t = e / dv, c = e - t * dv;
             float inter = 0.0f, intra = 0.0f;
             for (int j = 0; j < dk; ++j) inter = fmaf(Qs[t * ldk + j], S[j * lds + c], inter);
@@ -130,7 +133,7 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
         }
         __syncthreads();
         const float eB = es[kC - 1];
-        for (int e = tid; e < dk * dv; e += kThreads) {   // S_out
+        for (int e = tid; e < dk * dv; e += nt) {   // S_out
             const int j = e / dv, c = e - j * dv;
             float acc = 0.0f;
             for (int s = 0; s < n; ++s) acc = fmaf(ws[s] * Ks[s * ldk + j], Vs[s * ldv + c], acc);
@@ -139,7 +142,16 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
     }
     __syncthreads();
     if (hT)
-        for (int e = tid; e < dk * dv; e += kThreads) hT[so + e] = S[(e / dv) * lds + e % dv];
+        for (int e = tid; e < dk * dv; e += nt) hT[so + e] = S[(e / dv) * lds + e % dv];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+fwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ lg,
+           const float *__restrict__ h0, T *__restrict__ o, float *__restrict__ hT, int T_, int H, int dk, int dv) {
+    extern __shared__ float sm[];
+    const int bh = blockIdx.x, b = bh / H, h = bh - b * H;
+    fwd_body<T>(q, k, v, lg, h0, o, hT, T_, H, dk, dv, sm, b, h, bh);
 }
 
 // Forward sweep of the backward: dq of every token, q_t . dq_t in fp32 (for the reverse sweep's

@@ -61,7 +61,6 @@ struct __align__(8) Misc {
     uint64_t sdone, adone, ofree;           // TMEM-warp arrivals (128 each)
     uint32_t tmem_base;
     int bad_tile;                           // first chunk whose decay span is too wide
-    int sflag;                              // scalar decay: a chunk's total log g < kMinLogEB (for the backward)
     int waited_full;                        // q / log f arrivals the prep warps consumed
     int waited_v;                           // v arrivals the MMA thread consumed
     float EB[2][128];                       // E_B ring: read by the TMEM warps while that chunk is current
@@ -92,11 +91,10 @@ struct Params {
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
 // kScalar: the scalar-decay variant S_t = g_t S_{t-1} + k_t v_t^T (one decay per head and token,
-// key k loaded in place of log f).  Its decay factors exactly: A = Q K^T on the raw tiles, the
-// exact e^{b_t - b_s} applied where the TMEM warps mask A, Q rows scaled by e^{b_t} and K rows by
-// e^{B - b_t} after that MMA has read them, and the state scaled by e^{B} before the state MMA
-// adds to it.  Every exponent is <= 0, so the forward is exact for any decay; a pair whose chunk
-// decay leaves the backward's factorisation range is flagged for the backward.
+// key k loaded in place of log f).  The same chunk form with a decay shared by the key dims:
+// b_t = cumulative log g from the chunk start, Qt = q e^{b_t}, Kt = k e^{-b_t} (per-row factors),
+// E_B = e^{B} for every state row.  A chunk with B < kMinLogEB sends the pair to the exact
+// CUDA-core forward (its flag also routes the backward).
 template <bool kPacked, bool kScalar = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
@@ -151,7 +149,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->adone, 128);
         mbar_init(&m->ofree, 128);
         m->bad_tile = INT_MAX;
-        m->sflag = 0;
         m->waited_full = 0;
         m->waited_v = 0;
         fence_mbar_init();
@@ -209,8 +206,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
             for (int n = 0; n < N; ++n) {
                 const int s = n & 1;
-                // scalar decay: A needs only the raw tiles; otherwise the prepped Qt, Kt
-                if (!mbar_wait(kScalar ? &m->fullQG[s] : &m->prepped[s], (n >> 1) & 1)) {
+                if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) {
                     set_status(HGRN2_ERR_TIMEOUT);
                     break;
                 }
@@ -224,10 +220,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                                 sdesc_sw128(smem_u32(Gb[s]) + ko, 16, 1024), id_kk, kk > 0);
                 }
                 mma_commit(&m->barA);
-                if (kScalar) {   // the prep scales Q and K in place once A has read them
-                    if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-                    tc_fence_after();
-                }
                 // O = Qt bf16(S_in) once the S phase wrote it and the last epilogue read O;
                 // S' = S_in + Kt^T V
                 if (!mbar_wait(&m->sdone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -292,8 +284,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ld_volatile(&m->bad_tile) <= n) break;
             e_prev = e_cur;
-            if (kScalar) e_cur = __expf(m->Ppart[n % 3][kTile - 1]);   // e^{B}, B = the chunk's total log g
-            else e_cur = m->EB[s][r];   // the prep warps rewrite this slot only after this chunk's stage is released
+            e_cur = m->EB[s][kScalar ? 0 : r];   // the prep warps rewrite this slot only after this chunk's stage is released
             // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand),
             // once the previous chunk's o store has read X
             if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -302,22 +293,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 named_bar_sync(2, 128);
             }
             tc_fence_after();
-            // scalar decay: S_in is exact already; it is scaled by this chunk's e^{B} for the state MMA
-            const float e = kScalar ? e_cur : e_prev;
+            const float e = e_prev;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
                 tmem_ld32(tl + kColS + 32 * c, v);
                 tmem_wait_ld();
-                if (!kScalar) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] *= e;
-                }
+                for (int i = 0; i < 32; ++i) v[i] *= e;
                 store_chunk_bf16(X, r, c, v);
-                if (kScalar) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] *= e;
-                }
                 tmem_st32(tl + kColS + 32 * c, v);
             }
             tmem_wait_st();
@@ -348,21 +332,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (i > lane) v[i] = 0.0f;
-                    }
-                    if (kScalar) {   // A_rs = (q_r . k_s) e^{b_r - b_s} for s <= r
-                        const float *bv = m->Ppart[n % 3];
-                        const float br = bv[r];
-                        if (c < quad) {
-                            // every column precedes r: e^{b_r - b_e} e^{b_e - b_s} with b_e at the
-                            // block's last column, both factors <= 1; lane l forms column 32c + l's
-                            const float be = bv[32 * c + 31];
-                            const float alpha = __expf(br - be), beta = __expf(be - bv[32 * c + lane]);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] *= alpha * __shfl_sync(0xffffffffu, beta, i);
-                        } else {   // the diagonal block (columns past r were zeroed above)
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) v[i] *= i <= lane ? __expf(br - bv[32 * c + i]) : 0.0f;
-                        }
                     }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) pk[i] = __uint_as_float(pack_bf2(v[2 * i], v[2 * i + 1]));
@@ -427,7 +396,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
         if (n == N && (p.hT || p.hTs) && seg == p.nseg - 1 && r < p.D) {   // warp-uniform
-            const float e = kScalar ? 1.0f : e_cur;   // scalar decay: the state is complete
+            const float e = e_cur;
             float *dst = p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
             float *dsv = p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
 #pragma unroll
@@ -455,54 +424,78 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const int pc = ptid & 63, rr = ptid >> 6, col0 = 2 * pc;
         const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
         auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+        float gnx[4];   // scalar decay: log g of rows 4 lane .. 4 lane + 3 of the next chunk
+        auto load_lg = [&](int n) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = tok0 + n * kTile + 4 * lane + j;
+                gnx[j] = n < N && t < p.T ? __bfloat162float(p.lgs[((size_t)bc * p.T + t) * p.H + h]) : 0.0f;
+            }
+        };
+        if (kScalar) load_lg(0);
         for (int n = 0; n < N; ++n) {
             const int s = n & 1;
             if (!mbar_wait(&m->fullQG[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
             if (ptid == 0) m->waited_full = n + 1;
             if constexpr (kScalar) {
-                // b_t = cumulative log g from the chunk start into a 3-slot ring (the TMEM warps read
-                // slot n % 3 while masking chunk n, which may be after this stage is released: the
-                // prep two chunks ahead writes another slot); 0 past the sequence end
-                float *bv = m->Ppart[n % 3];
-                float *wtot = m->EB[0];   // warp totals of the scan (E_B is not kept for this variant)
-                float a = 0.0f;
-                if (ptid < kTile) {
-                    const int t = tok0 + n * kTile + ptid;
-                    if (t < p.T) a = __bfloat162float(p.lgs[((size_t)bc * p.T + t) * p.H + h]);
+                // b_t = cumulative log g from the chunk start (0 past the sequence end): every prep
+                // warp scans all 128 rows itself (rows 4l .. 4l+3 in lane l), so this prep needs no
+                // block barrier
+                float bl[4];
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, a, o);
-                        if (lane >= o) a += y;
+                for (int j = 0; j < 4; ++j) bl[j] = gnx[j];
+                load_lg(n + 1);
+                bl[1] += bl[0];
+                bl[2] += bl[1];
+                bl[3] += bl[2];
+                float x = bl[3];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                const float ex = x - bl[3];   // sum over the lanes before this one
+                float eq[4], ek[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    bl[j] += ex;
+                    eq[j] = __expf(bl[j]);
+                    ek[j] = __expf(-bl[j]);
+                }
+                const float Bt = __shfl_sync(0xffffffffu, bl[3], 31);
+                const bool bad = !(Bt >= kMinLogEB);   // also NaN
+                // Qt = q e^{b_t}, Kt = k e^{-b_t}, rows in batches of 8: row t = 32 rr + 8 bt + i has its
+                // factors in lane 8 rr + 2 bt + i / 4, slot i % 4
+#pragma unroll 1
+                for (int bt = 0; bt < 4; ++bt) {
+                    const int t0 = 32 * rr + 8 * bt;
+                    uint32_t wq[8], wk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        wq[i] = *reinterpret_cast<const uint32_t *>(Qb[s] + eoff(t0 + i));
+                        wk[i] = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(t0 + i));
                     }
-                    if (lane == 31) wtot[ptid >> 5] = a;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int src = 8 * rr + 2 * bt + (i >> 2);
+                        const float et = __shfl_sync(0xffffffffu, eq[i & 3], src);
+                        const float kt = __shfl_sync(0xffffffffu, ek[i & 3], src);
+                        wq[i] = pack_bf2(bf_lo(wq[i]) * et, bf_hi(wq[i]) * et);
+                        wk[i] = pack_bf2(bf_lo(wk[i]) * kt, bf_hi(wk[i]) * kt);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        *reinterpret_cast<uint32_t *>(Qb[s] + eoff(t0 + i)) = wq[i];
+                        *reinterpret_cast<uint32_t *>(Gb[s] + eoff(t0 + i)) = wk[i];
+                    }
                 }
-                named_bar_sync(1, 256);
-                if (ptid < kTile) {
-                    for (int w = 0; w < (ptid >> 5); ++w) a += wtot[w];
-                    bv[ptid] = a;
-                }
-                named_bar_sync(1, 256);
-                const float Bt = bv[kTile - 1];
-                // the forward is exact for any decay; the backward's factorised form is not past this
-                if (ptid == 0 && !(Bt >= kMinLogEB)) m->sflag = 1;
-                // Q rows times e^{b_t}, K rows times e^{B - b_t} (both <= 1) once the A MMA has read the
-                // raw tiles; lane l forms the factors of row 32 rr + l and the warp shares them
-                const float bl = bv[32 * rr + lane];
-                const float el = __expf(bl), wl = __expf(Bt - bl);
-                if (!mbar_wait(&m->barA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const int t = 32 * rr + i;
-                    const float et = __shfl_sync(0xffffffffu, el, i), wt = __shfl_sync(0xffffffffu, wl, i);
-                    uint32_t *pq = reinterpret_cast<uint32_t *>(Qb[s] + eoff(t));
-                    uint32_t *pk = reinterpret_cast<uint32_t *>(Gb[s] + eoff(t));
-                    const uint32_t wq = *pq, wk = *pk;
-                    *pq = pack_bf2(bf_lo(wq) * et, bf_hi(wq) * et);
-                    *pk = pack_bf2(bf_lo(wk) * wt, bf_hi(wk) * wt);
+                if (ptid == 0) {   // read after prepped[s] completes (this thread arrives after these)
+                    m->EB[s][0] = __expf(Bt);
+                    if (bad) atomicMin(&m->bad_tile, n);
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1, 256);
                 mbar_arrive(&m->prepped[s]);
+                if (bad) break;
                 continue;
             }
             const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
@@ -575,8 +568,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         for (int k = m->waited_v; k < issued_v; ++k) mbar_wait(&m->fullV[k & 1], (k >> 1) & 1, 2000000u);
     }
     if (tid == 0) {
-        if (kScalar) { if (p.flags) p.flags[bh] = m->sflag; }   // for the backward only
-        else if (p.nseg == 1) p.flags[bh] = fell_back ? 1 : 0;   // sole writer
+        if (p.nseg == 1) { if (p.flags) p.flags[bh] = fell_back ? 1 : 0; }   // sole writer
         else if (fell_back) p.flags[bh] = 1;                  // zeroed by the aggregate kernel
         if (fell_back) atomicAdd(&g_counters[0], 1ull);
         else atomicAdd(&g_counters[1], (unsigned long long)N);
@@ -585,11 +577,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
     // exact route for this (b,h) when it runs unsegmented: the pipeline is drained, so the
     // CTA's shared memory is free for the CUDA-core chunkwise forward of the whole sequence
-    if (!kScalar && fell_back && p.nseg == 1) {
+    if (fell_back && p.nseg == 1) {
         __syncthreads();
-        const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
-        simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T, p.H, p.D,
-                                     p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
+        if constexpr (kScalar) {   // the scalar-decay exact forward (key k in p.lf, value v in p.x)
+            sd::fwd_body<__nv_bfloat16>(p.q, p.lf, p.x, p.lgs, p.h0, p.o, p.hT, p.T, p.H, p.D, p.D,
+                                        reinterpret_cast<float *>(smem), b, h, bh);
+        } else {
+            const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
+            simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T,
+                                         p.H, p.D, p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
+        }
     }
 }
 
@@ -795,6 +792,7 @@ scan_kernel(const float *__restrict__ h0, float *__restrict__ U, const float *__
 // ------------------------------------------------------------------ host side
 static_assert(tcf::kSmemBytes <= 227 * 1024, "forward shared memory");
 static_assert(tcf::kAggSmem <= 227 * 1024, "aggregate shared memory");
+static_assert(sd::fwd_smem(128, 128) <= tcf::kSmemBytes, "scalar-decay exact forward inside the forward kernel");
 
 // Segments per (b,h): enough CTAs to cover the 148 SMs of a B200 once, at most one per chunk.
 void tc_fwd_segments(int B, int T, int H, int *nseg, int *tps) {

@@ -124,21 +124,26 @@ def test_scalar_empty_sequence_passes_states_through(cuda):
     assert torch.equal(got["hT"], g["h0"]) and torch.equal(got["dh0"], g["dhT"])
 
 
-@pytest.mark.parametrize("d,lb,strong", [(128, 0.5, False), (64, 0.9, False), (128, 0.5, True)],
-                         ids=["d128", "d64", "d128_strong_decay"])
+@pytest.mark.parametrize("d,lb,strong", [(128, 0.5, None), (64, 0.9, None), (128, 0.5, "all"), (64, 0.9, "one")],
+                         ids=["d128", "d64", "d128_strong_decay", "d64_one_flagged_head"])
 def test_scalar_tensor_core_forward(cuda, d, lb, strong):
     # bf16 with d = 128 or 64 runs the scalar-decay instance of the tensor-core forward: chunk
-    # passes are counted on the device, no pair takes another route; with log g = -12 per token
-    # the decay inside a 128-token chunk reaches e^{-1536}, and every factor it forms is <= 1
+    # passes and exact-route pairs are counted on the device.  A pair with a chunk whose summed
+    # log g is below -59.8 (log g = -12 per token: e^{-1536} over a chunk) is recomputed by the
+    # exact CUDA-core forward inside the same launch; the other pairs stay on the tensor cores.
     B, T, H = 2, 300, 3
+    nt = (T + 127) // 128
     inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, lb, seed=1300 + d, h0_sigma=0.1)
-    if strong:
+    if strong == "all":
         inp["log_g"][:] = -12.0
+    elif strong == "one":
+        inp["log_g"][1, :, 0] = -12.0
     g = to_cuda(inp)
     L.counters(reset=True)
     o, hT = L.scalar_fwd(g["q"], g["k"], g["v"], g["log_g"], g["h0"], want_hT=True)
     c = L.counters(reset=True)
-    assert c[1] == B * H * ((T + 127) // 128) and c[0] == 0 and c[2] == 1, c
+    exact = {None: 0, "all": B * H, "one": 1}[strong]
+    assert c[0] == exact and c[1] == (B * H - exact) * nt and c[2] == 1, c
     assert L.device_status() == L.OK
     assert np.isfinite(np64(o)).all() and np.isfinite(np64(hT)).all()
     for b in range(B):
