@@ -413,13 +413,14 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 // Shared memory (7 tiles of 32 KB): Qb q -> Qt, Gb log f -> Kt, Vb v, Ob dO, D16 bf16(dSh)
 // then the dq tile, AT mask(A)^T then di staging, DA mask(dA) then d log f staging.
 //
-// Two modes.  Recompute mode (kSaved = false) follows the forward-sweep kernel: as soon
-// as the MMAs of a chunk are done, dq of this chunk (written by that kernel) lands in D16
-// and v, dO of the next chunk in Vb, Ob; q and log f of the next chunk follow once the
-// epilogue has read Qt and Kt.  Saved-state mode (kSaved = true) needs no forward sweep:
-// the bf16 state entering each chunk, stored by the training forward, lands in D16 and a
-// third MMA phase forms dq itself, transposed (lane j, tokens along the columns),
-//     dq_pre^T = S_in dO^T + Kt^T mask(dA)^T,      dq = E * dq_pre,
+// Phase 2 issues its two products that read bf16(dSh) first, under a commit of their own, so
+// that D16 takes its next tile while the other two run.  Two modes.  Recompute mode (kSaved =
+// false) follows the forward-sweep kernel: dq of this chunk (written by that kernel) lands in
+// D16, v and dO of the next chunk in Vb, Ob once phase 2 is done; q and log f of the next chunk
+// follow once the epilogue has read Qt and Kt.  Saved-state mode (kSaved = true) needs no
+// forward sweep: the bf16 state entering each chunk, stored by the training forward, lands in
+// D16 and a third MMA phase forms dq itself, transposed (lane j, tokens along the columns),
+//     dq_pre^T = Kt^T mask(dA)^T + S_in dO^T,      dq = E * dq_pre,
 // reusing the masked dA of this chunk; q dq = Qt dq_pre then enters d log f without
 // reading dq back.  A (batch, head) that the forward flagged for the exact route runs
 // both exact sweeps here, on CUDA cores.
@@ -431,6 +432,7 @@ constexpr int kStoreTid = 256;   // issues the output TMA stores (thread 0 issue
 struct __align__(8) Misc {
     uint64_t barIn, barVO, barDQ, barP1, barP2, barP3;   // barDQ: dq (recompute) or S_in (saved)
     uint64_t barDS;                                      // all 512 threads wrote dSh into TMEM
+    uint64_t barD16;                                     // the phase-2 MMAs that read bf16(dSh) completed
     uint32_t tmem_base;
     int pad;
     int issued[3], waited[3];   // loads issued / arrivals waited for: [barIn, barVO, barDQ]
@@ -532,6 +534,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->barP2, 1);
         mbar_init(&m->barP3, 1);
         mbar_init(&m->barDS, kRevThreads);
+        mbar_init(&m->barD16, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -811,35 +814,52 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         fence_proxy_async_smem();
         tc_fence_before();
         if (__syncthreads_or(!ok)) { ok = false; break; }
-        // ---- phase 2
+        // ---- phase 2: the two products that read bf16(dSh) in D16 first, so that D16 can take the
+        // next tile (the saved state, or dq) while the other two run
         if (tid == 0) {
             tc_fence_after();
-            // di = mask(A)^T dO + Kt dSh          (M = s, N = v)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(AT) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
-            }
+            // di = Kt dSh + mask(A)^T dO          (M = s, N = v)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
                 mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(D16) + kk * 2048, kBlk, 1024), id_kmn, true);
+                            sdesc_sw128(smem_u32(D16) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
             }
-            // dk_pre^T = Qt^T mask(dA) + dSh V^T   (M = j, N = s)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(DA) + kk * 2048, kBlk, 1024), id_mnmn, kk > 0);
-            }
+            // dk_pre^T = dSh V^T + Qt^T mask(dA)   (M = j, N = s)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
                 mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, true);
+                            sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, kk > 0);
+            }
+            mma_commit(&m->barD16);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(AT) + ko, 16, 1024),
+                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_kmn, true);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
+                            sdesc_sw128(smem_u32(DA) + kk * 2048, kBlk, 1024), id_mnmn, true);
             }
             mma_commit(&m->barP2);   // also covers the recurrence step issued after the dS phase
+            // D16 once the first two products have read it: the saved bf16 state entering this chunk
+            // (saved mode) or dq of this chunk (recompute mode)
+            if (!mbar_wait(&m->barD16, par)) {
+                ok = false;
+            } else {
+                ++issued[2];
+                mbar_arrive_expect_tx(&m->barDQ, kTileBytes);
+                if (kSaved) {
+                    tma_load_4d(D16, &tm_st, &m->barDQ, 0, 0, 0, slot0 + n * sstride);
+                    tma_load_4d(D16 + kBlk, &tm_st, &m->barDQ, 64, 0, 0, slot0 + n * sstride);
+                } else {
+                    tma_load_4d(D16, &tm_dq, &m->barDQ, 0, h, n * kTile, b);
+                    tma_load_4d(D16 + kBlk, &tm_dq, &m->barDQ, 64, h, n * kTile, b);
+                }
+            }
         }
         // Qt and Kt to registers for the epilogue while the phase-2 MMAs run
         uint32_t qk[32];
@@ -849,20 +869,10 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             qk[i] = (uint32_t)*reinterpret_cast<const uint16_t *>(Qb + off) |
                     ((uint32_t)*reinterpret_cast<const uint16_t *>(Gb + off) << 16);
         }
-        if (__syncthreads_or(!mbar_wait(&m->barP2, par))) { ok = false; break; }
+        if (__syncthreads_or(!mbar_wait(&m->barP2, par) || !ok)) { ok = false; break; }
         tc_fence_after();
-        if (tid == 0) {
-            ++issued[2];
-            mbar_arrive_expect_tx(&m->barDQ, kTileBytes);
-            if (kSaved) {   // the saved bf16 state entering this chunk into D16
-                tma_load_4d(D16, &tm_st, &m->barDQ, 0, 0, 0, slot0 + n * sstride);
-                tma_load_4d(D16 + kBlk, &tm_st, &m->barDQ, 64, 0, 0, slot0 + n * sstride);
-            } else {        // dq of this chunk into D16; v and dO of the next chunk into Vb, Ob
-                tma_load_4d(D16, &tm_dq, &m->barDQ, 0, h, n * kTile, b);
-                tma_load_4d(D16 + kBlk, &tm_dq, &m->barDQ, 64, h, n * kTile, b);
-                if (n > 0) issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
-            }
-        }
+        // recompute mode: v and dO of the next chunk into Vb, Ob
+        if (!kSaved && tid == 0 && n > 0) issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
         // ---- di (lane s) -> AT (rows s) for the TMA store
         {
             float v[32];
@@ -875,27 +885,33 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // q = Qt / E, k dk = Kt dk_pre, f_t dk_t = dk_pre_t / E_{t-1}.  Qt and Kt were copied to
         // registers, so that q and log f of the next chunk can load during the epilogue.
         if (kSaved) {
-            // phase 3 once di has left X1: dq_pre^T = S_in dO^T + Kt^T mask(dA)^T   (M = j, N = t)
+            // phase 3 once di has left X1: dq_pre^T = Kt^T mask(dA)^T + S_in dO^T   (M = j, N = t),
+            // the product that needs no saved state first
             tc_fence_before();
-            if (__syncthreads_or(!mbar_wait(&m->barDQ, par))) { ok = false; break; }
+            __syncthreads();
             if (tid == 0) {
-                waited[2] = it + 1;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
-                                sdesc_sw128(smem_u32(Ob) + ko, 16, 1024), id_kk, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
                     mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + kk * 2048, kBlk, 1024),
-                                sdesc_sw128(smem_u32(DA) + ko, 16, 1024), id_mnk, true);
+                                sdesc_sw128(smem_u32(DA) + ko, 16, 1024), id_mnk, kk > 0);
                 }
-                mma_commit(&m->barP3);
+                if (!mbar_wait(&m->barDQ, par)) {
+                    ok = false;
+                } else {
+                    waited[2] = it + 1;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                        mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
+                                    sdesc_sw128(smem_u32(Ob) + ko, 16, 1024), id_kk, true);
+                    }
+                }
+                mma_commit(&m->barP3);   // also on a timeout: the waits below then end at once
             }
-            if (__syncthreads_or(!mbar_wait(&m->barP3, par))) { ok = false; break; }
+            if (__syncthreads_or(!mbar_wait(&m->barP3, par) || !ok)) { ok = false; break; }
             tc_fence_after();
             if (tid == 0 && n > 0) {   // every operand tile of this chunk has been read
                 issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, n - 1);
