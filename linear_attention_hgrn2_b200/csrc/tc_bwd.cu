@@ -710,6 +710,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tmem_st32(tl + kColE + c0, ev);
             tmem_wait_st();
             if (q4 == 3) m->EB[j] = __expf(bsum);
+            // the previous chunk's output stores have read their staging tiles (D16, AT, DA are
+            // written next, from the dS phase on): waited for by the issuing thread before this barrier
+            if (tid == kStoreTid) tma_store_wait_read0();
             fence_proxy_async_smem();
             tc_fence_before();
             if (__syncthreads_or(q4 == 3 && !(bsum >= kMinLogEB))) {
@@ -750,10 +753,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
             }
         }
-        // the previous chunk's output stores have read their staging tiles (the issuing thread)
-        if (tid == kStoreTid) tma_store_wait_read0();
-        __syncthreads();
-        // ---- dS phase: dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16
+        // ---- dS phase (thread 0 joins once it has issued phase 1): dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16
         {
             float v[32];
             tc_fence_after();
