@@ -172,8 +172,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColDA, sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024),
-                                sdesc_sw128(smem_u32(Vb[s]) + ko, 16, 1024), id_kk, kk > 0);
+                    mma_bf16_ss(tbase + kColDA, sdesc_add(sdesc_sw128(smem_u32(Ob[s]), 16, 1024), ko),
+                                sdesc_add(sdesc_sw128(smem_u32(Vb[s]), 16, 1024), ko), id_kk, kk > 0);
                 }
                 mma_commit(&m->barDA);
                 if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -188,14 +188,14 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(X) + ko, 16, 1024),
-                                sdesc_sw128(smem_u32(Ob[s]) + ko, 16, 1024), id_kk, kk > 0);
+                    mma_bf16_ss(tbase + kColDQ, sdesc_add(sdesc_sw128(smem_u32(X), 16, 1024), ko),
+                                sdesc_add(sdesc_sw128(smem_u32(Ob[s]), 16, 1024), ko), id_kk, kk > 0);
                 }
                 mma_commit(&m->barQ1);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                                sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                    mma_bf16_ss(tbase + kColS, sdesc_add(sdesc_sw128(smem_u32(Gb[s]), kBlk, 1024), kk * 2048),
+                                sdesc_add(sdesc_sw128(smem_u32(Vb[s]), kBlk, 1024), kk * 2048), id_mnmn, true);
                 mma_commit(&m->barS);
                 // dq_pre^T += Kt^T mask(dA)^T (M = j, N = t, K = s)
                 if (!mbar_wait(&m->dadone, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -203,8 +203,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColDQ, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                                sdesc_sw128(smem_u32(X) + ko, 16, 1024), id_mnk, true);
+                    mma_bf16_ss(tbase + kColDQ, sdesc_add(sdesc_sw128(smem_u32(Gb[s]), kBlk, 1024), kk * 2048),
+                                sdesc_add(sdesc_sw128(smem_u32(X), 16, 1024), ko), id_mnk, true);
                 }
                 mma_commit(&m->barQ);
                 mma_commit(&m->empty[s]);
@@ -729,14 +729,14 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Qb) + ko, 16, 1024), id_kk, kk > 0);
+                mma_bf16_ss(tbase + kColX1, sdesc_add(sdesc_sw128(smem_u32(Gb), 16, 1024), ko),
+                            sdesc_add(sdesc_sw128(smem_u32(Qb), 16, 1024), ko), id_kk, kk > 0);
             }
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(Ob) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, kk > 0);
+                mma_bf16_ss(tbase + kColX2, sdesc_add(sdesc_sw128(smem_u32(Ob), 16, 1024), ko),
+                            sdesc_add(sdesc_sw128(smem_u32(Vb), 16, 1024), ko), id_kk, kk > 0);
             }
             mma_commit(&m->barP1);
             // warm L2: this chunk's dq (or saved state), the next chunk's inputs.  Issued here,
@@ -773,8 +773,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + kColDS, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                mma_bf16_ss(tbase + kColDS, sdesc_add(sdesc_sw128(smem_u32(Qb), kBlk, 1024), kk * 2048),
+                            sdesc_add(sdesc_sw128(smem_u32(Ob), kBlk, 1024), kk * 2048), id_mnmn, true);
             }
         }
         // ---- masks: A^T keeps t >= s (lane s), dA keeps s <= t (lane t)
@@ -822,27 +822,27 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(D16) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
+                mma_bf16_ss(tbase + kColX1, sdesc_add(sdesc_sw128(smem_u32(Gb), 16, 1024), ko),
+                            sdesc_add(sdesc_sw128(smem_u32(D16), kBlk, 1024), kk * 2048), id_kmn, kk > 0);
             }
             // dk_pre^T = dSh V^T + Qt^T mask(dA)   (M = j, N = s)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Vb) + ko, 16, 1024), id_kk, kk > 0);
+                mma_bf16_ss(tbase + kColX2, sdesc_add(sdesc_sw128(smem_u32(D16), 16, 1024), ko),
+                            sdesc_add(sdesc_sw128(smem_u32(Vb), 16, 1024), ko), id_kk, kk > 0);
             }
             mma_commit(&m->barD16);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(AT) + ko, 16, 1024),
-                            sdesc_sw128(smem_u32(Ob) + kk * 2048, kBlk, 1024), id_kmn, true);
+                mma_bf16_ss(tbase + kColX1, sdesc_add(sdesc_sw128(smem_u32(AT), 16, 1024), ko),
+                            sdesc_add(sdesc_sw128(smem_u32(Ob), kBlk, 1024), kk * 2048), id_kmn, true);
             }
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16_ss(tbase + kColX2, sdesc_sw128(smem_u32(Qb) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(DA) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                mma_bf16_ss(tbase + kColX2, sdesc_add(sdesc_sw128(smem_u32(Qb), kBlk, 1024), kk * 2048),
+                            sdesc_add(sdesc_sw128(smem_u32(DA), kBlk, 1024), kk * 2048), id_mnmn, true);
             }
             mma_commit(&m->barP2);   // also covers the recurrence step issued after the dS phase
             // D16 once the first two products have read it: the saved bf16 state entering this chunk
@@ -894,8 +894,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(Gb) + kk * 2048, kBlk, 1024),
-                                sdesc_sw128(smem_u32(DA) + ko, 16, 1024), id_mnk, kk > 0);
+                    mma_bf16_ss(tbase + kColX1, sdesc_add(sdesc_sw128(smem_u32(Gb), kBlk, 1024), kk * 2048),
+                                sdesc_add(sdesc_sw128(smem_u32(DA), 16, 1024), ko), id_mnk, kk > 0);
                 }
                 if (!mbar_wait(&m->barDQ, par)) {
                     ok = false;
@@ -905,8 +905,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                        mma_bf16_ss(tbase + kColX1, sdesc_sw128(smem_u32(D16) + ko, 16, 1024),
-                                    sdesc_sw128(smem_u32(Ob) + ko, 16, 1024), id_kk, true);
+                        mma_bf16_ss(tbase + kColX1, sdesc_add(sdesc_sw128(smem_u32(D16), 16, 1024), ko),
+                                    sdesc_add(sdesc_sw128(smem_u32(Ob), 16, 1024), ko), id_kk, true);
                     }
                 }
                 mma_commit(&m->barP3);   // also on a timeout: the waits below then end at once

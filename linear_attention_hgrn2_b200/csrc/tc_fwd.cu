@@ -204,6 +204,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const uint32_t id_kk = idesc_bf16(128, 128, false, false);
             const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
             const uint32_t id_mnmn = idesc_bf16(128, 128, true, true);
+            const uint64_t dXm = sdesc_sw128(smem_u32(X), kBlk, 1024);   // bf16(S_in), MN-major
             for (int n = 0; n < N; ++n) {
                 const int s = n & 1;
                 if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) {
@@ -212,12 +213,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
                 if (ld_volatile(&m->bad_tile) <= n) break;
                 tc_fence_after();
+                // operand descriptors of this stage: K-major (for A, O) and MN-major (for S, O2) views
+                const uint64_t dQ = sdesc_sw128(smem_u32(Qb[s]), 16, 1024), dG = sdesc_sw128(smem_u32(Gb[s]), 16, 1024);
+                const uint64_t dGm = sdesc_sw128(smem_u32(Gb[s]), kBlk, 1024), dVm = sdesc_sw128(smem_u32(Vb[s]), kBlk, 1024);
                 // A = Qt Kt^T
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColA, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
-                                sdesc_sw128(smem_u32(Gb[s]) + ko, 16, 1024), id_kk, kk > 0);
+                    mma_bf16_ss(tbase + kColA, sdesc_add(dQ, ko), sdesc_add(dG, ko), id_kk, kk > 0);
                 }
                 mma_commit(&m->barA);
                 // O = Qt bf16(S_in) once the S phase wrote it and the last epilogue read O;
@@ -228,8 +231,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
-                    mma_bf16_ss(tbase + kColO, sdesc_sw128(smem_u32(Qb[s]) + ko, 16, 1024),
-                                sdesc_sw128(smem_u32(X) + kk * 2048, kBlk, 1024), id_kmn, kk > 0);
+                    mma_bf16_ss(tbase + kColO, sdesc_add(dQ, ko), sdesc_add(dXm, kk * 2048), id_kmn, kk > 0);
                 }
                 mma_commit(&m->barO1);
                 if (!mbar_wait(&m->fullV[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
@@ -237,8 +239,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ss(tbase + kColS, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                                sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                    mma_bf16_ss(tbase + kColS, sdesc_add(dGm, kk * 2048), sdesc_add(dVm, kk * 2048), id_mnmn, true);
                 mma_commit(&m->barS);
                 mma_commit(&m->emptyQG[s]);   // Qt and Kt of stage s are free once the MMAs above completed
                 // O += bf16(mask(A)) V once the TMEM warps wrote it (A operand in TMEM)
@@ -246,8 +247,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tbase + kColO, tbase + kColP + 8 * kk,
-                                sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_kmn, true);
+                    mma_bf16_ts(tbase + kColO, tbase + kColP + 8 * kk, sdesc_add(dVm, kk * 2048), id_kmn, true);
                 mma_commit(&m->barO2);
                 mma_commit(&m->emptyV[s]);   // v of stage s is free once every MMA above completed
             }

@@ -224,6 +224,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     d |= 2ull << 61;
     return d;
 }
+// The descriptor of the same layout `off` bytes further on (off a multiple of 16): the start address
+// field (bits 0-13, address >> 4) takes the offset directly, with no carry out of the field while
+// both addresses lie in the CTA's shared memory (below 2^18 bytes).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t off) {
+    const uint32_t lo = (uint32_t)d + (off >> 4);
+    return ((d >> 32) << 32) | lo;
+}
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   15 A major (0 = K, 1 = MN), 16 B major, 17-22 N >> 3, 24-28 M >> 4.
