@@ -753,7 +753,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
             }
         }
-        // ---- dS phase (thread 0 joins once it has issued phase 1): dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16
+        // ---- dS phase: dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16; thread 0
+        // joins once it has issued phase 1
         {
             float v[32];
             tc_fence_after();

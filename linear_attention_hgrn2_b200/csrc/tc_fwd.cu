@@ -214,8 +214,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 if (ld_volatile(&m->bad_tile) <= n) break;
                 tc_fence_after();
                 // operand descriptors of this stage: K-major (for A, O) and MN-major (for S, O2) views
-                const uint64_t dQ = sdesc_sw128(smem_u32(Qb[s]), 16, 1024), dG = sdesc_sw128(smem_u32(Gb[s]), 16, 1024);
-                const uint64_t dGm = sdesc_sw128(smem_u32(Gb[s]), kBlk, 1024), dVm = sdesc_sw128(smem_u32(Vb[s]), kBlk, 1024);
+                const uint64_t dQ = sdesc_sw128(smem_u32(Qb[s]), 16, 1024);
+                const uint64_t dG = sdesc_sw128(smem_u32(Gb[s]), 16, 1024);
+                const uint64_t dGm = sdesc_sw128(smem_u32(Gb[s]), kBlk, 1024);
+                const uint64_t dVm = sdesc_sw128(smem_u32(Vb[s]), kBlk, 1024);
                 // A = Qt Kt^T
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -736,8 +738,8 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ss(tbase, sdesc_sw128(smem_u32(Gb[s]) + kk * 2048, kBlk, 1024),
-                            sdesc_sw128(smem_u32(Vb[s]) + kk * 2048, kBlk, 1024), id_mnmn, true);
+                mma_bf16_ss(tbase, sdesc_add(sdesc_sw128(smem_u32(Gb[s]), kBlk, 1024), kk * 2048),
+                            sdesc_add(sdesc_sw128(smem_u32(Vb[s]), kBlk, 1024), kk * 2048), id_mnmn, true);
             mma_commit(&m->barM);
         }
         if (__syncthreads_or(!mbar_wait(&m->barM, n & 1))) { ok = false; break; }
