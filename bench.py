@@ -307,7 +307,11 @@ def run_ours(args, world, rank, local):
     if not args.no_varlen:
         out["varlen"] = run_varlen(args, dev, pk, rank)
     if not args.no_d64:
-        out["head_dim_64"] = run_d64(args, dev, pk, rank)
+        from linear_attention_hgrn2_b200 import inputs as I
+        out["head_dim_64"] = run_head_dim(args, dev, pk, rank, I.TRAIN_D64, 9)
+    if not args.no_d256:
+        from linear_attention_hgrn2_b200 import inputs as I
+        out["head_dim_256"] = run_head_dim(args, dev, pk, rank, I.TRAIN_D256, 17)
     if not args.no_fwd_configs:
         out["forward_configs"] = run_fwd_configs(args, dev, pk, rank)
     if not args.no_scalar:
@@ -511,12 +515,12 @@ def run_varlen(args, dev, pk, rank):
     return res
 
 
-def run_d64(args, dev, pk, rank):
-    """The training pair with 64-wide heads at the same hidden size (B=8, H=32, T=2048, d=64)."""
+def run_head_dim(args, dev, pk, rank, w, seed_off):
+    """The training pair at the same hidden size with another head size: 64-wide heads (B=8, H=32,
+    T=2048) or 256-wide heads (B=8, H=8, T=2048, run as 128-wide blocks)."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
-    w = I.TRAIN_D64
-    inp = I.make_workload(w, seed=rank_seed(rank) + 9)
+    inp = I.make_workload(w, seed=rank_seed(rank) + seed_off)
     q, lf, x, dO = (inp[k].to(dev) for k in ("q", "log_f", "i", "dO"))
     sv = L.new_saved(q)
     o = torch.empty_like(x)
@@ -555,6 +559,9 @@ def run_d64(args, dev, pk, rank):
     res = {"workload": w.name, "tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
            "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4), "bwd_achieved_gbs": round(gbs_b, 1),
            "bwd_frac": round(gbs_b / pk["hbm_gbs"], 4), "calls": "hgrn2_fwd_train + hgrn2_bwd_saved", "steps": K}
+    if w.dk > 128 or w.dv > 128:
+        res["route"] = ("128-wide blocks on the tensor cores (column copies in, partial outputs added in fp32); "
+                        "bwd_frac counts the algorithmic bytes of the wide head only")
     del inp, q, lf, x, dO, sv, o
     torch.cuda.empty_cache()
     return res
@@ -734,6 +741,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-d64", action="store_true")
+    ap.add_argument("--no-d256", action="store_true")
     ap.add_argument("--no-fwd-configs", action="store_true")
     ap.add_argument("--no-scalar", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

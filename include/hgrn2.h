@@ -36,10 +36,18 @@
  *    by the CUDA runtime returns HGRN2_ERR_CUDA.
  *  - No exception or abort crosses this ABI.
  *  - Supported sizes: B, H >= 1; T >= 0 (T = 0 writes hT = h0 and nothing else);
- *    1 <= d_k, d_v <= 128; chunk in {16, 32, 64, 128}.  The bf16 tensor-core
- *    path is used when dtype = BF16 and d_k = d_v = 128; every other supported
- *    shape runs the exact CUDA-core path.  Unsupported shapes return
+ *    1 <= d_k, d_v <= 256; chunk in {16, 32, 64, 128}.  The bf16 tensor-core
+ *    path is used when dtype = BF16 and d_k = d_v = 128 or 64; every other
+ *    shape up to 128 runs the exact CUDA-core path.  Unsupported shapes return
  *    HGRN2_ERR_UNSUPPORTED.
+ *  - A head wider than 128 (d_k or d_v in 129..256) runs as blocks: key dims
+ *    0..127 and 128..d_k-1, value dims likewise.  Diag(f) acts on each key dim and
+ *    the update on each value column alone (§3.2, §5), so every block pair (a, c)
+ *    is a head of its own: its state block S[a, c] evolves alone and o[c] is the
+ *    sum over a of the blocks' outputs; the gradients add the same way.  Each
+ *    block takes the route of its own sizes, on contiguous copies of its columns
+ *    in the workspace; partial outputs are added in fp32 and rounded once.
+ *    Packed sequences and the decode step take d_k, d_v <= 128.
  *  - `chunk` is the length of the chunks of the chunkwise algorithm (§3.2);
  *    results do not depend on it beyond rounding.  The CUDA-core path caps it at
  *    what fits in shared memory for the given d_k, d_v.
@@ -123,7 +131,8 @@ hgrn2_status hgrn2_bwd(const void *q, const void *log_f, const void *i, const fl
  * needed) is opaque.  For the bf16 tensor-core route it holds, per (b,h), the
  * bf16-rounded state entering each 128-token chunk (the same operand the forward
  * multiplies with; ceil(T/128) x 128 x 128 x 2 bytes), the float32 final state,
- * and which (b,h) took the exact route.
+ * and which (b,h) took the exact route.  For a head wider than 128 it holds one
+ * such region per block pair whose sizes take the tensor-core route.
  *
  * hgrn2_fwd_train: hgrn2_fwd (same arguments and results) that also fills
  *   `saved` (saved_bytes >= hgrn2_saved_size, else HGRN2_ERR_INVALID_ARG).

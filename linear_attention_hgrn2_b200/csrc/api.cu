@@ -40,7 +40,7 @@ hgrn2_status check_common(int B, int T, int H, int dk, int dv, int chunk, hgrn2_
     if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
     if (dt != HGRN2_FP32 && dt != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
     if (!chunk_ok(chunk)) return HGRN2_ERR_UNSUPPORTED;
-    if (dk > 128 || dv > 128) return HGRN2_ERR_UNSUPPORTED;
+    if (dk > 256 || dv > 256) return HGRN2_ERR_UNSUPPORTED;   // wider than 128: blocks of <= 128
     // index arithmetic is 64-bit; keep grid dimensions and per-tensor element counts sane
     if ((long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
     return HGRN2_OK;
@@ -52,6 +52,48 @@ hgrn2_status check_common(int B, int T, int H, int dk, int dv, int chunk, hgrn2_
 bool use_tc(int dk, int dv, hgrn2_dtype dt) { return dt == HGRN2_BF16 && dk == dv && (dk == 128 || dk == 64); }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Heads wider than 128 run as blocks of the 128-wide path (wide.cu): the key dims in blocks a
+// (w[0][a] dims from off[0][a]) and the value dims in blocks c (w[1][c] from off[1][c]).
+bool is_wide(int dk, int dv) { return dk > 128 || dv > 128; }
+struct WideSplit {
+    int n[2], off[2][2], w[2][2];
+};
+WideSplit wide_split(int dk, int dv) {
+    WideSplit s{};
+    const int d[2] = {dk, dv};
+    for (int x = 0; x < 2; ++x) {
+        s.w[x][0] = d[x] < 128 ? d[x] : 128;
+        s.w[x][1] = d[x] - s.w[x][0];
+        s.off[x][0] = 0;
+        s.off[x][1] = s.w[x][0];
+        s.n[x] = s.w[x][1] > 0 ? 2 : 1;
+    }
+    return s;
+}
+// Scratch of a wide-head call, carved from the workspace (sizes only when base is null).
+struct WideWs {
+    char *q[2], *f[2], *x[2], *dO[2];          // token blocks; null: the caller's tensor serves
+    char *part[2][2], *pq[2][2], *pf[2][2];    // per block pair: o (or di) and dq, d log f partials
+    float *h0[2][2], *hT[2][2], *dhT[2][2], *dh0[2][2];
+    char *sub;                                 // the block calls' own workspace
+    size_t sub_bytes, total;
+};
+WideWs wide_ws(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd, bool tc64, char *base);
+size_t wide_saved(int B, int T, int H, int dk, int dv, hgrn2_dtype dt, size_t off[2][2]);
+// Blocks of equal size (each of d_k, d_v is 256 or at most 128): the nb block pairs of a head run
+// as nb heads of one call of the 128-wide path, block pair (a, c) of head h as head
+// h * nb + a * n[1] + c, so that the whole problem is one launch over H * nb heads.
+bool wide_uniform(int dk, int dv) { return (dk == 256 || dk <= 128) && (dv == 256 || dv <= 128); }
+struct WideStack {
+    char *q, *f, *x, *dO;         // [B*T*H][nb][block width]
+    char *part, *pq, *pf;         // o (or di), dq, d log f of the H * nb heads
+    float *h0, *hT, *dhT, *dh0;   // [B*H*nb][kw][vw]
+    char *sub;
+    size_t sub_bytes, total;
+};
+WideStack wide_stack_ws(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd, bool tc64,
+                        char *base);
 
 // Saved-state buffer of the tensor-core route (written by hgrn2_fwd_train, read by
 // hgrn2_bwd_saved): bf16 state entering every 128-token chunk, fp32 final state, and the
@@ -81,7 +123,9 @@ size_t ws_bytes_base(int B, int H, int dk, int dv, hgrn2_dtype dt, int want_bwd)
 }
 size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd,
                        bool tc64 = true) {
-    (void)chunk;
+    if (is_wide(dk, dv))
+        return wide_uniform(dk, dv) ? wide_stack_ws(B, T, H, dk, dv, chunk, dt, want_bwd, tc64, nullptr).total
+                                    : wide_ws(B, T, H, dk, dv, chunk, dt, want_bwd, tc64, nullptr).total;
     size_t bytes = ws_bytes_base(B, H, dk, dv, dt, want_bwd);
     if (!want_bwd && use_tc(dk, dv, dt) && dk == 128 && T > 0) bytes += align256(tc_fwd_workspace(B, T, H));
     if (want_bwd && tc64 && use_tc(dk, dv, dt) && dk == 64 && T > 0)   // saved states + o scratch
@@ -90,7 +134,101 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
 }
 
 size_t saved_bytes_needed(int B, int T, int H, int dk, int dv, hgrn2_dtype dt) {
+    if (is_wide(dk, dv)) {
+        if (!wide_uniform(dk, dv)) return wide_saved(B, T, H, dk, dv, dt, nullptr);
+        const WideSplit s = wide_split(dk, dv);
+        return saved_bytes_needed(B, T, H * s.n[0] * s.n[1], s.w[0][0], s.w[1][0], dt);
+    }
     return (use_tc(dk, dv, dt) && T > 0) ? saved_layout(B, T, H).total : 0;
+}
+
+WideStack wide_stack_ws(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd, bool tc64,
+                        char *base) {
+    const WideSplit s = wide_split(dk, dv);
+    const int nb = s.n[0] * s.n[1], kw = s.w[0][0], vw = s.w[1][0];
+    const size_t es = dt == HGRN2_BF16 ? 2 : 4, rows = (size_t)B * T * H * nb;
+    const size_t sb = (size_t)B * H * nb * kw * vw * sizeof(float);
+    WideStack w{};
+    size_t p = 0;
+    auto take = [&](size_t n) -> char * {
+        char *r = base ? base + p : nullptr;
+        p += align256(n);
+        return r;
+    };
+    w.q = take(rows * kw * es);
+    w.f = take(rows * kw * es);
+    w.x = take(rows * vw * es);
+    w.part = take(rows * vw * es);
+    w.h0 = (float *)take(sb);
+    if (want_bwd) {
+        w.dO = take(rows * vw * es);
+        w.pq = take(rows * kw * es);
+        w.pf = take(rows * kw * es);
+        w.dhT = (float *)take(sb);
+        w.dh0 = (float *)take(sb);
+    } else {
+        w.hT = (float *)take(sb);
+    }
+    w.sub_bytes = ws_bytes_needed(B, T, H * nb, kw, vw, chunk, dt, want_bwd, tc64);
+    w.sub = take(w.sub_bytes);
+    w.total = p;
+    return w;
+}
+
+// Block (a, c) regions of a wide head's saved buffer, each as saved_bytes_needed for the block.
+size_t wide_saved(int B, int T, int H, int dk, int dv, hgrn2_dtype dt, size_t off[2][2]) {
+    const WideSplit s = wide_split(dk, dv);
+    size_t p = 0;
+    for (int a = 0; a < s.n[0]; ++a)
+        for (int c = 0; c < s.n[1]; ++c) {
+            if (off) off[a][c] = p;
+            p += align256(saved_bytes_needed(B, T, H, s.w[0][a], s.w[1][c], dt));
+        }
+    return p;
+}
+
+WideWs wide_ws(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd, bool tc64, char *base) {
+    const WideSplit s = wide_split(dk, dv);
+    const size_t es = dt == HGRN2_BF16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H;
+    WideWs w{};
+    size_t p = 0;
+    auto take = [&](size_t n) -> char * {
+        char *r = base ? base + p : nullptr;
+        p += align256(n);
+        return r;
+    };
+    if (s.n[0] > 1)
+        for (int a = 0; a < 2; ++a) {
+            w.q[a] = take(rows * s.w[0][a] * es);
+            w.f[a] = take(rows * s.w[0][a] * es);
+        }
+    if (s.n[1] > 1)
+        for (int c = 0; c < 2; ++c) {
+            w.x[c] = take(rows * s.w[1][c] * es);
+            if (want_bwd) w.dO[c] = take(rows * s.w[1][c] * es);
+        }
+    size_t sub = 0;
+    for (int a = 0; a < s.n[0]; ++a)
+        for (int c = 0; c < s.n[1]; ++c) {
+            const int kw = s.w[0][a], vw = s.w[1][c];
+            const size_t sb = BH * kw * vw * sizeof(float);
+            w.part[a][c] = take(rows * vw * es);
+            w.h0[a][c] = (float *)take(sb);
+            if (want_bwd) {
+                w.pq[a][c] = take(rows * kw * es);
+                w.pf[a][c] = take(rows * kw * es);
+                w.dhT[a][c] = (float *)take(sb);
+                w.dh0[a][c] = (float *)take(sb);
+            } else {
+                w.hT[a][c] = (float *)take(sb);
+            }
+            const size_t need = ws_bytes_needed(B, T, H, kw, vw, chunk, dt, want_bwd, tc64);
+            if (need > sub) sub = need;
+        }
+    w.sub_bytes = sub;
+    w.sub = take(sub);
+    w.total = p;
+    return w;
 }
 
 // Workspace of the packed-sequence calls: rowsum(dhT * hT) [nseq*H*dk], flags [nseq*H] and the
@@ -122,6 +260,21 @@ size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk, hgrn
 
 namespace {
 
+hgrn2_status wide_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
+                      void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                      void *workspace, cudaStream_t stream);
+hgrn2_status wide_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                      const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
+                      int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                      cudaStream_t stream, bool tc64);
+hgrn2_status stack_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
+                       void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                       void *workspace, cudaStream_t stream);
+hgrn2_status stack_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                       const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
+                       int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                       cudaStream_t stream, bool tc64);
+
 // Forward; `saved` (null, or saved_bytes_needed bytes) receives what hgrn2_bwd_saved reads.
 hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
                       void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
@@ -132,8 +285,12 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
     const void *ptrs[] = {q, log_f, i, h0, o, hT, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    if (cu && is_wide(dk, dv)) return HGRN2_ERR_UNSUPPORTED;   // packed sequences: d_k, d_v <= 128
     size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 0);
     if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
+    if (is_wide(dk, dv))
+        return (wide_uniform(dk, dv) ? stack_fwd : wide_fwd)(q, log_f, i, h0, o, hT, saved, B, T, H, dk, dv, chunk,
+                                                             dtype, workspace, stream);
     const bool bf16 = dtype == HGRN2_BF16;
     if (T == 0) {
         if (!hT) return HGRN2_OK;
@@ -188,8 +345,13 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     const void *ptrs[] = {q, log_f, i, h0, dO, dhT, dq, dlog_f, di, dh0, workspace, saved};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    if (cu && is_wide(dk, dv)) return HGRN2_ERR_UNSUPPORTED;
     size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1, tc64 && !saved);
     if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
+    if (is_wide(dk, dv))
+        return (wide_uniform(dk, dv) ? stack_bwd : wide_bwd)(q, log_f, i, h0, saved, dO, dhT, dq, dlog_f, di, dh0, B,
+                                                             T, H, dk, dv, chunk, dtype, workspace, stream,
+                                                             tc64 && !saved);
     const bool bf16 = dtype == HGRN2_BF16;
     if (T > 0 && !saved && !cu && tc64 && use_tc(dk, dv, dtype) && dk == 64) {
         // 64-wide heads: the tensor-core forward keeps the chunk states in the workspace (its o
@@ -242,6 +404,219 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     SimtBwdArgs a{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs, B, T, H, dk, dv, C, nullptr, cu, perm};
     g_launches += 2;
     return from_cuda(launch_simt_bwd(a, bf16, stream));
+}
+
+// Columns off .. off+w-1 of every row of a [rows][d] token tensor into contiguous [rows][w].
+cudaError_t copy_cols(void *dst, const void *src, size_t rows, int d, int off, int w, size_t es, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    return cudaMemcpy2DAsync(dst, w * es, (const char *)src + off * es, d * es, w * es, rows, cudaMemcpyDeviceToDevice,
+                             st);
+}
+
+// Columns off .. off+w-1 of every row of a [rows][d] token tensor into rows `dpitch` elements apart.
+cudaError_t copy_cols_to(void *dst, size_t dpitch, const void *src, size_t rows, int d, int off, int w, size_t es,
+                         cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    return cudaMemcpy2DAsync(dst, dpitch * es, (const char *)src + off * es, d * es, w * es, rows,
+                             cudaMemcpyDeviceToDevice, st);
+}
+
+// Equal blocks: the columns of block pair j = a * n[1] + c go to head slot j of the H * nb heads
+// (token rows nb blocks wide, state matrices nb per (b, h)); one forward call runs them all, and
+// o[c] = sum over a of slot a * n[1] + c, added in fp32.
+hgrn2_status stack_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
+                       void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                       void *workspace, cudaStream_t stream) {
+    const WideSplit s = wide_split(dk, dv);
+    const int nK = s.n[0], nV = s.n[1], nb = nK * nV, kw = s.w[0][0], vw = s.w[1][0];
+    const WideStack w = wide_stack_ws(B, T, H, dk, dv, chunk, dtype, 0, true, (char *)workspace);
+    const bool bf16 = dtype == HGRN2_BF16;
+    const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H, sm = (size_t)kw * vw;
+    for (int a = 0; a < nK; ++a)
+        for (int c = 0; c < nV; ++c) {
+            const int j = a * nV + c;
+            if (copy_cols_to(w.q + j * kw * es, (size_t)nb * kw, q, rows, dk, s.off[0][a], kw, es, stream) ||
+                copy_cols_to(w.f + j * kw * es, (size_t)nb * kw, log_f, rows, dk, s.off[0][a], kw, es, stream) ||
+                copy_cols_to(w.x + j * vw * es, (size_t)nb * vw, i, rows, dv, s.off[1][c], vw, es, stream))
+                return HGRN2_ERR_CUDA;
+            if (h0 && launch_state_block(const_cast<float *>(h0), w.h0 + j * sm, nb * sm, BH, dk, dv, s.off[0][a], kw,
+                                         s.off[1][c], vw, false, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+        }
+    const hgrn2_status st = fwd_impl(w.q, w.f, w.x, h0 ? w.h0 : nullptr, w.part, hT ? w.hT : nullptr, saved, B, T,
+                                     H * nb, kw, vw, chunk, dtype, w.sub, w.sub_bytes, stream);
+    if (st != HGRN2_OK) return st;
+    for (int a = 0; a < nK && hT; ++a)
+        for (int c = 0; c < nV; ++c)
+            if (launch_state_block(hT, w.hT + (a * nV + c) * sm, nb * sm, BH, dk, dv, s.off[0][a], kw, s.off[1][c], vw,
+                                   true, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+    for (int c = 0; c < nV; ++c)
+        if (launch_sum_blocks(o, dv, s.off[1][c], w.part + c * vw * es, nK > 1 ? w.part + (nV + c) * vw * es : nullptr,
+                              nb * vw, rows, vw, bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+    g_launches += (h0 ? nb : 0) + (hT ? nb : 0) + (rows ? nV : 0);
+    return HGRN2_OK;
+}
+
+// Backward of equal blocks: one backward call over the H * nb heads; dq[a], d log f[a] = sums of
+// slots a * n[1] + c over c, di[c] = sum of slots a * n[1] + c over a, dh0 blocks as they are.
+hgrn2_status stack_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                       const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
+                       int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                       cudaStream_t stream, bool tc64) {
+    const WideSplit s = wide_split(dk, dv);
+    const int nK = s.n[0], nV = s.n[1], nb = nK * nV, kw = s.w[0][0], vw = s.w[1][0];
+    const WideStack w = wide_stack_ws(B, T, H, dk, dv, chunk, dtype, 1, tc64, (char *)workspace);
+    const bool bf16 = dtype == HGRN2_BF16;
+    const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H, sm = (size_t)kw * vw;
+    for (int a = 0; a < nK; ++a)
+        for (int c = 0; c < nV; ++c) {
+            const int j = a * nV + c;
+            if (copy_cols_to(w.q + j * kw * es, (size_t)nb * kw, q, rows, dk, s.off[0][a], kw, es, stream) ||
+                copy_cols_to(w.f + j * kw * es, (size_t)nb * kw, log_f, rows, dk, s.off[0][a], kw, es, stream) ||
+                copy_cols_to(w.x + j * vw * es, (size_t)nb * vw, i, rows, dv, s.off[1][c], vw, es, stream) ||
+                copy_cols_to(w.dO + j * vw * es, (size_t)nb * vw, dO, rows, dv, s.off[1][c], vw, es, stream))
+                return HGRN2_ERR_CUDA;
+            if (h0 && launch_state_block(const_cast<float *>(h0), w.h0 + j * sm, nb * sm, BH, dk, dv, s.off[0][a], kw,
+                                         s.off[1][c], vw, false, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+            if (dhT && launch_state_block(const_cast<float *>(dhT), w.dhT + j * sm, nb * sm, BH, dk, dv, s.off[0][a],
+                                          kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+        }
+    const hgrn2_status st = bwd_impl(w.q, w.f, w.x, h0 ? w.h0 : nullptr, saved, w.dO, dhT ? w.dhT : nullptr, w.pq,
+                                     w.pf, w.part, dh0 ? w.dh0 : nullptr, B, T, H * nb, kw, vw, chunk, dtype, w.sub,
+                                     w.sub_bytes, stream, nullptr, tc64);
+    if (st != HGRN2_OK) return st;
+    for (int a = 0; a < nK && dh0; ++a)
+        for (int c = 0; c < nV; ++c)
+            if (launch_state_block(dh0, w.dh0 + (a * nV + c) * sm, nb * sm, BH, dk, dv, s.off[0][a], kw, s.off[1][c],
+                                   vw, true, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+    for (int a = 0; a < nK; ++a) {
+        const size_t j0 = (size_t)a * nV;
+        if (launch_sum_blocks(dq, dk, s.off[0][a], w.pq + j0 * kw * es, nV > 1 ? w.pq + (j0 + 1) * kw * es : nullptr,
+                              nb * kw, rows, kw, bf16, stream) != cudaSuccess ||
+            launch_sum_blocks(dlog_f, dk, s.off[0][a], w.pf + j0 * kw * es,
+                              nV > 1 ? w.pf + (j0 + 1) * kw * es : nullptr, nb * kw, rows, kw, bf16, stream) !=
+                cudaSuccess)
+            return HGRN2_ERR_CUDA;
+    }
+    for (int c = 0; c < nV; ++c)
+        if (launch_sum_blocks(di, dv, s.off[1][c], w.part + c * vw * es, nK > 1 ? w.part + (nV + c) * vw * es : nullptr,
+                              nb * vw, rows, vw, bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+    g_launches += (h0 ? nb : 0) + (dhT ? nb : 0) + (dh0 ? nb : 0) + (rows ? 2 * nK + nV : 0);
+    return HGRN2_OK;
+}
+
+// Heads wider than 128: every block pair (a, c) runs the forward of a head of d_k = w[0][a],
+// d_v = w[1][c] on contiguous copies of its columns, with its state block as h0 / hT and its own
+// region of the saved buffer; o[c] = sum over a of the blocks' outputs, added in fp32.
+hgrn2_status wide_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
+                      void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
+                      void *workspace, cudaStream_t stream) {
+    const WideSplit s = wide_split(dk, dv);
+    const WideWs w = wide_ws(B, T, H, dk, dv, chunk, dtype, 0, true, (char *)workspace);
+    size_t soff[2][2];
+    wide_saved(B, T, H, dk, dv, dtype, soff);
+    const bool bf16 = dtype == HGRN2_BF16;
+    const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H;
+    cudaError_t e = cudaSuccess;
+    for (int a = 0; a < 2 && s.n[0] > 1 && e == cudaSuccess; ++a) {
+        e = copy_cols(w.q[a], q, rows, dk, s.off[0][a], s.w[0][a], es, stream);
+        if (e == cudaSuccess) e = copy_cols(w.f[a], log_f, rows, dk, s.off[0][a], s.w[0][a], es, stream);
+    }
+    for (int c = 0; c < 2 && s.n[1] > 1 && e == cudaSuccess; ++c)
+        e = copy_cols(w.x[c], i, rows, dv, s.off[1][c], s.w[1][c], es, stream);
+    if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+    for (int a = 0; a < s.n[0]; ++a)
+        for (int c = 0; c < s.n[1]; ++c) {
+            const int kw = s.w[0][a], vw = s.w[1][c];
+            if (h0 && launch_state_block(const_cast<float *>(h0), w.h0[a][c], (size_t)kw * vw, BH, dk, dv,
+                                         s.off[0][a], kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+            void *sv = saved && saved_bytes_needed(B, T, H, kw, vw, dtype) ? (char *)saved + soff[a][c] : nullptr;
+            const hgrn2_status st = fwd_impl(s.n[0] > 1 ? w.q[a] : q, s.n[0] > 1 ? w.f[a] : log_f,
+                                             s.n[1] > 1 ? w.x[c] : i, h0 ? w.h0[a][c] : nullptr, w.part[a][c],
+                                             hT ? w.hT[a][c] : nullptr, sv, B, T, H, kw, vw, chunk, dtype, w.sub,
+                                             w.sub_bytes, stream);
+            if (st != HGRN2_OK) return st;
+            if (hT && launch_state_block(hT, w.hT[a][c], (size_t)kw * vw, BH, dk, dv, s.off[0][a], kw, s.off[1][c],
+                                         vw, true, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+            g_launches += (h0 ? 1 : 0) + (hT ? 1 : 0);
+        }
+    for (int c = 0; c < s.n[1]; ++c) {
+        if (launch_sum_blocks(o, dv, s.off[1][c], w.part[0][c], s.n[0] > 1 ? w.part[1][c] : nullptr, s.w[1][c], rows,
+                              s.w[1][c], bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+        g_launches += rows ? 1 : 0;
+    }
+    return HGRN2_OK;
+}
+
+// Backward of a wide head: every block pair runs the backward of its own head (from its saved
+// region, if any); dq[a], d log f[a] = sums over c, di[c] = sum over a, dh0 block (a,c) as is.
+hgrn2_status wide_bwd(const void *q, const void *log_f, const void *i, const float *h0, const void *saved,
+                      const void *dO, const float *dhT, void *dq, void *dlog_f, void *di, float *dh0, int B,
+                      int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
+                      cudaStream_t stream, bool tc64) {
+    const WideSplit s = wide_split(dk, dv);
+    const WideWs w = wide_ws(B, T, H, dk, dv, chunk, dtype, 1, tc64, (char *)workspace);
+    size_t soff[2][2];
+    wide_saved(B, T, H, dk, dv, dtype, soff);
+    const bool bf16 = dtype == HGRN2_BF16;
+    const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H;
+    cudaError_t e = cudaSuccess;
+    for (int a = 0; a < 2 && s.n[0] > 1 && e == cudaSuccess; ++a) {
+        e = copy_cols(w.q[a], q, rows, dk, s.off[0][a], s.w[0][a], es, stream);
+        if (e == cudaSuccess) e = copy_cols(w.f[a], log_f, rows, dk, s.off[0][a], s.w[0][a], es, stream);
+    }
+    for (int c = 0; c < 2 && s.n[1] > 1 && e == cudaSuccess; ++c) {
+        e = copy_cols(w.x[c], i, rows, dv, s.off[1][c], s.w[1][c], es, stream);
+        if (e == cudaSuccess) e = copy_cols(w.dO[c], dO, rows, dv, s.off[1][c], s.w[1][c], es, stream);
+    }
+    if (e != cudaSuccess) return HGRN2_ERR_CUDA;
+    for (int a = 0; a < s.n[0]; ++a)
+        for (int c = 0; c < s.n[1]; ++c) {
+            const int kw = s.w[0][a], vw = s.w[1][c];
+            if (h0 && launch_state_block(const_cast<float *>(h0), w.h0[a][c], (size_t)kw * vw, BH, dk, dv,
+                                         s.off[0][a], kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+            if (dhT && launch_state_block(const_cast<float *>(dhT), w.dhT[a][c], (size_t)kw * vw, BH, dk, dv,
+                                          s.off[0][a], kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+            const size_t need = saved_bytes_needed(B, T, H, kw, vw, dtype);
+            const void *sv = saved && need ? (const char *)saved + soff[a][c] : nullptr;
+            const hgrn2_status st = bwd_impl(s.n[0] > 1 ? w.q[a] : q, s.n[0] > 1 ? w.f[a] : log_f,
+                                             s.n[1] > 1 ? w.x[c] : i, h0 ? w.h0[a][c] : nullptr, sv,
+                                             s.n[1] > 1 ? w.dO[c] : dO, dhT ? w.dhT[a][c] : nullptr, w.pq[a][c],
+                                             w.pf[a][c], w.part[a][c], dh0 ? w.dh0[a][c] : nullptr, B, T, H, kw, vw,
+                                             chunk, dtype, w.sub, w.sub_bytes, stream, nullptr, tc64);
+            if (st != HGRN2_OK) return st;
+            if (dh0 && launch_state_block(dh0, w.dh0[a][c], (size_t)kw * vw, BH, dk, dv, s.off[0][a], kw,
+                                          s.off[1][c], vw, true, stream) != cudaSuccess)
+                return HGRN2_ERR_CUDA;
+            g_launches += (h0 ? 1 : 0) + (dhT ? 1 : 0) + (dh0 ? 1 : 0);
+        }
+    for (int a = 0; a < s.n[0]; ++a) {
+        const bool two = s.n[1] > 1;
+        if (launch_sum_blocks(dq, dk, s.off[0][a], w.pq[a][0], two ? w.pq[a][1] : nullptr, s.w[0][a], rows,
+                              s.w[0][a], bf16, stream) != cudaSuccess ||
+            launch_sum_blocks(dlog_f, dk, s.off[0][a], w.pf[a][0], two ? w.pf[a][1] : nullptr, s.w[0][a], rows,
+                              s.w[0][a], bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+        g_launches += rows ? 2 : 0;
+    }
+    for (int c = 0; c < s.n[1]; ++c) {
+        if (launch_sum_blocks(di, dv, s.off[1][c], w.part[0][c], s.n[0] > 1 ? w.part[1][c] : nullptr, s.w[1][c], rows,
+                              s.w[1][c], bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+        g_launches += rows ? 1 : 0;
+    }
+    return HGRN2_OK;
 }
 
 hgrn2_status step_impl(const void *q, const void *lf, const void *i, float *S, void *o, int B, int H, int dk, int dv,
@@ -328,12 +703,12 @@ hgrn2_status hgrn2_bwd_saved(const void *q, const void *log_f, const void *i, co
 }
 
 size_t hgrn2_saved_size_varlen(int nseq, int total_T, int H, int dk, int dv, hgrn2_dtype dtype) {
-    if (check_common(nseq, total_T, H, dk, dv, 64, dtype) != HGRN2_OK) return (size_t)-1;
+    if (check_common(nseq, total_T, H, dk, dv, 64, dtype) != HGRN2_OK || is_wide(dk, dv)) return (size_t)-1;
     return (use_tc(dk, dv, dtype) && total_T > 0) ? saved_layout(nseq, total_T, H, true).total : 0;
 }
 
 size_t hgrn2_workspace_size_varlen(int nseq, int total_T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype) {
-    if (check_common(nseq, total_T, H, dk, dv, chunk, dtype) != HGRN2_OK) return (size_t)-1;
+    if (check_common(nseq, total_T, H, dk, dv, chunk, dtype) != HGRN2_OK || is_wide(dk, dv)) return (size_t)-1;
     return ws_bytes_varlen(nseq, H, dk);
 }
 

@@ -9,5 +9,6 @@
 #include "varlen.cu"
 #include "scalar.cu"
 #include "selftest.cu"
+#include "wide.cu"
 #include "tc_fwd.cu"
 #include "tc_bwd.cu"

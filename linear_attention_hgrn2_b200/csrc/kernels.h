@@ -98,6 +98,13 @@ cudaError_t launch_scalar_bwd(const ScalarArgs &a, bool bf16, cudaStream_t st);
 // Longest-first launch order of packed sequences: perm[r] = the sequence that CTA row r runs,
 // ordered by decreasing number of 128-token chunks (one CTA; any nseq).
 cudaError_t launch_lpt_order(const int *cu, int nseq, int T, int *perm, cudaStream_t st);
+// Heads wider than 128 (wide.cu): state blocks between [nmat][dk][dv] and rw x cw matrices
+// `bstride` floats apart; dst[r][off + c] = p0[r][c] + p1[r][c] (p1 may be null) in fp32, dst rows
+// `pitch` elements apart, p0 / p1 rows `spitch` apart.
+cudaError_t launch_state_block(float *full, float *blk, size_t bstride, size_t nmat, int dk, int dv, int ro, int rw,
+                               int co, int cw, bool to_full, cudaStream_t st);
+cudaError_t launch_sum_blocks(void *dst, int pitch, int off, const void *p0, const void *p1, int spitch, size_t rows,
+                              int w, bool bf16, cudaStream_t st);
 
 size_t simt_fwd_smem(int C, int dk, int dv);
 size_t simt_bwd_dq_smem(int C, int dk, int dv);

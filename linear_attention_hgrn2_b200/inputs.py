@@ -57,8 +57,10 @@ VARLEN = dict(name="varlen_train_bf16_T16384_H16_d128_docmean512", total_T=16384
 
 # the training workload's hidden size (2048) with 64-wide heads
 TRAIN_D64 = Workload("train_fwdbwd_bf16_B8_H32_T2048_d64", 8, 32, 2048, 64, 64, torch.bfloat16, 0.95, 64, bwd=True)
+# ... and with 256-wide heads
+TRAIN_D256 = Workload("train_fwdbwd_bf16_B8_H8_T2048_d256", 8, 8, 2048, 256, 256, torch.bfloat16, 0.95, 64, bwd=True)
 
-WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG, TRAIN_D64)}
+WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG, TRAIN_D64, TRAIN_D256)}
 
 
 def _gen(seed: int) -> np.random.Generator:

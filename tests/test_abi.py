@@ -57,7 +57,8 @@ def test_workspace_size_rejects_bad_arguments(lib):
     f = lib.hgrn2_workspace_size
     assert f(0, 16, 1, 16, 16, 16, 0, 0) == bad          # B < 1
     assert f(1, -1, 1, 16, 16, 16, 0, 0) == bad          # T < 0
-    assert f(1, 16, 1, 256, 16, 16, 0, 0) == bad         # d_k > 128
+    assert f(1, 16, 1, 257, 16, 16, 0, 0) == bad         # d_k > 256
+    assert f(1, 16, 1, 16, 257, 16, 0, 0) == bad         # d_v > 256
     assert f(1, 16, 1, 16, 16, 48, 0, 0) == bad          # chunk not a power of two in [16,128]
     assert f(1, 16, 1, 16, 16, 16, 7, 0) == bad          # unknown dtype
     assert f(1, 16, 1, 16, 16, 16, 0, 0) != bad
@@ -244,3 +245,31 @@ def test_scalar_decay_argument_checks_before_any_launch(lib):
     assert g(*args, 2, 8, 3, 16, 16, L.BF16, None, 0, None) == L.ERR_INVALID_ARG
     assert g(*args, 2, 8, 3, 16, 16, L.BF16, vp(256), 255, None) == L.ERR_INVALID_ARG
     assert g(*args, 2, 300, 3, 128, 128, L.BF16, vp(256), 256, None) == L.ERR_INVALID_ARG   # no room for states
+
+
+def test_wide_heads_sizes(lib):
+    # heads wider than 128 run as blocks of <= 128: the workspace holds the column copies, the
+    # blocks' partial outputs, their state blocks and the block calls' own workspace; the saved
+    # buffer that of one call over all blocks (equal blocks) or one region per block pair
+    bad = ctypes.c_size_t(-1).value
+    B, T, H = 2, 300, 3
+    ws = lib.hgrn2_workspace_size
+    for dk, dv in ((256, 256), (192, 160), (100, 256), (256, 64)):
+        for want in (0, 1, 2):
+            assert ws(B, T, H, dk, dv, 64, L.BF16, want) not in (bad, 0)
+            assert ws(B, T, H, dk, dv, 64, L.FP32, want) not in (bad, 0)
+    one = lib.hgrn2_saved_size(B, T, H, 128, 128, L.BF16)
+    up = lambda x: (x + 255) // 256 * 256
+    # equal blocks run as one call over H * (blocks per head) heads
+    assert lib.hgrn2_saved_size(B, T, H, 256, 256, L.BF16) == lib.hgrn2_saved_size(B, T, 4 * H, 128, 128, L.BF16)
+    assert lib.hgrn2_saved_size(B, T, H, 256, 128, L.BF16) == lib.hgrn2_saved_size(B, T, 2 * H, 128, 128, L.BF16)
+    assert lib.hgrn2_saved_size(B, T, H, 64, 256, L.BF16) == 0   # 64 x 128 blocks: exact route
+    # blocks (0,0) 128 x 128 and (1,1) 64 x 64 take the tensor cores, (0,1) and (1,0) do not
+    assert lib.hgrn2_saved_size(B, T, H, 192, 192, L.BF16) == up(one) + up(lib.hgrn2_saved_size(B, T, H, 64, 64, L.BF16))
+    assert lib.hgrn2_saved_size(B, T, H, 256, 256, L.FP32) == 0
+    # packed sequences and the decode step stay at <= 128
+    assert lib.hgrn2_workspace_size_varlen(2, 300, H, 256, 256, 64, L.BF16) == bad
+    assert lib.hgrn2_saved_size_varlen(2, 300, H, 256, 256, L.BF16) == bad
+    vp = ctypes.c_void_p
+    st = lib.hgrn2_step(vp(256), vp(256), vp(256), vp(4096), vp(256), 1, 1, 256, 256, L.FP32, None)
+    assert st == L.ERR_UNSUPPORTED
