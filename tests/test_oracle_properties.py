@@ -83,3 +83,37 @@ def test_bwd_matches_central_difference_on_a_random_entry(shape, seed, scale, wh
     am[which][idx] -= h
     fd = (loss(ap) - loss(am)) / (2 * h)
     assert grads[which][idx] == pytest.approx(fd, rel=1e-5, abs=1e-6)
+
+
+@settings(max_examples=25, deadline=None)
+@given(B=st.integers(1, 2), T=st.integers(1, 9), H=st.integers(1, 2), dk=st.integers(2, 6), dv=st.integers(2, 6),
+       seed=st.integers(0, 10 ** 6), scale=st.sampled_from([0.05, 0.5, 3.0]), data=st.data())
+def test_blocks_of_key_and_value_dims_recombine_exactly(B, T, H, dk, dv, seed, scale, data):
+    # Diag(f) acts on each key dim and the update on each value column alone (§3.2, §5), so the
+    # state block S[a, c] of key block a and value block c is a recurrence of its own: o[c] sums
+    # the blocks' outputs over a, dq and d log f [a] sum over c, di[c] over a, and hT, dh0 blocks
+    # map one to one.  Heads wider than 128 run on exactly this split.
+    ka = data.draw(st.integers(1, dk - 1))
+    vc = data.draw(st.integers(1, dv - 1))
+    q, lf, x, h0 = _draw(seed, B, T, H, dk, dv, scale)
+    rng = np.random.default_rng(seed + 2)
+    dO = rng.standard_normal((B, T, H, dv))
+    dhT = rng.standard_normal((B, H, dk, dv))
+    o, hT = oracle.fwd(q, lf, x, h0)
+    dq, dlf, di, dh0 = oracle.bwd(q, lf, x, dO, h0, dhT)
+    K = [slice(0, ka), slice(ka, dk)]
+    V = [slice(0, vc), slice(vc, dv)]
+    o2, hT2 = np.zeros_like(o), np.zeros_like(hT)
+    dq2, dlf2, di2, dh02 = np.zeros_like(dq), np.zeros_like(dlf), np.zeros_like(di), np.zeros_like(dh0)
+    for a in K:
+        for c in V:
+            ob, hb = oracle.fwd(q[..., a], lf[..., a], x[..., c], h0[:, :, a, c])
+            o2[..., c] += ob
+            hT2[:, :, a, c] = hb
+            gq, gf, gi, gh = oracle.bwd(q[..., a], lf[..., a], x[..., c], dO[..., c], h0[:, :, a, c], dhT[:, :, a, c])
+            dq2[..., a] += gq
+            dlf2[..., a] += gf
+            di2[..., c] += gi
+            dh02[:, :, a, c] = gh
+    for got, ref in ((o2, o), (hT2, hT), (dq2, dq), (dlf2, dlf), (di2, di), (dh02, dh0)):
+        np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-11)
