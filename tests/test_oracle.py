@@ -60,6 +60,22 @@ def test_hand_worked_example_fwd_and_bwd():
     np.testing.assert_allclose(dh0[0, 0], g["dh0"], atol=1e-14)
 
 
+def test_scalar_decay_hand_worked_example():
+    g = _parse_golden(os.path.join(GOLDEN, "hand_example_scalar_decay_T2_dk2_dv1.txt"))
+    sh = lambda a: a[None, :, None, :]          # [T, D] -> [1, T, 1, D]
+    lg = g["log_g"][:, 0][None, :, None]        # [T, 1] -> [1, T, 1]
+    h0 = g["h0"][None, None]                    # [dk, dv] -> [1, 1, dk, dv]
+    o, hT = oracle.sd_fwd(sh(g["q"]), sh(g["k"]), sh(g["v"]), lg, h0)
+    np.testing.assert_allclose(o[0, :, 0], g["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(hT[0, 0], g["hT"], rtol=0, atol=1e-14)
+    dq, dk, dv, dlg, dh0 = oracle.sd_bwd(sh(g["q"]), sh(g["k"]), sh(g["v"]), lg, sh(g["dO"]), h0)
+    np.testing.assert_allclose(dq[0, :, 0], g["dq"], atol=1e-14)
+    np.testing.assert_allclose(dk[0, :, 0], g["dk"], atol=1e-14)
+    np.testing.assert_allclose(dv[0, :, 0], g["dv"], atol=1e-14)
+    np.testing.assert_allclose(dlg[0, :, 0], g["dlog_g"][:, 0], atol=1e-14)
+    np.testing.assert_allclose(dh0[0, 0], g["dh0"], atol=1e-14)
+
+
 # ---------------------------------------------------------------- forward pins
 @pytest.mark.parametrize("shape", [(1, 7, 1, 3, 2), (2, 9, 3, 4, 5), (1, 70, 2, 2, 3)])
 def test_fwd_matches_quadratic_form(shape):
