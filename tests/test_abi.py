@@ -273,3 +273,28 @@ def test_wide_heads_sizes(lib):
     vp = ctypes.c_void_p
     st = lib.hgrn2_step(vp(256), vp(256), vp(256), vp(4096), vp(256), 1, 1, 256, 256, L.FP32, None)
     assert st == L.ERR_UNSUPPORTED
+
+
+def test_no_fallback_without_the_library_or_a_device():
+    # a fresh process: the library handle is cached per process.  A missing .so raises at load
+    # time, and a call on host tensors raises instead of computing anything on the CPU.
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import linear_attention_hgrn2_b200 as L, torch\n"
+        "try:\n"
+        "    L.load_library('/nonexistent/libhgrn2.so'); print('loaded')\n"
+        "except ImportError:\n"
+        "    print('missing raises')\n"
+        "L._lib = None\n"
+        "q = torch.zeros(1, 4, 1, 8, dtype=torch.bfloat16)\n"
+        "try:\n"
+        "    L.fwd(q, q, q); print('computed on host')\n"
+        "except Exception as e:\n"
+        "    print('host tensors raise', type(e).__name__)\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = out.stdout.strip().splitlines()
+    assert lines[0] == "missing raises"
+    assert lines[1].startswith("host tensors raise"), lines
