@@ -298,3 +298,27 @@ def test_no_fallback_without_the_library_or_a_device():
     lines = out.stdout.strip().splitlines()
     assert lines[0] == "missing raises"
     assert lines[1].startswith("host tensors raise"), lines
+
+
+def test_wide_heads_reject_bad_arguments_before_any_launch(lib):
+    # the wide-head path checks like every other call before it launches anything; on a machine
+    # without a GPU a launch would surface as ERR_CUDA, so ERR_INVALID_ARG shows none was made
+    vp = ctypes.c_void_p
+    B, T, H, dk, dv = 1, 16, 1, 256, 256
+    need = lib.hgrn2_workspace_size(B, T, H, dk, dv, 64, L.BF16, 0)
+    assert need > 0
+    st = lib.hgrn2_fwd(vp(256), vp(256), vp(256), None, vp(256), None, B, T, H, dk, dv, 64, L.BF16, vp(256),
+                       need - 1, None)
+    assert st == L.ERR_INVALID_ARG       # workspace one byte short
+    st = lib.hgrn2_fwd(None, vp(256), vp(256), None, vp(256), None, B, T, H, dk, dv, 64, L.BF16, vp(256), need, None)
+    assert st == L.ERR_INVALID_ARG       # q missing
+    st = lib.hgrn2_fwd(vp(256), vp(256), vp(258), None, vp(256), None, B, T, H, dk, dv, 64, L.BF16, vp(256), need,
+                       None)
+    assert st == L.ERR_INVALID_ARG       # i not 16-byte aligned
+    needb = lib.hgrn2_workspace_size(B, T, H, dk, dv, 64, L.BF16, 1)
+    st = lib.hgrn2_bwd(vp(256), vp(256), vp(256), None, vp(256), None, vp(256), vp(256), vp(256), None,
+                       B, T, H, dk, dv, 64, L.BF16, vp(256), needb - 1, None)
+    assert st == L.ERR_INVALID_ARG
+    st = lib.hgrn2_fwd(vp(256), vp(256), vp(256), None, vp(256), None, B, T, H, 257, dv, 64, L.BF16, vp(256), need,
+                       None)
+    assert st == L.ERR_UNSUPPORTED       # wider than 256
