@@ -322,3 +322,34 @@ def test_wide_heads_reject_bad_arguments_before_any_launch(lib):
     st = lib.hgrn2_fwd(vp(256), vp(256), vp(256), None, vp(256), None, B, T, H, 257, dv, 64, L.BF16, vp(256), need,
                        None)
     assert st == L.ERR_UNSUPPORTED       # wider than 256
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: a C99 program includes the header, links the library and calls it
+    # (host-only calls: sizes, version, an argument error)
+    import shutil
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if gcc is None or not os.path.isdir(cuda_inc):
+        pytest.skip("no C compiler or CUDA headers")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "linear_attention_hgrn2_b200")
+    src = tmp_path / "t.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"hgrn2.h\"\n"
+        "int main(void) {\n"
+        "    size_t ws = hgrn2_workspace_size(8, 2048, 16, 128, 128, 64, HGRN2_BF16, 1);\n"
+        "    hgrn2_status st = hgrn2_fwd(NULL, NULL, NULL, NULL, NULL, NULL, 0, 16, 1, 16, 16, 16, HGRN2_FP32,\n"
+        "                                NULL, 0, NULL);\n"
+        "    printf(\"%s|%zu|%d|%s\\n\", hgrn2_version(), ws, (int)st, hgrn2_status_string(st));\n"
+        "    return 0;\n}\n")
+    exe = tmp_path / "t"
+    cc = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                         "-I", cuda_inc, str(src), "-L", pkg, "-lhgrn2", f"-Wl,-rpath,{pkg}", "-o", str(exe)],
+                        capture_output=True, text=True, timeout=120)
+    assert cc.returncode == 0, cc.stderr[-2000:]
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr[-2000:]
+    version, ws, st, msg = run.stdout.strip().split("|")
+    assert version.startswith("hgrn2-b200") and int(ws) > 0
+    assert int(st) == L.ERR_INVALID_ARG and msg
