@@ -204,7 +204,8 @@ hgrn2_status hgrn2_bwd_varlen(const void *q, const void *log_f, const void *i, c
  * more scratch than that (for d_k = 128 and bf16: B*H > 2032) return
  * HGRN2_ERR_UNSUPPORTED and launch nothing.  The first call on a device looks
  * up the array's device address on that device (make that first call before
- * any stream capture on it).  All calls share the one array and it keeps the
+ * any stream capture on it); the lookup is repeated when the device's current
+ * context has changed since, e.g. after cudaDeviceReset.  All calls share the one array and it keeps the
  * last call's contents; nothing in it needs to start at zero, because each call
  * writes what it reads.  Calls that may overlap on the GPU (on different
  * streams, or from different host threads) race on the array: serialise them.

@@ -7,6 +7,8 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <mutex>
 
 #include "common.cuh"
@@ -965,27 +967,51 @@ const char *hgrn2_version(void) { return "hgrn2-b200 0.1"; }
 // Scratch of hgrn2_bwd_noalloc: a fixed-size array in the library's own device
 // memory, present on every GPU the library is loaded on for the life of the
 // process.  Host code only ever sees a stand-in for this symbol; the device
-// address is looked up per device with cudaGetSymbolAddress and cached.
+// address is looked up with cudaGetSymbolAddress, once per device and context:
+// the cache is keyed on the current driver context, so a context made anew on
+// the same device (after cudaDeviceReset, say), whose copy of the array may sit
+// elsewhere, gets a fresh lookup instead of a stale address.
 namespace {
 constexpr size_t kNoAllocScratchBytes = HGRN2_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+struct NoAllocEntry {
+    CUcontext ctx;
+    void *ptr;
+};
+NoAllocEntry g_noalloc[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once per device).
+// The calling thread's current driver context (null if none is current yet).
+CUcontext current_context() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    }
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Device address of the scratch array in the current device's current context.
 hgrn2_status noalloc_scratch(void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return HGRN2_ERR_CUDA;
     if (dev >= kMaxDevices) return HGRN2_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
+    CUcontext ctx = current_context();
+    if (!ctx || g_noalloc[dev].ctx != ctx || !g_noalloc[dev].ptr) {
+        void *p = nullptr;   // the lookup also makes the device's primary context current if none is
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HGRN2_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        g_noalloc[dev].ctx = current_context();
+        g_noalloc[dev].ptr = p;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = g_noalloc[dev].ptr;
     return HGRN2_OK;
 }
 }  // namespace

@@ -141,6 +141,23 @@ def make_decode(B: int, H: int, dk: int, dv: int, steps: int, dtype: torch.dtype
     return {"q": q, "i": i, "log_f": lf, "S": S, "g": graw}
 
 
+def decode_state(B: int, H: int, dk: int, dv: int, seed: int, S_sigma: float = 1.0) -> torch.Tensor:
+    """Initial decode state S [B,H,dk,dv] float32, N(0, S_sigma^2), for the streamed decode
+    inputs below (its own PCG64 stream, so any number of steps can follow it)."""
+    return torch.from_numpy(_normal(_gen(seed), (B, H, dk, dv), S_sigma))
+
+
+def decode_token(B: int, H: int, dk: int, dv: int, dtype: torch.dtype, lb: float, seed: int, t: int) -> dict:
+    """Inputs of decode step t alone: q, log_f [B,H,dk] and i [B,H,dv] in ``dtype``, drawn from
+    a PCG64 stream keyed by (seed, t) in the order q, i, gate.  A long run of steps can then be
+    generated one token at a time on the host, with no tensor holding every step."""
+    g = np.random.Generator(np.random.PCG64([seed, t]))
+    q = _to(_normal(g, (B, H, dk)), dtype)
+    i = _to(_normal(g, (B, H, dv)), dtype)
+    lf = _to(gate_log_f(_normal(g, (B, H, dk)), lb), dtype)
+    return {"q": q, "i": i, "log_f": lf}
+
+
 def make_varlen(lens, H: int, dk: int, dv: int, dtype: torch.dtype, lb: float, seed: int,
                 h0_sigma: float = 0.0, with_dO: bool = False, dhT_sigma: float = 0.0) -> dict:
     """Packed variable-length sequences: CPU tensors q, log_f [total_T,H,dk], i (and dO)

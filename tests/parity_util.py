@@ -2,11 +2,13 @@
 
 Tolerances (the accuracy bar of the benchmark spec for this method):
   * float32 inputs: max relative error <= 1e-4, measured element-wise as
-        max_i |g_i - r_i| / max(|r_i|, 1e-2 * max_j |r_j|)
+        max_i |g_i - r_i| / max(|r_i|, FP32_FLOOR * max_j |r_j|)
     The floor keeps elements that are ~0 from dividing by ~0: an element-wise
-    ratio is unbounded there for any finite-precision arithmetic (a plain
-    sequential float32 recurrence reaches 1.9e-4 on the tiny workload with a
-    1e-3*rms floor, and 7.7e-6 with this one);
+    ratio is unbounded there for any finite-precision arithmetic.  Elements
+    below FP32_FLOOR of the tensor's largest magnitude are thus held to an
+    absolute error of 1e-4 * FP32_FLOOR * max|r|.  test_fp32_metric.py measures
+    a plain token-by-token float32 recurrence under each candidate floor (1.9e-4
+    with a 1e-3*rms floor, about 7e-5 with 1e-3*max, about 7e-6 with 1e-2*max);
   * bfloat16 inputs with a float32 state: normalised max-abs error <= 2e-2,
         max_i |g_i - r_i| / max_i |r_i|,
     per output tensor.
@@ -20,18 +22,20 @@ import oracle
 
 TOL_FP32 = 1e-4
 TOL_BF16 = 2e-2
+FP32_FLOOR = 1e-2   # relative to max|r|
 
 
 def np64(t):
     return None if t is None else t.detach().to("cpu", torch.float64).numpy()
 
 
-def rel_err(g, r):
+def rel_err(g, r, floor=None):
     g = np.asarray(g, np.float64)
     r = np.asarray(r, np.float64)
     if r.size == 0:
         return 0.0
-    den = np.maximum(np.abs(r), 1e-2 * np.max(np.abs(r)) + 1e-300)
+    fl = FP32_FLOOR if floor is None else floor
+    den = np.maximum(np.abs(r), fl * np.max(np.abs(r)) + 1e-300)
     return float(np.max(np.abs(g - r) / den))
 
 

@@ -353,3 +353,17 @@ def test_header_is_plain_c(tmp_path):
     version, ws, st, msg = run.stdout.strip().split("|")
     assert version.startswith("hgrn2-b200") and int(ws) > 0
     assert int(st) == L.ERR_INVALID_ARG and msg
+
+
+@pytest.mark.parametrize("dt,d,limit", [(L.BF16, 128, 2032), (L.FP32, 128, 2048), (L.BF16, 64, 4032)])
+def test_noalloc_size_limit_boundary(lib, dt, d, limit):
+    # the allocation-free backward needs hgrn2_workspace_size(..., want_bwd = 2) bytes of its fixed
+    # scratch: B*H = limit fits exactly, limit + 1 does not and is refused on the host, before any
+    # launch (so this runs without a GPU; the accepted size is only sized, never called)
+    cap = 1 << 20
+    f = lib.hgrn2_workspace_size
+    assert f(1, 64, limit, d, d, 64, dt, 2) <= cap
+    assert f(1, 64, limit + 1, d, d, 64, dt, 2) > cap
+    vp = ctypes.c_void_p(16)
+    st = lib.hgrn2_bwd_noalloc(vp, vp, vp, None, vp, None, vp, vp, vp, None, 1, 64, limit + 1, d, d, 64, dt, None)
+    assert st == L.ERR_UNSUPPORTED

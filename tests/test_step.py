@@ -45,6 +45,38 @@ def test_decode_workload_full_size_sampled(cuda):
         assert err(np64(S[b:b + 1, h:h + 1]), S_ref[(b, h)], torch.float32) <= 1e-5
 
 
+def test_decode_workload_1000_steps_sampled(cuda):
+    """The decode workload as specified: B=256, H=16, d=128, lb=0.8, S ~ N(0,1), and 1000
+    consecutive in-place steps on one state buffer.  Every token is drawn on the host as it
+    is needed (decode_token), so no tensor holds all 1000 steps.  o is compared at every step
+    and the state after the last step, for sampled (b,h) pairs that include the first and
+    the last, against the oracle run step by step on the same pairs: the fp32 state drift
+    over 1000 read-modify-write steps is inside the measurement."""
+    w = I.DECODE
+    B, H, dk, dv, steps = w["B"], w["H"], w["dk"], w["dv"], w["steps"]
+    seed = 1007
+    S0 = I.decode_state(B, H, dk, dv, seed, w["S_sigma"])
+    S = S0.cuda()
+    pairs = [(0, 0), (17, 3), (128, 9), (255, 15)]
+    bi = torch.tensor([p[0] for p in pairs])
+    hi = torch.tensor([p[1] for p in pairs])
+    S_ref = np64(S0[bi, hi])[:, None]          # [npairs, 1, dk, dv]: one batch row per pair
+    worst = 0.0
+    for t in range(steps):
+        tok = I.decode_token(B, H, dk, dv, w["dtype"], w["lb"], seed, t)
+        o = L.step(tok["q"].cuda(), tok["log_f"].cuda(), tok["i"].cuda(), S)
+        sl = lambda x: np64(x[bi, hi])[:, None]
+        o_ref, S_ref = oracle.step(sl(tok["q"]), sl(tok["log_f"]), sl(tok["i"]), S_ref)
+        e = err(np64(o[bi.cuda(), hi.cuda()])[:, None], o_ref, w["dtype"])
+        worst = max(worst, e)
+        assert e <= tol(w["dtype"]), (t, e)
+    torch.cuda.synchronize()
+    assert torch.isfinite(S).all()
+    e_S = err(np64(S[bi.cuda(), hi.cuda()])[:, None], S_ref, torch.float32)
+    print(f"1000-step decode: worst o error {worst:.3e} (bar {tol(w['dtype'])}), final-state error {e_S:.3e}")
+    assert e_S <= 1e-5
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_steps_equal_fwd(cuda, dtype):
     B, T, H, d = 2, 40, 3, 128

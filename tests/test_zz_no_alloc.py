@@ -6,8 +6,9 @@ must not allocate device memory once running, since cudaMalloc/cudaFree
 synchronise the device).  Its scratch is a fixed array inside the library.
 The test calls it through the C ABI and checks it against hgrn2_bwd on the
 same inputs, twice in a row (the second call sees the first call's leftovers in
-the shared scratch array, with different sizes and options).  The file is named
-so that pytest collects it last.
+the shared scratch array, with different sizes and options), and against the
+fp64 oracle, so that a fault shared by both library backwards cannot pass.  The
+file is named so that pytest collects it last.
 """
 import ctypes
 
@@ -16,7 +17,7 @@ import torch
 
 import linear_attention_hgrn2_b200 as L
 from linear_attention_hgrn2_b200 import inputs as I
-from parity_util import err, np64, tol
+from parity_util import err, np64, oracle_heads, tol
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +63,16 @@ def test_noalloc_matches_workspace_backward(cuda, calls):
             # 64-wide bf16 heads the two calls take different routes (exact / tensor cores)
             e = err(np64(a), np64(r), dtype)
             assert e <= tol(dtype), (n, name, e)
+        # and against the oracle, every (b, h) pair whole
+        pairs = [(b, h) for b in range(B) for h in range(H)]
+        orc = oracle_heads(inp, pairs, want_bwd=True, dhT=inp.get("dhT"))
+        for k, (b, h) in enumerate(pairs):
+            for name, a in zip(("dq", "dlog_f", "di", "dh0"), got):
+                if a is None:
+                    continue
+                sl = a[b, h] if name == "dh0" else a[b, :, h]
+                e = err(np64(sl), orc[name][k], dtype)
+                assert e <= tol(dtype), ("oracle", n, name, b, h, e)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda):
