@@ -228,26 +228,33 @@ def run_ours(args, world, rank, local):
     n_spin = max(1, int(0.05 / max((time.perf_counter() - w0) / 3, 1e-6)))
     stream = torch.cuda.current_stream()
     K = args.steps
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    step_est_ms = 1e3 * (time.perf_counter() - w0) / 3
+    # the K-step timed region is repeated until about 100 ms of steps have been timed (at most
+    # 25 regions); the reported time is the median region, with the spread beside it
+    reps = max(1, min(25, int(np.ceil(100.0 / max(K * step_est_ms, 1e-3)))))
     gate = 2_000_000   # cycles of a device-side sleep that holds the queue while the host fills it
+    region_ms = []
     with ClockSampler(local) as clk:
         time.sleep(0.1)              # nvidia-smi starting up
         for _ in range(n_spin):      # clocks back up after that idle period
             step()
         launches0 = L.counters()[2]  # synchronises
-        barrier(world)
-        torch.cuda.synchronize()
-        # timed region: only the two bracketing events, so nothing but the calls runs between
-        # them; the sleep ahead of t0 lets the host queue the K steps before the GPU reaches them
-        torch.cuda._sleep(gate)
-        t0.record(stream)
-        for _ in range(K):
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        launches = L.counters()[2] - launches0
+        for _ in range(reps):
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            torch.cuda.synchronize()
+            # timed region: only the two bracketing events, so nothing but the calls runs between
+            # them; the sleep ahead of t0 lets the host queue the K steps before the GPU reaches them
+            torch.cuda._sleep(gate)
+            t0.record(stream)
+            for _ in range(K):
+                step()
+            t1.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            region_ms.append(t0.elapsed_time(t1))
+        launches = (L.counters()[2] - launches0) // reps
         # per-call durations, same data and clocks: K forward calls, then K backward calls
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         torch.cuda._sleep(gate)
@@ -259,7 +266,7 @@ def run_ours(args, world, rank, local):
             bwd_call()
         ev[2].record(stream)
         torch.cuda.synchronize()
-    ms_local = t0.elapsed_time(t1)
+    ms_local = statistics.median(region_ms)
     ms = max_over_ranks(ms_local, world)
     fwd_ms = ev[0].elapsed_time(ev[1]) / K
     bwd_ms = ev[1].elapsed_time(ev[2]) / K
@@ -289,16 +296,28 @@ def run_ours(args, world, rank, local):
                  "bf16_peak_frac": round(tensor_frac, 4),
                  "bf16_peak_tflops": pk["bf16_tflops_sustained"]}
 
+    clocks = clk.summary()
+    timed = {"regions": reps, "steps_per_region": K,
+             "ms_per_step_median": round(ms_local / K, 5),
+             "ms_per_step_min": round(min(region_ms) / K, 5), "ms_per_step_max": round(max(region_ms) / K, 5),
+             "spread": round((max(region_ms) - min(region_ms)) / ms_local, 4),
+             "timed_ms_total": round(sum(region_ms), 2)}
+    if clocks.get("sm_mhz"):
+        # time x median SM clock: comparable across runs at different clocks
+        timed["ms_x_sm_ghz_per_step"] = round(ms_local / K * clocks["sm_mhz"] / 1e3, 5)
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K,
            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
            "config": {"workload": w.name, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv, "chunk": chunk,
+                      "tensor_core_chunk": 128,
+                      "chunk_note": "chunk is the call's argument (the exact route's chunk); the tensor-core "
+                                    "kernels that run this workload tile by 128 tokens",
                       "lb": w.lb, "global_batch": B * world, "seq_len": T,
                       "parallelism": f"dp{world} (independent replicas, no collective)",
                       "calls": "hgrn2_fwd_train + hgrn2_bwd_saved",
                       "l2": "no flush: 268 MB of token inputs per step > 126 MB L2"},
            "roofline": roofline, "step_roofline": step_roof, "gpu_launches": launches,
-           "clocks": clk.summary()}
+           "timed_regions": timed, "clocks": clocks}
 
     if not args.no_e2e:
         out["e2e"] = run_e2e(args, q, lf, x, dO, o, ws_f, ws_b, sv, w, world)
@@ -306,6 +325,9 @@ def run_ours(args, world, rank, local):
         out["decode_step"] = run_decode(args, dev, pk)
     if not args.no_varlen:
         out["varlen"] = run_varlen(args, dev, pk, rank)
+    if not args.no_lb0:
+        from linear_attention_hgrn2_b200 import inputs as I
+        out["lower_bound_zero"] = run_head_dim(args, dev, pk, rank, I.TRAIN_LB0, 19, ref_ms=ms_per_step)
     if not args.no_d64:
         from linear_attention_hgrn2_b200 import inputs as I
         out["head_dim_64"] = run_head_dim(args, dev, pk, rank, I.TRAIN_D64, 9)
@@ -318,6 +340,7 @@ def run_ours(args, world, rank, local):
         out["scalar_decay"] = run_scalar(args, dev, pk, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_seconds)
+        out["cpu_baseline_other_workloads"] = cpu_baseline_others(budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out), flush=True)
 
@@ -515,9 +538,11 @@ def run_varlen(args, dev, pk, rank):
     return res
 
 
-def run_head_dim(args, dev, pk, rank, w, seed_off):
-    """The training pair at the same hidden size with another head size: 64-wide heads (B=8, H=32,
-    T=2048) or 256-wide heads (B=8, H=8, T=2048, run as 128-wide blocks)."""
+def run_head_dim(args, dev, pk, rank, w, seed_off, ref_ms=None):
+    """The training pair on a variant of the training workload: 64-wide heads (B=8, H=32, T=2048),
+    256-wide heads (B=8, H=8, T=2048, run as 128-wide blocks), or the first layer's forget-gate
+    lower bound lb = 0 (the same shapes; with ref_ms, the headline step's time, for the ratio).
+    Exact-route passes over the timed steps are counted on the device."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
     inp = I.make_workload(w, seed=rank_seed(rank) + seed_off)
@@ -537,6 +562,7 @@ def run_head_dim(args, dev, pk, rank, w, seed_off):
     torch.cuda.synchronize()
     K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    L.counters(reset=True)
     torch.cuda._sleep(2_000_000)
     ev[0].record()
     for _ in range(K):
@@ -550,6 +576,7 @@ def run_head_dim(args, dev, pk, rank, w, seed_off):
         bwd_call()
     ev[3].record()
     torch.cuda.synchronize()
+    cnt = L.counters(reset=True)
     ms = ev[0].elapsed_time(ev[1]) / K
     fwd_ms = ev[1].elapsed_time(ev[2]) / K
     bwd_ms = ev[2].elapsed_time(ev[3]) / K
@@ -558,7 +585,10 @@ def run_head_dim(args, dev, pk, rank, w, seed_off):
     gbs_b = bwd_bytes / (bwd_ms / 1e3) / 1e9
     res = {"workload": w.name, "tokens_per_s": round(w.B * w.T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
            "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4), "bwd_achieved_gbs": round(gbs_b, 1),
-           "bwd_frac": round(gbs_b / pk["hbm_gbs"], 4), "calls": "hgrn2_fwd_train + hgrn2_bwd_saved", "steps": K}
+           "bwd_frac": round(gbs_b / pk["hbm_gbs"], 4), "calls": "hgrn2_fwd_train + hgrn2_bwd_saved", "steps": K,
+           "lb": w.lb, "exact_route_passes": int(cnt[0]), "tensor_core_chunk_passes": int(cnt[1])}
+    if ref_ms:
+        res["step_time_vs_headline"] = round(ms / ref_ms, 4)
     if w.dk > 128 or w.dv > 128:
         res["route"] = ("128-wide blocks on the tensor cores (column copies in, partial outputs added in fp32); "
                         "bwd_frac counts the algorithmic bytes of the wide head only")
@@ -690,6 +720,54 @@ def cpu_baseline(inp, w, budget_s=15.0):
             "seconds": round(dt, 3)}
 
 
+def cpu_baseline_others(budget_s=15.0):
+    """The oracle (unchanged) on the host cores for the other workloads, each on a bounded sample:
+    the forward layer (fwd, B=4, H=8, T=2048) and the long sequence (fwd, B=1, H=8, T=32768,
+    h0 in, hT out), whole (batch, head) sequences; the decode workload (B=256, H=16), its first
+    decode steps.  Each leg is sized from a first short run to about budget_s / 3 seconds."""
+    import oracle
+    from linear_attention_hgrn2_b200 import inputs as I
+    cores = oracle.num_threads()
+    f64 = lambda t: t.to(torch.float64).numpy()
+    out = {}
+    for w in (I.FWD_LAYER, I.LONG):
+        inp = I.make_workload(w, seed=1011)
+        def run(nb, nh):
+            sl = lambda t: f64(t[:nb, :, :nh].contiguous())
+            h0 = f64(inp["h0"][:nb, :nh].contiguous()) if "h0" in inp else None
+            t0 = time.perf_counter()
+            oracle.fwd(sl(inp["q"]), sl(inp["log_f"]), sl(inp["i"]), h0)
+            return time.perf_counter() - t0
+        nh = min(w.H, cores)
+        dt1 = run(1, nh)
+        nb = max(1, min(w.B, int(budget_s / 3 / max(dt1, 1e-3))))
+        dt = run(nb, nh) if nb > 1 else dt1
+        seqs = nb * nh
+        out[w.name] = {"value": round(seqs * w.T / w.H / dt, 2), "unit": "tokens/s", "cores": cores,
+                       "kind": "oracle", "seconds": round(dt, 3),
+                       "sample": f"fwd of {seqs} whole (batch,head) sequences of {w.B * w.H} (T={w.T}); "
+                                 f"tokens/s counts a token as all H heads"}
+    cfg = I.DECODE
+    S0 = f64(I.decode_state(cfg["B"], cfg["H"], cfg["dk"], cfg["dv"], 1005, cfg["S_sigma"]))
+    def steps(n):   # only the oracle's own calls are timed, not the drawing of the tokens
+        S, dt = S0, 0.0
+        for t in range(n):
+            tok = I.decode_token(cfg["B"], cfg["H"], cfg["dk"], cfg["dv"], cfg["dtype"], cfg["lb"], 1005, t)
+            a = [f64(tok[k]) for k in ("q", "log_f", "i")]
+            t0 = time.perf_counter()
+            _, S = oracle.step(*a, S)
+            dt += time.perf_counter() - t0
+        return dt
+    dt1 = steps(2) / 2
+    n = max(2, min(cfg["steps"], int(budget_s / 3 / max(dt1, 1e-3))))
+    dt = steps(n)
+    out[cfg["name"]] = {"value": round(cfg["B"] * n / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                        "ms_per_step": round(dt / n * 1e3, 2), "seconds": round(dt, 3),
+                        "sample": f"the first {n} of {cfg['steps']} decode steps, all {cfg['B']}x{cfg['H']} "
+                                  f"(batch,head) states (the oracle's calls only)"}
+    return out
+
+
 # ------------------------------------------------------------------------------------ reference arm
 def run_reference(args, world, rank):
     """The oracle as the reference arm: same metric and config, bounded samples per step, host cores."""
@@ -741,6 +819,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-d64", action="store_true")
+    ap.add_argument("--no-lb0", action="store_true")
     ap.add_argument("--no-d256", action="store_true")
     ap.add_argument("--no-fwd-configs", action="store_true")
     ap.add_argument("--no-scalar", action="store_true")

@@ -1,22 +1,26 @@
 // tc_bwd.cu -- chunkwise HGRN2 backward on 5th-generation tensor cores (sm_100a).
 //
 // Two sweeps per (batch, head), d_k = d_v = 128, bf16 token tensors, 128-token
-// chunks, same factorisation as the forward: E_t = prod_{r<=t} f_r inside a
-// chunk, Qt = q E, Kt = k / E, E_B = E at the chunk end.
+// chunks, same factorisation as the forward: with b the cumulative log decay from
+// the chunk start, B its chunk total and the balanced reference rho = B / 2 (per key
+// dim), E_t = e^{b_t - rho}, Qt = q E, Kt = k / E, and H = e^{B - rho} = e^{rho} the
+// scale of the state on either side of the chunk's MMAs (S_r = H S_in before them,
+// S_out = H S' after them).
 //
 // Forward sweep (dq_kernel): the fp32 state is recomputed in TMEM and
-//   dq = E * (dO S_in^T + mask(dO V^T) Kt)                                 (1)
+//   dq = E * (dO S_r^T + mask(dO V^T) Kt)                                  (1)
 // is formed transposed (TMEM lane = key dim j, column = token t), so the
 // decay factor E[j][t] that finishes it sits in the same thread's lane.  The
-// state is post-scaled: the MMA accumulates S_in + Kt^T V, and the next chunk
-// multiplies its rows by E_B before using it.  At the end it writes
-// rowsum(dhT * hT) for the reverse sweep's carry.
+// MMA accumulates S' = S_r + Kt^T V, and the next chunk multiplies its rows by
+// both state scales before using it.  At the end it writes rowsum(dhT * hT) for
+// the reverse sweep's carry.
 //
 // Reverse sweep (rev_kernel), chunks last to first, dS = dL/dS_out in TMEM:
-//   dSh  = Diag(E_B) dS                                   (also the new dS)
+//   dSh  = Diag(H) dS                                     (also the new dS)
 //   di   = mask(A)^T dO + Kt dSh                            A = Qt Kt^T
 //   dk^T = (Qt^T mask(dO V^T) + dSh V^T) / E               (lane j, column s)
-//   dS   = dSh + Qt^T dO
+//   dS   = Diag(H) (dSh + Qt^T dO)                          (dL/dS_in; the scale is
+//                                                            applied with the next dSh)
 //   dlog f_t = sum_{t'>=t} (q dq - k dk)_{t'} + rowsum(dhT hT) - f_t dk_t
 // The last line is the gradient through both the decay and the tied input gate
 // k = 1 - f ("HGRN2: Gated Linear RNNs with State Expansion", §2.1 tied gate,
@@ -69,6 +73,7 @@ struct __align__(8) Misc {
     int pad;
     float EB[2][128];
     float Bpart[128];                        // sum of log f over rows 0..63, per key dim
+    float Bpart2[128];                       // ... and over rows 64..127
     float rs_part[128];
 };
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
@@ -236,19 +241,25 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
             tmem_wait_st();
         }
         int n = 0;
-        float e_prev = 1.0f, e_cur = 1.0f;
+        // a wait given up by a lane of this warp (warp-uniform: TMEM loads and stores are
+        // warp-collective); the group leaves together at its next barrier
+        bool fail = false;
+        auto wait_all = [&](uint64_t *bar, uint32_t par) {
+            fail = __any_sync(0xffffffffu, fail || !mbar_wait(bar, par));
+        };
+        float e_prev = 1.0f, e_cur = 1.0f;   // e^{B/2} of the previous and the current chunk
         for (; n < N; ++n) {
             const int s = n & 1;
-            if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (ld_volatile(&m->bad_tile) <= n) break;
+            wait_all(&m->prepped[s], (n >> 1) & 1);
+            if (n >= 1) {
+                wait_all(&m->barS, (n - 1) & 1);
+                if (r == 0) tma_store_wait_read0();   // the previous dq store has read X
+            }
+            if (named_bar_or(2, 128, fail || ld_volatile(&m->bad_tile) <= n)) break;
             e_prev = e_cur;
             e_cur = m->EB[s][r];
-            // S phase
-            if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (n >= 1) {
-                if (r == 0) tma_store_wait_read0();   // the previous dq store has read X
-                named_bar_sync(2, 128);
-            }
+            // S phase: S_r = Diag(e^{B/2}) Diag(e^{B_prev/2}) S' of the previous chunk, one factor after
+            // the other (their product can fall below the fp32 range; the first gives S_out, O(1))
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -256,7 +267,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
                 tmem_ld32(tl + kColS + 32 * c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= e_prev;
+                for (int i = 0; i < 32; ++i) v[i] = (v[i] * e_prev) * e_cur;
                 store_chunk_bf16(X, r, c, v);
                 tmem_st32(tl + kColS + 32 * c, v);
             }
@@ -264,9 +275,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->sdone);
-            // causal mask of dA (lane = t), bf16 -> X (rows t) once S_in dO^T has read X
-            if (!mbar_wait(&m->barDA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (!mbar_wait(&m->barQ1, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            // causal mask of dA (lane = t), bf16 -> X (rows t) once S_r dO^T has read X.  (After a
+            // wait given up, this thread goes on with whatever TMEM holds; nothing it writes is used.)
+            wait_all(&m->barDA, n & 1);
+            wait_all(&m->barQ1, n & 1);
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -282,7 +294,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
             tc_fence_before();
             mbar_arrive(&m->dadone);
             // dq[t][j] = E[j][t] * dq_pre^T[j][t]  (lane j = r) -> X as the [t][j] tile
-            if (!mbar_wait(&m->barQ, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            wait_all(&m->barQ, n & 1);
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -301,18 +313,19 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
             tc_fence_before();
             mbar_arrive(&m->dqfree);
             mbar_arrive(&m->efree);
-            named_bar_sync(2, 128);
+            if (named_bar_or(2, 128, fail)) break;
             if (r == 0) {
                 tma_store_4d(&tm_dq, X, 0, h, n * kTile, b);
                 tma_store_4d(&tm_dq, X + kBlk, 64, h, n * kTile, b);
                 tma_store_commit();
             }
         }
+        if (fail) set_status(HGRN2_ERR_TIMEOUT);
         if (r == 0) tma_store_wait_all0();
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        if (n == N && p.dhT && p.rs) {
-            // hT = Diag(E_B of the last chunk) S';  rs[j] = sum_v dhT[j,v] hT[j,v]
+        if (n == N && !fail && p.dhT && p.rs) {
+            // hT = Diag(e^{B/2} of the last chunk) S';  rs[j] = sum_v dhT[j,v] hT[j,v]
             const float *g = p.dhT + ((size_t)bh * 128 + r) * 128;
             float acc = 0.0f;
 #pragma unroll
@@ -334,17 +347,23 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
         auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
         for (int n = 0; n < N; ++n) {
             const int s = n & 1;
-            if (!mbar_wait(&m->full[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (warp == 8 && lane == 0) m->waited_full = n + 1;
-            if (half == 1) {
+            const bool landed = mbar_wait(&m->full[s], (n >> 1) & 1);
+            if (warp == 8 && lane == 0 && landed) m->waited_full = n + 1;
+            {   // half 1 sums rows 0..63 (its prefix), half 0 rows 64..127: with both, the chunk total
                 float sum = 0.0f;
 #pragma unroll 16
                 for (int t = 0; t < 64; ++t)
-                    sum += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t)));
-                m->Bpart[j] = sum;
+                    sum += __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Gb[s] + eoff(t + 64 * (1 - half))));
+                (half ? m->Bpart : m->Bpart2)[j] = sum;
             }
-            named_bar_sync(1, 256);   // rows 0..63 of log f are read before the first half overwrites them
-            float bsum = half ? m->Bpart[j] : 0.0f;
+            // every row of log f is read before either half overwrites it; the group leaves
+            // together if a wait gave up
+            if (named_bar_or(1, 256, !landed)) {
+                if (!landed) set_status(HGRN2_ERR_TIMEOUT);
+                break;
+            }
+            const float rho = 0.5f * (m->Bpart[j] + m->Bpart2[j]);   // the balanced reference
+            float bsum = (half ? m->Bpart[j] : 0.0f) - rho;           // b - rho before this half
             float ev[64];
 #pragma unroll
             for (int bt = 0; bt < 8; ++bt) {
@@ -364,18 +383,23 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
 #pragma unroll
                 for (int i = 0; i < 8; ++i) *reinterpret_cast<__nv_bfloat16 *>(Gb[s] + eoff(t0 + i)) = ok[i];
             }
-            if (half == 1) {
+            if (half == 1) {   // bsum = B - rho = B / 2
                 m->EB[s][j] = __expf(bsum);
-                if (!(bsum >= kMinLogEB)) atomicMin(&m->bad_tile, n);
+                if (!(bsum >= -kMaxRefLog)) atomicMin(&m->bad_tile, n);   // also NaN
             }
             fence_proxy_async_smem();
             // E -> TMEM lane j once the previous chunk's dq epilogue has read it
-            if (n >= 1 && !mbar_wait(&m->efree, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(ev));
-            tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(ev + 32));
-            tmem_wait_st();
+            const bool efree = __all_sync(0xffffffffu, n < 1 || mbar_wait(&m->efree, (n - 1) & 1));
+            if (efree) {
+                tmem_st32(tl + kColE + 64 * half, *reinterpret_cast<float(*)[32]>(ev));
+                tmem_st32(tl + kColE + 64 * half + 32, *reinterpret_cast<float(*)[32]>(ev + 32));
+                tmem_wait_st();
+            }
             tc_fence_before();
-            named_bar_sync(1, 256);   // bad_tile settled, Bpart free
+            if (named_bar_or(1, 256, !efree)) {   // bad_tile settled, Bpart free
+                if (!efree) set_status(HGRN2_ERR_TIMEOUT);
+                break;
+            }
             mbar_arrive(&m->prepped[s]);
             if (ld_volatile(&m->bad_tile) <= n) break;
         }
@@ -617,16 +641,19 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     };
     bool ok = true;
     int it = 0, n = N - 1;
+    float g_later = 1.0f;   // e^{rho} of the chunk processed before this one (the later chunk), key dim j
     for (; n >= 0; --n, ++it) {
         const uint32_t par = it & 1;
         if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
         if (tid == 0) waited[0] = it + 1;
+        float em1 = 1.0f;   // E of the row before the chunk, e^{-rho}
+        float hh = 1.0f;    // the state scale e^{B - rho} = e^{rho} of this chunk, key dim j
         // ---- prep: column j, rows c0 .. c0+31: Qt = q E, Kt = k / E in place; E -> TMEM.
-        // f = e^a directly, so k = 1 - f has an absolute error of a few 1e-8; E is the running
-        // product of f from the range start, 1/E = e^{-b}.
+        // f = e^a directly, so k = 1 - f has an absolute error of a few 1e-8; E = e^{b - rho} is the
+        // running product of f from the range start, 1/E = e^{rho - b}.
         {
             const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
-            float bsum = 0.0f;   // per-dim: the running log-decay sum; scalar decay: the chunk's total
+            float bsum = 0.0f;   // the running b - rho; after the prep B - rho = B / 2
             float ev[32];
             if constexpr (kScalar) {
                 // b_t = cumulative log g from the chunk start (0 past the sequence end), threads 0..127
@@ -647,9 +674,12 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     m->Bpart[0][tid] = a;
                 }
                 __syncthreads();
-                bsum = m->Bpart[0][kTile - 1];
+                const float rho = 0.5f * m->Bpart[0][kTile - 1];   // the balanced reference
+                em1 = __expf(-rho);
+                bsum = rho;   // B - rho
+                hh = __expf(rho);
 #pragma unroll
-                for (int bt = 0; bt < 4; ++bt) {   // Qt = q e^{b_t}, Kt = k e^{-b_t} (b_t >= the range bound)
+                for (int bt = 0; bt < 4; ++bt) {   // Qt = q e^{b_t - rho}, Kt = k e^{rho - b_t}
                     const int t0 = c0 + 8 * bt;
                     float kv[8], qv[8];
 #pragma unroll
@@ -660,7 +690,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     __nv_bfloat16 oq[8], ok2[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float b = m->Bpart[0][t0 + i], E = __expf(b);
+                        const float b = m->Bpart[0][t0 + i] - rho, E = __expf(b);
                         ok2[i] = __float2bfloat16_rn(kv[i] * __expf(-b));
                         oq[i] = __float2bfloat16_rn(qv[i] * E);
                         ev[8 * bt + i] = E;
@@ -673,13 +703,20 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
             } else {
             float sum = 0.0f;
-            if (q4 < 3) {
 #pragma unroll 8
-                for (int i = 0; i < 32; ++i) sum += c0 + i < vr ? bfat(Gb, c0 + i) : 0.0f;
-                m->Bpart[q4][j] = sum;
-            }
+            for (int i = 0; i < 32; ++i) sum += c0 + i < vr ? bfat(Gb, c0 + i) : 0.0f;
+            // quarters 0..2 in Bpart, quarter 3 in EB (free from the start of the prep until the
+            // epilogue: the dS phase takes e^{B/2} from a register)
+            if (q4 < 3) m->Bpart[q4][j] = sum;
+            else m->EB[j] = sum;
             __syncthreads();
             for (int r2 = 0; r2 < q4; ++r2) bsum += m->Bpart[r2][j];
+            // the chunk total, summed in the same order by the four threads of key dim j
+            const float Btot = ((m->Bpart[0][j] + m->Bpart[1][j]) + m->Bpart[2][j]) + m->EB[j];
+            const float rho = 0.5f * Btot;   // the balanced reference
+            em1 = __expf(-rho);
+            hh = __expf(Btot - rho);
+            bsum -= rho;
             float E = __expf(bsum);
 #pragma unroll
             for (int bt = 0; bt < 4; ++bt) {
@@ -709,14 +746,15 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }   // per-dim prep
             tmem_st32(tl + kColE + c0, ev);
             tmem_wait_st();
-            if (q4 == 3) m->EB[j] = __expf(bsum);
             // the previous chunk's output stores have read their staging tiles (D16, AT, DA are
             // written next, from the dS phase on): waited for by the issuing thread before this barrier
             if (tid == kStoreTid) tma_store_wait_read0();
             fence_proxy_async_smem();
             tc_fence_before();
-            if (__syncthreads_or(q4 == 3 && !(bsum >= kMinLogEB))) {
-                if (tid == 0) set_status(HGRN2_ERR_DEVICE);   // the forward sweep passed this (b,h)
+            // the forward passed this (b,h): its chunks are in range (a unit of margin for the
+            // rounding of the two kernels' sums)
+            if (__syncthreads_or(q4 == 3 && !(bsum >= -kMaxRefLog - 1.0f))) {
+                if (tid == 0) set_status(HGRN2_ERR_DEVICE);
                 ok = false;
                 break;
             }
@@ -753,16 +791,19 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 }
             }
         }
-        // ---- dS phase: dSh = Diag(E_B) dS -> TMEM (becomes the new dS) and bf16 into D16; thread 0
-        // joins once it has issued phase 1
+        // ---- dS phase: dSh = Diag(e^{B - rho}) dL/dS_out -> TMEM (becomes the new dS) and bf16 into
+        // D16, with dL/dS_out = Diag(e^{rho_later}) dS of the later chunk; thread 0 joins once it has
+        // issued phase 1
         {
             float v[32];
             tc_fence_after();
             tmem_ld32(tl + kColDS + c0, v);
             tmem_wait_ld();
-            const float e = m->EB[j];
+            // one factor after the other: their product can fall below the fp32 range, while the first
+            // gives dL/dS_out of this chunk, O(1)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= e;
+            for (int i = 0; i < 32; ++i) v[i] = (v[i] * g_later) * hh;
+            g_later = hh;   // e^{rho} = e^{B - rho} of this chunk
             store_chunk_bf16(D16, j, q4, v);
             tmem_st32(tl + kColDS + c0, v);
             tmem_wait_st();
@@ -932,7 +973,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tmem_ld16(tl + kColX2 + col, dkp);
             tmem_ld16(tl + kColE + col, e);
             if (kSaved) tmem_ld16(tl + kColX1 + col, dap);   // dq_pre of these tokens
-            const float eprev = col > 0 ? tmem_ld1(tl + kColE + col - 1) : 1.0f;
+            const float eprev = col > 0 ? tmem_ld1(tl + kColE + col - 1) : em1;
             tmem_wait_ld();
             float invE = __fdividef(1.0f, e[15]);
 #pragma unroll
@@ -1038,9 +1079,11 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         float v[32];
         tmem_ld32(tl + kColDS + c0, v);
         tmem_wait_ld();
+        const float e = g_later;   // dh0 = Diag(e^{rho}) dL/dS_r of the first chunk
         float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * p.D + j) * p.D + c0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
     }
     if (tid == 0 && ok && n < 0) atomicAdd(&g_counters[1], (unsigned long long)N);
     tc_fence_before();

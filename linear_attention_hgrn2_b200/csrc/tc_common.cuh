@@ -13,8 +13,15 @@ namespace tcc {
 constexpr int kTile = 128;               // tokens per chunk (one M = 128 MMA tile)
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kBlk = 128 * 128;          // bytes of one 64-column block of a 128-row tile
-constexpr float kMinEB = 1e-26f;         // factorisation range: min_j E_B[j] (decay span ~60)
-constexpr float kMinLogEB = -59.8f;      // the same bound on the chunk's summed log decay
+// Factorisation range.  Inside a chunk the decay between tokens s <= t is split as
+// e^{b_t - b_s} = e^{b_t - rho} e^{rho - b_s}, with b the cumulative log decay from the chunk
+// start and the reference rho = B / 2, half the chunk's total B (per key dim).  Every factor
+// then lies in [e^{B/2}, e^{-B/2}], so a chunk is on the tensor cores while B / 2 >= -kMaxRefLog:
+// factors stay inside e^{+-75} (bf16 / fp32 overflow at e^{88.7}; a 128-term sum of products
+// of such a factor with O(1) values stays below 1e37, and values down to e^{-75} |x| stay
+// normal for |x| > 5e-6).  Beyond that span (an average log f below -1.17 over a 128-token
+// chunk) the pair takes the exact route.
+constexpr float kMaxRefLog = 75.0f;
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -79,6 +86,18 @@ __device__ __forceinline__ void store_row_bf16(uint8_t *blk, int row, const floa
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier over `count` threads that also ORs `pred` over them: every thread of the group
+// gets the same answer, so a group can leave a loop together (a thread that gave up a wait on
+// its own and skipped the next barrier would leave the others waiting there for good).
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 __device__ __forceinline__ int ld_volatile(const int *p) { return *reinterpret_cast<const volatile int *>(p); }
 

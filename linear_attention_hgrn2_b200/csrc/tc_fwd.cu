@@ -1,30 +1,38 @@
 // tc_fwd.cu -- chunkwise HGRN2 forward on 5th-generation tensor cores (sm_100a).
 //
 // One CTA walks the 128-token chunks of one (batch, head) (or of one segment of
-// it); d_k = d_v = 128, bf16 token tensors, fp32 state.  Per chunk, with
-// E_t = prod_{r<=t} f_r (cumulative inside the chunk, per key dim j),
-// k = 1 - f, S_in the state entering the chunk and E_B = E at the chunk end
-// ("HGRN2: Gated Linear RNNs with State Expansion", §3.2: gated linear attention
-// with key 1 - f, value i, query q, so chunkwise; §5: per-dimension decay):
+// it); d_k = d_v = 128, bf16 token tensors, fp32 state.  Per chunk and key dim j,
+// with b_t the cumulative log decay from the chunk start, B = b at the chunk end,
+// the reference rho = B / 2, E_t = e^{b_t - rho}, k = 1 - f and S_in the state
+// entering the chunk ("HGRN2: Gated Linear RNNs with State Expansion", §3.2: gated
+// linear attention with key 1 - f, value i, query q, so chunkwise; §5:
+// per-dimension decay):
 //
 //   Qt = q * E,  Kt = k / E                                    (bf16 in smem)
+//   S_r = Diag(e^rho) S_in                                     fp32 state in TMEM
 //   A  = mask_{s<=t}(Qt Kt^T)                                  tcgen05, fp32 in TMEM
-//   O  = Qt bf16(S_in) + bf16(A) V                             tcgen05, fp32 in TMEM
-//   S' = S_in + Kt^T V,   S_out = Diag(E_B) S'                 fp32 state in TMEM
+//   O  = Qt bf16(S_r) + bf16(A) V                              tcgen05, fp32 in TMEM
+//   S' = S_r + Kt^T V,   S_out = Diag(e^{B - rho}) S'          fp32 state in TMEM
 //
-// For training, the forward can also keep what the backward needs: bf16(S_in) of every
+// Qt Kt^T realises sum_j q_t[j] k_s[j] e^{b_t[j] - b_s[j]} through factors referenced
+// to rho, and Qt S_r realises sum_j q_t[j] e^{b_t[j]} S_in[j, :].  With rho = B / 2 (a
+// balanced reference, the stabilising second level of the chunk form: the decay is
+// split at the middle of its range instead of at the chunk start) every factor lies
+// in [e^{B/2}, e^{-B/2}], which halves the exponent range of the start-referenced
+// form.  A chunk is valid while B / 2 >= -75 for every key dim (an average log f of
+// -1.17 per token over the chunk; a first layer with lower bound 0 sums to about
+// -103 +- 6); a (batch, head) meeting a chunk beyond that is flagged and
+// recomputed afterwards by the exact CUDA-core route, which forms every exponent
+// as a difference of cumulative sums.
+//
+// For training, the forward can also keep what the backward needs: bf16(S_r) of every
 // chunk (the operand it builds anyway for the inter-chunk MMA, written out by a TMA store)
 // and the fp32 final state.
 //
-// The state is post-scaled: the MMA accumulates Kt^T V onto S_in, and the next
-// chunk multiplies the rows by this chunk's E_B before using it (the products
-// Kt * E_B = k * E_B / E <= k are never formed in bf16 at all).  Qt Kt^T realises
-// sum_j q_t[j] k_s[j] exp(b_t[j] - b_s[j]) through factors referenced to the
-// chunk start; it is valid while 1/E stays representable with margin, i.e.
-// min_j E_B[j] >= 1e-26 (a cumulative log-decay span of about 60 inside the
-// chunk).  A (batch, head) meeting a chunk beyond that is flagged and recomputed
-// afterwards by the exact CUDA-core route, which forms every exponent as a
-// difference of cumulative sums.
+// The two state scales of consecutive chunks are applied together: the next chunk's S
+// phase multiplies the rows by e^{B_n - rho_n} e^{rho_{n+1}} = e^{(B_n + B_{n+1}) / 2} <= 1
+// before building its operand (the products of Kt with these scales are never formed in
+// bf16 at all).
 //
 // Warp roles (16 warps), coordinated by mbarriers only:
 //   warp 0      TMA producer: q, log f, i tiles (128-byte swizzle) into a 2-stage ring; q and
@@ -64,7 +72,8 @@ struct __align__(8) Misc {
     int waited_full;                        // q / log f arrivals the prep warps consumed
     int waited_v;                           // v arrivals the MMA thread consumed
     float EB[2][128];                       // E_B ring: read by the TMEM warps while that chunk is current
-    float Ppart[3][128];                    // per 32-row range sums of log f (ranges 0..2)
+    float Ppart[3][128];                    // per 32-row range sums of log f (ranges 0..2; range 3's
+                                            // sums go to the stage's EB slot until the prep ends)
 };
 
 constexpr size_t kSmemBytes = 7 * (size_t)kTileBytes + sizeof(Misc);
@@ -92,9 +101,9 @@ struct Params {
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
 // kScalar: the scalar-decay variant S_t = g_t S_{t-1} + k_t v_t^T (one decay per head and token,
 // key k loaded in place of log f).  The same chunk form with a decay shared by the key dims:
-// b_t = cumulative log g from the chunk start, Qt = q e^{b_t}, Kt = k e^{-b_t} (per-row factors),
-// E_B = e^{B} for every state row.  A chunk with B < kMinLogEB sends the pair to the exact
-// CUDA-core forward (its flag also routes the backward).
+// b_t = cumulative log g from the chunk start, rho = B / 2, Qt = q e^{b_t - rho}, Kt = k e^{rho - b_t}
+// (per-row factors), the state scales e^{B/2} for every state row.  A chunk with B / 2 < -kMaxRefLog
+// sends the pair to the exact CUDA-core forward (its flag also routes the backward).
 template <bool kPacked, bool kScalar = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
@@ -280,29 +289,38 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tmem_wait_st();
         }
         int n = 0;
-        float e_prev = 1.0f, e_cur = 1.0f;   // E_B of the previous and the current chunk, key dim r
+        // a wait given up by a lane of this warp (warp-uniform, since the TMEM loads and stores
+        // are warp-collective): the group leaves together at its next barrier
+        bool fail = false;
+        auto wait_all = [&](uint64_t *bar, uint32_t par) {
+            fail = __any_sync(0xffffffffu, fail || !mbar_wait(bar, par));
+        };
+        // e^{B - rho} of the previous and the current chunk, key dim r (e^{B/2} for both scales)
+        float e_prev = 1.0f, e_cur = 1.0f;
         for (; n < N; ++n) {
             const int s = n & 1;
-            if (!mbar_wait(&m->prepped[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (ld_volatile(&m->bad_tile) <= n) break;
+            wait_all(&m->prepped[s], (n >> 1) & 1);
+            // the previous chunk's state MMA completed, and its o store has read X
+            if (n >= 1) {
+                wait_all(&m->barS, (n - 1) & 1);
+                if (r == 0) tma_store_wait_read0();
+            }
+            // one decision for the whole group: a wait given up anywhere in it, or a flagged chunk
+            if (named_bar_or(2, 128, fail || ld_volatile(&m->bad_tile) <= n)) break;
             e_prev = e_cur;
             e_cur = m->EB[s][kScalar ? 0 : r];   // the prep warps rewrite this slot only after this chunk's stage is released
-            // S phase: S_in = Diag(E_B of the previous chunk) S'; bf16(S_in) -> X (B operand),
-            // once the previous chunk's o store has read X
-            if (n >= 1 && !mbar_wait(&m->barS, (n - 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (n >= 1) {
-                if (r == 0) tma_store_wait_read0();
-                named_bar_sync(2, 128);
-            }
+            // S phase: S_r = Diag(e^{rho}) Diag(e^{B_prev - rho_prev}) S' of the previous chunk (both
+            // factors e^{B/2}); bf16(S_r) -> X (B operand).  The two factors are applied one after
+            // the other: the first gives S_out of the previous chunk, O(1), while their product can
+            // fall below the fp32 range (two strongly decaying chunks: e^{-52} e^{-52}).
             tc_fence_after();
-            const float e = e_prev;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
                 tmem_ld32(tl + kColS + 32 * c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= e;
+                for (int i = 0; i < 32; ++i) v[i] = (v[i] * e_prev) * e_cur;
                 store_chunk_bf16(X, r, c, v);
                 tmem_st32(tl + kColS + 32 * c, v);
             }
@@ -310,8 +328,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->sdone);
-            if (p.save) {   // bf16(S_in) of this chunk, kept for the backward
-                named_bar_sync(2, 128);
+            if (p.save) {   // bf16(S_r) of this chunk, kept for the backward
+                named_bar_sync(2, 128);   // no thread of the group has left since the barrier above
                 if (r == 0) {
                     const int slot = slot0 + n * sstride;
                     tma_store_4d(&tm_st, X, 0, 0, 0, slot);
@@ -322,7 +340,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             // causal mask of A -> bf16 pairs in TMEM columns P (the A operand of the intra MMA),
             // as soon as A is complete.  Column block c is kept (c < quad), dropped (c > quad) or
             // diagonal (per element).  The MMA that read the previous chunk's P completed before A.
-            if (!mbar_wait(&m->barA, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            // (After a wait given up, this thread goes on with whatever TMEM holds; nothing it
+            // writes is used, and the group leaves at its next barrier.)
+            wait_all(&m->barA, n & 1);
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -348,10 +368,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             mbar_arrive(&m->adone);
             // o epilogue: O -> bf16 rows in X (free: the last MMA of the chunk completed, and the
             // state store has read it) -> TMA store; the next S phase waits until the store has read X
-            if (!mbar_wait(&m->barO2, n & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
+            wait_all(&m->barO2, n & 1);
             if (p.save) {
                 if (r == 0) tma_store_wait_read0();
-                named_bar_sync(2, 128);
+                if (named_bar_or(2, 128, fail)) break;
             }
             tc_fence_after();
             const int vr = valid_rows(n);
@@ -366,13 +386,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&m->ofree);
-                named_bar_sync(2, 128);
+                if (named_bar_or(2, 128, fail)) break;
                 if (r == 0) {
                     tma_store_4d(&tm_o, X, 0, h, tok0 + n * kTile, bc);
                     if (nblk == 2) tma_store_4d(&tm_o, X + kBlk, 64, h, tok0 + n * kTile, bc);
                     tma_store_commit();
                 }
-            } else {   // a packed sequence's last chunk: its rows only, stored by their threads
+            } else if (!fail) {   // a packed sequence's last chunk: its rows only, stored by their threads
                 uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(tok0 + n * kTile + r) * p.H + h) * p.D);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -393,12 +413,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 mbar_arrive(&m->ofree);
             }
         }
+        if (fail) set_status(HGRN2_ERR_TIMEOUT);
         if (r == 0) tma_store_wait_all0();
         // the last state MMA must be complete before hT is read or TMEM is released
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        if (n == N && (p.hT || p.hTs) && seg == p.nseg - 1 && r < p.D) {   // warp-uniform
-            const float e = e_cur;
+        if (n == N && !fail && (p.hT || p.hTs) && seg == p.nseg - 1 && r < p.D) {   // warp-uniform
+            const float e = e_cur;   // hT = Diag(e^{B - rho}) S' of the last chunk
             float *dst = p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
             float *dsv = p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
 #pragma unroll
@@ -419,9 +440,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // ------------------------------------------------------------ prep warps
         // thread = one column pair (2 key dims, 4-byte smem accesses) and one 32-row range.
         // Each range first sums its own rows of log f; ranges exchange sums through shared
-        // memory.  Then f = e^a directly (so k = 1 - f has an absolute error of a few 1e-8),
-        // E = running product of f from the range start, 1/E = e^{-b} with b the running sum
-        // of log f.  Rows go in batches of 8: all loads, then the arithmetic, then all stores.
+        // memory, which also gives the chunk total B and the reference rho = B / 2.  Then
+        // f = e^a directly (so k = 1 - f has an absolute error of a few 1e-8), E = e^{b - rho}
+        // as the running product of f from the range start, 1/E = e^{rho - b} with b the
+        // running sum of log f.  Rows go in batches of 8: all loads, then the arithmetic, then
+        // all stores.
         const int ptid = tid - 256;
         const int pc = ptid & 63, rr = ptid >> 6, col0 = 2 * pc;
         const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
@@ -437,9 +460,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (kScalar) load_lg(0);
         for (int n = 0; n < N; ++n) {
             const int s = n & 1;
-            if (!mbar_wait(&m->fullQG[s], (n >> 1) & 1)) { set_status(HGRN2_ERR_TIMEOUT); break; }
-            if (ptid == 0) m->waited_full = n + 1;
+            const bool landed = mbar_wait(&m->fullQG[s], (n >> 1) & 1);
+            if (ptid == 0 && landed) m->waited_full = n + 1;
             if constexpr (kScalar) {
+                if (!__all_sync(0xffffffffu, landed)) {   // no group barrier here: each warp may leave alone
+                    set_status(HGRN2_ERR_TIMEOUT);
+                    break;
+                }
                 // b_t = cumulative log g from the chunk start (0 past the sequence end): every prep
                 // warp scans all 128 rows itself (rows 4l .. 4l+3 in lane l), so this prep needs no
                 // block barrier
@@ -457,17 +484,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     if (lane >= o) x += y;
                 }
                 const float ex = x - bl[3];   // sum over the lanes before this one
+                const float Bt = __shfl_sync(0xffffffffu, x, 31);   // the chunk total B
+                const float rho = 0.5f * Bt;                         // the balanced reference
                 float eq[4], ek[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    bl[j] += ex;
+                    bl[j] += ex - rho;
                     eq[j] = __expf(bl[j]);
                     ek[j] = __expf(-bl[j]);
                 }
-                const float Bt = __shfl_sync(0xffffffffu, bl[3], 31);
-                const bool bad = !(Bt >= kMinLogEB);   // also NaN
-                // Qt = q e^{b_t}, Kt = k e^{-b_t}, rows in batches of 8: row t = 32 rr + 8 bt + i has its
-                // factors in lane 8 rr + 2 bt + i / 4, slot i % 4
+                const bool bad = !(rho >= -kMaxRefLog);   // also NaN
+                // Qt = q e^{b_t - rho}, Kt = k e^{rho - b_t}, rows in batches of 8: row t = 32 rr + 8 bt + i
+                // has its factors in lane 8 rr + 2 bt + i / 4, slot i % 4
 #pragma unroll 1
                 for (int bt = 0; bt < 4; ++bt) {
                     const int t0 = 32 * rr + 8 * bt;
@@ -492,7 +520,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     }
                 }
                 if (ptid == 0) {   // read after prepped[s] completes (this thread arrives after these)
-                    m->EB[s][0] = __expf(Bt);
+                    m->EB[s][0] = __expf(Bt - rho);
                     if (bad) atomicMin(&m->bad_tile, n);
                 }
                 fence_proxy_async_smem();
@@ -501,25 +529,41 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 continue;
             }
             const int vr = valid_rows(n);   // rows from vr on: log f = 0 and q = 0 (no effect)
-            if (rr < 3) {
-                float s0 = 0.0f, s1 = 0.0f;
+            float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(32 * rr + i));
-                    if (32 * rr + i >= vr) w = 0u;
-                    s0 += bf_lo(w);
-                    s1 += bf_hi(w);
-                }
+            for (int i = 0; i < 32; ++i) {
+                uint32_t w = *reinterpret_cast<const uint32_t *>(Gb[s] + eoff(32 * rr + i));
+                if (32 * rr + i >= vr) w = 0u;
+                s0 += bf_lo(w);
+                s1 += bf_hi(w);
+            }
+            // ranges 0..2 in Ppart, range 3 in this stage's E_B slot (free until the end of this
+            // prep: the TMEM warps read it only after prepped[s], and its last reader, two chunks
+            // back, released the stage before these rows were loaded)
+            float *p3 = m->EB[s];
+            if (rr < 3) {
                 m->Ppart[rr][col0] = s0;
                 m->Ppart[rr][col0 + 1] = s1;
+            } else {
+                p3[col0] = s0;
+                p3[col0 + 1] = s1;
             }
-            named_bar_sync(1, 256);
-            float b0 = 0.0f, b1 = 0.0f;
+            // the whole prep group leaves together if any of its waits gave up (its later barriers
+            // would otherwise wait for the leavers)
+            if (named_bar_or(1, 256, !landed)) {
+                if (!landed) set_status(HGRN2_ERR_TIMEOUT);
+                break;
+            }
+            float b0 = 0.0f, b1 = 0.0f;   // sum of log f over the rows before this range
             for (int r2 = 0; r2 < rr; ++r2) {
                 b0 += m->Ppart[r2][col0];
                 b1 += m->Ppart[r2][col0 + 1];
             }
-            float E0 = __expf(b0), E1 = __expf(b1);   // E of the row before the range
+            // relative to the balanced reference rho = B / 2 (the chunk total, summed in the same
+            // order by the four threads of a column)
+            b0 -= 0.5f * (((m->Ppart[0][col0] + m->Ppart[1][col0]) + m->Ppart[2][col0]) + p3[col0]);
+            b1 -= 0.5f * (((m->Ppart[0][col0 + 1] + m->Ppart[1][col0 + 1]) + m->Ppart[2][col0 + 1]) + p3[col0 + 1]);
+            float E0 = __expf(b0), E1 = __expf(b1);   // E = e^{b - rho} of the row before the range
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
                 const int t0 = 32 * rr + 8 * bt;
@@ -547,13 +591,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     *reinterpret_cast<uint32_t *>(Gb[s] + eoff(t0 + i)) = wa[i];
                 }
             }
-            if (rr == 3) {
+            // b = B - rho = B / 2 now: the scale e^{B/2} of both state factors
+            if (rr == 3 && !(b0 >= -kMaxRefLog && b1 >= -kMaxRefLog)) atomicMin(&m->bad_tile, n);   // also NaN
+            fence_proxy_async_smem();
+            named_bar_sync(1, 256);   // bad_tile settled; Ppart and the range-3 sums read by all
+            if (rr == 3) {   // before this thread's arrival, which publishes it to the TMEM warps
                 m->EB[s][col0] = __expf(b0);
                 m->EB[s][col0 + 1] = __expf(b1);
-                if (!(b0 >= kMinLogEB && b1 >= kMinLogEB)) atomicMin(&m->bad_tile, n);
             }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 256);   // bad_tile settled; Ppart free for the next chunk
             mbar_arrive(&m->prepped[s]);
             if (ld_volatile(&m->bad_tile) <= n) break;
         }

@@ -55,6 +55,10 @@ DECODE = dict(name="decode_bf16_B256_H16_d128_1000steps", B=256, H=16, dk=128, d
 VARLEN = dict(name="varlen_train_bf16_T16384_H16_d128_docmean512", total_T=16384, H=16, dk=128, dv=128,
               dtype=torch.bfloat16, lb=0.95, mean_len=512, chunk=64)
 
+# the training workload with the first layer's forget-gate lower bound, lb = 0 (f = sigmoid(x))
+TRAIN_LB0 = Workload("train_fwdbwd_bf16_B8_H16_T2048_d128_lb0", 8, 16, 2048, 128, 128, torch.bfloat16,
+                     0.0, 64, bwd=True)
+
 # the training workload's hidden size (2048) with 64-wide heads
 TRAIN_D64 = Workload("train_fwdbwd_bf16_B8_H32_T2048_d64", 8, 32, 2048, 64, 64, torch.bfloat16, 0.95, 64, bwd=True)
 # ... and with 256-wide heads
@@ -89,15 +93,17 @@ def _to(x: np.ndarray, dtype: torch.dtype) -> torch.Tensor:
 
 def make_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: torch.dtype, lb: float,
                 seed: int, h0_sigma: float = 0.0, with_dO: bool = False,
-                dhT_sigma: float = 0.0) -> dict:
+                dhT_sigma: float = 0.0, gate_shift: float = 0.0) -> dict:
     """CPU tensors q, log_f, i [B,T,H,*] in ``dtype``; optional h0, dO, dhT.
 
+    The gate pre-activations are x ~ N(gate_shift, 1): a negative shift gives forget gates
+    near 0 (decays far stronger than the workloads', for edge cases).
     Draw order (fixed): q, i, gate pre-activations, dO, h0, dhT."""
     g = _gen(seed)
     out = {}
     out["q"] = _to(_normal(g, (B, T, H, dk)), dtype)
     out["i"] = _to(_normal(g, (B, T, H, dv)), dtype)
-    out["log_f"] = _to(gate_log_f(_normal(g, (B, T, H, dk)), lb), dtype)
+    out["log_f"] = _to(gate_log_f(_normal(g, (B, T, H, dk)) + np.float32(gate_shift), lb), dtype)
     if with_dO:
         out["dO"] = _to(_normal(g, (B, T, H, dv)), dtype)
     if h0_sigma > 0:

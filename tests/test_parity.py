@@ -199,14 +199,19 @@ def test_gate_zero_keeps_last_input(cuda, dtype):
 
 
 @pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
-def test_reports_exact_route_is_finite_for_strong_decay(cuda, saved):
-    # lb = 0 at chunk 128: cumulative log-decay spans of ~-100 inside a chunk (B*H = 2: the
-    # forward runs in sequence segments, then the exact route for the flagged pairs)
+def test_lower_bound_zero_stays_on_tensor_cores(cuda, saved):
+    # lb = 0 (the first layer's bound) at chunk 128: cumulative log-decay spans of about -103
+    # inside a chunk.  The balanced reference keeps every factor within e^{+-75}, so no pair
+    # leaves the tensor cores (B*H = 2: the forward runs in sequence segments)
     inp = I.make_inputs(1, 384, 2, 128, 128, torch.bfloat16, 0.0, seed=5, with_dO=True)
     g = to_cuda(inp)
     sv = L.new_saved(g["q"]) if saved else None
+    L.counters(reset=True)
     o, _ = L.fwd(g["q"], g["log_f"], g["i"], chunk=128, saved=sv)
     dq, dlf, di, _ = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], chunk=128, saved=sv)
+    c = L.counters(reset=True)
+    assert c[0] == 0, c   # no exact-route pass
+    assert L.device_status() == L.OK
     ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True)
     for n, h in enumerate((0, 1)):
         for name, got in (("o", o[0, :, h]), ("dq", dq[0, :, h]), ("dlog_f", dlf[0, :, h]),
@@ -215,14 +220,41 @@ def test_reports_exact_route_is_finite_for_strong_decay(cuda, saved):
             assert err(np64(got), ref[name][n], torch.bfloat16) <= 2e-2, name
 
 
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
+def test_workload_train_lower_bound_zero_full_size(cuda, saved):
+    # the training workload's shape with the first layer's lower bound, lb = 0 (forget gates
+    # sigmoid(x), x ~ N(0, 1)), in the launch configuration the benchmark times: every pair on
+    # the tensor cores, sampled pairs checked whole against the oracle
+    w = I.TRAIN
+    inp = I.make_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, 0.0, seed=1013, with_dO=True, h0_sigma=0.1,
+                        dhT_sigma=0.1)
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"]) if saved else None
+    L.counters(reset=True)
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=w.chunk, saved=sv)
+    dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True,
+                             chunk=w.chunk, saved=sv)
+    c = L.counters(reset=True)
+    assert c[0] == 0, c
+    assert L.device_status() == L.OK
+    pairs = _sample_pairs(w.B, w.H, 3, 3)
+    ref = oracle_heads(inp, pairs, want_bwd=True, dhT=inp["dhT"])
+    for n, (b, h) in enumerate(pairs):
+        for name, got in (("o", o[b, :, h]), ("hT", hT[b, h]), ("dq", dq[b, :, h]), ("dlog_f", dlf[b, :, h]),
+                          ("di", di[b, :, h]), ("dh0", dh0[b, h])):
+            e = err(np64(got), ref[name][n], w.dtype)
+            assert e <= 2e-2, (name, b, h, e)
+
+
 def test_saved_pair_launch_counts_and_mixed_routes(cuda):
-    # B*H = 80 > 148 / 2: one CTA per (b,h), no sequence segments.  Head 3 of batch 1 gets a
-    # strong decay (exact route), every other pair stays on the tensor cores; the saved
-    # backward is one launch and computes both kinds of pair.
+    # B*H = 80 > 148 / 2: one CTA per (b,h), no sequence segments.  Head 3 of batch 1 gets
+    # gates shifted down (chunk decays of ~-180, past the factorised range: exact route), every other
+    # pair stays on the tensor cores; the saved backward is one launch and computes both kinds
+    # of pair.
     B, T, H = 10, 600, 8
     inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.9, seed=77, h0_sigma=0.1, with_dO=True,
                         dhT_sigma=0.1)
-    strong = I.make_inputs(1, T, 1, 128, 128, torch.bfloat16, 0.0, seed=78)
+    strong = I.make_inputs(1, T, 1, 128, 128, torch.bfloat16, 0.0, seed=78, gate_shift=-1.0)
     inp["log_f"][1, :, 3] = strong["log_f"][0, :, 0]
     g = to_cuda(inp)
     sv = L.new_saved(g["q"])

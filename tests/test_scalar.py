@@ -124,12 +124,13 @@ def test_scalar_empty_sequence_passes_states_through(cuda):
     assert torch.equal(got["hT"], g["h0"]) and torch.equal(got["dh0"], g["dhT"])
 
 
-@pytest.mark.parametrize("d,lb,strong", [(128, 0.5, None), (64, 0.9, None), (128, 0.5, "all"), (64, 0.9, "one")],
-                         ids=["d128", "d64", "d128_strong_decay", "d64_one_flagged_head"])
+@pytest.mark.parametrize("d,lb,strong", [(128, 0.5, None), (64, 0.9, None), (128, 0.0, None), (128, 0.5, "all"),
+                                         (64, 0.9, "one")],
+                         ids=["d128", "d64", "d128_lb0", "d128_strong_decay", "d64_one_flagged_head"])
 def test_scalar_tensor_core_forward(cuda, d, lb, strong):
     # bf16 with d = 128 or 64 runs the scalar-decay instance of the tensor-core forward: chunk
     # passes and exact-route pairs are counted on the device.  A pair with a chunk whose summed
-    # log g is below -59.8 (log g = -12 per token: e^{-1536} over a chunk) is recomputed by the
+    # log g is below -150 (log g = -12 per token: e^{-1536} over a chunk) is recomputed by the
     # exact CUDA-core forward inside the same launch; the other pairs stay on the tensor cores.
     B, T, H = 2, 300, 3
     nt = (T + 127) // 128
@@ -159,13 +160,13 @@ def test_scalar_tensor_core_forward(cuda, d, lb, strong):
 def test_scalar_tensor_core_backward_with_a_flagged_head(cuda, d):
     # bf16 d = 128 / 64: the backward runs the forward again (chunk states saved into the workspace)
     # and the tensor-core reverse sweep: 4 launches (forward, reverse sweep, the exact route's two
-    # kernels for flagged pairs).  Head (1, 2) has log g = -1 per token, a chunk total of -128,
-    # past the factorised form's range: it is recomputed on CUDA cores; the rest stays on the
-    # tensor cores.  Every gradient must match the oracle.
+    # kernels for flagged pairs).  Head (1, 2) has log g = -2 per token, a chunk total of -256,
+    # past the factorised form's range (-150): it is recomputed on CUDA cores; the rest stays on
+    # the tensor cores.  Every gradient must match the oracle.
     B, T, H = 2, 300, 3
     inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, 0.9, seed=1400 + d, h0_sigma=0.1, with_dO=True,
                                dhT_sigma=0.1)
-    inp["log_g"][1, :, 2] = -1.0
+    inp["log_g"][1, :, 2] = -2.0
     g = to_cuda(inp)
     L.counters(reset=True)
     dq, dk, dv, dg, dh0 = L.scalar_bwd(g["q"], g["k"], g["v"], g["log_g"], g["dO"], g["h0"], g["dhT"],
@@ -185,7 +186,7 @@ def test_scalar_saved_state_pair(cuda, d):
     B, T, H = 2, 300, 3
     inp = I.make_scalar_inputs(B, T, H, d, d, torch.bfloat16, 0.9, seed=1500 + d, h0_sigma=0.1, with_dO=True,
                                dhT_sigma=0.1)
-    inp["log_g"][0, :, 1] = -1.0
+    inp["log_g"][0, :, 1] = -2.0
     g = to_cuda(inp)
     sv = L.new_scalar_saved(g["q"])
     assert sv is not None

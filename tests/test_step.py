@@ -5,7 +5,7 @@ import torch
 
 import linear_attention_hgrn2_b200 as L
 from linear_attention_hgrn2_b200 import inputs as I
-from parity_util import err, np64, tol
+from parity_util import err, norm_max_abs, np64, tol
 import oracle
 
 pytestmark = pytest.mark.gpu
@@ -72,9 +72,14 @@ def test_decode_workload_1000_steps_sampled(cuda):
         assert e <= tol(w["dtype"]), (t, e)
     torch.cuda.synchronize()
     assert torch.isfinite(S).all()
-    e_S = err(np64(S[bi.cuda(), hi.cuda()])[:, None], S_ref, torch.float32)
-    print(f"1000-step decode: worst o error {worst:.3e} (bar {tol(w['dtype'])}), final-state error {e_S:.3e}")
-    assert e_S <= 1e-5
+    S_got = np64(S[bi.cuda(), hi.cuda()])[:, None]
+    e_S = err(S_got, S_ref, torch.float32)
+    print(f"1000-step decode: worst o error {worst:.3e} (bar {tol(w['dtype'])}), final-state relative error "
+          f"{e_S:.3e}, normalised max-abs {norm_max_abs(S_got, S_ref):.3e}")
+    # the state is float32: the bar is the float32 accuracy statement (max relative error 1e-4).  A
+    # read-modify-write in float32 adds one rounding per step; 1000 steps of it measure ~1e-5 here.
+    assert e_S <= tol(torch.float32)
+    assert norm_max_abs(S_got, S_ref) <= tol(w["dtype"])
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])

@@ -112,13 +112,13 @@ def test_fp32_exact_route(cuda, case):
 
 
 def test_bf16_strong_decay_sequence_takes_the_exact_route(cuda):
-    # one sequence with lb = 0 at chunk 128 (log-decay spans of ~-100 inside a chunk): its
+    # one sequence with gates shifted down (log-decay spans of ~-180 inside a chunk): its
     # (sequence, head) pairs are flagged and recomputed by the exact route inside the same
     # launches, from the sequence's own offset; the others stay on the tensor cores
     lens = [200, 300, 150]
     inp = I.make_varlen(lens, 2, 128, 128, torch.bfloat16, 0.9, seed=604, h0_sigma=0.1, with_dO=True,
                         dhT_sigma=0.1)
-    strong = I.make_inputs(1, 300, 2, 128, 128, torch.bfloat16, 0.0, seed=605)
+    strong = I.make_inputs(1, 300, 2, 128, 128, torch.bfloat16, 0.0, seed=605, gate_shift=-1.0)
     inp["log_f"][200:500] = strong["log_f"][0]
     g = to_cuda(inp)
     L.counters(reset=True)

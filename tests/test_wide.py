@@ -65,7 +65,7 @@ def test_wide_strong_decay_head_takes_the_exact_route(cuda):
     # and recomputed on CUDA cores in both passes; the other head stays on the tensor cores
     B, T, H, d = 1, 300, 2, 256
     inp = I.make_inputs(B, T, H, d, d, torch.bfloat16, 0.9, seed=931, h0_sigma=0.1, with_dO=True, dhT_sigma=0.1)
-    strong = I.make_inputs(1, T, 1, d, d, torch.bfloat16, 0.0, seed=932)
+    strong = I.make_inputs(1, T, 1, d, d, torch.bfloat16, 0.0, seed=932, gate_shift=-1.0)
     inp["log_f"][0, :, 1] = strong["log_f"][0, :, 0]
     g = to_cuda(inp)
     sv = L.new_saved(g["q"])
