@@ -601,7 +601,7 @@ def run_fwd_configs(args, dev, pk, rank):
     """The two forward-only workloads: the forward layer (B=4, H=8, T=2048, lb=0.5) and the long
     sequence (B=1, H=8, T=32768, lb=0.9, h0 in, hT out).  With 32 and 8 (b,h) pairs they run the
     segmented forward: segment aggregates, an fp32 scan over segments, then every segment from
-    its incoming state (4 launches)."""
+    its incoming state (3 launches)."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
     res = {}

@@ -310,6 +310,43 @@ hgrn2_status hgrn2_scalar_bwd_saved(const void *q, const void *k, const void *v,
                                     int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
                                     void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* ---- One sequence across several GPUs (sequence parallelism) ----------------------
+ * Over a contiguous slice of tokens the recurrence (§3.2) is affine in the state that
+ * enters the slice, S_out = Diag(g) S_in + U, and its backward is affine in the gradient
+ * that leaves it, dL/dS_in = Diag(g) dL/dS_out + W, with
+ *   g = prod_t f_t,   U = sum_t (k_t * prod_{r>t} f_r) i_t^T,   W = sum_t (q_t * prod_{r<=t} f_r) dO_t^T.
+ * Each GPU computes the maps of its own slice, the maps are exchanged (the caller's
+ * all-gather), hgrn2_affine_scan gives each slice its boundary state, and each GPU then runs
+ * hgrn2_fwd / hgrn2_bwd on its slice from those boundary states (h0 = the state entering the
+ * slice, dhT = the gradient leaving it).  The chunkwise algorithm's state passing, with slices
+ * in place of chunks; the pages name linear-attention sequence parallelism (LASP) for running
+ * it across devices.
+ *
+ * hgrn2_state_map: the forward map of a slice.
+ *   log_f : [B,T,H,dk] (dtype)   i : [B,T,H,dv] (dtype)
+ *   g : out [B,H,dk] float32     U : out [B,H,dk,dv] float32
+ * hgrn2_state_map_bwd: the backward map of a slice (g is the same as the forward's).
+ *   q, log_f : [B,T,H,dk]   dO : [B,T,H,dv]   g : out [B,H,dk]   W : out [B,H,dk,dv]
+ * Both: dk <= 128, dv <= 256; T >= 0 (T = 0 gives g = 1, U = W = 0).  Exact for any decay
+ * strength (every product of gates is <= 1).  bf16 with dk = dv = 128 computes the forward map
+ * on the tensor cores; every other case steps the recurrence token by token on CUDA cores in
+ * fp32.  Asynchronous on `stream`; the library allocates nothing. */
+hgrn2_status hgrn2_state_map(const void *log_f, const void *i, int B, int T, int H, int dk, int dv,
+                             hgrn2_dtype dtype, float *g, float *U, cudaStream_t stream);
+hgrn2_status hgrn2_state_map_bwd(const void *q, const void *log_f, const void *dO, int B, int T, int H,
+                                 int dk, int dv, hgrn2_dtype dtype, float *g, float *W, cudaStream_t stream);
+
+/* Scan of R slice maps in fp32: S = init (zeros if NULL), then for `count` maps
+ * r = first, first + step, ... (step = +1 or -1, every r in [0, R)):
+ *   S <- Diag(g_r) S + M_r
+ *   g : [R][B,H,dk] float32   M : [R][B,H,dk,dv] float32   init, S : [B,H,dk,dv] float32
+ * Forward: r = 0 .. rank-1 from h0 gives the state entering slice `rank`; all R maps give
+ * hT.  Backward (M = W): r = R-1 down to rank+1 from dhT gives dL/dS leaving slice `rank`.
+ * S may be init (in place); it must not overlap g or M.  count = 0 copies init (or zeros). */
+hgrn2_status hgrn2_affine_scan(const float *g, const float *M, int R, int first, int count, int step,
+                               const float *init, float *S, int B, int H, int dk, int dv,
+                               cudaStream_t stream);
+
 /* Check of the failure reporting: launches one block that waits, through the bounded
  * wait every kernel of the library uses, on a barrier that nothing arrives at.  The
  * wait gives up after `polls` polls (1 .. 2^24; each poll lasts at most the hardware's

@@ -31,7 +31,8 @@ EXPORTS = ("hgrn2_workspace_size", "hgrn2_fwd", "hgrn2_bwd", "hgrn2_saved_size",
            "hgrn2_fwd_varlen", "hgrn2_bwd_varlen", "hgrn2_step", "hgrn2_step_lb", "hgrn2_step_bwd",
            "hgrn2_step_lb_bwd", "hgrn2_get_device_status", "hgrn2_get_counters", "hgrn2_status_string",
            "hgrn2_version", "hgrn2_selftest_wait_timeout", "hgrn2_scalar_workspace_size", "hgrn2_scalar_fwd",
-           "hgrn2_scalar_bwd", "hgrn2_scalar_saved_size", "hgrn2_scalar_fwd_train", "hgrn2_scalar_bwd_saved")
+           "hgrn2_scalar_bwd", "hgrn2_scalar_saved_size", "hgrn2_scalar_fwd_train", "hgrn2_scalar_bwd_saved",
+           "hgrn2_state_map", "hgrn2_state_map_bwd", "hgrn2_affine_scan")
 
 _lib = None
 
@@ -97,6 +98,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hgrn2_scalar_bwd.argtypes = [vp] * 12 + [i32] * 6 + [vp, sz, vp]
     lib.hgrn2_scalar_bwd.restype = i32
     lib.hgrn2_selftest_wait_timeout.restype = i32
+    lib.hgrn2_state_map.argtypes = [vp] * 2 + [i32] * 6 + [vp] * 3
+    lib.hgrn2_state_map.restype = i32
+    lib.hgrn2_state_map_bwd.argtypes = [vp] * 3 + [i32] * 6 + [vp] * 3
+    lib.hgrn2_state_map_bwd.restype = i32
+    lib.hgrn2_affine_scan.argtypes = [vp] * 2 + [i32] * 4 + [vp] * 2 + [i32] * 4 + [vp]
+    lib.hgrn2_affine_scan.restype = i32
     lib.hgrn2_get_device_status.restype = i32
     lib.hgrn2_get_counters.argtypes = [ctypes.POINTER(ctypes.c_longlong), i32, i32, vp]
     lib.hgrn2_get_counters.restype = i32
@@ -488,6 +495,54 @@ def scalar_bwd(q, k, v, log_g, dO, h0=None, dhT=None, want_dh0=False, saved=None
                               _stream())
     _raise(st, "hgrn2_scalar_bwd")
     return dq, dk_, dv_, dg, dh0
+
+
+# ---------------------------------------------------------------- one sequence across GPUs
+def state_map(log_f, i):
+    """The forward map of a token slice: S_out = Diag(g) S_in + U for every (b, h).
+
+    log_f: [B,T,H,dk]; i: [B,T,H,dv] (same dtype).  Returns (g [B,H,dk], U [B,H,dk,dv]), float32."""
+    B, T, H, dk = log_f.shape
+    dv = i.shape[-1]
+    _check(log_f, "log_f")
+    _check(i, "i", log_f.dtype, (B, T, H, dv))
+    g = torch.empty((B, H, dk), dtype=torch.float32, device=log_f.device)
+    U = torch.empty((B, H, dk, dv), dtype=torch.float32, device=log_f.device)
+    _raise(load_library().hgrn2_state_map(_ptr(log_f), _ptr(i), B, T, H, dk, dv, _dt(log_f), _ptr(g), _ptr(U),
+                                          _stream()), "hgrn2_state_map")
+    return g, U
+
+
+def state_map_bwd(q, log_f, dO):
+    """The backward map of a token slice: dL/dS_in = Diag(g) dL/dS_out + W.
+
+    q, log_f: [B,T,H,dk]; dO: [B,T,H,dv].  Returns (g [B,H,dk], W [B,H,dk,dv]), float32."""
+    B, T, H, dk = q.shape
+    dv = dO.shape[-1]
+    _check(q, "q")
+    _check(log_f, "log_f", q.dtype, q.shape)
+    _check(dO, "dO", q.dtype, (B, T, H, dv))
+    g = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
+    W = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _raise(load_library().hgrn2_state_map_bwd(_ptr(q), _ptr(log_f), _ptr(dO), B, T, H, dk, dv, _dt(q), _ptr(g),
+                                              _ptr(W), _stream()), "hgrn2_state_map_bwd")
+    return g, W
+
+
+def affine_scan(g, M, first: int, count: int, step: int = 1, init=None, out=None):
+    """S = init (or 0), then S <- Diag(g_r) S + M_r for r = first, first + step, ... (count maps).
+
+    g: [R,B,H,dk]; M: [R,B,H,dk,dv]; init, out: [B,H,dk,dv] float32 (out may be init)."""
+    R, B, H, dk, dv = M.shape
+    _check(g, "g", torch.float32, (R, B, H, dk))
+    _check(M, "M", torch.float32)
+    if init is not None:
+        _check(init, "init", torch.float32, (B, H, dk, dv))
+    S = out if out is not None else torch.empty((B, H, dk, dv), dtype=torch.float32, device=M.device)
+    _check(S, "out", torch.float32, (B, H, dk, dv))
+    _raise(load_library().hgrn2_affine_scan(_ptr(g), _ptr(M), R, first, count, step, _ptr(init), _ptr(S), B, H, dk,
+                                            dv, _stream()), "hgrn2_affine_scan")
+    return S
 
 
 def device_status() -> int:

@@ -322,14 +322,10 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
                     saved ? (float *)((char *)saved + sl.hTs) : nullptr, cu, perm, dk};
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
-        if (nseg == 1) {   // the exact route, if needed, runs inside the tensor-core kernel
-            g_launches += 1;
-            return HGRN2_OK;
-        }
-        // segmented: aggregate, scan, segments, then the exact route for flagged (b,h)
-        g_launches += 4;
-        SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, flags, nullptr, nullptr};
-        return from_cuda(launch_simt_fwd(a, bf16, stream));
+        // the exact route, if needed, runs inside the tensor-core kernel: in the pair's CTA, or with
+        // segments in the pair's last segment to finish (aggregate, scan, segments: 3 launches)
+        g_launches += nseg == 1 ? 1 : 3;
+        return HGRN2_OK;
     }
     SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr, cu, perm};
     g_launches += 1;
@@ -426,6 +422,12 @@ cudaError_t copy_cols_to(void *dst, size_t dpitch, const void *src, size_t rows,
 // Equal blocks: the columns of block pair j = a * n[1] + c go to head slot j of the H * nb heads
 // (token rows nb blocks wide, state matrices nb per (b, h)); one forward call runs them all, and
 // o[c] = sum over a of slot a * n[1] + c, added in fp32.
+// bf16 heads of 256 x 256 run on the tensor cores reading the caller's 256-wide rows in place (two
+// 128-wide half-heads each, key blocks for q and log f, value blocks for i and dO): no column
+// copies; the blocks' partial outputs land in summable layouts.  The backward does so from saved
+// states only.
+bool wide_inplace(int T, int dk, int dv, hgrn2_dtype dt) { return dt == HGRN2_BF16 && dk == 256 && dv == 256 && T > 0; }
+
 hgrn2_status stack_fwd(const void *q, const void *log_f, const void *i, const float *h0, void *o, float *hT,
                        void *saved, int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype,
                        void *workspace, cudaStream_t stream) {
@@ -434,6 +436,32 @@ hgrn2_status stack_fwd(const void *q, const void *log_f, const void *i, const fl
     const WideStack w = wide_stack_ws(B, T, H, dk, dv, chunk, dtype, 0, true, (char *)workspace);
     const bool bf16 = dtype == HGRN2_BF16;
     const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H, sm = (size_t)kw * vw;
+    if (wide_inplace(T, dk, dv, dtype)) {
+        for (int a = 0; a < nK && h0; ++a)
+            for (int c = 0; c < nV; ++c)
+                if (launch_state_block(const_cast<float *>(h0), w.h0 + (a * nV + c) * sm, nb * sm, BH, dk, dv,
+                                       s.off[0][a], kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                    return HGRN2_ERR_CUDA;
+        const int C = simt_chunk(chunk, kw, vw, false);
+        if (!C) return HGRN2_ERR_UNSUPPORTED;
+        const SavedLayout sl = saved_layout(B, T, H * nb);
+        int *flags = saved ? (int *)((char *)saved + sl.flags) : (int *)w.sub;
+        TcFwdArgs t{q, log_f, i, h0 ? w.h0 : nullptr, w.part, hT ? w.hT : nullptr, flags, nullptr, B, T, H * nb, C,
+                    saved, saved ? (float *)((char *)saved + sl.hTs) : nullptr, nullptr, nullptr, 128};
+        t.nK = nK;
+        t.nV = nV;
+        if (launch_tc_fwd(t, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+        for (int a = 0; a < nK && hT; ++a)
+            for (int c = 0; c < nV; ++c)
+                if (launch_state_block(hT, w.hT + (a * nV + c) * sm, nb * sm, BH, dk, dv, s.off[0][a], kw,
+                                       s.off[1][c], vw, true, stream) != cudaSuccess)
+                    return HGRN2_ERR_CUDA;
+        // o = the two key blocks' partials, [nK][B][T][H][256], added in fp32
+        if (launch_sum_blocks(o, dv, 0, w.part, w.part + rows * dv * es, dv, rows, dv, bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+        g_launches += (h0 ? nb : 0) + 1 + (hT ? nb : 0) + 1;
+        return HGRN2_OK;
+    }
     for (int a = 0; a < nK; ++a)
         for (int c = 0; c < nV; ++c) {
             const int j = a * nV + c;
@@ -472,6 +500,40 @@ hgrn2_status stack_bwd(const void *q, const void *log_f, const void *i, const fl
     const WideStack w = wide_stack_ws(B, T, H, dk, dv, chunk, dtype, 1, tc64, (char *)workspace);
     const bool bf16 = dtype == HGRN2_BF16;
     const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H, sm = (size_t)kw * vw;
+    if (saved && wide_inplace(T, dk, dv, dtype)) {
+        for (int a = 0; a < nK; ++a)
+            for (int c = 0; c < nV; ++c) {
+                const int j = a * nV + c;
+                if (h0 && launch_state_block(const_cast<float *>(h0), w.h0 + j * sm, nb * sm, BH, dk, dv, s.off[0][a],
+                                             kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                    return HGRN2_ERR_CUDA;
+                if (dhT && launch_state_block(const_cast<float *>(dhT), w.dhT + j * sm, nb * sm, BH, dk, dv,
+                                              s.off[0][a], kw, s.off[1][c], vw, false, stream) != cudaSuccess)
+                    return HGRN2_ERR_CUDA;
+            }
+        const int C = simt_chunk(chunk, kw, vw, true);
+        if (!C) return HGRN2_ERR_UNSUPPORTED;
+        const SavedLayout sl = saved_layout(B, T, H * nb);
+        TcBwdArgs t{q, log_f, i, dO, h0 ? w.h0 : nullptr, dhT ? w.dhT : nullptr, w.pq, w.pf, w.part,
+                    dh0 ? w.dh0 : nullptr, (float *)w.sub, (int *)((char *)saved + sl.flags), B, T, H * nb, C, saved,
+                    (const float *)((const char *)saved + sl.hTs), nullptr, nullptr, 128};
+        t.nK = nK;
+        t.nV = nV;
+        if (launch_tc_bwd(t, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+        for (int a = 0; a < nK && dh0; ++a)
+            for (int c = 0; c < nV; ++c)
+                if (launch_state_block(dh0, w.dh0 + (a * nV + c) * sm, nb * sm, BH, dk, dv, s.off[0][a], kw,
+                                       s.off[1][c], vw, true, stream) != cudaSuccess)
+                    return HGRN2_ERR_CUDA;
+        // dq, d log f: the value blocks' partials; di: the key blocks' ([2][B][T][H][256] each)
+        const size_t half = rows * 256 * es;
+        if (launch_sum_blocks(dq, dk, 0, w.pq, w.pq + half, dk, rows, dk, bf16, stream) != cudaSuccess ||
+            launch_sum_blocks(dlog_f, dk, 0, w.pf, w.pf + half, dk, rows, dk, bf16, stream) != cudaSuccess ||
+            launch_sum_blocks(di, dv, 0, w.part, w.part + half, dv, rows, dv, bf16, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+        g_launches += (h0 ? nb : 0) + (dhT ? nb : 0) + 1 + (dh0 ? nb : 0) + 3;
+        return HGRN2_OK;
+    }
     for (int a = 0; a < nK; ++a)
         for (int c = 0; c < nV; ++c) {
             const int j = a * nV + c;
@@ -764,6 +826,66 @@ hgrn2_status hgrn2_step_lb_bwd(const void *q, const void *g, const void *i, floa
     if (!(lb >= 0.0f && lb < 1.0f)) return HGRN2_ERR_INVALID_ARG;
     return step_bwd_impl(q, g, i, S, dO, dS, dS_prev, dq, dg, di, B, H, dk, dv, dtype, true, lb, stream);
 }
+
+// ------------------------------------------------------------------ sequence parallelism
+namespace {
+hgrn2_status state_map_impl(const void *q, const void *log_f, const void *v, int B, int T, int H, int dk, int dv,
+                            hgrn2_dtype dtype, float *g, float *M, bool backward, cudaStream_t stream) {
+    if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return HGRN2_ERR_INVALID_ARG;
+    if (dtype != HGRN2_FP32 && dtype != HGRN2_BF16) return HGRN2_ERR_INVALID_ARG;
+    if (dk > 128 || dv > 256 || (long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    if (!g || !M || (T > 0 && (!log_f || !v || (backward && !q)))) return HGRN2_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, log_f, v, g, M};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    if (!backward && T > 0 && dtype == HGRN2_BF16 && dk == 128 && dv == 128) {
+        g_launches += 1;
+        return from_cuda(launch_tc_state_map(log_f, v, B, T, H, g, M, stream));
+    }
+    StateMapArgs a{log_f, q, v, g, M, B, T, H, dk, dv, backward};
+    g_launches += 1;
+    return from_cuda(launch_state_map(a, dtype == HGRN2_BF16, stream));
+}
+}  // namespace
+
+extern "C" {
+
+hgrn2_status hgrn2_state_map(const void *log_f, const void *i, int B, int T, int H, int dk, int dv, hgrn2_dtype dtype,
+                             float *g, float *U, cudaStream_t stream) {
+    return state_map_impl(nullptr, log_f, i, B, T, H, dk, dv, dtype, g, U, false, stream);
+}
+
+hgrn2_status hgrn2_state_map_bwd(const void *q, const void *log_f, const void *dO, int B, int T, int H, int dk,
+                                 int dv, hgrn2_dtype dtype, float *g, float *W, cudaStream_t stream) {
+    return state_map_impl(q, log_f, dO, B, T, H, dk, dv, dtype, g, W, true, stream);
+}
+
+hgrn2_status hgrn2_affine_scan(const float *g, const float *M, int R, int first, int count, int step,
+                               const float *init, float *S, int B, int H, int dk, int dv, cudaStream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1 || R < 0 || count < 0 || (step != 1 && step != -1))
+        return HGRN2_ERR_INVALID_ARG;
+    if (dk > 256 || dv > 256 || (long long)B * H > (1ll << 30)) return HGRN2_ERR_UNSUPPORTED;
+    if (count > 0) {
+        const long long last = (long long)first + (long long)(count - 1) * step;
+        if (first < 0 || first >= R || last < 0 || last >= R || !g || !M) return HGRN2_ERR_INVALID_ARG;
+    }
+    if (!S) return HGRN2_ERR_INVALID_ARG;
+    const size_t nbh = (size_t)B * H, ns = nbh * dk * dv * sizeof(float);
+    const float *ptrs[] = {g, M, init, S};
+    for (const float *p : ptrs)
+        if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
+    if (count > 0) {   // S must not overlap the maps (init may be S itself)
+        auto overlap = [](const void *a, size_t na, const void *b, size_t nb) {
+            return (const char *)a < (const char *)b + nb && (const char *)b < (const char *)a + na;
+        };
+        if (overlap(S, ns, g, (size_t)R * nbh * dk * sizeof(float)) || overlap(S, ns, M, (size_t)R * ns))
+            return HGRN2_ERR_INVALID_ARG;
+    }
+    g_launches += 1;
+    return from_cuda(launch_affine_scan(g, M, init, S, nbh, dk, dv, first, count, step, stream));
+}
+
+}  // extern "C"
 
 // ------------------------------------------------------------------ scalar-decay variant
 namespace {

@@ -10,5 +10,6 @@
 #include "scalar.cu"
 #include "selftest.cu"
 #include "wide.cu"
+#include "seqpar.cu"
 #include "tc_fwd.cu"
 #include "tc_bwd.cu"

@@ -32,6 +32,10 @@ struct TcFwdArgs {
     const int *perm;   // with cu: launch order of the sequences (longest first), or null
     int D;             // head size d_k = d_v: 128 or 64
     const void *lgs;   // scalar-decay variant: log g [B][T][H] (lf is then the key k); else null
+    // Heads of width nK * 128 = nV * 128 read in place (nK = nV = 2: 256): H counts block pairs,
+    // H / (nK nV) the caller's heads; q, lf, x are the caller's [B][T][H / (nK nV)][256] tensors and
+    // o the key blocks' partials [nK][B][T][H / (nK nV)][256] (summed by the caller).
+    int nK = 1, nV = 1;
 };
 
 struct SimtBwdArgs {
@@ -62,6 +66,10 @@ struct TcBwdArgs {
     int D;             // head size d_k = d_v: 128 or 64 (64: saved-state mode only)
     const void *lgs;   // scalar-decay variant (saved mode): log g [B][T][H]; lf is then k, dlf dk
     void *dlg;         // scalar-decay variant: d log g [B][T][H]
+    // Heads read in place (saved mode, nK = nV = 2), as for TcFwdArgs: q, lf, x, dO are the caller's
+    // 256-wide tensors; dq, dlf the value blocks' partials [nV][B][T][Hw][256]; dx the key blocks'
+    // partials [nK][B][T][Hw][256].
+    int nK = 1, nV = 1;
 };
 
 struct StepBwdArgs {
@@ -105,6 +113,24 @@ cudaError_t launch_state_block(float *full, float *blk, size_t bstride, size_t n
                                int co, int cw, bool to_full, cudaStream_t st);
 cudaError_t launch_sum_blocks(void *dst, int pitch, int off, const void *p0, const void *p1, int spitch, size_t rows,
                               int w, bool bf16, cudaStream_t st);
+
+// State maps of a token slice (seqpar.cu): forward (g, U) from log f and v = i, or backward
+// (g, W) from log f, q and v = dO; [B][H][dk] and [B][H][dk][dv] fp32.  CUDA cores, any shape
+// with dk <= 128.
+struct StateMapArgs {
+    const void *lf, *q, *v;
+    float *g, *M;
+    int B, T, H, dk, dv;
+    bool backward;
+};
+cudaError_t launch_state_map(const StateMapArgs &a, bool bf16, cudaStream_t st);
+// The forward map of bf16 d = 128 slices on the tensor cores (the segment aggregate of tc_fwd.cu
+// over the whole slice).
+cudaError_t launch_tc_state_map(const void *lf, const void *x, int B, int T, int H, float *g, float *U,
+                                cudaStream_t st);
+// S = init (or 0); S <- Diag(g_r) S + M_r for r = first, first + step, ... (count maps).
+cudaError_t launch_affine_scan(const float *g, const float *M, const float *init, float *S, size_t nbh, int dk, int dv,
+                               int first, int count, int step, cudaStream_t st);
 
 size_t simt_fwd_smem(int C, int dk, int dv);
 size_t simt_bwd_dq_smem(int C, int dk, int dv);

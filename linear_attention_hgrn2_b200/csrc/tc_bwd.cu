@@ -487,6 +487,11 @@ struct RevParams {
                          // every operand tile is held at zero, which is exactly neutral)
     const __nv_bfloat16 *lgs;   // scalar decay: log g [B][T][H] (lf is then the key k, dlf its gradient)
     __nv_bfloat16 *dlg;         // scalar decay: d log g [B][T][H]
+    // Heads of width 256 read in place (saved mode; nK = nV = 2): head h of the call is block pair
+    // (a, c) of head h / (nK nV); q, log f at half-head (h / (nK nV)) nK + a and i, dO at * nV + c of
+    // the caller's tensors viewed as [B][T][2 Hw][128]; dq, d log f go to the value block's partial
+    // ([nV][B][T][Hw][256]), di to the key block's ([nK][B][T][Hw][256]).  nK = nV = 1 otherwise.
+    int nK, nV, Bo;
 };
 
 // kPacked (saved mode only): p.cu holds packed sequences; compiled apart so the dense path
@@ -496,7 +501,9 @@ struct RevParams {
 // the prep scans the gate per row instead of forming k = 1 - f; the epilogue writes dk = dk_pre /
 // E in place of d log f, has no tied-key term, and sums the per-dim reverse sums over d_k into
 // d log g_t.  Flagged pairs return at once; the host recomputes them on the exact route.
-template <bool kSaved, bool kPacked, bool kScalar = false>
+// kWide (saved mode only): heads of width 256 read in place (p.nK = p.nV = 2), compiled apart so
+// that the other instances carry none of its head arithmetic.
+template <bool kSaved, bool kPacked, bool kScalar = false, bool kWide = false>
 __global__ void __launch_bounds__(rsw::kRevThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
@@ -528,17 +535,38 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         sstride = p.H;
     }
     auto valid_rows = [&](int n) -> int { return kPacked ? min(kTile, len - n * kTile) : kTile; };
+    // head coordinates of the key-side (q, log f, dq, d log f) and value-side (i, dO, di) token
+    // tensors and the batch coordinates of the partial outputs; h and bc unless heads are read in place
+    static_assert(!kWide || (kSaved && !kPacked && !kScalar), "heads read in place: saved mode, dense, per-dim");
+    const int nK = kWide ? p.nK : 1, nV = kWide ? p.nV : 1, nbk = nK * nV;
+    const int hw = h / nbk, ka = (h - hw * nbk) / nV, vc = h - hw * nbk - ka * nV;
+    const int hk = hw * nK + ka, hv = hw * nV + vc, kbc = vc * p.Bo + bc, vbc = ka * p.Bo + bc;
     if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
         if (kSaved && !kScalar) {   // both sweeps here (recompute mode: in the forward-sweep kernel)
             float *sm = reinterpret_cast<float *>(smem);
             const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
             const int Tl = kPacked ? len : p.T;
-            simt_bwd_dq_body<__nv_bfloat16>(p.lf + ok, p.x + ok, p.h0, p.dO + ok, p.dhT, p.dq + ok, p.rs, Tl, p.H,
-                                            p.D, p.D, p.simt_chunk, sm, b, h, bh);
-            __syncthreads();
-            simt_bwd_rev_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.dO + ok, p.dhT, p.dq + ok, p.rs,
-                                             p.dlf + ok, p.dx + ok, p.dh0, Tl, p.H, p.D, p.D, p.simt_chunk, sm,
-                                             b, h, bh);
+            if constexpr (!kWide) {
+                simt_bwd_dq_body<__nv_bfloat16>(p.lf + ok, p.x + ok, p.h0, p.dO + ok, p.dhT, p.dq + ok, p.rs, Tl, p.H,
+                                                p.D, p.D, p.simt_chunk, sm, b, h, bh);
+                __syncthreads();
+                simt_bwd_rev_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.dO + ok, p.dhT, p.dq + ok, p.rs,
+                                                 p.dlf + ok, p.dx + ok, p.dh0, Tl, p.H, p.D, p.D, p.simt_chunk, sm,
+                                                 b, h, bh);
+            } else {
+                // heads read in place (nK = nV): every token tensor viewed with Hw nK half-heads of 128,
+                // indexed at the value-side half-head hv; key-side tensors shifted by hk - hv half-heads,
+                // the partial outputs by their block
+                const int Hh = (p.H / nbk) * p.nV;
+                const long long ks = (long long)(hk - hv) * p.D;
+                const size_t part = (size_t)p.Bo * p.T * Hh * p.D;
+                __nv_bfloat16 *dq = p.dq + vc * part + ks, *dlf = p.dlf + vc * part + ks, *dx = p.dx + ka * part;
+                simt_bwd_dq_body<__nv_bfloat16>(p.lf + ks, p.x, p.h0, p.dO, p.dhT, dq, p.rs, p.T, Hh, p.D, p.D,
+                                                p.simt_chunk, sm, b, hv, bh);
+                __syncthreads();
+                simt_bwd_rev_body<__nv_bfloat16>(p.q + ks, p.lf + ks, p.x, p.dO, p.dhT, dq, p.rs, dlf, dx, p.dh0, p.T,
+                                                 Hh, p.D, p.D, p.simt_chunk, sm, b, hv, bh);
+            }
             if (tid == 0) atomicAdd(&g_counters[0], 1ull);
         }
         return;
@@ -583,13 +611,15 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     int *issued = m->issued, *waited = m->waited;   // thread 0 issues; waits are recorded by thread 0
     if (tid == 0)
         for (int q = 0; q < 3; ++q) issued[q] = waited[q] = 0;
+    // two token tiles of one side (q, log f: key side, hk; i, dO: value side, hv)
     auto issue2 = [&](uint8_t *d0, const CUtensorMap *t0, uint8_t *d1, const CUtensorMap *t1, uint64_t *bar,
                       int q, int n) {
         ++issued[q];
+        const int hh = q == 0 ? hk : hv;
         mbar_arrive_expect_tx(bar, 2 * nblk * kBlk);
         for (int c = 0; c < nblk; ++c) {
-            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, h, tok0 + n * kTile, bc);
-            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, h, tok0 + n * kTile, bc);
+            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, hh, tok0 + n * kTile, bc);
+            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, hh, tok0 + n * kTile, bc);
         }
     };
     if (tid == 0 && N > 0) {
@@ -784,10 +814,10 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 if (kSaved) tma_prefetch_l2_4d(&tm_st, 64 * c, 0, 0, slot0 + n * sstride);
                 else tma_prefetch_l2_4d(&tm_dq, 64 * c, h, n * kTile, b);
                 if (n > 0) {
-                    tma_prefetch_l2_4d(&tm_q, 64 * c, h, tok0 + (n - 1) * kTile, bc);
-                    tma_prefetch_l2_4d(&tm_lf, 64 * c, h, tok0 + (n - 1) * kTile, bc);
-                    tma_prefetch_l2_4d(&tm_x, 64 * c, h, tok0 + (n - 1) * kTile, bc);
-                    tma_prefetch_l2_4d(&tm_do, 64 * c, h, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_q, 64 * c, hk, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_lf, 64 * c, hk, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_x, 64 * c, hv, tok0 + (n - 1) * kTile, bc);
+                    tma_prefetch_l2_4d(&tm_do, 64 * c, hv, tok0 + (n - 1) * kTile, bc);
                 }
             }
         }
@@ -1049,9 +1079,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (vr == kTile) {
             if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
                 for (int c = 0; c < nblk; ++c) {
-                    tma_store_4d(&tm_di, AT + c * kBlk, 64 * c, h, tok0 + n * kTile, bc);
-                    tma_store_4d(&tm_dlf, DA + c * kBlk, 64 * c, h, tok0 + n * kTile, bc);
-                    if (kSaved) tma_store_4d(&tm_dq, D16 + c * kBlk, 64 * c, h, tok0 + n * kTile, bc);
+                    tma_store_4d(&tm_di, AT + c * kBlk, 64 * c, hv, tok0 + n * kTile, vbc);
+                    tma_store_4d(&tm_dlf, DA + c * kBlk, 64 * c, hk, tok0 + n * kTile, kbc);
+                    if (kSaved) tma_store_4d(&tm_dq, D16 + c * kBlk, 64 * c, hk, tok0 + n * kTile, kbc);
                 }
                 tma_store_commit();
             }
@@ -1104,13 +1134,17 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     const bool packed = a.cu != nullptr;   // saved mode only; a.B is then the number of sequences
     if ((packed || a.D != 128 || a.lgs) && !saved) return cudaErrorInvalidValue;
     if (a.lgs && packed) return cudaErrorInvalidValue;
+    const int nbk = a.nK * a.nV;
+    const bool inplace = nbk > 1;
+    if (inplace && (!saved || packed || a.lgs || a.D != 128 || a.nK != a.nV || a.H % nbk)) return cudaErrorInvalidValue;
+    const int Hk = inplace ? a.H / nbk * a.nK : a.H, Hv = inplace ? a.H / nbk * a.nV : a.H;
     const int Bm = packed ? 1 : a.B, D = a.D;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl, mst;
-    if (!make_token_map(&mq, a.q, Bm, a.T, a.H, D) || !make_token_map(&ml, a.lf, Bm, a.T, a.H, D) ||
-        !make_token_map(&mx, a.x, Bm, a.T, a.H, D) || !make_token_map(&mdo, a.dO, Bm, a.T, a.H, D) ||
-        !make_token_map(&mdq, a.dq, Bm, a.T, a.H, D) || !make_token_map(&mdi, a.dx, Bm, a.T, a.H, D) ||
-        !make_token_map(&mdl, a.dlf, Bm, a.T, a.H, D))
+    if (!make_token_map(&mq, a.q, Bm, a.T, Hk, D) || !make_token_map(&ml, a.lf, Bm, a.T, Hk, D) ||
+        !make_token_map(&mx, a.x, Bm, a.T, Hv, D) || !make_token_map(&mdo, a.dO, Bm, a.T, Hv, D) ||
+        !make_token_map(&mdq, a.dq, Bm * a.nV, a.T, Hk, D) || !make_token_map(&mdi, a.dx, Bm * a.nK, a.T, Hv, D) ||
+        !make_token_map(&mdl, a.dlf, Bm * a.nV, a.T, Hk, D))
         return cudaErrorInvalidValue;
     // saved states: 128-row "token" tiles
     if (saved && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
@@ -1120,7 +1154,7 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
                       (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm, D, (const __nv_bfloat16 *)a.lgs,
-                      (__nv_bfloat16 *)a.dlg};
+                      (__nv_bfloat16 *)a.dlg, a.nK, a.nV, Bm};
     cudaError_t e;
     if (saved) {
         // one launch; the exact route of a flagged (b,h) runs in the same shared memory
@@ -1128,7 +1162,8 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
         if (simt_bwd_dq_smem(a.simt_C, D, D) > smem) smem = simt_bwd_dq_smem(a.simt_C, D, D);
         if (simt_bwd_rev_smem(a.simt_C, D, D) > smem) smem = simt_bwd_rev_smem(a.simt_C, D, D);
         auto kern = packed ? tcb::rev_kernel<true, true>
-                    : a.lgs ? tcb::rev_kernel<true, false, true> : tcb::rev_kernel<true, false>;
+                    : a.lgs ? tcb::rev_kernel<true, false, true>
+                    : inplace ? tcb::rev_kernel<true, false, false, true> : tcb::rev_kernel<true, false>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         kern<<<a.B * a.H, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);

@@ -85,7 +85,9 @@ struct Params {
     const __nv_bfloat16 *q, *lf, *x;   // for the in-kernel exact route
     int simt_chunk;
     int *flags;       // [B*H] set to 1 when the (b,h) must take the exact route
-    const float *Sin; // [B*H][nseg-1][128][128] state entering segments 1.. (from the scan)
+    float *Useg;      // with segments: [B*H][nseg][128][128] every segment's final state from its start
+                      // state (zero; h0 for segment 0), for the scan
+    float *gseg;      // with segments: [B*H][nseg][128] every segment's decay product (0 for segment 0)
     int T, H, ntiles;
     int nseg, tps;    // sequence segments per (b,h) and chunks per segment
     bool save;        // store bf16(S_in) of every chunk through tm_st
@@ -96,6 +98,12 @@ struct Params {
     int D;            // head size d_k = d_v: 128, or 64 (the second 64-column half of every operand
                       // tile is held at zero: log f = 0, q = i = 0 there, exactly neutral)
     const __nv_bfloat16 *lgs;   // scalar-decay variant: log g [B][T][H]; tm_lf then maps the key k
+    int *seg_done;    // with segments: [B*H] segments of the pair finished (zeroed by the aggregate kernel)
+    // Heads of width 256 read in place: head h of the call is block pair (a, c) of head
+    // h / (nK nV) of the caller's [B][T][Hw][256] tensors, a = key block, c = value block.  Those
+    // are read as [B][T][Hw nK][128] (q, log f: half-head Hw-index * nK + a) and [B][T][Hw nV][128]
+    // (i: * nV + c); o is the key block's partial, [nK][B][T][Hw nV][128].  nK = nV = 1 otherwise.
+    int nK, nV, Bo;   // Bo: the batch count of one o partial
 };
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
@@ -138,6 +146,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         sstride = p.H;
     }
     auto valid_rows = [&](int n) -> int { return kPacked ? min(kTile, len - n * kTile) : kTile; };
+    // head coordinates of the key-side (q, log f) and value-side (i, o) token tensors, and the
+    // batch coordinate of o (the key block's partial); all h and bc unless heads are read in place
+    const int nbk = p.nK * p.nV, hw = h / nbk, ka = (h - hw * nbk) / p.nV, vc = h - hw * nbk - ka * p.nV;
+    const int hk = hw * p.nK + ka, hv = hw * p.nV + vc, obc = ka * p.Bo + bc;
     if (smem_u32(smem) & 1023u) {   // the swizzled operand layout needs 1024-byte alignment
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
@@ -196,14 +208,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 if (n >= 2 && !wait_or_abort(&m->emptyQG[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
                 mbar_arrive_expect_tx(&m->fullQG[s], 2 * nblk * kBlk);
                 for (int c = 0; c < nblk; ++c) {
-                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, h, tok0 + n * kTile, bc);
-                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, h, tok0 + n * kTile, bc);
+                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, hk, tok0 + n * kTile, bc);
+                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, hk, tok0 + n * kTile, bc);
                 }
                 ++issued_qg;
                 if (n >= 2 && !wait_or_abort(&m->emptyV[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
                 mbar_arrive_expect_tx(&m->fullV[s], nblk * kBlk);
                 for (int c = 0; c < nblk; ++c)
-                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, h, tok0 + n * kTile, bc);
+                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, hv, tok0 + n * kTile, bc);
                 ++issued_v;
             }
         }
@@ -267,9 +279,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // ------------------------------------------------------------ TMEM warps
         const int quad = warp & 3, r = 32 * quad + lane;             // TMEM lane = tile row
         const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
-        {   // S = h0 / scanned incoming state / 0 (d x d, zero outside for d = 64)
-            const float *init = seg == 0 ? (p.h0 ? p.h0 + (size_t)bh * p.D * p.D : nullptr)
-                                         : p.Sin + ((size_t)bh * (p.nseg - 1) + seg - 1) * 16384;
+        {   // S = h0 for a sequence's first segment, else 0 (d x d, zero outside for d = 64): with
+            // segments, the carried state is added afterwards (fixup_kernel)
+            const float *init = seg == 0 && p.h0 ? p.h0 + (size_t)bh * p.D * p.D : nullptr;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 float v[32];
@@ -297,6 +309,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         };
         // e^{B - rho} of the previous and the current chunk, key dim r (e^{B/2} for both scales)
         float e_prev = 1.0f, e_cur = 1.0f;
+        float gprod = 1.0f;   // with segments: the segment's decay product, prod of e^{B} = (e^{B/2})^2
         for (; n < N; ++n) {
             const int s = n & 1;
             wait_all(&m->prepped[s], (n >> 1) & 1);
@@ -309,6 +322,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (named_bar_or(2, 128, fail || ld_volatile(&m->bad_tile) <= n)) break;
             e_prev = e_cur;
             e_cur = m->EB[s][kScalar ? 0 : r];   // the prep warps rewrite this slot only after this chunk's stage is released
+            gprod = (gprod * e_cur) * e_cur;
             // S phase: S_r = Diag(e^{rho}) Diag(e^{B_prev - rho_prev}) S' of the previous chunk (both
             // factors e^{B/2}); bf16(S_r) -> X (B operand).  The two factors are applied one after
             // the other: the first gives S_out of the previous chunk, O(1), while their product can
@@ -388,8 +402,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 mbar_arrive(&m->ofree);
                 if (named_bar_or(2, 128, fail)) break;
                 if (r == 0) {
-                    tma_store_4d(&tm_o, X, 0, h, tok0 + n * kTile, bc);
-                    if (nblk == 2) tma_store_4d(&tm_o, X + kBlk, 64, h, tok0 + n * kTile, bc);
+                    tma_store_4d(&tm_o, X, 0, hv, tok0 + n * kTile, obc);
+                    if (nblk == 2) tma_store_4d(&tm_o, X + kBlk, 64, hv, tok0 + n * kTile, obc);
                     tma_store_commit();
                 }
             } else if (!fail) {   // a packed sequence's last chunk: its rows only, stored by their threads
@@ -414,14 +428,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             }
         }
         if (fail) set_status(HGRN2_ERR_TIMEOUT);
-        if (r == 0) tma_store_wait_all0();
+        if (r == 0) {
+            tma_store_wait_all0();
+            fence_proxy_async_global();   // the stores are ordered before the segment count below
+        }
         // the last state MMA must be complete before hT is read or TMEM is released
         if (n >= 1) mbar_wait(&m->barS, (n - 1) & 1);
         tc_fence_after();
-        if (n == N && !fail && (p.hT || p.hTs) && seg == p.nseg - 1 && r < p.D) {   // warp-uniform
-            const float e = e_cur;   // hT = Diag(e^{B - rho}) S' of the last chunk
-            float *dst = p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
-            float *dsv = p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
+        if (p.nseg > 1 && n == N && !fail) {   // with segments: this segment's map (g, U) for the scan
+            if (r < p.D) p.gseg[((size_t)bh * p.nseg + seg) * 128 + r] = seg == 0 ? 0.0f : gprod;
+        }
+        if (n == N && !fail && (p.nseg > 1 || ((p.hT || p.hTs) && seg == p.nseg - 1)) && r < p.D) {   // warp-uniform
+            const float e = e_cur;   // hT (or the segment's U) = Diag(e^{B - rho}) S' of the last chunk
+            float *dst = p.nseg > 1 ? p.Useg + (((size_t)bh * p.nseg + seg) * 128 + r) * 128
+                                    : p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
+            float *dsv = p.nseg > 1 ? nullptr : p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 if (32 * c >= p.D) break;
@@ -548,6 +569,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 p3[col0] = s0;
                 p3[col0 + 1] = s1;
             }
+
             // the whole prep group leaves together if any of its waits gave up (its later barriers
             // would otherwise wait for the leavers)
             if (named_bar_or(1, 256, !landed)) {
@@ -559,10 +581,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 b0 += m->Ppart[r2][col0];
                 b1 += m->Ppart[r2][col0 + 1];
             }
-            // relative to the balanced reference rho = B / 2 (the chunk total, summed in the same
-            // order by the four threads of a column)
-            b0 -= 0.5f * (((m->Ppart[0][col0] + m->Ppart[1][col0]) + m->Ppart[2][col0]) + p3[col0]);
-            b1 -= 0.5f * (((m->Ppart[0][col0 + 1] + m->Ppart[1][col0 + 1]) + m->Ppart[2][col0 + 1]) + p3[col0 + 1]);
+            // the chunk total, summed in the same order by the four threads of a column
+            const float Bt0 = ((m->Ppart[0][col0] + m->Ppart[1][col0]) + m->Ppart[2][col0]) + p3[col0];
+            const float Bt1 = ((m->Ppart[0][col0 + 1] + m->Ppart[1][col0 + 1]) + m->Ppart[2][col0 + 1]) + p3[col0 + 1];
+            // relative to the balanced reference rho = B / 2
+            b0 -= 0.5f * Bt0;
+            b1 -= 0.5f * Bt1;
             float E0 = __expf(b0), E1 = __expf(b1);   // E = e^{b - rho} of the row before the range
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
@@ -622,29 +646,60 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     __syncwarp();
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
-    // exact route for this (b,h) when it runs unsegmented: the pipeline is drained, so the
-    // CTA's shared memory is free for the CUDA-core chunkwise forward of the whole sequence
-    if (fell_back && p.nseg == 1) {
+    // With segments, the last segment of the pair to finish runs the exact route for the whole
+    // sequence if any segment flagged the pair (every other segment's flag, o and hT stores are
+    // complete before its count: its stores were waited for, then the fence and the atomic)
+    bool exact = fell_back && p.nseg == 1;
+    if (p.nseg > 1) {
+        if (tid == 0) {
+            fence_proxy_async_global();   // this CTA's bulk-async o stores before the count
+            __threadfence();
+            const int prev = atomicAdd(&p.seg_done[bh], 1);
+            __threadfence();
+            m->waited_v = (prev == p.nseg - 1 && ld_volatile(&p.flags[bh]) != 0) ? 1 : 0;
+        }
+        __syncthreads();
+        exact = m->waited_v != 0;
+    }
+    // exact route for this (b,h): the pipeline is drained, so the CTA's shared memory is free for
+    // the CUDA-core chunkwise forward of the whole sequence
+    if (exact) {
         __syncthreads();
         if constexpr (kScalar) {   // the scalar-decay exact forward (key k in p.lf, value v in p.x)
             sd::fwd_body<__nv_bfloat16>(p.q, p.lf, p.x, p.lgs, p.h0, p.o, p.hT, p.T, p.H, p.D, p.D,
                                         reinterpret_cast<float *>(smem), b, h, bh);
         } else {
-            const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
-            simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T,
-                                         p.H, p.D, p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
+            // the whole sequence from its first token: a packed sequence's offset (a segmented
+            // launch's tok0 is its segment's first token, not the sequence's)
+            const size_t ok = kPacked ? (size_t)tok0 * p.H * p.D : 0;
+            if (nbk == 1) {
+                simt_fwd_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.h0, p.o + ok, p.hT, kPacked ? len : p.T,
+                                             p.H, p.D, p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, h, bh);
+            } else {
+                // heads read in place (nK = nV): every token tensor is viewed with Hw nK half-heads of
+                // 128 and indexed at the value-side half-head hv; the key-side tensors are shifted by
+                // the half-heads between hk and hv, and o by its key block's partial
+                const int Hh = (p.H / nbk) * p.nV;   // half-heads of the token tensors
+                const long long kshift = (long long)(hk - hv) * p.D;
+                const size_t opart = (size_t)ka * p.Bo * p.T * Hh * p.D;
+                simt_fwd_body<__nv_bfloat16>(p.q + kshift, p.lf + kshift, p.x, p.h0, p.o + opart, p.hT, p.T, Hh, p.D,
+                                             p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, hv, bh);
+            }
         }
     }
 }
 
 // ------------------------------------------------------------------ sequence segments
 // For few (batch, head) pairs, each sequence is cut into segments of `tps` chunks run by
-// separate CTAs.  The state map of a segment started from zero is affine in its incoming
-// state: S_out = Diag(g) S_in + U with g = prod of the chunks' E_B and U the state the
-// segment reaches from S_in = 0.  agg_kernel computes (g, U) for every segment but the
-// last, scan_kernel chains them in fp32 from h0, and fwd_kernel then runs each segment
-// from its incoming state.  The aggregate uses Kh = k * prod_{r>t} f_r directly
-// (suffix products inside the chunk), so it is exact for any decay strength.
+// separate CTAs.  The state map of a segment is affine in its incoming state:
+// S_out = Diag(g) S_in + U with g = prod of the chunks' e^{B} and U the state the segment
+// reaches from S_in = 0.  fwd_kernel runs every segment from zero (the first from h0) and
+// writes its (g, U); scan_kernel chains them in fp32 (the states entering the segments, and
+// hT); fixup_kernel adds the carried states to the segments' outputs.
+//
+// agg_kernel computes (g, U) of a run of chunks without its outputs, on the tensor cores, with
+// Kh = k * prod_{r>t} f_r directly (suffix products inside the chunk): exact for any decay
+// strength.  It serves hgrn2_state_map (one segment = a whole slice).
 struct AggMisc {
     uint64_t full[2];
     uint64_t barM;
@@ -657,7 +712,8 @@ constexpr size_t kAggSmem = 4 * (size_t)kTileBytes + sizeof(AggMisc);
 
 struct AggParams {
     float *U, *g;     // [B*H][nseg-1][128][128], [B*H][nseg-1][128]
-    int *flags;       // zeroed here (segment 0) before fwd_kernel sets exact-route flags
+    int *flags;       // zeroed here (segment 0) before fwd_kernel sets exact-route flags (or null)
+    int *seg_done;    // zeroed here (segment 0): fwd_kernel's finished-segment counts (or null)
     int H, nseg, tps;
 };
 
@@ -680,7 +736,8 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
         mbar_init(&m->full[1], 1);
         mbar_init(&m->barM, 1);
         fence_mbar_init();
-        if (seg == 0) p.flags[bh] = 0;
+        if (seg == 0 && p.flags) p.flags[bh] = 0;
+        if (seg == 0 && p.seg_done) p.seg_done[bh] = 0;
     }
     if (warp == 0) {
         tmem_alloc(&m->tmem_base, 128);
@@ -759,7 +816,15 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
             S1 *= f1[i];
         }
         fence_proxy_async_smem();
-        __syncthreads();
+        // the previous chunk's MMA ran under this prep: it must be done before S is scaled, and
+        // before its stage takes the chunk after this one
+        if (n >= 1) {
+            if (__syncthreads_or(!mbar_wait(&m->barM, (n - 1) & 1))) { ok = false; break; }
+            tc_fence_after();
+            if (tid == 0 && n + 1 < N) issue_load(n + 1);
+        } else {
+            __syncthreads();
+        }
         {   // S <- Diag(E_B) S
             float r0[32], r1[32];
             tc_fence_after();
@@ -779,7 +844,7 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
         }
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0) {   // S += Kh^T V, completing under the next chunk's prep
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
@@ -787,10 +852,9 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
                             sdesc_add(sdesc_sw128(smem_u32(Vb[s]), kBlk, 1024), kk * 2048), id_mnmn, true);
             mma_commit(&m->barM);
         }
-        if (__syncthreads_or(!mbar_wait(&m->barM, n & 1))) { ok = false; break; }
-        tc_fence_after();
-        if (tid == 0 && n + 2 < N) issue_load(n + 2);
     }
+    if (ok && N > 0 && __syncthreads_or(!mbar_wait(&m->barM, (N - 1) & 1))) ok = false;   // the last MMA
+    tc_fence_after();
     if (!ok && tid == 0) {
         set_status(HGRN2_ERR_TIMEOUT);
         for (int k = waited; k < issued; ++k) mbar_wait(&m->full[k & 1], (k >> 1) & 1, 2000000u);
@@ -815,23 +879,266 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
     if (warp == 0) tmem_dealloc(tbase, 128);
 }
 
-// S_in(segment 0) = h0 (or 0); S_in(seg+1) = Diag(g_seg) S_in(seg) + U_seg, in fp32, written
-// over U_seg.  One thread per 4 consecutive state elements of one (batch, head).
+// With segments: every segment ran from a zero state (segment 0 from h0), so its final state is
+// U_seg and the state entering segment k is the scan of the maps of segments 0..k-1 (segment 0's
+// g is 0: h0 is inside its U).  In fp32, over the U slots: slot k-1 becomes the state entering
+// segment k; the sequence's final state goes to hT (and the saved final state).  Pairs the exact
+// route recomputed whole (flagged) are left alone.  One thread per 4 consecutive state elements
+// of one (batch, head).
 __global__ void __launch_bounds__(256)
-scan_kernel(const float *__restrict__ h0, float *__restrict__ U, const float *__restrict__ g, int nseg) {
+scan_kernel(float *__restrict__ U, const float *__restrict__ g, int nseg, const int *__restrict__ flags,
+            float *__restrict__ hT, float *__restrict__ hTs) {
     const int bh = blockIdx.x >> 4;
+    if (flags[bh]) return;
     const int e = ((blockIdx.x & 15) * 256 + threadIdx.x) * 4;   // element offset in [0, 16384)
     const int jrow = e >> 7;
-    const int nagg = nseg - 1;
-    float4 S = h0 ? *reinterpret_cast<const float4 *>(h0 + (size_t)bh * 16384 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sg = 0; sg < nagg; ++sg) {
-        const size_t slot = (size_t)bh * nagg + sg;
+    float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sg = 0; sg < nseg; ++sg) {
+        const size_t slot = (size_t)bh * nseg + sg;
         float4 *u = reinterpret_cast<float4 *>(U + slot * 16384 + e);
         const float gj = g[slot * 128 + jrow];
         const float4 uv = *u;
         S = make_float4(fmaf(gj, S.x, uv.x), fmaf(gj, S.y, uv.y), fmaf(gj, S.z, uv.z), fmaf(gj, S.w, uv.w));
-        *u = S;
+        if (sg < nseg - 1) {
+            *u = S;
+        } else {
+            if (hT) *reinterpret_cast<float4 *>(hT + (size_t)bh * 16384 + e) = S;
+            if (hTs) *reinterpret_cast<float4 *>(hTs + (size_t)bh * 16384 + e) = S;
+        }
     }
+}
+
+// ------------------------------------------------------------------ carried-state fix-up
+// With segments, segment k >= 1 of a pair ran from a zero state; its outputs lack the state S_in
+// that enters it, carried through its chunks with no new input:
+//   o_t += (q_t * e^{b_t})^T S_c,      S_{c+1} = Diag(e^{B_c}) S_c,      S_0 = S_in
+// (b_t the cumulative log decay from chunk c's start, B_c its total; every factor <= 1), and,
+// when the chunk states are kept for the backward, the chunk's saved bf16(e^{rho} S_in) lacks
+// e^{rho_c} S_c.  One CTA per segment walks its chunks from the start and stops once
+// max_j decay_j max_v |S_in[j,v]| < 2^-40: no term it could still add exceeds 128 |q| 2^-40 (the
+// outputs are bf16, 2^-8 relative).  Single-stage: per chunk, load q, log f, o (and the saved
+// state), form Qt = q e^{b} in place, one MMA O = Qt bf16(S_c) into TMEM, add it to o, correct
+// the saved state, scale the carried state; 8 warps, thread (row r, half) holds 64 columns of
+// row r of the carried state in registers.
+struct FixMisc {
+    uint64_t full, barM;
+    uint32_t tmem_base;
+    int pad;
+    float EB[128];        // e^{B} of the chunk, key dim
+    float ER[128];        // e^{rho} = e^{B/2} of the chunk, key dim (the saved states' scale)
+    float Ppart[3][128];  // per 32-row range sums of log f (ranges 0..2)
+};
+constexpr size_t kFixSmem = 5 * (size_t)kTileBytes + sizeof(FixMisc);
+
+struct FixParams {
+    const float *Sin;   // [B*H][nseg][128][128]: slot k-1 = the state entering segment k (the scan)
+    const int *flags;   // [B*H] nonzero: recomputed whole by the exact route (skipped)
+    int H, nseg, tps, ntiles;
+    bool save;          // saved bf16 chunk states (slot bh * ntiles + chunk) to correct
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
+             const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_st, FixParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *Qb = smem, *Gb = smem + kTileBytes, *Ob = smem + 2 * kTileBytes, *Sb = smem + 3 * kTileBytes;
+    uint8_t *X = smem + 4 * kTileBytes;
+    FixMisc *m = reinterpret_cast<FixMisc *>(smem + 5 * kTileBytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nfix = p.nseg - 1;
+    const int bh = blockIdx.x / nfix, seg = 1 + blockIdx.x - bh * nfix, b = bh / p.H, h = bh - b * p.H;
+    if (p.flags[bh]) return;
+    const int g0 = seg * p.tps, N = min(p.ntiles - g0, p.tps);
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0) set_status(HGRN2_ERR_DEVICE);
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(&m->full, 1);
+        mbar_init(&m->barM, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = m->tmem_base;
+    const int quad = warp & 3, ch = warp >> 2, r = 32 * quad + lane;   // carried-state row / token row r
+    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+    // the carried state, row r, columns 64 ch .. 64 ch + 63
+    float S[64];
+    float smax = 0.0f;
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(p.Sin + ((size_t)bh * p.nseg + seg - 1) * 16384 +
+                                                             (size_t)r * 128 + 64 * ch);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float4 a = src[i];
+            S[4 * i] = a.x; S[4 * i + 1] = a.y; S[4 * i + 2] = a.z; S[4 * i + 3] = a.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 64; ++i) smax = fmaxf(smax, fabsf(S[i]));
+    }
+    float decay = 1.0f;   // the carried decay of row r so far
+    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
+    const int pc = tid & 63, rr = tid >> 6, col0 = 2 * pc;   // prep: column pair, 32-row range
+    const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
+    auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+    int issued = 0, waited = 0;
+    bool ok = true;
+    for (int c = 0; c < N; ++c) {
+        // stop once nothing the carried state could still add is above 2^-40
+        if (!__syncthreads_or(decay * smax >= 0x1p-40f)) break;
+        const int tok = (g0 + c) * kTile, slot = bh * p.ntiles + g0 + c;
+        if (tid == 0) {
+            tma_store_wait_read0();   // the previous chunk's stores have read Ob, Sb
+            ++issued;
+            mbar_arrive_expect_tx(&m->full, (p.save ? 4 : 3) * kTileBytes);
+            for (int k = 0; k < 2; ++k) {
+                tma_load_4d(Qb + k * kBlk, &tm_q, &m->full, 64 * k, h, tok, b);
+                tma_load_4d(Gb + k * kBlk, &tm_lf, &m->full, 64 * k, h, tok, b);
+                tma_load_4d(Ob + k * kBlk, &tm_o, &m->full, 64 * k, h, tok, b);
+                if (p.save) tma_load_4d(Sb + k * kBlk, &tm_st, &m->full, 64 * k, 0, 0, slot);
+            }
+        }
+        // bf16(S_c) -> X, the MN-major B operand (row r = key dim, columns = value dims)
+        {
+            float v[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = S[32 * hh + i];
+                store_chunk_bf16(X, r, 2 * ch + hh, v);
+            }
+        }
+        if (__syncthreads_or(!mbar_wait(&m->full, c & 1))) { ok = false; break; }
+        waited = issued;
+        // prep: b = cumulative log f from the chunk start; Qt = q e^{b} in place; e^{B}, e^{B/2}
+        {
+            float s0 = 0.0f, s1 = 0.0f;
+            if (rr < 3) {
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb + eoff(32 * rr + i));
+                    s0 += bf_lo(w);
+                    s1 += bf_hi(w);
+                }
+                m->Ppart[rr][col0] = s0;
+                m->Ppart[rr][col0 + 1] = s1;
+            }
+            __syncthreads();
+            float b0 = 0.0f, b1 = 0.0f;
+            for (int r2 = 0; r2 < rr; ++r2) {
+                b0 += m->Ppart[r2][col0];
+                b1 += m->Ppart[r2][col0 + 1];
+            }
+            float E0 = __expf(b0), E1 = __expf(b1);
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                const int t = 32 * rr + i;
+                const uint32_t wa = *reinterpret_cast<const uint32_t *>(Gb + eoff(t));
+                uint32_t *wq = reinterpret_cast<uint32_t *>(Qb + eoff(t));
+                b0 += bf_lo(wa);
+                b1 += bf_hi(wa);
+                E0 *= __expf(bf_lo(wa));
+                E1 *= __expf(bf_hi(wa));
+                *wq = pack_bf2(bf_lo(*wq) * E0, bf_hi(*wq) * E1);
+            }
+            if (rr == 3) {   // b = the chunk total B now (summed as the forward's prep sums it: the
+                             // three ranges' totals, then this range's rows)
+                m->EB[col0] = __expf(b0);
+                m->EB[col0 + 1] = __expf(b1);
+                m->ER[col0] = __expf(0.5f * b0);
+                m->ER[col0 + 1] = __expf(0.5f * b1);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {   // O = Qt bf16(S_c): M = tokens, N = value dims, K = key dims
+            tc_fence_after();
+            const uint64_t dQ = sdesc_sw128(smem_u32(Qb), 16, 1024);
+            const uint64_t dXm = sdesc_sw128(smem_u32(X), kBlk, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase, sdesc_add(dQ, ko), sdesc_add(dXm, kk * 2048), id_kmn, kk > 0);
+            }
+            mma_commit(&m->barM);
+        }
+        // the saved state of this chunk, row r (key dim): + e^{rho} S_c
+        if (p.save) {
+            const float er = m->ER[r];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+                const int cc = 2 * ch + hh;
+                uint8_t *base = Sb + (cc >> 1) * kBlk + r * 128;
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        v[8 * qd + 2 * k] = bf_lo(ws[k]) + er * S[32 * hh + 8 * qd + 2 * k];
+                        v[8 * qd + 2 * k + 1] = bf_hi(ws[k]) + er * S[32 * hh + 8 * qd + 2 * k + 1];
+                    }
+                }
+                store_chunk_bf16(Sb, r, cc, v);
+            }
+        }
+        if (__syncthreads_or(!mbar_wait(&m->barM, c & 1))) { ok = false; break; }
+        tc_fence_after();
+        // o row r (token) += O row r
+        {
+            float v[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int cc = 2 * ch + hh;
+                tmem_ld32(tl + 32 * cc, v);
+                tmem_wait_ld();
+                uint8_t *base = Ob + (cc >> 1) * kBlk + r * 128;
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        v[8 * qd + 2 * k] += bf_lo(ws[k]);
+                        v[8 * qd + 2 * k + 1] += bf_hi(ws[k]);
+                    }
+                }
+                store_chunk_bf16(Ob, r, cc, v);
+            }
+        }
+        // the carried state to the next chunk
+        const float eb = m->EB[r];
+        decay *= eb;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) S[i] *= eb;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            for (int k = 0; k < 2; ++k) {
+                tma_store_4d(&tm_o, Ob + k * kBlk, 64 * k, h, tok, b);
+                if (p.save) tma_store_4d(&tm_st, Sb + k * kBlk, 64 * k, 0, 0, slot);
+            }
+            tma_store_commit();
+        }
+    }
+    if (!ok && tid == 0) {
+        set_status(HGRN2_ERR_TIMEOUT);
+        for (int k = waited; k < issued; ++k) mbar_wait(&m->full, k & 1, 2000000u);
+    }
+    if (tid == 0) tma_store_wait_all0();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, 128);
 }
 
 }  // namespace tcf
@@ -839,6 +1146,7 @@ scan_kernel(const float *__restrict__ h0, float *__restrict__ U, const float *__
 // ------------------------------------------------------------------ host side
 static_assert(tcf::kSmemBytes <= 227 * 1024, "forward shared memory");
 static_assert(tcf::kAggSmem <= 227 * 1024, "aggregate shared memory");
+static_assert(tcf::kFixSmem <= 227 * 1024, "fix-up shared memory");
 static_assert(sd::fwd_smem(128, 128) <= tcf::kSmemBytes, "scalar-decay exact forward inside the forward kernel");
 
 // Segments per (b,h): enough CTAs to cover the 148 SMs of a B200 once, at most one per chunk.
@@ -856,7 +1164,9 @@ void tc_fwd_segments(int B, int T, int H, int *nseg, int *tps) {
 size_t tc_fwd_workspace(int B, int T, int H) {
     int nseg, tps;
     tc_fwd_segments(B, T, H, &nseg, &tps);
-    return (size_t)B * H * (nseg - 1) * (16384 + 128) * sizeof(float);
+    if (nseg <= 1) return 0;
+    // (U, g) of every segment, then the per-pair finished-segment counts
+    return (size_t)B * H * nseg * (16384 + 128) * sizeof(float) + (size_t)B * H * sizeof(int);
 }
 
 size_t tc_fwd_smem() { return tcf::kSmemBytes; }
@@ -868,12 +1178,29 @@ int tc_saved_slots(int B, int T, int H, bool packed) {
     return packed ? ((T >> 7) + B) * H : B * H * ((T + tcc::kTile - 1) / tcc::kTile);
 }
 
+// The whole slice as one segment: (g, U) of every (b,h), [B*H][128] and [B*H][128][128].
+cudaError_t launch_tc_state_map(const void *lf, const void *x, int B, int T, int H, float *g, float *U,
+                                cudaStream_t st) {
+    CUtensorMap ml, mx;
+    if (!make_token_map(&ml, lf, B, T, H, 128) || !make_token_map(&mx, x, B, T, H, 128)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(tcf::agg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kAggSmem);
+    if (e != cudaSuccess) return e;
+    const int ntiles = (T + tcc::kTile - 1) / tcc::kTile;
+    tcf::AggParams ap{U, g, nullptr, nullptr, H, 2, ntiles};
+    tcf::agg_kernel<<<B * H, tcf::kThreads, tcf::kAggSmem, st>>>(ml, mx, ap);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     const bool packed = a.cu != nullptr;   // a.B is then the number of sequences
     const int Bm = packed ? 1 : a.B;
+    const int nbk = a.nK * a.nV;
+    const bool inplace = nbk > 1;
+    if (inplace && (packed || a.lgs || a.D != 128 || a.nK != a.nV || a.H % nbk)) return cudaErrorInvalidValue;
+    const int Hk = inplace ? a.H / nbk * a.nK : a.H, Hv = inplace ? a.H / nbk * a.nV : a.H;
     CUtensorMap mq, ml, mx, mo, mst;
-    if (!make_token_map(&mq, a.q, Bm, a.T, a.H, a.D) || !make_token_map(&ml, a.lf, Bm, a.T, a.H, a.D) ||
-        !make_token_map(&mx, a.x, Bm, a.T, a.H, a.D) || !make_token_map(&mo, a.o, Bm, a.T, a.H, a.D))
+    if (!make_token_map(&mq, a.q, Bm, a.T, Hk, a.D) || !make_token_map(&ml, a.lf, Bm, a.T, Hk, a.D) ||
+        !make_token_map(&mx, a.x, Bm, a.T, Hv, a.D) || !make_token_map(&mo, a.o, Bm * a.nK, a.T, Hv, a.D))
         return cudaErrorInvalidValue;
     // saved states: 128-row "token" tiles
     if (a.st16 && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
@@ -885,23 +1212,29 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     int nseg = 1, tps = ntiles;
-    if (!packed && !scalar && a.D == 128) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);   // else one CTA per (b,h)
+    if (!packed && !scalar && !inplace && a.D == 128) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);   // else one CTA per (b,h)
     const int BH = a.B * a.H;
-    float *U = a.seg_ws, *g = a.seg_ws ? a.seg_ws + (size_t)BH * (nseg - 1) * 16384 : nullptr;
+    float *U = a.seg_ws, *g = a.seg_ws ? a.seg_ws + (size_t)BH * nseg * 16384 : nullptr;
+    int *seg_done = a.seg_ws ? reinterpret_cast<int *>(g + (size_t)BH * nseg * 128) : nullptr;
     if (nseg > 1) {
-        e = cudaFuncSetAttribute(tcf::agg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kAggSmem);
-        if (e != cudaSuccess) return e;
-        tcf::AggParams ap{U, g, a.flags, a.H, nseg, tps};
-        tcf::agg_kernel<<<BH * (nseg - 1), tcf::kThreads, tcf::kAggSmem, st>>>(ml, mx, ap);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        tcf::scan_kernel<<<BH * 16, 256, 0, st>>>(a.h0, U, g, nseg);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        // pass 1 only raises the exact-route flags and counts finished segments: both start at zero
+        if (!a.seg_ws || !a.flags) return cudaErrorInvalidValue;
+        if ((e = cudaMemsetAsync(a.flags, 0, sizeof(int) * (size_t)BH, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(seg_done, 0, sizeof(int) * (size_t)BH, st)) != cudaSuccess) return e;
     }
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
-                  (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, a.T, a.H, ntiles, nseg, tps,
+                  (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, g, a.T, a.H, ntiles, nseg, tps,
                   a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D,
-                  (const __nv_bfloat16 *)a.lgs};
+                  (const __nv_bfloat16 *)a.lgs, seg_done, a.nK, a.nV, Bm};
     kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
+    if ((e = cudaGetLastError()) != cudaSuccess || nseg == 1) return e;
+    // segments: the states entering them (and hT), then the carried states' contributions
+    tcf::scan_kernel<<<BH * 16, 256, 0, st>>>(U, g, nseg, a.flags, a.hT, a.st16 ? a.hTs : nullptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tcf::fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kFixSmem);
+    if (e != cudaSuccess) return e;
+    tcf::FixParams fp{U, a.flags, a.H, nseg, tps, ntiles, a.st16 != nullptr};
+    tcf::fixup_kernel<<<BH * (nseg - 1), tcf::kThreads, tcf::kFixSmem, st>>>(mq, ml, mo, mst, fp);
     return cudaGetLastError();
 }
 

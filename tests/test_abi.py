@@ -367,3 +367,22 @@ def test_noalloc_size_limit_boundary(lib, dt, d, limit):
     vp = ctypes.c_void_p(16)
     st = lib.hgrn2_bwd_noalloc(vp, vp, vp, None, vp, None, vp, vp, vp, None, 1, 64, limit + 1, d, d, 64, dt, None)
     assert st == L.ERR_UNSUPPORTED
+
+
+def test_sequence_parallel_entry_points_check_their_arguments(lib):
+    # host-side refusals, before any launch
+    vp = ctypes.c_void_p
+    a, b = vp(1 << 20), vp(1 << 24)   # two aligned, disjoint stand-in addresses (never dereferenced)
+    # state maps: key dims above 128, unknown dtype, null outputs, misaligned pointers
+    assert lib.hgrn2_state_map(a, a, 1, 8, 1, 129, 16, L.FP32, a, b, None) == L.ERR_UNSUPPORTED
+    assert lib.hgrn2_state_map(a, a, 1, 8, 1, 16, 16, 7, a, b, None) == L.ERR_INVALID_ARG
+    assert lib.hgrn2_state_map(a, a, 1, 8, 1, 16, 16, L.FP32, None, b, None) == L.ERR_INVALID_ARG
+    assert lib.hgrn2_state_map_bwd(None, a, a, 1, 8, 1, 16, 16, L.FP32, a, b, None) == L.ERR_INVALID_ARG
+    assert lib.hgrn2_state_map(vp((1 << 20) + 4), a, 1, 8, 1, 16, 16, L.FP32, a, b, None) == L.ERR_INVALID_ARG
+    # scan: maps outside [0, R), a step other than +-1, an output overlapping the maps
+    f = lib.hgrn2_affine_scan
+    assert f(a, b, 4, 3, 2, 1, None, vp(1 << 28), 1, 1, 16, 16, None) == L.ERR_INVALID_ARG   # maps 3, 4
+    assert f(a, b, 4, 1, 3, -1, None, vp(1 << 28), 1, 1, 16, 16, None) == L.ERR_INVALID_ARG  # maps 1, 0, -1
+    assert f(a, b, 4, 0, 2, 2, None, vp(1 << 28), 1, 1, 16, 16, None) == L.ERR_INVALID_ARG
+    assert f(a, b, 4, 0, 2, 1, None, b, 1, 1, 16, 16, None) == L.ERR_INVALID_ARG            # S on M
+    assert f(a, b, 4, 0, 2, 1, None, None, 1, 1, 16, 16, None) == L.ERR_INVALID_ARG          # no output

@@ -288,7 +288,7 @@ def test_autograd_function_uses_saved_states(cuda):
     loss = (o.float() * g["dO"].float()).sum() + (hT * g["dhT"]).sum()
     loss.backward()
     c = L.counters(reset=True)
-    assert c[2] == 4 + 1, c   # segmented forward (4 launches) + one saved backward launch
+    assert c[2] == 3 + 1, c   # segmented forward (3 launches) + one saved backward launch
     ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True, dhT=inp["dhT"])
     for n, h in enumerate((0, 1)):
         for name, got in (("dq", q.grad[0, :, h]), ("dlog_f", lf.grad[0, :, h]), ("di", x.grad[0, :, h]),
@@ -316,6 +316,37 @@ def test_more_pairs_than_sms(cuda, saved):
                           ("di", di[b, :, h]), ("dh0", dh0[b, h])):
             e = err(np64(got), ref[name][n], torch.bfloat16)
             assert e <= 2e-2, (name, b, h, e)
+
+
+@pytest.mark.parametrize("saved", [False, True], ids=["plain", "saved"])
+def test_segmented_forward_with_a_flagged_pair(cuda, saved):
+    # B*H = 2: the forward runs in sequence segments (aggregate, scan, segments: 3 launches).  Head 1
+    # has gates shifted below the factorised range: its segments flag it, and the last of its
+    # segments to finish recomputes the whole sequence on the exact route in the same launch
+    B, T, H = 1, 1000, 2
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.9, seed=61, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    strong = I.make_inputs(1, T, 1, 128, 128, torch.bfloat16, 0.0, seed=62, gate_shift=-1.0)
+    inp["log_f"][0, :, 1] = strong["log_f"][0, :, 0]
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"]) if saved else None
+    L.counters(reset=True)
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    c = L.counters(reset=True)
+    assert c[2] == 3 and c[0] >= 1, c
+    assert L.device_status() == L.OK
+    want_bwd = saved
+    if saved:
+        dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
+                                 saved=sv)
+    ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=want_bwd, dhT=inp["dhT"])
+    for n, h in enumerate((0, 1)):
+        got = [("o", o[0, :, h]), ("hT", hT[0, h])]
+        if saved:
+            got += [("dq", dq[0, :, h]), ("dlog_f", dlf[0, :, h]), ("di", di[0, :, h]), ("dh0", dh0[0, h])]
+        for name, t in got:
+            e = err(np64(t), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, h, e)
 
 
 def test_saved_pair_long_segmented_sequence(cuda):
