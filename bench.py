@@ -590,8 +590,8 @@ def run_head_dim(args, dev, pk, rank, w, seed_off, ref_ms=None):
     if ref_ms:
         res["step_time_vs_headline"] = round(ms / ref_ms, 4)
     if w.dk > 128 or w.dv > 128:
-        res["route"] = ("128-wide blocks on the tensor cores (column copies in, partial outputs added in fp32); "
-                        "bwd_frac counts the algorithmic bytes of the wide head only")
+        res["route"] = ("128-wide half-head blocks on the tensor cores, read in place; partial outputs added in "
+                        "fp32; bwd_frac counts the algorithmic bytes of the wide head only")
     del inp, q, lf, x, dO, sv, o
     torch.cuda.empty_cache()
     return res
@@ -600,8 +600,9 @@ def run_head_dim(args, dev, pk, rank, w, seed_off, ref_ms=None):
 def run_fwd_configs(args, dev, pk, rank):
     """The two forward-only workloads: the forward layer (B=4, H=8, T=2048, lb=0.5) and the long
     sequence (B=1, H=8, T=32768, lb=0.9, h0 in, hT out).  With 32 and 8 (b,h) pairs they run the
-    segmented forward: segment aggregates, an fp32 scan over segments, then every segment from
-    its incoming state (3 launches)."""
+    segmented forward: every segment from a zero state, then the carried states added to the
+    segments' first chunks (2 launches for the forward layer's 4 segments per pair; 3 for the
+    long sequence's 18, whose fp32 scan over segments is a launch of its own)."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
     res = {}

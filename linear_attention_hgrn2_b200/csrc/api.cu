@@ -323,8 +323,9 @@ hgrn2_status fwd_impl(const void *q, const void *log_f, const void *i, const flo
         cudaError_t e = launch_tc_fwd(t, stream);
         if (e != cudaSuccess) return HGRN2_ERR_CUDA;
         // the exact route, if needed, runs inside the tensor-core kernel: in the pair's CTA, or with
-        // segments in the pair's last segment to finish (aggregate, scan, segments: 3 launches)
-        g_launches += nseg == 1 ? 1 : 3;
+        // segments in the pair's last segment to finish (segments, the scan beyond a few segments,
+        // the carried-state fix-up)
+        g_launches += tc_fwd_launches(nseg);
         return HGRN2_OK;
     }
     SimtFwdArgs a{q, log_f, i, h0, o, hT, B, T, H, dk, dv, C, nullptr, cu, perm};

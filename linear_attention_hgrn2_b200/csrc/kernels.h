@@ -142,6 +142,8 @@ size_t tc_fwd_smem();
 int tc_saved_slots(int B, int T, int H, bool packed);
 void tc_fwd_segments(int B, int T, int H, int *nseg, int *tps);
 size_t tc_fwd_workspace(int B, int T, int H);
+// Kernel launches of one segmented forward call with nseg segments per pair (1 without segments).
+int tc_fwd_launches(int nseg);
 size_t tc_bwd_smem();
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st);

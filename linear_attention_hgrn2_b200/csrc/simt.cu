@@ -57,6 +57,30 @@ static __device__ __forceinline__ void load_tile(float *dst, int ld, const T *sr
     }
 }
 
+// A 16-bit token tensor carries fp32 values of dq between the exact backward's two sweeps: the
+// forward sweep writes each value's low half into the d log f row and its high half into the di
+// row of its token (rows the reverse sweep overwrites only after reading them back), so that the
+// reverse sweep's d log f sums q dq over the sequence from fp32 dq, not from the rounded output.
+// Needs d_v >= d_k; tok() indexes both tensors as usual.
+static __device__ __forceinline__ void stash_f32(void *lo, void *hi, size_t ilo, size_t ihi, float v) {
+    const uint32_t u = __float_as_uint(v);
+    reinterpret_cast<uint16_t *>(lo)[ilo] = (uint16_t)(u & 0xffffu);
+    reinterpret_cast<uint16_t *>(hi)[ihi] = (uint16_t)(u >> 16);
+}
+static __device__ __forceinline__ void load_stash(float *dst, int ld, const void *lo, const void *hi, int b, int h,
+                                                  int c0, int C, int n, int T_, int H, int dk, int dv) {
+    for (int idx = threadIdx.x; idx < C * dk; idx += blockDim.x) {
+        int t = idx / dk, j = idx - t * dk;
+        float v = 0.0f;
+        if (t < n) {
+            const uint32_t l = reinterpret_cast<const uint16_t *>(lo)[tok(b, c0 + t, h, T_, H, dk) + j];
+            const uint32_t u = reinterpret_cast<const uint16_t *>(hi)[tok(b, c0 + t, h, T_, H, dv) + j];
+            v = __uint_as_float(l | (u << 16));
+        }
+        dst[t * ld + j] = v;
+    }
+}
+
 // log f -> (inclusive cumsum b in place, k = 1 - f in K).  One thread per key dim.
 static __device__ __forceinline__ void cumsum_gates(float *Bs, float *Ks, int ld, int C, int dk) {
     for (int j = threadIdx.x; j < dk; j += blockDim.x) {
@@ -150,7 +174,8 @@ template <typename T>
 __device__ __noinline__ void
 simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
-                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
+                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx,
+                   T *stash_lo = nullptr, T *stash_hi = nullptr) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Bs = sm;              // [C][ldk]
     float *Ks = Bs + C * ldk;    // [C][ldk]
@@ -189,7 +214,11 @@ simt_bwd_dq_body(const T *__restrict__ lf, const T *__restrict__ x, const float 
             float acc = expf(bt) * inter;
             for (int s = 0; s <= t; ++s)
                 acc = fmaf(As[t * ldc + s] * Ks[s * ldk + j], expf(bt - Bs[s * ldk + j]), acc);
-            if (t < n) dq[tok(b, c0 + t, h, T_, H, dk) + j] = from_f<T>(acc);
+            if (t < n) {
+                dq[tok(b, c0 + t, h, T_, H, dk) + j] = from_f<T>(acc);
+                if (sizeof(T) == 2 && stash_lo)
+                    stash_f32(stash_lo, stash_hi, tok(b, c0 + t, h, T_, H, dk) + j, tok(b, c0 + t, h, T_, H, dv) + j, acc);
+            }
         }
         __syncthreads();
         for (int idx = tid; idx < C * dk; idx += blockDim.x) {
@@ -225,7 +254,8 @@ __device__ __noinline__ void
 simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__restrict__ x,
                     const T *__restrict__ dO, const float *__restrict__ dhT, const T *__restrict__ dq,
                     const float *__restrict__ rs, T *__restrict__ dlf, T *__restrict__ dx,
-                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx) {
+                    float *__restrict__ dh0, int T_, int H, int dk, int dv, int C, float *sm, int b, int h, int sidx,
+                    bool dq_stashed = false) {
     const int ldk = dk + 1, ldv = dv + 1, ldc = C + 1;
     float *Qs = sm;               // [C][ldk] q, later q e^{b}
     float *Bs = Qs + C * ldk;     // [C][ldk] b
@@ -254,7 +284,8 @@ simt_bwd_rev_body(const T *__restrict__ q, const T *__restrict__ lf, const T *__
         __syncthreads();
         load_tile(Qs, ldk, q, b, h, c0, C, n, T_, H, dk);
         load_tile(Bs, ldk, lf, b, h, c0, C, n, T_, H, dk);
-        load_tile(Ds, ldk, dq, b, h, c0, C, n, T_, H, dk);
+        if (dq_stashed) load_stash(Ds, ldk, dlf, dx, b, h, c0, C, n, T_, H, dk, dv);   // fp32 dq
+        else load_tile(Ds, ldk, dq, b, h, c0, C, n, T_, H, dk);
         load_tile(Vs, ldv, x, b, h, c0, C, n, T_, H, dv);
         load_tile(Gs, ldv, dO, b, h, c0, C, n, T_, H, dv);
         __syncthreads();
@@ -376,13 +407,15 @@ template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_bwd_dq_kernel(const T *__restrict__ lf, const T *__restrict__ x, const float *__restrict__ h0,
                    const T *__restrict__ dO, const float *__restrict__ dhT, T *__restrict__ dq,
-                   float *__restrict__ rs, int T_, int H, int dk, int dv, int C, const int *__restrict__ only,
-                   const int *__restrict__ cu, const int *__restrict__ perm) {
+                   float *__restrict__ rs, T *dlf, T *dx, int T_, int H, int dk, int dv, int C,
+                   const int *__restrict__ only, const int *__restrict__ cu, const int *__restrict__ perm) {
     if (only && only[blockIdx.x] == 0) return;
     extern __shared__ float sm[];
     const SeqView v = seq_view(cu, perm, blockIdx.x, H, T_);
     const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
-    simt_bwd_dq_body<T>(lf + ok, x + ov, h0, dO + ov, dhT, dq + ok, rs, v.T, H, dk, dv, C, sm, v.b, v.h, v.sidx);
+    const bool st = sizeof(T) == 2 && dv >= dk && dlf;
+    simt_bwd_dq_body<T>(lf + ok, x + ov, h0, dO + ov, dhT, dq + ok, rs, v.T, H, dk, dv, C, sm, v.b, v.h, v.sidx,
+                        st ? dlf + ok : nullptr, st ? dx + ov : nullptr);
 }
 
 template <typename T>
@@ -397,7 +430,7 @@ simt_bwd_rev_kernel(const T *__restrict__ q, const T *__restrict__ lf, const T *
     const SeqView v = seq_view(cu, perm, blockIdx.x, H, T_);
     const size_t ok = v.tok0 * H * dk, ov = v.tok0 * H * dv;
     simt_bwd_rev_body<T>(q + ok, lf + ok, x + ov, dO + ov, dhT, dq + ok, rs, dlf + ok, dx + ov, dh0, v.T, H, dk, dv, C,
-                         sm, v.b, v.h, v.sidx);
+                         sm, v.b, v.h, v.sidx, sizeof(T) == 2 && dv >= dk);
 }
 
 // ------------------------------------------------------------------ launchers
@@ -426,7 +459,8 @@ static cudaError_t launch_simt_bwd_t(const SimtBwdArgs &a, cudaStream_t st) {
     e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
     if (e != cudaSuccess) return e;
     k1<<<a.B * a.H, kSimtThreads, s1, st>>>((const T *)a.lf, (const T *)a.x, a.h0, (const T *)a.dO,
-                                            a.dhT, (T *)a.dq, a.rs, a.T, a.H, a.dk, a.dv, a.C, a.only, a.cu, a.perm);
+                                            a.dhT, (T *)a.dq, a.rs, (T *)a.dlf, (T *)a.dx, a.T, a.H, a.dk, a.dv,
+                                            a.C, a.only, a.cu, a.perm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k2<<<a.B * a.H, kSimtThreads, s2, st>>>((const T *)a.q, (const T *)a.lf, (const T *)a.x,

@@ -424,10 +424,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUt
         __syncthreads();
         float *sm = reinterpret_cast<float *>(smem);
         simt_bwd_dq_body<__nv_bfloat16>(p.lf, p.x, p.h0, p.dO, p.dhT, p.dq, p.rs, p.T, p.H, 128, 128,
-                                        p.simt_chunk, sm, b, h, bh);
+                                        p.simt_chunk, sm, b, h, bh, p.dlf, p.dx);
         __syncthreads();
         simt_bwd_rev_body<__nv_bfloat16>(p.q, p.lf, p.x, p.dO, p.dhT, p.dq, p.rs, p.dlf, p.dx, p.dh0, p.T, p.H,
-                                         128, 128, p.simt_chunk, sm, b, h, bh);
+                                         128, 128, p.simt_chunk, sm, b, h, bh, true);
     }
 }
 
@@ -548,11 +548,11 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             const int Tl = kPacked ? len : p.T;
             if constexpr (!kWide) {
                 simt_bwd_dq_body<__nv_bfloat16>(p.lf + ok, p.x + ok, p.h0, p.dO + ok, p.dhT, p.dq + ok, p.rs, Tl, p.H,
-                                                p.D, p.D, p.simt_chunk, sm, b, h, bh);
+                                                p.D, p.D, p.simt_chunk, sm, b, h, bh, p.dlf + ok, p.dx + ok);
                 __syncthreads();
                 simt_bwd_rev_body<__nv_bfloat16>(p.q + ok, p.lf + ok, p.x + ok, p.dO + ok, p.dhT, p.dq + ok, p.rs,
                                                  p.dlf + ok, p.dx + ok, p.dh0, Tl, p.H, p.D, p.D, p.simt_chunk, sm,
-                                                 b, h, bh);
+                                                 b, h, bh, true);
             } else {
                 // heads read in place (nK = nV): every token tensor viewed with Hw nK half-heads of 128,
                 // indexed at the value-side half-head hv; key-side tensors shifted by hk - hv half-heads,
@@ -562,10 +562,10 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 const size_t part = (size_t)p.Bo * p.T * Hh * p.D;
                 __nv_bfloat16 *dq = p.dq + vc * part + ks, *dlf = p.dlf + vc * part + ks, *dx = p.dx + ka * part;
                 simt_bwd_dq_body<__nv_bfloat16>(p.lf + ks, p.x, p.h0, p.dO, p.dhT, dq, p.rs, p.T, Hh, p.D, p.D,
-                                                p.simt_chunk, sm, b, hv, bh);
+                                                p.simt_chunk, sm, b, hv, bh, dlf, dx);
                 __syncthreads();
                 simt_bwd_rev_body<__nv_bfloat16>(p.q + ks, p.lf + ks, p.x, p.dO, p.dhT, dq, p.rs, dlf, dx, p.dh0, p.T,
-                                                 Hh, p.D, p.D, p.simt_chunk, sm, b, hv, bh);
+                                                 Hh, p.D, p.D, p.simt_chunk, sm, b, hv, bh, true);
             }
             if (tid == 0) atomicAdd(&g_counters[0], 1ull);
         }

@@ -98,12 +98,17 @@ struct Params {
     int D;            // head size d_k = d_v: 128, or 64 (the second 64-column half of every operand
                       // tile is held at zero: log f = 0, q = i = 0 there, exactly neutral)
     const __nv_bfloat16 *lgs;   // scalar-decay variant: log g [B][T][H]; tm_lf then maps the key k
-    int *seg_done;    // with segments: [B*H] segments of the pair finished (zeroed by the aggregate kernel)
+    int *seg_done;    // with segments: [B*H] segments of the pair finished (zeroed before the launch)
     // Heads of width 256 read in place: head h of the call is block pair (a, c) of head
     // h / (nK nV) of the caller's [B][T][Hw][256] tensors, a = key block, c = value block.  Those
     // are read as [B][T][Hw nK][128] (q, log f: half-head Hw-index * nK + a) and [B][T][Hw nV][128]
     // (i: * nV + c); o is the key block's partial, [nK][B][T][Hw nV][128].  nK = nV = 1 otherwise.
     int nK, nV, Bo;   // Bo: the batch count of one o partial
+    // With segments, for the carried-state fix-up of segments k >= 1: bf16(q e^{b}) of the
+    // segment's first chunk ([B*H][nseg][128][128], b the cumulative log f from the chunk start)
+    // and that chunk's total log decay B ([B*H][nseg][128])
+    __nv_bfloat16 *qtil;
+    float *bseg;
 };
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
@@ -112,7 +117,10 @@ struct Params {
 // b_t = cumulative log g from the chunk start, rho = B / 2, Qt = q e^{b_t - rho}, Kt = k e^{rho - b_t}
 // (per-row factors), the state scales e^{B/2} for every state row.  A chunk with B / 2 < -kMaxRefLog
 // sends the pair to the exact CUDA-core forward (its flag also routes the backward).
-template <bool kPacked, bool kScalar = false>
+// kSeg: dense launches with sequence segments (the first chunk's q e^{b} and B are written for the
+// fix-up; the kernel lets its dependent launch early), compiled apart from the one-CTA-per-pair
+// instance.
+template <bool kPacked, bool kScalar = false, bool kSeg = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o,
@@ -124,6 +132,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     uint8_t *X = smem + 6 * kTileBytes;
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
+    if constexpr (kSeg) grid_dep_launch();   // the scan or fix-up may be scheduled now; it waits for this grid
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int bh = blockIdx.x / p.nseg;
     const int seg = blockIdx.x - bh * p.nseg, h = bh % p.H;
@@ -588,6 +597,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             b0 -= 0.5f * Bt0;
             b1 -= 0.5f * Bt1;
             float E0 = __expf(b0), E1 = __expf(b1);   // E = e^{b - rho} of the row before the range
+            // a later segment's first chunk: bf16(q e^{b}) and B, for the fix-up
+            uint32_t *qt_out = nullptr;
+            float er0 = 0.0f, er1 = 0.0f;
+            if (kSeg && n == 0 && seg > 0 && p.qtil) {
+                const size_t slot = (size_t)bh * p.nseg + seg;
+                qt_out = reinterpret_cast<uint32_t *>(p.qtil + slot * 16384 + col0);
+                er0 = __expf(0.5f * Bt0);
+                er1 = __expf(0.5f * Bt1);
+                if (rr == 0) {
+                    p.bseg[slot * 128 + col0] = Bt0;
+                    p.bseg[slot * 128 + col0 + 1] = Bt1;
+                }
+            }
 #pragma unroll 1
             for (int bt = 0; bt < 4; ++bt) {
                 const int t0 = 32 * rr + 8 * bt;
@@ -615,6 +637,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     *reinterpret_cast<uint32_t *>(Gb[s] + eoff(t0 + i)) = wa[i];
                 }
             }
+            if (qt_out) {   // q e^{b} = Qt e^{rho}, from this thread's Qt rows (rounded to bf16 twice)
+#pragma unroll 4
+                for (int i = 0; i < 32; ++i) {
+                    const int t = 32 * rr + i;
+                    const uint32_t w = *reinterpret_cast<const uint32_t *>(Qb[s] + eoff(t));
+                    qt_out[(size_t)t * 64] = pack_bf2(bf_lo(w) * er0, bf_hi(w) * er1);
+                }
+            }
             // b = B - rho = B / 2 now: the scale e^{B/2} of both state factors
             if (rr == 3 && !(b0 >= -kMaxRefLog && b1 >= -kMaxRefLog)) atomicMin(&m->bad_tile, n);   // also NaN
             fence_proxy_async_smem();
@@ -640,7 +670,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
     if (tid == 0) {
         if (p.nseg == 1) { if (p.flags) p.flags[bh] = fell_back ? 1 : 0; }   // sole writer
-        else if (fell_back) p.flags[bh] = 1;                  // zeroed by the aggregate kernel
+        else if (fell_back) p.flags[bh] = 1;                  // zeroed before the launch
         if (fell_back) atomicAdd(&g_counters[0], 1ull);
         else atomicAdd(&g_counters[1], (unsigned long long)N);
     }
@@ -884,26 +914,43 @@ agg_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CU
 // g is 0: h0 is inside its U).  In fp32, over the U slots: slot k-1 becomes the state entering
 // segment k; the sequence's final state goes to hT (and the saved final state).  Pairs the exact
 // route recomputed whole (flagged) are left alone.  One thread per 4 consecutive state elements
-// of one (batch, head).
+// of one (batch, head); the maps are loaded kScanBatch segments at a time, so that one memory
+// latency covers a batch rather than each segment.  Launched as a programmatic dependent of the segments' kernel.
+constexpr int kScanBatch = 16;
 __global__ void __launch_bounds__(256)
 scan_kernel(float *__restrict__ U, const float *__restrict__ g, int nseg, const int *__restrict__ flags,
             float *__restrict__ hT, float *__restrict__ hTs) {
+    grid_dep_launch();   // the fix-up may be scheduled now; it waits for this grid itself
+    grid_dep_wait();     // the segments' maps and flags are complete
     const int bh = blockIdx.x >> 4;
     if (flags[bh]) return;
     const int e = ((blockIdx.x & 15) * 256 + threadIdx.x) * 4;   // element offset in [0, 16384)
     const int jrow = e >> 7;
     float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sg = 0; sg < nseg; ++sg) {
-        const size_t slot = (size_t)bh * nseg + sg;
-        float4 *u = reinterpret_cast<float4 *>(U + slot * 16384 + e);
-        const float gj = g[slot * 128 + jrow];
-        const float4 uv = *u;
-        S = make_float4(fmaf(gj, S.x, uv.x), fmaf(gj, S.y, uv.y), fmaf(gj, S.z, uv.z), fmaf(gj, S.w, uv.w));
-        if (sg < nseg - 1) {
-            *u = S;
-        } else {
-            if (hT) *reinterpret_cast<float4 *>(hT + (size_t)bh * 16384 + e) = S;
-            if (hTs) *reinterpret_cast<float4 *>(hTs + (size_t)bh * 16384 + e) = S;
+    for (int s0 = 0; s0 < nseg; s0 += kScanBatch) {
+        float4 uv[kScanBatch];
+        float gj[kScanBatch];
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) {
+            if (s0 + i < nseg) {
+                const size_t slot = (size_t)bh * nseg + s0 + i;
+                uv[i] = *reinterpret_cast<const float4 *>(U + slot * 16384 + e);
+                gj[i] = g[slot * 128 + jrow];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) {
+            const int sg = s0 + i;
+            if (sg < nseg) {
+                S = make_float4(fmaf(gj[i], S.x, uv[i].x), fmaf(gj[i], S.y, uv[i].y), fmaf(gj[i], S.z, uv[i].z),
+                                fmaf(gj[i], S.w, uv[i].w));
+                if (sg < nseg - 1) {
+                    *reinterpret_cast<float4 *>(U + ((size_t)bh * nseg + sg) * 16384 + e) = S;
+                } else {
+                    if (hT) *reinterpret_cast<float4 *>(hT + (size_t)bh * 16384 + e) = S;
+                    if (hTs) *reinterpret_cast<float4 *>(hTs + (size_t)bh * 16384 + e) = S;
+                }
+            }
         }
     }
 }
@@ -914,49 +961,79 @@ scan_kernel(float *__restrict__ U, const float *__restrict__ g, int nseg, const 
 //   o_t += (q_t * e^{b_t})^T S_c,      S_{c+1} = Diag(e^{B_c}) S_c,      S_0 = S_in
 // (b_t the cumulative log decay from chunk c's start, B_c its total; every factor <= 1), and,
 // when the chunk states are kept for the backward, the chunk's saved bf16(e^{rho} S_in) lacks
-// e^{rho_c} S_c.  One CTA per segment walks its chunks from the start and stops once
-// max_j decay_j max_v |S_in[j,v]| < 2^-40: no term it could still add exceeds 128 |q| 2^-40 (the
-// outputs are bf16, 2^-8 relative).  Single-stage: per chunk, load q, log f, o (and the saved
-// state), form Qt = q e^{b} in place, one MMA O = Qt bf16(S_c) into TMEM, add it to o, correct
-// the saved state, scale the carried state; 8 warps, thread (row r, half) holds 64 columns of
-// row r of the carried state in registers.
+// e^{rho_c} S_c.  One CTA per segment walks its chunks from the start while
+// max_j decay_j max_v |S_c[j,v]| >= kFixStop (decay_j the carried decay of key dim j so far): a
+// term left out is below 128 |q| kFixStop, 2^-15 of the relative rounding of the bf16 copy of the
+// state that every inter-chunk product reads.  Per chunk: q e^{b} (the first chunk's from the
+// segments' kernel, later ones from q and log f), o (and the saved state) in; one MMA
+// O = (q e^{b}) bf16(S_c) into TMEM; o += O; the saved state corrected; the carried state scaled.
+// 8 warps; thread (row r, half) holds 64 columns of row r of the carried state in registers.
+// Without saved states two stages: the next chunk's tiles load while this one is on the tensor
+// cores and in the epilogue (the decision to walk it is taken from this chunk's e^{B}, before
+// they are requested).
+// S_in is the scan kernel's (slot k-1 of Sin), or, with few segments (merged), summed here from
+// the segments' maps: S_in = sum_{m<k} Diag(prod_{m<l<k} g_l) U_m; the last segment's CTA then
+// also writes hT = Diag(g_k) S_in + U_k.  A programmatic dependent of the kernel before it: only
+// its set-up runs before grid_dep_wait().
+constexpr float kFixStop = 0x1p-24f;
+
 struct FixMisc {
-    uint64_t full, barM;
+    uint64_t fullQG[2], fullO[2], barM;
     uint32_t tmem_base;
     int pad;
     float EB[128];        // e^{B} of the chunk, key dim
     float ER[128];        // e^{rho} = e^{B/2} of the chunk, key dim (the saved states' scale)
     float Ppart[3][128];  // per 32-row range sums of log f (ranges 0..2)
 };
-constexpr size_t kFixSmem = 5 * (size_t)kTileBytes + sizeof(FixMisc);
+// one stage (q, log f, o, saved state) + X, or two stages (q, log f, o) + X
+constexpr size_t fix_smem(bool save) { return (save ? 5 : 7) * (size_t)kTileBytes + sizeof(FixMisc); }
+constexpr int kMergedScanMax = 4;   // segments per pair up to which the fix-up sums S_in itself
 
 struct FixParams {
-    const float *Sin;   // [B*H][nseg][128][128]: slot k-1 = the state entering segment k (the scan)
+    const float *U;     // [B*H][nseg][128][128]: the segments' U, or (after the scan kernel) slot k-1 =
+                        // the state entering segment k
+    const float *g;     // [B*H][nseg][128]: the segments' decay products (merged)
+    const float *B0;    // [B*H][nseg][128]: each segment's first-chunk total log decay
     const int *flags;   // [B*H] nonzero: recomputed whole by the exact route (skipped)
+    float *hT, *hTs;    // merged: the final state (either may be null)
     int H, nseg, tps, ntiles;
     bool save;          // saved bf16 chunk states (slot bh * ntiles + chunk) to correct
+    bool merged;        // S_in summed here (else read from the scan's slots)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
 fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
-             const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_st, FixParams p) {
+             const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_st,
+             const __grid_constant__ CUtensorMap tm_qt, FixParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t *Qb = smem, *Gb = smem + kTileBytes, *Ob = smem + 2 * kTileBytes, *Sb = smem + 3 * kTileBytes;
-    uint8_t *X = smem + 4 * kTileBytes;
-    FixMisc *m = reinterpret_cast<FixMisc *>(smem + 5 * kTileBytes);
+    const int NS = p.save ? 1 : 2;   // stages
+    // stage s: q, log f, o at smem + 3 s tiles (s = 0 with one stage)
+    auto Qb = [&](int s) { return smem + (size_t)s * 3 * kTileBytes; };
+    auto Gb = [&](int s) { return smem + ((size_t)s * 3 + 1) * kTileBytes; };
+    auto Ob = [&](int s) { return smem + ((size_t)s * 3 + 2) * kTileBytes; };
+    uint8_t *Sb = smem + 3 * kTileBytes;                              // one stage only
+    uint8_t *X = smem + (NS == 2 ? 6 : 4) * kTileBytes;
+    FixMisc *m = reinterpret_cast<FixMisc *>(smem + (NS == 2 ? 7 : 5) * kTileBytes);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nfix = p.nseg - 1;
     const int bh = blockIdx.x / nfix, seg = 1 + blockIdx.x - bh * nfix, b = bh / p.H, h = bh - b * p.H;
-    if (p.flags[bh]) return;
     const int g0 = seg * p.tps, N = min(p.ntiles - g0, p.tps);
+    const size_t myslot = (size_t)bh * p.nseg + seg;
     if (smem_u32(smem) & 1023u) {
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
     }
     if (tid == 0) {
-        mbar_init(&m->full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&m->fullQG[s], 1);
+            mbar_init(&m->fullO[s], 1);
+        }
         mbar_init(&m->barM, 1);
         fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_lf);
+        tma_prefetch_desc(&tm_o);
+        tma_prefetch_desc(&tm_qt);
     }
     if (warp == 0) {
         tmem_alloc(&m->tmem_base, 128);
@@ -968,42 +1045,159 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t tbase = m->tmem_base;
     const int quad = warp & 3, ch = warp >> 2, r = 32 * quad + lane;   // carried-state row / token row r
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
-    // the carried state, row r, columns 64 ch .. 64 ch + 63
-    float S[64];
-    float smax = 0.0f;
-    {
-        const float4 *src = reinterpret_cast<const float4 *>(p.Sin + ((size_t)bh * p.nseg + seg - 1) * 16384 +
-                                                             (size_t)r * 128 + 64 * ch);
+    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
+    const int pc = tid & 63, rr = tid >> 6, col0 = 2 * pc;   // prep: column pair, 32-row range
+    const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
+    auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+    // loads issued (thread 0) and waited for (every thread), per barrier kind, counted in chunks
+    int issued_qg = 0, issued_o = 0, waited_qg = 0, waited_o = 0;
+    auto load_qg = [&](int c) {   // thread 0; the first chunk: q e^{b} into the q tile
+        const int s = NS == 2 ? (c & 1) : 0, tok = (g0 + c) * kTile;
+        mbar_arrive_expect_tx(&m->fullQG[s], (c == 0 ? 1 : 2) * kTileBytes);
+        for (int k = 0; k < 2; ++k) {
+            if (c == 0) {
+                tma_load_4d(Qb(s) + k * kBlk, &tm_qt, &m->fullQG[s], 64 * k, 0, 0, (int)myslot);
+            } else {
+                tma_load_4d(Qb(s) + k * kBlk, &tm_q, &m->fullQG[s], 64 * k, h, tok, b);
+                tma_load_4d(Gb(s) + k * kBlk, &tm_lf, &m->fullQG[s], 64 * k, h, tok, b);
+            }
+        }
+        ++issued_qg;
+    };
+    auto load_o = [&](int c) {    // thread 0
+        const int s = NS == 2 ? (c & 1) : 0, tok = (g0 + c) * kTile, slot = bh * p.ntiles + g0 + c;
+        mbar_arrive_expect_tx(&m->fullO[s], (p.save ? 2 : 1) * kTileBytes);
+        for (int k = 0; k < 2; ++k) {
+            tma_load_4d(Ob(s) + k * kBlk, &tm_o, &m->fullO[s], 64 * k, h, tok, b);
+            if (p.save) tma_load_4d(Sb + k * kBlk, &tm_st, &m->fullO[s], 64 * k, 0, 0, slot);
+        }
+        ++issued_o;
+    };
+    // prep of stage s (chunks after the first): b = cumulative log f from the chunk start;
+    // Qt = q e^{b} in place; e^{B} and e^{B/2}, B summed as the forward's prep sums it
+    // (((P0 + P1) + P2) + P3, Pk the 32-row range totals)
+    auto prep = [&](int s) {
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb(s) + eoff(32 * rr + i));
+            s0 += bf_lo(w);
+            s1 += bf_hi(w);
+        }
+        if (rr < 3) {
+            m->Ppart[rr][col0] = s0;
+            m->Ppart[rr][col0 + 1] = s1;
+        }
+        __syncthreads();
+        float b0 = 0.0f, b1 = 0.0f;
+        for (int r2 = 0; r2 < rr; ++r2) {
+            b0 += m->Ppart[r2][col0];
+            b1 += m->Ppart[r2][col0 + 1];
+        }
+        if (rr == 3) {
+            const float B0 = b0 + s0, B1 = b1 + s1;
+            m->EB[col0] = __expf(B0);
+            m->EB[col0 + 1] = __expf(B1);
+            m->ER[col0] = __expf(0.5f * B0);
+            m->ER[col0 + 1] = __expf(0.5f * B1);
+        }
+        float E0 = __expf(b0), E1 = __expf(b1);
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const int t = 32 * rr + i;
+            const uint32_t wa = *reinterpret_cast<const uint32_t *>(Gb(s) + eoff(t));
+            uint32_t *wq = reinterpret_cast<uint32_t *>(Qb(s) + eoff(t));
+            E0 *= __expf(bf_lo(wa));
+            E1 *= __expf(bf_hi(wa));
+            *wq = pack_bf2(bf_lo(*wq) * E0, bf_hi(*wq) * E1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();   // Qt, e^{B}, e^{B/2} complete
+    };
+
+    grid_dep_wait();   // the segments' outputs (and the scan's) are complete from here on
+    bool ok = true, go = false;
+    float S[64];          // the carried state, row r, columns 64 ch .. 64 ch + 63
+    float smax = 0.0f;    // max |S| of the row's 64 columns as entered
+    float decay = 1.0f;   // the carried decay of row r so far
+    // the entering state (loaded before the flag is known; unused for a flagged pair)
+    const size_t rowoff = (size_t)r * 128 + 64 * ch;
+    auto slot_row = [&](int sg) {
+        return reinterpret_cast<const float4 *>(p.U + ((size_t)bh * p.nseg + sg) * 16384 + rowoff);
+    };
+    if (p.merged) {   // S_in = sum over the earlier segments' maps, two segments per round of loads
+#pragma unroll
+        for (int i = 0; i < 64; ++i) S[i] = 0.0f;
+        int mseg = 0;
+        for (; mseg + 1 < seg; mseg += 2) {
+            const float ga = p.g[((size_t)bh * p.nseg + mseg) * 128 + r];
+            const float gb = p.g[((size_t)bh * p.nseg + mseg + 1) * 128 + r];
+            const float4 *ua = slot_row(mseg), *ub = slot_row(mseg + 1);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float4 a = ua[i], c2 = ub[i];
+                S[4 * i] = fmaf(gb, fmaf(ga, S[4 * i], a.x), c2.x);
+                S[4 * i + 1] = fmaf(gb, fmaf(ga, S[4 * i + 1], a.y), c2.y);
+                S[4 * i + 2] = fmaf(gb, fmaf(ga, S[4 * i + 2], a.z), c2.z);
+                S[4 * i + 3] = fmaf(gb, fmaf(ga, S[4 * i + 3], a.w), c2.w);
+            }
+        }
+        if (mseg < seg) {
+            const float ga = p.g[((size_t)bh * p.nseg + mseg) * 128 + r];
+            const float4 *ua = slot_row(mseg);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float4 a = ua[i];
+                S[4 * i] = fmaf(ga, S[4 * i], a.x);
+                S[4 * i + 1] = fmaf(ga, S[4 * i + 1], a.y);
+                S[4 * i + 2] = fmaf(ga, S[4 * i + 2], a.z);
+                S[4 * i + 3] = fmaf(ga, S[4 * i + 3], a.w);
+            }
+        }
+    } else {
+        const float4 *src = slot_row(seg - 1);   // the scan's slot k-1
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float4 a = src[i];
             S[4 * i] = a.x; S[4 * i + 1] = a.y; S[4 * i + 2] = a.z; S[4 * i + 3] = a.w;
         }
-#pragma unroll
-        for (int i = 0; i < 64; ++i) smax = fmaxf(smax, fabsf(S[i]));
     }
-    float decay = 1.0f;   // the carried decay of row r so far
-    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
-    const int pc = tid & 63, rr = tid >> 6, col0 = 2 * pc;   // prep: column pair, 32-row range
-    const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
-    auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
-    int issued = 0, waited = 0;
-    bool ok = true;
-    for (int c = 0; c < N; ++c) {
-        // stop once nothing the carried state could still add is above 2^-40
-        if (!__syncthreads_or(decay * smax >= 0x1p-40f)) break;
-        const int tok = (g0 + c) * kTile, slot = bh * p.ntiles + g0 + c;
-        if (tid == 0) {
-            tma_store_wait_read0();   // the previous chunk's stores have read Ob, Sb
-            ++issued;
-            mbar_arrive_expect_tx(&m->full, (p.save ? 4 : 3) * kTileBytes);
-            for (int k = 0; k < 2; ++k) {
-                tma_load_4d(Qb + k * kBlk, &tm_q, &m->full, 64 * k, h, tok, b);
-                tma_load_4d(Gb + k * kBlk, &tm_lf, &m->full, 64 * k, h, tok, b);
-                tma_load_4d(Ob + k * kBlk, &tm_o, &m->full, 64 * k, h, tok, b);
-                if (p.save) tma_load_4d(Sb + k * kBlk, &tm_st, &m->full, 64 * k, 0, 0, slot);
+    if (!p.flags[bh]) {
+        if (tid == 0) {   // the first chunk's tiles
+            fence_proxy_async_global();
+            load_qg(0);
+            load_o(0);
+        }
+        if (tid < 128) {  // the first chunk's e^{B}, e^{B/2}
+            const float B = p.B0[myslot * 128 + tid];
+            m->EB[tid] = __expf(B);
+            m->ER[tid] = __expf(0.5f * B);
+        }
+        if (p.merged && seg == p.nseg - 1 && (p.hT || p.hTs)) {   // the sequence's final state
+            const float gk = p.g[myslot * 128 + r];
+            const float4 *src = slot_row(seg);
+            float4 *d1 = p.hT ? reinterpret_cast<float4 *>(p.hT + (size_t)bh * 16384 + rowoff) : nullptr;
+            float4 *d2 = p.hTs ? reinterpret_cast<float4 *>(p.hTs + (size_t)bh * 16384 + rowoff) : nullptr;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float4 a = src[i];
+                const float4 w = make_float4(fmaf(gk, S[4 * i], a.x), fmaf(gk, S[4 * i + 1], a.y),
+                                             fmaf(gk, S[4 * i + 2], a.z), fmaf(gk, S[4 * i + 3], a.w));
+                if (d1) d1[i] = w;
+                if (d2) d2[i] = w;
             }
         }
+#pragma unroll
+        for (int i = 0; i < 64; ++i) smax = fmaxf(smax, fabsf(S[i]));
+        go = __syncthreads_or(smax >= kFixStop);
+    }
+    for (int c = 0; go && c < N; ++c) {
+        const int s = NS == 2 ? (c & 1) : 0, par = (c / NS) & 1;
+        const int tok = (g0 + c) * kTile, slot = bh * p.ntiles + g0 + c;
+        if (__syncthreads_or(!mbar_wait(&m->fullQG[s], par))) { ok = false; break; }
+        waited_qg = c + 1;
+        if (c > 0) prep(s);   // the first chunk's q e^{b} came ready-made
         // bf16(S_c) -> X, the MN-major B operand (row r = key dim, columns = value dims)
         {
             float v[32];
@@ -1014,53 +1208,13 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 store_chunk_bf16(X, r, 2 * ch + hh, v);
             }
         }
-        if (__syncthreads_or(!mbar_wait(&m->full, c & 1))) { ok = false; break; }
-        waited = issued;
-        // prep: b = cumulative log f from the chunk start; Qt = q e^{b} in place; e^{B}, e^{B/2}
-        {
-            float s0 = 0.0f, s1 = 0.0f;
-            if (rr < 3) {
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t *>(Gb + eoff(32 * rr + i));
-                    s0 += bf_lo(w);
-                    s1 += bf_hi(w);
-                }
-                m->Ppart[rr][col0] = s0;
-                m->Ppart[rr][col0 + 1] = s1;
-            }
-            __syncthreads();
-            float b0 = 0.0f, b1 = 0.0f;
-            for (int r2 = 0; r2 < rr; ++r2) {
-                b0 += m->Ppart[r2][col0];
-                b1 += m->Ppart[r2][col0 + 1];
-            }
-            float E0 = __expf(b0), E1 = __expf(b1);
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) {
-                const int t = 32 * rr + i;
-                const uint32_t wa = *reinterpret_cast<const uint32_t *>(Gb + eoff(t));
-                uint32_t *wq = reinterpret_cast<uint32_t *>(Qb + eoff(t));
-                b0 += bf_lo(wa);
-                b1 += bf_hi(wa);
-                E0 *= __expf(bf_lo(wa));
-                E1 *= __expf(bf_hi(wa));
-                *wq = pack_bf2(bf_lo(*wq) * E0, bf_hi(*wq) * E1);
-            }
-            if (rr == 3) {   // b = the chunk total B now (summed as the forward's prep sums it: the
-                             // three ranges' totals, then this range's rows)
-                m->EB[col0] = __expf(b0);
-                m->EB[col0 + 1] = __expf(b1);
-                m->ER[col0] = __expf(0.5f * b0);
-                m->ER[col0 + 1] = __expf(0.5f * b1);
-            }
-        }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        // whether the carried state still matters after this chunk
+        const bool next = __syncthreads_or(decay * m->EB[r] * smax >= kFixStop) && c + 1 < N;
         if (tid == 0) {   // O = Qt bf16(S_c): M = tokens, N = value dims, K = key dims
             tc_fence_after();
-            const uint64_t dQ = sdesc_sw128(smem_u32(Qb), 16, 1024);
+            const uint64_t dQ = sdesc_sw128(smem_u32(Qb(s)), 16, 1024);
             const uint64_t dXm = sdesc_sw128(smem_u32(X), kBlk, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -1068,7 +1222,15 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mma_bf16_ss(tbase, sdesc_add(dQ, ko), sdesc_add(dXm, kk * 2048), id_kmn, kk > 0);
             }
             mma_commit(&m->barM);
+            if (next && NS == 2) {   // the other stage: chunk c-1's MMA is complete, its stores read
+                tma_store_wait_read0();
+                load_qg(c + 1);
+                load_o(c + 1);
+            }
         }
+        if (__syncthreads_or(!mbar_wait(&m->fullO[s], par) || !mbar_wait(&m->barM, c & 1))) { ok = false; break; }
+        waited_o = c + 1;
+        tc_fence_after();
         // the saved state of this chunk, row r (key dim): + e^{rho} S_c
         if (p.save) {
             const float er = m->ER[r];
@@ -1090,8 +1252,6 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 store_chunk_bf16(Sb, r, cc, v);
             }
         }
-        if (__syncthreads_or(!mbar_wait(&m->barM, c & 1))) { ok = false; break; }
-        tc_fence_after();
         // o row r (token) += O row r
         {
             float v[32];
@@ -1100,7 +1260,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const int cc = 2 * ch + hh;
                 tmem_ld32(tl + 32 * cc, v);
                 tmem_wait_ld();
-                uint8_t *base = Ob + (cc >> 1) * kBlk + r * 128;
+                uint8_t *base = Ob(s) + (cc >> 1) * kBlk + r * 128;
 #pragma unroll
                 for (int qd = 0; qd < 4; ++qd) {
                     const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
@@ -1111,7 +1271,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         v[8 * qd + 2 * k + 1] += bf_hi(ws[k]);
                     }
                 }
-                store_chunk_bf16(Ob, r, cc, v);
+                store_chunk_bf16(Ob(s), r, cc, v);
             }
         }
         // the carried state to the next chunk
@@ -1124,17 +1284,26 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         __syncthreads();
         if (tid == 0) {
             for (int k = 0; k < 2; ++k) {
-                tma_store_4d(&tm_o, Ob + k * kBlk, 64 * k, h, tok, b);
+                tma_store_4d(&tm_o, Ob(s) + k * kBlk, 64 * k, h, tok, b);
                 if (p.save) tma_store_4d(&tm_st, Sb + k * kBlk, 64 * k, 0, 0, slot);
             }
             tma_store_commit();
+            if (next && NS == 1) {   // the single stage, once this chunk's stores have read it
+                tma_store_wait_read0();
+                load_qg(c + 1);
+                load_o(c + 1);
+            }
         }
+        go = next;
     }
-    if (!ok && tid == 0) {
-        set_status(HGRN2_ERR_TIMEOUT);
-        for (int k = waited; k < issued; ++k) mbar_wait(&m->full, k & 1, 2000000u);
+    if (tid == 0) {
+        if (!ok) set_status(HGRN2_ERR_TIMEOUT);
+        // loads still in flight: the first chunk's when the carried state was negligible, or
+        // any after a timeout
+        for (int k = waited_qg; k < issued_qg; ++k) mbar_wait(&m->fullQG[NS == 2 ? (k & 1) : 0], (k / NS) & 1, 2000000u);
+        for (int k = waited_o; k < issued_o; ++k) mbar_wait(&m->fullO[NS == 2 ? (k & 1) : 0], (k / NS) & 1, 2000000u);
+        tma_store_wait_all0();
     }
-    if (tid == 0) tma_store_wait_all0();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1146,7 +1315,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 // ------------------------------------------------------------------ host side
 static_assert(tcf::kSmemBytes <= 227 * 1024, "forward shared memory");
 static_assert(tcf::kAggSmem <= 227 * 1024, "aggregate shared memory");
-static_assert(tcf::kFixSmem <= 227 * 1024, "fix-up shared memory");
+static_assert(tcf::fix_smem(false) <= 227 * 1024 && tcf::fix_smem(true) <= 227 * 1024, "fix-up shared memory");
 static_assert(sd::fwd_smem(128, 128) <= tcf::kSmemBytes, "scalar-decay exact forward inside the forward kernel");
 
 // Segments per (b,h): enough CTAs to cover the 148 SMs of a B200 once, at most one per chunk.
@@ -1165,11 +1334,16 @@ size_t tc_fwd_workspace(int B, int T, int H) {
     int nseg, tps;
     tc_fwd_segments(B, T, H, &nseg, &tps);
     if (nseg <= 1) return 0;
-    // (U, g) of every segment, then the per-pair finished-segment counts
-    return (size_t)B * H * nseg * (16384 + 128) * sizeof(float) + (size_t)B * H * sizeof(int);
+    // per segment: U, g, the first chunk's B (fp32) and q e^{b} (bf16); then the per-pair
+    // finished-segment counts
+    return (size_t)B * H * nseg * ((16384 + 2 * 128) * sizeof(float) + 16384 * sizeof(__nv_bfloat16)) +
+           (size_t)B * H * sizeof(int);
 }
 
 size_t tc_fwd_smem() { return tcf::kSmemBytes; }
+
+// segments, then the fix-up, with the scan between them beyond kMergedScanMax segments
+int tc_fwd_launches(int nseg) { return nseg <= 1 ? 1 : nseg <= tcf::kMergedScanMax ? 2 : 3; }
 
 // Slots of the saved bf16 chunk states: [B*H*ntiles] (slot bh * ntiles + n), or for packed
 // sequences [(T / 128 + nseq) * H] (slot ((cu[s] / 128) + s + n) * H + h: sequence s's chunks
@@ -1191,6 +1365,24 @@ cudaError_t launch_tc_state_map(const void *lf, const void *x, int B, int T, int
     return cudaGetLastError();
 }
 
+// Launches a kernel as a programmatic dependent of the previous work in the stream: it may be
+// scheduled before that work completes, and waits for it with grid_dep_wait().
+template <typename... Exp, typename... Act>
+static cudaError_t launch_dependent(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                    Act &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
+
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     const bool packed = a.cu != nullptr;   // a.B is then the number of sequences
     const int Bm = packed ? 1 : a.B;
@@ -1207,15 +1399,22 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     if (!a.st16) mst = mo;   // unused
     const bool scalar = a.lgs != nullptr;   // the scalar-decay variant (a.lf is then the key k)
-    auto kern = packed ? tcf::fwd_kernel<true> : scalar ? tcf::fwd_kernel<false, true> : tcf::fwd_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kSmemBytes);
-    if (e != cudaSuccess) return e;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     int nseg = 1, tps = ntiles;
     if (!packed && !scalar && !inplace && a.D == 128) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);   // else one CTA per (b,h)
+    auto kern = packed ? tcf::fwd_kernel<true>
+                : scalar ? tcf::fwd_kernel<false, true>
+                : nseg > 1 ? tcf::fwd_kernel<false, false, true>
+                : tcf::fwd_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kSmemBytes);
+    if (e != cudaSuccess) return e;
     const int BH = a.B * a.H;
-    float *U = a.seg_ws, *g = a.seg_ws ? a.seg_ws + (size_t)BH * nseg * 16384 : nullptr;
-    int *seg_done = a.seg_ws ? reinterpret_cast<int *>(g + (size_t)BH * nseg * 128) : nullptr;
+    // segment workspace: U [BH][nseg][128][128], g and the first chunk's B [BH][nseg][128] (fp32),
+    // the first chunk's q e^{b} [BH][nseg][128][128] (bf16), the finished-segment counts [BH]
+    const size_t nsl = (size_t)BH * nseg;
+    float *U = a.seg_ws, *g = a.seg_ws ? U + nsl * 16384 : nullptr, *bs = a.seg_ws ? g + nsl * 128 : nullptr;
+    __nv_bfloat16 *qtil = a.seg_ws ? reinterpret_cast<__nv_bfloat16 *>(bs + nsl * 128) : nullptr;
+    int *seg_done = a.seg_ws ? reinterpret_cast<int *>(qtil + nsl * 16384) : nullptr;
     if (nseg > 1) {
         // pass 1 only raises the exact-route flags and counts finished segments: both start at zero
         if (!a.seg_ws || !a.flags) return cudaErrorInvalidValue;
@@ -1225,16 +1424,30 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     tcf::Params p{a.h0, a.hT, (__nv_bfloat16 *)a.o, (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf,
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, g, a.T, a.H, ntiles, nseg, tps,
                   a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D,
-                  (const __nv_bfloat16 *)a.lgs, seg_done, a.nK, a.nV, Bm};
+                  (const __nv_bfloat16 *)a.lgs, seg_done, a.nK, a.nV, Bm,
+                  nseg > 1 ? qtil : nullptr, nseg > 1 ? bs : nullptr};
     kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     if ((e = cudaGetLastError()) != cudaSuccess || nseg == 1) return e;
-    // segments: the states entering them (and hT), then the carried states' contributions
-    tcf::scan_kernel<<<BH * 16, 256, 0, st>>>(U, g, nseg, a.flags, a.hT, a.st16 ? a.hTs : nullptr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tcf::fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kFixSmem);
+    // segments: the states entering them (and hT), then the carried states' contributions.  With
+    // few segments the fix-up sums the states itself; else the scan kernel chains them first.
+    // Each launch is a programmatic dependent of the one before it, so that its start-up overlaps
+    // that kernel's end.
+    const bool merged = nseg <= tcf::kMergedScanMax;
+    if (!merged) {
+        e = launch_dependent(tcf::scan_kernel, dim3(BH * 16), dim3(256), 0, st, U, (const float *)g, nseg,
+                             (const int *)a.flags, a.hT, a.st16 ? a.hTs : nullptr);
+        if (e != cudaSuccess) return e;
+    }
+    CUtensorMap mqt;   // the first chunks' q e^{b}: 128-row tiles, one per segment slot
+    if (!make_token_map(&mqt, qtil, (int)nsl, 128, 1)) return cudaErrorInvalidValue;
+    const size_t fsm = tcf::fix_smem(a.st16 != nullptr);
+    e = cudaFuncSetAttribute(tcf::fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
     if (e != cudaSuccess) return e;
-    tcf::FixParams fp{U, a.flags, a.H, nseg, tps, ntiles, a.st16 != nullptr};
-    tcf::fixup_kernel<<<BH * (nseg - 1), tcf::kThreads, tcf::kFixSmem, st>>>(mq, ml, mo, mst, fp);
+    tcf::FixParams fp{U, g, bs, a.flags, merged ? a.hT : nullptr, merged && a.st16 ? a.hTs : nullptr,
+                      a.H, nseg, tps, ntiles, a.st16 != nullptr, merged};
+    e = launch_dependent(tcf::fixup_kernel, dim3(BH * (nseg - 1)), dim3(tcf::kThreads), fsm, st, mq, ml, mo, mst,
+                         mqt, fp);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

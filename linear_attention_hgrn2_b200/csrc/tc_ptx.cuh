@@ -108,6 +108,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // Orders this thread's bulk-async (TMA) global accesses with its later generic-proxy accesses.
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched as a programmatic dependent of the one before it in the stream may start
+// while that one still runs.  grid_dep_wait() returns once every earlier grid it depends on has
+// completed and its memory operations are visible; nothing those grids write may be read before
+// it.  grid_dep_launch() lets the dependent grid be scheduled as soon as every CTA of this grid
+// has executed it (without it, as the CTAs exit).  Both are no-ops for a normal launch.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),

@@ -288,7 +288,9 @@ def test_autograd_function_uses_saved_states(cuda):
     loss = (o.float() * g["dO"].float()).sum() + (hT * g["dhT"]).sum()
     loss.backward()
     c = L.counters(reset=True)
-    assert c[2] == 3 + 1, c   # segmented forward (3 launches) + one saved backward launch
+    # segmented forward (3 segments per pair: segments, then the fix-up that sums the entering states
+    # itself) + one saved backward launch
+    assert c[2] == 2 + 1, c
     ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True, dhT=inp["dhT"])
     for n, h in enumerate((0, 1)):
         for name, got in (("dq", q.grad[0, :, h]), ("dlog_f", lf.grad[0, :, h]), ("di", x.grad[0, :, h]),
@@ -320,7 +322,7 @@ def test_more_pairs_than_sms(cuda, saved):
 
 @pytest.mark.parametrize("saved", [False, True], ids=["plain", "saved"])
 def test_segmented_forward_with_a_flagged_pair(cuda, saved):
-    # B*H = 2: the forward runs in sequence segments (aggregate, scan, segments: 3 launches).  Head 1
+    # B*H = 2: the forward runs in 8 sequence segments (segments, scan, fix-up: 3 launches).  Head 1
     # has gates shifted below the factorised range: its segments flag it, and the last of its
     # segments to finish recomputes the whole sequence on the exact route in the same launch
     B, T, H = 1, 1000, 2
@@ -349,9 +351,42 @@ def test_segmented_forward_with_a_flagged_pair(cuda, saved):
             assert e <= 2e-2, (name, h, e)
 
 
+@pytest.mark.parametrize("saved", [False, True], ids=["plain", "saved"])
+@pytest.mark.parametrize("lb", [0.9, 0.5])
+def test_segmented_forward_few_segments(cuda, saved, lb):
+    # B*H = 40: 3 segments of 3 chunks per pair (ragged T), so the fix-up sums the entering states
+    # itself and writes hT (2 launches).  At lb = 0.9 the carried state matters through whole
+    # segments (the fix-up walks every chunk of them, from one or two stages); at 0.5 for one chunk.
+    # Head 7 of batch 1 has gates below the factorised range and is recomputed on the exact route.
+    B, T, H = 2, 1000, 20
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, lb, seed=63, h0_sigma=0.1, with_dO=True,
+                        dhT_sigma=0.1)
+    strong = I.make_inputs(1, T, 1, 128, 128, torch.bfloat16, 0.0, seed=64, gate_shift=-1.0)
+    inp["log_f"][1, :, 7] = strong["log_f"][0, :, 0]
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"]) if saved else None
+    L.counters(reset=True)
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    c = L.counters(reset=True)
+    assert c[2] == 2 and c[0] >= 1, c
+    assert L.device_status() == L.OK
+    if saved:
+        dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
+                                 saved=sv)
+    pairs = [(0, 0), (0, 19), (1, 6), (1, 7), (1, 19)]
+    ref = oracle_heads(inp, pairs, want_bwd=saved, dhT=inp["dhT"])
+    for n, (b, h) in enumerate(pairs):
+        got = [("o", o[b, :, h]), ("hT", hT[b, h])]
+        if saved:
+            got += [("dq", dq[b, :, h]), ("dlog_f", dlf[b, :, h]), ("di", di[b, :, h]), ("dh0", dh0[b, h])]
+        for name, t in got:
+            e = err(np64(t), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, b, h, e)
+
+
 def test_saved_pair_long_segmented_sequence(cuda):
-    # B*H = 2: the forward cuts each sequence into up to 74 segments (aggregate, fp32 scan, then
-    # every segment from its incoming state) and saves the chunk states of all of them; the
+    # B*H = 2: the forward cuts each sequence into 32 one-chunk segments (segments from zero states,
+    # fp32 scan, carried-state fix-up) and saves the chunk states of all of them; the
     # backward walks all 32 chunks of each sequence from the saved states
     B, T, H = 1, 4096, 2
     inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.95, seed=41, h0_sigma=0.1, with_dO=True,
