@@ -334,6 +334,9 @@ def run_ours(args, world, rank, local):
     if not args.no_d256:
         from linear_attention_hgrn2_b200 import inputs as I
         out["head_dim_256"] = run_head_dim(args, dev, pk, rank, I.TRAIN_D256, 17)
+    if not args.no_long_train:
+        from linear_attention_hgrn2_b200 import inputs as I
+        out["long_sequence_train"] = run_head_dim(args, dev, pk, rank, I.TRAIN_LONG, 23)
     if not args.no_fwd_configs:
         out["forward_configs"] = run_fwd_configs(args, dev, pk, rank)
     if not args.no_scalar:
@@ -540,8 +543,9 @@ def run_varlen(args, dev, pk, rank):
 
 def run_head_dim(args, dev, pk, rank, w, seed_off, ref_ms=None):
     """The training pair on a variant of the training workload: 64-wide heads (B=8, H=32, T=2048),
-    256-wide heads (B=8, H=8, T=2048, run as 128-wide blocks), or the first layer's forget-gate
-    lower bound lb = 0 (the same shapes; with ref_ms, the headline step's time, for the ratio).
+    256-wide heads (B=8, H=8, T=2048, run as 128-wide blocks), the first layer's forget-gate
+    lower bound lb = 0 (the same shapes; with ref_ms, the headline step's time, for the ratio), or
+    the long sequence's shape (B=1, H=8, T=32768: 8 (b,h), both calls in sequence segments).
     Exact-route passes over the timed steps are counted on the device."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
@@ -823,6 +827,7 @@ def main():
     ap.add_argument("--no-lb0", action="store_true")
     ap.add_argument("--no-d256", action="store_true")
     ap.add_argument("--no-fwd-configs", action="store_true")
+    ap.add_argument("--no-long-train", action="store_true")
     ap.add_argument("--no-scalar", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -130,6 +130,7 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
                                     : wide_ws(B, T, H, dk, dv, chunk, dt, want_bwd, tc64, nullptr).total;
     size_t bytes = ws_bytes_base(B, H, dk, dv, dt, want_bwd);
     if (!want_bwd && use_tc(dk, dv, dt) && dk == 128 && T > 0) bytes += align256(tc_fwd_workspace(B, T, H));
+    if (want_bwd == 2 && use_tc(dk, dv, dt) && dk == 128 && T > 0) bytes += align256(tc_bwd_workspace(B, T, H));
     if (want_bwd && tc64 && use_tc(dk, dv, dt) && dk == 64 && T > 0)   // saved states + o scratch
         bytes += saved_layout(B, T, H).total + align256((size_t)B * T * H * dv * 2);
     return bytes;
@@ -255,7 +256,7 @@ size_t hgrn2_workspace_size(int B, int T, int H, int dk, int dv, int chunk, hgrn
                             int want_bwd) {
     if (check_common(B, T, H, dk, dv, chunk, dtype) != HGRN2_OK) return (size_t)-1;
     if (want_bwd < 0 || want_bwd > 2) return (size_t)-1;
-    return ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, want_bwd != 0, want_bwd != 2);
+    return ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, want_bwd, want_bwd != 2);
 }
 
 }  // extern "C"
@@ -345,7 +346,8 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return HGRN2_ERR_INVALID_ARG;
     if (cu && is_wide(dk, dv)) return HGRN2_ERR_UNSUPPORTED;
-    size_t need = cu ? ws_bytes_varlen(B, H, dk) : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, 1, tc64 && !saved);
+    size_t need = cu ? ws_bytes_varlen(B, H, dk)
+                     : ws_bytes_needed(B, T, H, dk, dv, chunk, dtype, saved ? 2 : 1, tc64 && !saved);
     if (ws_bytes < need || (need && !workspace)) return HGRN2_ERR_INVALID_ARG;
     if (is_wide(dk, dv))
         return (wide_uniform(dk, dv) ? stack_bwd : wide_bwd)(q, log_f, i, h0, saved, dO, dhT, dq, dlog_f, di, dh0, B,
@@ -387,11 +389,13 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
     // without saved states only d = 128 has a tensor-core backward (recompute); the rest take the
     // exact route
     if (use_tc(dk, dv, dtype) && (saved || (!cu && dk == 128))) {
-        if (saved) {   // one launch: reverse sweep from the saved states (exact route inside)
+        if (saved) {   // reverse sweep from the saved states (exact route inside); few (b,h): segments
             TcBwdArgs t{q, log_f, i, dO, h0, dhT, dq, dlog_f, di, dh0, rs,
                         (int *)((char *)saved + sl.flags), B, T, H, C, saved,
                         (const float *)((const char *)saved + sl.hTs), cu, perm, dk};
-            g_launches += 1;
+            const bool segs = !cu && dk == 128 && tc_bwd_workspace(B, T, H) > 0;
+            if (segs) t.seg_ws = (float *)((char *)workspace + ws_bytes_base(B, H, dk, dv, dtype, 1));
+            g_launches += segs ? tc_bwd_launches(B, T, H) : 1;
             return from_cuda(launch_tc_bwd(t, stream));
         }
         int *flags = (int *)((char *)workspace + align256(sizeof(float) * (size_t)B * H * dk));
@@ -498,7 +502,7 @@ hgrn2_status stack_bwd(const void *q, const void *log_f, const void *i, const fl
                        cudaStream_t stream, bool tc64) {
     const WideSplit s = wide_split(dk, dv);
     const int nK = s.n[0], nV = s.n[1], nb = nK * nV, kw = s.w[0][0], vw = s.w[1][0];
-    const WideStack w = wide_stack_ws(B, T, H, dk, dv, chunk, dtype, 1, tc64, (char *)workspace);
+    const WideStack w = wide_stack_ws(B, T, H, dk, dv, chunk, dtype, saved ? 2 : 1, tc64, (char *)workspace);
     const bool bf16 = dtype == HGRN2_BF16;
     const size_t es = bf16 ? 2 : 4, rows = (size_t)B * T * H, BH = (size_t)B * H, sm = (size_t)kw * vw;
     if (saved && wide_inplace(T, dk, dv, dtype)) {
@@ -629,7 +633,7 @@ hgrn2_status wide_bwd(const void *q, const void *log_f, const void *i, const flo
                       int T, int H, int dk, int dv, int chunk, hgrn2_dtype dtype, void *workspace,
                       cudaStream_t stream, bool tc64) {
     const WideSplit s = wide_split(dk, dv);
-    const WideWs w = wide_ws(B, T, H, dk, dv, chunk, dtype, 1, tc64, (char *)workspace);
+    const WideWs w = wide_ws(B, T, H, dk, dv, chunk, dtype, saved ? 2 : 1, tc64, (char *)workspace);
     size_t soff[2][2];
     wide_saved(B, T, H, dk, dv, dtype, soff);
     const bool bf16 = dtype == HGRN2_BF16;

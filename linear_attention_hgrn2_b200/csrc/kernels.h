@@ -70,6 +70,9 @@ struct TcBwdArgs {
     // 256-wide tensors; dq, dlf the value blocks' partials [nV][B][T][Hw][256]; dx the key blocks'
     // partials [nK][B][T][Hw][256].
     int nK = 1, nV = 1;
+    // saved states, dense d = 128, few (b,h): sequence segments' workspace, tc_bwd_workspace(B, T, H)
+    // bytes (null: one CTA per (b,h))
+    float *seg_ws = nullptr;
 };
 
 struct StepBwdArgs {
@@ -144,6 +147,10 @@ void tc_fwd_segments(int B, int T, int H, int *nseg, int *tps);
 size_t tc_fwd_workspace(int B, int T, int H);
 // Kernel launches of one segmented forward call with nseg segments per pair (1 without segments).
 int tc_fwd_launches(int nseg);
+// Sequence segments of the saved-state backward (dense, d = 128, bf16): workspace bytes (0: one
+// CTA per (b,h)) and kernel launches of one call.
+size_t tc_bwd_workspace(int B, int T, int H);
+int tc_bwd_launches(int B, int T, int H);
 size_t tc_bwd_smem();
 cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st);

@@ -492,6 +492,12 @@ struct RevParams {
     // the caller's tensors viewed as [B][T][2 Hw][128]; dq, d log f go to the value block's partial
     // ([nV][B][T][Hw][256]), di to the key block's ([nK][B][T][Hw][256]).  nK = nV = 1 otherwise.
     int nK, nV, Bo;
+    // Sequence segments (kSeg): [B*H][nseg] segments of tps chunks each; every segment's reverse
+    // sweep starts from a zero gradient (the last from dhT) and writes its backward map: W, the
+    // gradient it hands to the state entering it ([B*H][nseg][128][128]), and g, its decay product
+    // ([B*H][nseg][128])
+    int nseg, tps;
+    float *Wseg, *gseg;
 };
 
 // kPacked (saved mode only): p.cu holds packed sequences; compiled apart so the dense path
@@ -503,7 +509,9 @@ struct RevParams {
 // d log g_t.  Flagged pairs return at once; the host recomputes them on the exact route.
 // kWide (saved mode only): heads of width 256 read in place (p.nK = p.nV = 2), compiled apart so
 // that the other instances carry none of its head arithmetic.
-template <bool kSaved, bool kPacked, bool kScalar = false, bool kWide = false>
+// kSeg (saved mode, dense, per-dim): one CTA per sequence segment (p.nseg per pair); a flagged
+// pair is recomputed whole by its first segment's CTA.
+template <bool kSaved, bool kPacked, bool kScalar = false, bool kWide = false, bool kSeg = false>
 __global__ void __launch_bounds__(rsw::kRevThreads, 1)
 rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_do,
@@ -515,13 +523,24 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     uint8_t *D16 = smem + 4 * kTileBytes, *AT = smem + 5 * kTileBytes, *DA = smem + 6 * kTileBytes;
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
+    if constexpr (kSeg) grid_dep_launch();   // the scan may be scheduled now; it waits for this grid
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    int bh = blockIdx.x;
+    static_assert(!kSeg || (kSaved && !kPacked && !kScalar && !kWide), "segments: saved mode, dense, per-dim");
+    const int seg = kSeg ? (int)blockIdx.x % p.nseg : 0;
+    int bh = kSeg ? (int)blockIdx.x / p.nseg : (int)blockIdx.x;
     const int h = bh % p.H;
     // token of chunk n: tok0 + n * kTile of batch bc; saved-state slot: slot0 + n * sstride.
     // Packed sequences (saved mode only): rows from the sequence's end on (valid(n) < kTile)
     // are masked in the prep and not stored.
     int b = bh / p.H, bc = b, tok0 = 0, len = p.T, N = p.ntiles, slot0 = bh * p.ntiles, sstride = 1;
+    if (kSeg) {   // this segment's chunks
+        const int g0 = seg * p.tps;
+        N = min(p.ntiles - g0, p.tps);
+        tok0 = g0 * kTile;
+        slot0 += g0;
+    }
+    // the sequence's last segment starts from dhT (and the carry rowsum(dhT * hT)); others from zero
+    const bool from_dhT = !kSeg || seg == p.nseg - 1;
     static_assert(kSaved || !kPacked, "packed sequences need the saved states");
     if (kPacked) {
         const int sq = packed_seq(p.perm, bh / p.H, gridDim.x / p.H);
@@ -542,6 +561,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int hw = h / nbk, ka = (h - hw * nbk) / nV, vc = h - hw * nbk - ka * nV;
     const int hk = hw * nK + ka, hv = hw * nV + vc, kbc = vc * p.Bo + bc, vbc = ka * p.Bo + bc;
     if (p.flags[bh] != 0) {   // this (b,h) takes the exact route
+        if (kSeg && seg != 0) return;   // recomputed whole by the first segment's CTA
         if (kSaved && !kScalar) {   // both sweeps here (recompute mode: in the forward-sweep kernel)
             float *sm = reinterpret_cast<float *>(smem);
             const size_t ok = (size_t)tok0 * p.H * p.D;   // 0 unless packed sequences
@@ -629,7 +649,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
         float v[32];
         float part = 0.0f;   // saved mode: this quarter's share of rowsum(dhT * hT)
-        if (p.dhT && j < p.D && c0 < p.D) {   // d x d; zero outside for d = 64
+        if (from_dhT && p.dhT && j < p.D && c0 < p.D) {   // d x d; zero outside for d = 64
             const float4 *src = reinterpret_cast<const float4 *>(p.dhT + ((size_t)bh * p.D + j) * p.D + c0);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -656,7 +676,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             __syncthreads();
             if (q4 == 0) m->carry[j] = m->Bpart[0][j] + m->Bpart[1][j] + m->Bpart[2][j] + m->EB[j];
         } else if (q4 == 0) {
-            m->carry[j] = (p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
+            m->carry[j] = (from_dhT && p.dhT && p.rs) ? p.rs[(size_t)bh * 128 + j] : 0.0f;
         }
     }
 
@@ -672,6 +692,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     bool ok = true;
     int it = 0, n = N - 1;
     float g_later = 1.0f;   // e^{rho} of the chunk processed before this one (the later chunk), key dim j
+    float gprod = 1.0f;     // segments: the product of this segment's chunk decays e^{B}, key dim j
     for (; n >= 0; --n, ++it) {
         const uint32_t par = it & 1;
         if (__syncthreads_or(!mbar_wait(&m->barIn, par))) { ok = false; break; }
@@ -834,6 +855,7 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = (v[i] * g_later) * hh;
             g_later = hh;   // e^{rho} = e^{B - rho} of this chunk
+            if (kSeg) gprod = (gprod * hh) * hh;
             store_chunk_bf16(D16, j, q4, v);
             tmem_st32(tl + kColDS + c0, v);
             tmem_wait_st();
@@ -1104,13 +1126,16 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             for (int k = waited[q]; k < issued[q]; ++k) mbar_wait(bars[q], k & 1, 2000000u);
     }
     if (tid == kStoreTid) tma_store_wait_all0();
-    if (ok && n < 0 && p.dh0 && j < p.D && c0 < p.D) {   // warp-uniform
+    // dh0 (or, with segments, the segment's W; its g alongside)
+    float *dhout = kSeg ? p.Wseg + ((size_t)bh * p.nseg + seg) * 16384 : p.dh0 ? p.dh0 + (size_t)bh * p.D * p.D : nullptr;
+    if (kSeg && ok && n < 0 && q4 == 0) p.gseg[((size_t)bh * p.nseg + seg) * 128 + j] = gprod;
+    if (ok && n < 0 && dhout && j < p.D && c0 < p.D) {   // warp-uniform
         tc_fence_after();
         float v[32];
         tmem_ld32(tl + kColDS + c0, v);
         tmem_wait_ld();
         const float e = g_later;   // dh0 = Diag(e^{rho}) dL/dS_r of the first chunk
-        float4 *dst = reinterpret_cast<float4 *>(p.dh0 + ((size_t)bh * p.D + j) * p.D + c0);
+        float4 *dst = reinterpret_cast<float4 *>(dhout + (size_t)j * p.D + c0);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
@@ -1122,10 +1147,361 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (warp == 0) tmem_dealloc(tbase, kTmemCols);
 }
 
+// ------------------------------------------------------------------ backward segments
+// With segments, every segment's reverse sweep started from a zero gradient (the last from dhT):
+// W_k is the gradient it hands to the state entering it, g_k its decay product.  The gradient
+// carried into the last state of segment k from the segments after it is
+//   D_{last-1} = W_last,     D_{k-1} = Diag(g_k) D_k + W_k,     dh0 = Diag(g_0) D_0 + W_0.
+// In fp32, in place: slot k of W becomes D_{k-1} (k >= 1); slot 0 gives dh0.  Flagged pairs
+// (recomputed whole on the exact route) are left alone.  One thread per 4 consecutive elements
+// of one (batch, head); the maps are loaded 16 segments at a time.  A programmatic dependent of
+// the segments' kernel.
+__global__ void __launch_bounds__(256)
+bwd_scan_kernel(float *__restrict__ W, const float *__restrict__ g, int nseg, const int *__restrict__ flags,
+                float *__restrict__ dh0) {
+    grid_dep_launch();
+    grid_dep_wait();
+    const int bh = blockIdx.x >> 4;
+    if (flags[bh]) return;
+    const int e = ((blockIdx.x & 15) * 256 + threadIdx.x) * 4;
+    const int jrow = e >> 7;
+    constexpr int kBatch = 16;
+    float4 D = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = nseg - 1; s0 >= 0; s0 -= kBatch) {
+        float4 wv[kBatch];
+        float gj[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            if (s0 - i >= 0) {
+                const size_t slot = (size_t)bh * nseg + s0 - i;
+                wv[i] = *reinterpret_cast<const float4 *>(W + slot * 16384 + e);
+                gj[i] = g[slot * 128 + jrow];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int sg = s0 - i;
+            if (sg >= 0) {
+                D = make_float4(fmaf(gj[i], D.x, wv[i].x), fmaf(gj[i], D.y, wv[i].y), fmaf(gj[i], D.z, wv[i].z),
+                                fmaf(gj[i], D.w, wv[i].w));
+                if (sg > 0) *reinterpret_cast<float4 *>(W + ((size_t)bh * nseg + sg) * 16384 + e) = D;
+                else if (dh0) *reinterpret_cast<float4 *>(dh0 + (size_t)bh * 16384 + e) = D;
+            }
+        }
+    }
+}
+
+// The gradient D carried into the last state of segment k < last from later segments reaches its
+// tokens through the decays since: at token t of a chunk (b_t the cumulative log decay from the
+// chunk start, B its total) the state gradient misses Diag(e^{B - b_t}) D.  So, per chunk from the
+// segment's end (k_t = 1 - f_t, i_t the input, S_in the state entering the chunk):
+//   di_t       += D^T (k_t * e^{B - b_t})
+//   dK_t[j]     = e^{B - b_t[j]} (D i_t)[j]           (the missing part of dL/dk_t)
+//   d log f_t  += e^{B} rowsum(S_in * D) + sum_{s<t} k_s dK_s - f_t dK_t
+//   D          <- Diag(e^{B}) D                        (into the chunk before)
+// (the d log f term is f_t rowsum(S_{t-1} * missing gradient of S_t), written with the forward
+// state S_{t-1} expanded over the chunk; it decays with D, so nothing beyond the walked chunks
+// changes).  The saved state holds bf16(e^{rho} S_in), rho = B/2, so e^{B} rowsum(S_in * D) =
+// e^{B - rho} rowsum(S_r * D).  Two MMAs per chunk: DI = Kd bf16(D) (lane t) and
+// Y^T = bf16(D) I^T (lane j), Kd = k e^{B - b}.  One CTA per segment k < last walks its chunks from
+// the end while max_j decay_j max |D[j,:]| >= kFixStop (as the forward's fix-up); di and d log f are
+// read, corrected and stored back.  8 warps: thread (row r, half) holds 64 columns of row r of D.
+namespace bfx {
+constexpr float kStop = 0x1p-24f;
+struct Misc {
+    uint64_t full, barM;
+    uint32_t tmem_base;
+    int pad;
+    float Ppart[4][128];   // 32-row range sums of log f
+    float BT[128];         // the chunk's total log decay B, key dim
+    float Rp[2][128];      // halves of rowsum(S_r * D)
+};
+// log f, i, saved state (then Kd), di, d log f, bf16(D)
+constexpr size_t kSmem = 6 * (size_t)kTileBytes + sizeof(Misc);
+}  // namespace bfx
+
+struct BwdFixParams {
+    const float *D;     // [B*H][nseg][128][128]: slot k+1 = the gradient carried into segment k's end
+    const int *flags;
+    int H, nseg, tps, ntiles;
+};
+
+__global__ void __launch_bounds__(256, 1)
+bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constant__ CUtensorMap tm_x,
+                 const __grid_constant__ CUtensorMap tm_st, const __grid_constant__ CUtensorMap tm_di,
+                 const __grid_constant__ CUtensorMap tm_dlf, BwdFixParams p) {
+    using namespace bfx;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *Lb = smem, *Ib = smem + kTileBytes, *Sb = smem + 2 * kTileBytes, *DIb = smem + 3 * kTileBytes;
+    uint8_t *DLb = smem + 4 * kTileBytes, *X = smem + 5 * kTileBytes;
+    uint8_t *Kd = Sb;   // once rowsum(S_r * D) has been formed
+    Misc *m = reinterpret_cast<Misc *>(smem + 6 * kTileBytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nfix = p.nseg - 1;
+    const int bh = blockIdx.x / nfix, seg = blockIdx.x - bh * nfix, b = bh / p.H, h = bh - b * p.H;
+    const int g0 = seg * p.tps, N = p.tps;   // a segment before the last: tps whole chunks
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0) set_status(HGRN2_ERR_DEVICE);
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(&m->full, 1);
+        mbar_init(&m->barM, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_lf);
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_st);
+        tma_prefetch_desc(&tm_di);
+        tma_prefetch_desc(&tm_dlf);
+    }
+    if (warp == 0) {
+        tmem_alloc(&m->tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = m->tmem_base;
+    const int quad = warp & 3, ch = warp >> 2, r = 32 * quad + lane;
+    const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
+    const uint32_t id_kk = idesc_bf16(128, 128, false, false);
+    const uint32_t id_kmn = idesc_bf16(128, 128, false, true);
+    const int pc = tid & 63, rr = tid >> 6, col0 = 2 * pc;   // prep: column pair, 32-row range
+    const uint32_t cblk = (uint32_t)(col0 >> 6) * kBlk, cch = (uint32_t)((col0 & 63) >> 3), cin = (uint32_t)(col0 & 7) * 2;
+    auto eoff = [&](int t) -> uint32_t { return cblk + t * 128 + ((cch ^ (t & 7)) << 4) + cin; };
+    // element (t, j) of a tile (lane j's column)
+    const uint32_t jblk = (uint32_t)(r >> 6) * kBlk, jch = (uint32_t)((r & 63) >> 3), jin = (uint32_t)(r & 7) * 2;
+    auto joff = [&](int t) -> uint32_t { return jblk + t * 128 + ((jch ^ (t & 7)) << 4) + jin; };
+    int issued = 0, waited = 0;
+    auto load = [&](int c) {   // thread 0: chunk g0 + c
+        const int tok = (g0 + c) * kTile, slot = bh * p.ntiles + g0 + c;
+        mbar_arrive_expect_tx(&m->full, 5 * kTileBytes);
+        for (int k = 0; k < 2; ++k) {
+            tma_load_4d(Lb + k * kBlk, &tm_lf, &m->full, 64 * k, h, tok, b);
+            tma_load_4d(Ib + k * kBlk, &tm_x, &m->full, 64 * k, h, tok, b);
+            tma_load_4d(Sb + k * kBlk, &tm_st, &m->full, 64 * k, 0, 0, slot);
+            tma_load_4d(DIb + k * kBlk, &tm_di, &m->full, 64 * k, h, tok, b);
+            tma_load_4d(DLb + k * kBlk, &tm_dlf, &m->full, 64 * k, h, tok, b);
+        }
+        ++issued;
+    };
+
+    grid_dep_wait();   // the segments' outputs and the scan's gradients are complete from here on
+    float Dr[64];      // the carried gradient, row r, columns 64 ch .. 64 ch + 63
+    float dmax = 0.0f, decay = 1.0f;
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(p.D + ((size_t)bh * p.nseg + seg + 1) * 16384 +
+                                                             (size_t)r * 128 + 64 * ch);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float4 a = src[i];
+            Dr[4 * i] = a.x; Dr[4 * i + 1] = a.y; Dr[4 * i + 2] = a.z; Dr[4 * i + 3] = a.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 64; ++i) dmax = fmaxf(dmax, fabsf(Dr[i]));
+    }
+    bool ok = true;
+    bool go = !p.flags[bh] && __syncthreads_or(dmax >= kStop);
+    if (go && tid == 0) load(N - 1);
+    for (int c = N - 1; go && c >= 0; --c) {
+        const int tok = (g0 + c) * kTile;
+        // bf16(D) -> X (row r = key dim, columns = value dims)
+        {
+            float v[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = Dr[32 * hh + i];
+                store_chunk_bf16(X, r, 2 * ch + hh, v);
+            }
+        }
+        if (__syncthreads_or(!mbar_wait(&m->full, waited & 1))) { ok = false; break; }
+        ++waited;
+        // rowsum(S_r * D), this thread's half of row r
+        {
+            float acc = 0.0f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int cc = 2 * ch + hh;
+                const uint8_t *base = Sb + (cc >> 1) * kBlk + r * 128;
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        acc = fmaf(bf_lo(ws[k]), Dr[32 * hh + 8 * qd + 2 * k], acc);
+                        acc = fmaf(bf_hi(ws[k]), Dr[32 * hh + 8 * qd + 2 * k + 1], acc);
+                    }
+                }
+            }
+            m->Rp[ch][r] = acc;
+        }
+        // prep: range sums of log f; B (summed as the forward's prep sums it); Kd = k e^{B - b}
+        // over the saved state's tile (read above)
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(Lb + eoff(32 * rr + i));
+            s0 += bf_lo(w);
+            s1 += bf_hi(w);
+        }
+        m->Ppart[rr][col0] = s0;
+        m->Ppart[rr][col0 + 1] = s1;
+        __syncthreads();   // Ppart complete; every thread has read S_r
+        {
+            float b0 = 0.0f, b1 = 0.0f;
+            for (int r2 = 0; r2 < rr; ++r2) {
+                b0 += m->Ppart[r2][col0];
+                b1 += m->Ppart[r2][col0 + 1];
+            }
+            const float B0 = ((m->Ppart[0][col0] + m->Ppart[1][col0]) + m->Ppart[2][col0]) + m->Ppart[3][col0];
+            const float B1 = ((m->Ppart[0][col0 + 1] + m->Ppart[1][col0 + 1]) + m->Ppart[2][col0 + 1]) +
+                             m->Ppart[3][col0 + 1];
+            if (rr == 0) {
+                m->BT[col0] = B0;
+                m->BT[col0 + 1] = B1;
+            }
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                const int t = 32 * rr + i;
+                const uint32_t wa = *reinterpret_cast<const uint32_t *>(Lb + eoff(t));
+                b0 += bf_lo(wa);
+                b1 += bf_hi(wa);
+                const float k0 = 1.0f - __expf(bf_lo(wa)), k1 = 1.0f - __expf(bf_hi(wa));
+                *reinterpret_cast<uint32_t *>(Kd + eoff(t)) = pack_bf2(k0 * __expf(B0 - b0), k1 * __expf(B1 - b1));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();   // Kd, X, B, rowsum halves complete
+        if (tid == 0) {    // DI = Kd bf16(D) (cols 0..127, lane t); Y^T = bf16(D) I^T (cols 128..255, lane j)
+            tc_fence_after();
+            const uint64_t dK = sdesc_sw128(smem_u32(Kd), 16, 1024);
+            const uint64_t dXm = sdesc_sw128(smem_u32(X), kBlk, 1024);
+            const uint64_t dXk = sdesc_sw128(smem_u32(X), 16, 1024);
+            const uint64_t dI = sdesc_sw128(smem_u32(Ib), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase, sdesc_add(dK, ko), sdesc_add(dXm, kk * 2048), id_kmn, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ko = (kk >> 2) * kBlk + (kk & 3) * 32;
+                mma_bf16_ss(tbase + 128, sdesc_add(dXk, ko), sdesc_add(dI, ko), id_kk, kk > 0);
+            }
+            mma_commit(&m->barM);
+        }
+        if (__syncthreads_or(!mbar_wait(&m->barM, (N - 1 - c) & 1))) { ok = false; break; }   // chunk N-1-c walked
+        tc_fence_after();
+        if (ch == 1) {
+            // di row r (token) += DI row r
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld32(tl + 32 * cc, v);
+                tmem_wait_ld();
+                const uint8_t *base = DIb + (cc >> 1) * kBlk + r * 128;
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        v[8 * qd + 2 * k] += bf_lo(ws[k]);
+                        v[8 * qd + 2 * k + 1] += bf_hi(ws[k]);
+                    }
+                }
+                store_chunk_bf16(DIb, r, cc, v);
+            }
+        } else {
+            // d log f column r (key dim) over the chunk's tokens, in order
+            const float Bt = m->BT[r];
+            const float rho = 0.5f * Bt;
+            const float base = __expf(Bt - rho) * (m->Rp[0][r] + m->Rp[1][r]);   // e^{B} rowsum(S_in * D)
+            float bsum = 0.0f, pre = 0.0f;
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                float y[32];
+                tmem_ld32(tl + 128 + 32 * cb, y);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int t = 32 * cb + i;
+                    const float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Lb + joff(t)));
+                    bsum += a;
+                    const float f = __expf(a);
+                    const float dK = __expf(Bt - bsum) * y[i];
+                    __nv_bfloat16 *dl = reinterpret_cast<__nv_bfloat16 *>(DLb + joff(t));
+                    *dl = __float2bfloat16_rn(__bfloat162float(*dl) + (base + pre - f * dK));
+                    pre = fmaf(1.0f - f, dK, pre);
+                }
+            }
+        }
+        // the carried gradient into the chunk before
+        const float eb = __expf(m->BT[r]);
+        decay *= eb;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) Dr[i] *= eb;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        const bool next = __syncthreads_or(decay * dmax >= kStop) && c > 0;
+        if (tid == 0) {
+            for (int k = 0; k < 2; ++k) {
+                tma_store_4d(&tm_di, DIb + k * kBlk, 64 * k, h, tok, b);
+                tma_store_4d(&tm_dlf, DLb + k * kBlk, 64 * k, h, tok, b);
+            }
+            tma_store_commit();
+            if (next) {   // the tiles, once this chunk's stores have read them
+                tma_store_wait_read0();
+                load(c - 1);
+            }
+        }
+        go = next;
+    }
+    if (tid == 0) {
+        if (!ok) set_status(HGRN2_ERR_TIMEOUT);
+        for (int k = waited; k < issued; ++k) mbar_wait(&m->full, k & 1, 2000000u);
+        tma_store_wait_all0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
 }  // namespace tcb
 
 static_assert(tcb::fsw::kSmemBytes <= 227 * 1024, "forward-sweep shared memory");
 static_assert(tcb::rsw::kSmemBytes <= 227 * 1024, "reverse-sweep shared memory");
+
+static_assert(tcb::bfx::kSmem <= 227 * 1024, "backward fix-up shared memory");
+
+size_t tc_bwd_workspace(int B, int T, int H) {
+    int nseg, tps;
+    tc_fwd_segments(B, T, H, &nseg, &tps);   // the forward's cut
+    return nseg > 1 ? (size_t)B * H * nseg * (16384 + 128) * sizeof(float) : 0;
+}
+int tc_bwd_launches(int B, int T, int H) { return tc_bwd_workspace(B, T, H) ? 3 : 1; }
+
+// Launches a kernel as a programmatic dependent of the previous work in the stream: it may be
+// scheduled before that work completes, and waits for it with grid_dep_wait().
+template <typename... Exp, typename... Act>
+static cudaError_t launch_dependent_b(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                      Act &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
 
 size_t tc_bwd_smem() { return tcb::fsw::kSmemBytes > tcb::rsw::kSmemBytes ? tcb::fsw::kSmemBytes : tcb::rsw::kSmemBytes; }
 
@@ -1154,8 +1530,37 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
                       (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm, D, (const __nv_bfloat16 *)a.lgs,
-                      (__nv_bfloat16 *)a.dlg, a.nK, a.nV, Bm};
+                      (__nv_bfloat16 *)a.dlg, a.nK, a.nV, Bm, 1, ntiles, nullptr, nullptr};
     cudaError_t e;
+    int nseg = 1, tps = ntiles;
+    if (saved && !packed && !a.lgs && !inplace && D == 128 && a.seg_ws) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);
+    if (nseg > 1) {
+        // sequence segments: every segment from a zero gradient (the last from dhT), the reverse
+        // scan of their maps (and dh0), then the carried gradients added to each segment's last chunks
+        const int BH = a.B * a.H;
+        float *W = a.seg_ws, *g = a.seg_ws + (size_t)BH * nseg * 16384;
+        p2.nseg = nseg;
+        p2.tps = tps;
+        p2.Wseg = W;
+        p2.gseg = g;
+        size_t smem = tcb::rsw::kSmemBytes;
+        if (simt_bwd_dq_smem(a.simt_C, D, D) > smem) smem = simt_bwd_dq_smem(a.simt_C, D, D);
+        if (simt_bwd_rev_smem(a.simt_C, D, D) > smem) smem = simt_bwd_rev_smem(a.simt_C, D, D);
+        auto kern = tcb::rev_kernel<true, false, false, false, true>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        kern<<<BH * nseg, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_dependent_b(tcb::bwd_scan_kernel, dim3(BH * 16), dim3(256), 0, st, W, (const float *)g, nseg,
+                               (const int *)a.flags, a.dh0);
+        if (e != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(tcb::bwd_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)tcb::bfx::kSmem)) != cudaSuccess)
+            return e;
+        tcb::BwdFixParams fp{W, a.flags, a.H, nseg, tps, ntiles};
+        return launch_dependent_b(tcb::bwd_fixup_kernel, dim3(BH * (nseg - 1)), dim3(256), tcb::bfx::kSmem, st, ml,
+                                  mx, mst, mdi, mdl, fp);
+    }
     if (saved) {
         // one launch; the exact route of a flagged (b,h) runs in the same shared memory
         size_t smem = tcb::rsw::kSmemBytes;

@@ -63,6 +63,9 @@ TRAIN_LB0 = Workload("train_fwdbwd_bf16_B8_H16_T2048_d128_lb0", 8, 16, 2048, 128
 TRAIN_D64 = Workload("train_fwdbwd_bf16_B8_H32_T2048_d64", 8, 32, 2048, 64, 64, torch.bfloat16, 0.95, 64, bwd=True)
 # ... and with 256-wide heads
 TRAIN_D256 = Workload("train_fwdbwd_bf16_B8_H8_T2048_d256", 8, 8, 2048, 256, 256, torch.bfloat16, 0.95, 64, bwd=True)
+# ... and the long sequence's shape as a training pair (few (b,h): both directions in segments)
+TRAIN_LONG = Workload("train_fwdbwd_bf16_B1_H8_T32768_d128", 1, 8, 32768, 128, 128, torch.bfloat16, 0.9, 64,
+                      bwd=True)
 
 WORKLOADS = {w.name: w for w in (TINY, FWD_LAYER, TRAIN, LONG, TRAIN_D64, TRAIN_D256)}
 

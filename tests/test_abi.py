@@ -196,12 +196,23 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
     bad = ctypes.c_size_t(-1).value
     up = lambda x: (x + 255) // 256 * 256
     B, T, H = 2, 300, 3
-    for d in (128, 64):
-        assert f(B, T, H, d, d, 64, L.BF16, 2) <= f(B, T, H, d, d, 64, L.BF16, 1)
+    assert f(B, T, H, 64, 64, 64, L.BF16, 2) <= f(B, T, H, 64, 64, 64, L.BF16, 1)
     # d = 64 without saved states: room for the chunk states and an o scratch on top
     extra = lib.hgrn2_saved_size(B, T, H, 64, 64, L.BF16) + up(B * T * H * 64 * 2)
     assert f(B, T, H, 64, 64, 64, L.BF16, 1) == f(B, T, H, 64, 64, 64, L.BF16, 2) + extra
-    assert f(B, T, H, 128, 128, 64, L.BF16, 1) == f(B, T, H, 128, 128, 64, L.BF16, 2)
+    # d = 128 with saved states and few (b,h): the backward runs in sequence segments, cut as the
+    # forward cuts them (148 // (B*H) per pair, at most one per chunk), and keeps every segment's
+    # backward map (128 x 128 + 128 floats)
+    def nseg(B, T, H):
+        ntiles = (T + 127) // 128
+        ns = min(max(1, 148 // (B * H)), ntiles)
+        tps = (ntiles + ns - 1) // ns
+        return (ntiles + tps - 1) // tps
+    for (B, T, H) in ((2, 300, 3), (1, 32768, 8), (8, 2048, 16)):
+        ns = nseg(B, T, H)
+        seg = up(B * H * ns * (128 * 128 + 128) * 4) if ns > 1 else 0
+        assert f(B, T, H, 128, 128, 64, L.BF16, 2) == f(B, T, H, 128, 128, 64, L.BF16, 1) + seg, (B, T, H)
+    assert nseg(8, 2048, 16) == 1 and nseg(1, 32768, 8) == 18
     assert f(B, T, H, 64, 64, 64, L.BF16, 3) == bad
     assert f(B, T, H, 64, 64, 64, L.BF16, -1) == bad
 
