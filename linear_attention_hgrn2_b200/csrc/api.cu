@@ -451,20 +451,20 @@ hgrn2_status stack_fwd(const void *q, const void *log_f, const void *i, const fl
         if (!C) return HGRN2_ERR_UNSUPPORTED;
         const SavedLayout sl = saved_layout(B, T, H * nb);
         int *flags = saved ? (int *)((char *)saved + sl.flags) : (int *)w.sub;
-        TcFwdArgs t{q, log_f, i, h0 ? w.h0 : nullptr, w.part, hT ? w.hT : nullptr, flags, nullptr, B, T, H * nb, C,
+        // every block pair adds its share of o into o: zeroed first
+        if (cudaMemsetAsync(o, 0, rows * dv * es, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
+        TcFwdArgs t{q, log_f, i, h0 ? w.h0 : nullptr, o, hT ? w.hT : nullptr, flags, nullptr, B, T, H * nb, C,
                     saved, saved ? (float *)((char *)saved + sl.hTs) : nullptr, nullptr, nullptr, 128};
         t.nK = nK;
         t.nV = nV;
+        t.opart = w.part;
         if (launch_tc_fwd(t, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
         for (int a = 0; a < nK && hT; ++a)
             for (int c = 0; c < nV; ++c)
                 if (launch_state_block(hT, w.hT + (a * nV + c) * sm, nb * sm, BH, dk, dv, s.off[0][a], kw,
                                        s.off[1][c], vw, true, stream) != cudaSuccess)
                     return HGRN2_ERR_CUDA;
-        // o = the two key blocks' partials, [nK][B][T][H][256], added in fp32
-        if (launch_sum_blocks(o, dv, 0, w.part, w.part + rows * dv * es, dv, rows, dv, bf16, stream) != cudaSuccess)
-            return HGRN2_ERR_CUDA;
-        g_launches += (h0 ? nb : 0) + 1 + (hT ? nb : 0) + 1;
+        g_launches += (h0 ? nb : 0) + 1 + (hT ? nb : 0);
         return HGRN2_OK;
     }
     for (int a = 0; a < nK; ++a)
@@ -519,24 +519,26 @@ hgrn2_status stack_bwd(const void *q, const void *log_f, const void *i, const fl
         const int C = simt_chunk(chunk, kw, vw, true);
         if (!C) return HGRN2_ERR_UNSUPPORTED;
         const SavedLayout sl = saved_layout(B, T, H * nb);
-        TcBwdArgs t{q, log_f, i, dO, h0 ? w.h0 : nullptr, dhT ? w.dhT : nullptr, w.pq, w.pf, w.part,
+        // every block pair adds its shares of dq, d log f and di into them: zeroed first
+        if (cudaMemsetAsync(dq, 0, rows * dk * es, stream) != cudaSuccess ||
+            cudaMemsetAsync(dlog_f, 0, rows * dk * es, stream) != cudaSuccess ||
+            cudaMemsetAsync(di, 0, rows * dv * es, stream) != cudaSuccess)
+            return HGRN2_ERR_CUDA;
+        TcBwdArgs t{q, log_f, i, dO, h0 ? w.h0 : nullptr, dhT ? w.dhT : nullptr, dq, dlog_f, di,
                     dh0 ? w.dh0 : nullptr, (float *)w.sub, (int *)((char *)saved + sl.flags), B, T, H * nb, C, saved,
                     (const float *)((const char *)saved + sl.hTs), nullptr, nullptr, 128};
         t.nK = nK;
         t.nV = nV;
+        t.dq_part = w.pq;
+        t.dlf_part = w.pf;
+        t.dx_part = w.part;
         if (launch_tc_bwd(t, stream) != cudaSuccess) return HGRN2_ERR_CUDA;
         for (int a = 0; a < nK && dh0; ++a)
             for (int c = 0; c < nV; ++c)
                 if (launch_state_block(dh0, w.dh0 + (a * nV + c) * sm, nb * sm, BH, dk, dv, s.off[0][a], kw,
                                        s.off[1][c], vw, true, stream) != cudaSuccess)
                     return HGRN2_ERR_CUDA;
-        // dq, d log f: the value blocks' partials; di: the key blocks' ([2][B][T][H][256] each)
-        const size_t half = rows * 256 * es;
-        if (launch_sum_blocks(dq, dk, 0, w.pq, w.pq + half, dk, rows, dk, bf16, stream) != cudaSuccess ||
-            launch_sum_blocks(dlog_f, dk, 0, w.pf, w.pf + half, dk, rows, dk, bf16, stream) != cudaSuccess ||
-            launch_sum_blocks(di, dv, 0, w.part, w.part + half, dv, rows, dv, bf16, stream) != cudaSuccess)
-            return HGRN2_ERR_CUDA;
-        g_launches += (h0 ? nb : 0) + (dhT ? nb : 0) + 1 + (dh0 ? nb : 0) + 3;
+        g_launches += (h0 ? nb : 0) + (dhT ? nb : 0) + 1 + (dh0 ? nb : 0);
         return HGRN2_OK;
     }
     for (int a = 0; a < nK; ++a)

@@ -33,9 +33,11 @@ struct TcFwdArgs {
     int D;             // head size d_k = d_v: 128 or 64
     const void *lgs;   // scalar-decay variant: log g [B][T][H] (lf is then the key k); else null
     // Heads of width nK * 128 = nV * 128 read in place (nK = nV = 2: 256): H counts block pairs,
-    // H / (nK nV) the caller's heads; q, lf, x are the caller's [B][T][H / (nK nV)][256] tensors and
-    // o the key blocks' partials [nK][B][T][H / (nK nV)][256] (summed by the caller).
+    // H / (nK nV) the caller's heads; q, lf, x, o are the caller's [B][T][H / (nK nV)][256] tensors.
+    // o must be zero on entry: every block pair adds its share into it.  opart: scratch
+    // [nK][B][T][H / (nK nV)][256] for the shares of pairs flagged for the exact route.
     int nK = 1, nV = 1;
+    void *opart = nullptr;
 };
 
 struct SimtBwdArgs {
@@ -66,10 +68,12 @@ struct TcBwdArgs {
     int D;             // head size d_k = d_v: 128 or 64 (64: saved-state mode only)
     const void *lgs;   // scalar-decay variant (saved mode): log g [B][T][H]; lf is then k, dlf dk
     void *dlg;         // scalar-decay variant: d log g [B][T][H]
-    // Heads read in place (saved mode, nK = nV = 2), as for TcFwdArgs: q, lf, x, dO are the caller's
-    // 256-wide tensors; dq, dlf the value blocks' partials [nV][B][T][Hw][256]; dx the key blocks'
-    // partials [nK][B][T][Hw][256].
+    // Heads read in place (saved mode, nK = nV = 2), as for TcFwdArgs: q, lf, x, dO, dq, dlf, dx are
+    // the caller's 256-wide tensors; dq, dlf, dx must be zero on entry (every block pair adds its
+    // share).  Scratch for the shares of flagged pairs: dq, dlf as the value blocks' partials
+    // [nV][B][T][Hw][256] (dq_part, dlf_part), dx as the key blocks' [nK][B][T][Hw][256] (dx_part).
     int nK = 1, nV = 1;
+    void *dq_part = nullptr, *dlf_part = nullptr, *dx_part = nullptr;
     // saved states, dense d = 128, few (b,h): sequence segments' workspace, tc_bwd_workspace(B, T, H)
     // bytes (null: one CTA per (b,h))
     float *seg_ws = nullptr;

@@ -489,9 +489,13 @@ struct RevParams {
     __nv_bfloat16 *dlg;         // scalar decay: d log g [B][T][H]
     // Heads of width 256 read in place (saved mode; nK = nV = 2): head h of the call is block pair
     // (a, c) of head h / (nK nV); q, log f at half-head (h / (nK nV)) nK + a and i, dO at * nV + c of
-    // the caller's tensors viewed as [B][T][2 Hw][128]; dq, d log f go to the value block's partial
-    // ([nV][B][T][Hw][256]), di to the key block's ([nK][B][T][Hw][256]).  nK = nV = 1 otherwise.
+    // the caller's tensors viewed as [B][T][2 Hw][128].  Every block pair adds its shares of dq,
+    // d log f (key-side half-heads) and di (value-side) into the outputs, zeroed by the host, by TMA
+    // reduce-add; a flagged pair's exact route writes its shares into the partials (dq, d log f: the
+    // value block's, [nV][B][T][Hw][256]; di: the key block's, [nK][B][T][Hw][256]) and adds them
+    // from there.  nK = nV = 1 otherwise.
     int nK, nV, Bo;
+    __nv_bfloat16 *dq_part, *dlf_part, *dx_part;   // heads read in place: the exact route's partials
     // Sequence segments (kSeg): [B*H][nseg] segments of tps chunks each; every segment's reverse
     // sweep starts from a zero gradient (the last from dhT) and writes its backward map: W, the
     // gradient it hands to the state entering it ([B*H][nseg][128][128]), and g, its decay product
@@ -577,15 +581,22 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 // heads read in place (nK = nV): every token tensor viewed with Hw nK half-heads of 128,
                 // indexed at the value-side half-head hv; key-side tensors shifted by hk - hv half-heads,
                 // the partial outputs by their block
+                // The shares go to the partials first (the reverse sweep reads its dq share back),
+                // then are added into the outputs (other block pairs add theirs by TMA reduce-add)
                 const int Hh = (p.H / nbk) * p.nV;
                 const long long ks = (long long)(hk - hv) * p.D;
                 const size_t part = (size_t)p.Bo * p.T * Hh * p.D;
-                __nv_bfloat16 *dq = p.dq + vc * part + ks, *dlf = p.dlf + vc * part + ks, *dx = p.dx + ka * part;
+                __nv_bfloat16 *dq = p.dq_part + vc * part + ks, *dlf = p.dlf_part + vc * part + ks;
+                __nv_bfloat16 *dx = p.dx_part + ka * part;
                 simt_bwd_dq_body<__nv_bfloat16>(p.lf + ks, p.x, p.h0, p.dO, p.dhT, dq, p.rs, p.T, Hh, p.D, p.D,
                                                 p.simt_chunk, sm, b, hv, bh, dlf, dx);
                 __syncthreads();
                 simt_bwd_rev_body<__nv_bfloat16>(p.q + ks, p.lf + ks, p.x, p.dO, p.dhT, dq, p.rs, dlf, dx, p.dh0, p.T,
                                                  Hh, p.D, p.D, p.simt_chunk, sm, b, hv, bh, true);
+                __syncthreads();
+                add_rows_bf16(p.dq + ks, dq, b, hv, p.T, Hh);
+                add_rows_bf16(p.dlf + ks, dlf, b, hv, p.T, Hh);
+                add_rows_bf16(p.dx, dx, b, hv, p.T, Hh);
             }
             if (tid == 0) atomicAdd(&g_counters[0], 1ull);
         }
@@ -1101,9 +1112,15 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (vr == kTile) {
             if (tid == kStoreTid) {   // a thread of another warp than the one issuing loads and MMAs
                 for (int c = 0; c < nblk; ++c) {
-                    tma_store_4d(&tm_di, AT + c * kBlk, 64 * c, hv, tok0 + n * kTile, vbc);
-                    tma_store_4d(&tm_dlf, DA + c * kBlk, 64 * c, hk, tok0 + n * kTile, kbc);
-                    if (kSaved) tma_store_4d(&tm_dq, D16 + c * kBlk, 64 * c, hk, tok0 + n * kTile, kbc);
+                    if constexpr (kWide) {   // this block pair's shares, added into the outputs
+                        tma_reduce_add_4d(&tm_di, AT + c * kBlk, 64 * c, hv, tok0 + n * kTile, bc);
+                        tma_reduce_add_4d(&tm_dlf, DA + c * kBlk, 64 * c, hk, tok0 + n * kTile, bc);
+                        tma_reduce_add_4d(&tm_dq, D16 + c * kBlk, 64 * c, hk, tok0 + n * kTile, bc);
+                    } else {
+                        tma_store_4d(&tm_di, AT + c * kBlk, 64 * c, hv, tok0 + n * kTile, vbc);
+                        tma_store_4d(&tm_dlf, DA + c * kBlk, 64 * c, hk, tok0 + n * kTile, kbc);
+                        if (kSaved) tma_store_4d(&tm_dq, D16 + c * kBlk, 64 * c, hk, tok0 + n * kTile, kbc);
+                    }
                 }
                 tma_store_commit();
             }
@@ -1512,15 +1529,17 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     if (a.lgs && packed) return cudaErrorInvalidValue;
     const int nbk = a.nK * a.nV;
     const bool inplace = nbk > 1;
-    if (inplace && (!saved || packed || a.lgs || a.D != 128 || a.nK != a.nV || a.H % nbk)) return cudaErrorInvalidValue;
+    if (inplace && (!saved || packed || a.lgs || a.D != 128 || a.nK != a.nV || a.H % nbk || !a.dq_part ||
+                    !a.dlf_part || !a.dx_part))
+        return cudaErrorInvalidValue;
     const int Hk = inplace ? a.H / nbk * a.nK : a.H, Hv = inplace ? a.H / nbk * a.nV : a.H;
     const int Bm = packed ? 1 : a.B, D = a.D;
     const int ntiles = (a.T + tcc::kTile - 1) / tcc::kTile;
     CUtensorMap mq, ml, mx, mdo, mdq, mdi, mdl, mst;
     if (!make_token_map(&mq, a.q, Bm, a.T, Hk, D) || !make_token_map(&ml, a.lf, Bm, a.T, Hk, D) ||
         !make_token_map(&mx, a.x, Bm, a.T, Hv, D) || !make_token_map(&mdo, a.dO, Bm, a.T, Hv, D) ||
-        !make_token_map(&mdq, a.dq, Bm * a.nV, a.T, Hk, D) || !make_token_map(&mdi, a.dx, Bm * a.nK, a.T, Hv, D) ||
-        !make_token_map(&mdl, a.dlf, Bm * a.nV, a.T, Hk, D))
+        !make_token_map(&mdq, a.dq, Bm, a.T, Hk, D) || !make_token_map(&mdi, a.dx, Bm, a.T, Hv, D) ||
+        !make_token_map(&mdl, a.dlf, Bm, a.T, Hk, D))
         return cudaErrorInvalidValue;
     // saved states: 128-row "token" tiles
     if (saved && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
@@ -1530,7 +1549,8 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
                       (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.lf, (const __nv_bfloat16 *)a.x,
                       (const __nv_bfloat16 *)a.dO, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dlf,
                       (__nv_bfloat16 *)a.dx, a.simt_C, a.cu, a.perm, D, (const __nv_bfloat16 *)a.lgs,
-                      (__nv_bfloat16 *)a.dlg, a.nK, a.nV, Bm, 1, ntiles, nullptr, nullptr};
+                      (__nv_bfloat16 *)a.dlg, a.nK, a.nV, Bm, (__nv_bfloat16 *)a.dq_part,
+                      (__nv_bfloat16 *)a.dlf_part, (__nv_bfloat16 *)a.dx_part, 1, ntiles, nullptr, nullptr};
     cudaError_t e;
     int nseg = 1, tps = ntiles;
     if (saved && !packed && !a.lgs && !inplace && D == 128 && a.seg_ws) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);

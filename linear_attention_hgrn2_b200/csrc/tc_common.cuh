@@ -114,6 +114,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, co
 }
 
 // One 32-column chunk (c = 0..3) of a TMEM row -> bf16 into row `row` of a swizzled 128 x 128 tile.
+// dst += src over rows t of batch b, half-head hv of [B][T][Hh][128] bf16 tensors (atomically: other
+// CTAs add into the same rows).
+__device__ __forceinline__ void add_rows_bf16(__nv_bfloat16 *dst, const __nv_bfloat16 *src, int b, int hv, int T,
+                                              int Hh) {
+    for (size_t idx = threadIdx.x; idx < (size_t)T * 64; idx += blockDim.x) {
+        const size_t t = idx >> 6, cp = idx & 63;
+        const size_t off = (((size_t)b * T + t) * Hh + hv) * 128 + 2 * cp;
+        atomicAdd(reinterpret_cast<__nv_bfloat162 *>(dst + off), *reinterpret_cast<const __nv_bfloat162 *>(src + off));
+    }
+}
+
 __device__ __forceinline__ void store_chunk_bf16(uint8_t *tile, int row, int c, const float (&r)[32]) {
     uint8_t *base = tile + (c >> 1) * kBlk + row * 128;
 #pragma unroll

@@ -102,13 +102,16 @@ struct Params {
     // Heads of width 256 read in place: head h of the call is block pair (a, c) of head
     // h / (nK nV) of the caller's [B][T][Hw][256] tensors, a = key block, c = value block.  Those
     // are read as [B][T][Hw nK][128] (q, log f: half-head Hw-index * nK + a) and [B][T][Hw nV][128]
-    // (i: * nV + c); o is the key block's partial, [nK][B][T][Hw nV][128].  nK = nV = 1 otherwise.
+    // (i: * nV + c).  Every block pair adds its share of o into o ([B][T][Hw nV][128], zeroed by the
+    // host) by TMA reduce-add; a flagged pair's exact route writes its share into its key block's
+    // partial of opart ([nK][B][T][Hw nV][128]) and adds it from there.  nK = nV = 1 otherwise.
     int nK, nV, Bo;   // Bo: the batch count of one o partial
     // With segments, for the carried-state fix-up of segments k >= 1: bf16(q e^{b}) of the
     // segment's first chunk ([B*H][nseg][128][128], b the cumulative log f from the chunk start)
     // and that chunk's total log decay B ([B*H][nseg][128])
     __nv_bfloat16 *qtil;
     float *bseg;
+    __nv_bfloat16 *opart;   // heads read in place: the exact route's partial outputs
 };
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
@@ -411,8 +414,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 mbar_arrive(&m->ofree);
                 if (named_bar_or(2, 128, fail)) break;
                 if (r == 0) {
-                    tma_store_4d(&tm_o, X, 0, hv, tok0 + n * kTile, obc);
-                    if (nblk == 2) tma_store_4d(&tm_o, X + kBlk, 64, hv, tok0 + n * kTile, obc);
+                    if (nbk > 1) {   // heads read in place: this block pair's share, added into o
+                        tma_reduce_add_4d(&tm_o, X, 0, hv, tok0 + n * kTile, bc);
+                        tma_reduce_add_4d(&tm_o, X + kBlk, 64, hv, tok0 + n * kTile, bc);
+                    } else {
+                        tma_store_4d(&tm_o, X, 0, hv, tok0 + n * kTile, obc);
+                        if (nblk == 2) tma_store_4d(&tm_o, X + kBlk, 64, hv, tok0 + n * kTile, obc);
+                    }
                     tma_store_commit();
                 }
             } else if (!fail) {   // a packed sequence's last chunk: its rows only, stored by their threads
@@ -708,12 +716,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             } else {
                 // heads read in place (nK = nV): every token tensor is viewed with Hw nK half-heads of
                 // 128 and indexed at the value-side half-head hv; the key-side tensors are shifted by
-                // the half-heads between hk and hv, and o by its key block's partial
+                // the half-heads between hk and hv.  The share goes to the key block's partial, then
+                // is added into o (other block pairs add theirs by TMA reduce-add, in any order)
                 const int Hh = (p.H / nbk) * p.nV;   // half-heads of the token tensors
                 const long long kshift = (long long)(hk - hv) * p.D;
                 const size_t opart = (size_t)ka * p.Bo * p.T * Hh * p.D;
-                simt_fwd_body<__nv_bfloat16>(p.q + kshift, p.lf + kshift, p.x, p.h0, p.o + opart, p.hT, p.T, Hh, p.D,
-                                             p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, hv, bh);
+                simt_fwd_body<__nv_bfloat16>(p.q + kshift, p.lf + kshift, p.x, p.h0, p.opart + opart, p.hT, p.T, Hh,
+                                             p.D, p.D, p.simt_chunk, reinterpret_cast<float *>(smem), b, hv, bh);
+                __syncthreads();
+                add_rows_bf16(p.o, p.opart + opart, b, hv, p.T, Hh);
             }
         }
     }
@@ -1388,11 +1399,11 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     const int Bm = packed ? 1 : a.B;
     const int nbk = a.nK * a.nV;
     const bool inplace = nbk > 1;
-    if (inplace && (packed || a.lgs || a.D != 128 || a.nK != a.nV || a.H % nbk)) return cudaErrorInvalidValue;
+    if (inplace && (packed || a.lgs || a.D != 128 || a.nK != a.nV || a.H % nbk || !a.opart)) return cudaErrorInvalidValue;
     const int Hk = inplace ? a.H / nbk * a.nK : a.H, Hv = inplace ? a.H / nbk * a.nV : a.H;
     CUtensorMap mq, ml, mx, mo, mst;
     if (!make_token_map(&mq, a.q, Bm, a.T, Hk, a.D) || !make_token_map(&ml, a.lf, Bm, a.T, Hk, a.D) ||
-        !make_token_map(&mx, a.x, Bm, a.T, Hv, a.D) || !make_token_map(&mo, a.o, Bm * a.nK, a.T, Hv, a.D))
+        !make_token_map(&mx, a.x, Bm, a.T, Hv, a.D) || !make_token_map(&mo, a.o, Bm, a.T, Hv, a.D))
         return cudaErrorInvalidValue;
     // saved states: 128-row "token" tiles
     if (a.st16 && !make_token_map(&mst, a.st16, tc_saved_slots(a.B, a.T, a.H, packed), 128, 1))
@@ -1425,7 +1436,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, g, a.T, a.H, ntiles, nseg, tps,
                   a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D,
                   (const __nv_bfloat16 *)a.lgs, seg_done, a.nK, a.nV, Bm,
-                  nseg > 1 ? qtil : nullptr, nseg > 1 ? bs : nullptr};
+                  nseg > 1 ? qtil : nullptr, nseg > 1 ? bs : nullptr, (__nv_bfloat16 *)a.opart};
     kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
     if ((e = cudaGetLastError()) != cudaSuccess || nseg == 1) return e;
     // segments: the states entering them (and hT), then the carried states' contributions.  With
