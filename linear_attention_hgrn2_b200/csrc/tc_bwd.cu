@@ -1226,7 +1226,7 @@ bwd_scan_kernel(float *__restrict__ W, const float *__restrict__ g, int nseg, co
 namespace bfx {
 constexpr float kStop = 0x1p-24f;
 struct Misc {
-    uint64_t full, barM;
+    uint64_t fullA, fullB, barM;   // A: i and the saved state; B: log f, di, d log f
     uint32_t tmem_base;
     int pad;
     float Ppart[4][128];   // 32-row range sums of log f
@@ -1262,7 +1262,8 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
         return;
     }
     if (tid == 0) {
-        mbar_init(&m->full, 1);
+        mbar_init(&m->fullA, 1);
+        mbar_init(&m->fullB, 1);
         mbar_init(&m->barM, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_lf);
@@ -1289,21 +1290,36 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
     // element (t, j) of a tile (lane j's column)
     const uint32_t jblk = (uint32_t)(r >> 6) * kBlk, jch = (uint32_t)((r & 63) >> 3), jin = (uint32_t)(r & 7) * 2;
     auto joff = [&](int t) -> uint32_t { return jblk + t * 128 + ((jch ^ (t & 7)) << 4) + jin; };
-    int issued = 0, waited = 0;
-    auto load = [&](int c) {   // thread 0: chunk g0 + c
+    // Loads per chunk, in two groups: A (i, the saved state) once the chunk before's MMAs have read
+    // Ib and Sb; B (log f, di, d log f) once its epilogue and stores are done (prefetched to L2
+    // while it is on the tensor cores).  Counted in chunks walked.
+    int issuedA = 0, issuedB = 0, waited = 0;
+    auto load_a = [&](int c) {   // thread 0: chunk g0 + c
         const int tok = (g0 + c) * kTile, slot = bh * p.ntiles + g0 + c;
-        mbar_arrive_expect_tx(&m->full, 5 * kTileBytes);
+        mbar_arrive_expect_tx(&m->fullA, 2 * kTileBytes);
         for (int k = 0; k < 2; ++k) {
-            tma_load_4d(Lb + k * kBlk, &tm_lf, &m->full, 64 * k, h, tok, b);
-            tma_load_4d(Ib + k * kBlk, &tm_x, &m->full, 64 * k, h, tok, b);
-            tma_load_4d(Sb + k * kBlk, &tm_st, &m->full, 64 * k, 0, 0, slot);
-            tma_load_4d(DIb + k * kBlk, &tm_di, &m->full, 64 * k, h, tok, b);
-            tma_load_4d(DLb + k * kBlk, &tm_dlf, &m->full, 64 * k, h, tok, b);
+            tma_load_4d(Ib + k * kBlk, &tm_x, &m->fullA, 64 * k, h, tok, b);
+            tma_load_4d(Sb + k * kBlk, &tm_st, &m->fullA, 64 * k, 0, 0, slot);
         }
-        ++issued;
+        ++issuedA;
+    };
+    auto load_b = [&](int c) {
+        const int tok = (g0 + c) * kTile;
+        mbar_arrive_expect_tx(&m->fullB, 3 * kTileBytes);
+        for (int k = 0; k < 2; ++k) {
+            tma_load_4d(Lb + k * kBlk, &tm_lf, &m->fullB, 64 * k, h, tok, b);
+            tma_load_4d(DIb + k * kBlk, &tm_di, &m->fullB, 64 * k, h, tok, b);
+            tma_load_4d(DLb + k * kBlk, &tm_dlf, &m->fullB, 64 * k, h, tok, b);
+        }
+        ++issuedB;
     };
 
     grid_dep_wait();   // the segments' outputs and the scan's gradients are complete from here on
+    const bool flagged = p.flags[bh] != 0;
+    if (!flagged && tid == 0) {   // the last chunk's tiles, while the carried gradient is read
+        load_a(N - 1);
+        load_b(N - 1);
+    }
     float Dr[64];      // the carried gradient, row r, columns 64 ch .. 64 ch + 63
     float dmax = 0.0f, decay = 1.0f;
     {
@@ -1318,8 +1334,7 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
         for (int i = 0; i < 64; ++i) dmax = fmaxf(dmax, fabsf(Dr[i]));
     }
     bool ok = true;
-    bool go = !p.flags[bh] && __syncthreads_or(dmax >= kStop);
-    if (go && tid == 0) load(N - 1);
+    bool go = !flagged && __syncthreads_or(dmax >= kStop);
     for (int c = N - 1; go && c >= 0; --c) {
         const int tok = (g0 + c) * kTile;
         // bf16(D) -> X (row r = key dim, columns = value dims)
@@ -1332,7 +1347,10 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
                 store_chunk_bf16(X, r, 2 * ch + hh, v);
             }
         }
-        if (__syncthreads_or(!mbar_wait(&m->full, waited & 1))) { ok = false; break; }
+        if (__syncthreads_or(!mbar_wait(&m->fullA, waited & 1) || !mbar_wait(&m->fullB, waited & 1))) {
+            ok = false;
+            break;
+        }
         ++waited;
         // rowsum(S_r * D), this thread's half of row r
         {
@@ -1409,9 +1427,20 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
                 mma_bf16_ss(tbase + 128, sdesc_add(dXk, ko), sdesc_add(dI, ko), id_kk, kk > 0);
             }
             mma_commit(&m->barM);
+            if (c > 0) {   // the chunk before's log f, di, d log f into L2 for its loads after the stores
+                const int tp = (g0 + c - 1) * kTile;
+                for (int k = 0; k < 2; ++k) {
+                    tma_prefetch_l2_4d(&tm_lf, 64 * k, h, tp, b);
+                    tma_prefetch_l2_4d(&tm_di, 64 * k, h, tp, b);
+                    tma_prefetch_l2_4d(&tm_dlf, 64 * k, h, tp, b);
+                }
+            }
         }
         if (__syncthreads_or(!mbar_wait(&m->barM, (N - 1 - c) & 1))) { ok = false; break; }   // chunk N-1-c walked
         tc_fence_after();
+        // whether the chunk before will be walked: the carried gradient after this chunk's decay
+        const bool next = __syncthreads_or(decay * __expf(m->BT[r]) * dmax >= kStop) && c > 0;
+        if (next && tid == 0) load_a(c - 1);   // Ib and Sb were read by the MMAs above
         if (ch == 1) {
             // di row r (token) += DI row r
 #pragma unroll
@@ -1433,27 +1462,33 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
                 store_chunk_bf16(DIb, r, cc, v);
             }
         } else {
-            // d log f column r (key dim) over the chunk's tokens, in order
+            // d log f column r (key dim) over the chunk's tokens, in order, 32 tokens at a time:
+            // their log f and d log f first, then the running sums in registers, then the stores
             const float Bt = m->BT[r];
             const float rho = 0.5f * Bt;
             const float base = __expf(Bt - rho) * (m->Rp[0][r] + m->Rp[1][r]);   // e^{B} rowsum(S_in * D)
             float bsum = 0.0f, pre = 0.0f;
 #pragma unroll 1
             for (int cb = 0; cb < 4; ++cb) {
-                float y[32];
+                float y[32], av[32], dv[32];
                 tmem_ld32(tl + 128 + 32 * cb, y);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    av[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Lb + joff(32 * cb + i)));
+                    dv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(DLb + joff(32 * cb + i)));
+                }
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int t = 32 * cb + i;
-                    const float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Lb + joff(t)));
-                    bsum += a;
-                    const float f = __expf(a);
+                    bsum += av[i];
+                    const float f = __expf(av[i]);
                     const float dK = __expf(Bt - bsum) * y[i];
-                    __nv_bfloat16 *dl = reinterpret_cast<__nv_bfloat16 *>(DLb + joff(t));
-                    *dl = __float2bfloat16_rn(__bfloat162float(*dl) + (base + pre - f * dK));
+                    dv[i] += base + pre - f * dK;
                     pre = fmaf(1.0f - f, dK, pre);
                 }
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(DLb + joff(32 * cb + i)) = __float2bfloat16_rn(dv[i]);
             }
         }
         // the carried gradient into the chunk before
@@ -1463,23 +1498,25 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
         for (int i = 0; i < 64; ++i) Dr[i] *= eb;
         fence_proxy_async_smem();
         tc_fence_before();
-        const bool next = __syncthreads_or(decay * dmax >= kStop) && c > 0;
+        __syncthreads();
         if (tid == 0) {
             for (int k = 0; k < 2; ++k) {
                 tma_store_4d(&tm_di, DIb + k * kBlk, 64 * k, h, tok, b);
                 tma_store_4d(&tm_dlf, DLb + k * kBlk, 64 * k, h, tok, b);
             }
             tma_store_commit();
-            if (next) {   // the tiles, once this chunk's stores have read them
+            if (next) {   // log f, di, d log f tiles, once this chunk's stores have read them
                 tma_store_wait_read0();
-                load(c - 1);
+                load_b(c - 1);
             }
         }
         go = next;
     }
     if (tid == 0) {
         if (!ok) set_status(HGRN2_ERR_TIMEOUT);
-        for (int k = waited; k < issued; ++k) mbar_wait(&m->full, k & 1, 2000000u);
+        // loads still landing: the last chunk's when nothing was walked, or any after a timeout
+        for (int k = waited; k < issuedA; ++k) mbar_wait(&m->fullA, k & 1, 2000000u);
+        for (int k = waited; k < issuedB; ++k) mbar_wait(&m->fullB, k & 1, 2000000u);
         tma_store_wait_all0();
     }
     tc_fence_before();

@@ -1237,6 +1237,14 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tma_store_wait_read0();
                 load_qg(c + 1);
                 load_o(c + 1);
+            } else if (next) {   // one stage: the next chunk's tiles into L2 for its loads after the stores
+                const int tn = (g0 + c + 1) * kTile, sn = bh * p.ntiles + g0 + c + 1;
+                for (int k = 0; k < 2; ++k) {
+                    tma_prefetch_l2_4d(&tm_q, 64 * k, h, tn, b);
+                    tma_prefetch_l2_4d(&tm_lf, 64 * k, h, tn, b);
+                    tma_prefetch_l2_4d(&tm_o, 64 * k, h, tn, b);
+                    tma_prefetch_l2_4d(&tm_st, 64 * k, 0, 0, sn);
+                }
             }
         }
         if (__syncthreads_or(!mbar_wait(&m->fullO[s], par) || !mbar_wait(&m->barM, c & 1))) { ok = false; break; }
