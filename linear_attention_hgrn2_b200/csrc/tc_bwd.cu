@@ -1232,6 +1232,7 @@ struct Misc {
     float Ppart[4][128];   // 32-row range sums of log f
     float BT[128];         // the chunk's total log decay B, key dim
     float Rp[2][128];      // halves of rowsum(S_r * D)
+    float Pre0[128];       // the first 64 tokens' sum of k dK, key dim
 };
 // log f, i, saved state (then Kd), di, d log f, bf16(D)
 constexpr size_t kSmem = 6 * (size_t)kTileBytes + sizeof(Misc);
@@ -1441,41 +1442,44 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
         // whether the chunk before will be walked: the carried gradient after this chunk's decay
         const bool next = __syncthreads_or(decay * __expf(m->BT[r]) * dmax >= kStop) && c > 0;
         if (next && tid == 0) load_a(c - 1);   // Ib and Sb were read by the MMAs above
-        if (ch == 1) {
-            // di row r (token) += DI row r
+        // di row r (token) += DI row r: this half's 64 columns
+#pragma unroll 1
+        for (int cc = 2 * ch; cc < 2 * ch + 2; ++cc) {
+            float v[32];
+            tmem_ld32(tl + 32 * cc, v);
+            tmem_wait_ld();
+            const uint8_t *base = DIb + (cc >> 1) * kBlk + r * 128;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float v[32];
-                tmem_ld32(tl + 32 * cc, v);
-                tmem_wait_ld();
-                const uint8_t *base = DIb + (cc >> 1) * kBlk + r * 128;
+            for (int qd = 0; qd < 4; ++qd) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int qd = 0; qd < 4; ++qd) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(base + (((4 * (cc & 1) + qd) ^ (r & 7)) << 4));
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        v[8 * qd + 2 * k] += bf_lo(ws[k]);
-                        v[8 * qd + 2 * k + 1] += bf_hi(ws[k]);
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    v[8 * qd + 2 * k] += bf_lo(ws[k]);
+                    v[8 * qd + 2 * k + 1] += bf_hi(ws[k]);
                 }
-                store_chunk_bf16(DIb, r, cc, v);
             }
-        } else {
-            // d log f column r (key dim) over the chunk's tokens, in order, 32 tokens at a time:
-            // their log f and d log f first, then the running sums in registers, then the stores
+            store_chunk_bf16(DIb, r, cc, v);
+        }
+        // d log f column r (key dim), this half's 64 tokens in order, 32 at a time: their log f and
+        // d log f first, then the running sums in registers.  The second half's sum of k dK
+        // starts from the first half's total, exchanged through shared memory.
+        {
             const float Bt = m->BT[r];
             const float rho = 0.5f * Bt;
             const float base = __expf(Bt - rho) * (m->Rp[0][r] + m->Rp[1][r]);   // e^{B} rowsum(S_in * D)
-            float bsum = 0.0f, pre = 0.0f;
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                float y[32], av[32], dv[32];
-                tmem_ld32(tl + 128 + 32 * cb, y);
+            float bsum = ch ? m->Ppart[0][r] + m->Ppart[1][r] : 0.0f;   // log decay before the half
+            float pre = 0.0f;
+            float dv[64];   // d log f + this half's own terms
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                const int t0 = 64 * ch + 32 * cb;
+                float y[32], av[32];
+                tmem_ld32(tl + 128 + t0, y);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    av[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Lb + joff(32 * cb + i)));
-                    dv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(DLb + joff(32 * cb + i)));
+                    av[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(Lb + joff(t0 + i)));
+                    dv[32 * cb + i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(DLb + joff(t0 + i)));
                 }
                 tmem_wait_ld();
 #pragma unroll
@@ -1483,13 +1487,16 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
                     bsum += av[i];
                     const float f = __expf(av[i]);
                     const float dK = __expf(Bt - bsum) * y[i];
-                    dv[i] += base + pre - f * dK;
+                    dv[32 * cb + i] += pre - f * dK;
                     pre = fmaf(1.0f - f, dK, pre);
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    *reinterpret_cast<__nv_bfloat16 *>(DLb + joff(32 * cb + i)) = __float2bfloat16_rn(dv[i]);
             }
+            if (ch == 0) m->Pre0[r] = pre;
+            __syncthreads();
+            const float off = base + (ch ? m->Pre0[r] : 0.0f);
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+                *reinterpret_cast<__nv_bfloat16 *>(DLb + joff(64 * ch + i)) = __float2bfloat16_rn(dv[i] + off);
         }
         // the carried gradient into the chunk before
         const float eb = __expf(m->BT[r]);
