@@ -989,7 +989,7 @@ scan_kernel(float *__restrict__ U, const float *__restrict__ g, int nseg, const 
 constexpr float kFixStop = 0x1p-24f;
 
 struct FixMisc {
-    uint64_t fullQG[2], fullO[2], barM;
+    uint64_t fullQG[2], fullO[2], barM, fullU[2];   // fullU: the segments' state slots
     uint32_t tmem_base;
     int pad;
     float EB[128];        // e^{B} of the chunk, key dim
@@ -1015,7 +1015,7 @@ struct FixParams {
 __global__ void __launch_bounds__(kThreads, 1)
 fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
              const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_st,
-             const __grid_constant__ CUtensorMap tm_qt, FixParams p) {
+             const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_u, FixParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int NS = p.save ? 1 : 2;   // stages
     // stage s: q, log f, o at smem + 3 s tiles (s = 0 with one stage)
@@ -1038,6 +1038,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int s = 0; s < 2; ++s) {
             mbar_init(&m->fullQG[s], 1);
             mbar_init(&m->fullO[s], 1);
+            mbar_init(&m->fullU[s], 1);
         }
         mbar_init(&m->barM, 1);
         fence_mbar_init();
@@ -1045,6 +1046,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tma_prefetch_desc(&tm_lf);
         tma_prefetch_desc(&tm_o);
         tma_prefetch_desc(&tm_qt);
+        tma_prefetch_desc(&tm_u);
     }
     if (warp == 0) {
         tmem_alloc(&m->tmem_base, 128);
@@ -1132,49 +1134,28 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     float S[64];          // the carried state, row r, columns 64 ch .. 64 ch + 63
     float smax = 0.0f;    // max |S| of the row's 64 columns as entered
     float decay = 1.0f;   // the carried decay of row r so far
-    // the entering state (loaded before the flag is known; unused for a flagged pair)
-    const size_t rowoff = (size_t)r * 128 + 64 * ch;
-    auto slot_row = [&](int sg) {
-        return reinterpret_cast<const float4 *>(p.U + ((size_t)bh * p.nseg + sg) * 16384 + rowoff);
+    const bool flagged = p.flags[bh] != 0;
+    const bool want_hT = p.merged && seg == p.nseg - 1 && (p.hT || p.hTs);
+    // The segments' state slots it reads, 64 KB each, staged through shared memory by TMA (tiles
+    // the first chunk does not use yet): merged, segments 0 .. seg-1 (and its own for hT); else
+    // the scan's slot seg-1.  Two buffers with two stages, one with one.
+    const int nslots = flagged ? 0 : p.merged ? seg + (want_hT ? 1 : 0) : 1;
+    const int nbuf = NS;
+    auto ubox = [&](int buf, int bx) -> uint8_t * {   // 32 columns x 128 rows of fp32, swizzled
+        if (NS == 2) return smem + (size_t)(3 + 2 * buf) * kTileBytes + (size_t)bx * 16384;
+        return smem + (size_t)(bx < 2 ? 1 : 4) * kTileBytes + (size_t)(bx & 1) * 16384;
     };
-    if (p.merged) {   // S_in = sum over the earlier segments' maps, two segments per round of loads
-#pragma unroll
-        for (int i = 0; i < 64; ++i) S[i] = 0.0f;
-        int mseg = 0;
-        for (; mseg + 1 < seg; mseg += 2) {
-            const float ga = p.g[((size_t)bh * p.nseg + mseg) * 128 + r];
-            const float gb = p.g[((size_t)bh * p.nseg + mseg + 1) * 128 + r];
-            const float4 *ua = slot_row(mseg), *ub = slot_row(mseg + 1);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float4 a = ua[i], c2 = ub[i];
-                S[4 * i] = fmaf(gb, fmaf(ga, S[4 * i], a.x), c2.x);
-                S[4 * i + 1] = fmaf(gb, fmaf(ga, S[4 * i + 1], a.y), c2.y);
-                S[4 * i + 2] = fmaf(gb, fmaf(ga, S[4 * i + 2], a.z), c2.z);
-                S[4 * i + 3] = fmaf(gb, fmaf(ga, S[4 * i + 3], a.w), c2.w);
-            }
-        }
-        if (mseg < seg) {
-            const float ga = p.g[((size_t)bh * p.nseg + mseg) * 128 + r];
-            const float4 *ua = slot_row(mseg);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float4 a = ua[i];
-                S[4 * i] = fmaf(ga, S[4 * i], a.x);
-                S[4 * i + 1] = fmaf(ga, S[4 * i + 1], a.y);
-                S[4 * i + 2] = fmaf(ga, S[4 * i + 2], a.z);
-                S[4 * i + 3] = fmaf(ga, S[4 * i + 3], a.w);
-            }
-        }
-    } else {
-        const float4 *src = slot_row(seg - 1);   // the scan's slot k-1
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 a = src[i];
-            S[4 * i] = a.x; S[4 * i + 1] = a.y; S[4 * i + 2] = a.z; S[4 * i + 3] = a.w;
-        }
-    }
-    if (!p.flags[bh]) {
+    auto slot_of = [&](int i) { return (size_t)bh * p.nseg + (p.merged ? i : seg - 1); };
+    int issuedU = 0, waitedU = 0;
+    auto load_u = [&](int i) {   // thread 0: slot i into buffer i % nbuf
+        const int buf = i % nbuf;
+        mbar_arrive_expect_tx(&m->fullU[buf], 4 * 16384);
+        for (int bx = 0; bx < 4; ++bx) tma_load_2d(ubox(buf, bx), &tm_u, &m->fullU[buf], 32 * bx, (int)slot_of(i) * 128);
+        ++issuedU;
+    };
+    if (tid == 0)
+        for (int i = 0; i < nslots && i < nbuf; ++i) load_u(i);
+    if (!flagged) {
         if (tid == 0) {   // the first chunk's tiles
             fence_proxy_async_global();
             load_qg(0);
@@ -1185,20 +1166,48 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             m->EB[tid] = __expf(B);
             m->ER[tid] = __expf(0.5f * B);
         }
-        if (p.merged && seg == p.nseg - 1 && (p.hT || p.hTs)) {   // the sequence's final state
-            const float gk = p.g[myslot * 128 + r];
-            const float4 *src = slot_row(seg);
-            float4 *d1 = p.hT ? reinterpret_cast<float4 *>(p.hT + (size_t)bh * 16384 + rowoff) : nullptr;
-            float4 *d2 = p.hTs ? reinterpret_cast<float4 *>(p.hTs + (size_t)bh * 16384 + rowoff) : nullptr;
+    }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float4 a = src[i];
-                const float4 w = make_float4(fmaf(gk, S[4 * i], a.x), fmaf(gk, S[4 * i + 1], a.y),
-                                             fmaf(gk, S[4 * i + 2], a.z), fmaf(gk, S[4 * i + 3], a.w));
-                if (d1) d1[i] = w;
-                if (d2) d2[i] = w;
+    for (int i = 0; i < 64; ++i) S[i] = 0.0f;
+    for (int i = 0; i < nslots; ++i) {
+        const int buf = i % nbuf;
+        if (__syncthreads_or(!mbar_wait(&m->fullU[buf], (i / nbuf) & 1))) { ok = false; break; }
+        waitedU = i + 1;
+        float u[64];   // row r, columns 64 ch .. 64 ch + 63 of the slot
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+            const uint8_t *row = ubox(buf, 2 * ch + hb) + r * 128;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 a = *reinterpret_cast<const float4 *>(row + ((k ^ (r & 7)) << 4));
+                u[32 * hb + 4 * k] = a.x; u[32 * hb + 4 * k + 1] = a.y;
+                u[32 * hb + 4 * k + 2] = a.z; u[32 * hb + 4 * k + 3] = a.w;
             }
         }
+        if (!p.merged) {          // the scan's state entering this segment
+#pragma unroll
+            for (int k = 0; k < 64; ++k) S[k] = u[k];
+        } else if (i < seg) {     // S_in = Diag(g_i) S + U_i over the earlier segments
+            const float gi = p.g[slot_of(i) * 128 + r];
+#pragma unroll
+            for (int k = 0; k < 64; ++k) S[k] = fmaf(gi, S[k], u[k]);
+        } else {                  // the sequence's final state: Diag(g_k) S_in + U_k
+            const float gk = p.g[myslot * 128 + r];
+            const size_t rowoff = (size_t)bh * 16384 + (size_t)r * 128 + 64 * ch;
+            float4 *d1 = p.hT ? reinterpret_cast<float4 *>(p.hT + rowoff) : nullptr;
+            float4 *d2 = p.hTs ? reinterpret_cast<float4 *>(p.hTs + rowoff) : nullptr;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float4 w = make_float4(fmaf(gk, S[4 * k], u[4 * k]), fmaf(gk, S[4 * k + 1], u[4 * k + 1]),
+                                             fmaf(gk, S[4 * k + 2], u[4 * k + 2]), fmaf(gk, S[4 * k + 3], u[4 * k + 3]));
+                if (d1) d1[k] = w;
+                if (d2) d2[k] = w;
+            }
+        }
+        __syncthreads();   // the buffer has been read
+        if (tid == 0 && i + nbuf < nslots) load_u(i + nbuf);
+    }
+    if (!flagged && ok) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) smax = fmaxf(smax, fabsf(S[i]));
         go = __syncthreads_or(smax >= kFixStop);
@@ -1319,6 +1328,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (!ok) set_status(HGRN2_ERR_TIMEOUT);
         // loads still in flight: the first chunk's when the carried state was negligible, or
         // any after a timeout
+        for (int k = waitedU; k < issuedU; ++k) mbar_wait(&m->fullU[k % nbuf], (k / nbuf) & 1, 2000000u);
         for (int k = waited_qg; k < issued_qg; ++k) mbar_wait(&m->fullQG[NS == 2 ? (k & 1) : 0], (k / NS) & 1, 2000000u);
         for (int k = waited_o; k < issued_o; ++k) mbar_wait(&m->fullO[NS == 2 ? (k & 1) : 0], (k / NS) & 1, 2000000u);
         tma_store_wait_all0();
@@ -1457,15 +1467,15 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
                              (const int *)a.flags, a.hT, a.st16 ? a.hTs : nullptr);
         if (e != cudaSuccess) return e;
     }
-    CUtensorMap mqt;   // the first chunks' q e^{b}: 128-row tiles, one per segment slot
-    if (!make_token_map(&mqt, qtil, (int)nsl, 128, 1)) return cudaErrorInvalidValue;
+    CUtensorMap mqt, mu;   // the first chunks' q e^{b}: 128-row tiles, one per segment slot; the state slots
+    if (!make_token_map(&mqt, qtil, (int)nsl, 128, 1) || !make_state_map(&mu, U, nsl * 128)) return cudaErrorInvalidValue;
     const size_t fsm = tcf::fix_smem(a.st16 != nullptr);
     e = cudaFuncSetAttribute(tcf::fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
     if (e != cudaSuccess) return e;
     tcf::FixParams fp{U, g, bs, a.flags, merged ? a.hT : nullptr, merged && a.st16 ? a.hTs : nullptr,
                       a.H, nseg, tps, ntiles, a.st16 != nullptr, merged};
     e = launch_dependent(tcf::fixup_kernel, dim3(BH * (nseg - 1)), dim3(tcf::kThreads), fsm, st, mq, ml, mo, mst,
-                         mqt, fp);
+                         mqt, mu, fp);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
