@@ -33,7 +33,10 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
  *    stream).  Argument checks run on the host before anything is launched: a
  *    call that returns an error has launched nothing.  A launch failure reported
- *    by the CUDA runtime returns HGRN2_ERR_CUDA.
+ *    by the CUDA runtime returns HGRN2_ERR_CUDA.  Everything a call puts on the
+ *    stream (kernel launches, some as programmatic dependents of the launch
+ *    before them, and cudaMemsetAsync of workspace or outputs) is stream-ordered,
+ *    so a call can be captured into a CUDA graph (hgrn2_bwd_noalloc: see there).
  *  - No exception or abort crosses this ABI.
  *  - Supported sizes: B, H >= 1; T >= 0 (T = 0 writes hT = h0 and nothing else);
  *    1 <= d_k, d_v <= 256; chunk in {16, 32, 64, 128}.  The bf16 tensor-core

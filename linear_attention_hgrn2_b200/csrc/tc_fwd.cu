@@ -112,6 +112,11 @@ struct Params {
     __nv_bfloat16 *qtil;
     float *bseg;
     __nv_bfloat16 *opart;   // heads read in place: the exact route's partial outputs
+    // Final states (hT, the saved final state, or a segment's U) leave through shared memory by
+    // TMA: tm_h1 / tm_h2 map them as fp32 [rows][128] (bit 0 / bit 1 of hmaps set when mapped;
+    // d = 128 only); h1row0 / h2row0: this CTA's first row = its slot times 128.
+    int hmaps;
+    int hslot1, hslot2;   // 0: the pair's index; 1: the segment slot (b,h) nseg + seg
 };
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
@@ -127,7 +132,8 @@ template <bool kPacked, bool kScalar = false, bool kSeg = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
            const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_o,
-           const __grid_constant__ CUtensorMap tm_st, Params p) {
+           const __grid_constant__ CUtensorMap tm_st, const __grid_constant__ CUtensorMap tm_h1,
+           const __grid_constant__ CUtensorMap tm_h2, Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *Qb[2] = {smem, smem + 3 * kTileBytes};
     uint8_t *Gb[2] = {smem + kTileBytes, smem + 4 * kTileBytes};
@@ -457,20 +463,49 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         if (n == N && !fail && (p.nseg > 1 || ((p.hT || p.hTs) && seg == p.nseg - 1)) && r < p.D) {   // warp-uniform
             const float e = e_cur;   // hT (or the segment's U) = Diag(e^{B - rho}) S' of the last chunk
-            float *dst = p.nseg > 1 ? p.Useg + (((size_t)bh * p.nseg + seg) * 128 + r) * 128
-                                    : p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
-            float *dsv = p.nseg > 1 ? nullptr : p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
+            if (p.hmaps) {
+                // d = 128: every row into four swizzled 32-column boxes of fp32 in the (now idle) first
+                // two ring tiles, then TMA stores (the group's condition here is uniform: all 128
+                // threads finished the loop together, and r < 128)
+                uint8_t *stg = smem;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (32 * c >= p.D) break;
-                float v[32];
-                tmem_ld32(tl + kColS + 32 * c, v);
-                tmem_wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tl + kColS + 32 * c, v);
+                    tmem_wait_ld();
+                    uint8_t *row = stg + (size_t)c * 16384 + r * 128;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 w = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
-                    if (dst) reinterpret_cast<float4 *>(dst + 32 * c)[i] = w;
-                    if (dsv) reinterpret_cast<float4 *>(dsv + 32 * c)[i] = w;
+                    for (int k = 0; k < 8; ++k)
+                        *reinterpret_cast<float4 *>(row + ((k ^ (r & 7)) << 4)) =
+                            make_float4(v[4 * k] * e, v[4 * k + 1] * e, v[4 * k + 2] * e, v[4 * k + 3] * e);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(2, 128);
+                if (r == 0) {
+                    const int seg_slot = bh * p.nseg + seg;
+                    for (int c = 0; c < 4; ++c) {
+                        if (p.hmaps & 1) tma_store_2d(&tm_h1, stg + (size_t)c * 16384, 32 * c, (p.hslot1 ? seg_slot : bh) * 128);
+                        if (p.hmaps & 2) tma_store_2d(&tm_h2, stg + (size_t)c * 16384, 32 * c, (p.hslot2 ? seg_slot : bh) * 128);
+                    }
+                    tma_store_commit();
+                    tma_store_wait_all0();
+                }
+            } else {
+                float *dst = p.nseg > 1 ? p.Useg + (((size_t)bh * p.nseg + seg) * 128 + r) * 128
+                                        : p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
+                float *dsv = p.nseg > 1 ? nullptr : p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (32 * c >= p.D) break;
+                    float v[32];
+                    tmem_ld32(tl + kColS + 32 * c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 w = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
+                        if (dst) reinterpret_cast<float4 *>(dst + 32 * c)[i] = w;
+                        if (dsv) reinterpret_cast<float4 *>(dsv + 32 * c)[i] = w;
+                    }
                 }
             }
         }
@@ -1454,8 +1489,16 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
                   (const __nv_bfloat16 *)a.x, a.simt_C, a.flags, U, g, a.T, a.H, ntiles, nseg, tps,
                   a.st16 != nullptr, a.st16 ? a.hTs : nullptr, a.cu, a.perm, a.D,
                   (const __nv_bfloat16 *)a.lgs, seg_done, a.nK, a.nV, Bm,
-                  nseg > 1 ? qtil : nullptr, nseg > 1 ? bs : nullptr, (__nv_bfloat16 *)a.opart};
-    kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, p);
+                  nseg > 1 ? qtil : nullptr, nseg > 1 ? bs : nullptr, (__nv_bfloat16 *)a.opart, 0, 0, 0};
+    // the segments' final states U leave through shared memory by TMA (measured: U stores 4 us
+    // sooner on the long sequence; for one CTA per pair the row stores of hT, whose drain does not
+    // hold the CTA, measured 1 us faster than the TMA store and its wait)
+    CUtensorMap mh1 = mo, mh2 = mo;
+    if (a.D == 128 && nseg > 1 && U && make_state_map(&mh1, U, (size_t)BH * nseg * 128)) {
+        p.hmaps = 1;
+        p.hslot1 = 1;
+    }
+    kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, mh1, mh2, p);
     if ((e = cudaGetLastError()) != cudaSuccess || nseg == 1) return e;
     // segments: the states entering them (and hT), then the carried states' contributions.  With
     // few segments the fix-up sums the states itself; else the scan kernel chains them first.
