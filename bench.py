@@ -594,8 +594,9 @@ def run_head_dim(args, dev, pk, rank, w, seed_off, ref_ms=None):
     if ref_ms:
         res["step_time_vs_headline"] = round(ms / ref_ms, 4)
     if w.dk > 128 or w.dv > 128:
-        res["route"] = ("128-wide half-head blocks on the tensor cores, read in place; partial outputs added in "
-                        "fp32; bwd_frac counts the algorithmic bytes of the wide head only")
+        res["route"] = ("128-wide half-head blocks on the tensor cores, read in place; each block pair adds its "
+                        "share of the outputs by TMA reduce-add into zeroed outputs; bwd_frac counts the algorithmic "
+                        "bytes of the wide head only")
     del inp, q, lf, x, dO, sv, o
     torch.cuda.empty_cache()
     return res
