@@ -123,6 +123,25 @@ size_t ws_bytes_base(int B, int H, int dk, int dv, hgrn2_dtype dt, int want_bwd)
     if (use_tc(dk, dv, dt)) bytes += align256(sizeof(int) * (size_t)B * H);  // exact-route flags
     return bytes;
 }
+// The backward without saved states for few (b,h) (sequence segments): it runs the training
+// forward into its workspace and then the saved-state backward, which both run in segments,
+// instead of one CTA per (b,h) walking every chunk twice.
+bool segmented_recompute(int B, int T, int H, int dk, int dv, hgrn2_dtype dt) {
+    return dt == HGRN2_BF16 && dk == 128 && dv == 128 && T > 0 && tc_bwd_workspace(B, T, H) > 0;
+}
+struct RecomputeLayout {
+    size_t saved, o, fws, total;   // offsets of the saved buffer, the o scratch, the forward's workspace
+};
+size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd, bool tc64);
+// [the saved-state backward's workspace][saved buffer][o scratch][the forward's workspace]
+RecomputeLayout recompute_layout(int B, int T, int H, int dv, hgrn2_dtype dt) {
+    RecomputeLayout l;
+    l.saved = ws_bytes_needed(B, T, H, 128, dv, 64, dt, 2, false);
+    l.o = l.saved + align256(saved_layout(B, T, H).total);
+    l.fws = l.o + align256((size_t)B * T * H * dv * 2);
+    l.total = l.fws + ws_bytes_needed(B, T, H, 128, dv, 64, dt, 0, true);
+    return l;
+}
 size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dtype dt, int want_bwd,
                        bool tc64 = true) {
     if (is_wide(dk, dv))
@@ -131,6 +150,7 @@ size_t ws_bytes_needed(int B, int T, int H, int dk, int dv, int chunk, hgrn2_dty
     size_t bytes = ws_bytes_base(B, H, dk, dv, dt, want_bwd);
     if (!want_bwd && use_tc(dk, dv, dt) && dk == 128 && T > 0) bytes += align256(tc_fwd_workspace(B, T, H));
     if (want_bwd == 2 && use_tc(dk, dv, dt) && dk == 128 && T > 0) bytes += align256(tc_bwd_workspace(B, T, H));
+    if (want_bwd == 1 && tc64 && segmented_recompute(B, T, H, dk, dv, dt)) bytes = recompute_layout(B, T, H, dv, dt).total;
     if (want_bwd && tc64 && use_tc(dk, dv, dt) && dk == 64 && T > 0)   // saved states + o scratch
         bytes += saved_layout(B, T, H).total + align256((size_t)B * T * H * dv * 2);
     return bytes;
@@ -365,6 +385,17 @@ hgrn2_status bwd_impl(const void *q, const void *log_f, const void *i, const flo
         if (st != HGRN2_OK) return st;
         return bwd_impl(q, log_f, i, h0, sv, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype, workspace,
                         base, stream);
+    }
+    if (!saved && !cu && tc64 && segmented_recompute(B, T, H, dk, dv, dtype)) {
+        // few (b,h): the training forward (segments) into the workspace, then the saved-state
+        // backward (segments)
+        const RecomputeLayout l = recompute_layout(B, T, H, dv, dtype);
+        char *sv = (char *)workspace + l.saved;
+        hgrn2_status st = fwd_impl(q, log_f, i, h0, sv + (l.o - l.saved), nullptr, sv, B, T, H, dk, dv, chunk, dtype,
+                                   (char *)workspace + l.fws, l.total - l.fws, stream);
+        if (st != HGRN2_OK) return st;
+        return bwd_impl(q, log_f, i, h0, sv, dO, dhT, dq, dlog_f, di, dh0, B, T, H, dk, dv, chunk, dtype, workspace,
+                        l.saved, stream);
     }
     if (T == 0) {
         if (!dh0) return HGRN2_OK;
