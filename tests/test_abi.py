@@ -208,10 +208,19 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
         ns = min(max(1, 148 // (B * H)), ntiles)
         tps = (ntiles + ns - 1) // ns
         return (ntiles + tps - 1) // tps
+    # Without saved states and with segments, the backward runs the training forward into its
+    # workspace and then the saved-state backward: room for both, the saved buffer and an o scratch.
     for (B, T, H) in ((2, 300, 3), (1, 32768, 8), (8, 2048, 16)):
         ns = nseg(B, T, H)
         seg = up(B * H * ns * (128 * 128 + 128) * 4) if ns > 1 else 0
-        assert f(B, T, H, 128, 128, 64, L.BF16, 2) == f(B, T, H, 128, 128, 64, L.BF16, 1) + seg, (B, T, H)
+        base = up(B * H * 128 * 4) + up(B * H * 4)   # rowsum(dhT * hT), exact-route flags
+        assert f(B, T, H, 128, 128, 64, L.BF16, 2) == base + seg, (B, T, H)
+        if ns > 1:
+            extra = up(lib.hgrn2_saved_size(B, T, H, 128, 128, L.BF16)) + up(B * T * H * 128 * 2) + \
+                f(B, T, H, 128, 128, 64, L.BF16, 0)
+            assert f(B, T, H, 128, 128, 64, L.BF16, 1) == base + seg + extra, (B, T, H)
+        else:
+            assert f(B, T, H, 128, 128, 64, L.BF16, 1) == base, (B, T, H)
     assert nseg(8, 2048, 16) == 1 and nseg(1, 32768, 8) == 18
     assert f(B, T, H, 64, 64, 64, L.BF16, 3) == bad
     assert f(B, T, H, 64, 64, 64, L.BF16, -1) == bad

@@ -384,24 +384,26 @@ def test_segmented_forward_few_segments(cuda, saved, lb):
             assert e <= 2e-2, (name, b, h, e)
 
 
+@pytest.mark.parametrize("saved", [True, False], ids=["saved", "recompute"])
 @pytest.mark.parametrize("lb,T", [(0.9, 32768), (0.0, 4096)])
-def test_segmented_backward_long_sequence(cuda, lb, T):
+def test_segmented_backward_long_sequence(cuda, lb, T, saved):
     # B*H = 8, the long workload's shape as a training pair: the saved-state backward runs in
     # segments (18 of 15 chunks per pair at T = 32768; 16 of 2 at T = 4096): every segment's reverse
-    # sweep from a zero
-    # gradient (the last from dhT), the reverse scan of their maps (giving dh0), then the carried
-    # gradients added to di and d log f of each segment's last chunks.  lb = 0: strong decay.
+    # sweep from a zero gradient (the last from dhT), the reverse scan of their maps (giving dh0),
+    # then the carried gradients added to di and d log f of each segment's last chunks.  Without
+    # saved states the backward first runs the training forward into its workspace (3 more
+    # launches).  lb = 0: strong decay.
     B, H = 1, 8
     inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, lb, seed=1090 + T, h0_sigma=0.1, with_dO=True,
                         dhT_sigma=0.1)
     g = to_cuda(inp)
-    sv = L.new_saved(g["q"])
+    sv = L.new_saved(g["q"]) if saved else None
     o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
     L.counters(reset=True)
     dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
                              saved=sv)
     c = L.counters(reset=True)
-    assert c[2] == 3 and c[0] == 0, c
+    assert c[2] == (3 if saved else 6) and c[0] == 0, c
     assert L.device_status() == L.OK
     pairs = [(0, 0), (0, 5)]
     ref = oracle_heads(inp, pairs, want_bwd=True, dhT=inp["dhT"])
