@@ -609,6 +609,19 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int quad = warp & 3, q4 = warp >> 2;
     const int j = 32 * quad + lane;      // TMEM lane / key dim / tile row
     const int c0 = 32 * q4;              // this thread's 32 TMEM columns (or rows, in the prep)
+    const int nblk = p.D >> 6;   // 64-column blocks loaded and stored per tile
+    int *issued = m->issued, *waited = m->waited;   // thread 0 issues; waits are recorded by thread 0
+    // two token tiles of one side (q, log f: key side, hk; i, dO: value side, hv)
+    auto issue2 = [&](uint8_t *d0, const CUtensorMap *t0, uint8_t *d1, const CUtensorMap *t1, uint64_t *bar,
+                      int q, int n) {
+        ++issued[q];
+        const int hh = q == 0 ? hk : hv;
+        mbar_arrive_expect_tx(bar, 2 * nblk * kBlk);
+        for (int c = 0; c < nblk; ++c) {
+            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, hh, tok0 + n * kTile, bc);
+            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, hh, tok0 + n * kTile, bc);
+        }
+    };
     if (tid == 0) {
         mbar_init(&m->barIn, 1);
         mbar_init(&m->barVO, 1);
@@ -619,12 +632,18 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mbar_init(&m->barDS, kRevThreads);
         mbar_init(&m->barD16, 1);
         fence_mbar_init();
+        for (int q = 0; q < 3; ++q) issued[q] = waited[q] = 0;
+        // the last chunk's tiles before the TMEM allocation and the block barrier (the d = 64 zero
+        // fill below writes only the tiles' upper halves, which TMA does not load)
+        if (N > 0) {
+            issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, N - 1);
+            issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, N - 1);
+        }
     }
     if (warp == 0) {
         tmem_alloc(&m->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    const int nblk = p.D >> 6;   // 64-column blocks loaded and stored per tile
     if (nblk == 1) {             // d = 64: the unloaded halves of the input tiles stay zero
         for (int i = tid; i < 4 * (int)(kBlk / 16); i += kRevThreads) {
             const int t = i / (int)(kBlk / 16), o = i - t * (int)(kBlk / 16);
@@ -639,24 +658,6 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t tbase = m->tmem_base;
     const uint32_t tl = tbase + ((uint32_t)(32 * quad) << 16);
 
-    int *issued = m->issued, *waited = m->waited;   // thread 0 issues; waits are recorded by thread 0
-    if (tid == 0)
-        for (int q = 0; q < 3; ++q) issued[q] = waited[q] = 0;
-    // two token tiles of one side (q, log f: key side, hk; i, dO: value side, hv)
-    auto issue2 = [&](uint8_t *d0, const CUtensorMap *t0, uint8_t *d1, const CUtensorMap *t1, uint64_t *bar,
-                      int q, int n) {
-        ++issued[q];
-        const int hh = q == 0 ? hk : hv;
-        mbar_arrive_expect_tx(bar, 2 * nblk * kBlk);
-        for (int c = 0; c < nblk; ++c) {
-            tma_load_4d(d0 + c * kBlk, t0, bar, 64 * c, hh, tok0 + n * kTile, bc);
-            tma_load_4d(d1 + c * kBlk, t1, bar, 64 * c, hh, tok0 + n * kTile, bc);
-        }
-    };
-    if (tid == 0 && N > 0) {
-        issue2(Qb, &tm_q, Gb, &tm_lf, &m->barIn, 0, N - 1);
-        issue2(Vb, &tm_x, Ob, &tm_do, &m->barVO, 1, N - 1);
-    }
     {   // dS = dhT (or 0); carry = rowsum(dhT * hT) (or 0)
         float v[32];
         float part = 0.0f;   // saved mode: this quarter's share of rowsum(dhT * hT)

@@ -172,6 +172,25 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         if (tid == 0) set_status(HGRN2_ERR_DEVICE);
         return;
     }
+    const int nblk = p.D >> 6;   // 64-column blocks loaded and stored per tile
+    int issued_qg = 0, issued_v = 0;   // producer (thread 0): loads issued per barrier pair
+    // chunk n's q and log f into stage n & 1, and its i (thread 0)
+    auto load_qg = [&](int n) {
+        const int s = n & 1;
+        mbar_arrive_expect_tx(&m->fullQG[s], 2 * nblk * kBlk);
+        for (int c = 0; c < nblk; ++c) {
+            tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, hk, tok0 + n * kTile, bc);
+            tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, hk, tok0 + n * kTile, bc);
+        }
+        ++issued_qg;
+    };
+    auto load_v = [&](int n) {
+        const int s = n & 1;
+        mbar_arrive_expect_tx(&m->fullV[s], nblk * kBlk);
+        for (int c = 0; c < nblk; ++c)
+            tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, hv, tok0 + n * kTile, bc);
+        ++issued_v;
+    };
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&m->fullQG[s], 1);
@@ -191,6 +210,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         m->waited_full = 0;
         m->waited_v = 0;
         fence_mbar_init();
+        // the first chunk's tiles before the TMEM allocation and the block barrier (the d = 64
+        // zero fill below writes only the tiles' upper halves, which TMA does not load)
+        if (N > 0) {
+            load_qg(0);
+            load_v(0);
+        }
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_lf);
         tma_prefetch_desc(&tm_x);
@@ -200,7 +225,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tmem_alloc(&m->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    const int nblk = p.D >> 6;   // 64-column blocks loaded and stored per tile
     if (nblk == 1) {             // d = 64: the unloaded halves of the input tiles stay zero
         for (int i = tid; i < 6 * (int)(kBlk / 16); i += kFwdThreads) {
             const int t = i / (int)(kBlk / 16), o = i - t * (int)(kBlk / 16);
@@ -213,28 +237,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = m->tmem_base;
-    int issued_qg = 0, issued_v = 0;   // producer: loads issued per barrier pair
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            for (int n = 0; n < N; ++n) {
+            for (int n = 1; n < N; ++n) {   // chunk 0's loads went out with the set-up
                 const int s = n & 1;
                 if (ld_volatile(&m->bad_tile) < n) break;
                 // q and log f once the state MMA of chunk n-2 has read Qt, Kt; i once its last
                 // MMA has read v
                 if (n >= 2 && !wait_or_abort(&m->emptyQG[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
-                mbar_arrive_expect_tx(&m->fullQG[s], 2 * nblk * kBlk);
-                for (int c = 0; c < nblk; ++c) {
-                    tma_load_4d(Qb[s] + c * kBlk, &tm_q, &m->fullQG[s], 64 * c, hk, tok0 + n * kTile, bc);
-                    tma_load_4d(Gb[s] + c * kBlk, &tm_lf, &m->fullQG[s], 64 * c, hk, tok0 + n * kTile, bc);
-                }
-                ++issued_qg;
+                load_qg(n);
                 if (n >= 2 && !wait_or_abort(&m->emptyV[s], ((n - 2) >> 1) & 1, &m->bad_tile, n - 2)) break;
-                mbar_arrive_expect_tx(&m->fullV[s], nblk * kBlk);
-                for (int c = 0; c < nblk; ++c)
-                    tma_load_4d(Vb[s] + c * kBlk, &tm_x, &m->fullV[s], 64 * c, hv, tok0 + n * kTile, bc);
-                ++issued_v;
+                load_v(n);
             }
         }
     } else if (warp == 1) {
