@@ -606,8 +606,8 @@ def run_fwd_configs(args, dev, pk, rank):
     """The two forward-only workloads: the forward layer (B=4, H=8, T=2048, lb=0.5) and the long
     sequence (B=1, H=8, T=32768, lb=0.9, h0 in, hT out).  With 32 and 8 (b,h) pairs they run the
     segmented forward: every segment from a zero state, then the carried states added to the
-    segments' first chunks (2 launches for the forward layer's 4 segments per pair; 3 for the
-    long sequence's 18, whose fp32 scan over segments is a launch of its own)."""
+    segments' first chunks by a fix-up that sums the entering states itself (2 launches: the
+    forward layer's 4 segments per pair, the long sequence's 18)."""
     import linear_attention_hgrn2_b200 as L
     from linear_attention_hgrn2_b200 import inputs as I
     res = {}

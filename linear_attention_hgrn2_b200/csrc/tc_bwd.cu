@@ -502,6 +502,9 @@ struct RevParams {
     // ([B*H][nseg][128])
     int nseg, tps;
     float *Wseg, *gseg;
+    // and sum_v |W[j,v]| over each quarter of the value dims ([B*H][nseg][128][4]; the fix-up's
+    // bound on what the maps it leaves out could add)
+    float *Wabs;
 };
 
 // kPacked (saved mode only): p.cu holds packed sequences; compiled apart so the dense path
@@ -527,7 +530,9 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     uint8_t *D16 = smem + 4 * kTileBytes, *AT = smem + 5 * kTileBytes, *DA = smem + 6 * kTileBytes;
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
-    if constexpr (kSeg) grid_dep_launch();   // the scan may be scheduled now; it waits for this grid
+    // (kSeg: no early trigger of the dependent scan or fix-up, as in the forward's segments: the
+    // fix-up scheduled at this kernel's start made the long-sequence backward slower, A/B on one
+    // B200 240.4 -> 224.9 us without the trigger.)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     static_assert(!kSeg || (kSaved && !kPacked && !kScalar && !kWide), "segments: saved mode, dense, per-dim");
     const int seg = kSeg ? (int)blockIdx.x % p.nseg : 0;
@@ -1154,9 +1159,14 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         tmem_wait_ld();
         const float e = g_later;   // dh0 = Diag(e^{rho}) dL/dS_r of the first chunk
         float4 *dst = reinterpret_cast<float4 *>(dhout + (size_t)j * p.D + c0);
+        float wabs = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
+        for (int i = 0; i < 8; ++i) {
+            const float4 w = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
+            wabs += (fabsf(w.x) + fabsf(w.y)) + (fabsf(w.z) + fabsf(w.w));
+            dst[i] = w;
+        }
+        if (kSeg && p.Wabs) p.Wabs[(((size_t)bh * p.nseg + seg) * 128 + j) * 4 + q4] = wabs;
     }
     if (tid == 0 && ok && n < 0) atomicAdd(&g_counters[1], (unsigned long long)N);
     tc_fence_before();
@@ -1173,7 +1183,8 @@ rev_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 // In fp32, in place: slot k of W becomes D_{k-1} (k >= 1); slot 0 gives dh0.  Flagged pairs
 // (recomputed whole on the exact route) are left alone.  One thread per 4 consecutive elements
 // of one (batch, head); the maps are loaded 16 segments at a time.  A programmatic dependent of
-// the segments' kernel.
+// the segments' kernel.  Used beyond kBwdMergedMax segments per pair; with fewer, the fix-up
+// sums what it needs of the maps itself.
 __global__ void __launch_bounds__(256)
 bwd_scan_kernel(float *__restrict__ W, const float *__restrict__ g, int nseg, const int *__restrict__ flags,
                 float *__restrict__ dh0) {
@@ -1224,8 +1235,14 @@ bwd_scan_kernel(float *__restrict__ W, const float *__restrict__ g, int nseg, co
 // Y^T = bf16(D) I^T (lane j), Kd = k e^{B - b}.  One CTA per segment k < last walks its chunks from
 // the end while max_j decay_j max |D[j,:]| >= kFixStop (as the forward's fix-up); di and d log f are
 // read, corrected and stored back.  8 warps: thread (row r, half) holds 64 columns of row r of D.
+// D_k is the scan's, or, with up to kBwdMergedMax segments (merged), summed here from the maps,
+// nearest first: D_k = sum_{m>k} Diag(w_m) W_m, w_m = prod_{k<l<m} g_l, each thread for its own
+// row r while w_m (nseg - m) M[r] >= kStop, M[r] = max_{m>k} sum_v |W_m[r,v]| (the maps left out
+// add less than that to any entry, as in the forward's fix-up).  Segment 0's CTA then writes
+// dh0 = Diag(g_0) D_0 + W_0.
 namespace bfx {
 constexpr float kStop = 0x1p-24f;
+constexpr int kBwdMergedMax = 18;   // segments per pair up to which the fix-up sums D itself
 struct Misc {
     uint64_t fullA, fullB, barM;   // A: i and the saved state; B: log f, di, d log f
     uint32_t tmem_base;
@@ -1241,8 +1258,13 @@ constexpr size_t kSmem = 6 * (size_t)kTileBytes + sizeof(Misc);
 
 struct BwdFixParams {
     const float *D;     // [B*H][nseg][128][128]: slot k+1 = the gradient carried into segment k's end
+                        // (the scan's), or (merged) the segments' maps W
     const int *flags;
     int H, nseg, tps, ntiles;
+    bool merged;
+    const float *g;     // merged: [B*H][nseg][128] the segments' decay products
+    const float *Wabs;  // merged: [B*H][nseg][128][4] quarter sums of |W| per row
+    float *dh0;         // merged: dh0 [B*H][128][128] (may be null)
 };
 
 __global__ void __launch_bounds__(256, 1)
@@ -1324,14 +1346,61 @@ bwd_fixup_kernel(const __grid_constant__ CUtensorMap tm_lf, const __grid_constan
     }
     float Dr[64];      // the carried gradient, row r, columns 64 ch .. 64 ch + 63
     float dmax = 0.0f, decay = 1.0f;
-    {
-        const float4 *src = reinterpret_cast<const float4 *>(p.D + ((size_t)bh * p.nseg + seg + 1) * 16384 +
-                                                             (size_t)r * 128 + 64 * ch);
+    const size_t s0 = (size_t)bh * p.nseg;
+    if (!p.merged) {
+        const float4 *src = reinterpret_cast<const float4 *>(p.D + (s0 + seg + 1) * 16384 + (size_t)r * 128 + 64 * ch);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float4 a = src[i];
             Dr[4 * i] = a.x; Dr[4 * i + 1] = a.y; Dr[4 * i + 2] = a.z; Dr[4 * i + 3] = a.w;
         }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) Dr[i] = 0.0f;
+    }
+    if (p.merged && !flagged) {
+        // map m = seg+1+i, row r: x[i] = sum_v |W_m[r,v]|, loaded at once (indices clamped to the
+        // last segment, the extra values unused); M = max over the later segments (NaN kept); the
+        // maps m' >= m add at most w_m (nseg - m) M to an entry of row r
+        constexpr int kMaps = kBwdMergedMax - 1;
+        const int nl = p.nseg - 1 - seg;   // later segments
+        float xr[kMaps];
+#pragma unroll
+        for (int i = 0; i < kMaps; ++i) {
+            const float4 a = *reinterpret_cast<const float4 *>(p.Wabs + ((s0 + (size_t)min(seg + 1 + i, p.nseg - 1)) * 128 + r) * 4);
+            xr[i] = (a.x + a.y) + (a.z + a.w);
+        }
+        float M = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kMaps; ++i)
+            if (i < nl) M = (xr[i] > M || isnan(xr[i])) ? xr[i] : M;
+        float w = 1.0f;
+        for (int i = 0; i < nl; ++i) {
+            if (w * ((float)(nl - i) * M) < kStop) break;   // false for NaN: the row walks on
+            const size_t sl = s0 + seg + 1 + i;
+            const float4 *src = reinterpret_cast<const float4 *>(p.D + sl * 16384 + (size_t)r * 128 + 64 * ch);
+            const float gm = p.g[sl * 128 + r];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float4 a = src[k];
+                Dr[4 * k] = fmaf(w, a.x, Dr[4 * k]); Dr[4 * k + 1] = fmaf(w, a.y, Dr[4 * k + 1]);
+                Dr[4 * k + 2] = fmaf(w, a.z, Dr[4 * k + 2]); Dr[4 * k + 3] = fmaf(w, a.w, Dr[4 * k + 3]);
+            }
+            w *= gm;
+        }
+        if (seg == 0 && p.dh0) {   // dh0 = Diag(g_0) D_0 + W_0
+            const float gz = p.g[s0 * 128 + r];
+            const float4 *src = reinterpret_cast<const float4 *>(p.D + s0 * 16384 + (size_t)r * 128 + 64 * ch);
+            float4 *dst = reinterpret_cast<float4 *>(p.dh0 + (size_t)bh * 16384 + (size_t)r * 128 + 64 * ch);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float4 a = src[i];
+                dst[i] = make_float4(fmaf(gz, Dr[4 * i], a.x), fmaf(gz, Dr[4 * i + 1], a.y),
+                                     fmaf(gz, Dr[4 * i + 2], a.z), fmaf(gz, Dr[4 * i + 3], a.w));
+            }
+        }
+    }
+    if (!flagged) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) dmax = fmaxf(dmax, fabsf(Dr[i]));
     }
@@ -1543,9 +1612,14 @@ static_assert(tcb::bfx::kSmem <= 227 * 1024, "backward fix-up shared memory");
 size_t tc_bwd_workspace(int B, int T, int H) {
     int nseg, tps;
     tc_fwd_segments(B, T, H, &nseg, &tps);   // the forward's cut
-    return nseg > 1 ? (size_t)B * H * nseg * (16384 + 128) * sizeof(float) : 0;
+    // per segment: W, g and the quarter sums of |W| per row
+    return nseg > 1 ? (size_t)B * H * nseg * (16384 + 128 + 512) * sizeof(float) : 0;
 }
-int tc_bwd_launches(int B, int T, int H) { return tc_bwd_workspace(B, T, H) ? 3 : 1; }
+int tc_bwd_launches(int B, int T, int H) {
+    int nseg, tps;
+    tc_fwd_segments(B, T, H, &nseg, &tps);
+    return tc_bwd_workspace(B, T, H) ? (nseg <= tcb::bfx::kBwdMergedMax ? 2 : 3) : 1;
+}
 
 // Launches a kernel as a programmatic dependent of the previous work in the stream: it may be
 // scheduled before that work completes, and waits for it with grid_dep_wait().
@@ -1601,13 +1675,16 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
     if (saved && !packed && !a.lgs && !inplace && D == 128 && a.seg_ws) tc_fwd_segments(a.B, a.T, a.H, &nseg, &tps);
     if (nseg > 1) {
         // sequence segments: every segment from a zero gradient (the last from dhT), the reverse
-        // scan of their maps (and dh0), then the carried gradients added to each segment's last chunks
+        // scan of their maps (and dh0) unless the fix-up sums them itself, then the carried
+        // gradients added to each segment's last chunks
         const int BH = a.B * a.H;
-        float *W = a.seg_ws, *g = a.seg_ws + (size_t)BH * nseg * 16384;
+        float *W = a.seg_ws, *g = a.seg_ws + (size_t)BH * nseg * 16384, *Wabs = g + (size_t)BH * nseg * 128;
+        const bool merged = nseg <= tcb::bfx::kBwdMergedMax;
         p2.nseg = nseg;
         p2.tps = tps;
         p2.Wseg = W;
         p2.gseg = g;
+        p2.Wabs = Wabs;
         size_t smem = tcb::rsw::kSmemBytes;
         if (simt_bwd_dq_smem(a.simt_C, D, D) > smem) smem = simt_bwd_dq_smem(a.simt_C, D, D);
         if (simt_bwd_rev_smem(a.simt_C, D, D) > smem) smem = simt_bwd_rev_smem(a.simt_C, D, D);
@@ -1616,13 +1693,15 @@ cudaError_t launch_tc_bwd(const TcBwdArgs &a, cudaStream_t st) {
             return e;
         kern<<<BH * nseg, tcb::rsw::kRevThreads, smem, st>>>(mq, ml, mx, mdo, mdq, mdi, mdl, mst, p2);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        e = launch_dependent_b(tcb::bwd_scan_kernel, dim3(BH * 16), dim3(256), 0, st, W, (const float *)g, nseg,
-                               (const int *)a.flags, a.dh0);
-        if (e != cudaSuccess) return e;
+        if (!merged) {
+            e = launch_dependent_b(tcb::bwd_scan_kernel, dim3(BH * 16), dim3(256), 0, st, W, (const float *)g, nseg,
+                                   (const int *)a.flags, a.dh0);
+            if (e != cudaSuccess) return e;
+        }
         if ((e = cudaFuncSetAttribute(tcb::bwd_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)tcb::bfx::kSmem)) != cudaSuccess)
             return e;
-        tcb::BwdFixParams fp{W, a.flags, a.H, nseg, tps, ntiles};
+        tcb::BwdFixParams fp{W, a.flags, a.H, nseg, tps, ntiles, merged, g, Wabs, a.dh0};
         return launch_dependent_b(tcb::bwd_fixup_kernel, dim3(BH * (nseg - 1)), dim3(256), tcb::bfx::kSmem, st, ml,
                                   mx, mst, mdi, mdl, fp);
     }

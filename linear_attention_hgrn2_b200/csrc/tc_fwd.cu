@@ -117,6 +117,9 @@ struct Params {
     // d = 128 only); h1row0 / h2row0: this CTA's first row = its slot times 128.
     int hmaps;
     int hslot1, hslot2;   // 0: the pair's index; 1: the segment slot (b,h) nseg + seg
+    // With segments: [B*H][nseg][128] sum_v |U[j,v]| of every segment's U, row j (the fix-up's
+    // bound on what the maps it leaves out could add; a sum, so that inf and NaN carry into it)
+    float *uabs;
 };
 
 // kPacked: p.cu holds packed sequences (compiled apart so the dense path carries no row masks).
@@ -126,8 +129,7 @@ struct Params {
 // (per-row factors), the state scales e^{B/2} for every state row.  A chunk with B / 2 < -kMaxRefLog
 // sends the pair to the exact CUDA-core forward (its flag also routes the backward).
 // kSeg: dense launches with sequence segments (the first chunk's q e^{b} and B are written for the
-// fix-up; the kernel lets its dependent launch early), compiled apart from the one-CTA-per-pair
-// instance.
+// fix-up), compiled apart from the one-CTA-per-pair instance.
 template <bool kPacked, bool kScalar = false, bool kSeg = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_lf,
@@ -141,7 +143,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     uint8_t *X = smem + 6 * kTileBytes;
     Misc *m = reinterpret_cast<Misc *>(smem + 7 * kTileBytes);
 
-    if constexpr (kSeg) grid_dep_launch();   // the scan or fix-up may be scheduled now; it waits for this grid
+    // (kSeg: no early trigger of the dependent scan or fix-up; it launches as this grid's CTAs
+    // exit.  Triggered at this kernel's start, the fix-up's CTAs took the SMs this grid leaves free
+    // and waited there, and the calls measured slower: A/B on one B200, forward layer 48.4 -> 45.8
+    // us, long sequence 128.1 -> 119.9 us without the trigger.)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int bh = blockIdx.x / p.nseg;
     const int seg = blockIdx.x - bh * p.nseg, h = bh % p.H;
@@ -483,6 +488,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 // two ring tiles, then TMA stores (the group's condition here is uniform: all 128
                 // threads finished the loop together, and r < 128)
                 uint8_t *stg = smem;
+                float rabs = 0.0f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     float v[32];
@@ -490,10 +496,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                     tmem_wait_ld();
                     uint8_t *row = stg + (size_t)c * 16384 + r * 128;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        *reinterpret_cast<float4 *>(row + ((k ^ (r & 7)) << 4)) =
-                            make_float4(v[4 * k] * e, v[4 * k + 1] * e, v[4 * k + 2] * e, v[4 * k + 3] * e);
+                    for (int k = 0; k < 8; ++k) {
+                        const float4 w = make_float4(v[4 * k] * e, v[4 * k + 1] * e, v[4 * k + 2] * e, v[4 * k + 3] * e);
+                        rabs += (fabsf(w.x) + fabsf(w.y)) + (fabsf(w.z) + fabsf(w.w));
+                        *reinterpret_cast<float4 *>(row + ((k ^ (r & 7)) << 4)) = w;
+                    }
                 }
+                if (p.nseg > 1 && p.uabs) p.uabs[((size_t)bh * p.nseg + seg) * 128 + r] = rabs;
                 fence_proxy_async_smem();
                 named_bar_sync(2, 128);
                 if (r == 0) {
@@ -509,6 +518,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 float *dst = p.nseg > 1 ? p.Useg + (((size_t)bh * p.nseg + seg) * 128 + r) * 128
                                         : p.hT ? p.hT + ((size_t)bh * p.D + r) * p.D : nullptr;
                 float *dsv = p.nseg > 1 ? nullptr : p.hTs ? p.hTs + ((size_t)bh * p.D + r) * p.D : nullptr;
+                float rabs = 0.0f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     if (32 * c >= p.D) break;
@@ -518,10 +528,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float4 w = make_float4(v[4 * i] * e, v[4 * i + 1] * e, v[4 * i + 2] * e, v[4 * i + 3] * e);
+                        rabs += (fabsf(w.x) + fabsf(w.y)) + (fabsf(w.z) + fabsf(w.w));
                         if (dst) reinterpret_cast<float4 *>(dst + 32 * c)[i] = w;
                         if (dsv) reinterpret_cast<float4 *>(dsv + 32 * c)[i] = w;
                     }
                 }
+                if (p.nseg > 1 && p.uabs) p.uabs[((size_t)bh * p.nseg + seg) * 128 + r] = rabs;
             }
         }
     } else if (warp >= 8) {
@@ -1032,28 +1044,32 @@ scan_kernel(float *__restrict__ U, const float *__restrict__ g, int nseg, const 
 // Without saved states two stages: the next chunk's tiles load while this one is on the tensor
 // cores and in the epilogue (the decision to walk it is taken from this chunk's e^{B}, before
 // they are requested).
-// S_in is the scan kernel's (slot k-1 of Sin), or, with few segments (merged), summed here from
-// the segments' maps: S_in = sum_{m<k} Diag(prod_{m<l<k} g_l) U_m; the last segment's CTA then
-// also writes hT = Diag(g_k) S_in + U_k.  A programmatic dependent of the kernel before it: only
-// its set-up runs before grid_dep_wait().
+// S_in is the scan kernel's (slot k-1 of Sin), or, with up to kMergedScanMax segments (merged),
+// summed here from the segments' maps, nearest first: S_in = sum_{m<k} Diag(w_m) U_m with
+// w_m = prod_{m<l<k} g_l.  The walk ends at the first m where max_j w_m[j] (m + 1) M[j] <
+// kFixStop, M[j] = max_{m'<k} sum_v |U_m'[j,v]|: the maps m' <= m left out add less than that to
+// any entry (w only shrinks further back), the bar the carried state itself is held to.  The last
+// segment's CTA then also writes hT = Diag(g_k) S_in + U_k.  A programmatic dependent of the
+// kernel before it: only its set-up runs before grid_dep_wait().
 constexpr float kFixStop = 0x1p-24f;
 
 struct FixMisc {
     uint64_t fullQG[2], fullO[2], barM, fullU[2];   // fullU: the segments' state slots
     uint32_t tmem_base;
-    int pad;
+    int nmaps;            // merged: the segments' maps the walk takes
     float EB[128];        // e^{B} of the chunk, key dim
     float ER[128];        // e^{rho} = e^{B/2} of the chunk, key dim (the saved states' scale)
     float Ppart[3][128];  // per 32-row range sums of log f (ranges 0..2)
 };
 // one stage (q, log f, o, saved state) + X, or two stages (q, log f, o) + X
 constexpr size_t fix_smem(bool save) { return (save ? 5 : 7) * (size_t)kTileBytes + sizeof(FixMisc); }
-constexpr int kMergedScanMax = 4;   // segments per pair up to which the fix-up sums S_in itself
+constexpr int kMergedScanMax = 18;   // segments per pair up to which the fix-up sums S_in itself
 
 struct FixParams {
     const float *U;     // [B*H][nseg][128][128]: the segments' U, or (after the scan kernel) slot k-1 =
                         // the state entering segment k
     const float *g;     // [B*H][nseg][128]: the segments' decay products (merged)
+    const float *uabs;  // [B*H][nseg][128]: sum_v |U[j,v]| of the segments' U, row j (merged)
     const float *B0;    // [B*H][nseg][128]: each segment's first-chunk total log decay
     const int *flags;   // [B*H] nonzero: recomputed whole by the exact route (skipped)
     float *hT, *hTs;    // merged: the final state (either may be null)
@@ -1091,6 +1107,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             mbar_init(&m->fullU[s], 1);
         }
         mbar_init(&m->barM, 1);
+        m->nmaps = 1;
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_lf);
@@ -1187,15 +1204,17 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const bool flagged = p.flags[bh] != 0;
     const bool want_hT = p.merged && seg == p.nseg - 1 && (p.hT || p.hTs);
     // The segments' state slots it reads, 64 KB each, staged through shared memory by TMA (tiles
-    // the first chunk does not use yet): merged, segments 0 .. seg-1 (and its own for hT); else
-    // the scan's slot seg-1.  Two buffers with two stages, one with one.
-    const int nslots = flagged ? 0 : p.merged ? seg + (want_hT ? 1 : 0) : 1;
+    // the first chunk does not use yet): merged, segments seg-1, seg-2, ... (nmaps of them) and its
+    // own for hT; else the scan's slot seg-1.  Two buffers with two stages, one with one.
     const int nbuf = NS;
     auto ubox = [&](int buf, int bx) -> uint8_t * {   // 32 columns x 128 rows of fp32, swizzled
         if (NS == 2) return smem + (size_t)(3 + 2 * buf) * kTileBytes + (size_t)bx * 16384;
         return smem + (size_t)(bx < 2 ? 1 : 4) * kTileBytes + (size_t)(bx & 1) * 16384;
     };
-    auto slot_of = [&](int i) { return (size_t)bh * p.nseg + (p.merged ? i : seg - 1); };
+    int nmaps = 1;   // slots i < nmaps: segment seg-1-i (merged); i = nmaps: its own (hT)
+    auto slot_of = [&](int i) {
+        return (size_t)bh * p.nseg + (!p.merged ? seg - 1 : i < nmaps ? seg - 1 - i : seg);
+    };
     int issuedU = 0, waitedU = 0;
     auto load_u = [&](int i) {   // thread 0: slot i into buffer i % nbuf
         const int buf = i % nbuf;
@@ -1203,8 +1222,7 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int bx = 0; bx < 4; ++bx) tma_load_2d(ubox(buf, bx), &tm_u, &m->fullU[buf], 32 * bx, (int)slot_of(i) * 128);
         ++issuedU;
     };
-    if (tid == 0)
-        for (int i = 0; i < nslots && i < nbuf; ++i) load_u(i);
+    if (tid == 0 && !flagged) load_u(0);   // segment seg-1 (merged) or the scan's slot: always read
     if (!flagged) {
         if (tid == 0) {   // the first chunk's tiles
             fence_proxy_async_global();
@@ -1217,10 +1235,48 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             m->ER[tid] = __expf(0.5f * B);
         }
     }
+    if (p.merged && !flagged) {   // how far back the walk goes, from this thread's row r
+        // map m = seg-1-i, row r: x[i] = sum_v |U_m[r,v]| and g_m[r], all loaded at once (indices
+        // clamped to segment 0, the extra values unused).  M = max_{i<seg} x[i] (NaN kept): the maps
+        // m' <= m add at most w_m (m + 1) M to an entry of row r.
+        const size_t s0 = (size_t)bh * p.nseg;
+        constexpr int kMaps = kMergedScanMax - 1;
+        float xr[kMaps], gr[kMaps];
+#pragma unroll
+        for (int i = 0; i < kMaps; ++i) {
+            const size_t sl = s0 + (size_t)max(seg - 1 - i, 0);
+            xr[i] = p.uabs[sl * 128 + r];
+            gr[i] = p.g[sl * 128 + r];
+        }
+        float M = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kMaps; ++i)
+            if (i < seg) M = (xr[i] > M || isnan(xr[i])) ? xr[i] : M;
+        float w = 1.0f;
+        int n = 0;
+        bool on = true;
+#pragma unroll
+        for (int i = 0; i < kMaps; ++i) {   // "not below" is true for NaN: such a row walks on
+            on = on && i < seg && !(w * ((float)(seg - i) * M) < kFixStop);
+            if (on) {
+                ++n;
+                w *= gr[i];
+            }
+        }
+        n = __reduce_max_sync(0xffffffffu, n);
+        if (lane == 0 && n > 1) atomicMax(&m->nmaps, n);
+        __syncthreads();
+        nmaps = m->nmaps;
+    }
+    const int nslots = flagged ? 0 : p.merged ? nmaps + (want_hT ? 1 : 0) : 1;
+    if (tid == 0)
+        for (int i = 1; i < nslots && i < nbuf; ++i) load_u(i);
 #pragma unroll
     for (int i = 0; i < 64; ++i) S[i] = 0.0f;
+    float wr = 1.0f;   // merged: the weight of the next map, row r
     for (int i = 0; i < nslots; ++i) {
         const int buf = i % nbuf;
+        const float gi = p.merged ? p.g[slot_of(i) * 128 + r] : 0.0f;   // issued before the wait
         if (__syncthreads_or(!mbar_wait(&m->fullU[buf], (i / nbuf) & 1))) { ok = false; break; }
         waitedU = i + 1;
         float u[64];   // row r, columns 64 ch .. 64 ch + 63 of the slot
@@ -1237,12 +1293,12 @@ fixup_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (!p.merged) {          // the scan's state entering this segment
 #pragma unroll
             for (int k = 0; k < 64; ++k) S[k] = u[k];
-        } else if (i < seg) {     // S_in = Diag(g_i) S + U_i over the earlier segments
-            const float gi = p.g[slot_of(i) * 128 + r];
+        } else if (i < nmaps) {   // S_in += Diag(w) U_m, m = seg-1-i; then w *= g_m
 #pragma unroll
-            for (int k = 0; k < 64; ++k) S[k] = fmaf(gi, S[k], u[k]);
+            for (int k = 0; k < 64; ++k) S[k] = fmaf(wr, u[k], S[k]);
+            wr *= gi;
         } else {                  // the sequence's final state: Diag(g_k) S_in + U_k
-            const float gk = p.g[myslot * 128 + r];
+            const float gk = gi;
             const size_t rowoff = (size_t)bh * 16384 + (size_t)r * 128 + 64 * ch;
             float4 *d1 = p.hT ? reinterpret_cast<float4 *>(p.hT + rowoff) : nullptr;
             float4 *d2 = p.hTs ? reinterpret_cast<float4 *>(p.hTs + rowoff) : nullptr;
@@ -1413,9 +1469,9 @@ size_t tc_fwd_workspace(int B, int T, int H) {
     int nseg, tps;
     tc_fwd_segments(B, T, H, &nseg, &tps);
     if (nseg <= 1) return 0;
-    // per segment: U, g, the first chunk's B (fp32) and q e^{b} (bf16); then the per-pair
-    // finished-segment counts
-    return (size_t)B * H * nseg * ((16384 + 2 * 128) * sizeof(float) + 16384 * sizeof(__nv_bfloat16)) +
+    // per segment: U, g, the first chunk's B, the row sums of |U| (fp32) and q e^{b} (bf16); then
+    // the per-pair finished-segment counts
+    return (size_t)B * H * nseg * ((16384 + 3 * 128) * sizeof(float) + 16384 * sizeof(__nv_bfloat16)) +
            (size_t)B * H * sizeof(int);
 }
 
@@ -1488,11 +1544,13 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcf::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int BH = a.B * a.H;
-    // segment workspace: U [BH][nseg][128][128], g and the first chunk's B [BH][nseg][128] (fp32),
-    // the first chunk's q e^{b} [BH][nseg][128][128] (bf16), the finished-segment counts [BH]
+    // segment workspace: U [BH][nseg][128][128], g, the first chunk's B and the row sums of |U|
+    // [BH][nseg][128] (fp32), the first chunk's q e^{b} [BH][nseg][128][128] (bf16), the
+    // finished-segment counts [BH]
     const size_t nsl = (size_t)BH * nseg;
     float *U = a.seg_ws, *g = a.seg_ws ? U + nsl * 16384 : nullptr, *bs = a.seg_ws ? g + nsl * 128 : nullptr;
-    __nv_bfloat16 *qtil = a.seg_ws ? reinterpret_cast<__nv_bfloat16 *>(bs + nsl * 128) : nullptr;
+    float *uabs = a.seg_ws ? bs + nsl * 128 : nullptr;
+    __nv_bfloat16 *qtil = a.seg_ws ? reinterpret_cast<__nv_bfloat16 *>(uabs + nsl * 128) : nullptr;
     int *seg_done = a.seg_ws ? reinterpret_cast<int *>(qtil + nsl * 16384) : nullptr;
     if (nseg > 1) {
         // pass 1 only raises the exact-route flags and counts finished segments: both start at zero
@@ -1508,6 +1566,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     // the segments' final states U leave through shared memory by TMA (measured: U stores 4 us
     // sooner on the long sequence; for one CTA per pair the row stores of hT, whose drain does not
     // hold the CTA, measured 1 us faster than the TMA store and its wait)
+    p.uabs = nseg > 1 ? uabs : nullptr;
     CUtensorMap mh1 = mo, mh2 = mo;
     if (a.D == 128 && nseg > 1 && U && make_state_map(&mh1, U, (size_t)BH * nseg * 128)) {
         p.hmaps = 1;
@@ -1516,7 +1575,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     kern<<<BH * nseg, tcf::kFwdThreads, tcf::kSmemBytes, st>>>(mq, ml, mx, mo, mst, mh1, mh2, p);
     if ((e = cudaGetLastError()) != cudaSuccess || nseg == 1) return e;
     // segments: the states entering them (and hT), then the carried states' contributions.  With
-    // few segments the fix-up sums the states itself; else the scan kernel chains them first.
+    // up to kMergedScanMax segments the fix-up sums the states it needs itself, nearest first;
+    // else the scan kernel chains them first.
     // Each launch is a programmatic dependent of the one before it, so that its start-up overlaps
     // that kernel's end.
     const bool merged = nseg <= tcf::kMergedScanMax;
@@ -1530,7 +1590,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t st) {
     const size_t fsm = tcf::fix_smem(a.st16 != nullptr);
     e = cudaFuncSetAttribute(tcf::fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
     if (e != cudaSuccess) return e;
-    tcf::FixParams fp{U, g, bs, a.flags, merged ? a.hT : nullptr, merged && a.st16 ? a.hTs : nullptr,
+    tcf::FixParams fp{U, g, uabs, bs, a.flags, merged ? a.hT : nullptr, merged && a.st16 ? a.hTs : nullptr,
                       a.H, nseg, tps, ntiles, a.st16 != nullptr, merged};
     e = launch_dependent(tcf::fixup_kernel, dim3(BH * (nseg - 1)), dim3(tcf::kThreads), fsm, st, mq, ml, mo, mst,
                          mqt, mu, fp);

@@ -202,7 +202,7 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
     assert f(B, T, H, 64, 64, 64, L.BF16, 1) == f(B, T, H, 64, 64, 64, L.BF16, 2) + extra
     # d = 128 with saved states and few (b,h): the backward runs in sequence segments, cut as the
     # forward cuts them (148 // (B*H) per pair, at most one per chunk), and keeps every segment's
-    # backward map (128 x 128 + 128 floats)
+    # backward map (128 x 128 + 128 floats) and the quarter sums of |W| per row (4 x 128 floats)
     def nseg(B, T, H):
         ntiles = (T + 127) // 128
         ns = min(max(1, 148 // (B * H)), ntiles)
@@ -212,7 +212,7 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
     # workspace and then the saved-state backward: room for both, the saved buffer and an o scratch.
     for (B, T, H) in ((2, 300, 3), (1, 32768, 8), (8, 2048, 16)):
         ns = nseg(B, T, H)
-        seg = up(B * H * ns * (128 * 128 + 128) * 4) if ns > 1 else 0
+        seg = up(B * H * ns * (128 * 128 + 128 + 512) * 4) if ns > 1 else 0
         base = up(B * H * 128 * 4) + up(B * H * 4)   # rowsum(dhT * hT), exact-route flags
         assert f(B, T, H, 128, 128, 64, L.BF16, 2) == base + seg, (B, T, H)
         if ns > 1:

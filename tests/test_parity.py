@@ -289,8 +289,9 @@ def test_autograd_function_uses_saved_states(cuda):
     loss.backward()
     c = L.counters(reset=True)
     # segmented forward (3 segments per pair: segments, then the fix-up that sums the entering states
-    # itself) + segmented saved backward (segments, reverse scan, fix-up)
-    assert c[2] == 2 + 3, c
+    # itself) + segmented saved backward (segments, then the fix-up that sums the carried gradients
+    # itself)
+    assert c[2] == 2 + 2, c
     ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True, dhT=inp["dhT"])
     for n, h in enumerate((0, 1)):
         for name, got in (("dq", q.grad[0, :, h]), ("dlog_f", lf.grad[0, :, h]), ("di", x.grad[0, :, h]),
@@ -322,7 +323,8 @@ def test_more_pairs_than_sms(cuda, saved):
 
 @pytest.mark.parametrize("saved", [False, True], ids=["plain", "saved"])
 def test_segmented_forward_with_a_flagged_pair(cuda, saved):
-    # B*H = 2: the forward runs in 8 sequence segments (segments, scan, fix-up: 3 launches).  Head 1
+    # B*H = 2: the forward runs in 8 sequence segments (segments, then the fix-up, which sums the
+    # states entering them itself: 2 launches).  Head 1
     # has gates shifted below the factorised range: its segments flag it, and the last of its
     # segments to finish recomputes the whole sequence on the exact route in the same launch
     B, T, H = 1, 1000, 2
@@ -335,7 +337,7 @@ def test_segmented_forward_with_a_flagged_pair(cuda, saved):
     L.counters(reset=True)
     o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
     c = L.counters(reset=True)
-    assert c[2] == 3 and c[0] >= 1, c
+    assert c[2] == 2 and c[0] >= 1, c
     assert L.device_status() == L.OK
     want_bwd = saved
     if saved:
@@ -384,14 +386,46 @@ def test_segmented_forward_few_segments(cuda, saved, lb):
             assert e <= 2e-2, (name, b, h, e)
 
 
+@pytest.mark.parametrize("saved", [False, True], ids=["plain", "saved"])
+@pytest.mark.parametrize("lb", [0.999, 0.9])
+def test_segmented_forward_walks_back_as_far_as_the_states_matter(cuda, saved, lb):
+    # B*H = 8, T = 2304: 18 one-chunk segments per pair.  The fix-up of segment k sums the maps of
+    # segments k-1, k-2, ... while what the rest could add is at least 2^-24: at lb = 0.999 (a
+    # chunk keeps ~94% of the state) that is every earlier segment, and the last segment's hT sums
+    # all 17; at lb = 0.9 a few.  Checked against the oracle with h0 and hT, and (saved) through
+    # the corrected chunk states that the backward reads.
+    B, T, H = 1, 2304, 8
+    inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, lb, seed=1170 + int(lb * 1000), h0_sigma=0.1,
+                        with_dO=True, dhT_sigma=0.1)
+    g = to_cuda(inp)
+    sv = L.new_saved(g["q"]) if saved else None
+    L.counters(reset=True)
+    o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    c = L.counters(reset=True)
+    assert c[2] == 2 and c[0] == 0, c
+    assert L.device_status() == L.OK
+    if saved:
+        dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
+                                 saved=sv)
+    pairs = [(0, 0), (0, 3), (0, 7)]
+    ref = oracle_heads(inp, pairs, want_bwd=saved, dhT=inp["dhT"])
+    for n, (b, h) in enumerate(pairs):
+        got = [("o", o[b, :, h]), ("hT", hT[b, h])]
+        if saved:
+            got += [("dq", dq[b, :, h]), ("dlog_f", dlf[b, :, h]), ("di", di[b, :, h]), ("dh0", dh0[b, h])]
+        for name, t in got:
+            e = err(np64(t), ref[name][n], torch.bfloat16)
+            assert e <= 2e-2, (name, b, h, e)
+
+
 @pytest.mark.parametrize("saved", [True, False], ids=["saved", "recompute"])
 @pytest.mark.parametrize("lb,T", [(0.9, 32768), (0.0, 4096)])
 def test_segmented_backward_long_sequence(cuda, lb, T, saved):
     # B*H = 8, the long workload's shape as a training pair: the saved-state backward runs in
     # segments (18 of 15 chunks per pair at T = 32768; 16 of 2 at T = 4096): every segment's reverse
-    # sweep from a zero gradient (the last from dhT), the reverse scan of their maps (giving dh0),
-    # then the carried gradients added to di and d log f of each segment's last chunks.  Without
-    # saved states the backward first runs the training forward into its workspace (3 more
+    # sweep from a zero gradient (the last from dhT), then the carried gradients, summed from the
+    # later segments' maps, added to di and d log f of each segment's last chunks (and dh0).
+    # Without saved states the backward first runs the training forward into its workspace (2 more
     # launches).  lb = 0: strong decay.
     B, H = 1, 8
     inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, lb, seed=1090 + T, h0_sigma=0.1, with_dO=True,
@@ -403,7 +437,7 @@ def test_segmented_backward_long_sequence(cuda, lb, T, saved):
     dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
                              saved=sv)
     c = L.counters(reset=True)
-    assert c[2] == (3 if saved else 6) and c[0] == 0, c
+    assert c[2] == (2 if saved else 4) and c[0] == 0, c
     assert L.device_status() == L.OK
     pairs = [(0, 0), (0, 5)]
     ref = oracle_heads(inp, pairs, want_bwd=True, dhT=inp["dhT"])
@@ -416,16 +450,20 @@ def test_segmented_backward_long_sequence(cuda, lb, T, saved):
 
 def test_saved_pair_long_segmented_sequence(cuda):
     # B*H = 2: the forward cuts each sequence into 32 one-chunk segments (segments from zero states,
-    # fp32 scan, carried-state fix-up) and saves the chunk states of all of them; the
-    # backward walks all 32 chunks of each sequence from the saved states
+    # fp32 scan, carried-state fix-up) and saves the chunk states of all of them; the backward runs
+    # the same 32 segments (reverse sweeps, reverse fp32 scan of their maps, carried-gradient
+    # fix-up).  More than 18 segments per pair: both scans are launches of their own.
     B, T, H = 1, 4096, 2
     inp = I.make_inputs(B, T, H, 128, 128, torch.bfloat16, 0.95, seed=41, h0_sigma=0.1, with_dO=True,
                         dhT_sigma=0.1)
     g = to_cuda(inp)
     sv = L.new_saved(g["q"])
+    L.counters(reset=True)
     o, hT = L.fwd(g["q"], g["log_f"], g["i"], g["h0"], want_hT=True, chunk=64, saved=sv)
+    assert L.counters(reset=True)[2] == 3
     dq, dlf, di, dh0 = L.bwd(g["q"], g["log_f"], g["i"], g["dO"], g["h0"], g["dhT"], want_dh0=True, chunk=64,
                              saved=sv)
+    assert L.counters(reset=True)[2] == 3
     assert L.device_status() == L.OK
     ref = oracle_heads(inp, [(0, 0), (0, 1)], want_bwd=True, dhT=inp["dhT"])
     for n, h in enumerate((0, 1)):
