@@ -15,7 +15,7 @@ Recorded (worst over the seeds and over o, hT, dq, d log f, di):
   * floor 1e-3 * max|r|: about 7e-5;
   * floor 1e-2 * max|r|: about 7e-6.
 The parity tests use the floor in ``parity_util.FP32_FLOOR``; this test checks
-that plain float32 passes it with room to spare and that the survey's rms
+that plain float32 passes it with room to spare and that the 1e-3 * rms(r)
 floor is indeed out of reach, so the choice of floor is reproducible.
 """
 import numpy as np
