@@ -1,6 +1,6 @@
 """Error metrics and oracle helpers shared by the GPU parity tests.
 
-Tolerances (the accuracy bar of the benchmark spec for this method):
+Tolerances (the accuracy bar set for this method: fp32 relative, bf16 normalised max-abs):
   * float32 inputs: max relative error <= 1e-4, measured element-wise as
         max_i |g_i - r_i| / max(|r_i|, FP32_FLOOR * max_j |r_j|)
     The floor keeps elements that are ~0 from dividing by ~0: an element-wise
