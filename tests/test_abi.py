@@ -222,6 +222,13 @@ def test_workspace_size_of_the_backward_with_saved_states(lib):
         else:
             assert f(B, T, H, 128, 128, 64, L.BF16, 1) == base, (B, T, H)
     assert nseg(8, 2048, 16) == 1 and nseg(1, 32768, 8) == 18
+    # the forward with segments: per segment its U (128 x 128), g, the first chunk's total decay and
+    # the row sums of |U| (3 x 128 floats), the first chunk's bf16 q e^{b} (128 x 128); then the
+    # per-pair finished-segment counts
+    for (B, T, H) in ((2, 300, 3), (1, 32768, 8), (8, 2048, 16), (4, 2048, 8)):
+        ns = nseg(B, T, H)
+        fseg = up(B * H * ns * ((128 * 128 + 3 * 128) * 4 + 128 * 128 * 2) + B * H * 4) if ns > 1 else 0
+        assert f(B, T, H, 128, 128, 64, L.BF16, 0) == up(B * H * 4) + fseg, (B, T, H)
     assert f(B, T, H, 64, 64, 64, L.BF16, 3) == bad
     assert f(B, T, H, 64, 64, 64, L.BF16, -1) == bad
 
